@@ -1,0 +1,121 @@
+"""fp64 CPU oracle of softmax attention, forward and backward.
+
+Test infrastructure only (see the package docstring): the product path never
+imports this module.
+
+What it computes.  DASH summary §1 fixes the object of the method: the attention
+backward pass, whose dQ gradient must be accumulated in a fixed order to be
+bit-reproducible.  The pages print no formulas, so this module writes out the
+textbook definition of softmax attention and its gradient, per (batch, head),
+in float64, with no tiling, blocking or reordering:
+
+  forward   s_ij  = scale * q_i . k_j          (masked to -inf if causal and j > i)
+            LSE_i = log sum_j exp(s_ij)        (natural log)
+            P_ij  = exp(s_ij - LSE_i)
+            O_i   = sum_j P_ij v_j
+  backward  dV_j  = sum_i P_ij dO_i
+            dP_ij = dO_i . v_j
+            Delta_i = dO_i . O_i               (= sum_j P_ij dP_ij)
+            dS_ij = P_ij (dP_ij - Delta_i)
+            dQ_i  = scale * sum_j dS_ij k_j
+            dK_j  = scale * sum_i dS_ij q_i
+
+Causal masking is top-left aligned with equal query and key lengths: query row
+i attends to keys j <= i.  Inputs may be any float dtype (e.g. bf16 values held
+in float32); they are widened exactly to float64.  A matrix product (numpy's
+``@``) serves as a library step.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def _f64(x) -> np.ndarray:
+    """Widen to float64 (exact for bf16 / fp16 / fp32 inputs)."""
+    if hasattr(x, "detach"):  # a torch tensor: go through float32 (exact for bf16)
+        x = x.detach().to("cpu").float().numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def _mask(S: int, causal: bool) -> np.ndarray:
+    """Boolean [S,S] matrix of allowed (query i, key j) pairs."""
+    if not causal:
+        return np.ones((S, S), dtype=bool)
+    return np.tril(np.ones((S, S), dtype=bool))
+
+
+def head_forward(q, k, v, causal: bool, scale: float):
+    """Forward of one head: returns (O [S,D], LSE [S]) from the definition."""
+    S = q.shape[0]
+    s = scale * (q @ k.T)
+    allowed = _mask(S, causal)
+    s = np.where(allowed, s, -np.inf)
+    m = s.max(axis=1, keepdims=True)
+    lse = (m + np.log(np.exp(s - m).sum(axis=1, keepdims=True)))[:, 0]
+    p = np.where(allowed, np.exp(s - lse[:, None]), 0.0)
+    return p @ v, lse
+
+
+def head_backward(q, k, v, do, causal: bool, scale: float):
+    """Backward of one head: returns (dQ, dK, dV, Delta) from the definition.
+
+    O and LSE are recomputed here in float64; the backward's own formula
+    Delta_i = dO_i . O_i uses that O.
+    """
+    S = q.shape[0]
+    allowed = _mask(S, causal)
+    o, lse = head_forward(q, k, v, causal, scale)
+    s = np.where(allowed, scale * (q @ k.T), -np.inf)
+    p = np.where(allowed, np.exp(s - lse[:, None]), 0.0)
+    dv = p.T @ do
+    dp = do @ v.T
+    delta = (do * o).sum(axis=1)
+    ds = p * (dp - delta[:, None])
+    dq = scale * (ds @ k)
+    dk = scale * (ds.T @ q)
+    return dq, dk, dv, delta
+
+
+def forward(q, k, v, causal: bool, scale: float | None = None, heads=None):
+    """Batched forward over [B,H,S,D] inputs.
+
+    heads: optional iterable of (b, h) to compute; other heads are left NaN.
+    Returns (O [B,H,S,D] float64, LSE [B,H,S] float64).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, S, D = q.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    o = np.full((B, H, S, D), np.nan)
+    lse = np.full((B, H, S), np.nan)
+    for b, h in (heads if heads is not None else np.ndindex(B, H)):
+        o[b, h], lse[b, h] = head_forward(q[b, h], k[b, h], v[b, h], causal, scale)
+    return o, lse
+
+
+def backward(q, k, v, do, causal: bool, scale: float | None = None, heads=None):
+    """Batched backward over [B,H,S,D] inputs.
+
+    heads: optional iterable of (b, h) to compute; other heads are left NaN.
+    Returns (dQ, dK, dV [B,H,S,D], Delta [B,H,S]) in float64.
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, H, S, D = q.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    dq = np.full((B, H, S, D), np.nan)
+    dk = np.full((B, H, S, D), np.nan)
+    dv = np.full((B, H, S, D), np.nan)
+    delta = np.full((B, H, S), np.nan)
+    for b, h in (heads if heads is not None else np.ndindex(B, H)):
+        dq[b, h], dk[b, h], dv[b, h], delta[b, h] = head_backward(
+            q[b, h], k[b, h], v[b, h], do[b, h], causal, scale)
+    return dq, dk, dv, delta
+
+
+def rel_fro(x, ref) -> float:
+    """Relative Frobenius error ||x - ref||_F / ||ref||_F (the parity metric)."""
+    x, ref = _f64(x), _f64(ref)
+    den = np.linalg.norm(ref.ravel())
+    num = np.linalg.norm((x - ref).ravel())
+    return float(num / den) if den > 0 else float(num)

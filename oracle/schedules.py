@@ -1,0 +1,128 @@
+"""Oracle of the DASH tile schedules: visiting order and dQ accumulation order.
+
+Test infrastructure only (see the package docstring).
+
+Vocabulary.  A head has N = S/128 key/value (KV) tiles and N query (Q) tiles.
+A *pair* (kv, q) is the work of one KV tile against one Q tile; with a causal
+mask only pairs with q >= kv exist.  DASH summary §2.1 requires that all pairs of
+one KV tile run back to back on one SM (a *chain*), with dK/dV held on chip.  A
+*unit* is the work one CTA slot does for one head: one chain, or for the
+symmetric shift two chains.  Step t of a unit is its t-th pair.  Each Q tile's
+dQ block receives one partial per contributing KV tile; the *position* of a
+pair is the index of its partial in that block's fixed accumulation order.
+
+Schedules (names follow the pages):
+
+* ``naive_asc``  -- the serialised deterministic baseline of DASH summary §1:
+  every chain visits Q tiles ascending, and each dQ block accumulates its
+  partials in ascending KV order.
+* ``descending`` -- DASH summary §2.2.A: Q tiles visited from the last to the
+  first ("N to 0" on the page, read as N-1 down to 0 for N tiles numbered from
+  0).  The page does not change the accumulation order, so it stays ascending
+  in KV.
+* ``shift``      -- DASH summary §2.2.B, full masks: the SM holding KV tile k
+  visits k, k+1, ..., N-1, 0, ..., k-1 (the page prints this sequence; with one
+  KV tile per SM it is read as the sequence of Q tiles, i.e. dQ blocks, that
+  chain visits).  Each dQ block accumulates in step order.
+* ``sym_shift``  -- DASH summary §2.2.B, causal masks: KV tiles k and N-1-k are
+  paired (one CTA serves both, one after the other) so the triangle of causal
+  pairs folds into an N/2 x (N+1) rectangle, run in two phases: the dense
+  lower-left rectangle (Q in [N/2, N) x KV in [0, N/2)) and then the folded
+  upper triangle.  Accumulation follows (phase, step).  Requires even N.
+"""
+from __future__ import annotations
+
+NAIVE_ASC, DESCENDING, SHIFT, SYM_SHIFT = "naive_asc", "descending", "shift", "sym_shift"
+ALL = (NAIVE_ASC, DESCENDING, SHIFT, SYM_SHIFT)
+
+
+def supported(name: str, N: int, causal: bool) -> bool:
+    """Which (schedule, mask) combinations the pages define."""
+    if name == SHIFT:
+        return not causal
+    if name == SYM_SHIFT:
+        return causal and N % 2 == 0
+    return name in (NAIVE_ASC, DESCENDING)
+
+
+def units(name: str, N: int, causal: bool):
+    """Per-head units: a list, one entry per CTA slot of the head, each a list
+    of (kv, q) pairs in visiting order."""
+    if not supported(name, N, causal):
+        raise ValueError(f"schedule {name} undefined for N={N} causal={causal}")
+    out = []
+    if name == NAIVE_ASC:
+        for k in range(N):
+            qs = range(k, N) if causal else range(N)
+            out.append([(k, q) for q in qs])
+    elif name == DESCENDING:
+        for k in range(N):
+            lo = k if causal else 0
+            out.append([(k, q) for q in range(N - 1, lo - 1, -1)])
+    elif name == SHIFT:
+        for k in range(N):
+            out.append([(k, (k + t) % N) for t in range(N)])
+    elif name == SYM_SHIFT:
+        h = N // 2
+        for k in range(h):
+            seq = []
+            # phase 1: dense lower-left rectangle Q in [h, N) x KV in [0, h)
+            for t in range(h):
+                seq.append((k, h + (k + t) % h))
+            # phase 2: upper-left triangle of KV k, folded with the
+            # 180-degree-rotated lower-right triangle of KV N-1-k
+            for t in range(h):
+                r = (k + t) % h
+                seq.append((k, r) if r >= k else (N - 1 - k, N - 1 - r))
+            seq.append((N - 1 - k, N - 1 - k))  # the shared diagonal, last
+            out.append(seq)
+    return out
+
+
+def accumulation_order(name: str, N: int, causal: bool):
+    """dQ accumulation order per block: dict q -> list of (unit, step), first
+    partial first."""
+    us = units(name, N, causal)
+    contrib = {q: [] for q in range(N)}
+    for u, seq in enumerate(us):
+        for t, (kv, q) in enumerate(seq):
+            contrib[q].append((u, t, kv))
+    order = {}
+    for q, lst in contrib.items():
+        if name in (NAIVE_ASC, DESCENDING):
+            lst = sorted(lst, key=lambda e: e[2])        # ascending KV
+        else:
+            lst = sorted(lst, key=lambda e: e[1])        # step (phase, step) order
+        order[q] = [(u, t) for (u, t, _kv) in lst]
+    return order
+
+
+def positions(name: str, N: int, causal: bool):
+    """Per-head table: list per unit of (kv, q, position, n_contributors)."""
+    us = units(name, N, causal)
+    order = accumulation_order(name, N, causal)
+    pos = {}
+    for q, lst in order.items():
+        for p, ut in enumerate(lst):
+            pos[ut] = (p, len(lst))
+    return [[(kv, q) + pos[(u, t)] for t, (kv, q) in enumerate(seq)]
+            for u, seq in enumerate(us)]
+
+
+def packed_table(name: str, n_heads: int, N: int, causal: bool, num_slots: int):
+    """Whole-grid table: per CTA slot, the list of (head, kv, q, position,
+    n_contributors) it runs, in order.
+
+    Heads are taken in order, each head's units in consecutive global unit
+    numbers; global unit g runs on slot g mod num_slots, in round g div
+    num_slots.  (The pages only say that later heads follow; this static
+    round-robin packing is the plainest reading.)
+    """
+    per_head = positions(name, N, causal)
+    U = len(per_head)
+    slots = [[] for _ in range(num_slots)]
+    for hd in range(n_heads):
+        for k in range(U):
+            g = hd * U + k
+            slots[g % num_slots].extend((hd,) + e for e in per_head[k])
+    return slots
