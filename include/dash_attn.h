@@ -1,0 +1,160 @@
+/*
+ * dash_attn.h -- C ABI of the deterministic attention backward for B200.
+ *
+ * The library computes the FlashAttention-style backward pass of softmax
+ * attention (dQ, dK, dV from Q, K, V, O, dO and the row log-sum-exp) with a
+ * persistent sm_100a kernel.  Each CTA runs whole KV-tile chains with dK/dV
+ * resident in tensor memory; dQ is accumulated in fp32 through per-block
+ * integer tickets so that the partials of every dQ block are added in the
+ * fixed order that the chosen schedule defines.  With the same shape, mask,
+ * schedule and SM count, results are bitwise identical from run to run.
+ *
+ * Sources (cited by page title and section):
+ *   "Resumen Técnico: DASH – Programación de Atención Determinista para el
+ *    Entrenamiento de LLM de Alto Rendimiento" (the DASH technical summary):
+ *   §1   deterministic backward = fixed dQ accumulation order; the serialised
+ *        baseline and its nondeterministic counterpart
+ *   §2.1 the DAG model: compute and reduction phases, accumulation-order
+ *        edges, critical path objective, one KV tile per SM as a chain
+ *   §2.2.A descending Q-tile iteration; §2.2.B shift scheduling (full masks),
+ *        symmetric shift (causal masks) and the zero-weight-edge lemma
+ *   §5   the choice between heuristic and optimal schedules is left to the user
+ * The pages print no interface and no formulas: the signatures below and the
+ * attention definitions are this library's own.
+ *
+ * Conventions for every GPU entry point:
+ *   - Tensors are caller-owned DEVICE memory on the current CUDA device.
+ *     q, k, v, o, dout, dq, dk, dv: bf16, contiguous [B, H, S, D], 16-byte
+ *     aligned.  lse: fp32 [B, H, S], natural log of sum_j exp(scale * q.k_j).
+ *     The softmax scale is 1/sqrt(D).  Causal masks are top-left aligned:
+ *     query i attends to keys j <= i.
+ *   - Supported shapes: D in {64, 128}, S a positive multiple of 128,
+ *     B * H * S < 2^31.  Other shapes return DASH_ERR_UNSUPPORTED.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     asynchronous: DASH_OK means the work was enqueued.  Argument and launch
+ *     errors are returned at once; errors found on the device (a spin wait
+ *     that ran out) are reported by dash_attn_sync_status().
+ *   - The library owns its workspace (fp32 dQ accumulator, tickets, the
+ *     per-row Delta and scaled LSE, an error word) and caches it per
+ *     (device, stream); schedule tables are cached per shape.  Calls on
+ *     different streams use different workspaces.  Workspace memory is
+ *     released by dash_release_workspace().
+ */
+#ifndef DASH_ATTN_H_
+#define DASH_ATTN_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DASH_SCHED_NAIVE_ASC = 0,   /* §1 baseline: Q ascending, dQ order ascending KV       */
+  DASH_SCHED_DESCENDING = 1,  /* §2.2.A: Q tiles last to first, dQ order ascending KV  */
+  DASH_SCHED_SHIFT = 2,       /* §2.2.B full masks: cyclic shift, conflict-free order  */
+  DASH_SCHED_SYM_SHIFT = 3,   /* §2.2.B causal masks: KV i and N-1-i folded, 2 phases  */
+  DASH_SCHED_ATOMIC = 4       /* §1 nondeterministic counterpart: fp32 atomic dQ adds  */
+} dash_schedule_t;
+
+typedef enum {
+  DASH_OK = 0,
+  DASH_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, bad enum, negative size   */
+  DASH_ERR_UNSUPPORTED = 2,   /* shape or schedule/mask combination not provided       */
+  DASH_ERR_CUDA = 3,          /* a CUDA runtime call failed                            */
+  DASH_ERR_TIMEOUT = 4,       /* a device spin wait ran out (see dash_attn_sync_status)*/
+  DASH_ERR_OOM = 5,           /* workspace allocation failed                           */
+  DASH_ERR_SCHEDULE = 6       /* schedule table failed validation (e.g. would deadlock)*/
+} dash_status_t;
+
+/*
+ * Forward pass, provided only to produce O and LSE for the backward.
+ * o: bf16 [B,H,S,D] output.  lse: fp32 [B,H,S] output (natural log).
+ * Computes O = softmax(scale * Q K^T + mask) V with fp32 accumulation.
+ */
+int dash_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                  int B, int H, int S, int D, int causal, void* stream);
+
+/*
+ * Backward pass (DASH summary §1, §2.1, §2.2).
+ * Inputs q, k, v, o, dout (bf16 [B,H,S,D]) and lse (fp32 [B,H,S]); outputs
+ * dq, dk, dv (bf16 [B,H,S,D]), fully overwritten.
+ *   dV_j = sum_i P_ij dO_i,  dS_ij = P_ij (dO_i.v_j - dO_i.O_i),
+ *   dQ_i = scale sum_j dS_ij k_j,  dK_j = scale sum_i dS_ij q_i,
+ *   with P_ij = exp(scale q_i.k_j - LSE_i) (0 where masked).
+ * schedule: a dash_schedule_t.  SHIFT needs causal == 0; SYM_SHIFT needs
+ * causal == 1 and an even number of 128-row tiles.  Every schedule except
+ * ATOMIC is deterministic: dQ partials are added in fp32 in the schedule's
+ * fixed order, then rounded once to bf16.
+ */
+int dash_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                  const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                  int B, int H, int S, int D, int causal, int schedule, void* stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the device error word of
+ * that stream's workspace: DASH_ERR_TIMEOUT if a ticket or pipeline wait of a
+ * previous backward on this stream ran out (its outputs are then invalid),
+ * DASH_ERR_CUDA if the stream reported an error, else DASH_OK.
+ */
+int dash_attn_sync_status(void* stream);
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char* dash_status_string(int status);
+
+/*
+ * Upper bound, in microseconds, of every device spin wait of later launches
+ * (ticket waits and pipeline waits).  Default 10 s, or the environment
+ * variable DASH_SPIN_LIMIT_US when set.  us <= 0 restores the default.
+ */
+int dash_set_spin_limit_us(long long us);
+
+/* Number of persistent CTAs the backward uses on `device` for head dim D. */
+int dash_bwd_num_ctas(int device, int D, int* num_ctas);
+
+/* Frees every cached workspace and schedule table of the current device
+ * (synchronises the device first). */
+int dash_release_workspace(void);
+
+/* ---------------------------------------------------------------------------
+ * Host-only entry points (no GPU needed).
+ */
+
+/*
+ * Schedule table of a whole grid (DASH summary §2.2), in CTA order.
+ * n_heads = B*H heads of N = S/128 tiles on num_ctas persistent CTAs.
+ * If rows != NULL, writes up to cap rows of 6 ints:
+ *   (cta, head, kv_tile, q_tile, position_in_dQ_order, chain_index).
+ * Returns the total number of rows (pairs), or a negative dash_status_t
+ * (-DASH_ERR_UNSUPPORTED, -DASH_ERR_SCHEDULE if validation fails).
+ */
+long long dash_sched_table(int n_heads, int N, int causal, int schedule, int num_ctas,
+                           int* rows, long long cap);
+
+/*
+ * DAG simulation of a schedule table (DASH summary §2.1): per pair the events
+ * start, partial ready, reduction start, reduction done; arcs of weight
+ * w_compute (tile compute) and w_reduce (ordered reduction), zero-weight
+ * accumulation-order and chain arcs, and with dq_buffers >= 1 at most that
+ * many partials in flight per CTA (<= 0: unbounded).  Outputs (any may be
+ * NULL): critical_path (longest path), makespan (latest end of a compute
+ * phase), bubble_time (sum over used CTAs of critical_path minus the CTA's
+ * compute time), stalls (pairs whose partial waited for a free buffer).
+ */
+int dash_sched_simulate(int n_heads, int N, int causal, int schedule, int num_ctas,
+                        double w_compute, double w_reduce, int dq_buffers,
+                        double* critical_path, double* makespan, double* bubble_time,
+                        long long* stalls);
+
+/*
+ * Longest paths of a general DAG with n_nodes nodes and n_edges weighted
+ * edges src[e] -> dst[e] (weight w[e]); host arrays.  Writes depth[n] (longest
+ * path ending at the node), height[n] (longest path starting there) and *cp
+ * (any may be NULL).  Used to check the lemma of DASH summary §2.2.B.
+ * Returns DASH_ERR_INVALID_ARG on a cycle or an out-of-range node.
+ */
+int dash_dag_longest_path(int n_nodes, int n_edges, const int* src, const int* dst,
+                          const double* w, double* depth, double* height, double* cp);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DASH_ATTN_H_ */

@@ -119,3 +119,45 @@ def rel_fro(x, ref) -> float:
     den = np.linalg.norm(ref.ravel())
     num = np.linalg.norm((x - ref).ravel())
     return float(num / den) if den > 0 else float(num)
+
+
+def head_backward_rows(q, k, v, do, causal: bool, scale: float, rows_q, rows_kv, chunk=1024):
+    """The backward of one head evaluated only at chosen rows, for heads too
+    large to hold S x S matrices: dQ at query rows ``rows_q`` and dK, dV at
+    key rows ``rows_kv``, each row from the same definitions as
+    ``head_backward``.
+
+    dK_j and dV_j sum over every query i, so O_i, LSE_i and Delta_i are first
+    formed for all rows; those per-row quantities are independent of one
+    another and are computed ``chunk`` rows at a time only to bound memory.
+    Returns (dq [len(rows_q), D], dk, dv [len(rows_kv), D]).
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    S, D = q.shape
+    rows_q = np.asarray(rows_q)
+    rows_kv = np.asarray(rows_kv)
+    keys = np.arange(S)
+    lse = np.empty(S)
+    o = np.empty((S, D))
+    for a in range(0, S, chunk):
+        i = np.arange(a, min(S, a + chunk))
+        allowed = (keys[None, :] <= i[:, None]) if causal else np.ones((len(i), S), bool)
+        s = np.where(allowed, scale * (q[i] @ k.T), -np.inf)
+        m = s.max(axis=1, keepdims=True)
+        lse[i] = (m + np.log(np.exp(s - m).sum(axis=1, keepdims=True)))[:, 0]
+        o[i] = np.where(allowed, np.exp(s - lse[i][:, None]), 0.0) @ v
+    delta = (do * o).sum(axis=1)
+    # dQ rows
+    allowed = (keys[None, :] <= rows_q[:, None]) if causal else np.ones((len(rows_q), S), bool)
+    s = np.where(allowed, scale * (q[rows_q] @ k.T), -np.inf)
+    p = np.where(allowed, np.exp(s - lse[rows_q][:, None]), 0.0)
+    ds = p * (do[rows_q] @ v.T - delta[rows_q][:, None])
+    dq = scale * (ds @ k)
+    # dK, dV rows (columns j of P for all queries i)
+    allowed = (keys[:, None] >= rows_kv[None, :]) if causal else np.ones((S, len(rows_kv)), bool)
+    s = np.where(allowed, scale * (q @ k[rows_kv].T), -np.inf)
+    p = np.where(allowed, np.exp(s - lse[:, None]), 0.0)
+    dv = p.T @ do
+    ds = p * (do @ v[rows_kv].T - delta[:, None])
+    dk = scale * (ds.T @ q)
+    return dq, dk, dv

@@ -1,0 +1,182 @@
+"""ctypes binding of libdash_attn.so (argument marshalling only).
+
+Every step of the backward runs in the library's CUDA kernels; this module
+turns torch tensors into pointers and a stream handle, and raises
+``DashError`` on a non-zero status.  It never falls back to another
+implementation: if the library is missing or fails to load, ``load()``
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libdash_attn.so")
+
+SCHEDULES = {"naive_asc": 0, "descending": 1, "shift": 2, "sym_shift": 3, "atomic": 4}
+STATUS = {0: "DASH_OK", 1: "DASH_ERR_INVALID_ARG", 2: "DASH_ERR_UNSUPPORTED", 3: "DASH_ERR_CUDA",
+          4: "DASH_ERR_TIMEOUT", 5: "DASH_ERR_OOM", 6: "DASH_ERR_SCHEDULE"}
+
+EXPORTS = ("dash_attn_fwd", "dash_attn_bwd", "dash_attn_sync_status", "dash_status_string",
+           "dash_set_spin_limit_us", "dash_bwd_num_ctas", "dash_release_workspace",
+           "dash_sched_table", "dash_sched_simulate", "dash_dag_longest_path")
+
+
+class DashError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(status, status)}")
+        self.status = status
+
+
+_lib = None
+
+
+def load(path: str | None = None):
+    """Load (building first if absent or stale) the shared library."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    if path is None:
+        from . import build as _build
+        try:
+            _build.build()
+        except Exception as e:  # no compiler on this machine: use what is there
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"libdash_attn.so is missing and could not be built: {e}")
+        path = LIB_PATH
+    lib = ctypes.CDLL(path)
+    vp, i, ll, d = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_double
+    P = ctypes.POINTER
+    lib.dash_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, vp]
+    lib.dash_attn_bwd.argtypes = [vp] * 9 + [i, i, i, i, i, i, vp]
+    lib.dash_attn_sync_status.argtypes = [vp]
+    lib.dash_status_string.argtypes = [i]
+    lib.dash_status_string.restype = ctypes.c_char_p
+    lib.dash_set_spin_limit_us.argtypes = [ll]
+    lib.dash_bwd_num_ctas.argtypes = [i, i, P(i)]
+    lib.dash_release_workspace.argtypes = []
+    lib.dash_sched_table.argtypes = [i, i, i, i, i, vp, ll]
+    lib.dash_sched_table.restype = ll
+    lib.dash_sched_simulate.argtypes = [i, i, i, i, i, d, d, i, P(d), P(d), P(d), P(ll)]
+    lib.dash_dag_longest_path.argtypes = [i, i, vp, vp, vp, vp, vp, P(d)]
+    for name in EXPORTS:
+        if name not in ("dash_status_string", "dash_sched_table"):
+            getattr(lib, name).restype = ctypes.c_int
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise DashError(rc, what)
+
+
+def _stream_handle(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _sched_id(schedule) -> int:
+    return SCHEDULES[schedule] if isinstance(schedule, str) else int(schedule)
+
+
+def dash_status_string(status: int) -> str:
+    return load().dash_status_string(int(status)).decode()
+
+
+def dash_attn_fwd(q, k, v, causal: bool, out=None, lse=None, stream=None):
+    """O, LSE = attention forward (bf16 [B,H,S,D] CUDA tensors)."""
+    import torch
+    B, H, S, D = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    rc = load().dash_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S, D,
+                              int(bool(causal)), _stream_handle(stream))
+    _check(rc, "dash_attn_fwd")
+    return out, lse
+
+
+def dash_attn_bwd(q, k, v, o, do, lse, causal: bool, schedule="shift", dq=None, dk=None,
+                  dv=None, stream=None):
+    """dQ, dK, dV of attention (bf16 [B,H,S,D], lse fp32 [B,H,S]; CUDA tensors)."""
+    import torch
+    for t in (q, k, v, o, do, lse):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("inputs must be contiguous CUDA tensors")
+    B, H, S, D = q.shape
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    rc = load().dash_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
+                              _ptr(dk), _ptr(dv), B, H, S, D, int(bool(causal)),
+                              _sched_id(schedule), _stream_handle(stream))
+    _check(rc, "dash_attn_bwd")
+    return dq, dk, dv
+
+
+def dash_attn_sync_status(stream=None) -> int:
+    return int(load().dash_attn_sync_status(_stream_handle(stream)))
+
+
+def dash_set_spin_limit_us(us: int) -> None:
+    _check(load().dash_set_spin_limit_us(int(us)), "dash_set_spin_limit_us")
+
+
+def dash_bwd_num_ctas(device: int = 0, D: int = 128) -> int:
+    n = ctypes.c_int(0)
+    _check(load().dash_bwd_num_ctas(device, D, ctypes.byref(n)), "dash_bwd_num_ctas")
+    return n.value
+
+
+def dash_release_workspace() -> None:
+    _check(load().dash_release_workspace(), "dash_release_workspace")
+
+
+def dash_sched_table(n_heads: int, N: int, causal: bool, schedule, num_ctas: int):
+    """Rows (cta, head, kv, q, position, chain_index) as a list of tuples."""
+    lib = load()
+    sid = _sched_id(schedule)
+    n = lib.dash_sched_table(n_heads, N, int(bool(causal)), sid, num_ctas, None, 0)
+    if n < 0:
+        raise DashError(int(-n), "dash_sched_table")
+    buf = (ctypes.c_int * (6 * n))()
+    lib.dash_sched_table(n_heads, N, int(bool(causal)), sid, num_ctas, buf, n)
+    flat = list(buf)
+    return [tuple(flat[6 * r: 6 * r + 6]) for r in range(n)]
+
+
+def dash_sched_simulate(n_heads: int, N: int, causal: bool, schedule, num_ctas: int,
+                        w_compute: float, w_reduce: float, dq_buffers: int = 0):
+    """(critical_path, makespan, bubble_time, stalls) of a schedule's DAG."""
+    cp, mk, bt = ctypes.c_double(), ctypes.c_double(), ctypes.c_double()
+    st = ctypes.c_longlong()
+    rc = load().dash_sched_simulate(n_heads, N, int(bool(causal)), _sched_id(schedule), num_ctas,
+                                    float(w_compute), float(w_reduce), int(dq_buffers),
+                                    ctypes.byref(cp), ctypes.byref(mk), ctypes.byref(bt),
+                                    ctypes.byref(st))
+    _check(rc, "dash_sched_simulate")
+    return cp.value, mk.value, bt.value, st.value
+
+
+def dash_dag_longest_path(n_nodes: int, edges):
+    """(cp, depth list, height list) of a weighted DAG given as (u, v, w) edges."""
+    m = len(edges)
+    src = (ctypes.c_int * max(m, 1))(*[e[0] for e in edges])
+    dst = (ctypes.c_int * max(m, 1))(*[e[1] for e in edges])
+    w = (ctypes.c_double * max(m, 1))(*[float(e[2]) for e in edges])
+    depth = (ctypes.c_double * max(n_nodes, 1))()
+    height = (ctypes.c_double * max(n_nodes, 1))()
+    cp = ctypes.c_double()
+    rc = load().dash_dag_longest_path(n_nodes, m, src, dst, w, depth, height, ctypes.byref(cp))
+    _check(rc, "dash_dag_longest_path")
+    return cp.value, list(depth)[:n_nodes], list(height)[:n_nodes]

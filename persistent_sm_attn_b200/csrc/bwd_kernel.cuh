@@ -1,0 +1,435 @@
+// Persistent deterministic attention backward for sm_100a.
+//
+// One CTA per SM runs the chains its schedule table lists ("Resumen Técnico:
+// DASH ..." §2.1: all pairs of one KV tile run back to back on one SM, with
+// the dK/dV accumulators on chip).  Per (KV tile j, Q tile i) pair:
+//
+//   S^T  = K_j Q_i^T                  tcgen05.mma, TMEM cols [0,128)
+//   dP^T = V_j dO_i^T                 tcgen05.mma, TMEM cols [128,256)
+//   P^T  = exp(scale S^T - LSE_i),  dS^T = P^T (dP^T - Delta_i)   (softmax warps -> smem)
+//   dV_j += P^T dO_i,  dK_j += dS^T Q_i      tcgen05.mma into TMEM (resident per chain)
+//   dQp  = dS K_j                     tcgen05.mma into TMEM
+//   ordered reduction of dQp into the fp32 accumulator of block (b,h,i): wait
+//   until the block's ticket equals this pair's position, add, publish, bump
+//   the ticket (§1: the fixed accumulation order is what makes dQ bitwise
+//   reproducible; §2.2 chooses the order).  The last contributor rounds the
+//   sum once to bf16 and writes dQ.
+//
+// Warp roles (320 threads): warp 0 TMA producer, warp 1 MMA issuer and TMEM
+// owner, warps 2-5 softmax / dS, warps 6-9 dQ reduction and the dK/dV
+// epilogue.  TMEM lane quarter of a warp is (warp % 4), so each group of four
+// consecutive warps covers the 128 lanes.
+//
+// Shared-memory tiles are [128 rows][D] bf16 stored as D/64 column blocks of
+// 128 rows x 128 bytes with the 128-byte swizzle (the layout a TMA load with
+// SWIZZLE_128B and a 64 x 128 box produces).  The same bytes serve as a
+// K-major operand (rows = M or N, contiguous along K) or as an MN-major one
+// (rows = K, contiguous along M or N): leading byte offset 16 KiB between
+// 64-element column blocks, stride byte offset 1 KiB between 8-row groups.
+#pragma once
+#include "ptx.cuh"
+
+namespace dash {
+
+struct BwdParams {
+  const float* lse2;      // [B*H*S] LSE * log2(e)
+  const float* delta;     // [B*H*S] Delta_i = dO_i . O_i (fp32)
+  const int* cta_off;     // [grid + 1]
+  const int4* chains;     // {bh, kv, pair_off, pair_cnt}
+  const uint32_t* pairs;  // q | position << 16
+  float* acc;             // fp32 dQ accumulator, per block [D/4][128][4]
+  uint32_t* tickets;      // [B*H*N]
+  unsigned* err;          // device error word (accumulates until read by the host)
+  unsigned* abort_flag;   // per-launch: set by the first timeout, cleared before each launch
+  __nv_bfloat16* dq;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  int S, N, causal;
+  float scale, scale_log2;
+  unsigned long long spin_ns;
+};
+
+template <int D>
+struct BwdCfg {
+  static constexpr int kThreads = 320;
+  static constexpr int kTile = 128 * D * 2;              // one [128][D] bf16 tile
+  static constexpr int kStages = (D == 64) ? 2 : 1;      // Q/dO pipeline depth
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + kTile;
+  static constexpr int OFF_Q = OFF_V + kTile;
+  static constexpr int OFF_DO = OFF_Q + kStages * kTile;
+  static constexpr int OFF_PT = OFF_DO + kStages * kTile;  // P^T  [128 kv][128 q]
+  static constexpr int OFF_DST = OFF_PT + 32768;           // dS^T [128 kv][128 q]
+  static constexpr int OFF_LSE = OFF_DST + 32768;          // kStages x 128 fp32
+  static constexpr int OFF_DEL = OFF_LSE + kStages * 512;
+  static constexpr int OFF_BAR = OFF_DEL + kStages * 512;
+  static constexpr int kBars = 14 + 2 * kStages;
+  static constexpr int OFF_TMEM_SLOT = OFF_BAR + kBars * 8;
+  static constexpr int kSmemBytes = OFF_TMEM_SLOT + 16 + 1024;  // + alignment slack
+  // TMEM columns
+  static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 256 + D;
+  static constexpr uint32_t TM_DQ = (D == 64) ? 384 : 128;  // D=128 shares dP^T's columns
+  static constexpr bool kDqAliasesDp = (D != 64);
+};
+
+// barrier indices
+enum {
+  B_KV_FULL = 0, B_KV_EMPTY, B_S_FULL, B_DP_FULL, B_DS_READY, B_DS_FREE, B_DQ_FULL, B_DQ_EMPTY,
+  B_DKDV_FULL, B_DKDV_EMPTY, B_FINAL, B_Q_FULL0 = 14
+};
+
+template <int D, bool kAtomic>
+__global__ void __launch_bounds__(320, 1)
+    dash_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                    const BwdParams p) {
+  using namespace dev;
+  using C = BwdCfg<D>;
+  constexpr int ST = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sb = (raw + 1023u) & ~1023u;
+  uint8_t* gb = smem_raw + (sb - raw);
+  const uint32_t sK = sb + C::OFF_K, sV = sb + C::OFF_V, sQ = sb + C::OFF_Q, sDO = sb + C::OFF_DO;
+  const uint32_t sPt = sb + C::OFF_PT, sDSt = sb + C::OFF_DST;
+  const float* lse_s = reinterpret_cast<const float*>(gb + C::OFF_LSE);
+  const float* del_s = reinterpret_cast<const float*>(gb + C::OFF_DEL);
+  const uint32_t bar0 = sb + C::OFF_BAR;
+  auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  auto Q_FULL = [&](int s) { return BAR(B_Q_FULL0 + s); };
+  auto Q_EMPTY = [&](int s) { return BAR(B_Q_FULL0 + ST + s); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gb + C::OFF_TMEM_SLOT);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint64_t lim = p.spin_ns;
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR(B_KV_FULL), 1);
+    mbar_init(BAR(B_KV_EMPTY), 1);
+    mbar_init(BAR(B_S_FULL), 1);
+    mbar_init(BAR(B_DP_FULL), 1);
+    mbar_init(BAR(B_DS_READY), 128);
+    mbar_init(BAR(B_DS_FREE), 1);
+    mbar_init(BAR(B_DQ_FULL), 1);
+    mbar_init(BAR(B_DQ_EMPTY), 128);
+    mbar_init(BAR(B_DKDV_FULL), 1);
+    mbar_init(BAR(B_DKDV_EMPTY), 128);
+    mbar_init(BAR(B_FINAL), 1);
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(Q_FULL(s), 1);
+      mbar_init(Q_EMPTY(s), 1);
+    }
+    fence_mbar_init();
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+    prefetch_tmap(&tmDO);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int cbeg = p.cta_off[blockIdx.x], cend = p.cta_off[blockIdx.x + 1];
+  const int S = p.S, N = p.N;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int it = 0, cn = 0;
+      for (int ci = cbeg; ci < cend; ++ci, ++cn) {
+        const int4 ch = p.chains[ci];
+        if (cn > 0) mbar_wait(BAR(B_KV_EMPTY), (cn - 1) & 1, lim, p.err, p.abort_flag);
+        mbar_expect_tx(BAR(B_KV_FULL), 2 * C::kTile);
+        const int row_kv = ch.x * S + ch.y * 128;
+#pragma unroll
+        for (int cb = 0; cb < D / 64; ++cb) {
+          tma_load_2d(sK + cb * 16384, &tmK, cb * 64, row_kv, BAR(B_KV_FULL));
+          tma_load_2d(sV + cb * 16384, &tmV, cb * 64, row_kv, BAR(B_KV_FULL));
+        }
+        for (int t = 0; t < ch.w; ++t, ++it) {
+          const int q = (int)(p.pairs[ch.z + t] & 0xffffu);
+          const int s = it % ST;
+          if (it >= ST) mbar_wait(Q_EMPTY(s), ((it / ST) - 1) & 1, lim, p.err, p.abort_flag);
+          mbar_expect_tx(Q_FULL(s), 2 * C::kTile + 1024);
+          const int row_q = ch.x * S + q * 128;
+#pragma unroll
+          for (int cb = 0; cb < D / 64; ++cb) {
+            tma_load_2d(sQ + s * C::kTile + cb * 16384, &tmQ, cb * 64, row_q, Q_FULL(s));
+            tma_load_2d(sDO + s * C::kTile + cb * 16384, &tmDO, cb * 64, row_q, Q_FULL(s));
+          }
+          bulk_load(sb + C::OFF_LSE + s * 512, p.lse2 + row_q, 512, Q_FULL(s));
+          bulk_load(sb + C::OFF_DEL + s * 512, p.delta + row_q, 512, Q_FULL(s));
+        }
+      }
+      // drain: every issued load has landed before the CTA can exit
+      for (int s = 0; s < ST && s < it; ++s) {
+        const int last_use = ((it - 1 - s) / ST) * ST + s;
+        mbar_wait(Q_FULL(s), (last_use / ST) & 1, lim, p.err, p.abort_flag);
+      }
+      if (cn > 0) mbar_wait(BAR(B_KV_FULL), (cn - 1) & 1, lim, p.err, p.abort_flag);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t ID_SS = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t ID_KV = idesc_bf16_f32(128, D, 0, 1);
+      constexpr uint32_t ID_Q = idesc_bf16_f32(128, D, 1, 1);
+      const uint32_t tS = tmem + C::TM_S, tDP = tmem + C::TM_DP, tDV = tmem + C::TM_DV,
+                     tDK = tmem + C::TM_DK, tDQ = tmem + C::TM_DQ;
+      int it = 0, cn = 0;
+      for (int ci = cbeg; ci < cend; ++ci, ++cn) {
+        const int cnt = p.chains[ci].w;
+        mbar_wait(BAR(B_KV_FULL), cn & 1, lim, p.err, p.abort_flag);
+        if (cn > 0) mbar_wait(BAR(B_DKDV_EMPTY), (cn - 1) & 1, lim, p.err, p.abort_flag);
+        tc_fence_after();
+        for (int t = 0; t < cnt; ++t, ++it) {
+          const int s = it % ST;
+          const uint32_t q_s = sQ + s * C::kTile, do_s = sDO + s * C::kTile;
+          mbar_wait(Q_FULL(s), (it / ST) & 1, lim, p.err, p.abort_flag);
+          tc_fence_after();
+          // S^T = K Q^T : M = kv, N = q, K = D (both operands K-major)
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            tc_mma_ss(tS, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(q_s + off, 16, 1024), ID_SS,
+                      kk > 0);
+          }
+          tc_commit(BAR(B_S_FULL));
+          if (C::kDqAliasesDp && it > 0) {
+            mbar_wait(BAR(B_DQ_EMPTY), (it - 1) & 1, lim, p.err, p.abort_flag);
+            tc_fence_after();
+          }
+          // dP^T = V dO^T
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            tc_mma_ss(tDP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(do_s + off, 16, 1024),
+                      ID_SS, kk > 0);
+          }
+          tc_commit(BAR(B_DP_FULL));
+          mbar_wait(BAR(B_DS_READY), it & 1, lim, p.err, p.abort_flag);
+          tc_fence_after();
+          // dV += P^T dO ; dK += dS^T Q : M = kv, N = D, K = q (A K-major, B MN-major)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t offA = (kk >> 2) * 16384 + (kk & 3) * 32;
+            const uint32_t offB = kk * 2048;
+            tc_mma_ss(tDV, sdesc_sw128(sPt + offA, 16, 1024), sdesc_sw128(do_s + offB, 16384, 1024),
+                      ID_KV, (t > 0 || kk > 0) ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t offA = (kk >> 2) * 16384 + (kk & 3) * 32;
+            const uint32_t offB = kk * 2048;
+            tc_mma_ss(tDK, sdesc_sw128(sDSt + offA, 16, 1024), sdesc_sw128(q_s + offB, 16384, 1024),
+                      ID_KV, (t > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(Q_EMPTY(s));
+          if (t == cnt - 1) tc_commit(BAR(B_DKDV_FULL));
+          if (!C::kDqAliasesDp && it > 0) {
+            mbar_wait(BAR(B_DQ_EMPTY), (it - 1) & 1, lim, p.err, p.abort_flag);
+            tc_fence_after();
+          }
+          // dQp = dS K : M = q, N = D, K = kv (both operands MN-major)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            tc_mma_ss(tDQ, sdesc_sw128(sDSt + kk * 2048, 16384, 1024),
+                      sdesc_sw128(sK + kk * 2048, 16384, 1024), ID_Q, kk > 0);
+          }
+          tc_commit(BAR(B_DQ_FULL));
+          tc_commit(BAR(B_DS_FREE));
+        }
+        tc_commit(BAR(B_KV_EMPTY));
+      }
+      // drain: all issued MMAs complete before TMEM is released
+      tc_commit(BAR(B_FINAL));
+      mbar_wait(BAR(B_FINAL), 0, lim, p.err, p.abort_flag);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ softmax / dS
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // KV row of the tile
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const float sl2 = p.scale_log2;
+    int it = 0;
+    for (int ci = cbeg; ci < cend; ++ci) {
+      const int4 ch = p.chains[ci];
+      for (int t = 0; t < ch.w; ++t, ++it) {
+        const int q = (int)(p.pairs[ch.z + t] & 0xffffu);
+        const int s = it % ST;
+        mbar_wait(Q_FULL(s), (it / ST) & 1, lim, p.err, p.abort_flag);
+        mbar_wait(BAR(B_S_FULL), it & 1, lim, p.err, p.abort_flag);
+        mbar_wait(BAR(B_DP_FULL), it & 1, lim, p.err, p.abort_flag);
+        if (it > 0) mbar_wait(BAR(B_DS_FREE), (it - 1) & 1, lim, p.err, p.abort_flag);
+        tc_fence_after();
+        const bool diag = p.causal && (q == ch.y);
+        const float* lse_t = lse_s + s * 128;
+        const float* del_t = del_s + s * 128;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t sv[32], dv[32];
+          tmem_ld32x2(tmem + lane_off + C::TM_S + c * 32, tmem + lane_off + C::TM_DP + c * 32, sv,
+                      dv);
+          uint32_t pk[16], dk[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const int qc = c * 32 + j;
+            float p0 = exp2f(fmaf(__uint_as_float(sv[j]), sl2, -lse_t[qc]));
+            float p1 = exp2f(fmaf(__uint_as_float(sv[j + 1]), sl2, -lse_t[qc + 1]));
+            if (diag) {
+              if (qc < r) p0 = 0.f;
+              if (qc + 1 < r) p1 = 0.f;
+            }
+            const float d0 = p0 * (__uint_as_float(dv[j]) - del_t[qc]);
+            const float d1 = p1 * (__uint_as_float(dv[j + 1]) - del_t[qc + 1]);
+            pk[j >> 1] = pack_bf16x2(p0, p1);
+            dk[j >> 1] = pack_bf16x2(d0, d1);
+          }
+          const uint32_t row = (uint32_t)(c >> 1) * 16384 + (uint32_t)(r >> 3) * 1024 +
+                               (uint32_t)(r & 7) * 128;
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const uint32_t chunk = (uint32_t)((((c & 1) * 4 + m) ^ (r & 7)) * 16);
+            st_shared_v4(sPt + row + chunk, pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
+            st_shared_v4(sDSt + row + chunk, dk[4 * m], dk[4 * m + 1], dk[4 * m + 2],
+                         dk[4 * m + 3]);
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(BAR(B_DS_READY));
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ dQ reduction + dK/dV epilogue
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // row of the tile (Q row for dQ, KV row for dK/dV)
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    int it = 0, cn = 0;
+    for (int ci = cbeg; ci < cend; ++ci, ++cn) {
+      const int4 ch = p.chains[ci];
+      for (int t = 0; t < ch.w; ++t, ++it) {
+        const uint32_t w = p.pairs[ch.z + t];
+        const int q = (int)(w & 0xffffu), pos = (int)(w >> 16);
+        const int ncontrib = p.causal ? q + 1 : N;
+        const bool last = (pos == ncontrib - 1);
+        mbar_wait(BAR(B_DQ_FULL), it & 1, lim, p.err, p.abort_flag);
+        tc_fence_after();
+        float a[D];
+#pragma unroll
+        for (int c2 = 0; c2 < D / 32; ++c2) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_off + C::TM_DQ + c2 * 32, v);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) a[c2 * 32 + j] = __uint_as_float(v[j]);
+        }
+        tc_fence_before();
+        mbar_arrive(BAR(B_DQ_EMPTY));
+        const long long blk = (long long)ch.x * N + q;
+        float4* accp = reinterpret_cast<float4*>(p.acc + blk * 128 * D);
+        if constexpr (!kAtomic) {
+          if (pos > 0) {
+            uint32_t* tk = p.tickets + blk;
+            if (lane == 0) {
+              if (ld_acquire_gpu(tk) != (uint32_t)pos) {
+                const uint64_t t0 = globaltimer();
+                bool ok = false;
+                while (!ok) {
+#pragma unroll 1
+                  for (int i = 0; i < 32 && !ok; ++i) ok = (ld_acquire_gpu(tk) == (uint32_t)pos);
+                  if (!ok && (aborted(p.abort_flag) || globaltimer() - t0 > lim)) {
+                    if (!aborted(p.abort_flag)) raise_timeout(p.err, p.abort_flag, ERR_WHERE_TICKET);
+                    break;
+                  }
+                }
+              }
+            }
+            __syncwarp();
+            (void)ld_acquire_gpu(tk);
+          }
+          if (last) {
+            __nv_bfloat16* out = p.dq + ((size_t)ch.x * S + (size_t)q * 128 + r) * D;
+#pragma unroll
+            for (int c8 = 0; c8 < D / 8; ++c8) {
+              float4 x0 = make_float4(a[8 * c8], a[8 * c8 + 1], a[8 * c8 + 2], a[8 * c8 + 3]);
+              float4 x1 = make_float4(a[8 * c8 + 4], a[8 * c8 + 5], a[8 * c8 + 6], a[8 * c8 + 7]);
+              if (pos > 0) {
+                const float4 o0 = ld_cg_f4(accp + (2 * c8) * 128 + r);
+                const float4 o1 = ld_cg_f4(accp + (2 * c8 + 1) * 128 + r);
+                x0.x = o0.x + x0.x; x0.y = o0.y + x0.y; x0.z = o0.z + x0.z; x0.w = o0.w + x0.w;
+                x1.x = o1.x + x1.x; x1.y = o1.y + x1.y; x1.z = o1.z + x1.z; x1.w = o1.w + x1.w;
+              }
+              const float sc = p.scale;
+              uint4 pk;
+              pk.x = pack_bf16x2(x0.x * sc, x0.y * sc);
+              pk.y = pack_bf16x2(x0.z * sc, x0.w * sc);
+              pk.z = pack_bf16x2(x1.x * sc, x1.y * sc);
+              pk.w = pack_bf16x2(x1.z * sc, x1.w * sc);
+              *reinterpret_cast<uint4*>(out + 8 * c8) = pk;
+            }
+          } else {
+#pragma unroll
+            for (int c4 = 0; c4 < D / 4; ++c4) {
+              float4 x = make_float4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]);
+              if (pos > 0) {
+                const float4 o = ld_cg_f4(accp + c4 * 128 + r);
+                x.x = o.x + x.x; x.y = o.y + x.y; x.z = o.z + x.z; x.w = o.w + x.w;
+              }
+              st_cg_f4(accp + c4 * 128 + r, x);
+            }
+            named_bar_sync(1, 128);
+            if (threadIdx.x == 192) {
+              __threadfence();
+              st_release_gpu(p.tickets + blk, (uint32_t)(pos + 1));
+            }
+          }
+        } else {
+#pragma unroll
+          for (int c4 = 0; c4 < D / 4; ++c4)
+            atomicAdd(accp + c4 * 128 + r,
+                      make_float4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]));
+        }
+      }
+      // chain epilogue: dV_j and scale * dK_j (rows of KV tile ch.y) to global bf16
+      mbar_wait(BAR(B_DKDV_FULL), cn & 1, lim, p.err, p.abort_flag);
+      tc_fence_after();
+      const size_t row = (size_t)ch.x * S + (size_t)ch.y * 128 + r;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t col = which ? C::TM_DK : C::TM_DV;
+        const float sc = which ? p.scale : 1.0f;
+        __nv_bfloat16* out = (which ? p.dk : p.dv) + row * D;
+#pragma unroll
+        for (int c2 = 0; c2 < D / 32; ++c2) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_off + col + c2 * 32, v);
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8) {
+            uint4 pk;
+            pk.x = pack_bf16x2(__uint_as_float(v[8 * c8]) * sc, __uint_as_float(v[8 * c8 + 1]) * sc);
+            pk.y = pack_bf16x2(__uint_as_float(v[8 * c8 + 2]) * sc, __uint_as_float(v[8 * c8 + 3]) * sc);
+            pk.z = pack_bf16x2(__uint_as_float(v[8 * c8 + 4]) * sc, __uint_as_float(v[8 * c8 + 5]) * sc);
+            pk.w = pack_bf16x2(__uint_as_float(v[8 * c8 + 6]) * sc, __uint_as_float(v[8 * c8 + 7]) * sc);
+            *reinterpret_cast<uint4*>(out + c2 * 32 + c8 * 8) = pk;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(BAR(B_DKDV_EMPTY));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace dash

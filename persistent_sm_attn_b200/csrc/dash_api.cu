@@ -1,0 +1,470 @@
+// C ABI of the deterministic attention backward: argument checks, workspace
+// and schedule-table caches, TMA descriptors and launches.  The operation
+// itself is documented in include/dash_attn.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <map>
+#include <mutex>
+#include <string>
+#include <tuple>
+
+#include "../../include/dash_attn.h"
+#include "aux_kernels.cuh"
+#include "bwd_kernel.cuh"
+#include "sched.h"
+
+namespace {
+
+using dash::BwdCfg;
+using dash::BwdParams;
+
+// ------------------------------------------------------------------ settings
+long long default_spin_us() {
+  const char* e = std::getenv("DASH_SPIN_LIMIT_US");
+  if (e) {
+    const long long v = std::atoll(e);
+    if (v > 0) return v;
+  }
+  return 10LL * 1000 * 1000;
+}
+std::atomic<long long> g_spin_us{0};
+long long spin_us() {
+  long long v = g_spin_us.load();
+  return v > 0 ? v : default_spin_us();
+}
+
+// ------------------------------------------------------------------ caches
+struct Workspace {
+  float* acc = nullptr;
+  size_t acc_bytes = 0;
+  uint32_t* tickets = nullptr;
+  size_t tk_bytes = 0;
+  float* rowbuf = nullptr;  // lse2 then delta, each rows_cap floats
+  size_t rows_cap = 0;
+  unsigned* err = nullptr;   // [0] error word, [1] per-launch abort flag
+};
+
+struct DevTable {
+  int* cta_off = nullptr;
+  int4* chains = nullptr;
+  uint32_t* pairs = nullptr;
+};
+
+std::mutex g_mu;
+std::map<std::pair<int, uintptr_t>, Workspace> g_ws;                  // (device, stream)
+std::map<std::tuple<int, int, int, int, int, int>, DevTable> g_tables;  // device,heads,N,causal,sched,ctas
+std::map<std::pair<int, int>, int> g_num_ctas;                        // (device, D)
+
+#define DASH_CUDA(call)                    \
+  do {                                     \
+    if ((call) != cudaSuccess) return DASH_ERR_CUDA; \
+  } while (0)
+
+int grow(void** p, size_t* have, size_t need) {
+  if (*have >= need) return DASH_OK;
+  if (*p) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return DASH_ERR_CUDA;
+    cudaFree(*p);
+    *p = nullptr;
+    *have = 0;
+  }
+  if (cudaMalloc(p, need) != cudaSuccess) {
+    cudaGetLastError();
+    return DASH_ERR_OOM;
+  }
+  *have = need;
+  return DASH_OK;
+}
+
+int get_workspace(int dev, void* stream, size_t acc_bytes, size_t tk_bytes, size_t rows,
+                  Workspace** out) {
+  Workspace& w = g_ws[{dev, reinterpret_cast<uintptr_t>(stream)}];
+  int rc;
+  if ((rc = grow(reinterpret_cast<void**>(&w.acc), &w.acc_bytes, acc_bytes))) return rc;
+  if ((rc = grow(reinterpret_cast<void**>(&w.tickets), &w.tk_bytes, tk_bytes))) return rc;
+  size_t rb = w.rows_cap * 2 * sizeof(float);
+  if (rows > w.rows_cap) {
+    if ((rc = grow(reinterpret_cast<void**>(&w.rowbuf), &rb, rows * 2 * sizeof(float)))) return rc;
+    w.rows_cap = rows;
+  }
+  if (!w.err) {
+    if (cudaMalloc(&w.err, 2 * sizeof(unsigned)) != cudaSuccess) return DASH_ERR_OOM;
+    if (cudaMemset(w.err, 0, 2 * sizeof(unsigned)) != cudaSuccess) return DASH_ERR_CUDA;
+  }
+  *out = &w;
+  return DASH_OK;
+}
+
+int get_table(int dev, int heads, int N, int causal, int sched, int ctas, DevTable** out) {
+  auto key = std::make_tuple(dev, heads, N, causal, sched, ctas);
+  auto itb = g_tables.find(key);
+  if (itb != g_tables.end()) {
+    *out = &itb->second;
+    return DASH_OK;
+  }
+  dash::Table t;
+  std::string err;
+  if (!dash::build_table(heads, N, causal, sched, ctas, &t, &err)) return DASH_ERR_UNSUPPORTED;
+  if (!dash::validate_table(t, &err)) return DASH_ERR_SCHEDULE;
+  DevTable d;
+  if (cudaMalloc(&d.cta_off, t.cta_off.size() * sizeof(int)) != cudaSuccess ||
+      cudaMalloc(&d.chains, t.chains.size() * sizeof(int4)) != cudaSuccess ||
+      cudaMalloc(&d.pairs, t.pairs.size() * sizeof(uint32_t)) != cudaSuccess) {
+    cudaGetLastError();
+    cudaFree(d.cta_off);
+    cudaFree(d.chains);
+    cudaFree(d.pairs);
+    return DASH_ERR_OOM;
+  }
+  static_assert(sizeof(dash::Chain) == sizeof(int4), "chain layout");
+  DASH_CUDA(cudaMemcpy(d.cta_off, t.cta_off.data(), t.cta_off.size() * sizeof(int),
+                       cudaMemcpyHostToDevice));
+  DASH_CUDA(cudaMemcpy(d.chains, t.chains.data(), t.chains.size() * sizeof(int4),
+                       cudaMemcpyHostToDevice));
+  DASH_CUDA(cudaMemcpy(d.pairs, t.pairs.data(), t.pairs.size() * sizeof(uint32_t),
+                       cudaMemcpyHostToDevice));
+  auto res = g_tables.emplace(key, d);
+  *out = &res.first->second;
+  return DASH_OK;
+}
+
+// ------------------------------------------------------------------ TMA descriptors
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// [rows][D] bf16 viewed with a 64-column x 128-row box and the 128-byte swizzle.
+int make_tmap(CUtensorMap* m, const void* base, long long rows, int D) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return DASH_ERR_CUDA;
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DASH_OK : DASH_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ helpers
+bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_shape(int B, int H, int S, int D) {
+  if (B < 0 || H < 0 || S < 0 || D < 0) return DASH_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return DASH_ERR_UNSUPPORTED;
+  if (S == 0 || S % 128 != 0 || S / 128 > 32767) return DASH_ERR_UNSUPPORTED;
+  if ((long long)B * H * S >= (1LL << 31)) return DASH_ERR_UNSUPPORTED;
+  return DASH_OK;
+}
+
+template <int D, bool kAtomic>
+int num_ctas_for(int dev, int* out) {
+  using C = BwdCfg<D>;
+  auto key = std::make_pair(dev, D * 2 + (kAtomic ? 1 : 0));
+  auto itn = g_num_ctas.find(key);
+  if (itn != g_num_ctas.end()) {
+    *out = itn->second;
+    return DASH_OK;
+  }
+  auto kern = dash::dash_bwd_kernel<D, kAtomic>;
+  DASH_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes));
+  int per_sm = 0, sms = 0;
+  DASH_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, C::kThreads, C::kSmemBytes));
+  DASH_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  if (per_sm < 1) return DASH_ERR_UNSUPPORTED;
+  *out = per_sm * sms;
+  g_num_ctas[key] = *out;
+  return DASH_OK;
+}
+
+template <int D, bool kAtomic>
+int launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+               const float* lse, void* dq, void* dk, void* dv, int B, int H, int S, int causal,
+               int sched, cudaStream_t stream, int dev) {
+  using C = BwdCfg<D>;
+  const int N = S / 128;
+  const long long rows = (long long)B * H * S;
+  int ctas = 0;
+  int rc = num_ctas_for<D, kAtomic>(dev, &ctas);
+  if (rc) return rc;
+  DevTable* tab = nullptr;
+  Workspace* ws = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if ((rc = get_table(dev, B * H, N, causal, sched, ctas, &tab))) return rc;
+    if ((rc = get_workspace(dev, stream, (size_t)rows * D * sizeof(float),
+                            (size_t)B * H * N * sizeof(uint32_t), (size_t)rows, &ws)))
+      return rc;
+  }
+  CUtensorMap tq, tk, tv, tdo;
+  if ((rc = make_tmap(&tq, q, rows, D)) || (rc = make_tmap(&tk, k, rows, D)) ||
+      (rc = make_tmap(&tv, v, rows, D)) || (rc = make_tmap(&tdo, dout, rows, D)))
+    return rc;
+  float* lse2 = ws->rowbuf;
+  float* delta = ws->rowbuf + ws->rows_cap;
+  {
+    const long long threads = rows * (D / 8);
+    const int blocks = (int)((threads + 255) / 256);
+    dash::dash_delta_kernel<D><<<blocks, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, delta,
+        lse2, rows);
+  }
+  DASH_CUDA(cudaMemsetAsync(ws->err + 1, 0, sizeof(unsigned), stream));
+  if (kAtomic) {
+    DASH_CUDA(cudaMemsetAsync(ws->acc, 0, (size_t)rows * D * sizeof(float), stream));
+  } else {
+    DASH_CUDA(cudaMemsetAsync(ws->tickets, 0, (size_t)B * H * N * sizeof(uint32_t), stream));
+  }
+  BwdParams p;
+  p.lse2 = lse2;
+  p.delta = delta;
+  p.cta_off = tab->cta_off;
+  p.chains = tab->chains;
+  p.pairs = tab->pairs;
+  p.acc = ws->acc;
+  p.tickets = ws->tickets;
+  p.err = ws->err;
+  p.abort_flag = ws->err + 1;
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.S = S;
+  p.N = N;
+  p.causal = causal;
+  p.scale = 1.0f / sqrtf((float)D);
+  p.scale_log2 = p.scale * 1.4426950408889634f;
+  p.spin_ns = (unsigned long long)spin_us() * 1000ull;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ctas);
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  DASH_CUDA(cudaLaunchKernelEx(&cfg, dash::dash_bwd_kernel<D, kAtomic>, tq, tk, tv, tdo, p));
+  if (kAtomic) {
+    const long long n_blocks = (long long)B * H * N;
+    const long long threads = n_blocks * 128 * (D / 4);
+    dash::dash_dq_convert<D><<<(int)((threads + 255) / 256), 256, 0, stream>>>(
+        ws->acc, static_cast<__nv_bfloat16*>(dq), n_blocks, p.scale);
+  }
+  DASH_CUDA(cudaGetLastError());
+  return DASH_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* dash_status_string(int s) {
+  switch (s) {
+    case DASH_OK: return "DASH_OK";
+    case DASH_ERR_INVALID_ARG: return "DASH_ERR_INVALID_ARG";
+    case DASH_ERR_UNSUPPORTED: return "DASH_ERR_UNSUPPORTED";
+    case DASH_ERR_CUDA: return "DASH_ERR_CUDA";
+    case DASH_ERR_TIMEOUT: return "DASH_ERR_TIMEOUT";
+    case DASH_ERR_OOM: return "DASH_ERR_OOM";
+    case DASH_ERR_SCHEDULE: return "DASH_ERR_SCHEDULE";
+    default: return "DASH_ERR_UNKNOWN";
+  }
+}
+
+int dash_set_spin_limit_us(long long us) {
+  g_spin_us.store(us > 0 ? us : 0);
+  return DASH_OK;
+}
+
+int dash_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                  int S, int D, int causal, void* stream) {
+  int rc = check_shape(B, H, S, D);
+  if (rc) return rc;
+  if (causal != 0 && causal != 1) return DASH_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !lse)
+    return DASH_ERR_INVALID_ARG;
+  if (B == 0 || H == 0) return DASH_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  dim3 grid(S / 64, B * H);
+  const float sl2 = (1.0f / sqrtf((float)D)) * 1.4426950408889634f;
+  if (D == 64)
+    dash::dash_fwd_kernel<64><<<grid, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+        static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(o), lse, S, causal, sl2);
+  else
+    dash::dash_fwd_kernel<128><<<grid, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+        static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(o), lse, S, causal, sl2);
+  DASH_CUDA(cudaGetLastError());
+  return DASH_OK;
+}
+
+int dash_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                  const float* lse, void* dq, void* dk, void* dv, int B, int H, int S, int D,
+                  int causal, int schedule, void* stream) {
+  int rc = check_shape(B, H, S, D);
+  if (rc) return rc;
+  if (causal != 0 && causal != 1) return DASH_ERR_INVALID_ARG;
+  if (schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_ATOMIC) return DASH_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return DASH_ERR_INVALID_ARG;
+  if (!dash::schedule_supported(schedule, S / 128, causal)) return DASH_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0) return DASH_OK;
+  int dev = 0;
+  DASH_CUDA(cudaGetDevice(&dev));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool atomic = (schedule == DASH_SCHED_ATOMIC);
+  if (D == 64)
+    return atomic ? launch_bwd<64, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
+                                         schedule, st, dev)
+                  : launch_bwd<64, false>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
+                                          schedule, st, dev);
+  return atomic ? launch_bwd<128, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
+                                        schedule, st, dev)
+                : launch_bwd<128, false>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
+                                         schedule, st, dev);
+}
+
+int dash_attn_sync_status(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return DASH_ERR_CUDA;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DASH_ERR_CUDA;
+  unsigned* err = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto itw = g_ws.find({dev, reinterpret_cast<uintptr_t>(stream)});
+    if (itw == g_ws.end()) return DASH_OK;
+    err = itw->second.err;
+  }
+  unsigned h = 0;
+  if (!err) return DASH_OK;
+  if (cudaMemcpy(&h, err, sizeof(unsigned), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return DASH_ERR_CUDA;
+  if (h) {
+    if (cudaMemset(err, 0, sizeof(unsigned)) != cudaSuccess) return DASH_ERR_CUDA;
+    return DASH_ERR_TIMEOUT;
+  }
+  return DASH_OK;
+}
+
+int dash_bwd_num_ctas(int device, int D, int* num_ctas) {
+  if (!num_ctas) return DASH_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return DASH_ERR_UNSUPPORTED;
+  int prev = 0;
+  DASH_CUDA(cudaGetDevice(&prev));
+  DASH_CUDA(cudaSetDevice(device));
+  std::lock_guard<std::mutex> lk(g_mu);
+  const int rc = (D == 64) ? num_ctas_for<64, false>(device, num_ctas)
+                           : num_ctas_for<128, false>(device, num_ctas);
+  cudaSetDevice(prev);
+  return rc;
+}
+
+int dash_release_workspace(void) {
+  int dev = 0;
+  DASH_CUDA(cudaGetDevice(&dev));
+  DASH_CUDA(cudaDeviceSynchronize());
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (auto itw = g_ws.begin(); itw != g_ws.end();) {
+    if (itw->first.first == dev) {
+      cudaFree(itw->second.acc);
+      cudaFree(itw->second.tickets);
+      cudaFree(itw->second.rowbuf);
+      cudaFree(itw->second.err);
+      itw = g_ws.erase(itw);
+    } else {
+      ++itw;
+    }
+  }
+  for (auto itt = g_tables.begin(); itt != g_tables.end();) {
+    if (std::get<0>(itt->first) == dev) {
+      cudaFree(itt->second.cta_off);
+      cudaFree(itt->second.chains);
+      cudaFree(itt->second.pairs);
+      itt = g_tables.erase(itt);
+    } else {
+      ++itt;
+    }
+  }
+  return DASH_OK;
+}
+
+long long dash_sched_table(int n_heads, int N, int causal, int schedule, int num_ctas, int* rows,
+                           long long cap) {
+  dash::Table t;
+  std::string err;
+  if (!dash::build_table(n_heads, N, causal, schedule, num_ctas, &t, &err))
+    return -DASH_ERR_UNSUPPORTED;
+  if (!dash::validate_table(t, &err)) return -DASH_ERR_SCHEDULE;
+  long long n = 0;
+  for (int c = 0; c < t.num_ctas; ++c)
+    for (int ci = t.cta_off[c]; ci < t.cta_off[c + 1]; ++ci) {
+      const dash::Chain& ch = t.chains[ci];
+      for (int i = 0; i < ch.pair_cnt; ++i, ++n) {
+        if (rows && n < cap) {
+          const uint32_t w = t.pairs[ch.pair_off + i];
+          int* r = rows + 6 * n;
+          r[0] = c;
+          r[1] = ch.bh;
+          r[2] = ch.kv;
+          r[3] = dash::pair_q(w);
+          r[4] = dash::pair_pos(w);
+          r[5] = ci;
+        }
+      }
+    }
+  return n;
+}
+
+int dash_sched_simulate(int n_heads, int N, int causal, int schedule, int num_ctas,
+                        double w_compute, double w_reduce, int dq_buffers, double* critical_path,
+                        double* makespan, double* bubble_time, long long* stalls) {
+  if (w_compute < 0 || w_reduce < 0) return DASH_ERR_INVALID_ARG;
+  dash::Table t;
+  std::string err;
+  if (!dash::build_table(n_heads, N, causal, schedule, num_ctas, &t, &err))
+    return DASH_ERR_UNSUPPORTED;
+  if (!dash::validate_table(t, &err)) return DASH_ERR_SCHEDULE;
+  dash::SimResult r;
+  if (!dash::simulate_table(t, w_compute, w_reduce, dq_buffers, &r, &err)) return DASH_ERR_SCHEDULE;
+  if (critical_path) *critical_path = r.critical_path;
+  if (makespan) *makespan = r.makespan;
+  if (bubble_time) *bubble_time = r.bubble_time;
+  if (stalls) *stalls = r.stalls;
+  return DASH_OK;
+}
+
+int dash_dag_longest_path(int n_nodes, int n_edges, const int* src, const int* dst, const double* w,
+                          double* depth, double* height, double* cp) {
+  if (n_nodes < 0 || n_edges < 0 || (n_edges > 0 && (!src || !dst || !w)))
+    return DASH_ERR_INVALID_ARG;
+  if (!dash::dag_longest_path(n_nodes, n_edges, src, dst, w, depth, height, cp))
+    return DASH_ERR_INVALID_ARG;
+  return DASH_OK;
+}
+
+}  // extern "C"

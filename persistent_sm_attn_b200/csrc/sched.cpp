@@ -1,0 +1,330 @@
+// DASH schedule tables, validator and DAG simulator (host C++).
+//
+// Schedules follow "Resumen Técnico: DASH – Programación de Atención
+// Determinista ..." §2.2:
+//   NAIVE_ASC   serialised baseline of §1: Q tiles ascending, dQ order by KV.
+//   DESCENDING  §2.2.A: Q tiles from the last to the first, dQ order by KV.
+//   SHIFT       §2.2.B full masks: the chain of KV tile k visits Q tiles
+//               k, k+1, ..., N-1, 0, ..., k-1; dQ blocks accumulate in step
+//               order, so every step touches N distinct blocks.
+//   SYM_SHIFT   §2.2.B causal masks: KV tiles k and N-1-k share one CTA; a
+//               dense phase over Q in [N/2, N) x KV in [0, N/2) is followed by
+//               the folded triangle; dQ blocks accumulate in (phase, step)
+//               order.  Needs even N.
+//   ATOMIC      the unordered comparison variant: SHIFT's visiting order for
+//               full masks, SYM_SHIFT's for causal masks (NAIVE_ASC for odd
+//               N); positions are unused.
+#include "sched.h"
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <deque>
+#include <queue>
+
+namespace dash {
+
+bool schedule_supported(int schedule, int N, int causal) {
+  if (N < 1 || N > 32767) return false;
+  switch (schedule) {
+    case NAIVE_ASC:
+    case DESCENDING:
+    case ATOMIC: return true;
+    case SHIFT: return !causal;
+    case SYM_SHIFT: return causal && (N % 2 == 0);
+    default: return false;
+  }
+}
+
+using Units = std::vector<std::vector<std::pair<int, int>>>;
+
+static Units units_of(int schedule, int N, int causal) {
+  Units u;
+  if (schedule == ATOMIC) {
+    if (!causal) schedule = SHIFT;
+    else schedule = (N % 2 == 0) ? SYM_SHIFT : NAIVE_ASC;
+  }
+  switch (schedule) {
+    case NAIVE_ASC:
+      for (int k = 0; k < N; ++k) {
+        std::vector<std::pair<int, int>> seq;
+        for (int q = causal ? k : 0; q < N; ++q) seq.push_back({k, q});
+        u.push_back(seq);
+      }
+      break;
+    case DESCENDING:
+      for (int k = 0; k < N; ++k) {
+        std::vector<std::pair<int, int>> seq;
+        for (int q = N - 1; q >= (causal ? k : 0); --q) seq.push_back({k, q});
+        u.push_back(seq);
+      }
+      break;
+    case SHIFT:
+      for (int k = 0; k < N; ++k) {
+        std::vector<std::pair<int, int>> seq;
+        for (int t = 0; t < N; ++t) seq.push_back({k, (k + t) % N});
+        u.push_back(seq);
+      }
+      break;
+    case SYM_SHIFT: {
+      const int h = N / 2;
+      for (int k = 0; k < h; ++k) {
+        std::vector<std::pair<int, int>> seq;
+        for (int t = 0; t < h; ++t) seq.push_back({k, h + (k + t) % h});       // dense phase
+        for (int t = 0; t < h; ++t) {                                            // folded phase
+          const int r = (k + t) % h;
+          if (r >= k) seq.push_back({k, r});
+          else seq.push_back({N - 1 - k, N - 1 - r});
+        }
+        seq.push_back({N - 1 - k, N - 1 - k});                                   // shared diagonal
+        u.push_back(seq);
+      }
+      break;
+    }
+    default: break;
+  }
+  return u;
+}
+
+std::vector<std::vector<std::pair<int, int>>> head_units(int schedule, int N, int causal) {
+  return units_of(schedule, N, causal);
+}
+
+bool build_table(int n_heads, int N, int causal, int schedule, int num_ctas, Table* out,
+                 std::string* err) {
+  if (n_heads < 1 || num_ctas < 1 || !schedule_supported(schedule, N, causal)) {
+    if (err) *err = "schedule not defined for this mask / tile count";
+    return false;
+  }
+  const Units units = units_of(schedule, N, causal);
+  const int U = (int)units.size();
+  // positions within each dQ block, for one head
+  // key: NAIVE_ASC / DESCENDING order by KV; SHIFT / SYM_SHIFT / ATOMIC by step
+  const bool by_kv = (schedule == NAIVE_ASC || schedule == DESCENDING);
+  std::vector<std::vector<std::pair<long long, int>>> contrib(N);  // per q: (key, unit*65536+step)
+  for (int k = 0; k < U; ++k)
+    for (int t = 0; t < (int)units[k].size(); ++t) {
+      const int kv = units[k][t].first, q = units[k][t].second;
+      const long long key = by_kv ? kv : (long long)t * 65536 + k;
+      contrib[q].push_back({key, k * 65536 + t});
+    }
+  std::vector<std::vector<int>> pos(U);
+  for (int k = 0; k < U; ++k) pos[k].assign(units[k].size(), -1);
+  for (int q = 0; q < N; ++q) {
+    auto& c = contrib[q];
+    std::sort(c.begin(), c.end());
+    for (int p = 0; p < (int)c.size(); ++p) pos[c[p].second >> 16][c[p].second & 0xffff] = p;
+  }
+  Table t;
+  t.n_heads = n_heads; t.N = N; t.causal = causal; t.schedule = schedule; t.num_ctas = num_ctas;
+  // per CTA, the global units it runs, in round order
+  std::vector<std::vector<long long>> per_cta(num_ctas);
+  const long long total_units = (long long)n_heads * U;
+  for (long long g = 0; g < total_units; ++g) per_cta[g % num_ctas].push_back(g);
+  t.cta_off.assign(num_ctas + 1, 0);
+  for (int c = 0; c < num_ctas; ++c) {
+    t.cta_off[c] = (int32_t)t.chains.size();
+    for (long long g : per_cta[c]) {
+      const int bh = (int)(g / U), k = (int)(g % U);
+      const auto& seq = units[k];
+      for (int i = 0; i < (int)seq.size(); ++i) {
+        if (i == 0 || seq[i].first != seq[i - 1].first) {
+          Chain ch{bh, seq[i].first, (int32_t)t.pairs.size(), 0};
+          t.chains.push_back(ch);
+        }
+        t.chains.back().pair_cnt++;
+        t.pairs.push_back(pack_pair(seq[i].second, pos[k][i]));
+      }
+    }
+  }
+  t.cta_off[num_ctas] = (int32_t)t.chains.size();
+  *out = std::move(t);
+  return true;
+}
+
+bool validate_table(const Table& t, std::string* err) {
+  auto fail = [&](const char* m) { if (err) *err = m; return false; };
+  const int N = t.N;
+  if ((int)t.cta_off.size() != t.num_ctas + 1) return fail("bad cta offsets");
+  const long long nblk = (long long)t.n_heads * N;
+  std::vector<uint8_t> seen((size_t)nblk * N, 0);       // (bh, kv, q)
+  std::vector<uint8_t> chain_seen((size_t)nblk, 0);     // (bh, kv)
+  std::vector<int> n_contrib(nblk, 0);
+  std::vector<uint8_t> pos_seen((size_t)nblk * N, 0);   // (bh, q, pos)
+  for (int c = 0; c < t.num_ctas; ++c) {
+    if (t.cta_off[c] > t.cta_off[c + 1]) return fail("cta offsets not monotone");
+    for (int ci = t.cta_off[c]; ci < t.cta_off[c + 1]; ++ci) {
+      const Chain& ch = t.chains[ci];
+      if (ch.bh < 0 || ch.bh >= t.n_heads || ch.kv < 0 || ch.kv >= N || ch.pair_cnt < 1)
+        return fail("chain out of range");
+      if (ch.pair_off < 0 || (long long)ch.pair_off + ch.pair_cnt > t.n_pairs())
+        return fail("chain pair range out of bounds");
+      uint8_t& cs = chain_seen[(size_t)ch.bh * N + ch.kv];
+      if (cs) return fail("KV tile split over two chains");
+      cs = 1;
+      for (int i = 0; i < ch.pair_cnt; ++i) {
+        const uint32_t w = t.pairs[ch.pair_off + i];
+        const int q = pair_q(w), p = pair_pos(w);
+        if (q < 0 || q >= N) return fail("q tile out of range");
+        if (t.causal && q < ch.kv) return fail("pair above the causal diagonal");
+        uint8_t& s = seen[((size_t)ch.bh * N + ch.kv) * N + q];
+        if (s) return fail("pair visited twice");
+        s = 1;
+        const long long blk = (long long)ch.bh * N + q;
+        if (p < 0 || p >= N) return fail("position out of range");
+        uint8_t& ps = pos_seen[(size_t)blk * N + p];
+        if (ps) return fail("position used twice in a dQ block");
+        ps = 1;
+        n_contrib[blk]++;
+      }
+    }
+  }
+  for (long long blk = 0; blk < nblk; ++blk) {
+    const int q = (int)(blk % N);
+    const int want = t.causal ? q + 1 : N;
+    if (n_contrib[blk] != want) return fail("dQ block has missing or extra contributors");
+    for (int p = 0; p < want; ++p)
+      if (!pos_seen[(size_t)blk * N + p]) return fail("positions are not a permutation");
+  }
+  if (t.schedule == ATOMIC) return true;  // no ordering to deadlock on
+  // Deadlock freedom: every CTA reduces its pairs in table order and waits for
+  // the block's ticket to equal the pair's position.
+  std::vector<int> ticket(nblk, 0);
+  std::vector<long long> next(t.num_ctas), end(t.num_ctas);
+  std::vector<std::vector<int>> waiters(nblk);
+  // flatten each CTA's pairs as (chain index, pair index) via a cursor
+  std::vector<int> cur_chain(t.num_ctas), cur_pair(t.num_ctas);
+  for (int c = 0; c < t.num_ctas; ++c) { cur_chain[c] = t.cta_off[c]; cur_pair[c] = 0; }
+  std::deque<int> work;
+  for (int c = 0; c < t.num_ctas; ++c) work.push_back(c);
+  long long done = 0;
+  while (!work.empty()) {
+    const int c = work.front();
+    work.pop_front();
+    while (cur_chain[c] < t.cta_off[c + 1]) {
+      const Chain& ch = t.chains[cur_chain[c]];
+      const uint32_t w = t.pairs[ch.pair_off + cur_pair[c]];
+      const long long blk = (long long)ch.bh * N + pair_q(w);
+      if (ticket[blk] != pair_pos(w)) { waiters[blk].push_back(c); break; }
+      ticket[blk]++;
+      ++done;
+      for (int wc : waiters[blk]) work.push_back(wc);
+      waiters[blk].clear();
+      if (++cur_pair[c] == ch.pair_cnt) { cur_pair[c] = 0; ++cur_chain[c]; }
+    }
+  }
+  if (done != t.n_pairs()) return fail("ticket order deadlocks with this many CTAs");
+  return true;
+}
+
+bool dag_longest_path(int n, int m, const int* src, const int* dst, const double* w,
+                      double* depth, double* height, double* cp) {
+  std::vector<int> indeg(n, 0), head(n + 1, 0), order;
+  for (int e = 0; e < m; ++e) {
+    if (src[e] < 0 || src[e] >= n || dst[e] < 0 || dst[e] >= n) return false;
+    indeg[dst[e]]++;
+    head[src[e] + 1]++;
+  }
+  for (int i = 0; i < n; ++i) head[i + 1] += head[i];
+  std::vector<int> adj(m), fill(head.begin(), head.end() - 1);
+  for (int e = 0; e < m; ++e) adj[fill[src[e]]++] = e;
+  std::vector<int> deg = indeg;
+  std::queue<int> qu;
+  for (int i = 0; i < n; ++i) if (!deg[i]) qu.push(i);
+  std::vector<double> d(n, 0.0), h(n, 0.0);
+  while (!qu.empty()) {
+    const int u = qu.front(); qu.pop();
+    order.push_back(u);
+    for (int j = head[u]; j < head[u + 1]; ++j) {
+      const int e = adj[j];
+      d[dst[e]] = std::max(d[dst[e]], d[u] + w[e]);
+      if (--deg[dst[e]] == 0) qu.push(dst[e]);
+    }
+  }
+  if ((int)order.size() != n) return false;  // cycle
+  for (int i = n - 1; i >= 0; --i) {
+    const int u = order[i];
+    for (int j = head[u]; j < head[u + 1]; ++j) {
+      const int e = adj[j];
+      h[u] = std::max(h[u], w[e] + h[dst[e]]);
+    }
+  }
+  double best = 0.0;
+  for (int i = 0; i < n; ++i) best = std::max(best, d[i]);
+  if (depth) std::copy(d.begin(), d.end(), depth);
+  if (height) std::copy(h.begin(), h.end(), height);
+  if (cp) *cp = best;
+  return true;
+}
+
+bool simulate_table(const Table& t, double c, double r, int beta, SimResult* res,
+                    std::string* err) {
+  const long long P = t.n_pairs();
+  if (P * 4 > (1LL << 31) - 1) { if (err) *err = "table too large to simulate"; return false; }
+  const int N = t.N;
+  // node id of event a of each pair, in CTA order
+  std::vector<int> a_of(P);
+  std::vector<int> blk_pos_node((size_t)t.n_heads * N * N, -1);
+  int nid = 0;
+  std::vector<int> src, dst;
+  std::vector<double> wt;
+  auto edge = [&](int u, int v, double w) { src.push_back(u); dst.push_back(v); wt.push_back(w); };
+  std::vector<std::vector<int>> cta_nodes(t.num_ctas);
+  for (int cta = 0; cta < t.num_ctas; ++cta)
+    for (int ci = t.cta_off[cta]; ci < t.cta_off[cta + 1]; ++ci) {
+      const Chain& ch = t.chains[ci];
+      for (int i = 0; i < ch.pair_cnt; ++i) {
+        const uint32_t w = t.pairs[ch.pair_off + i];
+        const size_t key = ((size_t)ch.bh * N + pair_q(w)) * N + pair_pos(w);
+        blk_pos_node[key] = nid;
+        cta_nodes[cta].push_back(nid);
+        nid += 4;
+      }
+    }
+  for (int cta = 0; cta < t.num_ctas; ++cta) {
+    const auto& nodes = cta_nodes[cta];
+    size_t n = 0;
+    for (int ci = t.cta_off[cta]; ci < t.cta_off[cta + 1]; ++ci) {
+      const Chain& ch = t.chains[ci];
+      for (int i = 0; i < ch.pair_cnt; ++i, ++n) {
+        const int a = nodes[n];
+        const uint32_t w = t.pairs[ch.pair_off + i];
+        edge(a, a + 1, c);
+        edge(a + 1, a + 2, 0.0);
+        edge(a + 2, a + 3, r);
+        const int p = pair_pos(w);
+        if (p > 0) {
+          const size_t key = ((size_t)ch.bh * N + pair_q(w)) * N + (p - 1);
+          const int y = blk_pos_node[key];
+          if (y < 0) { if (err) *err = "missing predecessor in dQ order"; return false; }
+          edge(y + 3, a + 2, 0.0);
+        }
+        if (n > 0) {
+          edge(nodes[n - 1] + 1, a, 0.0);
+          if (beta >= 1 && (long long)n - beta >= 0) edge(nodes[n - beta] + 3, a + 1, 0.0);
+        }
+      }
+    }
+  }
+  std::vector<double> depth(nid);
+  double cp = 0;
+  if (!dag_longest_path(nid, (int)src.size(), src.data(), dst.data(), wt.data(), depth.data(),
+                        nullptr, &cp)) {
+    if (err) *err = "schedule graph has a cycle (ticket deadlock)";
+    return false;
+  }
+  SimResult out;
+  out.critical_path = cp;
+  for (int cta = 0; cta < t.num_ctas; ++cta) {
+    const auto& nodes = cta_nodes[cta];
+    if (nodes.empty()) continue;
+    for (int a : nodes)
+      if (depth[a + 1] > depth[a] + c + 1e-12 * std::max(1.0, std::fabs(depth[a]))) out.stalls++;
+    out.makespan = std::max(out.makespan, depth[nodes.back() + 1]);
+    out.bubble_time += cp - c * (double)nodes.size();
+  }
+  *res = out;
+  return true;
+}
+
+}  // namespace dash

@@ -1,0 +1,72 @@
+// Host-side DASH schedule tables, their validator and the DAG simulator.
+//
+// A table tells each CTA of the persistent backward kernel which chains it
+// runs and, for every (KV tile, Q tile) pair of a chain, the Q tile and the
+// pair's position in that dQ block's fixed accumulation order.
+//
+// Source: "Resumen Técnico: DASH – Programación de Atención Determinista ...",
+// §2.1 (DAG formulation, one KV tile per SM as an unbroken chain) and §2.2
+// (descending Q-tile iteration, shift and symmetric shift scheduling).
+#pragma once
+#include <cstdint>
+#include <string>
+#include <vector>
+
+namespace dash {
+
+enum Schedule { NAIVE_ASC = 0, DESCENDING = 1, SHIFT = 2, SYM_SHIFT = 3, ATOMIC = 4 };
+
+struct Chain {           // one KV tile of one head, run back to back on one CTA
+  int32_t bh;            // b * H + h
+  int32_t kv;            // KV tile index
+  int32_t pair_off;      // first entry in Table::pairs
+  int32_t pair_cnt;      // number of pairs (Q tiles) of this chain
+};
+
+// Packed pair word: bits [0,16) Q tile, bits [16,32) position in the dQ order.
+inline uint32_t pack_pair(int q, int pos) { return uint32_t(q) | (uint32_t(pos) << 16); }
+inline int pair_q(uint32_t w) { return int(w & 0xffffu); }
+inline int pair_pos(uint32_t w) { return int(w >> 16); }
+
+struct Table {
+  int n_heads = 0, N = 0, causal = 0, schedule = 0, num_ctas = 0;
+  std::vector<int32_t> cta_off;   // num_ctas + 1 offsets into chains
+  std::vector<Chain> chains;      // grouped by CTA, in execution order
+  std::vector<uint32_t> pairs;    // packed (q, position)
+  long long n_pairs() const { return (long long)pairs.size(); }
+};
+
+// True when the pages define `schedule` for this mask and tile count.
+bool schedule_supported(int schedule, int N, int causal);
+
+// Units of one head: each a list of (kv, q) in visiting order.
+std::vector<std::vector<std::pair<int, int>>> head_units(int schedule, int N, int causal);
+
+// Build the whole-grid table: heads in order, unit g on CTA g mod num_ctas.
+// Returns false (with a message) if the combination is unsupported.
+bool build_table(int n_heads, int N, int causal, int schedule, int num_ctas, Table* out,
+                 std::string* err);
+
+// Checks coverage (every allowed pair once), positions (a permutation per dQ
+// block), unbroken chains, pair-word ranges, and deadlock freedom of the
+// ticket order when all num_ctas CTAs run concurrently and each CTA performs
+// its reductions in table order.  Returns false with a message on failure.
+bool validate_table(const Table& t, std::string* err);
+
+// Longest path of a general DAG (Kahn order).  Returns false on a cycle.
+bool dag_longest_path(int n_nodes, int n_edges, const int* src, const int* dst,
+                      const double* w, double* depth, double* height, double* cp);
+
+struct SimResult {
+  double critical_path = 0, makespan = 0, bubble_time = 0;
+  long long stalls = 0;
+};
+
+// Event-graph simulation of a table: per pair, events a (start), b (partial
+// ready), s (reduction start), d (reduction done); arcs a->b weight c,
+// b->s 0, d(prev in order)->s 0, s->d weight r, b(prev on slot)->a 0, and with
+// beta >= 1 buffers d(pair n-beta on slot)->b(pair n).  beta <= 0 = unbounded.
+bool simulate_table(const Table& t, double c, double r, int beta, SimResult* res,
+                    std::string* err);
+
+}  // namespace dash

@@ -1,0 +1,115 @@
+"""The library's schedule tables and DAG simulator against the oracle.
+
+Tables must equal the oracle's packed tables bit for bit (integer work); the
+simulator must reproduce the brute-force critical paths on tiny tables, the
+closed forms on larger ones, and the zero-weight-edge lemma of DASH summary
+§2.2.B through its general longest-path entry point.
+"""
+import random
+
+import pytest
+
+from oracle import dag, schedules as sc
+from persistent_sm_attn_b200 import binding
+
+SID = {sc.NAIVE_ASC: "naive_asc", sc.DESCENDING: "descending", sc.SHIFT: "shift",
+       sc.SYM_SHIFT: "sym_shift"}
+
+
+def _lib_table(name, heads, N, causal, ctas):
+    rows = binding.dash_sched_table(heads, N, causal, SID[name], ctas)
+    slots = [[] for _ in range(ctas)]
+    for cta, hd, kv, q, pos, _chain in rows:
+        ncontrib = q + 1 if causal else N
+        slots[cta].append((hd, kv, q, pos, ncontrib))
+    return slots
+
+
+CASES = [(name, N, causal, heads, ctas)
+         for name in sc.ALL
+         for causal in (False, True)
+         for N in (1, 2, 3, 4, 7, 8, 16)
+         for heads, ctas in ((1, 148), (3, 5), (5, 16), (2, 7))
+         if sc.supported(name, N, causal)
+         and len(sc.units(name, N, causal)) <= ctas]
+
+
+@pytest.mark.parametrize("name,N,causal,heads,ctas", CASES)
+def test_table_equals_oracle(name, N, causal, heads, ctas):
+    assert _lib_table(name, heads, N, causal, ctas) == sc.packed_table(name, heads, N, causal, ctas)
+
+
+def test_full_size_tables_validate():
+    # the workload shapes on a 148-SM grid
+    for heads, N, causal, name in ((32, 32, False, "shift"), (32, 32, False, "descending"),
+                                   (32, 32, False, "naive_asc"), (64, 64, True, "descending"),
+                                   (64, 64, True, "sym_shift"), (128, 128, True, "sym_shift"),
+                                   (24, 128, False, "shift")):
+        rows = binding.dash_sched_table(heads, N, causal, name, 148)
+        assert len(rows) == heads * (N * (N + 1) // 2 if causal else N * N)
+
+
+def test_deadlock_detected():
+    # a shift head needs all its N chains co-resident; 4 CTAs cannot hold 8
+    with pytest.raises(binding.DashError) as e:
+        binding.dash_sched_table(1, 8, False, "shift", 4)
+    assert e.value.status == 6
+    # the descending order only waits on lower KV tiles: it never deadlocks
+    assert len(binding.dash_sched_table(1, 8, False, "descending", 4)) == 64
+
+
+@pytest.mark.parametrize("name,N,causal,heads,ctas", [
+    (sc.SHIFT, 3, False, 1, 3), (sc.SHIFT, 4, False, 2, 5), (sc.NAIVE_ASC, 3, False, 1, 3),
+    (sc.NAIVE_ASC, 4, True, 2, 3), (sc.DESCENDING, 4, True, 1, 4), (sc.DESCENDING, 3, False, 2, 4),
+    (sc.SYM_SHIFT, 4, True, 2, 3), (sc.SYM_SHIFT, 2, True, 3, 2)])
+@pytest.mark.parametrize("beta", [None, 1, 2])
+def test_simulator_matches_bruteforce(name, N, causal, heads, ctas, beta):
+    c, r = 1.0, 0.35
+    table = sc.packed_table(name, heads, N, causal, ctas)
+    want = dag.simulate(table, c, r, beta)
+    got = binding.dash_sched_simulate(heads, N, causal, SID[name], ctas, c, r, beta or 0)
+    assert got[3] == want[3]
+    for g, w in zip(got[:3], want[:3]):
+        assert abs(g - w) < 1e-9
+
+
+@pytest.mark.parametrize("N", [8, 16, 32, 64])
+def test_simulator_closed_forms(N):
+    """One head, one CTA per unit, unbounded buffers, r <= c."""
+    c, r = 1.0, 0.15
+    cp = lambda name, causal: binding.dash_sched_simulate(1, N, causal, name, 148, c, r, 0)[0]
+    assert abs(cp("naive_asc", False) - (N * c + N * r)) < 1e-9
+    assert abs(cp("shift", False) - (N * c + r)) < 1e-9
+    assert abs(cp("descending", True) - (N * c + r)) < 1e-9
+    assert abs(cp("sym_shift", True) - ((N + 1) * c + r)) < 1e-9
+
+
+def test_predicted_ordering_on_workload_shapes():
+    """The simulator's ranking of schedules on the benchmark shapes (148 CTAs,
+    a partial-buffer depth of 2 as in the kernel, reduction ~ 1/4 of compute)."""
+    c, r = 1.0, 0.25
+    f = lambda heads, N, causal, name: binding.dash_sched_simulate(
+        heads, N, causal, name, 148, c, r, 2)[0]
+    # full mask: shift is never worse than the serialised orders
+    assert f(32, 32, False, "shift") <= f(32, 32, False, "descending")
+    assert f(32, 32, False, "shift") <= f(32, 32, False, "naive_asc")
+    # causal: descending beats the ascending baseline
+    assert f(64, 64, True, "descending") < f(64, 64, True, "naive_asc")
+
+
+def test_longest_path_matches_bruteforce_and_lemma():
+    rng = random.Random(3)
+    for _ in range(150):
+        n = rng.randint(2, 8)
+        edges = [(u, v, float(rng.randint(0, 4))) for u in range(n) for v in range(u + 1, n)
+                 if rng.random() < 0.35]
+        cp, depth, height = binding.dash_dag_longest_path(n, edges)
+        bcp, bdepth, bheight = dag.paths_longest(n, edges)
+        assert cp == bcp and depth == bdepth and height == bheight
+        for u in range(n):
+            for v in range(u + 1, n):
+                cp2, _, _ = binding.dash_dag_longest_path(n, edges + [(u, v, 0.0)])
+                if depth[u] <= depth[v]:
+                    assert cp2 == cp
+                if depth[v] + height[v] == cp:
+                    assert (cp2 == cp) == (depth[u] <= depth[v])
