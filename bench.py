@@ -1,0 +1,350 @@
+"""Benchmark of the deterministic attention backward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload INDEX] [--schedule NAME] [--all-workloads]
+
+One step = one backward pass (Delta preprocess + persistent kernel) of the
+workload through the C ABI, inputs resident in HBM.  L2 is flushed (a 512 MiB
+write) before every timed step; each step is timed with CUDA events on the
+launching stream and the steps are bracketed by a barrier and synchronisation.
+Rank 0 prints one JSON line.  With torchrun (N > 1) every rank runs the same
+workload on its own GPU (weak scaling: the B*H heads of one workload per GPU;
+heads are independent, so no data-path collective exists) and the time is the
+maximum over ranks.
+
+--impl reference times the fp64 CPU oracle (the only other implementation of
+the same computation) on a bounded sample of heads of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from persistent_sm_attn_b200.inputs import WORKLOADS, seed_of  # noqa: E402
+
+METRIC = "deterministic attn-bwd TFLOPS (% of B200 bf16 peak); det/nondet throughput ratio"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["bf16_tflops"]), float(pk["hbm_gbs"]), "measured"
+    except Exception:
+        return 1590.0, 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        mhz, maxmhz, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                maxmhz.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not mhz:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max(maxmhz),
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+def _dist_init(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_ours(args):
+    import datetime
+
+    import torch
+
+    from persistent_sm_attn_b200 import binding
+    from persistent_sm_attn_b200.inputs import draw
+
+    world, rank, local = _dist_init(args)
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    w = WORKLOADS[args.workload]
+    sched = args.schedule or w.schedules[0]
+    q, k, v, do = draw(w.B, w.H, w.S, w.D, w.sigma, seed_of(args.workload) + 1000 * rank,
+                       device="cuda")
+    o, lse = binding.dash_attn_fwd(q, k, v, w.causal)
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def time_schedule(name, steps, warmup, clocks=None):
+        dq = torch.empty_like(q)
+        dk = torch.empty_like(k)
+        dv = torch.empty_like(v)
+        for _ in range(warmup):
+            binding.dash_attn_bwd(q, k, v, o, do, lse, w.causal, name, dq, dk, dv)
+        st = binding.dash_attn_sync_status()
+        if st != 0:
+            raise RuntimeError(f"warm-up status {binding.dash_status_string(st)}")
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        barrier()
+        binding.dash_profile_begin()
+        ctx = clocks if clocks is not None else _Null()
+        with ctx:
+            for i in range(steps):
+                flush.fill_(float(i))
+                evs[i][0].record(stream)
+                binding.dash_attn_bwd(q, k, v, o, do, lse, w.causal, name, dq, dk, dv)
+                evs[i][1].record(stream)
+            barrier()
+        main_ms, aux_ms, n_calls = binding.dash_profile_end()
+        st = binding.dash_attn_sync_status()
+        if st != 0:
+            raise RuntimeError(f"timed status {binding.dash_status_string(st)}")
+        step_ms = sum(a.elapsed_time(b) for a, b in evs)
+        t = torch.tensor([step_ms, main_ms], dtype=torch.float64, device="cuda")
+        if dist is not None:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t[0]) / steps, float(t[1]) / steps, aux_ms / steps, n_calls
+
+    clocks = ClockSampler(local)
+    ms, main_ms, aux_ms, n_calls = time_schedule(sched, args.steps, args.warmup, clocks)
+    results = {sched: ms}
+    compare = [s for s in w.schedules if s != sched] if not args.no_compare else []
+    for other in compare:
+        results[other] = time_schedule(other, max(5, args.steps // 2), 3)[0]
+
+    # end to end through the public API: pinned host inputs in, results out
+    host_in = [t.cpu().pin_memory() for t in (q, k, v, o, do, lse)]
+    host_out = [torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(3)]
+    dev_in = [torch.empty_like(t) for t in (q, k, v, o, do, lse)]
+    dev_out = [torch.empty_like(q) for _ in range(3)]
+    e2e_steps = max(3, args.steps // 2)
+    for it in range(e2e_steps + 2):
+        if it == 2:
+            barrier()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        for d_, h_ in zip(dev_in, host_in):
+            d_.copy_(h_, non_blocking=True)
+        binding.dash_attn_bwd(*dev_in, w.causal, sched, *dev_out)
+        for h_, d_ in zip(host_out, dev_out):
+            h_.copy_(d_, non_blocking=True)
+    e1.record(stream)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_ms = float(t[0])
+    h2d = sum(x.numel() * x.element_size() for x in host_in)
+    d2h = sum(x.numel() * x.element_size() for x in host_out)
+
+    if rank == 0:
+        peak, _, peak_kind = _peaks()
+        tflops = lambda msec: w.flops * world / (msec * 1e-3) / 1e12
+        value = tflops(ms)
+        kern = w.flops / (main_ms * 1e-3) / 1e12
+        atomic_ms = results.get("atomic")
+        det = {s: round(tflops(m), 2) for s, m in results.items()}
+        best_det = max((v_ for s, v_ in det.items() if s != "atomic"), default=None)
+        line = {
+            "metric": METRIC,
+            "value": round(value, 2),
+            "unit": "TFLOP/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(ms, 4),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic (seeded normal bf16 Q, K, V, dO; O and LSE from the library forward)",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "S": w.S, "D": w.D,
+                       "mask": "causal" if w.causal else "full", "sigma": w.sigma,
+                       "schedule": sched, "parallelism": f"dp{world} (independent heads)",
+                       "l2": "flushed before every timed step (512 MiB write)"},
+            "pct_of_peak": round(100 * value / (peak * world), 2),
+            "schedules_tflops": det,
+            "det_nondet_ratio": (round(best_det / det["atomic"], 4)
+                                 if atomic_ms and best_det else None),
+            "roofline": {"bound": "tensor", "achieved": round(kern, 2), "peak": peak,
+                         "unit": "TFLOP/s", "frac": round(kern / peak, 4), "traffic": None,
+                         "kernel": "dash_bwd_kernel", "peak_kind": f"{peak_kind} bf16 burst",
+                         "kernel_ms": round(main_ms, 4), "aux_ms": round(aux_ms, 4)},
+            "e2e": {"value": round(tflops(e2e_ms), 2), "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": int(n_calls) * (3 if sched == "atomic" else 2),
+            "clocks": clocks.summary(),
+        }
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def _oracle_heads_tflops(w, seconds: float, index: int):
+    """Time the fp64 oracle's per-head backward on seeded heads of workload w
+    until ``seconds`` of CPU work have been spent (at least one head)."""
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    from oracle import attention as A
+    from persistent_sm_attn_b200.inputs import draw
+
+    flops_per_head = w.flops / (w.B * w.H)
+    heads = 0
+    t_total = 0.0
+    scale = 1.0 / np.sqrt(w.D)
+    while heads == 0 or t_total < seconds:
+        q, k, v, do = (t[0, 0].float().numpy()
+                       for t in draw(1, 1, w.S, w.D, w.sigma, seed_of(index) + heads))
+        t0 = time.perf_counter()
+        A.head_backward(q, k, v, do, w.causal, scale)
+        t_total += time.perf_counter() - t0
+        heads += 1
+    threads = max([d.get("num_threads", 1) for d in threadpool_info()] or [1])
+    return flops_per_head * heads / t_total / 1e12, heads, t_total, threads
+
+
+def cpu_baseline(w, seconds):
+    index = WORKLOADS.index(w)
+    tf, heads, t, cores = _oracle_heads_tflops(w, seconds, index)
+    return {"value": round(tf, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{heads} head(s) of {w.name} (S={w.S}, D={w.D}), fp64 numpy oracle, "
+                      f"{t:.1f} s; backward FLOPs counted as in the metric"}
+
+
+def run_reference(args):
+    world, rank, _ = _dist_init(args)
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    per_step = []
+    last = None
+    for _ in range(args.warmup):
+        _oracle_heads_tflops(w, 0.0, args.workload)
+    for _ in range(args.steps):
+        last = _oracle_heads_tflops(w, args.cpu_seconds / max(1, args.steps), args.workload)
+        per_step.append(last[0])
+    value = statistics.mean(per_step)
+    tf, heads, t, cores = last
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (seeded normal bf16 Q, K, V, dO widened to fp64)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "S": w.S, "D": w.D,
+                   "mask": "causal" if w.causal else "full", "schedule": "none (order-free)"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores,
+                         "kind": "oracle",
+                         "sample": f"each step: >= {args.cpu_seconds / max(1, args.steps):.1f} s "
+                                   f"of per-head fp64 backward of {w.name}"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", type=int, default=1)
+    ap.add_argument("--schedule", default=None)
+    ap.add_argument("--no-compare", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--all-workloads", action="store_true",
+                    help="one JSON line per workload (1-4), rank 0 only")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    if args.all_workloads:
+        for i in range(1, len(WORKLOADS)):
+            args.workload = i
+            run_ours(args)
+        return
+    run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -110,6 +110,17 @@ int dash_set_spin_limit_us(long long us);
 /* Number of persistent CTAs the backward uses on `device` for head dim D. */
 int dash_bwd_num_ctas(int device, int D, int* num_ctas);
 
+/*
+ * Device timing of backward launches.  Between dash_profile_begin() and
+ * dash_profile_end(), every dash_attn_bwd records CUDA events on its stream
+ * around its kernels.  dash_profile_end() waits for them and returns the
+ * summed milliseconds of the main (persistent) kernel, of the auxiliary
+ * kernels (Delta preprocess, and the fp32-to-bf16 dQ pass of ATOMIC), and the
+ * number of backward calls recorded.  Outputs may be NULL.
+ */
+int dash_profile_begin(void);
+int dash_profile_end(double* main_ms, double* aux_ms, long long* launches);
+
 /* Frees every cached workspace and schedule table of the current device
  * (synchronises the device first). */
 int dash_release_workspace(void);

@@ -20,7 +20,8 @@ STATUS = {0: "DASH_OK", 1: "DASH_ERR_INVALID_ARG", 2: "DASH_ERR_UNSUPPORTED", 3:
 
 EXPORTS = ("dash_attn_fwd", "dash_attn_bwd", "dash_attn_sync_status", "dash_status_string",
            "dash_set_spin_limit_us", "dash_bwd_num_ctas", "dash_release_workspace",
-           "dash_sched_table", "dash_sched_simulate", "dash_dag_longest_path")
+           "dash_sched_table", "dash_sched_simulate", "dash_dag_longest_path",
+           "dash_profile_begin", "dash_profile_end")
 
 
 class DashError(RuntimeError):
@@ -60,6 +61,8 @@ def load(path: str | None = None):
     lib.dash_sched_table.restype = ll
     lib.dash_sched_simulate.argtypes = [i, i, i, i, i, d, d, i, P(d), P(d), P(d), P(ll)]
     lib.dash_dag_longest_path.argtypes = [i, i, vp, vp, vp, vp, vp, P(d)]
+    lib.dash_profile_begin.argtypes = []
+    lib.dash_profile_end.argtypes = [P(d), P(d), P(ll)]
     for name in EXPORTS:
         if name not in ("dash_status_string", "dash_sched_table"):
             getattr(lib, name).restype = ctypes.c_int
@@ -180,3 +183,15 @@ def dash_dag_longest_path(n_nodes: int, edges):
     rc = load().dash_dag_longest_path(n_nodes, m, src, dst, w, depth, height, ctypes.byref(cp))
     _check(rc, "dash_dag_longest_path")
     return cp.value, list(depth)[:n_nodes], list(height)[:n_nodes]
+
+
+def dash_profile_begin() -> None:
+    _check(load().dash_profile_begin(), "dash_profile_begin")
+
+
+def dash_profile_end():
+    """(main kernel ms summed, auxiliary kernels ms summed, backward calls)."""
+    m, a, n = ctypes.c_double(), ctypes.c_double(), ctypes.c_longlong()
+    _check(load().dash_profile_end(ctypes.byref(m), ctypes.byref(a), ctypes.byref(n)),
+           "dash_profile_end")
+    return m.value, a.value, n.value

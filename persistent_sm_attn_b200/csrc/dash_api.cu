@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <array>
 #include <atomic>
 #include <cstdint>
 #include <cstdio>
@@ -12,6 +13,7 @@
 #include <mutex>
 #include <string>
 #include <tuple>
+#include <vector>
 
 #include "../../include/dash_attn.h"
 #include "aux_kernels.cuh"
@@ -59,6 +61,21 @@ std::mutex g_mu;
 std::map<std::pair<int, uintptr_t>, Workspace> g_ws;                  // (device, stream)
 std::map<std::tuple<int, int, int, int, int, int>, DevTable> g_tables;  // device,heads,N,causal,sched,ctas
 std::map<std::pair<int, int>, int> g_num_ctas;                        // (device, D)
+
+// Optional per-launch device timing: while enabled, each backward records four
+// events (before the Delta kernel, before and after the main kernel, after the
+// last auxiliary kernel) on its stream.
+std::atomic<bool> g_prof_on{false};
+std::mutex g_prof_mu;
+std::vector<std::array<cudaEvent_t, 4>> g_prof;
+
+bool prof_record(int slot, std::array<cudaEvent_t, 4>* ev, cudaStream_t st) {
+  if (!g_prof_on.load()) return true;
+  if (slot == 0)
+    for (auto& e : *ev)
+      if (cudaEventCreate(&e) != cudaSuccess) return false;
+  return cudaEventRecord((*ev)[slot], st) == cudaSuccess;
+}
 
 #define DASH_CUDA(call)                    \
   do {                                     \
@@ -222,6 +239,8 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
     return rc;
   float* lse2 = ws->rowbuf;
   float* delta = ws->rowbuf + ws->rows_cap;
+  std::array<cudaEvent_t, 4> ev{};
+  if (!prof_record(0, &ev, stream)) return DASH_ERR_CUDA;
   {
     const long long threads = rows * (D / 8);
     const int blocks = (int)((threads + 255) / 256);
@@ -265,12 +284,19 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (!prof_record(1, &ev, stream)) return DASH_ERR_CUDA;
   DASH_CUDA(cudaLaunchKernelEx(&cfg, dash::dash_bwd_kernel<D, kAtomic>, tq, tk, tv, tdo, p));
+  if (!prof_record(2, &ev, stream)) return DASH_ERR_CUDA;
   if (kAtomic) {
     const long long n_blocks = (long long)B * H * N;
     const long long threads = n_blocks * 128 * (D / 4);
     dash::dash_dq_convert<D><<<(int)((threads + 255) / 256), 256, 0, stream>>>(
         ws->acc, static_cast<__nv_bfloat16*>(dq), n_blocks, p.scale);
+  }
+  if (!prof_record(3, &ev, stream)) return DASH_ERR_CUDA;
+  if (g_prof_on.load()) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof.push_back(ev);
   }
   DASH_CUDA(cudaGetLastError());
   return DASH_OK;
@@ -381,6 +407,38 @@ int dash_bwd_num_ctas(int device, int D, int* num_ctas) {
   const int rc = (D == 64) ? num_ctas_for<64, false>(device, num_ctas)
                            : num_ctas_for<128, false>(device, num_ctas);
   cudaSetDevice(prev);
+  return rc;
+}
+
+int dash_profile_begin(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (auto& ev : g_prof)
+    for (auto e : ev) cudaEventDestroy(e);
+  g_prof.clear();
+  g_prof_on.store(true);
+  return DASH_OK;
+}
+
+int dash_profile_end(double* main_ms, double* aux_ms, long long* launches) {
+  g_prof_on.store(false);
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  double m = 0, a = 0;
+  int rc = DASH_OK;
+  for (auto& ev : g_prof) {
+    float t01 = 0, t12 = 0, t23 = 0;
+    if (cudaEventSynchronize(ev[3]) != cudaSuccess ||
+        cudaEventElapsedTime(&t01, ev[0], ev[1]) != cudaSuccess ||
+        cudaEventElapsedTime(&t12, ev[1], ev[2]) != cudaSuccess ||
+        cudaEventElapsedTime(&t23, ev[2], ev[3]) != cudaSuccess)
+      rc = DASH_ERR_CUDA;
+    m += t12;
+    a += t01 + t23;
+    for (auto e : ev) cudaEventDestroy(e);
+  }
+  if (main_ms) *main_ms = m;
+  if (aux_ms) *aux_ms = a;
+  if (launches) *launches = (long long)g_prof.size();
+  g_prof.clear();
   return rc;
 }
 
