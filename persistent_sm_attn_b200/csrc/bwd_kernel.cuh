@@ -4,21 +4,22 @@
 // DASH ..." §2.1: all pairs of one KV tile run back to back on one SM, with
 // the dK/dV accumulators on chip).  Per (KV tile j, Q tile i) pair:
 //
-//   S^T  = K_j Q_i^T                  tcgen05.mma, TMEM cols [0,128)
-//   dP^T = V_j dO_i^T                 tcgen05.mma, TMEM cols [128,256)
+//   dP^T = V_j dO_i^T                 tcgen05.mma -> TMEM
+//   S^T  = K_j Q_i^T                  tcgen05.mma -> TMEM
 //   P^T  = exp(scale S^T - LSE_i),  dS^T = P^T (dP^T - Delta_i)   (softmax warps -> smem)
-//   dV_j += P^T dO_i,  dK_j += dS^T Q_i      tcgen05.mma into TMEM (resident per chain)
-//   dQp  = dS K_j                     tcgen05.mma into TMEM
+//   dV_j += P^T dO_i,  dK_j += dS^T Q_i      tcgen05.mma, accumulators resident in TMEM
+//   dQp  = dS K_j                     tcgen05.mma -> TMEM
 //   ordered reduction of dQp into the fp32 accumulator of block (b,h,i): wait
-//   until the block's ticket equals this pair's position, add, publish, bump
-//   the ticket (§1: the fixed accumulation order is what makes dQ bitwise
-//   reproducible; §2.2 chooses the order).  The last contributor rounds the
-//   sum once to bf16 and writes dQ.
+//   until the block's ticket equals this pair's position, add with plain
+//   loads and stores, publish, bump the ticket (§1: a fixed accumulation
+//   order makes dQ bitwise reproducible; §2.2 chooses the order).  The last
+//   contributor rounds the sum once to bf16 and writes dQ.
 //
-// Warp roles (320 threads): warp 0 TMA producer, warp 1 MMA issuer and TMEM
-// owner, warps 2-5 softmax / dS, warps 6-9 dQ reduction and the dK/dV
-// epilogue.  TMEM lane quarter of a warp is (warp % 4), so each group of four
-// consecutive warps covers the 128 lanes.
+// Warp roles (512 threads, four warpgroups):
+//   WG0, WG1  softmax / dS; WG0 owns Q columns 0-63, WG1 columns 64-127
+//   WG2       dQ reduction and the dK/dV epilogue (176 registers)
+//   WG3       warp 12 TMA producer, warp 13 MMA issuer and TMEM owner (80 registers)
+// TMEM lane quarter of a warp is (warp % 4), so each warpgroup covers the 128 lanes.
 //
 // Shared-memory tiles are [128 rows][D] bf16 stored as D/64 column blocks of
 // 128 rows x 128 bytes with the 128-byte swizzle (the layout a TMA load with
@@ -51,7 +52,12 @@ struct BwdParams {
 
 template <int D>
 struct BwdCfg {
-  static constexpr int kThreads = 320;
+  static constexpr int kThreads = 512;
+  static constexpr int kLaunchRegs = 65536 / kThreads;   // 128: the setmaxnreg split below
+  static constexpr int kRegsReduce = 176;                // WG2
+  static constexpr int kRegsCtrl = 80;                   // WG3
+  static_assert(2 * kLaunchRegs + kRegsReduce + kRegsCtrl == 4 * kLaunchRegs,
+                "register split must equal the launch allocation");
   static constexpr int kTile = 128 * D * 2;              // one [128][D] bf16 tile
   static constexpr int kStages = (D == 64) ? 2 : 1;      // Q/dO pipeline depth
   static constexpr int OFF_K = 0;
@@ -63,23 +69,23 @@ struct BwdCfg {
   static constexpr int OFF_LSE = OFF_DST + 32768;          // kStages x 128 fp32
   static constexpr int OFF_DEL = OFF_LSE + kStages * 512;
   static constexpr int OFF_BAR = OFF_DEL + kStages * 512;
-  static constexpr int kBars = 14 + 2 * kStages;
+  static constexpr int kBars = 16 + 4 * kStages;
   static constexpr int OFF_TMEM_SLOT = OFF_BAR + kBars * 8;
   static constexpr int kSmemBytes = OFF_TMEM_SLOT + 16 + 1024;  // + alignment slack
   // TMEM columns
   static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 256 + D;
-  static constexpr uint32_t TM_DQ = (D == 64) ? 384 : 128;  // D=128 shares dP^T's columns
-  static constexpr bool kDqAliasesDp = (D != 64);
+  static constexpr uint32_t TM_DQ = (D == 64) ? 384 : 0;  // D=128 reuses S^T's columns
+  static constexpr bool kDqAliasesS = (D != 64);
 };
 
 // barrier indices
 enum {
   B_KV_FULL = 0, B_KV_EMPTY, B_S_FULL, B_DP_FULL, B_DS_READY, B_DS_FREE, B_DQ_FULL, B_DQ_EMPTY,
-  B_DKDV_FULL, B_DKDV_EMPTY, B_FINAL, B_Q_FULL0 = 14
+  B_DKDV_FULL, B_DKDV_EMPTY, B_FINAL, B_STAGE0 = 16
 };
 
 template <int D, bool kAtomic>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(512, 1)
     dash_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                     const BwdParams p) {
@@ -96,8 +102,10 @@ __global__ void __launch_bounds__(320, 1)
   const float* del_s = reinterpret_cast<const float*>(gb + C::OFF_DEL);
   const uint32_t bar0 = sb + C::OFF_BAR;
   auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
-  auto Q_FULL = [&](int s) { return BAR(B_Q_FULL0 + s); };
-  auto Q_EMPTY = [&](int s) { return BAR(B_Q_FULL0 + ST + s); };
+  auto Q_FULL = [&](int s) { return BAR(B_STAGE0 + s); };
+  auto Q_EMPTY = [&](int s) { return BAR(B_STAGE0 + ST + s); };
+  auto DO_FULL = [&](int s) { return BAR(B_STAGE0 + 2 * ST + s); };
+  auto DO_EMPTY = [&](int s) { return BAR(B_STAGE0 + 3 * ST + s); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gb + C::OFF_TMEM_SLOT);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -108,7 +116,7 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(BAR(B_KV_EMPTY), 1);
     mbar_init(BAR(B_S_FULL), 1);
     mbar_init(BAR(B_DP_FULL), 1);
-    mbar_init(BAR(B_DS_READY), 128);
+    mbar_init(BAR(B_DS_READY), 256);
     mbar_init(BAR(B_DS_FREE), 1);
     mbar_init(BAR(B_DQ_FULL), 1);
     mbar_init(BAR(B_DQ_EMPTY), 128);
@@ -118,6 +126,8 @@ __global__ void __launch_bounds__(320, 1)
     for (int s = 0; s < ST; ++s) {
       mbar_init(Q_FULL(s), 1);
       mbar_init(Q_EMPTY(s), 1);
+      mbar_init(DO_FULL(s), 1);
+      mbar_init(DO_EMPTY(s), 1);
     }
     fence_mbar_init();
     prefetch_tmap(&tmQ);
@@ -125,7 +135,7 @@ __global__ void __launch_bounds__(320, 1)
     prefetch_tmap(&tmV);
     prefetch_tmap(&tmDO);
   }
-  if (warp == 1) {
+  if (warp == 13) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
@@ -137,9 +147,10 @@ __global__ void __launch_bounds__(320, 1)
   const int cbeg = p.cta_off[blockIdx.x], cend = p.cta_off[blockIdx.x + 1];
   const int S = p.S, N = p.N;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+  if (warp >= 12) {
+    setmaxnreg_dec<C::kRegsCtrl>();
+    if (warp == 12 && lane == 0) {
+      // ---------------------------------------------------------- TMA producer
       int it = 0, cn = 0;
       for (int ci = cbeg; ci < cend; ++ci, ++cn) {
         const int4 ch = p.chains[ci];
@@ -148,34 +159,37 @@ __global__ void __launch_bounds__(320, 1)
         const int row_kv = ch.x * S + ch.y * 128;
 #pragma unroll
         for (int cb = 0; cb < D / 64; ++cb) {
-          tma_load_2d(sK + cb * 16384, &tmK, cb * 64, row_kv, BAR(B_KV_FULL));
           tma_load_2d(sV + cb * 16384, &tmV, cb * 64, row_kv, BAR(B_KV_FULL));
+          tma_load_2d(sK + cb * 16384, &tmK, cb * 64, row_kv, BAR(B_KV_FULL));
         }
         for (int t = 0; t < ch.w; ++t, ++it) {
           const int q = (int)(p.pairs[ch.z + t] & 0xffffu);
           const int s = it % ST;
-          if (it >= ST) mbar_wait(Q_EMPTY(s), ((it / ST) - 1) & 1, lim, p.err, p.abort_flag);
-          mbar_expect_tx(Q_FULL(s), 2 * C::kTile + 1024);
           const int row_q = ch.x * S + q * 128;
+          // dO first: the MMA issuer consumes it first (dP^T) and frees it first (after dV)
+          if (it >= ST) mbar_wait(DO_EMPTY(s), ((it / ST) - 1) & 1, lim, p.err, p.abort_flag);
+          mbar_expect_tx(DO_FULL(s), C::kTile + 512);
 #pragma unroll
-          for (int cb = 0; cb < D / 64; ++cb) {
+          for (int cb = 0; cb < D / 64; ++cb)
+            tma_load_2d(sDO + s * C::kTile + cb * 16384, &tmDO, cb * 64, row_q, DO_FULL(s));
+          bulk_load(sb + C::OFF_DEL + s * 512, p.delta + row_q, 512, DO_FULL(s));
+          if (it >= ST) mbar_wait(Q_EMPTY(s), ((it / ST) - 1) & 1, lim, p.err, p.abort_flag);
+          mbar_expect_tx(Q_FULL(s), C::kTile + 512);
+#pragma unroll
+          for (int cb = 0; cb < D / 64; ++cb)
             tma_load_2d(sQ + s * C::kTile + cb * 16384, &tmQ, cb * 64, row_q, Q_FULL(s));
-            tma_load_2d(sDO + s * C::kTile + cb * 16384, &tmDO, cb * 64, row_q, Q_FULL(s));
-          }
           bulk_load(sb + C::OFF_LSE + s * 512, p.lse2 + row_q, 512, Q_FULL(s));
-          bulk_load(sb + C::OFF_DEL + s * 512, p.delta + row_q, 512, Q_FULL(s));
         }
       }
       // drain: every issued load has landed before the CTA can exit
       for (int s = 0; s < ST && s < it; ++s) {
         const int last_use = ((it - 1 - s) / ST) * ST + s;
+        mbar_wait(DO_FULL(s), (last_use / ST) & 1, lim, p.err, p.abort_flag);
         mbar_wait(Q_FULL(s), (last_use / ST) & 1, lim, p.err, p.abort_flag);
       }
       if (cn > 0) mbar_wait(BAR(B_KV_FULL), (cn - 1) & 1, lim, p.err, p.abort_flag);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    } else if (warp == 13 && lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
       constexpr uint32_t ID_SS = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t ID_KV = idesc_bf16_f32(128, D, 0, 1);
       constexpr uint32_t ID_Q = idesc_bf16_f32(128, D, 1, 1);
@@ -190,21 +204,9 @@ __global__ void __launch_bounds__(320, 1)
         for (int t = 0; t < cnt; ++t, ++it) {
           const int s = it % ST;
           const uint32_t q_s = sQ + s * C::kTile, do_s = sDO + s * C::kTile;
-          mbar_wait(Q_FULL(s), (it / ST) & 1, lim, p.err, p.abort_flag);
+          // dP^T = V dO^T : M = kv, N = q, K = D (both operands K-major)
+          mbar_wait(DO_FULL(s), (it / ST) & 1, lim, p.err, p.abort_flag);
           tc_fence_after();
-          // S^T = K Q^T : M = kv, N = q, K = D (both operands K-major)
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            tc_mma_ss(tS, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(q_s + off, 16, 1024), ID_SS,
-                      kk > 0);
-          }
-          tc_commit(BAR(B_S_FULL));
-          if (C::kDqAliasesDp && it > 0) {
-            mbar_wait(BAR(B_DQ_EMPTY), (it - 1) & 1, lim, p.err, p.abort_flag);
-            tc_fence_after();
-          }
-          // dP^T = V dO^T
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -212,26 +214,38 @@ __global__ void __launch_bounds__(320, 1)
                       ID_SS, kk > 0);
           }
           tc_commit(BAR(B_DP_FULL));
+          // S^T = K Q^T
+          mbar_wait(Q_FULL(s), (it / ST) & 1, lim, p.err, p.abort_flag);
+          if (C::kDqAliasesS && it > 0) mbar_wait(BAR(B_DQ_EMPTY), (it - 1) & 1, lim, p.err, p.abort_flag);
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            tc_mma_ss(tS, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(q_s + off, 16, 1024), ID_SS,
+                      kk > 0);
+          }
+          tc_commit(BAR(B_S_FULL));
           mbar_wait(BAR(B_DS_READY), it & 1, lim, p.err, p.abort_flag);
           tc_fence_after();
           // dV += P^T dO ; dK += dS^T Q : M = kv, N = D, K = q (A K-major, B MN-major)
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t offA = (kk >> 2) * 16384 + (kk & 3) * 32;
-            const uint32_t offB = kk * 2048;
-            tc_mma_ss(tDV, sdesc_sw128(sPt + offA, 16, 1024), sdesc_sw128(do_s + offB, 16384, 1024),
-                      ID_KV, (t > 0 || kk > 0) ? 1u : 0u);
+            tc_mma_ss(tDV, sdesc_sw128(sPt + offA, 16, 1024),
+                      sdesc_sw128(do_s + kk * 2048, 16384, 1024), ID_KV,
+                      (t > 0 || kk > 0) ? 1u : 0u);
           }
+          tc_commit(DO_EMPTY(s));
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t offA = (kk >> 2) * 16384 + (kk & 3) * 32;
-            const uint32_t offB = kk * 2048;
-            tc_mma_ss(tDK, sdesc_sw128(sDSt + offA, 16, 1024), sdesc_sw128(q_s + offB, 16384, 1024),
-                      ID_KV, (t > 0 || kk > 0) ? 1u : 0u);
+            tc_mma_ss(tDK, sdesc_sw128(sDSt + offA, 16, 1024),
+                      sdesc_sw128(q_s + kk * 2048, 16384, 1024), ID_KV,
+                      (t > 0 || kk > 0) ? 1u : 0u);
           }
           tc_commit(Q_EMPTY(s));
           if (t == cnt - 1) tc_commit(BAR(B_DKDV_FULL));
-          if (!C::kDqAliasesDp && it > 0) {
+          if (!C::kDqAliasesS && it > 0) {
             mbar_wait(BAR(B_DQ_EMPTY), (it - 1) & 1, lim, p.err, p.abort_flag);
             tc_fence_after();
           }
@@ -250,9 +264,9 @@ __global__ void __launch_bounds__(320, 1)
       tc_commit(BAR(B_FINAL));
       mbar_wait(BAR(B_FINAL), 0, lim, p.err, p.abort_flag);
     }
-  } else if (warp < 6) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ softmax / dS
-    const int quarter = warp & 3;
+    const int quarter = warp & 3, half = warp >> 2;
     const int r = quarter * 32 + lane;  // KV row of the tile
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float sl2 = p.scale_log2;
@@ -262,23 +276,24 @@ __global__ void __launch_bounds__(320, 1)
       for (int t = 0; t < ch.w; ++t, ++it) {
         const int q = (int)(p.pairs[ch.z + t] & 0xffffu);
         const int s = it % ST;
+        mbar_wait(DO_FULL(s), (it / ST) & 1, lim, p.err, p.abort_flag);
         mbar_wait(Q_FULL(s), (it / ST) & 1, lim, p.err, p.abort_flag);
-        mbar_wait(BAR(B_S_FULL), it & 1, lim, p.err, p.abort_flag);
         mbar_wait(BAR(B_DP_FULL), it & 1, lim, p.err, p.abort_flag);
+        mbar_wait(BAR(B_S_FULL), it & 1, lim, p.err, p.abort_flag);
         if (it > 0) mbar_wait(BAR(B_DS_FREE), (it - 1) & 1, lim, p.err, p.abort_flag);
         tc_fence_after();
         const bool diag = p.causal && (q == ch.y);
         const float* lse_t = lse_s + s * 128;
         const float* del_t = del_s + s * 128;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
+          const int col0 = half * 64 + c * 32;
           uint32_t sv[32], dv[32];
-          tmem_ld32x2(tmem + lane_off + C::TM_S + c * 32, tmem + lane_off + C::TM_DP + c * 32, sv,
-                      dv);
+          tmem_ld32x2(tmem + lane_off + C::TM_S + col0, tmem + lane_off + C::TM_DP + col0, sv, dv);
           uint32_t pk[16], dk[16];
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
-            const int qc = c * 32 + j;
+            const int qc = col0 + j;
             float p0 = exp2f(fmaf(__uint_as_float(sv[j]), sl2, -lse_t[qc]));
             float p1 = exp2f(fmaf(__uint_as_float(sv[j + 1]), sl2, -lse_t[qc + 1]));
             if (diag) {
@@ -290,11 +305,11 @@ __global__ void __launch_bounds__(320, 1)
             pk[j >> 1] = pack_bf16x2(p0, p1);
             dk[j >> 1] = pack_bf16x2(d0, d1);
           }
-          const uint32_t row = (uint32_t)(c >> 1) * 16384 + (uint32_t)(r >> 3) * 1024 +
+          const uint32_t row = (uint32_t)half * 16384 + (uint32_t)(r >> 3) * 1024 +
                                (uint32_t)(r & 7) * 128;
 #pragma unroll
           for (int m = 0; m < 4; ++m) {
-            const uint32_t chunk = (uint32_t)((((c & 1) * 4 + m) ^ (r & 7)) * 16);
+            const uint32_t chunk = (uint32_t)(((c * 4 + m) ^ (r & 7)) * 16);
             st_shared_v4(sPt + row + chunk, pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
             st_shared_v4(sDSt + row + chunk, dk[4 * m], dk[4 * m + 1], dk[4 * m + 2],
                          dk[4 * m + 3]);
@@ -307,9 +322,12 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else {
     // ------------------------------------------------------------ dQ reduction + dK/dV epilogue
+    setmaxnreg_inc<C::kRegsReduce>();
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // row of the tile (Q row for dQ, KV row for dK/dV)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    constexpr int NV = D / 4;           // float4 per row
+    constexpr int G = 16;               // loads in flight per group
     int it = 0, cn = 0;
     for (int ci = cbeg; ci < cend; ++ci, ++cn) {
       const int4 ch = p.chains[ci];
@@ -351,46 +369,47 @@ __global__ void __launch_bounds__(320, 1)
             }
             __syncwarp();
             (void)ld_acquire_gpu(tk);
+            // acc += partial, G loads in flight before their adds
+#pragma unroll
+            for (int g0 = 0; g0 < NV; g0 += G) {
+              float4 old[G];
+#pragma unroll
+              for (int j = 0; j < G; ++j) old[j] = ld_cg_f4(accp + (g0 + j) * 128 + r);
+#pragma unroll
+              for (int j = 0; j < G; ++j) {
+                float* x = a + 4 * (g0 + j);
+                x[0] = old[j].x + x[0];
+                x[1] = old[j].y + x[1];
+                x[2] = old[j].z + x[2];
+                x[3] = old[j].w + x[3];
+              }
+            }
           }
           if (last) {
             __nv_bfloat16* out = p.dq + ((size_t)ch.x * S + (size_t)q * 128 + r) * D;
+            const float sc = p.scale;
 #pragma unroll
             for (int c8 = 0; c8 < D / 8; ++c8) {
-              float4 x0 = make_float4(a[8 * c8], a[8 * c8 + 1], a[8 * c8 + 2], a[8 * c8 + 3]);
-              float4 x1 = make_float4(a[8 * c8 + 4], a[8 * c8 + 5], a[8 * c8 + 6], a[8 * c8 + 7]);
-              if (pos > 0) {
-                const float4 o0 = ld_cg_f4(accp + (2 * c8) * 128 + r);
-                const float4 o1 = ld_cg_f4(accp + (2 * c8 + 1) * 128 + r);
-                x0.x = o0.x + x0.x; x0.y = o0.y + x0.y; x0.z = o0.z + x0.z; x0.w = o0.w + x0.w;
-                x1.x = o1.x + x1.x; x1.y = o1.y + x1.y; x1.z = o1.z + x1.z; x1.w = o1.w + x1.w;
-              }
-              const float sc = p.scale;
+              const float* x = a + 8 * c8;
               uint4 pk;
-              pk.x = pack_bf16x2(x0.x * sc, x0.y * sc);
-              pk.y = pack_bf16x2(x0.z * sc, x0.w * sc);
-              pk.z = pack_bf16x2(x1.x * sc, x1.y * sc);
-              pk.w = pack_bf16x2(x1.z * sc, x1.w * sc);
+              pk.x = pack_bf16x2(x[0] * sc, x[1] * sc);
+              pk.y = pack_bf16x2(x[2] * sc, x[3] * sc);
+              pk.z = pack_bf16x2(x[4] * sc, x[5] * sc);
+              pk.w = pack_bf16x2(x[6] * sc, x[7] * sc);
               *reinterpret_cast<uint4*>(out + 8 * c8) = pk;
             }
           } else {
 #pragma unroll
-            for (int c4 = 0; c4 < D / 4; ++c4) {
-              float4 x = make_float4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]);
-              if (pos > 0) {
-                const float4 o = ld_cg_f4(accp + c4 * 128 + r);
-                x.x = o.x + x.x; x.y = o.y + x.y; x.z = o.z + x.z; x.w = o.w + x.w;
-              }
-              st_cg_f4(accp + c4 * 128 + r, x);
-            }
+            for (int c4 = 0; c4 < NV; ++c4)
+              st_cg_f4(accp + c4 * 128 + r,
+                       make_float4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]));
+            __threadfence();
             named_bar_sync(1, 128);
-            if (threadIdx.x == 192) {
-              __threadfence();
-              st_release_gpu(p.tickets + blk, (uint32_t)(pos + 1));
-            }
+            if (threadIdx.x == 256) st_release_gpu(p.tickets + blk, (uint32_t)(pos + 1));
           }
         } else {
 #pragma unroll
-          for (int c4 = 0; c4 < D / 4; ++c4)
+          for (int c4 = 0; c4 < NV; ++c4)
             atomicAdd(accp + c4 * 128 + r,
                       make_float4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]));
         }
@@ -426,7 +445,7 @@ __global__ void __launch_bounds__(320, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

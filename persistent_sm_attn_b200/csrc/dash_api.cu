@@ -205,6 +205,11 @@ int num_ctas_for(int dev, int* out) {
   }
   auto kern = dash::dash_bwd_kernel<D, kAtomic>;
   DASH_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes));
+  // The kernel moves registers between warpgroups with setmaxnreg; the split
+  // adds up to exactly kLaunchRegs per thread, so refuse any other allocation.
+  cudaFuncAttributes fa;
+  DASH_CUDA(cudaFuncGetAttributes(&fa, kern));
+  if (fa.numRegs != C::kLaunchRegs) return DASH_ERR_UNSUPPORTED;
   int per_sm = 0, sms = 0;
   DASH_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, C::kThreads, C::kSmemBytes));
   DASH_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));

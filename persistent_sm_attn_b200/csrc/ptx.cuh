@@ -59,11 +59,11 @@ enum : unsigned {
 __device__ __forceinline__ bool aborted(const unsigned* abort_flag) {
   return *reinterpret_cast<const volatile unsigned*>(abort_flag) != 0u;
 }
-__device__ __noinline__ void raise_timeout(unsigned* err, unsigned* abort_flag, unsigned where) {
+__device__ __forceinline__ void raise_timeout(unsigned* err, unsigned* abort_flag, unsigned where) {
   atomicOr(err, ERR_TIMEOUT | where);
   atomicOr(abort_flag, 1u);
 }
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns,
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns,
                                        unsigned* err, unsigned* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
@@ -215,6 +215,14 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                                              uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
                : "memory");
+}
+template <uint32_t R>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
+}
+template <uint32_t R>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
 }
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
