@@ -126,6 +126,40 @@ int dash_profile_end(double* main_ms, double* aux_ms, long long* launches);
 int dash_release_workspace(void);
 
 /* ---------------------------------------------------------------------------
+ * Backward pass that allocates nothing.
+ *
+ * The paper has no counterpart to this entry point; it serves callers that
+ * cannot call cudaMalloc: code running while a stream is captured into a CUDA
+ * graph, runtimes that hand out all device memory from their own pool, and
+ * embedded users that must fix their device footprint in advance.
+ *
+ * Same arguments, supported shapes, schedules and results as dash_attn_bwd
+ * (q..dv caller-owned device memory; the caller still passes every input and
+ * output).  All scratch memory comes from one statically allocated device
+ * array of DASH_NOALLOC_SCRATCH_BYTES bytes, which every GPU that loads the
+ * library holds until the process exits.  The call never calls cudaMalloc,
+ * cudaFree or an allocating library routine.
+ *   - Size limit: the array must hold the fp32 dQ accumulator (B*H*S*D*4
+ *     bytes), the per-row Delta and scaled LSE (2*B*H*S*4), one ticket per
+ *     128-row dQ block and the schedule table; larger calls return
+ *     DASH_ERR_OOM without touching the device.
+ *   - Set-up: the first call on a device (with that device current) looks up
+ *     the array's device address and sizes the persistent grid; make that
+ *     first call before any stream capture begins.
+ *   - Sharing: every call uses the same array, which keeps the previous call's
+ *     contents; the call clears what must start at zero.  Calls that overlap
+ *     on the GPU (for example on two streams without ordering between them)
+ *     race on the array and give wrong results.
+ *   - Device-side timeouts of this entry point are recorded in the array, not
+ *     in the per-stream workspaces, so dash_attn_sync_status does not report
+ *     them; the spin limit is DASH_SPIN_LIMIT_US (default 10 s).
+ */
+#define DASH_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+int dash_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                          const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                          int B, int H, int S, int D, int causal, int schedule, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Host-only entry points (no GPU needed).
  */
 

@@ -21,7 +21,7 @@ STATUS = {0: "DASH_OK", 1: "DASH_ERR_INVALID_ARG", 2: "DASH_ERR_UNSUPPORTED", 3:
 EXPORTS = ("dash_attn_fwd", "dash_attn_bwd", "dash_attn_sync_status", "dash_status_string",
            "dash_set_spin_limit_us", "dash_bwd_num_ctas", "dash_release_workspace",
            "dash_sched_table", "dash_sched_simulate", "dash_dag_longest_path",
-           "dash_profile_begin", "dash_profile_end")
+           "dash_profile_begin", "dash_profile_end", "dash_attn_bwd_noalloc")
 
 
 class DashError(RuntimeError):
@@ -51,6 +51,7 @@ def load(path: str | None = None):
     P = ctypes.POINTER
     lib.dash_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, vp]
     lib.dash_attn_bwd.argtypes = [vp] * 9 + [i, i, i, i, i, i, vp]
+    lib.dash_attn_bwd_noalloc.argtypes = [vp] * 9 + [i, i, i, i, i, i, vp]
     lib.dash_attn_sync_status.argtypes = [vp]
     lib.dash_status_string.argtypes = [i]
     lib.dash_status_string.restype = ctypes.c_char_p
@@ -124,6 +125,23 @@ def dash_attn_bwd(q, k, v, o, do, lse, causal: bool, schedule="shift", dq=None, 
                               _ptr(dk), _ptr(dv), B, H, S, D, int(bool(causal)),
                               _sched_id(schedule), _stream_handle(stream))
     _check(rc, "dash_attn_bwd")
+    return dq, dk, dv
+
+
+def dash_attn_bwd_noalloc(q, k, v, o, do, lse, causal: bool, schedule, dq, dk, dv,
+                          stream=None):
+    """The backward through the entry point that allocates no device memory.
+    Outputs must be preallocated; all scratch comes from the library's static
+    device array (see include/dash_attn.h)."""
+    for t in (q, k, v, o, do, lse, dq, dk, dv):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("tensors must be contiguous CUDA tensors")
+    B, H, S, D = q.shape
+    rc = load().dash_attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse),
+                                      _ptr(dq), _ptr(dk), _ptr(dv), B, H, S, D,
+                                      int(bool(causal)), _sched_id(schedule),
+                                      _stream_handle(stream))
+    _check(rc, "dash_attn_bwd_noalloc")
     return dq, dk, dv
 
 

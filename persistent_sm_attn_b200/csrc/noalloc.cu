@@ -1,0 +1,280 @@
+// dash_attn_bwd_noalloc: the backward pass without any device allocation.
+//
+// Some callers cannot call cudaMalloc: code that runs while a stream is being
+// captured into a CUDA graph, runtimes that own all device memory through
+// their own pool and forbid other allocations, or embedded callers that must
+// know their whole device footprint up front.  This entry point runs the same
+// kernels as dash_attn_bwd, but takes every byte of scratch memory (the fp32
+// dQ accumulator, the tickets, the per-row Delta and scaled LSE, the error
+// words and the schedule table) from one statically allocated device array of
+// kNoallocScratchBytes.  Every device that loads the library holds that array
+// until the process exits.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/dash_attn.h"
+#include "aux_kernels.cuh"
+#include "bwd_kernel.cuh"
+#include "sched.h"
+
+namespace {
+
+constexpr size_t kNoallocScratchBytes = size_t(DASH_NOALLOC_SCRATCH_BYTES);
+constexpr int kMaxDevices = 64;
+
+// The scratch array.  In host code `g_noalloc_scratch` names a host-side
+// stand-in, not device memory: its device address is obtained once per device
+// with cudaGetSymbolAddress and passed to the kernels.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+struct DeviceState {
+  bool ready = false;
+  unsigned char* base = nullptr;  // device address of g_noalloc_scratch on this device
+  int ctas[2][2] = {{0, 0}, {0, 0}};  // [D==128][atomic]
+  // key of the schedule table currently held in the scratch array
+  long long table_key[6] = {-1, -1, -1, -1, -1, -1};
+};
+DeviceState g_dev[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn noalloc_encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+int noalloc_tmap(CUtensorMap* m, const void* base, long long rows, int D) {
+  EncodeTiledFn fn = noalloc_encode_fn();
+  if (!fn) return DASH_ERR_CUDA;
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DASH_OK : DASH_ERR_CUDA;
+}
+
+template <int D, bool kAtomic>
+int noalloc_ctas(int dev) {
+  using C = dash::BwdCfg<D>;
+  auto kern = dash::dash_bwd_kernel<D, kAtomic>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+      cudaSuccess)
+    return -DASH_ERR_CUDA;
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return -DASH_ERR_CUDA;
+  if (fa.numRegs != C::kLaunchRegs) return -DASH_ERR_UNSUPPORTED;
+  int per_sm = 0, sms = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, C::kThreads, C::kSmemBytes) !=
+          cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return -DASH_ERR_CUDA;
+  if (per_sm < 1) return -DASH_ERR_UNSUPPORTED;
+  return per_sm * sms;
+}
+
+// Once per device, with that device current: the scratch array's device
+// address and the persistent grid sizes.
+int noalloc_setup(int dev, DeviceState** out) {
+  DeviceState& st = g_dev[dev];
+  if (!st.ready) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) {
+      cudaGetLastError();
+      return DASH_ERR_CUDA;
+    }
+    st.base = static_cast<unsigned char*>(ptr);
+    const int c[4] = {noalloc_ctas<64, false>(dev), noalloc_ctas<64, true>(dev),
+                      noalloc_ctas<128, false>(dev), noalloc_ctas<128, true>(dev)};
+    for (int i = 0; i < 4; ++i)
+      if (c[i] < 0) return -c[i];
+    st.ctas[0][0] = c[0];
+    st.ctas[0][1] = c[1];
+    st.ctas[1][0] = c[2];
+    st.ctas[1][1] = c[3];
+    st.ready = true;
+  }
+  *out = &st;
+  return DASH_OK;
+}
+
+// Spin limit of the device waits: DASH_SPIN_LIMIT_US if set, else 10 s.
+unsigned long long noalloc_spin_ns() {
+  const char* e = std::getenv("DASH_SPIN_LIMIT_US");
+  const long long us = e ? std::atoll(e) : 0;
+  return (unsigned long long)(us > 0 ? us : 10LL * 1000 * 1000) * 1000ull;
+}
+
+// Scratch bytes a call needs, table excluded.
+size_t fixed_scratch(long long rows, int D, long long blocks) {
+  return 256                                         // error word + abort flag
+         + align256((size_t)blocks * 4)              // tickets
+         + 2 * align256((size_t)rows * 4)            // scaled LSE, Delta
+         + align256((size_t)rows * D * 4);           // fp32 dQ accumulator
+}
+
+template <int D, bool kAtomic>
+int noalloc_launch(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                   const float* lse, void* dq, void* dk, void* dv, int B, int H, int S,
+                   int causal, int sched, cudaStream_t stream, DeviceState* st) {
+  using C = dash::BwdCfg<D>;
+  const int N = S / 128;
+  const long long rows = (long long)B * H * S;
+  const long long blocks = (long long)B * H * N;
+  const int ctas = st->ctas[D == 128][kAtomic ? 1 : 0];
+  // lay out the scratch array
+  unsigned char* p0 = st->base;
+  unsigned* err = reinterpret_cast<unsigned*>(p0);
+  size_t off = 256;
+  uint32_t* tickets = reinterpret_cast<uint32_t*>(p0 + off);
+  off += align256((size_t)blocks * 4);
+  float* lse2 = reinterpret_cast<float*>(p0 + off);
+  off += align256((size_t)rows * 4);
+  float* delta = reinterpret_cast<float*>(p0 + off);
+  off += align256((size_t)rows * 4);
+  float* acc = reinterpret_cast<float*>(p0 + off);
+  off += align256((size_t)rows * D * 4);
+  // the schedule table, built and checked on the host, then copied in
+  const long long key[6] = {B * (long long)H, N, causal, sched, ctas, (long long)off};
+  dash::Table t;
+  std::string msg;
+  if (!dash::build_table(B * H, N, causal, sched, ctas, &t, &msg)) return DASH_ERR_UNSUPPORTED;
+  const size_t off_cta = off;
+  const size_t off_chain = off_cta + align256(t.cta_off.size() * sizeof(int));
+  const size_t off_pair = off_chain + align256(t.chains.size() * sizeof(int4));
+  const size_t end = off_pair + align256(t.pairs.size() * sizeof(uint32_t));
+  if (end > kNoallocScratchBytes) return DASH_ERR_OOM;
+  if (std::memcmp(key, st->table_key, sizeof(key)) != 0) {
+    if (!dash::validate_table(t, &msg)) return DASH_ERR_SCHEDULE;
+    if (cudaMemcpyAsync(p0 + off_cta, t.cta_off.data(), t.cta_off.size() * sizeof(int),
+                        cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+        cudaMemcpyAsync(p0 + off_chain, t.chains.data(), t.chains.size() * sizeof(int4),
+                        cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+        cudaMemcpyAsync(p0 + off_pair, t.pairs.data(), t.pairs.size() * sizeof(uint32_t),
+                        cudaMemcpyHostToDevice, stream) != cudaSuccess)
+      return DASH_ERR_CUDA;
+    std::memcpy(st->table_key, key, sizeof(key));
+  }
+  CUtensorMap tq, tk, tv, tdo;
+  int rc;
+  if ((rc = noalloc_tmap(&tq, q, rows, D)) || (rc = noalloc_tmap(&tk, k, rows, D)) ||
+      (rc = noalloc_tmap(&tv, v, rows, D)) || (rc = noalloc_tmap(&tdo, dout, rows, D)))
+    return rc;
+  // the array keeps the previous call's contents: clear what must start at zero
+  if (cudaMemsetAsync(err, 0, 2 * sizeof(unsigned), stream) != cudaSuccess) return DASH_ERR_CUDA;
+  if (kAtomic) {
+    if (cudaMemsetAsync(acc, 0, (size_t)rows * D * 4, stream) != cudaSuccess) return DASH_ERR_CUDA;
+  } else {
+    if (cudaMemsetAsync(tickets, 0, (size_t)blocks * 4, stream) != cudaSuccess)
+      return DASH_ERR_CUDA;
+  }
+  {
+    const long long threads = rows * (D / 8);
+    dash::dash_delta_kernel<D><<<(int)((threads + 255) / 256), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, delta,
+        lse2, rows);
+  }
+  dash::BwdParams p;
+  p.lse2 = lse2;
+  p.delta = delta;
+  p.cta_off = reinterpret_cast<const int*>(p0 + off_cta);
+  p.chains = reinterpret_cast<const int4*>(p0 + off_chain);
+  p.pairs = reinterpret_cast<const uint32_t*>(p0 + off_pair);
+  p.acc = acc;
+  p.tickets = tickets;
+  p.err = err;
+  p.abort_flag = err + 1;
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.S = S;
+  p.N = N;
+  p.causal = causal;
+  p.scale = 1.0f / sqrtf((float)D);
+  p.scale_log2 = p.scale * 1.4426950408889634f;
+  p.spin_ns = noalloc_spin_ns();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ctas);
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, dash::dash_bwd_kernel<D, kAtomic>, tq, tk, tv, tdo, p) !=
+      cudaSuccess)
+    return DASH_ERR_CUDA;
+  if (kAtomic) {
+    const long long threads = blocks * 128 * (D / 4);
+    dash::dash_dq_convert<D><<<(int)((threads + 255) / 256), 256, 0, stream>>>(
+        acc, static_cast<__nv_bfloat16*>(dq), blocks, p.scale);
+  }
+  return cudaGetLastError() == cudaSuccess ? DASH_OK : DASH_ERR_CUDA;
+}
+
+bool aligned16(const void* ptr) { return ptr && (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" int dash_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                                     const void* dout, const float* lse, void* dq, void* dk,
+                                     void* dv, int B, int H, int S, int D, int causal,
+                                     int schedule, void* stream) {
+  if (B < 0 || H < 0 || S < 0 || D < 0) return DASH_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return DASH_ERR_INVALID_ARG;
+  if (schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_ATOMIC) return DASH_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return DASH_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return DASH_ERR_UNSUPPORTED;
+  if (S == 0 || S % 128 != 0 || S / 128 > 32767) return DASH_ERR_UNSUPPORTED;
+  if ((long long)B * H * S >= (1LL << 31)) return DASH_ERR_UNSUPPORTED;
+  if (!dash::schedule_supported(schedule, S / 128, causal)) return DASH_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0) return DASH_OK;
+  // reject sizes beyond the array before touching the device
+  const long long rows = (long long)B * H * S, blocks = (long long)B * H * (S / 128);
+  if (fixed_scratch(rows, D, blocks) > kNoallocScratchBytes) return DASH_ERR_OOM;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DASH_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return DASH_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  DeviceState* st = nullptr;
+  int rc = noalloc_setup(dev, &st);
+  if (rc) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool atomic = (schedule == DASH_SCHED_ATOMIC);
+  if (D == 64)
+    return atomic ? noalloc_launch<64, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
+                                             schedule, s, st)
+                  : noalloc_launch<64, false>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
+                                              schedule, s, st);
+  return atomic ? noalloc_launch<128, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
+                                            schedule, s, st)
+                : noalloc_launch<128, false>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
+                                             schedule, s, st);
+}
