@@ -121,6 +121,22 @@ int dash_bwd_num_ctas(int device, int D, int* num_ctas);
 int dash_profile_begin(void);
 int dash_profile_end(double* main_ms, double* aux_ms, long long* launches);
 
+/*
+ * Diagnostic: one synchronous backward (same arguments as dash_attn_bwd) with
+ * a %globaltimer trace of every (KV tile, Q tile) pair, for measuring the
+ * compute time c and the reduction time r of the DAG model (DASH summary
+ * §2.1).  host_trace receives up to `cap` u64 entries laid out
+ * [num_ctas][rows_per_cta][8] (unused rows stay 0); events per pair: 0 tile
+ * start at the MMA issuer, 1 softmax done, 2 tile MMAs issued, 3 softmax start,
+ * 4 dQ partial ready at the reducers, 5 partial drained from TMEM, 6 ticket
+ * granted (0 for a block's first contributor), 7 reduction published.
+ * Allocates and frees its own trace buffer.
+ */
+int dash_trace_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                   const float* lse, void* dq, void* dk, void* dv, int B, int H, int S, int D,
+                   int causal, int schedule, void* stream, unsigned long long* host_trace,
+                   long long cap, int* num_ctas, int* rows_per_cta);
+
 /* Frees every cached workspace and schedule table of the current device
  * (synchronises the device first). */
 int dash_release_workspace(void);

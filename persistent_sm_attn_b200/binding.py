@@ -21,7 +21,8 @@ STATUS = {0: "DASH_OK", 1: "DASH_ERR_INVALID_ARG", 2: "DASH_ERR_UNSUPPORTED", 3:
 EXPORTS = ("dash_attn_fwd", "dash_attn_bwd", "dash_attn_sync_status", "dash_status_string",
            "dash_set_spin_limit_us", "dash_bwd_num_ctas", "dash_release_workspace",
            "dash_sched_table", "dash_sched_simulate", "dash_dag_longest_path",
-           "dash_profile_begin", "dash_profile_end", "dash_attn_bwd_noalloc")
+           "dash_profile_begin", "dash_profile_end", "dash_attn_bwd_noalloc",
+           "dash_trace_bwd")
 
 
 class DashError(RuntimeError):
@@ -62,6 +63,7 @@ def load(path: str | None = None):
     lib.dash_sched_table.restype = ll
     lib.dash_sched_simulate.argtypes = [i, i, i, i, i, d, d, i, P(d), P(d), P(d), P(ll)]
     lib.dash_dag_longest_path.argtypes = [i, i, vp, vp, vp, vp, vp, P(d)]
+    lib.dash_trace_bwd.argtypes = [vp] * 9 + [i, i, i, i, i, i, vp, vp, ll, P(i), P(i)]
     lib.dash_profile_begin.argtypes = []
     lib.dash_profile_end.argtypes = [P(d), P(d), P(ll)]
     for name in EXPORTS:
@@ -213,3 +215,25 @@ def dash_profile_end():
     _check(load().dash_profile_end(ctypes.byref(m), ctypes.byref(a), ctypes.byref(n)),
            "dash_profile_end")
     return m.value, a.value, n.value
+
+
+def dash_trace_bwd(q, k, v, o, do, lse, causal: bool, schedule="shift", stream=None):
+    """One traced backward; returns (dq, dk, dv, trace [ctas, rows, 8] uint64 ns)."""
+    import numpy as np
+    import torch
+    B, H, S, D = q.shape
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    N = S // 128
+    cap = 8 * (B * H * N * N + 1024 * (N + 1))   # >= ctas * rows_per_cta * 8
+    buf = np.zeros(cap, dtype=np.uint64)
+    nc, rows = ctypes.c_int(), ctypes.c_int()
+    rc = load().dash_trace_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
+                               _ptr(dk), _ptr(dv), B, H, S, D, int(bool(causal)),
+                               _sched_id(schedule), _stream_handle(stream),
+                               buf.ctypes.data_as(ctypes.c_void_p), cap, ctypes.byref(nc),
+                               ctypes.byref(rows))
+    _check(rc, "dash_trace_bwd")
+    n = nc.value * rows.value * 8
+    if n > cap:
+        raise RuntimeError("trace buffer too small")
+    return dq, dk, dv, buf[:n].reshape(nc.value, rows.value, 8)

@@ -48,6 +48,10 @@ struct BwdParams {
   int S, N, causal;
   float scale, scale_log2;
   unsigned long long spin_ns;
+  // Optional %globaltimer trace (kernels instantiated with kTrace only):
+  // trace[(cta * trace_rows + pair) * 8 + event], events listed at kTrace.
+  unsigned long long* trace = nullptr;
+  int trace_rows = 0;
 };
 
 template <int D>
@@ -84,7 +88,11 @@ enum {
   B_DKDV_FULL, B_DKDV_EMPTY, B_FINAL, B_STAGE0 = 16
 };
 
-template <int D, bool kAtomic>
+// kTrace: record %globaltimer per pair of this CTA: 0 MMA tile start, 1 softmax
+// done (seen by the MMA issuer), 2 tile MMAs issued, 3 softmax start, 4 dQ
+// partial ready (seen by the reducers), 5 partial drained, 6 ticket granted,
+// 7 reduction published.
+template <int D, bool kAtomic, bool kTrace = false>
 __global__ void __launch_bounds__(512, 1)
     dash_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -110,6 +118,12 @@ __global__ void __launch_bounds__(512, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint64_t lim = p.spin_ns;
+  auto trace = [&](int pair, int ev) {
+    if constexpr (kTrace) {
+      if (pair < p.trace_rows)
+        p.trace[((size_t)blockIdx.x * p.trace_rows + pair) * 8 + ev] = globaltimer();
+    }
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(BAR(B_KV_FULL), 1);
@@ -205,6 +219,7 @@ __global__ void __launch_bounds__(512, 1)
           const int s = it % ST;
           const uint32_t q_s = sQ + s * C::kTile, do_s = sDO + s * C::kTile;
           // dP^T = V dO^T : M = kv, N = q, K = D (both operands K-major)
+          trace(it, 0);
           mbar_wait(DO_FULL(s), (it / ST) & 1, lim, p.err, p.abort_flag);
           tc_fence_after();
 #pragma unroll
@@ -226,6 +241,7 @@ __global__ void __launch_bounds__(512, 1)
           }
           tc_commit(BAR(B_S_FULL));
           mbar_wait(BAR(B_DS_READY), it & 1, lim, p.err, p.abort_flag);
+          trace(it, 1);
           tc_fence_after();
           // dV += P^T dO ; dK += dS^T Q : M = kv, N = D, K = q (A K-major, B MN-major)
 #pragma unroll
@@ -257,6 +273,7 @@ __global__ void __launch_bounds__(512, 1)
           }
           tc_commit(BAR(B_DQ_FULL));
           tc_commit(BAR(B_DS_FREE));
+          trace(it, 2);
         }
         tc_commit(BAR(B_KV_EMPTY));
       }
@@ -281,6 +298,7 @@ __global__ void __launch_bounds__(512, 1)
         mbar_wait(BAR(B_DP_FULL), it & 1, lim, p.err, p.abort_flag);
         mbar_wait(BAR(B_S_FULL), it & 1, lim, p.err, p.abort_flag);
         if (it > 0) mbar_wait(BAR(B_DS_FREE), (it - 1) & 1, lim, p.err, p.abort_flag);
+        if (threadIdx.x == 0) trace(it, 3);
         tc_fence_after();
         const bool diag = p.causal && (q == ch.y);
         const float* lse_t = lse_s + s * 128;
@@ -337,6 +355,7 @@ __global__ void __launch_bounds__(512, 1)
         const int ncontrib = p.causal ? q + 1 : N;
         const bool last = (pos == ncontrib - 1);
         mbar_wait(BAR(B_DQ_FULL), it & 1, lim, p.err, p.abort_flag);
+        if (threadIdx.x == 256) trace(it, 4);
         tc_fence_after();
         float a[D];
 #pragma unroll
@@ -348,6 +367,7 @@ __global__ void __launch_bounds__(512, 1)
         }
         tc_fence_before();
         mbar_arrive(BAR(B_DQ_EMPTY));
+        if (threadIdx.x == 256) trace(it, 5);
         const long long blk = (long long)ch.x * N + q;
         float4* accp = reinterpret_cast<float4*>(p.acc + blk * 128 * D);
         if constexpr (!kAtomic) {
@@ -369,6 +389,7 @@ __global__ void __launch_bounds__(512, 1)
             }
             __syncwarp();
             (void)ld_acquire_gpu(tk);
+            if (threadIdx.x == 256) trace(it, 6);
             // acc += partial, G loads in flight before their adds
 #pragma unroll
             for (int g0 = 0; g0 < NV; g0 += G) {
@@ -407,6 +428,7 @@ __global__ void __launch_bounds__(512, 1)
             named_bar_sync(1, 128);
             if (threadIdx.x == 256) st_release_gpu(p.tickets + blk, (uint32_t)(pos + 1));
           }
+          if (threadIdx.x == 256) trace(it, 7);
         } else {
 #pragma unroll
           for (int c4 = 0; c4 < NV; ++c4)

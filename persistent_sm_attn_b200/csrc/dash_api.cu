@@ -219,10 +219,11 @@ int num_ctas_for(int dev, int* out) {
   return DASH_OK;
 }
 
-template <int D, bool kAtomic>
+template <int D, bool kAtomic, bool kTrace = false>
 int launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                const float* lse, void* dq, void* dk, void* dv, int B, int H, int S, int causal,
-               int sched, cudaStream_t stream, int dev) {
+               int sched, cudaStream_t stream, int dev, unsigned long long* trace = nullptr,
+               int trace_rows = 0) {
   using C = BwdCfg<D>;
   const int N = S / 128;
   const long long rows = (long long)B * H * S;
@@ -278,6 +279,8 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   p.scale = 1.0f / sqrtf((float)D);
   p.scale_log2 = p.scale * 1.4426950408889634f;
   p.spin_ns = (unsigned long long)spin_us() * 1000ull;
+  p.trace = trace;
+  p.trace_rows = trace_rows;
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ctas);
@@ -290,7 +293,16 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (!prof_record(1, &ev, stream)) return DASH_ERR_CUDA;
-  DASH_CUDA(cudaLaunchKernelEx(&cfg, dash::dash_bwd_kernel<D, kAtomic>, tq, tk, tv, tdo, p));
+  if (kTrace) {
+    auto kt = dash::dash_bwd_kernel<D, kAtomic, true>;
+    DASH_CUDA(cudaFuncSetAttribute(kt, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes));
+    cudaFuncAttributes fa;
+    DASH_CUDA(cudaFuncGetAttributes(&fa, kt));
+    if (fa.numRegs != C::kLaunchRegs) return DASH_ERR_UNSUPPORTED;
+    DASH_CUDA(cudaLaunchKernelEx(&cfg, kt, tq, tk, tv, tdo, p));
+  } else {
+    DASH_CUDA(cudaLaunchKernelEx(&cfg, dash::dash_bwd_kernel<D, kAtomic>, tq, tk, tv, tdo, p));
+  }
   if (!prof_record(2, &ev, stream)) return DASH_ERR_CUDA;
   if (kAtomic) {
     const long long n_blocks = (long long)B * H * N;
@@ -474,6 +486,70 @@ int dash_release_workspace(void) {
     }
   }
   return DASH_OK;
+}
+
+int dash_trace_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                   const float* lse, void* dq, void* dk, void* dv, int B, int H, int S, int D,
+                   int causal, int schedule, void* stream, unsigned long long* host_trace,
+                   long long cap, int* num_ctas, int* rows_per_cta) {
+  int rc = check_shape(B, H, S, D);
+  if (rc) return rc;
+  if (causal != 0 && causal != 1) return DASH_ERR_INVALID_ARG;
+  if (schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_ATOMIC) return DASH_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !host_trace ||
+      !num_ctas || !rows_per_cta)
+    return DASH_ERR_INVALID_ARG;
+  if (!dash::schedule_supported(schedule, S / 128, causal)) return DASH_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0) return DASH_ERR_INVALID_ARG;
+  int dev = 0;
+  DASH_CUDA(cudaGetDevice(&dev));
+  const bool atomic = (schedule == DASH_SCHED_ATOMIC);
+  int ctas = 0;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    rc = (D == 64) ? (atomic ? num_ctas_for<64, true>(dev, &ctas) : num_ctas_for<64, false>(dev, &ctas))
+                   : (atomic ? num_ctas_for<128, true>(dev, &ctas) : num_ctas_for<128, false>(dev, &ctas));
+  }
+  if (rc) return rc;
+  dash::Table t;
+  std::string err;
+  if (!dash::build_table(B * H, S / 128, causal, schedule, ctas, &t, &err)) return DASH_ERR_UNSUPPORTED;
+  int rows = 0;
+  for (int c = 0; c < ctas; ++c) {
+    int n = 0;
+    for (int ci = t.cta_off[c]; ci < t.cta_off[c + 1]; ++ci) n += t.chains[ci].pair_cnt;
+    rows = n > rows ? n : rows;
+  }
+  const size_t n_entries = (size_t)ctas * rows * 8;
+  unsigned long long* dtrace = nullptr;
+  if (cudaMalloc(&dtrace, n_entries * sizeof(unsigned long long)) != cudaSuccess) return DASH_ERR_OOM;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  rc = cudaMemsetAsync(dtrace, 0, n_entries * sizeof(unsigned long long), st) == cudaSuccess
+           ? DASH_OK : DASH_ERR_CUDA;
+  if (!rc) {
+    if (D == 64)
+      rc = atomic ? launch_bwd<64, true, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
+                                               schedule, st, dev, dtrace, rows)
+                  : launch_bwd<64, false, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
+                                                schedule, st, dev, dtrace, rows);
+    else
+      rc = atomic ? launch_bwd<128, true, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
+                                                schedule, st, dev, dtrace, rows)
+                  : launch_bwd<128, false, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S,
+                                                 causal, schedule, st, dev, dtrace, rows);
+  }
+  if (!rc && cudaStreamSynchronize(st) != cudaSuccess) rc = DASH_ERR_CUDA;
+  if (!rc) {
+    const size_t n = n_entries < (size_t)cap ? n_entries : (size_t)cap;
+    if (cudaMemcpy(host_trace, dtrace, n * sizeof(unsigned long long), cudaMemcpyDeviceToHost) !=
+        cudaSuccess)
+      rc = DASH_ERR_CUDA;
+  }
+  cudaFree(dtrace);
+  *num_ctas = ctas;
+  *rows_per_cta = rows;
+  return rc;
 }
 
 long long dash_sched_table(int n_heads, int N, int causal, int schedule, int num_ctas, int* rows,
