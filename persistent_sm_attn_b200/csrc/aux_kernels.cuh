@@ -48,19 +48,19 @@ __global__ void __launch_bounds__(256) dash_delta_kernel(const __nv_bfloat16* __
   }
 }
 
-// acc layout per 128-row block: [D/4][128][4] fp32.  One thread per (row, 4 columns).
+// fp32 accumulator -> bf16 dQ.  One accumulator block per 128-row Q tile,
+// laid out [D/4][128][4]: slot (c4, r) holds head dims 4*c4..4*c4+3 of row r.
+// One thread per float4 slot.
 template <int D>
 __global__ void __launch_bounds__(256) dash_dq_convert(const float* __restrict__ acc,
                                                        __nv_bfloat16* __restrict__ dq,
                                                        long long n_blocks, float scale) {
   const long long gt = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  const long long total = n_blocks * 128 * (D / 4);
-  if (gt >= total) return;
+  if (gt >= n_blocks * 32 * D) return;
   const int r = (int)(gt % 128);
-  const long long rest = gt / 128;
-  const int c4 = (int)(rest % (D / 4));
-  const long long blk = rest / (D / 4);
-  const float4 v = reinterpret_cast<const float4*>(acc)[(blk * (D / 4) + c4) * 128 + r];
+  const int c4 = (int)((gt / 128) % (D / 4));
+  const long long blk = gt / (32 * D);
+  const float4 v = reinterpret_cast<const float4*>(acc)[gt];
   __nv_bfloat162 lo = __floats2bfloat162_rn(v.x * scale, v.y * scale);
   __nv_bfloat162 hi = __floats2bfloat162_rn(v.z * scale, v.w * scale);
   uint2 pk;

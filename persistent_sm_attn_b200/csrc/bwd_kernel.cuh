@@ -1,25 +1,36 @@
 // Persistent deterministic attention backward for sm_100a.
 //
 // One CTA per SM runs the chains its schedule table lists ("Resumen Técnico:
-// DASH ..." §2.1: all pairs of one KV tile run back to back on one SM, with
-// the dK/dV accumulators on chip).  Per (KV tile j, Q tile i) pair:
+// DASH ..." §2.1: all pairs of one KV tile run back to back on one SM, with the
+// dK/dV accumulators on chip).  Per (KV tile j, Q tile i) pair of 128 x 128:
 //
-//   dP^T = V_j dO_i^T                 tcgen05.mma -> TMEM
-//   S^T  = K_j Q_i^T                  tcgen05.mma -> TMEM
-//   P^T  = exp(scale S^T - LSE_i),  dS^T = P^T (dP^T - Delta_i)   (softmax warps -> smem)
-//   dV_j += P^T dO_i,  dK_j += dS^T Q_i      tcgen05.mma, accumulators resident in TMEM
-//   dQp  = dS K_j                     tcgen05.mma -> TMEM
+//   dP^T = V_j dO_i^T                 tcgen05.mma (smem x smem) -> TMEM [128, 256)
+//   S^T  = K_j Q_i^T                  tcgen05.mma (smem x smem) -> TMEM [0, 128)
+//   P^T  = exp(scale S^T - LSE_i), dS^T = P^T (dP^T - Delta_i)     (softmax warps)
+//          P^T and dS^T go back to TMEM as bf16 in the columns S^T occupied;
+//          dS^T also goes to shared memory for the dQ product
+//   dV_j += P^T dO_i, dK_j += dS^T Q_i       tcgen05.mma with A in TMEM, accumulators in TMEM
+//   dQp  = dS K_j                     tcgen05.mma (smem x smem) -> TMEM
 //   ordered reduction of dQp into the fp32 accumulator of block (b,h,i): wait
-//   until the block's ticket equals this pair's position, add with plain
-//   loads and stores, publish, bump the ticket (§1: a fixed accumulation
-//   order makes dQ bitwise reproducible; §2.2 chooses the order).  The last
-//   contributor rounds the sum once to bf16 and writes dQ.
+//   until the block's ticket equals this pair's position, add with plain loads
+//   and stores, publish, bump the ticket (§1: a fixed accumulation order makes
+//   dQ bitwise reproducible; §2.2 chooses the order).  The last contributor
+//   rounds the sum once to bf16 and writes dQ.
+//
+// Taking P^T and dS^T from TMEM keeps two of the five products off the
+// shared-memory read path, which bounds the 1-CTA tensor cores here.
 //
 // Warp roles (512 threads, four warpgroups):
 //   WG0, WG1  softmax / dS; WG0 owns Q columns 0-63, WG1 columns 64-127
 //   WG2       dQ reduction and the dK/dV epilogue (176 registers)
 //   WG3       warp 12 TMA producer, warp 13 MMA issuer and TMEM owner (80 registers)
 // TMEM lane quarter of a warp is (warp % 4), so each warpgroup covers the 128 lanes.
+//
+// TMEM columns (512): S^T [0,128) then packed P^T/dS^T, dP^T [128,256),
+// dV [256,256+D), dK after it; dQp in the dP^T columns (D = 128) or in two
+// buffers [384,448) [448,512) (D = 64).  Packed layout after the softmax: the
+// 32 fp32 columns of chunk c (Q columns 32c..32c+31) hold P^T of those columns
+// in 32c..32c+15 and dS^T in 32c+16..32c+31, two bf16 per column.
 //
 // Shared-memory tiles are [128 rows][D] bf16 stored as D/64 column blocks of
 // 128 rows x 128 bytes with the 128-byte swizzle (the layout a TMA load with
@@ -39,7 +50,7 @@ struct BwdParams {
   const int4* chains;     // {bh, kv, pair_off, pair_cnt}
   const uint32_t* pairs;  // q | position << 16
   float* acc;             // fp32 dQ accumulator, per block [D/4][128][4]
-  uint32_t* tickets;      // [B*H*N]
+  uint32_t* tickets;      // one per 128-row dQ block
   unsigned* err;          // device error word (accumulates until read by the host)
   unsigned* abort_flag;   // per-launch: set by the first timeout, cleared before each launch
   __nv_bfloat16* dq;
@@ -63,29 +74,35 @@ struct BwdCfg {
   static_assert(2 * kLaunchRegs + kRegsReduce + kRegsCtrl == 4 * kLaunchRegs,
                 "register split must equal the launch allocation");
   static constexpr int kTile = 128 * D * 2;              // one [128][D] bf16 tile
-  static constexpr int kStages = (D == 64) ? 2 : 1;      // Q/dO pipeline depth
+  static constexpr int kStages = (D == 64) ? 3 : 2;      // Q/dO pipeline depth
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + kTile;
   static constexpr int OFF_Q = OFF_V + kTile;
   static constexpr int OFF_DO = OFF_Q + kStages * kTile;
-  static constexpr int OFF_PT = OFF_DO + kStages * kTile;  // P^T  [128 kv][128 q]
-  static constexpr int OFF_DST = OFF_PT + 32768;           // dS^T [128 kv][128 q]
-  static constexpr int OFF_LSE = OFF_DST + 32768;          // kStages x 128 fp32
+  static constexpr int OFF_DST = OFF_DO + kStages * kTile;  // dS^T [128 kv][128 q]
+  static constexpr int OFF_LSE = OFF_DST + 32768;           // kStages x 128 fp32
   static constexpr int OFF_DEL = OFF_LSE + kStages * 512;
   static constexpr int OFF_BAR = OFF_DEL + kStages * 512;
   static constexpr int kBars = 16 + 4 * kStages;
   static constexpr int OFF_TMEM_SLOT = OFF_BAR + kBars * 8;
-  static constexpr int kSmemBytes = OFF_TMEM_SLOT + 16 + 1024;  // + alignment slack
-  // TMEM columns
+  // The swizzled tiles need a 1 KiB aligned base; the kernel checks it.
+  static constexpr int kSmemBytes = OFF_TMEM_SLOT + 16;
+  static_assert(kSmemBytes <= 232448, "shared memory per block exceeded");
   static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 256 + D;
-  static constexpr uint32_t TM_DQ = (D == 64) ? 384 : 0;  // D=128 reuses S^T's columns
-  static constexpr bool kDqAliasesS = (D != 64);
+  static constexpr uint32_t TM_DQ = (D == 128) ? 128 : 384;
+  static constexpr bool kDqInDp = (D == 128);  // dQp reuses dP^T's columns
 };
+
+// Number of dQ reduction units (tickets): one per 128-row block.
+template <int D>
+constexpr long long dq_units(long long bh_times_n) {
+  return bh_times_n;
+}
 
 // barrier indices
 enum {
-  B_KV_FULL = 0, B_KV_EMPTY, B_S_FULL, B_DP_FULL, B_DS_READY, B_DS_FREE, B_DQ_FULL, B_DQ_EMPTY,
-  B_DKDV_FULL, B_DKDV_EMPTY, B_FINAL, B_STAGE0 = 16
+  B_KV_FULL = 0, B_KV_EMPTY, B_S_FULL, B_DP_FULL, B_DS_READY, B_DS_FREE, B_DQ_FULL0, B_DQ_FULL1,
+  B_DQ_EMPTY0, B_DQ_EMPTY1, B_DVDK_DONE, B_DKDV_FULL, B_DKDV_EMPTY, B_FINAL, B_STAGE0 = 16
 };
 
 // kTrace: record %globaltimer per pair of this CTA: 0 MMA tile start, 1 softmax
@@ -100,12 +117,18 @@ __global__ void __launch_bounds__(512, 1)
   using namespace dev;
   using C = BwdCfg<D>;
   constexpr int ST = C::kStages;
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t sb = (raw + 1023u) & ~1023u;
-  uint8_t* gb = smem_raw + (sb - raw);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t sb = smem_u32(smem_raw);
+  if (sb & 1023u) {  // the launch gave an unaligned base: refuse rather than misread
+    if (threadIdx.x == 0) {
+      atomicOr(p.err, ERR_MISALIGNED);
+      atomicOr(p.abort_flag, 1u);
+    }
+    return;
+  }
+  uint8_t* gb = smem_raw;
   const uint32_t sK = sb + C::OFF_K, sV = sb + C::OFF_V, sQ = sb + C::OFF_Q, sDO = sb + C::OFF_DO;
-  const uint32_t sPt = sb + C::OFF_PT, sDSt = sb + C::OFF_DST;
+  const uint32_t sDSt = sb + C::OFF_DST;
   const float* lse_s = reinterpret_cast<const float*>(gb + C::OFF_LSE);
   const float* del_s = reinterpret_cast<const float*>(gb + C::OFF_DEL);
   const uint32_t bar0 = sb + C::OFF_BAR;
@@ -118,12 +141,13 @@ __global__ void __launch_bounds__(512, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint64_t lim = p.spin_ns;
-  auto trace = [&](int pair, int ev) {
+  auto trace = [&](int row, int ev) {
     if constexpr (kTrace) {
-      if (pair < p.trace_rows)
-        p.trace[((size_t)blockIdx.x * p.trace_rows + pair) * 8 + ev] = globaltimer();
+      if (row < p.trace_rows)
+        p.trace[((size_t)blockIdx.x * p.trace_rows + row) * 8 + ev] = globaltimer();
     }
   };
+  auto wait = [&](uint32_t bar, uint32_t phase) { mbar_wait(bar, phase, lim, p.err, p.abort_flag); };
 
   if (threadIdx.x == 0) {
     mbar_init(BAR(B_KV_FULL), 1);
@@ -132,8 +156,11 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(BAR(B_DP_FULL), 1);
     mbar_init(BAR(B_DS_READY), 256);
     mbar_init(BAR(B_DS_FREE), 1);
-    mbar_init(BAR(B_DQ_FULL), 1);
-    mbar_init(BAR(B_DQ_EMPTY), 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(BAR(B_DQ_FULL0 + b), 1);
+      mbar_init(BAR(B_DQ_EMPTY0 + b), 128);
+    }
+    mbar_init(BAR(B_DVDK_DONE), 1);
     mbar_init(BAR(B_DKDV_FULL), 1);
     mbar_init(BAR(B_DKDV_EMPTY), 128);
     mbar_init(BAR(B_FINAL), 1);
@@ -168,7 +195,7 @@ __global__ void __launch_bounds__(512, 1)
       int it = 0, cn = 0;
       for (int ci = cbeg; ci < cend; ++ci, ++cn) {
         const int4 ch = p.chains[ci];
-        if (cn > 0) mbar_wait(BAR(B_KV_EMPTY), (cn - 1) & 1, lim, p.err, p.abort_flag);
+        if (cn > 0) wait(BAR(B_KV_EMPTY), (cn - 1) & 1);
         mbar_expect_tx(BAR(B_KV_FULL), 2 * C::kTile);
         const int row_kv = ch.x * S + ch.y * 128;
 #pragma unroll
@@ -181,13 +208,13 @@ __global__ void __launch_bounds__(512, 1)
           const int s = it % ST;
           const int row_q = ch.x * S + q * 128;
           // dO first: the MMA issuer consumes it first (dP^T) and frees it first (after dV)
-          if (it >= ST) mbar_wait(DO_EMPTY(s), ((it / ST) - 1) & 1, lim, p.err, p.abort_flag);
+          if (it >= ST) wait(DO_EMPTY(s), ((it / ST) - 1) & 1);
           mbar_expect_tx(DO_FULL(s), C::kTile + 512);
 #pragma unroll
           for (int cb = 0; cb < D / 64; ++cb)
             tma_load_2d(sDO + s * C::kTile + cb * 16384, &tmDO, cb * 64, row_q, DO_FULL(s));
           bulk_load(sb + C::OFF_DEL + s * 512, p.delta + row_q, 512, DO_FULL(s));
-          if (it >= ST) mbar_wait(Q_EMPTY(s), ((it / ST) - 1) & 1, lim, p.err, p.abort_flag);
+          if (it >= ST) wait(Q_EMPTY(s), ((it / ST) - 1) & 1);
           mbar_expect_tx(Q_FULL(s), C::kTile + 512);
 #pragma unroll
           for (int cb = 0; cb < D / 64; ++cb)
@@ -198,29 +225,30 @@ __global__ void __launch_bounds__(512, 1)
       // drain: every issued load has landed before the CTA can exit
       for (int s = 0; s < ST && s < it; ++s) {
         const int last_use = ((it - 1 - s) / ST) * ST + s;
-        mbar_wait(DO_FULL(s), (last_use / ST) & 1, lim, p.err, p.abort_flag);
-        mbar_wait(Q_FULL(s), (last_use / ST) & 1, lim, p.err, p.abort_flag);
+        wait(DO_FULL(s), (last_use / ST) & 1);
+        wait(Q_FULL(s), (last_use / ST) & 1);
       }
-      if (cn > 0) mbar_wait(BAR(B_KV_FULL), (cn - 1) & 1, lim, p.err, p.abort_flag);
+      if (cn > 0) wait(BAR(B_KV_FULL), (cn - 1) & 1);
     } else if (warp == 13 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
-      constexpr uint32_t ID_SS = idesc_bf16_f32(128, 128, 0, 0);
-      constexpr uint32_t ID_KV = idesc_bf16_f32(128, D, 0, 1);
-      constexpr uint32_t ID_Q = idesc_bf16_f32(128, D, 1, 1);
+      constexpr uint32_t ID_SS = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
+      constexpr uint32_t ID_KV = idesc_bf16_f32(128, D, 0, 1);    // dV, dK (A in TMEM)
+      constexpr uint32_t ID_Q = idesc_bf16_f32(128, D, 1, 1);     // dQ
       const uint32_t tS = tmem + C::TM_S, tDP = tmem + C::TM_DP, tDV = tmem + C::TM_DV,
-                     tDK = tmem + C::TM_DK, tDQ = tmem + C::TM_DQ;
+                     tDK = tmem + C::TM_DK;
       int it = 0, cn = 0;
       for (int ci = cbeg; ci < cend; ++ci, ++cn) {
         const int cnt = p.chains[ci].w;
-        mbar_wait(BAR(B_KV_FULL), cn & 1, lim, p.err, p.abort_flag);
-        if (cn > 0) mbar_wait(BAR(B_DKDV_EMPTY), (cn - 1) & 1, lim, p.err, p.abort_flag);
+        wait(BAR(B_KV_FULL), cn & 1);
+        if (cn > 0) wait(BAR(B_DKDV_EMPTY), (cn - 1) & 1);
         tc_fence_after();
         for (int t = 0; t < cnt; ++t, ++it) {
           const int s = it % ST;
           const uint32_t q_s = sQ + s * C::kTile, do_s = sDO + s * C::kTile;
-          // dP^T = V dO^T : M = kv, N = q, K = D (both operands K-major)
           trace(it, 0);
-          mbar_wait(DO_FULL(s), (it / ST) & 1, lim, p.err, p.abort_flag);
+          // dP^T = V dO^T : M = kv, N = q, K = D (both operands K-major)
+          wait(DO_FULL(s), (it / ST) & 1);
+          if (C::kDqInDp && it > 0) wait(BAR(B_DQ_EMPTY0), (it - 1) & 1);
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
@@ -229,9 +257,9 @@ __global__ void __launch_bounds__(512, 1)
                       ID_SS, kk > 0);
           }
           tc_commit(BAR(B_DP_FULL));
-          // S^T = K Q^T
-          mbar_wait(Q_FULL(s), (it / ST) & 1, lim, p.err, p.abort_flag);
-          if (C::kDqAliasesS && it > 0) mbar_wait(BAR(B_DQ_EMPTY), (it - 1) & 1, lim, p.err, p.abort_flag);
+          // S^T = K Q^T, after the previous dV/dK finished reading these columns
+          wait(Q_FULL(s), (it / ST) & 1);
+          if (it > 0) wait(BAR(B_DVDK_DONE), (it - 1) & 1);
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
@@ -240,38 +268,35 @@ __global__ void __launch_bounds__(512, 1)
                       kk > 0);
           }
           tc_commit(BAR(B_S_FULL));
-          mbar_wait(BAR(B_DS_READY), it & 1, lim, p.err, p.abort_flag);
+          wait(BAR(B_DS_READY), it & 1);
           trace(it, 1);
           tc_fence_after();
-          // dV += P^T dO ; dK += dS^T Q : M = kv, N = D, K = q (A K-major, B MN-major)
+          // dV += P^T dO ; dK += dS^T Q : M = kv, N = D, K = q (A in TMEM, B MN-major)
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t offA = (kk >> 2) * 16384 + (kk & 3) * 32;
-            tc_mma_ss(tDV, sdesc_sw128(sPt + offA, 16, 1024),
+          for (int kk = 0; kk < 8; ++kk)
+            tc_mma_ts(tDV, tS + 32 * (kk >> 1) + 8 * (kk & 1),
                       sdesc_sw128(do_s + kk * 2048, 16384, 1024), ID_KV,
                       (t > 0 || kk > 0) ? 1u : 0u);
-          }
           tc_commit(DO_EMPTY(s));
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t offA = (kk >> 2) * 16384 + (kk & 3) * 32;
-            tc_mma_ss(tDK, sdesc_sw128(sDSt + offA, 16, 1024),
+          for (int kk = 0; kk < 8; ++kk)
+            tc_mma_ts(tDK, tS + 32 * (kk >> 1) + 16 + 8 * (kk & 1),
                       sdesc_sw128(q_s + kk * 2048, 16384, 1024), ID_KV,
                       (t > 0 || kk > 0) ? 1u : 0u);
-          }
           tc_commit(Q_EMPTY(s));
+          tc_commit(BAR(B_DVDK_DONE));
           if (t == cnt - 1) tc_commit(BAR(B_DKDV_FULL));
-          if (!C::kDqAliasesS && it > 0) {
-            mbar_wait(BAR(B_DQ_EMPTY), (it - 1) & 1, lim, p.err, p.abort_flag);
+          // dQp = dS K : M = q, N = D, K = kv (both operands MN-major)
+          const int buf = C::kDqInDp ? 0 : (it & 1);
+          if (!C::kDqInDp && it >= 2) {
+            wait(BAR(B_DQ_EMPTY0 + buf), ((it - 2) >> 1) & 1);
             tc_fence_after();
           }
-          // dQp = dS K : M = q, N = D, K = kv (both operands MN-major)
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            tc_mma_ss(tDQ, sdesc_sw128(sDSt + kk * 2048, 16384, 1024),
+          for (int kk = 0; kk < 8; ++kk)
+            tc_mma_ss(tmem + C::TM_DQ + 64 * buf, sdesc_sw128(sDSt + kk * 2048, 16384, 1024),
                       sdesc_sw128(sK + kk * 2048, 16384, 1024), ID_Q, kk > 0);
-          }
-          tc_commit(BAR(B_DQ_FULL));
+          tc_commit(BAR(B_DQ_FULL0 + buf));
           tc_commit(BAR(B_DS_FREE));
           trace(it, 2);
         }
@@ -279,13 +304,15 @@ __global__ void __launch_bounds__(512, 1)
       }
       // drain: all issued MMAs complete before TMEM is released
       tc_commit(BAR(B_FINAL));
-      mbar_wait(BAR(B_FINAL), 0, lim, p.err, p.abort_flag);
+      wait(BAR(B_FINAL), 0);
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------ softmax / dS
     const int quarter = warp & 3, half = warp >> 2;
-    const int r = quarter * 32 + lane;  // KV row of the tile
+    const int r = quarter * 32 + lane;  // KV row of the tile = TMEM lane
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t rowoff =
+        (uint32_t)half * 16384 + (uint32_t)(r >> 3) * 1024 + (uint32_t)(r & 7) * 128;
     const float sl2 = p.scale_log2;
     int it = 0;
     for (int ci = cbeg; ci < cend; ++ci) {
@@ -293,46 +320,50 @@ __global__ void __launch_bounds__(512, 1)
       for (int t = 0; t < ch.w; ++t, ++it) {
         const int q = (int)(p.pairs[ch.z + t] & 0xffffu);
         const int s = it % ST;
-        mbar_wait(DO_FULL(s), (it / ST) & 1, lim, p.err, p.abort_flag);
-        mbar_wait(Q_FULL(s), (it / ST) & 1, lim, p.err, p.abort_flag);
-        mbar_wait(BAR(B_DP_FULL), it & 1, lim, p.err, p.abort_flag);
-        mbar_wait(BAR(B_S_FULL), it & 1, lim, p.err, p.abort_flag);
-        if (it > 0) mbar_wait(BAR(B_DS_FREE), (it - 1) & 1, lim, p.err, p.abort_flag);
+        wait(DO_FULL(s), (it / ST) & 1);
+        wait(Q_FULL(s), (it / ST) & 1);
+        wait(BAR(B_DP_FULL), it & 1);
+        wait(BAR(B_S_FULL), it & 1);
+        if (it > 0) wait(BAR(B_DS_FREE), (it - 1) & 1);
         if (threadIdx.x == 0) trace(it, 3);
         tc_fence_after();
-        const bool diag = p.causal && (q == ch.y);
+        // causal: on the diagonal tile Q column qc sees KV row r only if qc >= r
+        const int lim_c = (p.causal && q == ch.y) ? r : -1;
         const float* lse_t = lse_s + s * 128;
         const float* del_t = del_s + s * 128;
 #pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
-          const int col0 = half * 64 + c * 32;
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = half * 2 + cc;  // 32-column chunk of the tile
           uint32_t sv[32], dv[32];
-          tmem_ld32x2(tmem + lane_off + C::TM_S + col0, tmem + lane_off + C::TM_DP + col0, sv, dv);
+          tmem_ld32x2(tmem + lane_off + C::TM_S + 32 * c, tmem + lane_off + C::TM_DP + 32 * c, sv,
+                      dv);
           uint32_t pk[16], dk[16];
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
-            const int qc = col0 + j;
-            float p0 = exp2f(fmaf(__uint_as_float(sv[j]), sl2, -lse_t[qc]));
-            float p1 = exp2f(fmaf(__uint_as_float(sv[j + 1]), sl2, -lse_t[qc + 1]));
-            if (diag) {
-              if (qc < r) p0 = 0.f;
-              if (qc + 1 < r) p1 = 0.f;
-            }
-            const float d0 = p0 * (__uint_as_float(dv[j]) - del_t[qc]);
-            const float d1 = p1 * (__uint_as_float(dv[j + 1]) - del_t[qc + 1]);
+            const int qc = 32 * c + j;
+            const float2 l2 = *reinterpret_cast<const float2*>(lse_t + qc);
+            const float2 d2 = *reinterpret_cast<const float2*>(del_t + qc);
+            float p0 = ex2_approx(fmaf(__uint_as_float(sv[j]), sl2, -l2.x));
+            float p1 = ex2_approx(fmaf(__uint_as_float(sv[j + 1]), sl2, -l2.y));
+            if (qc < lim_c) p0 = 0.f;
+            if (qc + 1 < lim_c) p1 = 0.f;
+            const float d0 = p0 * (__uint_as_float(dv[j]) - d2.x);
+            const float d1 = p1 * (__uint_as_float(dv[j + 1]) - d2.y);
             pk[j >> 1] = pack_bf16x2(p0, p1);
             dk[j >> 1] = pack_bf16x2(d0, d1);
           }
-          const uint32_t row = (uint32_t)half * 16384 + (uint32_t)(r >> 3) * 1024 +
-                               (uint32_t)(r & 7) * 128;
+          // P^T and dS^T back into the columns of chunk c (this lane's own row)
+          tmem_st16(tmem + lane_off + C::TM_S + 32 * c, pk);
+          tmem_st16(tmem + lane_off + C::TM_S + 32 * c + 16, dk);
+          // dS^T to shared memory (128-byte swizzle, 64-column block `half`)
 #pragma unroll
           for (int m = 0; m < 4; ++m) {
-            const uint32_t chunk = (uint32_t)(((c * 4 + m) ^ (r & 7)) * 16);
-            st_shared_v4(sPt + row + chunk, pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
-            st_shared_v4(sDSt + row + chunk, dk[4 * m], dk[4 * m + 1], dk[4 * m + 2],
+            const uint32_t chunk = (uint32_t)(((cc * 4 + m) ^ (r & 7)) * 16);
+            st_shared_v4(sDSt + rowoff + chunk, dk[4 * m], dk[4 * m + 1], dk[4 * m + 2],
                          dk[4 * m + 3]);
           }
         }
+        tmem_wait_st();
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(BAR(B_DS_READY));
@@ -342,7 +373,7 @@ __global__ void __launch_bounds__(512, 1)
     // ------------------------------------------------------------ dQ reduction + dK/dV epilogue
     setmaxnreg_inc<C::kRegsReduce>();
     const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;  // row of the tile (Q row for dQ, KV row for dK/dV)
+    const int r = quarter * 32 + lane;  // Q row for dQ, KV row for dK/dV
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     constexpr int NV = D / 4;           // float4 per row
     constexpr int G = 16;               // loads in flight per group
@@ -354,19 +385,21 @@ __global__ void __launch_bounds__(512, 1)
         const int q = (int)(w & 0xffffu), pos = (int)(w >> 16);
         const int ncontrib = p.causal ? q + 1 : N;
         const bool last = (pos == ncontrib - 1);
-        mbar_wait(BAR(B_DQ_FULL), it & 1, lim, p.err, p.abort_flag);
+        const int buf = C::kDqInDp ? 0 : (it & 1);
+        const int ph = C::kDqInDp ? (it & 1) : ((it >> 1) & 1);
+        wait(BAR(B_DQ_FULL0 + buf), ph);
         if (threadIdx.x == 256) trace(it, 4);
         tc_fence_after();
         float a[D];
 #pragma unroll
         for (int c2 = 0; c2 < D / 32; ++c2) {
           uint32_t v[32];
-          tmem_ld32(tmem + lane_off + C::TM_DQ + c2 * 32, v);
+          tmem_ld32(tmem + lane_off + C::TM_DQ + 64 * buf + c2 * 32, v);
 #pragma unroll
           for (int j = 0; j < 32; ++j) a[c2 * 32 + j] = __uint_as_float(v[j]);
         }
         tc_fence_before();
-        mbar_arrive(BAR(B_DQ_EMPTY));
+        mbar_arrive(BAR(B_DQ_EMPTY0 + buf));
         if (threadIdx.x == 256) trace(it, 5);
         const long long blk = (long long)ch.x * N + q;
         float4* accp = reinterpret_cast<float4*>(p.acc + blk * 128 * D);
@@ -424,20 +457,22 @@ __global__ void __launch_bounds__(512, 1)
             for (int c4 = 0; c4 < NV; ++c4)
               st_cg_f4(accp + c4 * 128 + r,
                        make_float4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]));
-            __threadfence();
             named_bar_sync(1, 128);
-            if (threadIdx.x == 256) st_release_gpu(p.tickets + blk, (uint32_t)(pos + 1));
+            if (threadIdx.x == 256) {
+              __threadfence();
+              st_release_gpu(p.tickets + blk, (uint32_t)(pos + 1));
+            }
           }
-          if (threadIdx.x == 256) trace(it, 7);
         } else {
 #pragma unroll
           for (int c4 = 0; c4 < NV; ++c4)
             atomicAdd(accp + c4 * 128 + r,
                       make_float4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]));
         }
+        if (threadIdx.x == 256) trace(it, 7);
       }
       // chain epilogue: dV_j and scale * dK_j (rows of KV tile ch.y) to global bf16
-      mbar_wait(BAR(B_DKDV_FULL), cn & 1, lim, p.err, p.abort_flag);
+      wait(BAR(B_DKDV_FULL), cn & 1);
       tc_fence_after();
       const size_t row = (size_t)ch.x * S + (size_t)ch.y * 128 + r;
 #pragma unroll

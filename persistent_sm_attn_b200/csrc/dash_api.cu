@@ -169,13 +169,13 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [rows][D] bf16 viewed with a 64-column x 128-row box and the 128-byte swizzle.
-int make_tmap(CUtensorMap* m, const void* base, long long rows, int D) {
+// [rows][D] bf16 viewed with a 64-column x box_rows box and the 128-byte swizzle.
+int make_tmap(CUtensorMap* m, const void* base, long long rows, int D, int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return DASH_ERR_CUDA;
   cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-  cuuint32_t box[2] = {64, 128};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -236,12 +236,13 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
     std::lock_guard<std::mutex> lk(g_mu);
     if ((rc = get_table(dev, B * H, N, causal, sched, ctas, &tab))) return rc;
     if ((rc = get_workspace(dev, stream, (size_t)rows * D * sizeof(float),
-                            (size_t)B * H * N * sizeof(uint32_t), (size_t)rows, &ws)))
+                            (size_t)dash::dq_units<D>((long long)B * H * N) * sizeof(uint32_t),
+                            (size_t)rows, &ws)))
       return rc;
   }
   CUtensorMap tq, tk, tv, tdo;
-  if ((rc = make_tmap(&tq, q, rows, D)) || (rc = make_tmap(&tk, k, rows, D)) ||
-      (rc = make_tmap(&tv, v, rows, D)) || (rc = make_tmap(&tdo, dout, rows, D)))
+  if ((rc = make_tmap(&tq, q, rows, D, 128)) || (rc = make_tmap(&tk, k, rows, D, 128)) ||
+      (rc = make_tmap(&tv, v, rows, D, 128)) || (rc = make_tmap(&tdo, dout, rows, D, 128)))
     return rc;
   float* lse2 = ws->rowbuf;
   float* delta = ws->rowbuf + ws->rows_cap;
@@ -258,7 +259,9 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   if (kAtomic) {
     DASH_CUDA(cudaMemsetAsync(ws->acc, 0, (size_t)rows * D * sizeof(float), stream));
   } else {
-    DASH_CUDA(cudaMemsetAsync(ws->tickets, 0, (size_t)B * H * N * sizeof(uint32_t), stream));
+    DASH_CUDA(cudaMemsetAsync(ws->tickets, 0,
+                              (size_t)dash::dq_units<D>((long long)B * H * N) * sizeof(uint32_t),
+                              stream));
   }
   BwdParams p;
   p.lse2 = lse2;
@@ -305,10 +308,10 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   }
   if (!prof_record(2, &ev, stream)) return DASH_ERR_CUDA;
   if (kAtomic) {
-    const long long n_blocks = (long long)B * H * N;
-    const long long threads = n_blocks * 128 * (D / 4);
+    const long long n_units = dash::dq_units<D>((long long)B * H * N);
+    const long long threads = n_units * 32 * D;
     dash::dash_dq_convert<D><<<(int)((threads + 255) / 256), 256, 0, stream>>>(
-        ws->acc, static_cast<__nv_bfloat16*>(dq), n_blocks, p.scale);
+        ws->acc, static_cast<__nv_bfloat16*>(dq), n_units, p.scale);
   }
   if (!prof_record(3, &ev, stream)) return DASH_ERR_CUDA;
   if (g_prof_on.load()) {
@@ -409,7 +412,7 @@ int dash_attn_sync_status(void* stream) {
     return DASH_ERR_CUDA;
   if (h) {
     if (cudaMemset(err, 0, sizeof(unsigned)) != cudaSuccess) return DASH_ERR_CUDA;
-    return DASH_ERR_TIMEOUT;
+    return (h & dash::dev::ERR_TIMEOUT) ? DASH_ERR_TIMEOUT : DASH_ERR_UNSUPPORTED;
   }
   return DASH_OK;
 }

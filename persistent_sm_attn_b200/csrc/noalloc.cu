@@ -64,12 +64,12 @@ EncodeTiledFn noalloc_encode_fn() {
   return fn;
 }
 
-int noalloc_tmap(CUtensorMap* m, const void* base, long long rows, int D) {
+int noalloc_tmap(CUtensorMap* m, const void* base, long long rows, int D, int box_rows) {
   EncodeTiledFn fn = noalloc_encode_fn();
   if (!fn) return DASH_ERR_CUDA;
   cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-  cuuint32_t box[2] = {64, 128};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -143,7 +143,7 @@ int noalloc_launch(const void* q, const void* k, const void* v, const void* o, c
   using C = dash::BwdCfg<D>;
   const int N = S / 128;
   const long long rows = (long long)B * H * S;
-  const long long blocks = (long long)B * H * N;
+  const long long blocks = dash::dq_units<D>((long long)B * H * N);  // reduction units
   const int ctas = st->ctas[D == 128][kAtomic ? 1 : 0];
   // lay out the scratch array
   unsigned char* p0 = st->base;
@@ -180,8 +180,8 @@ int noalloc_launch(const void* q, const void* k, const void* v, const void* o, c
   }
   CUtensorMap tq, tk, tv, tdo;
   int rc;
-  if ((rc = noalloc_tmap(&tq, q, rows, D)) || (rc = noalloc_tmap(&tk, k, rows, D)) ||
-      (rc = noalloc_tmap(&tv, v, rows, D)) || (rc = noalloc_tmap(&tdo, dout, rows, D)))
+  if ((rc = noalloc_tmap(&tq, q, rows, D, 128)) || (rc = noalloc_tmap(&tk, k, rows, D, 128)) ||
+      (rc = noalloc_tmap(&tv, v, rows, D, 128)) || (rc = noalloc_tmap(&tdo, dout, rows, D, 128)))
     return rc;
   // the array keeps the previous call's contents: clear what must start at zero
   if (cudaMemsetAsync(err, 0, 2 * sizeof(unsigned), stream) != cudaSuccess) return DASH_ERR_CUDA;
@@ -230,7 +230,7 @@ int noalloc_launch(const void* q, const void* k, const void* v, const void* o, c
       cudaSuccess)
     return DASH_ERR_CUDA;
   if (kAtomic) {
-    const long long threads = blocks * 128 * (D / 4);
+    const long long threads = blocks * 32 * D;
     dash::dash_dq_convert<D><<<(int)((threads + 255) / 256), 256, 0, stream>>>(
         acc, static_cast<__nv_bfloat16*>(dq), blocks, p.scale);
   }
@@ -257,7 +257,7 @@ extern "C" int dash_attn_bwd_noalloc(const void* q, const void* k, const void* v
   if (!dash::schedule_supported(schedule, S / 128, causal)) return DASH_ERR_UNSUPPORTED;
   if (B == 0 || H == 0) return DASH_OK;
   // reject sizes beyond the array before touching the device
-  const long long rows = (long long)B * H * S, blocks = (long long)B * H * (S / 128);
+  const long long rows = (long long)B * H * S, blocks = 2LL * B * H * (S / 128);
   if (fixed_scratch(rows, D, blocks) > kNoallocScratchBytes) return DASH_ERR_OOM;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return DASH_ERR_CUDA;
