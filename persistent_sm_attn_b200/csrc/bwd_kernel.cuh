@@ -39,6 +39,8 @@
 // (rows = K, contiguous along M or N): leading byte offset 16 KiB between
 // 64-element column blocks, stride byte offset 1 KiB between 8-row groups.
 #pragma once
+#include <type_traits>
+
 #include "ptx.cuh"
 
 namespace dash {
@@ -338,20 +340,26 @@ __global__ void __launch_bounds__(512, 1)
           tmem_ld32x2(tmem + lane_off + C::TM_S + 32 * c, tmem + lane_off + C::TM_DP + 32 * c, sv,
                       dv);
           uint32_t pk[16], dk[16];
+          // the causal mask only touches chunks that reach the diagonal
+          auto body = [&](auto masked) {
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const int qc = 32 * c + j;
-            const float2 l2 = *reinterpret_cast<const float2*>(lse_t + qc);
-            const float2 d2 = *reinterpret_cast<const float2*>(del_t + qc);
-            float p0 = ex2_approx(fmaf(__uint_as_float(sv[j]), sl2, -l2.x));
-            float p1 = ex2_approx(fmaf(__uint_as_float(sv[j + 1]), sl2, -l2.y));
-            if (qc < lim_c) p0 = 0.f;
-            if (qc + 1 < lim_c) p1 = 0.f;
-            const float d0 = p0 * (__uint_as_float(dv[j]) - d2.x);
-            const float d1 = p1 * (__uint_as_float(dv[j + 1]) - d2.y);
-            pk[j >> 1] = pack_bf16x2(p0, p1);
-            dk[j >> 1] = pack_bf16x2(d0, d1);
-          }
+            for (int j = 0; j < 32; j += 2) {
+              const int qc = 32 * c + j;
+              const float2 l2 = *reinterpret_cast<const float2*>(lse_t + qc);
+              const float2 d2 = *reinterpret_cast<const float2*>(del_t + qc);
+              float p0 = ex2_approx(fmaf(__uint_as_float(sv[j]), sl2, -l2.x));
+              float p1 = ex2_approx(fmaf(__uint_as_float(sv[j + 1]), sl2, -l2.y));
+              if constexpr (decltype(masked)::value) {
+                if (qc < lim_c) p0 = 0.f;
+                if (qc + 1 < lim_c) p1 = 0.f;
+              }
+              pk[j >> 1] = pack_bf16x2(p0, p1);
+              dk[j >> 1] = pack_bf16x2(p0 * (__uint_as_float(dv[j]) - d2.x),
+                                       p1 * (__uint_as_float(dv[j + 1]) - d2.y));
+            }
+          };
+          if (lim_c > 32 * c) body(std::true_type{});
+          else body(std::false_type{});
           // P^T and dS^T back into the columns of chunk c (this lane's own row)
           tmem_st16(tmem + lane_off + C::TM_S + 32 * c, pk);
           tmem_st16(tmem + lane_off + C::TM_S + 32 * c + 16, dk);

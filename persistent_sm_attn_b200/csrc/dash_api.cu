@@ -308,10 +308,10 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   }
   if (!prof_record(2, &ev, stream)) return DASH_ERR_CUDA;
   if (kAtomic) {
-    const long long n_units = dash::dq_units<D>((long long)B * H * N);
-    const long long threads = n_units * 32 * D;
+    const long long n_blocks = (long long)B * H * N;  // 128-row accumulator blocks
+    const long long threads = n_blocks * 32 * D;
     dash::dash_dq_convert<D><<<(int)((threads + 255) / 256), 256, 0, stream>>>(
-        ws->acc, static_cast<__nv_bfloat16*>(dq), n_units, p.scale);
+        ws->acc, static_cast<__nv_bfloat16*>(dq), n_blocks, p.scale);
   }
   if (!prof_record(3, &ev, stream)) return DASH_ERR_CUDA;
   if (g_prof_on.load()) {

@@ -143,7 +143,7 @@ int noalloc_launch(const void* q, const void* k, const void* v, const void* o, c
   using C = dash::BwdCfg<D>;
   const int N = S / 128;
   const long long rows = (long long)B * H * S;
-  const long long blocks = dash::dq_units<D>((long long)B * H * N);  // reduction units
+  const long long blocks = dash::dq_units<D>((long long)B * H * N);  // tickets (reduction units)
   const int ctas = st->ctas[D == 128][kAtomic ? 1 : 0];
   // lay out the scratch array
   unsigned char* p0 = st->base;
@@ -230,9 +230,10 @@ int noalloc_launch(const void* q, const void* k, const void* v, const void* o, c
       cudaSuccess)
     return DASH_ERR_CUDA;
   if (kAtomic) {
-    const long long threads = blocks * 32 * D;
+    const long long n_blocks = (long long)B * H * N;  // 128-row accumulator blocks
+    const long long threads = n_blocks * 32 * D;
     dash::dash_dq_convert<D><<<(int)((threads + 255) / 256), 256, 0, stream>>>(
-        acc, static_cast<__nv_bfloat16*>(dq), blocks, p.scale);
+        acc, static_cast<__nv_bfloat16*>(dq), n_blocks, p.scale);
   }
   return cudaGetLastError() == cudaSuccess ? DASH_OK : DASH_ERR_CUDA;
 }
