@@ -116,6 +116,7 @@ def run_ours(args):
 
     from persistent_sm_attn_b200 import binding
     from persistent_sm_attn_b200.inputs import draw
+    from persistent_sm_attn_b200.parallel import max_over_ranks
 
     world, rank, local = _dist_init(args)
     torch.cuda.set_device(local)
@@ -163,10 +164,9 @@ def run_ours(args):
         if st != 0:
             raise RuntimeError(f"timed status {binding.dash_status_string(st)}")
         step_ms = sum(a.elapsed_time(b) for a, b in evs)
-        t = torch.tensor([step_ms, main_ms], dtype=torch.float64, device="cuda")
-        if dist is not None:
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t[0]) / steps, float(t[1]) / steps, aux_ms / steps, n_calls
+        step_ms = max_over_ranks(step_ms, "cuda")
+        main_ms = max_over_ranks(main_ms, "cuda")
+        return step_ms / steps, main_ms / steps, aux_ms / steps, n_calls
 
     clocks = ClockSampler(local)
     ms, main_ms, aux_ms, n_calls = time_schedule(sched, args.steps, args.warmup, clocks)
@@ -174,6 +174,10 @@ def run_ours(args):
     compare = [s for s in w.schedules if s != sched] if not args.no_compare else []
     for other in compare:
         results[other] = time_schedule(other, max(5, args.steps // 2), 3)[0]
+
+    sim = None
+    if rank == 0 and not args.no_compare:
+        sim = simulator_vs_measured(w, q, k, v, o, do, lse, sched, results)
 
     # end to end through the public API: pinned host inputs in, results out
     host_in = [t.cpu().pin_memory() for t in (q, k, v, o, do, lse)]
@@ -194,11 +198,7 @@ def run_ours(args):
             h_.copy_(d_, non_blocking=True)
     e1.record(stream)
     barrier()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_ms = float(t[0])
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, "cuda")
     h2d = sum(x.numel() * x.element_size() for x in host_in)
     d2h = sum(x.numel() * x.element_size() for x in host_out)
 
@@ -240,12 +240,49 @@ def run_ours(args):
             "gpu_launches": int(n_calls) * (3 if sched == "atomic" else 2),
             "clocks": clocks.summary(),
         }
+        if sim is not None:
+            line["simulator"] = sim
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def simulator_vs_measured(w, q, k, v, o, do, lse, main_sched, measured_ms):
+    """DAG-simulator prediction of the deterministic schedules' order, with
+    weights taken from two traced launches (outside the timed region): c = the
+    atomic kernel's median pair period on a CTA, r = the deterministic
+    kernel's median time from ticket grant to published reduction."""
+    import numpy as np
+
+    from persistent_sm_attn_b200 import binding
+
+    *_, tr_a = binding.dash_trace_bwd(q, k, v, o, do, lse, w.causal, "atomic")
+    *_, tr_d = binding.dash_trace_bwd(q, k, v, o, do, lse, w.causal, main_sched)
+    periods = []
+    for c in range(tr_a.shape[0]):
+        e0 = tr_a[c, :, 0].astype(np.int64)
+        e0 = e0[e0 > 0]
+        periods += list(np.diff(e0))
+    e6, e7 = tr_d[:, :, 6].astype(np.int64), tr_d[:, :, 7].astype(np.int64)
+    m = (e6 > 0) & (e7 > 0)
+    c_us = float(np.median(periods)) / 1000.0 if periods else 1.0
+    r_us = float(np.median(e7[m] - e6[m])) / 1000.0 if m.any() else 0.0
+    ctas = binding.dash_bwd_num_ctas(0, w.D)
+    pred = {}
+    for s_ in measured_ms:
+        if s_ == "atomic":
+            continue
+        cp, *_ = binding.dash_sched_simulate(w.B * w.H, w.n_tiles, w.causal, s_, ctas, c_us,
+                                             r_us, 2)
+        pred[s_] = round(cp / 1000.0, 4)
+    det = {s_: m_ for s_, m_ in measured_ms.items() if s_ != "atomic"}
+    return {"c_us": round(c_us, 3), "r_us": round(r_us, 3), "dq_buffers": 2, "ctas": ctas,
+            "predicted_ms": pred, "predicted_order": sorted(pred, key=pred.get),
+            "measured_ms": {s_: round(m_, 4) for s_, m_ in det.items()},
+            "measured_order": sorted(det, key=det.get)}
 
 
 class _Null:

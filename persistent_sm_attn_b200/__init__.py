@@ -10,7 +10,7 @@ from __future__ import annotations
 _BINDING_NAMES = {
     "dash_attn_fwd", "dash_attn_bwd", "dash_attn_sync_status", "dash_status_string",
     "dash_sched_simulate", "dash_sched_table", "dash_dag_longest_path", "dash_set_spin_limit_us",
-    "dash_bwd_num_ctas", "dash_release_workspace", "dash_profile_begin", "dash_profile_end", "dash_trace_bwd", "dash_attn_bwd_noalloc", "SCHEDULES", "DashError", "load",
+    "dash_bwd_num_ctas", "dash_release_workspace", "dash_profile_begin", "dash_profile_end", "dash_trace_bwd", "dash_attn_bwd_noalloc", "dash_inject_fault", "SCHEDULES", "DashError", "load",
 }
 
 

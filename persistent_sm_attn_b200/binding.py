@@ -22,7 +22,7 @@ EXPORTS = ("dash_attn_fwd", "dash_attn_bwd", "dash_attn_sync_status", "dash_stat
            "dash_set_spin_limit_us", "dash_bwd_num_ctas", "dash_release_workspace",
            "dash_sched_table", "dash_sched_simulate", "dash_dag_longest_path",
            "dash_profile_begin", "dash_profile_end", "dash_attn_bwd_noalloc",
-           "dash_trace_bwd")
+           "dash_trace_bwd", "dash_inject_fault")
 
 
 class DashError(RuntimeError):
@@ -57,6 +57,7 @@ def load(path: str | None = None):
     lib.dash_status_string.argtypes = [i]
     lib.dash_status_string.restype = ctypes.c_char_p
     lib.dash_set_spin_limit_us.argtypes = [ll]
+    lib.dash_inject_fault.argtypes = [i]
     lib.dash_bwd_num_ctas.argtypes = [i, i, P(i)]
     lib.dash_release_workspace.argtypes = []
     lib.dash_sched_table.argtypes = [i, i, i, i, i, vp, ll]
@@ -153,6 +154,11 @@ def dash_attn_sync_status(stream=None) -> int:
 
 def dash_set_spin_limit_us(us: int) -> None:
     _check(load().dash_set_spin_limit_us(int(us)), "dash_set_spin_limit_us")
+
+
+def dash_inject_fault(mode: int) -> None:
+    """Arm (1) or cancel (0) the host-side fault for the next backward."""
+    _check(load().dash_inject_fault(int(mode)), "dash_inject_fault")
 
 
 def dash_bwd_num_ctas(device: int = 0, D: int = 128) -> int:

@@ -150,6 +150,9 @@ __global__ void __launch_bounds__(512, 1)
     }
   };
   auto wait = [&](uint32_t bar, uint32_t phase) { mbar_wait(bar, phase, lim, p.err, p.abort_flag); };
+  auto drain = [&](uint32_t bar, uint32_t phase) {
+    mbar_wait_drain(bar, phase, lim, p.err, p.abort_flag);
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(BAR(B_KV_FULL), 1);
@@ -227,10 +230,10 @@ __global__ void __launch_bounds__(512, 1)
       // drain: every issued load has landed before the CTA can exit
       for (int s = 0; s < ST && s < it; ++s) {
         const int last_use = ((it - 1 - s) / ST) * ST + s;
-        wait(DO_FULL(s), (last_use / ST) & 1);
-        wait(Q_FULL(s), (last_use / ST) & 1);
+        drain(DO_FULL(s), (last_use / ST) & 1);
+        drain(Q_FULL(s), (last_use / ST) & 1);
       }
-      if (cn > 0) wait(BAR(B_KV_FULL), (cn - 1) & 1);
+      if (cn > 0) drain(BAR(B_KV_FULL), (cn - 1) & 1);
     } else if (warp == 13 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
       constexpr uint32_t ID_SS = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
@@ -306,7 +309,7 @@ __global__ void __launch_bounds__(512, 1)
       }
       // drain: all issued MMAs complete before TMEM is released
       tc_commit(BAR(B_FINAL));
-      wait(BAR(B_FINAL), 0);
+      drain(BAR(B_FINAL), 0);
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------ softmax / dS

@@ -35,6 +35,7 @@ long long default_spin_us() {
   return 10LL * 1000 * 1000;
 }
 std::atomic<long long> g_spin_us{0};
+std::atomic<int> g_fault{0};  // host-side fault injection for the next backward (tests only)
 long long spin_us() {
   long long v = g_spin_us.load();
   return v > 0 ? v : default_spin_us();
@@ -150,6 +151,42 @@ int get_table(int dev, int heads, int N, int causal, int sched, int ctas, DevTab
   return DASH_OK;
 }
 
+// A deliberately broken table for failure-detection tests: every partial of
+// dQ block (head 0, Q tile 0) moves one position later, so its first position
+// is never filled and the waits on it must run out.  All indices stay in range.
+DevTable g_fault_table;
+int get_fault_table(int dev, int heads, int N, int causal, int sched, int ctas, DevTable** out) {
+  dash::Table t;
+  std::string err;
+  if (!dash::build_table(heads, N, causal, sched, ctas, &t, &err)) return DASH_ERR_UNSUPPORTED;
+  for (const dash::Chain& ch : t.chains)
+    if (ch.bh == 0)
+      for (int i = 0; i < ch.pair_cnt; ++i) {
+        uint32_t& w = t.pairs[ch.pair_off + i];
+        if (dash::pair_q(w) == 0) w = dash::pack_pair(0, dash::pair_pos(w) + 1);
+      }
+  cudaFree(g_fault_table.cta_off);
+  cudaFree(g_fault_table.chains);
+  cudaFree(g_fault_table.pairs);
+  g_fault_table = DevTable{};
+  DevTable& d = g_fault_table;
+  if (cudaMalloc(&d.cta_off, t.cta_off.size() * sizeof(int)) != cudaSuccess ||
+      cudaMalloc(&d.chains, t.chains.size() * sizeof(int4)) != cudaSuccess ||
+      cudaMalloc(&d.pairs, t.pairs.size() * sizeof(uint32_t)) != cudaSuccess) {
+    cudaGetLastError();
+    return DASH_ERR_OOM;
+  }
+  DASH_CUDA(cudaMemcpy(d.cta_off, t.cta_off.data(), t.cta_off.size() * sizeof(int),
+                       cudaMemcpyHostToDevice));
+  DASH_CUDA(cudaMemcpy(d.chains, t.chains.data(), t.chains.size() * sizeof(int4),
+                       cudaMemcpyHostToDevice));
+  DASH_CUDA(cudaMemcpy(d.pairs, t.pairs.data(), t.pairs.size() * sizeof(uint32_t),
+                       cudaMemcpyHostToDevice));
+  (void)dev;
+  *out = &d;
+  return DASH_OK;
+}
+
 // ------------------------------------------------------------------ TMA descriptors
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -234,7 +271,12 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   Workspace* ws = nullptr;
   {
     std::lock_guard<std::mutex> lk(g_mu);
-    if ((rc = get_table(dev, B * H, N, causal, sched, ctas, &tab))) return rc;
+    const int fault = g_fault.exchange(0);
+    if (fault == 1 && !kAtomic) {
+      if ((rc = get_fault_table(dev, B * H, N, causal, sched, ctas, &tab))) return rc;
+    } else if ((rc = get_table(dev, B * H, N, causal, sched, ctas, &tab))) {
+      return rc;
+    }
     if ((rc = get_workspace(dev, stream, (size_t)rows * D * sizeof(float),
                             (size_t)dash::dq_units<D>((long long)B * H * N) * sizeof(uint32_t),
                             (size_t)rows, &ws)))
@@ -337,6 +379,12 @@ const char* dash_status_string(int s) {
     case DASH_ERR_SCHEDULE: return "DASH_ERR_SCHEDULE";
     default: return "DASH_ERR_UNKNOWN";
   }
+}
+
+int dash_inject_fault(int mode) {
+  if (mode != 0 && mode != 1) return DASH_ERR_INVALID_ARG;
+  g_fault.store(mode);
+  return DASH_OK;
 }
 
 int dash_set_spin_limit_us(long long us) {

@@ -1,0 +1,59 @@
+"""Head sharding and max-over-ranks timing, with world_size 2 gloo ranks on CPU."""
+import os
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+from persistent_sm_attn_b200.parallel import head_range, max_over_ranks
+
+
+@pytest.mark.parametrize("n_heads", [0, 1, 5, 32, 128, 97])
+@pytest.mark.parametrize("world", [1, 2, 3, 8])
+def test_head_ranges_partition(n_heads, world):
+    seen = []
+    sizes = []
+    for r in range(world):
+        a, b = head_range(n_heads, r, world)
+        seen.extend(range(a, b))
+        sizes.append(b - a)
+    assert seen == list(range(n_heads))
+    assert max(sizes) - min(sizes) <= 1
+
+
+def test_head_range_rejects_bad_ranks():
+    with pytest.raises(ValueError):
+        head_range(4, 2, 2)
+
+
+def _worker(rank, world, port, out):
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        a, b = head_range(64, rank, world)
+        # each rank "times" its own shard; the job time is the slowest rank's
+        t = max_over_ranks(1.0 + rank * 0.5)
+        gathered = [None] * world
+        dist.all_gather_object(gathered, (a, b))
+        out[rank] = (t, gathered)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks():
+    world = 2
+    port = 29500 + (os.getpid() % 1000)
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    for r in range(world):
+        t, ranges = res[r]
+        assert t == 1.5
+        assert ranges == [(0, 32), (32, 64)]
+
+
+def test_max_over_ranks_without_group():
+    assert max_over_ranks(3.25) == 3.25
