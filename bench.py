@@ -44,6 +44,29 @@ def _peaks():
         return 1590.0, 6650.0, "fallback"
 
 
+def _recorded_traffic(workload: str, schedule: str):
+    """DRAM bytes per launch recorded from an ncu capture, or None when no
+    capture exists for this workload/schedule or the kernel sources changed
+    since it was taken."""
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in ("bwd_kernel.cuh", "ptx.cuh"):
+        with open(os.path.join(ROOT, "persistent_sm_attn_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    digest = h.hexdigest()[:16]
+    try:
+        with open(os.path.join(ROOT, "profiles", "roofline_traffic.txt")) as fh:
+            for line in fh:
+                parts = line.split()
+                if len(parts) == 4 and not line.startswith("#"):
+                    if parts[0] == workload and parts[1] == schedule and parts[3] == digest:
+                        return int(parts[2])
+    except OSError:
+        pass
+    return None
+
+
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons during a region."""
 
@@ -232,7 +255,8 @@ def run_ours(args):
             "det_nondet_ratio": (round(best_det / det["atomic"], 4)
                                  if atomic_ms and best_det else None),
             "roofline": {"bound": "tensor", "achieved": round(kern, 2), "peak": peak,
-                         "unit": "TFLOP/s", "frac": round(kern / peak, 4), "traffic": None,
+                         "unit": "TFLOP/s", "frac": round(kern / peak, 4),
+                         "traffic": _recorded_traffic(w.name, sched),
                          "kernel": "dash_bwd_kernel", "peak_kind": f"{peak_kind} bf16 burst",
                          "kernel_ms": round(main_ms, 4), "aux_ms": round(aux_ms, 4)},
             "e2e": {"value": round(tflops(e2e_ms), 2), "unit": "TFLOP/s",

@@ -42,10 +42,17 @@ def _worker(rank, world, port, out):
         dist.destroy_process_group()
 
 
+def _free_port():
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
 def test_two_gloo_ranks():
     world = 2
-    port = 29500 + (os.getpid() % 1000)
-    with mp.Manager() as m:
+    port = _free_port()
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)
