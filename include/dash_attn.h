@@ -110,7 +110,7 @@ int dash_set_spin_limit_us(long long us);
 /*
  * Failure-detection testing.  mode 1: the next deterministic dash_attn_bwd
  * (any stream) runs with a schedule table in which dQ block (head 0, Q tile 0)
- * never receives its first partial, so its ticket waits run out; the kernel
+ * never receives its first two partials, so its ticket waits run out; the kernel
  * still ends, with DASH_ERR_TIMEOUT reported by dash_attn_sync_status and
  * invalid outputs.  The fault is made on the host; no memory outside the
  * call's buffers is touched.  mode 0 cancels.  Other modes: INVALID_ARG.

@@ -4,21 +4,26 @@
 // DASH ..." §2.1: all pairs of one KV tile run back to back on one SM, with the
 // dK/dV accumulators on chip).  Per (KV tile j, Q tile i) pair of 128 x 128:
 //
-//   dP^T = V_j dO_i^T                 tcgen05.mma (smem x smem) -> TMEM [128, 256)
 //   S^T  = K_j Q_i^T                  tcgen05.mma (smem x smem) -> TMEM [0, 128)
-//   P^T  = exp(scale S^T - LSE_i), dS^T = P^T (dP^T - Delta_i)     (softmax warps)
-//          P^T and dS^T go back to TMEM as bf16 in the columns S^T occupied;
-//          dS^T also goes to shared memory for the dQ product
-//   dV_j += P^T dO_i, dK_j += dS^T Q_i       tcgen05.mma with A in TMEM, accumulators in TMEM
+//   dP^T = V_j dO_i^T                 tcgen05.mma (smem x smem) -> TMEM [128, 256)
+//   P^T  = exp(scale S^T - LSE_i)     softmax warps, packed bf16 back into S^T's columns
+//   dV_j += P^T dO_i                  tcgen05.mma with A in TMEM, as soon as P^T is packed
+//   dS^T = P^T (dP^T - Delta_i)       softmax warps, into S^T's columns and shared memory
+//   dK_j += dS^T Q_i                  tcgen05.mma with A in TMEM
 //   dQp  = dS K_j                     tcgen05.mma (smem x smem) -> TMEM
-//   ordered reduction of dQp into the fp32 accumulator of block (b,h,i): wait
-//   until the block's ticket equals this pair's position, add with plain loads
-//   and stores, publish, bump the ticket (§1: a fixed accumulation order makes
-//   dQ bitwise reproducible; §2.2 chooses the order).  The last contributor
-//   rounds the sum once to bf16 and writes dQ.
+//   ordered reduction of dQp into an fp32 accumulator of block (b,h,i): wait
+//   until the accumulator's ticket says it is this pair's turn, add with plain
+//   loads and stores, publish, bump the ticket (§1: a fixed accumulation order
+//   makes dQ bitwise reproducible; §2.2 chooses the order).  Each block has two
+//   accumulators, one for the even and one for the odd positions of its order,
+//   so a contributor waits on the one two positions ahead of it; the last
+//   contributor adds the two sums, rounds once to bf16 and writes dQ.
 //
-// Taking P^T and dS^T from TMEM keeps two of the five products off the
-// shared-memory read path, which bounds the 1-CTA tensor cores here.
+// The MMA issuer queues S^T and dP^T of the next tile right behind dK and dQp,
+// so the exponentials of tile i+1 run while the tensor pipe finishes tile i,
+// and dV of tile i+1 runs while its dS is formed.  Taking P^T and dS^T from
+// TMEM keeps two of the five products off the shared-memory read path, which
+// bounds the 1-CTA tensor cores here.
 //
 // Warp roles (512 threads, four warpgroups):
 //   WG0, WG1  softmax / dS; WG0 owns Q columns 0-63, WG1 columns 64-127
@@ -38,6 +43,9 @@
 // K-major operand (rows = M or N, contiguous along K) or as an MN-major one
 // (rows = K, contiguous along M or N): leading byte offset 16 KiB between
 // 64-element column blocks, stride byte offset 1 KiB between 8-row groups.
+// A descriptor's start address field holds (address >> 4) in its low 14 bits;
+// every tile here ends below 256 KiB, so adding (byte offset >> 4) to a base
+// descriptor moves its start without carrying into the other fields.
 #pragma once
 #include <type_traits>
 
@@ -51,8 +59,9 @@ struct BwdParams {
   const int* cta_off;     // [grid + 1]
   const int4* chains;     // {bh, kv, pair_off, pair_cnt}
   const uint32_t* pairs;  // q | position << 16
-  float* acc;             // fp32 dQ accumulator, per block [D/4][128][4]
-  uint32_t* tickets;      // one per 128-row dQ block
+  float* acc;             // fp32 dQ accumulators, [D/4][128][4] each: two per 128-row block
+                          // (the atomic variant uses the first per block)
+  uint32_t* tickets;      // one per accumulator
   unsigned* err;          // device error word (accumulates until read by the host)
   unsigned* abort_flag;   // per-launch: set by the first timeout, cleared before each launch
   __nv_bfloat16* dq;
@@ -75,6 +84,8 @@ struct BwdCfg {
   static constexpr int kRegsCtrl = 80;                   // WG3
   static_assert(2 * kLaunchRegs + kRegsReduce + kRegsCtrl == 4 * kLaunchRegs,
                 "register split must equal the launch allocation");
+  static constexpr int kKVRows = 128;                    // TMA box rows of K and V
+  static constexpr int kQRows = 128;                     // TMA box rows of Q and dO
   static constexpr int kTile = 128 * D * 2;              // one [128][D] bf16 tile
   static constexpr int kStages = (D == 64) ? 3 : 2;      // Q/dO pipeline depth
   static constexpr int OFF_K = 0;
@@ -82,8 +93,8 @@ struct BwdCfg {
   static constexpr int OFF_Q = OFF_V + kTile;
   static constexpr int OFF_DO = OFF_Q + kStages * kTile;
   static constexpr int OFF_DST = OFF_DO + kStages * kTile;  // dS^T [128 kv][128 q]
-  static constexpr int OFF_LSE = OFF_DST + 32768;           // kStages x 128 fp32
-  static constexpr int OFF_DEL = OFF_LSE + kStages * 512;
+  static constexpr int OFF_LSE = OFF_DST + 32768;           // kStages x 128 fp32 (with Q)
+  static constexpr int OFF_DEL = OFF_LSE + kStages * 512;  // kStages x 128 fp32 (with Q)
   static constexpr int OFF_BAR = OFF_DEL + kStages * 512;
   static constexpr int kBars = 16 + 4 * kStages;
   static constexpr int OFF_TMEM_SLOT = OFF_BAR + kBars * 8;
@@ -95,19 +106,21 @@ struct BwdCfg {
   static constexpr bool kDqInDp = (D == 128);  // dQp reuses dP^T's columns
 };
 
-// Number of dQ reduction units (tickets): one per 128-row block.
+// Number of dQ accumulation chains (tickets, and fp32 accumulators of 128 x D):
+// two per 128-row block.
 template <int D>
 constexpr long long dq_units(long long bh_times_n) {
-  return bh_times_n;
+  return 2 * bh_times_n;
 }
 
 // barrier indices
 enum {
   B_KV_FULL = 0, B_KV_EMPTY, B_S_FULL, B_DP_FULL, B_DS_READY, B_DS_FREE, B_DQ_FULL0, B_DQ_FULL1,
-  B_DQ_EMPTY0, B_DQ_EMPTY1, B_DVDK_DONE, B_DKDV_FULL, B_DKDV_EMPTY, B_FINAL, B_STAGE0 = 16
+  B_DQ_EMPTY0, B_DQ_EMPTY1, B_DVDK_DONE, B_DKDV_FULL, B_DKDV_EMPTY, B_FINAL, B_P_READY,
+  B_STAGE0 = 16
 };
 
-// kTrace: record %globaltimer per pair of this CTA: 0 MMA tile start, 1 softmax
+// kTrace: record %globaltimer per pair of this CTA: 0 S^T issued, 1 softmax
 // done (seen by the MMA issuer), 2 tile MMAs issued, 3 softmax start, 4 dQ
 // partial ready (seen by the reducers), 5 partial drained, 6 ticket granted,
 // 7 reduction published.
@@ -169,6 +182,7 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(BAR(B_DKDV_FULL), 1);
     mbar_init(BAR(B_DKDV_EMPTY), 128);
     mbar_init(BAR(B_FINAL), 1);
+    mbar_init(BAR(B_P_READY), 256);
     for (int s = 0; s < ST; ++s) {
       mbar_init(Q_FULL(s), 1);
       mbar_init(Q_EMPTY(s), 1);
@@ -205,105 +219,126 @@ __global__ void __launch_bounds__(512, 1)
         const int row_kv = ch.x * S + ch.y * 128;
 #pragma unroll
         for (int cb = 0; cb < D / 64; ++cb) {
-          tma_load_2d(sV + cb * 16384, &tmV, cb * 64, row_kv, BAR(B_KV_FULL));
           tma_load_2d(sK + cb * 16384, &tmK, cb * 64, row_kv, BAR(B_KV_FULL));
+          tma_load_2d(sV + cb * 16384, &tmV, cb * 64, row_kv, BAR(B_KV_FULL));
         }
         for (int t = 0; t < ch.w; ++t, ++it) {
           const int q = (int)(p.pairs[ch.z + t] & 0xffffu);
           const int s = it % ST;
           const int row_q = ch.x * S + q * 128;
-          // dO first: the MMA issuer consumes it first (dP^T) and frees it first (after dV)
-          if (it >= ST) wait(DO_EMPTY(s), ((it / ST) - 1) & 1);
-          mbar_expect_tx(DO_FULL(s), C::kTile + 512);
-#pragma unroll
-          for (int cb = 0; cb < D / 64; ++cb)
-            tma_load_2d(sDO + s * C::kTile + cb * 16384, &tmDO, cb * 64, row_q, DO_FULL(s));
-          bulk_load(sb + C::OFF_DEL + s * 512, p.delta + row_q, 512, DO_FULL(s));
+          // Q with LSE and Delta (the softmax reads both until dS is done, which is
+          // before dK releases this stage); dO is released earlier, after dV
           if (it >= ST) wait(Q_EMPTY(s), ((it / ST) - 1) & 1);
-          mbar_expect_tx(Q_FULL(s), C::kTile + 512);
+          mbar_expect_tx(Q_FULL(s), C::kTile + 1024);
 #pragma unroll
           for (int cb = 0; cb < D / 64; ++cb)
             tma_load_2d(sQ + s * C::kTile + cb * 16384, &tmQ, cb * 64, row_q, Q_FULL(s));
           bulk_load(sb + C::OFF_LSE + s * 512, p.lse2 + row_q, 512, Q_FULL(s));
+          bulk_load(sb + C::OFF_DEL + s * 512, p.delta + row_q, 512, Q_FULL(s));
+          if (it >= ST) wait(DO_EMPTY(s), ((it / ST) - 1) & 1);
+          mbar_expect_tx(DO_FULL(s), C::kTile);
+#pragma unroll
+          for (int cb = 0; cb < D / 64; ++cb)
+            tma_load_2d(sDO + s * C::kTile + cb * 16384, &tmDO, cb * 64, row_q, DO_FULL(s));
         }
       }
       // drain: every issued load has landed before the CTA can exit
       for (int s = 0; s < ST && s < it; ++s) {
         const int last_use = ((it - 1 - s) / ST) * ST + s;
-        drain(DO_FULL(s), (last_use / ST) & 1);
         drain(Q_FULL(s), (last_use / ST) & 1);
+        drain(DO_FULL(s), (last_use / ST) & 1);
       }
       if (cn > 0) drain(BAR(B_KV_FULL), (cn - 1) & 1);
     } else if (warp == 13 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
+      // One thread issues every MMA; its instruction stream between MMAs is the
+      // issue cost, so the loops are unrolled with constant operand offsets added
+      // to descriptor words, and each product is written out once.
       constexpr uint32_t ID_SS = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
       constexpr uint32_t ID_KV = idesc_bf16_f32(128, D, 0, 1);    // dV, dK (A in TMEM)
       constexpr uint32_t ID_Q = idesc_bf16_f32(128, D, 1, 1);     // dQ
       const uint32_t tS = tmem + C::TM_S, tDP = tmem + C::TM_DP, tDV = tmem + C::TM_DV,
                      tDK = tmem + C::TM_DK;
+      const uint32_t hi = sdesc_hi(1024);  // every operand here: 1 KiB between 8-row groups
+      const uint32_t kK = sdesc_lo(sK, 16), kV = sdesc_lo(sV, 16);            // K-major
+      const uint32_t mK = sdesc_lo(sK, 16384), mDS = sdesc_lo(sDSt, 16384);  // MN-major
       int it = 0, cn = 0;
       for (int ci = cbeg; ci < cend; ++ci, ++cn) {
         const int cnt = p.chains[ci].w;
         wait(BAR(B_KV_FULL), cn & 1);
-        if (cn > 0) wait(BAR(B_DKDV_EMPTY), (cn - 1) & 1);
         tc_fence_after();
-        for (int t = 0; t < cnt; ++t, ++it) {
-          const int s = it % ST;
-          const uint32_t q_s = sQ + s * C::kTile, do_s = sDO + s * C::kTile;
-          trace(it, 0);
-          // dP^T = V dO^T : M = kv, N = q, K = D (both operands K-major)
-          wait(DO_FULL(s), (it / ST) & 1);
-          if (C::kDqInDp && it > 0) wait(BAR(B_DQ_EMPTY0), (it - 1) & 1);
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            tc_mma_ss(tDP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(do_s + off, 16, 1024),
-                      ID_SS, kk > 0);
-          }
-          tc_commit(BAR(B_DP_FULL));
-          // S^T = K Q^T, after the previous dV/dK finished reading these columns
-          wait(Q_FULL(s), (it / ST) & 1);
-          if (it > 0) wait(BAR(B_DVDK_DONE), (it - 1) & 1);
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            tc_mma_ss(tS, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(q_s + off, 16, 1024), ID_SS,
-                      kk > 0);
-          }
-          tc_commit(BAR(B_S_FULL));
-          wait(BAR(B_DS_READY), it & 1);
-          trace(it, 1);
-          tc_fence_after();
-          // dV += P^T dO ; dK += dS^T Q : M = kv, N = D, K = q (A in TMEM, B MN-major)
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            tc_mma_ts(tDV, tS + 32 * (kk >> 1) + 8 * (kk & 1),
-                      sdesc_sw128(do_s + kk * 2048, 16384, 1024), ID_KV,
-                      (t > 0 || kk > 0) ? 1u : 0u);
-          tc_commit(DO_EMPTY(s));
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            tc_mma_ts(tDK, tS + 32 * (kk >> 1) + 16 + 8 * (kk & 1),
-                      sdesc_sw128(q_s + kk * 2048, 16384, 1024), ID_KV,
-                      (t > 0 || kk > 0) ? 1u : 0u);
-          tc_commit(Q_EMPTY(s));
-          tc_commit(BAR(B_DVDK_DONE));
-          if (t == cnt - 1) tc_commit(BAR(B_DKDV_FULL));
-          // dQp = dS K : M = q, N = D, K = kv (both operands MN-major)
-          const int buf = C::kDqInDp ? 0 : (it & 1);
-          if (!C::kDqInDp && it >= 2) {
-            wait(BAR(B_DQ_EMPTY0 + buf), ((it - 2) >> 1) & 1);
+        // t = -1 only issues the chain's first S^T/dP^T; each later step finishes
+        // tile `it` and then issues S^T/dP^T of the next tile behind it
+        for (int t = -1; t < cnt; ++t) {
+          if (t >= 0) {
+            const int s = it % ST;
+            const uint32_t mQ = sdesc_lo(sQ + s * C::kTile, 16384);
+            const uint32_t mDO = sdesc_lo(sDO + s * C::kTile, 16384);
+            // dV += P^T dO : M = kv, N = D, K = q (A in TMEM, B MN-major), once P is packed
+            wait(BAR(B_P_READY), it & 1);
+            // the previous chain's dV/dK must have been read out before they restart
+            if (t == 0 && cn > 0) wait(BAR(B_DKDV_EMPTY), (cn - 1) & 1);
             tc_fence_after();
-          }
+            const uint32_t acc0 = t > 0 ? 1u : 0u;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            tc_mma_ss(tmem + C::TM_DQ + 64 * buf, sdesc_sw128(sDSt + kk * 2048, 16384, 1024),
-                      sdesc_sw128(sK + kk * 2048, 16384, 1024), ID_Q, kk > 0);
-          tc_commit(BAR(B_DQ_FULL0 + buf));
-          tc_commit(BAR(B_DS_FREE));
-          trace(it, 2);
+            for (int kk = 0; kk < 8; ++kk)
+              tc_mma_ts_w(tDV, tS + 32 * (kk >> 1) + 8 * (kk & 1), mDO + kk * 128, hi, ID_KV,
+                          kk > 0 ? 1u : acc0);
+            tc_commit(DO_EMPTY(s));
+            // dK += dS^T Q
+            wait(BAR(B_DS_READY), it & 1);
+            trace(it, 1);
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              tc_mma_ts_w(tDK, tS + 32 * (kk >> 1) + 16 + 8 * (kk & 1), mQ + kk * 128, hi, ID_KV,
+                          kk > 0 ? 1u : acc0);
+            tc_commit(Q_EMPTY(s));
+            tc_commit(BAR(B_DVDK_DONE));
+            if (t == cnt - 1) tc_commit(BAR(B_DKDV_FULL));
+            // dQp = dS K : M = q, N = D, K = kv (both operands MN-major)
+            const int buf = C::kDqInDp ? 0 : (it & 1);
+            if (!C::kDqInDp && it >= 2) {
+              wait(BAR(B_DQ_EMPTY0 + buf), ((it - 2) >> 1) & 1);
+              tc_fence_after();
+            }
+            const uint32_t tDQ = tmem + C::TM_DQ + 64 * buf;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              tc_mma_ss_w(tDQ, mDS + kk * 128, mK + kk * 128, hi, ID_Q, kk > 0 ? 1u : 0u);
+            tc_commit(BAR(B_DQ_FULL0 + buf));
+            tc_commit(BAR(B_DS_FREE));
+            trace(it, 2);
+            ++it;
+          }
+          if (t + 1 < cnt) {
+            // S^T = K Q^T of tile `it`: M = kv, N = q, K = D (both K-major), once dV/dK
+            // of the previous tile have read packed P^T/dS^T out of these columns
+            const int s = it % ST;
+            const uint32_t kQ = sdesc_lo(sQ + s * C::kTile, 16);
+            const uint32_t kDO = sdesc_lo(sDO + s * C::kTile, 16);
+            wait(Q_FULL(s), (it / ST) & 1);
+            if (it > 0) wait(BAR(B_DVDK_DONE), (it - 1) & 1);
+            tc_fence_after();
+            trace(it, 0);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (uint32_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+              tc_mma_ss_w(tS, kK + off, kQ + off, hi, ID_SS, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(BAR(B_S_FULL));
+            // dP^T = V dO^T; at D = 128 these columns hold dQp of the previous tile
+            // until the reducers have drained it
+            wait(DO_FULL(s), (it / ST) & 1);
+            if (C::kDqInDp && it > 0) wait(BAR(B_DQ_EMPTY0), (it - 1) & 1);
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (uint32_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+              tc_mma_ss_w(tDP, kV + off, kDO + off, hi, ID_SS, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(BAR(B_DP_FULL));
+          }
         }
         tc_commit(BAR(B_KV_EMPTY));
       }
@@ -313,11 +348,14 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------ softmax / dS
+    // Two phases per tile: P first (all the exponentials), published so that the
+    // MMA issuer can start dV while dS is computed; then dS once dP^T is in TMEM.
     const int quarter = warp & 3, half = warp >> 2;
     const int r = quarter * 32 + lane;  // KV row of the tile = TMEM lane
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t rowoff =
         (uint32_t)half * 16384 + (uint32_t)(r >> 3) * 1024 + (uint32_t)(r & 7) * 128;
+    const uint32_t tS = tmem + lane_off + C::TM_S, tDP = tmem + lane_off + C::TM_DP;
     const float sl2 = p.scale_log2;
     int it = 0;
     for (int ci = cbeg; ci < cend; ++ci) {
@@ -325,11 +363,8 @@ __global__ void __launch_bounds__(512, 1)
       for (int t = 0; t < ch.w; ++t, ++it) {
         const int q = (int)(p.pairs[ch.z + t] & 0xffffu);
         const int s = it % ST;
-        wait(DO_FULL(s), (it / ST) & 1);
-        wait(Q_FULL(s), (it / ST) & 1);
-        wait(BAR(B_DP_FULL), it & 1);
         wait(BAR(B_S_FULL), it & 1);
-        if (it > 0) wait(BAR(B_DS_FREE), (it - 1) & 1);
+        wait(Q_FULL(s), (it / ST) & 1);
         if (threadIdx.x == 0) trace(it, 3);
         tc_fence_after();
         // causal: on the diagonal tile Q column qc sees KV row r only if qc >= r
@@ -339,17 +374,15 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll 1
         for (int cc = 0; cc < 2; ++cc) {
           const int c = half * 2 + cc;  // 32-column chunk of the tile
-          uint32_t sv[32], dv[32];
-          tmem_ld32x2(tmem + lane_off + C::TM_S + 32 * c, tmem + lane_off + C::TM_DP + 32 * c, sv,
-                      dv);
-          uint32_t pk[16], dk[16];
+          uint32_t sv[32];
+          tmem_ld32(tS + 32 * c, sv);
+          uint32_t pk[16];
           // the causal mask only touches chunks that reach the diagonal
           auto body = [&](auto masked) {
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
               const int qc = 32 * c + j;
               const float2 l2 = *reinterpret_cast<const float2*>(lse_t + qc);
-              const float2 d2 = *reinterpret_cast<const float2*>(del_t + qc);
               float p0 = ex2_approx(fmaf(__uint_as_float(sv[j]), sl2, -l2.x));
               float p1 = ex2_approx(fmaf(__uint_as_float(sv[j + 1]), sl2, -l2.y));
               if constexpr (decltype(masked)::value) {
@@ -357,16 +390,39 @@ __global__ void __launch_bounds__(512, 1)
                 if (qc + 1 < lim_c) p1 = 0.f;
               }
               pk[j >> 1] = pack_bf16x2(p0, p1);
-              dk[j >> 1] = pack_bf16x2(p0 * (__uint_as_float(dv[j]) - d2.x),
-                                       p1 * (__uint_as_float(dv[j + 1]) - d2.y));
             }
           };
           if (lim_c > 32 * c) body(std::true_type{});
           else body(std::false_type{});
-          // P^T and dS^T back into the columns of chunk c (this lane's own row)
-          tmem_st16(tmem + lane_off + C::TM_S + 32 * c, pk);
-          tmem_st16(tmem + lane_off + C::TM_S + 32 * c + 16, dk);
-          // dS^T to shared memory (128-byte swizzle, 64-column block `half`)
+          // P^T into the first 16 columns of chunk c (this lane's own row)
+          tmem_st16(tS + 32 * c, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(BAR(B_P_READY));
+        wait(BAR(B_DP_FULL), it & 1);
+        if (it > 0) wait(BAR(B_DS_FREE), (it - 1) & 1);
+        tc_fence_after();
+        // dS from the bf16 P just packed: the registers are not there to keep P in
+        // fp32 across the wait, and the extra rounding stays far inside the error bound
+#pragma unroll 1
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = half * 2 + cc;
+          uint32_t pk[16], dv[32];
+          tmem_ld16(tS + 32 * c, pk);
+          tmem_ld32(tDP + 32 * c, dv);
+          uint32_t dk[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const float2 d2 = *reinterpret_cast<const float2*>(del_t + 32 * c + j);
+            const float p0 = __uint_as_float(pk[j >> 1] << 16);
+            const float p1 = __uint_as_float(pk[j >> 1] & 0xffff0000u);
+            dk[j >> 1] = pack_bf16x2(p0 * (__uint_as_float(dv[j]) - d2.x),
+                                     p1 * (__uint_as_float(dv[j + 1]) - d2.y));
+          }
+          // dS^T into the last 16 columns of chunk c, and to shared memory
+          // (128-byte swizzle, 64-column block `half`)
+          tmem_st16(tS + 32 * c + 16, dk);
 #pragma unroll
           for (int m = 0; m < 4; ++m) {
             const uint32_t chunk = (uint32_t)(((cc * 4 + m) ^ (r & 7)) * 16);
@@ -413,17 +469,23 @@ __global__ void __launch_bounds__(512, 1)
         mbar_arrive(BAR(B_DQ_EMPTY0 + buf));
         if (threadIdx.x == 256) trace(it, 5);
         const long long blk = (long long)ch.x * N + q;
-        float4* accp = reinterpret_cast<float4*>(p.acc + blk * 128 * D);
         if constexpr (!kAtomic) {
-          if (pos > 0) {
-            uint32_t* tk = p.tickets + blk;
+          // Two accumulation chains per dQ block: the contributions at even and at
+          // odd positions each add, in position order, into an fp32 accumulator of
+          // their own, so consecutive contributors to a block do not wait on each
+          // other.  The block's last contributor adds the two chain sums.
+          const int chain = pos & 1, idx = pos >> 1;
+          const long long unit = blk * 2 + chain;
+          float4* accp = reinterpret_cast<float4*>(p.acc) + unit * (32 * D);
+          // wait (bounded) until a chain's ticket reaches `want`
+          auto ticket_wait = [&](uint32_t* tk, uint32_t want) {
             if (lane == 0) {
-              if (ld_acquire_gpu(tk) != (uint32_t)pos) {
+              if (ld_acquire_gpu(tk) != want) {
                 const uint64_t t0 = globaltimer();
                 bool ok = false;
                 while (!ok) {
 #pragma unroll 1
-                  for (int i = 0; i < 32 && !ok; ++i) ok = (ld_acquire_gpu(tk) == (uint32_t)pos);
+                  for (int i = 0; i < 32 && !ok; ++i) ok = (ld_acquire_gpu(tk) == want);
                   if (!ok && (aborted(p.abort_flag) || globaltimer() - t0 > lim)) {
                     if (!aborted(p.abort_flag)) raise_timeout(p.err, p.abort_flag, ERR_WHERE_TICKET);
                     break;
@@ -433,13 +495,14 @@ __global__ void __launch_bounds__(512, 1)
             }
             __syncwarp();
             (void)ld_acquire_gpu(tk);
-            if (threadIdx.x == 256) trace(it, 6);
-            // acc += partial, G loads in flight before their adds
+          };
+          // a = acc + a over this thread's slots, G loads in flight before their adds
+          auto add_from = [&](const float4* src) {
 #pragma unroll
             for (int g0 = 0; g0 < NV; g0 += G) {
               float4 old[G];
 #pragma unroll
-              for (int j = 0; j < G; ++j) old[j] = ld_cg_f4(accp + (g0 + j) * 128 + r);
+              for (int j = 0; j < G; ++j) old[j] = ld_cg_f4(src + (g0 + j) * 128 + r);
 #pragma unroll
               for (int j = 0; j < G; ++j) {
                 float* x = a + 4 * (g0 + j);
@@ -449,8 +512,20 @@ __global__ void __launch_bounds__(512, 1)
                 x[3] = old[j].w + x[3];
               }
             }
+          };
+          if (idx > 0) {
+            ticket_wait(p.tickets + unit, (uint32_t)idx);
+            if (threadIdx.x == 256) trace(it, 6);
+            add_from(accp);
           }
           if (last) {
+            if (ncontrib > 1) {
+              // the other chain is complete once its ticket counts all its positions
+              const int other = chain ^ 1;
+              const long long ounit = blk * 2 + other;
+              ticket_wait(p.tickets + ounit, (uint32_t)((ncontrib + 1 - other) / 2));
+              add_from(reinterpret_cast<const float4*>(p.acc) + ounit * (32 * D));
+            }
             __nv_bfloat16* out = p.dq + ((size_t)ch.x * S + (size_t)q * 128 + r) * D;
             const float sc = p.scale;
 #pragma unroll
@@ -471,10 +546,11 @@ __global__ void __launch_bounds__(512, 1)
             named_bar_sync(1, 128);
             if (threadIdx.x == 256) {
               __threadfence();
-              st_release_gpu(p.tickets + blk, (uint32_t)(pos + 1));
+              st_release_gpu(p.tickets + unit, (uint32_t)(idx + 1));
             }
           }
         } else {
+          float4* accp = reinterpret_cast<float4*>(p.acc + blk * 128 * D);
 #pragma unroll
           for (int c4 = 0; c4 < NV; ++c4)
             atomicAdd(accp + c4 * 128 + r,

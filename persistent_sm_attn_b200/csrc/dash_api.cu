@@ -163,7 +163,9 @@ int get_fault_table(int dev, int heads, int N, int causal, int sched, int ctas, 
     if (ch.bh == 0)
       for (int i = 0; i < ch.pair_cnt; ++i) {
         uint32_t& w = t.pairs[ch.pair_off + i];
-        if (dash::pair_q(w) == 0) w = dash::pack_pair(0, dash::pair_pos(w) + 1);
+        // the block's first two positions never arrive, so the first wait of both
+        // of its accumulation chains runs out
+        if (dash::pair_q(w) == 0) w = dash::pack_pair(0, dash::pair_pos(w) + 2);
       }
   cudaFree(g_fault_table.cta_off);
   cudaFree(g_fault_table.chains);
@@ -277,14 +279,16 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
     } else if ((rc = get_table(dev, B * H, N, causal, sched, ctas, &tab))) {
       return rc;
     }
-    if ((rc = get_workspace(dev, stream, (size_t)rows * D * sizeof(float),
+    if ((rc = get_workspace(dev, stream, 2 * (size_t)rows * D * sizeof(float),
                             (size_t)dash::dq_units<D>((long long)B * H * N) * sizeof(uint32_t),
                             (size_t)rows, &ws)))
       return rc;
   }
   CUtensorMap tq, tk, tv, tdo;
-  if ((rc = make_tmap(&tq, q, rows, D, 128)) || (rc = make_tmap(&tk, k, rows, D, 128)) ||
-      (rc = make_tmap(&tv, v, rows, D, 128)) || (rc = make_tmap(&tdo, dout, rows, D, 128)))
+  if ((rc = make_tmap(&tq, q, rows, D, C::kQRows)) ||
+      (rc = make_tmap(&tk, k, rows, D, C::kKVRows)) ||
+      (rc = make_tmap(&tv, v, rows, D, C::kKVRows)) ||
+      (rc = make_tmap(&tdo, dout, rows, D, C::kQRows)))
     return rc;
   float* lse2 = ws->rowbuf;
   float* delta = ws->rowbuf + ws->rows_cap;

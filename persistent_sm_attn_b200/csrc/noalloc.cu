@@ -133,7 +133,7 @@ size_t fixed_scratch(long long rows, int D, long long blocks) {
   return 256                                         // error word + abort flag
          + align256((size_t)blocks * 4)              // tickets
          + 2 * align256((size_t)rows * 4)            // scaled LSE, Delta
-         + align256((size_t)rows * D * 4);           // fp32 dQ accumulator
+         + align256(2 * (size_t)rows * D * 4);       // fp32 dQ accumulators (two per block)
 }
 
 template <int D, bool kAtomic>
@@ -156,7 +156,7 @@ int noalloc_launch(const void* q, const void* k, const void* v, const void* o, c
   float* delta = reinterpret_cast<float*>(p0 + off);
   off += align256((size_t)rows * 4);
   float* acc = reinterpret_cast<float*>(p0 + off);
-  off += align256((size_t)rows * D * 4);
+  off += align256(2 * (size_t)rows * D * 4);
   // the schedule table, built and checked on the host, then copied in
   const long long key[6] = {B * (long long)H, N, causal, sched, ctas, (long long)off};
   dash::Table t;
@@ -180,8 +180,10 @@ int noalloc_launch(const void* q, const void* k, const void* v, const void* o, c
   }
   CUtensorMap tq, tk, tv, tdo;
   int rc;
-  if ((rc = noalloc_tmap(&tq, q, rows, D, 128)) || (rc = noalloc_tmap(&tk, k, rows, D, 128)) ||
-      (rc = noalloc_tmap(&tv, v, rows, D, 128)) || (rc = noalloc_tmap(&tdo, dout, rows, D, 128)))
+  if ((rc = noalloc_tmap(&tq, q, rows, D, C::kQRows)) ||
+      (rc = noalloc_tmap(&tk, k, rows, D, C::kKVRows)) ||
+      (rc = noalloc_tmap(&tv, v, rows, D, C::kKVRows)) ||
+      (rc = noalloc_tmap(&tdo, dout, rows, D, C::kQRows)))
     return rc;
   // the array keeps the previous call's contents: clear what must start at zero
   if (cudaMemsetAsync(err, 0, 2 * sizeof(unsigned), stream) != cudaSuccess) return DASH_ERR_CUDA;
