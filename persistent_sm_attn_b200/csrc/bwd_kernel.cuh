@@ -26,8 +26,8 @@
 // bounds the 1-CTA tensor cores here.
 //
 // Warp roles (512 threads, four warpgroups):
-//   WG0, WG1  softmax / dS; WG0 owns Q columns 0-63, WG1 columns 64-127
-//   WG2       dQ reduction and the dK/dV epilogue (176 registers)
+//   WG0, WG1  softmax / dS; WG0 owns Q columns 0-63, WG1 columns 64-127 (120 registers)
+//   WG2       dQ reduction and the dK/dV epilogue (192 registers)
 //   WG3       warp 12 TMA producer, warp 13 MMA issuer and TMEM owner (80 registers)
 // TMEM lane quarter of a warp is (warp % 4), so each warpgroup covers the 128 lanes.
 //
@@ -80,9 +80,10 @@ template <int D>
 struct BwdCfg {
   static constexpr int kThreads = 512;
   static constexpr int kLaunchRegs = 65536 / kThreads;   // 128: the setmaxnreg split below
-  static constexpr int kRegsReduce = 176;                // WG2
+  static constexpr int kRegsSoftmax = 120;               // WG0, WG1
+  static constexpr int kRegsReduce = 192;                // WG2
   static constexpr int kRegsCtrl = 80;                   // WG3
-  static_assert(2 * kLaunchRegs + kRegsReduce + kRegsCtrl == 4 * kLaunchRegs,
+  static_assert(2 * kRegsSoftmax + kRegsReduce + kRegsCtrl == 4 * kLaunchRegs,
                 "register split must equal the launch allocation");
   static constexpr int kKVRows = 128;                    // TMA box rows of K and V
   static constexpr int kQRows = 128;                     // TMA box rows of Q and dO
@@ -350,6 +351,7 @@ __global__ void __launch_bounds__(512, 1)
     // ------------------------------------------------------------ softmax / dS
     // Two phases per tile: P first (all the exponentials), published so that the
     // MMA issuer can start dV while dS is computed; then dS once dP^T is in TMEM.
+    setmaxnreg_dec<C::kRegsSoftmax>();
     const int quarter = warp & 3, half = warp >> 2;
     const int r = quarter * 32 + lane;  // KV row of the tile = TMEM lane
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
@@ -477,10 +479,13 @@ __global__ void __launch_bounds__(512, 1)
           const int chain = pos & 1, idx = pos >> 1;
           const long long unit = blk * 2 + chain;
           float4* accp = reinterpret_cast<float4*>(p.acc) + unit * (32 * D);
-          // wait (bounded) until a chain's ticket reaches `want`
-          auto ticket_wait = [&](uint32_t* tk, uint32_t want) {
+          // wait (bounded) until a chain's ticket reaches `want`.  Lane 0 acquires
+          // (its acquire pairs with the publisher's release) and the warp barrier
+          // orders the other lanes' accumulator loads after it.  `seen` is a value
+          // lane 0 already acquired (~0u: none).
+          auto ticket_wait = [&](uint32_t* tk, uint32_t want, uint32_t seen) {
             if (lane == 0) {
-              if (ld_acquire_gpu(tk) != want) {
+              if (seen != want && ld_acquire_gpu(tk) != want) {
                 const uint64_t t0 = globaltimer();
                 bool ok = false;
                 while (!ok) {
@@ -494,7 +499,6 @@ __global__ void __launch_bounds__(512, 1)
               }
             }
             __syncwarp();
-            (void)ld_acquire_gpu(tk);
           };
           // a = acc + a over this thread's slots, G loads in flight before their adds
           auto add_from = [&](const float4* src) {
@@ -514,7 +518,7 @@ __global__ void __launch_bounds__(512, 1)
             }
           };
           if (idx > 0) {
-            ticket_wait(p.tickets + unit, (uint32_t)idx);
+            ticket_wait(p.tickets + unit, (uint32_t)idx, ~0u);
             if (threadIdx.x == 256) trace(it, 6);
             add_from(accp);
           }
@@ -523,7 +527,7 @@ __global__ void __launch_bounds__(512, 1)
               // the other chain is complete once its ticket counts all its positions
               const int other = chain ^ 1;
               const long long ounit = blk * 2 + other;
-              ticket_wait(p.tickets + ounit, (uint32_t)((ncontrib + 1 - other) / 2));
+              ticket_wait(p.tickets + ounit, (uint32_t)((ncontrib + 1 - other) / 2), ~0u);
               add_from(reinterpret_cast<const float4*>(p.acc) + ounit * (32 * D));
             }
             __nv_bfloat16* out = p.dq + ((size_t)ch.x * S + (size_t)q * 128 + r) * D;
@@ -543,11 +547,10 @@ __global__ void __launch_bounds__(512, 1)
             for (int c4 = 0; c4 < NV; ++c4)
               st_cg_f4(accp + c4 * 128 + r,
                        make_float4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]));
+            // the barrier orders every thread's stores before thread 256's release,
+            // which publishes them at gpu scope
             named_bar_sync(1, 128);
-            if (threadIdx.x == 256) {
-              __threadfence();
-              st_release_gpu(p.tickets + unit, (uint32_t)(idx + 1));
-            }
+            if (threadIdx.x == 256) st_release_gpu(p.tickets + unit, (uint32_t)(idx + 1));
           }
         } else {
           float4* accp = reinterpret_cast<float4*>(p.acc + blk * 128 * D);
