@@ -300,10 +300,11 @@ def simulator_vs_measured(w, q, k, v, o, do, lse, main_sched, measured_ms):
         if s_ == "atomic":
             continue
         cp, *_ = binding.dash_sched_simulate(w.B * w.H, w.n_tiles, w.causal, s_, ctas, c_us,
-                                             r_us, 2)
+                                             r_us, 2, 2)
         pred[s_] = round(cp / 1000.0, 4)
     det = {s_: m_ for s_, m_ in measured_ms.items() if s_ != "atomic"}
-    return {"c_us": round(c_us, 3), "r_us": round(r_us, 3), "dq_buffers": 2, "ctas": ctas,
+    return {"c_us": round(c_us, 3), "r_us": round(r_us, 3), "dq_buffers": 2, "dq_chains": 2,
+            "ctas": ctas,
             "predicted_ms": pred, "predicted_order": sorted(pred, key=pred.get),
             "measured_ms": {s_: round(m_, 4) for s_, m_ in det.items()},
             "measured_order": sorted(det, key=det.get)}

@@ -204,16 +204,35 @@ long long dash_sched_table(int n_heads, int N, int causal, int schedule, int num
  * DAG simulation of a schedule table (DASH summary §2.1): per pair the events
  * start, partial ready, reduction start, reduction done; arcs of weight
  * w_compute (tile compute) and w_reduce (ordered reduction), zero-weight
- * accumulation-order and chain arcs, and with dq_buffers >= 1 at most that
- * many partials in flight per CTA (<= 0: unbounded).  Outputs (any may be
- * NULL): critical_path (longest path), makespan (latest end of a compute
- * phase), bubble_time (sum over used CTAs of critical_path minus the CTA's
- * compute time), stalls (pairs whose partial waited for a free buffer).
+ * chain arcs, one reduction at a time per CTA, and with dq_buffers >= 1 at
+ * most that many partials in flight per CTA (<= 0: unbounded).  The
+ * accumulation order of a dQ block is one fixed chain when dq_chains = 1 (the
+ * pages' model); with dq_chains = K > 1 (the kernel uses 2) position p waits
+ * for position p - K and the block's last contributor for the last position
+ * of every other chain.  Outputs (any may be NULL): critical_path (longest
+ * path), makespan (latest end of a compute phase), bubble_time (sum over used
+ * CTAs of critical_path minus the CTA's compute time), stalls (pairs whose
+ * partial waited for a free buffer).  Returns DASH_ERR_INVALID_ARG for
+ * negative weights or dq_chains < 1.
  */
 int dash_sched_simulate(int n_heads, int N, int causal, int schedule, int num_ctas,
-                        double w_compute, double w_reduce, int dq_buffers,
+                        double w_compute, double w_reduce, int dq_buffers, int dq_chains,
                         double* critical_path, double* makespan, double* bubble_time,
                         long long* stalls);
+
+/*
+ * Checks a schedule table supplied by the caller, in the row format of
+ * dash_sched_table: n_rows rows of 6 ints (cta, head, kv_tile, q_tile,
+ * position, chain_index), grouped by CTA in ascending order, each CTA's rows in
+ * execution order, consecutive rows of one chain sharing its chain index.
+ * Checks that every pair of the mask appears once, that positions form a
+ * permutation per dQ block, that chains are unbroken, and that the ticket
+ * order cannot deadlock when all num_ctas CTAs run concurrently (DASH summary
+ * §2.1).  rows is read only.  Returns DASH_OK, DASH_ERR_INVALID_ARG for a
+ * malformed row list, or DASH_ERR_SCHEDULE when a check fails.
+ */
+int dash_sched_check(int n_heads, int N, int causal, int num_ctas, const int* rows,
+                     long long n_rows);
 
 /*
  * Longest paths of a general DAG with n_nodes nodes and n_edges weighted

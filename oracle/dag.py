@@ -14,7 +14,15 @@ four events per pair x = (kv, q)):
   d(y) -> s(x)  weight 0   accumulation order: y is x's predecessor in its dQ block
   s(x) -> d(x)  weight r   the reduction of the partial into the block
   b(x_n) -> a(x_n+1)  0    next pair on the same CTA slot (chain / resource order)
+  d(x_n) -> s(x_n+1)  0    one reduction at a time per slot (the SM's reducer)
   d(x_n+1-beta) -> b(x_n+1)  0   at most beta partials in flight per slot
+
+With K accumulation chains per dQ block (the block's positions split by
+position mod K, each residue class accumulating into an accumulator of its
+own in position order, and the last contributor adding the K sums), the
+predecessor of position p is position p - K, and the block's last contributor
+also waits for the last position of every other chain.  K = 1 is the single
+fixed order of the pages.
 
 The times of events are their longest-path depths from time 0.  This module
 finds them by enumerating every path explicitly, with no dynamic programming,
@@ -73,14 +81,14 @@ def paths_longest(n_nodes: int, edges):
     return cp, depth, height
 
 
-def schedule_graph(table, c: float, r: float, beta: int | None):
+def schedule_graph(table, c: float, r: float, beta: int | None, chains: int = 1):
     """Build the event graph of a packed schedule table.
 
     table: per slot, a list of (head, kv, q, position, n_contributors) as
     returned by ``oracle.schedules.packed_table``.  beta: dQ partial buffers
-    per slot, None for unbounded.  Returns (n_nodes, edges, index) where
-    index[(slot, n)] = node id of event a of the n-th pair on that slot
-    (b, s, d follow as +1, +2, +3).
+    per slot, None for unbounded.  chains: accumulation chains per dQ block.
+    Returns (n_nodes, edges, index) where index[(slot, n)] = node id of event
+    a of the n-th pair on that slot (b, s, d follow as +1, +2, +3).
     """
     index = {}
     nid = 0
@@ -97,17 +105,21 @@ def schedule_graph(table, c: float, r: float, beta: int | None):
         for n, (hd, kv, q, p, nc) in enumerate(seq):
             a = index[(sl, n)]
             edges += [(a, a + 1, c), (a + 1, a + 2, 0.0), (a + 2, a + 3, r)]
-            if p > 0:
-                y = by_block[(hd, q, p - 1)]
-                edges.append((y + 3, a + 2, 0.0))
+            preds = [p - chains] if p >= chains else []
+            if p == nc - 1:
+                preds += list(range(max(0, p - chains + 1), p))
+            for pp in preds:
+                edges.append((by_block[(hd, q, pp)] + 3, a + 2, 0.0))
             if n > 0:
-                edges.append((index[(sl, n - 1)] + 1, a, 0.0))
+                prev = index[(sl, n - 1)]
+                edges.append((prev + 1, a, 0.0))
+                edges.append((prev + 3, a + 2, 0.0))
                 if beta is not None and n - beta >= 0:
                     edges.append((index[(sl, n - beta)] + 3, a + 1, 0.0))
     return nid, edges, index
 
 
-def simulate(table, c: float, r: float, beta: int | None):
+def simulate(table, c: float, r: float, beta: int | None, chains: int = 1):
     """Critical path, compute makespan, idle (bubble) time and stall count of
     a schedule table, all by brute-force path enumeration.
 
@@ -116,7 +128,7 @@ def simulate(table, c: float, r: float, beta: int | None):
     bubble_time:   sum over used slots of (critical_path - that slot's compute).
     stalls:        pairs whose partial-ready event waits on a full buffer.
     """
-    n, edges, index = schedule_graph(table, c, r, beta)
+    n, edges, index = schedule_graph(table, c, r, beta, chains)
     cp, depth, _ = paths_longest(n, edges)
     makespan = 0.0
     bubble = 0.0

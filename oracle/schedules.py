@@ -79,10 +79,21 @@ def units(name: str, N: int, causal: bool):
     return out
 
 
-def accumulation_order(name: str, N: int, causal: bool):
+def accumulation_order(name: str, N: int, causal: bool, rounds=None):
     """dQ accumulation order per block: dict q -> list of (unit, step), first
-    partial first."""
+    partial first.
+
+    rounds[u] is the round in which unit u of the head runs (all 0 when every
+    unit of the head has a CTA slot of its own).  For the step-ordered
+    schedules a block accumulates in execution order: by round, then by step
+    within the round.  The pages only treat one unit per SM; taking the round
+    first is the plainest extension when a head has more units than slots or
+    straddles two rounds, and it keeps every wait pointing to an earlier
+    (round, step), so no table deadlocks.
+    """
     us = units(name, N, causal)
+    if rounds is None:
+        rounds = [0] * len(us)
     contrib = {q: [] for q in range(N)}
     for u, seq in enumerate(us):
         for t, (kv, q) in enumerate(seq):
@@ -90,17 +101,17 @@ def accumulation_order(name: str, N: int, causal: bool):
     order = {}
     for q, lst in contrib.items():
         if name in (NAIVE_ASC, DESCENDING):
-            lst = sorted(lst, key=lambda e: e[2])        # ascending KV
+            lst = sorted(lst, key=lambda e: e[2])                 # ascending KV
         else:
-            lst = sorted(lst, key=lambda e: e[1])        # step (phase, step) order
+            lst = sorted(lst, key=lambda e: (rounds[e[0]], e[1]))  # (round, step)
         order[q] = [(u, t) for (u, t, _kv) in lst]
     return order
 
 
-def positions(name: str, N: int, causal: bool):
+def positions(name: str, N: int, causal: bool, rounds=None):
     """Per-head table: list per unit of (kv, q, position, n_contributors)."""
     us = units(name, N, causal)
-    order = accumulation_order(name, N, causal)
+    order = accumulation_order(name, N, causal, rounds)
     pos = {}
     for q, lst in order.items():
         for p, ut in enumerate(lst):
@@ -118,10 +129,11 @@ def packed_table(name: str, n_heads: int, N: int, causal: bool, num_slots: int):
     num_slots.  (The pages only say that later heads follow; this static
     round-robin packing is the plainest reading.)
     """
-    per_head = positions(name, N, causal)
-    U = len(per_head)
+    U = len(units(name, N, causal))
     slots = [[] for _ in range(num_slots)]
     for hd in range(n_heads):
+        rounds = [(hd * U + k) // num_slots for k in range(U)]
+        per_head = positions(name, N, causal, rounds)
         for k in range(U):
             g = hd * U + k
             slots[g % num_slots].extend((hd,) + e for e in per_head[k])

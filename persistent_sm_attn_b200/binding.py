@@ -22,7 +22,7 @@ EXPORTS = ("dash_attn_fwd", "dash_attn_bwd", "dash_attn_sync_status", "dash_stat
            "dash_set_spin_limit_us", "dash_bwd_num_ctas", "dash_release_workspace",
            "dash_sched_table", "dash_sched_simulate", "dash_dag_longest_path",
            "dash_profile_begin", "dash_profile_end", "dash_attn_bwd_noalloc",
-           "dash_trace_bwd", "dash_inject_fault")
+           "dash_trace_bwd", "dash_inject_fault", "dash_sched_check")
 
 
 class DashError(RuntimeError):
@@ -62,7 +62,8 @@ def load(path: str | None = None):
     lib.dash_release_workspace.argtypes = []
     lib.dash_sched_table.argtypes = [i, i, i, i, i, vp, ll]
     lib.dash_sched_table.restype = ll
-    lib.dash_sched_simulate.argtypes = [i, i, i, i, i, d, d, i, P(d), P(d), P(d), P(ll)]
+    lib.dash_sched_simulate.argtypes = [i, i, i, i, i, d, d, i, i, P(d), P(d), P(d), P(ll)]
+    lib.dash_sched_check.argtypes = [i, i, i, i, vp, ll]
     lib.dash_dag_longest_path.argtypes = [i, i, vp, vp, vp, vp, vp, P(d)]
     lib.dash_trace_bwd.argtypes = [vp] * 9 + [i, i, i, i, i, i, vp, vp, ll, P(i), P(i)]
     lib.dash_profile_begin.argtypes = []
@@ -185,16 +186,27 @@ def dash_sched_table(n_heads: int, N: int, causal: bool, schedule, num_ctas: int
 
 
 def dash_sched_simulate(n_heads: int, N: int, causal: bool, schedule, num_ctas: int,
-                        w_compute: float, w_reduce: float, dq_buffers: int = 0):
-    """(critical_path, makespan, bubble_time, stalls) of a schedule's DAG."""
+                        w_compute: float, w_reduce: float, dq_buffers: int = 0,
+                        dq_chains: int = 1):
+    """(critical_path, makespan, bubble_time, stalls) of a schedule's DAG;
+    dq_chains = 2 models the kernel's two accumulators per dQ block."""
     cp, mk, bt = ctypes.c_double(), ctypes.c_double(), ctypes.c_double()
     st = ctypes.c_longlong()
     rc = load().dash_sched_simulate(n_heads, N, int(bool(causal)), _sched_id(schedule), num_ctas,
                                     float(w_compute), float(w_reduce), int(dq_buffers),
-                                    ctypes.byref(cp), ctypes.byref(mk), ctypes.byref(bt),
-                                    ctypes.byref(st))
+                                    int(dq_chains), ctypes.byref(cp), ctypes.byref(mk),
+                                    ctypes.byref(bt), ctypes.byref(st))
     _check(rc, "dash_sched_simulate")
     return cp.value, mk.value, bt.value, st.value
+
+
+def dash_sched_check(n_heads: int, N: int, causal: bool, num_ctas: int, rows) -> int:
+    """Status of the library's checks on a caller-supplied table given as rows
+    (cta, head, kv, q, position, chain_index): 0 valid, 6 a failed check
+    (coverage, positions or a deadlocking ticket order), 1 malformed rows."""
+    flat = [int(x) for r in rows for x in r]
+    buf = (ctypes.c_int * max(len(flat), 1))(*flat)
+    return int(load().dash_sched_check(n_heads, N, int(bool(causal)), num_ctas, buf, len(rows)))
 
 
 def dash_dag_longest_path(n_nodes: int, edges):

@@ -635,21 +635,33 @@ long long dash_sched_table(int n_heads, int N, int causal, int schedule, int num
 }
 
 int dash_sched_simulate(int n_heads, int N, int causal, int schedule, int num_ctas,
-                        double w_compute, double w_reduce, int dq_buffers, double* critical_path,
-                        double* makespan, double* bubble_time, long long* stalls) {
-  if (w_compute < 0 || w_reduce < 0) return DASH_ERR_INVALID_ARG;
+                        double w_compute, double w_reduce, int dq_buffers, int dq_chains,
+                        double* critical_path, double* makespan, double* bubble_time,
+                        long long* stalls) {
+  if (w_compute < 0 || w_reduce < 0 || dq_chains < 1) return DASH_ERR_INVALID_ARG;
   dash::Table t;
   std::string err;
   if (!dash::build_table(n_heads, N, causal, schedule, num_ctas, &t, &err))
     return DASH_ERR_UNSUPPORTED;
   if (!dash::validate_table(t, &err)) return DASH_ERR_SCHEDULE;
   dash::SimResult r;
-  if (!dash::simulate_table(t, w_compute, w_reduce, dq_buffers, &r, &err)) return DASH_ERR_SCHEDULE;
+  if (!dash::simulate_table(t, w_compute, w_reduce, dq_buffers, dq_chains, &r, &err))
+    return DASH_ERR_SCHEDULE;
   if (critical_path) *critical_path = r.critical_path;
   if (makespan) *makespan = r.makespan;
   if (bubble_time) *bubble_time = r.bubble_time;
   if (stalls) *stalls = r.stalls;
   return DASH_OK;
+}
+
+int dash_sched_check(int n_heads, int N, int causal, int num_ctas, const int* rows,
+                     long long n_rows) {
+  if (causal != 0 && causal != 1) return DASH_ERR_INVALID_ARG;
+  dash::Table t;
+  std::string err;
+  if (!dash::table_from_rows(n_heads, N, causal, num_ctas, rows, n_rows, &t, &err))
+    return DASH_ERR_INVALID_ARG;
+  return dash::validate_table(t, &err) ? DASH_OK : DASH_ERR_SCHEDULE;
 }
 
 int dash_dag_longest_path(int n_nodes, int n_edges, const int* src, const int* dst, const double* w,

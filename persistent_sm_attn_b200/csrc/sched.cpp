@@ -5,8 +5,9 @@
 //   NAIVE_ASC   serialised baseline of §1: Q tiles ascending, dQ order by KV.
 //   DESCENDING  §2.2.A: Q tiles from the last to the first, dQ order by KV.
 //   SHIFT       §2.2.B full masks: the chain of KV tile k visits Q tiles
-//               k, k+1, ..., N-1, 0, ..., k-1; dQ blocks accumulate in step
-//               order, so every step touches N distinct blocks.
+//               k, k+1, ..., N-1, 0, ..., k-1; dQ blocks accumulate in
+//               execution order (round, then step), so every step touches N
+//               distinct blocks.
 //   SYM_SHIFT   §2.2.B causal masks: KV tiles k and N-1-k share one CTA; a
 //               dense phase over Q in [N/2, N) x KV in [0, N/2) is followed by
 //               the folded triangle; dQ blocks accumulate in (phase, step)
@@ -20,6 +21,7 @@
 #include <cmath>
 #include <cstdio>
 #include <deque>
+#include <map>
 #include <queue>
 
 namespace dash {
@@ -98,23 +100,39 @@ bool build_table(int n_heads, int N, int causal, int schedule, int num_ctas, Tab
   }
   const Units units = units_of(schedule, N, causal);
   const int U = (int)units.size();
-  // positions within each dQ block, for one head
-  // key: NAIVE_ASC / DESCENDING order by KV; SHIFT / SYM_SHIFT / ATOMIC by step
+  // Positions within each dQ block, per head.  NAIVE_ASC / DESCENDING order a
+  // block by KV; SHIFT / SYM_SHIFT / ATOMIC by execution order: the round in
+  // which the unit runs (global unit g runs in round g / num_ctas), then the
+  // step.  The round only matters for heads whose units span two rounds;
+  // heads with the same first-unit offset in their round share one table.
   const bool by_kv = (schedule == NAIVE_ASC || schedule == DESCENDING);
-  std::vector<std::vector<std::pair<long long, int>>> contrib(N);  // per q: (key, unit*65536+step)
-  for (int k = 0; k < U; ++k)
-    for (int t = 0; t < (int)units[k].size(); ++t) {
-      const int kv = units[k][t].first, q = units[k][t].second;
-      const long long key = by_kv ? kv : (long long)t * 65536 + k;
-      contrib[q].push_back({key, k * 65536 + t});
+  auto head_positions = [&](long long first_g) {
+    std::vector<std::vector<std::pair<long long, int>>> contrib(N);  // per q: (key, unit*65536+step)
+    for (int k = 0; k < U; ++k) {
+      const long long rnd = (first_g + k) / num_ctas - first_g / num_ctas;
+      for (int t = 0; t < (int)units[k].size(); ++t) {
+        const int kv = units[k][t].first, q = units[k][t].second;
+        const long long key = by_kv ? kv : (rnd << 40) + (long long)t * 65536 + k;
+        contrib[q].push_back({key, k * 65536 + t});
+      }
     }
-  std::vector<std::vector<int>> pos(U);
-  for (int k = 0; k < U; ++k) pos[k].assign(units[k].size(), -1);
-  for (int q = 0; q < N; ++q) {
-    auto& c = contrib[q];
-    std::sort(c.begin(), c.end());
-    for (int p = 0; p < (int)c.size(); ++p) pos[c[p].second >> 16][c[p].second & 0xffff] = p;
-  }
+    std::vector<std::vector<int>> pos(U);
+    for (int k = 0; k < U; ++k) pos[k].assign(units[k].size(), -1);
+    for (int q = 0; q < N; ++q) {
+      auto& c = contrib[q];
+      std::sort(c.begin(), c.end());
+      for (int p = 0; p < (int)c.size(); ++p) pos[c[p].second >> 16][c[p].second & 0xffff] = p;
+    }
+    return pos;
+  };
+  std::map<long long, std::vector<std::vector<int>>> pos_by_offset;
+  auto positions_of = [&](int bh) -> const std::vector<std::vector<int>>& {
+    const long long first_g = (long long)bh * U;
+    const long long key = by_kv ? 0 : first_g % num_ctas;
+    auto f = pos_by_offset.find(key);
+    if (f == pos_by_offset.end()) f = pos_by_offset.emplace(key, head_positions(first_g)).first;
+    return f->second;
+  };
   Table t;
   t.n_heads = n_heads; t.N = N; t.causal = causal; t.schedule = schedule; t.num_ctas = num_ctas;
   // per CTA, the global units it runs, in round order
@@ -127,6 +145,7 @@ bool build_table(int n_heads, int N, int causal, int schedule, int num_ctas, Tab
     for (long long g : per_cta[c]) {
       const int bh = (int)(g / U), k = (int)(g % U);
       const auto& seq = units[k];
+      const auto& pos = positions_of(bh);
       for (int i = 0; i < (int)seq.size(); ++i) {
         if (i == 0 || seq[i].first != seq[i - 1].first) {
           Chain ch{bh, seq[i].first, (int32_t)t.pairs.size(), 0};
@@ -138,6 +157,36 @@ bool build_table(int n_heads, int N, int causal, int schedule, int num_ctas, Tab
     }
   }
   t.cta_off[num_ctas] = (int32_t)t.chains.size();
+  *out = std::move(t);
+  return true;
+}
+
+bool table_from_rows(int n_heads, int N, int causal, int num_ctas, const int* rows,
+                     long long n_rows, Table* out, std::string* err) {
+  auto fail = [&](const char* m) { if (err) *err = m; return false; };
+  if (n_heads < 1 || N < 1 || N > 32767 || num_ctas < 1 || n_rows < 0 || (n_rows > 0 && !rows))
+    return fail("bad table shape");
+  Table t;
+  t.n_heads = n_heads; t.N = N; t.causal = causal; t.schedule = NAIVE_ASC; t.num_ctas = num_ctas;
+  t.cta_off.assign(num_ctas + 1, 0);
+  int prev_cta = 0, prev_chain = -1;
+  for (long long i = 0; i < n_rows; ++i) {
+    const int* r = rows + 6 * i;
+    const int cta = r[0], bh = r[1], kv = r[2], q = r[3], pos = r[4], chain = r[5];
+    if (cta < prev_cta || cta >= num_ctas) return fail("rows not grouped by CTA in order");
+    if (q < 0 || q >= N || pos < 0 || pos >= N) return fail("q tile or position out of range");
+    if (t.chains.empty() || cta != prev_cta || chain != prev_chain) {
+      for (int c = prev_cta + 1; c <= cta; ++c) t.cta_off[c] = (int32_t)t.chains.size();
+      t.chains.push_back(Chain{bh, kv, (int32_t)t.pairs.size(), 0});
+    } else if (t.chains.back().bh != bh || t.chains.back().kv != kv) {
+      return fail("a chain changes head or KV tile");
+    }
+    t.chains.back().pair_cnt++;
+    t.pairs.push_back(pack_pair(q, pos));
+    prev_cta = cta;
+    prev_chain = chain;
+  }
+  for (int c = prev_cta + 1; c <= num_ctas; ++c) t.cta_off[c] = (int32_t)t.chains.size();
   *out = std::move(t);
   return true;
 }
@@ -257,8 +306,9 @@ bool dag_longest_path(int n, int m, const int* src, const int* dst, const double
   return true;
 }
 
-bool simulate_table(const Table& t, double c, double r, int beta, SimResult* res,
+bool simulate_table(const Table& t, double c, double r, int beta, int chains, SimResult* res,
                     std::string* err) {
+  if (chains < 1) { if (err) *err = "chains must be >= 1"; return false; }
   const long long P = t.n_pairs();
   if (P * 4 > (1LL << 31) - 1) { if (err) *err = "table too large to simulate"; return false; }
   const int N = t.N;
@@ -293,14 +343,26 @@ bool simulate_table(const Table& t, double c, double r, int beta, SimResult* res
         edge(a + 1, a + 2, 0.0);
         edge(a + 2, a + 3, r);
         const int p = pair_pos(w);
-        if (p > 0) {
-          const size_t key = ((size_t)ch.bh * N + pair_q(w)) * N + (p - 1);
+        const int nc = t.causal ? pair_q(w) + 1 : N;
+        // accumulation order: position p - chains of the same chain, and for the
+        // block's last contributor the last position of every other chain
+        auto pred = [&](int pp) {
+          const size_t key = ((size_t)ch.bh * N + pair_q(w)) * N + pp;
           const int y = blk_pos_node[key];
-          if (y < 0) { if (err) *err = "missing predecessor in dQ order"; return false; }
+          if (y < 0) return false;
           edge(y + 3, a + 2, 0.0);
+          return true;
+        };
+        if (p >= chains && !pred(p - chains)) {
+          if (err) *err = "missing predecessor in dQ order";
+          return false;
         }
+        if (p == nc - 1)
+          for (int pp = std::max(0, p - chains + 1); pp < p; ++pp)
+            if (!pred(pp)) { if (err) *err = "missing predecessor in dQ order"; return false; }
         if (n > 0) {
           edge(nodes[n - 1] + 1, a, 0.0);
+          edge(nodes[n - 1] + 3, a + 2, 0.0);  // one reduction at a time per CTA
           if (beta >= 1 && (long long)n - beta >= 0) edge(nodes[n - beta] + 3, a + 1, 0.0);
         }
       }

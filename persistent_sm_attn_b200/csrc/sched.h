@@ -42,7 +42,9 @@ bool schedule_supported(int schedule, int N, int causal);
 // Units of one head: each a list of (kv, q) in visiting order.
 std::vector<std::vector<std::pair<int, int>>> head_units(int schedule, int N, int causal);
 
-// Build the whole-grid table: heads in order, unit g on CTA g mod num_ctas.
+// Build the whole-grid table: heads in order, unit g on CTA g mod num_ctas in
+// round g / num_ctas; step-ordered schedules accumulate each dQ block in
+// (round, step) order.
 // Returns false (with a message) if the combination is unsupported.
 bool build_table(int n_heads, int N, int causal, int schedule, int num_ctas, Table* out,
                  std::string* err);
@@ -64,9 +66,20 @@ struct SimResult {
 
 // Event-graph simulation of a table: per pair, events a (start), b (partial
 // ready), s (reduction start), d (reduction done); arcs a->b weight c,
-// b->s 0, d(prev in order)->s 0, s->d weight r, b(prev on slot)->a 0, and with
-// beta >= 1 buffers d(pair n-beta on slot)->b(pair n).  beta <= 0 = unbounded.
-bool simulate_table(const Table& t, double c, double r, int beta, SimResult* res,
+// b->s 0, s->d weight r, b(prev on slot)->a 0, d(prev on slot)->s 0 (one
+// reducer per CTA), with beta >= 1 buffers d(pair n-beta on slot)->b(pair n)
+// (beta <= 0 = unbounded), and the accumulation order: with `chains`
+// accumulators per dQ block, d(position p - chains)->s(p), and for the block's
+// last contributor d(last position of every other chain)->s.  chains = 1 is
+// the single fixed order.
+bool simulate_table(const Table& t, double c, double r, int beta, int chains, SimResult* res,
                     std::string* err);
+
+// A table given as rows of six ints {cta, bh, kv, q, position, chain id}, the
+// format dash_sched_table writes: rows grouped by CTA in ascending order, each
+// CTA's rows in execution order, consecutive rows of one chain sharing the
+// chain id.  Only the shape is checked here; validate_table checks the rest.
+bool table_from_rows(int n_heads, int N, int causal, int num_ctas, const int* rows,
+                     long long n_rows, Table* out, std::string* err);
 
 }  // namespace dash

@@ -57,7 +57,9 @@ def test_argument_errors_need_no_gpu(lib):
     assert _bwd(lib, good, S=384, causal=1, sched=3) == 2   # odd tile count
     assert _bwd(lib, good, causal=2) == 1
     assert lib.dash_attn_fwd(*good[:5], 1, 1, 128, 80, 0, None) == 2
-    assert lib.dash_sched_simulate(1, 4, 0, 2, 4, -1.0, 0.0, 0, None, None, None, None) == 1
+    assert lib.dash_sched_simulate(1, 4, 0, 2, 4, -1.0, 0.0, 0, 1, None, None, None, None) == 1
+    assert lib.dash_sched_simulate(1, 4, 0, 2, 4, 1.0, 0.0, 0, 0, None, None, None, None) == 1
+    assert lib.dash_sched_check(1, 4, 2, 4, None, 0) == 1
 
 
 def test_dag_cycle_rejected():

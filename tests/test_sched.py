@@ -49,13 +49,48 @@ def test_full_size_tables_validate():
         assert len(rows) == heads * (N * (N + 1) // 2 if causal else N * N)
 
 
-def test_deadlock_detected():
-    # a shift head needs all its N chains co-resident; 4 CTAs cannot hold 8
-    with pytest.raises(binding.DashError) as e:
-        binding.dash_sched_table(1, 8, False, "shift", 4)
-    assert e.value.status == 6
-    # the descending order only waits on lower KV tiles: it never deadlocks
+def test_more_units_than_ctas_never_deadlock():
+    # a shift head of 8 chains on 4 CTAs runs in two rounds; its dQ blocks
+    # accumulate round by round, so the table is valid
+    rows = binding.dash_sched_table(1, 8, False, "shift", 4)
+    assert len(rows) == 64
+    assert binding.dash_sched_check(1, 8, False, 4, rows) == 0
+    # the descending order only waits on lower KV tiles
     assert len(binding.dash_sched_table(1, 8, False, "descending", 4)) == 64
+
+
+def _step_ordered_shift_rows(N, ctas):
+    """Shift visiting order with every dQ block accumulated in step order
+    regardless of rounds: with fewer CTAs than chains a CTA of the first round
+    waits for a partial that only a chain of the second round produces."""
+    rows = []
+    for g in range(N):  # global unit g = KV tile g of head 0
+        for t in range(N):
+            rows.append((g % ctas, g // ctas, g, (g + t) % N, t))
+    out = []
+    for c in range(ctas):
+        for rnd, kv, t, q in sorted((r[1], r[2], r[4], r[3]) for r in rows if r[0] == c):
+            out.append((c, 0, kv, q, t, kv))
+    return out
+
+
+def test_deadlock_detected():
+    rows = _step_ordered_shift_rows(8, 4)
+    assert binding.dash_sched_check(1, 8, False, 4, rows) == 6
+    # with one CTA per chain the same order is valid
+    assert binding.dash_sched_check(1, 8, False, 8, _step_ordered_shift_rows(8, 8)) == 0
+
+
+def test_check_rejects_coverage_and_position_errors():
+    rows = binding.dash_sched_table(1, 4, False, "shift", 4)
+    assert binding.dash_sched_check(1, 4, False, 4, rows) == 0
+    assert binding.dash_sched_check(1, 4, False, 4, rows[:-1]) == 6        # a pair missing
+    bad = [list(r) for r in rows]
+    bad[0][4], bad[1][4] = bad[1][4], bad[0][4]    # two blocks' positions swapped
+    a, b = rows[0], rows[1]
+    if a[3] != b[3]:
+        assert binding.dash_sched_check(1, 4, False, 4, bad) == 6
+    assert binding.dash_sched_check(1, 4, False, 4, [(5, 0, 0, 0, 0, 0)]) == 1   # CTA out of range
 
 
 @pytest.mark.parametrize("name,N,causal,heads,ctas", [
@@ -63,11 +98,12 @@ def test_deadlock_detected():
     (sc.NAIVE_ASC, 4, True, 2, 3), (sc.DESCENDING, 4, True, 1, 4), (sc.DESCENDING, 3, False, 2, 4),
     (sc.SYM_SHIFT, 4, True, 2, 3), (sc.SYM_SHIFT, 2, True, 3, 2)])
 @pytest.mark.parametrize("beta", [None, 1, 2])
-def test_simulator_matches_bruteforce(name, N, causal, heads, ctas, beta):
+@pytest.mark.parametrize("chains", [1, 2])
+def test_simulator_matches_bruteforce(name, N, causal, heads, ctas, beta, chains):
     c, r = 1.0, 0.35
     table = sc.packed_table(name, heads, N, causal, ctas)
-    want = dag.simulate(table, c, r, beta)
-    got = binding.dash_sched_simulate(heads, N, causal, SID[name], ctas, c, r, beta or 0)
+    want = dag.simulate(table, c, r, beta, chains)
+    got = binding.dash_sched_simulate(heads, N, causal, SID[name], ctas, c, r, beta or 0, chains)
     assert got[3] == want[3]
     for g, w in zip(got[:3], want[:3]):
         assert abs(g - w) < 1e-9
