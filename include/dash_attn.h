@@ -34,7 +34,7 @@
  *     asynchronous: DASH_OK means the work was enqueued.  Argument and launch
  *     errors are returned at once; errors found on the device (a spin wait
  *     that ran out) are reported by dash_attn_sync_status().
- *   - The library owns its workspace (fp32 dQ accumulator, tickets, the
+ *   - The library owns its workspace (fp32 dQ accumulators, tickets, the
  *     per-row Delta and scaled LSE, an error word) and caches it per
  *     (device, stream); schedule tables are cached per shape.  Calls on
  *     different streams use different workspaces.  Workspace memory is
@@ -136,10 +136,11 @@ int dash_profile_end(double* main_ms, double* aux_ms, long long* launches);
  * a %globaltimer trace of every (KV tile, Q tile) pair, for measuring the
  * compute time c and the reduction time r of the DAG model (DASH summary
  * §2.1).  host_trace receives up to `cap` u64 entries laid out
- * [num_ctas][rows_per_cta][8] (unused rows stay 0); events per pair: 0 tile
- * start at the MMA issuer, 1 softmax done, 2 tile MMAs issued, 3 softmax start,
- * 4 dQ partial ready at the reducers, 5 partial drained from TMEM, 6 ticket
- * granted (0 for a block's first contributor), 7 reduction published.
+ * [num_ctas][rows_per_cta][8] (unused rows stay 0); events per pair: 0 S^T
+ * issued, 1 softmax done (seen by the MMA issuer), 2 tile MMAs issued, 3
+ * softmax start, 4 dQ partial ready at the reducers, 5 partial drained from
+ * TMEM, 6 ticket granted (0 for the first contributor of each of the block's
+ * two accumulation chains), 7 reduction published or dQ written.
  * Allocates and frees its own trace buffer.
  */
 int dash_trace_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -165,9 +166,9 @@ int dash_release_workspace(void);
  * array of DASH_NOALLOC_SCRATCH_BYTES bytes, which every GPU that loads the
  * library holds until the process exits.  The call never calls cudaMalloc,
  * cudaFree or an allocating library routine.
- *   - Size limit: the array must hold the fp32 dQ accumulator (B*H*S*D*4
- *     bytes), the per-row Delta and scaled LSE (2*B*H*S*4), one ticket per
- *     128-row dQ block and the schedule table; larger calls return
+ *   - Size limit: the array must hold the two fp32 dQ accumulators per block
+ *     (2*B*H*S*D*4 bytes), the per-row Delta and scaled LSE (2*B*H*S*4), two
+ *     tickets per 128-row dQ block and the schedule table; larger calls return
  *     DASH_ERR_OOM without touching the device.
  *   - Set-up: the first call on a device (with that device current) looks up
  *     the array's device address and sizes the persistent grid; make that
