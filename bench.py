@@ -18,6 +18,7 @@ the same computation) on a bounded sample of heads of the same workload.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -149,6 +150,9 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     w = WORKLOADS[args.workload]
+    if args.heads:
+        # a smaller case of the same kernel (profiling): B=1 and the given head count
+        w = dataclasses.replace(w, B=1, H=args.heads, name=f"{w.name}_as_b1_h{args.heads}")
     sched = args.schedule or w.schedules[0]
     q, k, v, do = draw(w.B, w.H, w.S, w.D, w.sigma, seed_of(args.workload) + 1000 * rank,
                        device="cuda")
@@ -394,6 +398,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--all-workloads", action="store_true",
                     help="one JSON line per workload (1-4), rank 0 only")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run the workload's shape with B=1 and this many heads (a smaller "
+                         "case of the same kernel, for profiling); 0 = the workload as named")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
