@@ -1,5 +1,7 @@
 // Supporting kernels of the backward path:
-//   dash_delta_kernel   Delta_i = sum_d dO_id O_id (fp32) and LSE_i * log2(e) per row
+//   dash_delta_kernel   Delta_i = sum_d dO_id O_id (fp32), and per row the column
+//                       terms the backward's S^T and dP^T products add (LSE_i / scale
+//                       and Delta_i, each as three bf16 parts)
 //   dash_dq_convert     fp32 accumulator -> bf16 dQ (atomic comparison variant only)
 //   dash_fwd_kernel     softmax-attention forward producing O and LSE; it only
 //                       feeds the backward, so it uses plain fp32 FMAs.
@@ -19,13 +21,25 @@ __device__ __forceinline__ void bf16x8_to_f32(uint4 v, float* f) {
   }
 }
 
-// One group of D/8 lanes per row; 16-byte loads of O and dO.
+// x as three bf16 parts whose fp32 sum is x to about 24 bits: hi = bf16(x),
+// mid = bf16(x - hi), lo = bf16(x - hi - mid).
+__device__ __forceinline__ void split3_bf16(float x, __nv_bfloat16* part) {
+  part[0] = __float2bfloat16_rn(x);
+  const float r1 = x - __bfloat162float(part[0]);
+  part[1] = __float2bfloat16_rn(r1);
+  part[2] = __float2bfloat16_rn(r1 - __bfloat162float(part[1]));
+}
+
+// One group of D/8 lanes per row; 16-byte loads of O and dO.  Writes cols[row] =
+// 8 bf16: -(LSE_row / scale) in three parts, -Delta_row in three parts, two zeros.
+// The backward adds them to S^T and dP^T through one extra K-step of each product
+// (against constant ones), so S' = S - LSE/scale and dP' = dP - Delta.
 template <int D>
 __global__ void __launch_bounds__(256) dash_delta_kernel(const __nv_bfloat16* __restrict__ o,
                                                          const __nv_bfloat16* __restrict__ dout,
                                                          const float* __restrict__ lse,
-                                                         float* __restrict__ delta,
-                                                         float* __restrict__ lse2, long long rows) {
+                                                         uint4* __restrict__ cols, long long rows,
+                                                         float inv_scale) {
   constexpr int L = D / 8;  // lanes per row
   const long long gt = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long row = gt / L;
@@ -43,8 +57,11 @@ __global__ void __launch_bounds__(256) dash_delta_kernel(const __nv_bfloat16* __
 #pragma unroll
   for (int m = L / 2; m >= 1; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
   if (row < rows && sub == 0) {
-    delta[row] = acc;
-    lse2[row] = lse[row] * 1.4426950408889634f;
+    __align__(16) __nv_bfloat16 part[8];
+    split3_bf16(-lse[row] * inv_scale, part);
+    split3_bf16(-acc, part + 3);
+    part[6] = part[7] = __float2bfloat16_rn(0.f);
+    cols[row] = *reinterpret_cast<const uint4*>(part);
   }
 }
 

@@ -26,9 +26,9 @@
 // bounds the 1-CTA tensor cores here.
 //
 // Warp roles (512 threads, four warpgroups):
-//   WG0, WG1  softmax / dS; WG0 owns Q columns 0-63, WG1 columns 64-127 (120 registers)
-//   WG2       dQ reduction and the dK/dV epilogue (192 registers)
-//   WG3       warp 12 TMA producer, warp 13 MMA issuer and TMEM owner (80 registers)
+//   WG0, WG1  softmax / dS; WG0 owns Q columns 0-63, WG1 columns 64-127 (96 registers)
+//   WG2       dQ reduction and the dK/dV epilogue (224 registers)
+//   WG3       warp 12 TMA producer, warp 13 MMA issuer and TMEM owner (96 registers)
 // TMEM lane quarter of a warp is (warp % 4), so each warpgroup covers the 128 lanes.
 //
 // TMEM columns (512): S^T [0,128) then packed P^T/dS^T, dP^T [128,256),
@@ -54,8 +54,6 @@
 namespace dash {
 
 struct BwdParams {
-  const float* lse2;      // [B*H*S] LSE * log2(e)
-  const float* delta;     // [B*H*S] Delta_i = dO_i . O_i (fp32)
   const int* cta_off;     // [grid + 1]
   const int4* chains;     // {bh, kv, pair_off, pair_cnt}
   const uint32_t* pairs;  // q | position << 16
@@ -80,24 +78,33 @@ template <int D>
 struct BwdCfg {
   static constexpr int kThreads = 512;
   static constexpr int kLaunchRegs = 65536 / kThreads;   // 128: the setmaxnreg split below
-  static constexpr int kRegsSoftmax = 120;               // WG0, WG1
-  static constexpr int kRegsReduce = 192;                // WG2
-  static constexpr int kRegsCtrl = 80;                   // WG3
+  static constexpr int kRegsSoftmax = 96;                // WG0, WG1
+  static constexpr int kRegsReduce = 224;                // WG2
+  static constexpr int kRegsCtrl = 96;                   // WG3
   static_assert(2 * kRegsSoftmax + kRegsReduce + kRegsCtrl == 4 * kLaunchRegs,
                 "register split must equal the launch allocation");
   static constexpr int kKVRows = 128;                    // TMA box rows of K and V
   static constexpr int kQRows = 128;                     // TMA box rows of Q and dO
   static constexpr int kTile = 128 * D * 2;              // one [128][D] bf16 tile
-  static constexpr int kStages = (D == 64) ? 3 : 2;      // Q/dO pipeline depth
-  static constexpr int OFF_K = 0;
+  // Q is double-buffered (the next S^T follows dK right away); at D = 128 dO has one
+  // buffer, refilled between dV of a tile and dP^T of the next, to fit the smem budget.
+  static constexpr int kStagesQ = (D == 64) ? 3 : 2;
+  static constexpr int kStagesDO = (D == 64) ? 3 : 1;
+  // LSE and Delta enter the S^T and dP^T products as one extra K-step each: a per-Q-row
+  // column tile ([128 rows][8] bf16, loaded with Q) against a constant tile of ones.
+  // Each tile is 2 KiB of core matrices (8 rows x 16 bytes, no swizzle) followed by
+  // 2 KiB of zeros for the K-step's second half.  They sit first in shared memory.
+  static constexpr int kColTile = 4096;
+  static constexpr int OFF_ONES = 0;                       // ones for S^T, then for dP^T
+  static constexpr int OFF_COL = OFF_ONES + 2 * kColTile;  // kStagesQ column tiles
+  static constexpr int OFF_K = OFF_COL + kStagesQ * kColTile;
+  static_assert(OFF_K % 1024 == 0, "swizzled tiles need 1 KiB alignment");
   static constexpr int OFF_V = OFF_K + kTile;
   static constexpr int OFF_Q = OFF_V + kTile;
-  static constexpr int OFF_DO = OFF_Q + kStages * kTile;
-  static constexpr int OFF_DST = OFF_DO + kStages * kTile;  // dS^T [128 kv][128 q]
-  static constexpr int OFF_LSE = OFF_DST + 32768;           // kStages x 128 fp32 (with Q)
-  static constexpr int OFF_DEL = OFF_LSE + kStages * 512;  // kStages x 128 fp32 (with Q)
-  static constexpr int OFF_BAR = OFF_DEL + kStages * 512;
-  static constexpr int kBars = 16 + 4 * kStages;
+  static constexpr int OFF_DO = OFF_Q + kStagesQ * kTile;
+  static constexpr int OFF_DST = OFF_DO + kStagesDO * kTile;  // dS^T [128 kv][128 q]
+  static constexpr int OFF_BAR = OFF_DST + 32768;
+  static constexpr int kBars = 16 + 2 * kStagesQ + 2 * kStagesDO;
   static constexpr int OFF_TMEM_SLOT = OFF_BAR + kBars * 8;
   // The swizzled tiles need a 1 KiB aligned base; the kernel checks it.
   static constexpr int kSmemBytes = OFF_TMEM_SLOT + 16;
@@ -129,10 +136,10 @@ template <int D, bool kAtomic, bool kTrace = false>
 __global__ void __launch_bounds__(512, 1)
     dash_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                    const BwdParams p) {
+                    const __grid_constant__ CUtensorMap tmC, const BwdParams p) {
   using namespace dev;
   using C = BwdCfg<D>;
-  constexpr int ST = C::kStages;
+  constexpr int ST = C::kStagesQ, SD = C::kStagesDO;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t sb = smem_u32(smem_raw);
   if (sb & 1023u) {  // the launch gave an unaligned base: refuse rather than misread
@@ -145,14 +152,12 @@ __global__ void __launch_bounds__(512, 1)
   uint8_t* gb = smem_raw;
   const uint32_t sK = sb + C::OFF_K, sV = sb + C::OFF_V, sQ = sb + C::OFF_Q, sDO = sb + C::OFF_DO;
   const uint32_t sDSt = sb + C::OFF_DST;
-  const float* lse_s = reinterpret_cast<const float*>(gb + C::OFF_LSE);
-  const float* del_s = reinterpret_cast<const float*>(gb + C::OFF_DEL);
   const uint32_t bar0 = sb + C::OFF_BAR;
   auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
   auto Q_FULL = [&](int s) { return BAR(B_STAGE0 + s); };
   auto Q_EMPTY = [&](int s) { return BAR(B_STAGE0 + ST + s); };
   auto DO_FULL = [&](int s) { return BAR(B_STAGE0 + 2 * ST + s); };
-  auto DO_EMPTY = [&](int s) { return BAR(B_STAGE0 + 3 * ST + s); };
+  auto DO_EMPTY = [&](int s) { return BAR(B_STAGE0 + 2 * ST + SD + s); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gb + C::OFF_TMEM_SLOT);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -187,6 +192,8 @@ __global__ void __launch_bounds__(512, 1)
     for (int s = 0; s < ST; ++s) {
       mbar_init(Q_FULL(s), 1);
       mbar_init(Q_EMPTY(s), 1);
+    }
+    for (int s = 0; s < SD; ++s) {
       mbar_init(DO_FULL(s), 1);
       mbar_init(DO_EMPTY(s), 1);
     }
@@ -195,7 +202,19 @@ __global__ void __launch_bounds__(512, 1)
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
     prefetch_tmap(&tmDO);
+    prefetch_tmap(&tmC);
   }
+  // the constant tiles of the extra K-step: row r of the first holds bf16 ones in columns
+  // 0-2 (they meet the LSE terms), of the second in columns 3-5 (the Delta terms); the
+  // second 2 KiB of every column tile and of both constant tiles stay zero
+  for (int i = threadIdx.x; i < 128; i += blockDim.x) {
+    const uint32_t one = 0x3F80u;  // bf16 1.0
+    st_shared_v4(sb + C::OFF_ONES + i * 16, one | (one << 16), one, 0u, 0u);
+    st_shared_v4(sb + C::OFF_ONES + C::kColTile + i * 16, 0u, one << 16, one | (one << 16), 0u);
+  }
+  for (int i = threadIdx.x; i < 128 * (2 + ST); i += blockDim.x)
+    st_shared_v4(sb + C::OFF_ONES + (i >> 7) * C::kColTile + 2048 + (i & 127) * 16, 0u, 0u, 0u, 0u);
+  fence_proxy_async_smem();
   if (warp == 13) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
@@ -225,29 +244,31 @@ __global__ void __launch_bounds__(512, 1)
         }
         for (int t = 0; t < ch.w; ++t, ++it) {
           const int q = (int)(p.pairs[ch.z + t] & 0xffffu);
-          const int s = it % ST;
+          const int s = it % ST, sd = it % SD;
           const int row_q = ch.x * S + q * 128;
-          // Q with LSE and Delta (the softmax reads both until dS is done, which is
-          // before dK releases this stage); dO is released earlier, after dV
+          // Q with its column tile (LSE and Delta terms, read by S^T and dP^T, which
+          // finish before dK frees the stage); dO is released earlier, after dV
           if (it >= ST) wait(Q_EMPTY(s), ((it / ST) - 1) & 1);
-          mbar_expect_tx(Q_FULL(s), C::kTile + 1024);
+          mbar_expect_tx(Q_FULL(s), C::kTile + 2048);
 #pragma unroll
           for (int cb = 0; cb < D / 64; ++cb)
             tma_load_2d(sQ + s * C::kTile + cb * 16384, &tmQ, cb * 64, row_q, Q_FULL(s));
-          bulk_load(sb + C::OFF_LSE + s * 512, p.lse2 + row_q, 512, Q_FULL(s));
-          bulk_load(sb + C::OFF_DEL + s * 512, p.delta + row_q, 512, Q_FULL(s));
-          if (it >= ST) wait(DO_EMPTY(s), ((it / ST) - 1) & 1);
-          mbar_expect_tx(DO_FULL(s), C::kTile);
+          tma_load_2d(sb + C::OFF_COL + s * C::kColTile, &tmC, 0, row_q, Q_FULL(s));
+          if (it >= SD) wait(DO_EMPTY(sd), ((it / SD) - 1) & 1);
+          mbar_expect_tx(DO_FULL(sd), C::kTile);
 #pragma unroll
           for (int cb = 0; cb < D / 64; ++cb)
-            tma_load_2d(sDO + s * C::kTile + cb * 16384, &tmDO, cb * 64, row_q, DO_FULL(s));
+            tma_load_2d(sDO + sd * C::kTile + cb * 16384, &tmDO, cb * 64, row_q, DO_FULL(sd));
         }
       }
       // drain: every issued load has landed before the CTA can exit
       for (int s = 0; s < ST && s < it; ++s) {
         const int last_use = ((it - 1 - s) / ST) * ST + s;
         drain(Q_FULL(s), (last_use / ST) & 1);
-        drain(DO_FULL(s), (last_use / ST) & 1);
+      }
+      for (int s = 0; s < SD && s < it; ++s) {
+        const int last_use = ((it - 1 - s) / SD) * SD + s;
+        drain(DO_FULL(s), (last_use / SD) & 1);
       }
       if (cn > 0) drain(BAR(B_KV_FULL), (cn - 1) & 1);
     } else if (warp == 13 && lane == 0) {
@@ -263,6 +284,11 @@ __global__ void __launch_bounds__(512, 1)
       const uint32_t hi = sdesc_hi(1024);  // every operand here: 1 KiB between 8-row groups
       const uint32_t kK = sdesc_lo(sK, 16), kV = sdesc_lo(sV, 16);            // K-major
       const uint32_t mK = sdesc_lo(sK, 16384), mDS = sdesc_lo(sDSt, 16384);  // MN-major
+      // the extra K-step's operands: K-major core matrices without swizzle, 2 KiB
+      // between the two 8-column halves of the step, 128 bytes between 8-row groups
+      const uint32_t hi_none = sdesc_hi_none(128);
+      const uint32_t kOnesS = sdesc_lo_none(sb + C::OFF_ONES, 2048);
+      const uint32_t kOnesDP = sdesc_lo_none(sb + C::OFF_ONES + C::kColTile, 2048);
       int it = 0, cn = 0;
       for (int ci = cbeg; ci < cend; ++ci, ++cn) {
         const int cnt = p.chains[ci].w;
@@ -272,9 +298,9 @@ __global__ void __launch_bounds__(512, 1)
         // tile `it` and then issues S^T/dP^T of the next tile behind it
         for (int t = -1; t < cnt; ++t) {
           if (t >= 0) {
-            const int s = it % ST;
+            const int s = it % ST, sd = it % SD;
             const uint32_t mQ = sdesc_lo(sQ + s * C::kTile, 16384);
-            const uint32_t mDO = sdesc_lo(sDO + s * C::kTile, 16384);
+            const uint32_t mDO = sdesc_lo(sDO + sd * C::kTile, 16384);
             // dV += P^T dO : M = kv, N = D, K = q (A in TMEM, B MN-major), once P is packed
             wait(BAR(B_P_READY), it & 1);
             // the previous chain's dV/dK must have been read out before they restart
@@ -285,7 +311,7 @@ __global__ void __launch_bounds__(512, 1)
             for (int kk = 0; kk < 8; ++kk)
               tc_mma_ts_w(tDV, tS + 32 * (kk >> 1) + 8 * (kk & 1), mDO + kk * 128, hi, ID_KV,
                           kk > 0 ? 1u : acc0);
-            tc_commit(DO_EMPTY(s));
+            tc_commit(DO_EMPTY(sd));
             // dK += dS^T Q
             wait(BAR(B_DS_READY), it & 1);
             trace(it, 1);
@@ -315,9 +341,10 @@ __global__ void __launch_bounds__(512, 1)
           if (t + 1 < cnt) {
             // S^T = K Q^T of tile `it`: M = kv, N = q, K = D (both K-major), once dV/dK
             // of the previous tile have read packed P^T/dS^T out of these columns
-            const int s = it % ST;
+            const int s = it % ST, sd = it % SD;
             const uint32_t kQ = sdesc_lo(sQ + s * C::kTile, 16);
-            const uint32_t kDO = sdesc_lo(sDO + s * C::kTile, 16);
+            const uint32_t kDO = sdesc_lo(sDO + sd * C::kTile, 16);
+            const uint32_t kCol = sdesc_lo_none(sb + C::OFF_COL + s * C::kColTile, 2048);
             wait(Q_FULL(s), (it / ST) & 1);
             if (it > 0) wait(BAR(B_DVDK_DONE), (it - 1) & 1);
             tc_fence_after();
@@ -327,10 +354,12 @@ __global__ void __launch_bounds__(512, 1)
               const uint32_t off = (uint32_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
               tc_mma_ss_w(tS, kK + off, kQ + off, hi, ID_SS, kk > 0 ? 1u : 0u);
             }
+            // S'^T = S^T - LSE / scale, so the softmax takes P = 2^(scale log2e S')
+            tc_mma_ss_w(tS, kOnesS, kCol, hi_none, ID_SS, 1u);
             tc_commit(BAR(B_S_FULL));
             // dP^T = V dO^T; at D = 128 these columns hold dQp of the previous tile
             // until the reducers have drained it
-            wait(DO_FULL(s), (it / ST) & 1);
+            wait(DO_FULL(sd), (it / SD) & 1);
             if (C::kDqInDp && it > 0) wait(BAR(B_DQ_EMPTY0), (it - 1) & 1);
             tc_fence_after();
 #pragma unroll
@@ -338,6 +367,8 @@ __global__ void __launch_bounds__(512, 1)
               const uint32_t off = (uint32_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
               tc_mma_ss_w(tDP, kV + off, kDO + off, hi, ID_SS, kk > 0 ? 1u : 0u);
             }
+            // dP'^T = dP^T - Delta, so the softmax forms dS = P dP'
+            tc_mma_ss_w(tDP, kOnesDP, kCol, hi_none, ID_SS, 1u);
             tc_commit(BAR(B_DP_FULL));
           }
         }
@@ -364,15 +395,11 @@ __global__ void __launch_bounds__(512, 1)
       const int4 ch = p.chains[ci];
       for (int t = 0; t < ch.w; ++t, ++it) {
         const int q = (int)(p.pairs[ch.z + t] & 0xffffu);
-        const int s = it % ST;
         wait(BAR(B_S_FULL), it & 1);
-        wait(Q_FULL(s), (it / ST) & 1);
         if (threadIdx.x == 0) trace(it, 3);
         tc_fence_after();
         // causal: on the diagonal tile Q column qc sees KV row r only if qc >= r
         const int lim_c = (p.causal && q == ch.y) ? r : -1;
-        const float* lse_t = lse_s + s * 128;
-        const float* del_t = del_s + s * 128;
 #pragma unroll 1
         for (int cc = 0; cc < 2; ++cc) {
           const int c = half * 2 + cc;  // 32-column chunk of the tile
@@ -384,9 +411,9 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
               const int qc = 32 * c + j;
-              const float2 l2 = *reinterpret_cast<const float2*>(lse_t + qc);
-              float p0 = ex2_approx(fmaf(__uint_as_float(sv[j]), sl2, -l2.x));
-              float p1 = ex2_approx(fmaf(__uint_as_float(sv[j + 1]), sl2, -l2.y));
+              // S'^T already has LSE / scale taken off by the tensor core
+              float p0 = ex2_approx(__uint_as_float(sv[j]) * sl2);
+              float p1 = ex2_approx(__uint_as_float(sv[j + 1]) * sl2);
               if constexpr (decltype(masked)::value) {
                 if (qc < lim_c) p0 = 0.f;
                 if (qc + 1 < lim_c) p1 = 0.f;
@@ -416,11 +443,10 @@ __global__ void __launch_bounds__(512, 1)
           uint32_t dk[16];
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
-            const float2 d2 = *reinterpret_cast<const float2*>(del_t + 32 * c + j);
+            // dP'^T already has Delta taken off by the tensor core
             const float p0 = __uint_as_float(pk[j >> 1] << 16);
             const float p1 = __uint_as_float(pk[j >> 1] & 0xffff0000u);
-            dk[j >> 1] = pack_bf16x2(p0 * (__uint_as_float(dv[j]) - d2.x),
-                                     p1 * (__uint_as_float(dv[j + 1]) - d2.y));
+            dk[j >> 1] = pack_bf16x2(p0 * __uint_as_float(dv[j]), p1 * __uint_as_float(dv[j + 1]));
           }
           // dS^T into the last 16 columns of chunk c, and to shared memory
           // (128-byte swizzle, 64-column block `half`)
@@ -445,7 +471,7 @@ __global__ void __launch_bounds__(512, 1)
     const int r = quarter * 32 + lane;  // Q row for dQ, KV row for dK/dV
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     constexpr int NV = D / 4;           // float4 per row
-    constexpr int G = 16;               // loads in flight per group
+    constexpr int G = 24;               // loads in flight per group
     int it = 0, cn = 0;
     for (int ci = cbeg; ci < cend; ++ci, ++cn) {
       const int4 ch = p.chains[ci];

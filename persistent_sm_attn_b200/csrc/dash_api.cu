@@ -47,7 +47,7 @@ struct Workspace {
   size_t acc_bytes = 0;
   uint32_t* tickets = nullptr;
   size_t tk_bytes = 0;
-  float* rowbuf = nullptr;  // lse2 then delta, each rows_cap floats
+  float* rowbuf = nullptr;  // per-row column terms of the backward, 16 bytes per row
   size_t rows_cap = 0;
   unsigned* err = nullptr;   // [0] error word, [1] per-launch abort flag
 };
@@ -105,9 +105,9 @@ int get_workspace(int dev, void* stream, size_t acc_bytes, size_t tk_bytes, size
   int rc;
   if ((rc = grow(reinterpret_cast<void**>(&w.acc), &w.acc_bytes, acc_bytes))) return rc;
   if ((rc = grow(reinterpret_cast<void**>(&w.tickets), &w.tk_bytes, tk_bytes))) return rc;
-  size_t rb = w.rows_cap * 2 * sizeof(float);
+  size_t rb = w.rows_cap * 16;
   if (rows > w.rows_cap) {
-    if ((rc = grow(reinterpret_cast<void**>(&w.rowbuf), &rb, rows * 2 * sizeof(float)))) return rc;
+    if ((rc = grow(reinterpret_cast<void**>(&w.rowbuf), &rb, rows * 16))) return rc;
     w.rows_cap = rows;
   }
   if (!w.err) {
@@ -222,6 +222,21 @@ int make_tmap(CUtensorMap* m, const void* base, long long rows, int D, int box_r
   return r == CUDA_SUCCESS ? DASH_OK : DASH_ERR_CUDA;
 }
 
+// [rows][8] bf16 column terms viewed with an 8 x 128 box, no swizzle: the box lands as
+// 8-row x 16-byte core matrices, the layout of the backward's extra K-step operand.
+int make_tmap_cols(CUtensorMap* m, const void* base, long long rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return DASH_ERR_CUDA;
+  cuuint64_t dims[2] = {8, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {16};
+  cuuint32_t box[2] = {8, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DASH_OK : DASH_ERR_CUDA;
+}
+
 // ------------------------------------------------------------------ helpers
 bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -284,22 +299,22 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
                             (size_t)rows, &ws)))
       return rc;
   }
-  CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tq, tk, tv, tdo, tc;
   if ((rc = make_tmap(&tq, q, rows, D, C::kQRows)) ||
       (rc = make_tmap(&tk, k, rows, D, C::kKVRows)) ||
       (rc = make_tmap(&tv, v, rows, D, C::kKVRows)) ||
-      (rc = make_tmap(&tdo, dout, rows, D, C::kQRows)))
+      (rc = make_tmap(&tdo, dout, rows, D, C::kQRows)) ||
+      (rc = make_tmap_cols(&tc, ws->rowbuf, rows)))
     return rc;
-  float* lse2 = ws->rowbuf;
-  float* delta = ws->rowbuf + ws->rows_cap;
+  const float scale = 1.0f / sqrtf((float)D);
   std::array<cudaEvent_t, 4> ev{};
   if (!prof_record(0, &ev, stream)) return DASH_ERR_CUDA;
   {
     const long long threads = rows * (D / 8);
     const int blocks = (int)((threads + 255) / 256);
     dash::dash_delta_kernel<D><<<blocks, 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, delta,
-        lse2, rows);
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse,
+        reinterpret_cast<uint4*>(ws->rowbuf), rows, 1.0f / scale);
   }
   DASH_CUDA(cudaMemsetAsync(ws->err + 1, 0, sizeof(unsigned), stream));
   if (kAtomic) {
@@ -310,8 +325,6 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
                               stream));
   }
   BwdParams p;
-  p.lse2 = lse2;
-  p.delta = delta;
   p.cta_off = tab->cta_off;
   p.chains = tab->chains;
   p.pairs = tab->pairs;
@@ -325,7 +338,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   p.S = S;
   p.N = N;
   p.causal = causal;
-  p.scale = 1.0f / sqrtf((float)D);
+  p.scale = scale;
   p.scale_log2 = p.scale * 1.4426950408889634f;
   p.spin_ns = (unsigned long long)spin_us() * 1000ull;
   p.trace = trace;
@@ -348,9 +361,9 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
     cudaFuncAttributes fa;
     DASH_CUDA(cudaFuncGetAttributes(&fa, kt));
     if (fa.numRegs != C::kLaunchRegs) return DASH_ERR_UNSUPPORTED;
-    DASH_CUDA(cudaLaunchKernelEx(&cfg, kt, tq, tk, tv, tdo, p));
+    DASH_CUDA(cudaLaunchKernelEx(&cfg, kt, tq, tk, tv, tdo, tc, p));
   } else {
-    DASH_CUDA(cudaLaunchKernelEx(&cfg, dash::dash_bwd_kernel<D, kAtomic>, tq, tk, tv, tdo, p));
+    DASH_CUDA(cudaLaunchKernelEx(&cfg, dash::dash_bwd_kernel<D, kAtomic>, tq, tk, tv, tdo, tc, p));
   }
   if (!prof_record(2, &ev, stream)) return DASH_ERR_CUDA;
   if (kAtomic) {

@@ -64,6 +64,20 @@ EncodeTiledFn noalloc_encode_fn() {
   return fn;
 }
 
+// [rows][8] bf16 column terms: an 8 x 128 box without swizzle (core-matrix layout).
+int noalloc_tmap_cols(CUtensorMap* m, const void* base, long long rows) {
+  EncodeTiledFn fn = noalloc_encode_fn();
+  if (!fn) return DASH_ERR_CUDA;
+  cuuint64_t dims[2] = {8, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {16};
+  cuuint32_t box[2] = {8, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DASH_OK : DASH_ERR_CUDA;
+}
+
 int noalloc_tmap(CUtensorMap* m, const void* base, long long rows, int D, int box_rows) {
   EncodeTiledFn fn = noalloc_encode_fn();
   if (!fn) return DASH_ERR_CUDA;
@@ -132,7 +146,7 @@ unsigned long long noalloc_spin_ns() {
 size_t fixed_scratch(long long rows, int D, long long blocks) {
   return 256                                         // error word + abort flag
          + align256((size_t)blocks * 4)              // tickets
-         + 2 * align256((size_t)rows * 4)            // scaled LSE, Delta
+         + align256((size_t)rows * 16)               // per-row column terms (LSE, Delta)
          + align256(2 * (size_t)rows * D * 4);       // fp32 dQ accumulators (two per block)
 }
 
@@ -151,10 +165,8 @@ int noalloc_launch(const void* q, const void* k, const void* v, const void* o, c
   size_t off = 256;
   uint32_t* tickets = reinterpret_cast<uint32_t*>(p0 + off);
   off += align256((size_t)blocks * 4);
-  float* lse2 = reinterpret_cast<float*>(p0 + off);
-  off += align256((size_t)rows * 4);
-  float* delta = reinterpret_cast<float*>(p0 + off);
-  off += align256((size_t)rows * 4);
+  uint4* cols = reinterpret_cast<uint4*>(p0 + off);
+  off += align256((size_t)rows * 16);
   float* acc = reinterpret_cast<float*>(p0 + off);
   off += align256(2 * (size_t)rows * D * 4);
   // the schedule table, built and checked on the host, then copied in
@@ -178,13 +190,15 @@ int noalloc_launch(const void* q, const void* k, const void* v, const void* o, c
       return DASH_ERR_CUDA;
     std::memcpy(st->table_key, key, sizeof(key));
   }
-  CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tq, tk, tv, tdo, tc;
   int rc;
   if ((rc = noalloc_tmap(&tq, q, rows, D, C::kQRows)) ||
       (rc = noalloc_tmap(&tk, k, rows, D, C::kKVRows)) ||
       (rc = noalloc_tmap(&tv, v, rows, D, C::kKVRows)) ||
-      (rc = noalloc_tmap(&tdo, dout, rows, D, C::kQRows)))
+      (rc = noalloc_tmap(&tdo, dout, rows, D, C::kQRows)) ||
+      (rc = noalloc_tmap_cols(&tc, cols, rows)))
     return rc;
+  const float scale = 1.0f / sqrtf((float)D);
   // the array keeps the previous call's contents: clear what must start at zero
   if (cudaMemsetAsync(err, 0, 2 * sizeof(unsigned), stream) != cudaSuccess) return DASH_ERR_CUDA;
   if (kAtomic) {
@@ -196,12 +210,10 @@ int noalloc_launch(const void* q, const void* k, const void* v, const void* o, c
   {
     const long long threads = rows * (D / 8);
     dash::dash_delta_kernel<D><<<(int)((threads + 255) / 256), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, delta,
-        lse2, rows);
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, cols,
+        rows, 1.0f / scale);
   }
   dash::BwdParams p;
-  p.lse2 = lse2;
-  p.delta = delta;
   p.cta_off = reinterpret_cast<const int*>(p0 + off_cta);
   p.chains = reinterpret_cast<const int4*>(p0 + off_chain);
   p.pairs = reinterpret_cast<const uint32_t*>(p0 + off_pair);
@@ -215,7 +227,7 @@ int noalloc_launch(const void* q, const void* k, const void* v, const void* o, c
   p.S = S;
   p.N = N;
   p.causal = causal;
-  p.scale = 1.0f / sqrtf((float)D);
+  p.scale = scale;
   p.scale_log2 = p.scale * 1.4426950408889634f;
   p.spin_ns = noalloc_spin_ns();
   cudaLaunchConfig_t cfg = {};
@@ -228,7 +240,7 @@ int noalloc_launch(const void* q, const void* k, const void* v, const void* o, c
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, dash::dash_bwd_kernel<D, kAtomic>, tq, tk, tv, tdo, p) !=
+  if (cudaLaunchKernelEx(&cfg, dash::dash_bwd_kernel<D, kAtomic>, tq, tk, tv, tdo, tc, p) !=
       cudaSuccess)
     return DASH_ERR_CUDA;
   if (kAtomic) {

@@ -209,6 +209,16 @@ static_assert((((uint64_t)sdesc_hi(1024) << 32) | sdesc_lo(0x12340u, 16384)) ==
                   sdesc_sw128(0x12340u, 16384, 1024),
               "descriptor words");
 
+// Descriptor words of a K-major operand without swizzle (layout type 0): 8-row x
+// 16-byte core matrices, `lbo` bytes between core matrices along K, `sbo` bytes
+// between core matrices along M or N.
+__host__ __device__ constexpr uint32_t sdesc_lo_none(uint32_t saddr, uint32_t lbo) {
+  return ((saddr & 0x3FFFFu) >> 4) | (((lbo >> 4) & 0x3FFFu) << 16);
+}
+__host__ __device__ constexpr uint32_t sdesc_hi_none(uint32_t sbo) {
+  return ((sbo >> 4) & 0x3FFFu) | (1u << 14);
+}
+
 // MMA issue with descriptors given as words: the issuing thread does one add
 // per operand per MMA, which keeps the single-thread issue stream short.
 __device__ __forceinline__ void tc_mma_ss_w(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
