@@ -35,7 +35,7 @@
  *     errors are returned at once; errors found on the device (a spin wait
  *     that ran out) are reported by dash_attn_sync_status().
  *   - The library owns its workspace (fp32 dQ accumulators, tickets, the
- *     per-row Delta and scaled LSE, an error word) and caches it per
+ *     per-row LSE and Delta terms, an error word) and caches it per
  *     (device, stream); schedule tables are cached per shape.  Calls on
  *     different streams use different workspaces.  Workspace memory is
  *     released by dash_release_workspace().
@@ -167,7 +167,7 @@ int dash_release_workspace(void);
  * library holds until the process exits.  The call never calls cudaMalloc,
  * cudaFree or an allocating library routine.
  *   - Size limit: the array must hold the two fp32 dQ accumulators per block
- *     (2*B*H*S*D*4 bytes), the per-row Delta and scaled LSE (2*B*H*S*4), two
+ *     (2*B*H*S*D*4 bytes), 16 bytes of LSE and Delta terms per row (B*H*S*16), two
  *     tickets per 128-row dQ block and the schedule table; larger calls return
  *     DASH_ERR_OOM without touching the device.
  *   - Set-up: the first call on a device (with that device current) looks up

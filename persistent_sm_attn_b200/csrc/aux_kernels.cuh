@@ -30,39 +30,77 @@ __device__ __forceinline__ void split3_bf16(float x, __nv_bfloat16* part) {
   part[2] = __float2bfloat16_rn(r1 - __bfloat162float(part[1]));
 }
 
-// One group of D/8 lanes per row; 16-byte loads of O and dO.  Writes cols[row] =
+// One group of L = D/8 lanes per row; 16-byte loads of O and dO.  Writes cols[row] =
 // 8 bf16: -(LSE_row / scale) in three parts, -Delta_row in three parts, two zeros.
 // The backward adds them to S^T and dP^T through one extra K-step of each product
 // (against constant ones), so S' = S - LSE/scale and dP' = dP - Delta.
+// Each thread takes kDeltaRows rows one grid-width apart and issues all their loads
+// before any arithmetic, so a grid of a few CTAs per SM keeps enough bytes in flight
+// to stream HBM.  The same launch clears the words the backward needs at zero:
+// `clear[0..n_clear)` (error words, block 0) and `tickets[0..n_tickets)`.
+constexpr int kDeltaRows = 4;
 template <int D>
 __global__ void __launch_bounds__(256) dash_delta_kernel(const __nv_bfloat16* __restrict__ o,
                                                          const __nv_bfloat16* __restrict__ dout,
                                                          const float* __restrict__ lse,
                                                          uint4* __restrict__ cols, long long rows,
-                                                         float inv_scale) {
+                                                         float inv_scale,
+                                                         uint32_t* __restrict__ tickets,
+                                                         long long n_tickets,
+                                                         unsigned* __restrict__ clear,
+                                                         int n_clear) {
   constexpr int L = D / 8;  // lanes per row
+  static_assert(32 % L == 0, "a warp holds whole rows");
+  const long long nthreads = (long long)gridDim.x * blockDim.x;
   const long long gt = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  const long long row = gt / L;
+  if (blockIdx.x == 0 && threadIdx.x < n_clear) clear[threadIdx.x] = 0u;
+  for (long long i = gt; i < n_tickets; i += nthreads) tickets[i] = 0u;
+  const long long per_pass = nthreads / L;  // rows one pass covers (blockDim is a multiple of 32)
   const int sub = (int)(gt % L);
-  float acc = 0.f;
-  if (row < rows) {
-    const uint4 ov = reinterpret_cast<const uint4*>(o + row * D)[sub];
-    const uint4 dv = reinterpret_cast<const uint4*>(dout + row * D)[sub];
-    float fo[8], fd[8];
-    bf16x8_to_f32(ov, fo);
-    bf16x8_to_f32(dv, fd);
+  // the loop bound is taken from the warp's first row, so every lane of a warp runs the
+  // same iterations and the shuffles below see full warps
+  const long long row0 = gt / L, warp_row0 = (gt & ~31LL) / L;
+  for (long long base = 0; warp_row0 + base < rows; base += kDeltaRows * per_pass) {
+    uint4 ov[kDeltaRows], dv[kDeltaRows];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc = fmaf(fo[i], fd[i], acc);
-  }
+    for (int u = 0; u < kDeltaRows; ++u) {
+      const long long row = row0 + base + u * per_pass;
+      if (row < rows) {
+        ov[u] = reinterpret_cast<const uint4*>(o + row * D)[sub];
+        dv[u] = reinterpret_cast<const uint4*>(dout + row * D)[sub];
+      } else {
+        ov[u] = make_uint4(0u, 0u, 0u, 0u);
+        dv[u] = ov[u];
+      }
+    }
 #pragma unroll
-  for (int m = L / 2; m >= 1; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
-  if (row < rows && sub == 0) {
-    __align__(16) __nv_bfloat16 part[8];
-    split3_bf16(-lse[row] * inv_scale, part);
-    split3_bf16(-acc, part + 3);
-    part[6] = part[7] = __float2bfloat16_rn(0.f);
-    cols[row] = *reinterpret_cast<const uint4*>(part);
+    for (int u = 0; u < kDeltaRows; ++u) {
+      const long long row = row0 + base + u * per_pass;
+      float fo[8], fd[8], acc = 0.f;
+      bf16x8_to_f32(ov[u], fo);
+      bf16x8_to_f32(dv[u], fd);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc = fmaf(fo[i], fd[i], acc);
+#pragma unroll
+      for (int m = L / 2; m >= 1; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+      if (row < rows && sub == 0) {
+        __align__(16) __nv_bfloat16 part[8];
+        split3_bf16(-lse[row] * inv_scale, part);
+        split3_bf16(-acc, part + 3);
+        part[6] = part[7] = __float2bfloat16_rn(0.f);
+        cols[row] = *reinterpret_cast<const uint4*>(part);
+      }
+    }
   }
+}
+
+// Grid of the Delta kernel: enough CTAs for kDeltaRows rows per thread, at most four
+// per SM (what its 64 registers a thread leave resident), so it runs as one wave.
+template <int D>
+inline int delta_grid(long long rows, int num_sms) {
+  const long long need = (rows * (D / 8) + 256LL * kDeltaRows - 1) / (256LL * kDeltaRows);
+  const long long cap = 4LL * (num_sms > 0 ? num_sms : 1);
+  return (int)(need < 1 ? 1 : (need < cap ? need : cap));
 }
 
 // fp32 accumulator -> bf16 dQ.  One accumulator block per 128-row Q tile,

@@ -526,20 +526,24 @@ __global__ void __launch_bounds__(512, 1)
             }
             __syncwarp();
           };
-          // a = acc + a over this thread's slots, G loads in flight before their adds
+          // a = acc + a over this thread's NV slots, up to G loads in flight before their
+          // adds (the last group holds the remaining NV mod G slots)
           auto add_from = [&](const float4* src) {
 #pragma unroll
             for (int g0 = 0; g0 < NV; g0 += G) {
               float4 old[G];
 #pragma unroll
-              for (int j = 0; j < G; ++j) old[j] = ld_cg_f4(src + (g0 + j) * 128 + r);
+              for (int j = 0; j < G; ++j)
+                if (g0 + j < NV) old[j] = ld_cg_f4(src + (g0 + j) * 128 + r);
 #pragma unroll
               for (int j = 0; j < G; ++j) {
-                float* x = a + 4 * (g0 + j);
-                x[0] = old[j].x + x[0];
-                x[1] = old[j].y + x[1];
-                x[2] = old[j].z + x[2];
-                x[3] = old[j].w + x[3];
+                if (g0 + j < NV) {
+                  float* x = a + 4 * (g0 + j);
+                  x[0] = old[j].x + x[0];
+                  x[1] = old[j].y + x[1];
+                  x[2] = old[j].z + x[2];
+                  x[3] = old[j].w + x[3];
+                }
               }
             }
           };

@@ -309,21 +309,13 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   const float scale = 1.0f / sqrtf((float)D);
   std::array<cudaEvent_t, 4> ev{};
   if (!prof_record(0, &ev, stream)) return DASH_ERR_CUDA;
-  {
-    const long long threads = rows * (D / 8);
-    const int blocks = (int)((threads + 255) / 256);
-    dash::dash_delta_kernel<D><<<blocks, 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse,
-        reinterpret_cast<uint4*>(ws->rowbuf), rows, 1.0f / scale);
-  }
-  DASH_CUDA(cudaMemsetAsync(ws->err + 1, 0, sizeof(unsigned), stream));
-  if (kAtomic) {
-    DASH_CUDA(cudaMemsetAsync(ws->acc, 0, (size_t)rows * D * sizeof(float), stream));
-  } else {
-    DASH_CUDA(cudaMemsetAsync(ws->tickets, 0,
-                              (size_t)dash::dq_units<D>((long long)B * H * N) * sizeof(uint32_t),
-                              stream));
-  }
+  // Delta and the column terms; the same launch clears the abort flag and, on the
+  // deterministic path, the tickets
+  dash::dash_delta_kernel<D><<<dash::delta_grid<D>(rows, ctas), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse,
+      reinterpret_cast<uint4*>(ws->rowbuf), rows, 1.0f / scale, ws->tickets,
+      kAtomic ? 0LL : dash::dq_units<D>((long long)B * H * N), ws->err + 1, 1);
+  if (kAtomic) DASH_CUDA(cudaMemsetAsync(ws->acc, 0, (size_t)rows * D * sizeof(float), stream));
   BwdParams p;
   p.cta_off = tab->cta_off;
   p.chains = tab->chains;

@@ -199,20 +199,14 @@ int noalloc_launch(const void* q, const void* k, const void* v, const void* o, c
       (rc = noalloc_tmap_cols(&tc, cols, rows)))
     return rc;
   const float scale = 1.0f / sqrtf((float)D);
-  // the array keeps the previous call's contents: clear what must start at zero
-  if (cudaMemsetAsync(err, 0, 2 * sizeof(unsigned), stream) != cudaSuccess) return DASH_ERR_CUDA;
-  if (kAtomic) {
-    if (cudaMemsetAsync(acc, 0, (size_t)rows * D * 4, stream) != cudaSuccess) return DASH_ERR_CUDA;
-  } else {
-    if (cudaMemsetAsync(tickets, 0, (size_t)blocks * 4, stream) != cudaSuccess)
-      return DASH_ERR_CUDA;
-  }
-  {
-    const long long threads = rows * (D / 8);
-    dash::dash_delta_kernel<D><<<(int)((threads + 255) / 256), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, cols,
-        rows, 1.0f / scale);
-  }
+  // The array keeps the previous call's contents: the Delta launch clears the error
+  // word, the abort flag and (deterministic path) the tickets; the atomic variant's
+  // accumulator is cleared here.
+  if (kAtomic && cudaMemsetAsync(acc, 0, (size_t)rows * D * 4, stream) != cudaSuccess)
+    return DASH_ERR_CUDA;
+  dash::dash_delta_kernel<D><<<dash::delta_grid<D>(rows, ctas), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, cols,
+      rows, 1.0f / scale, tickets, kAtomic ? 0LL : blocks, err, 2);
   dash::BwdParams p;
   p.cta_off = reinterpret_cast<const int*>(p0 + off_cta);
   p.chains = reinterpret_cast<const int4*>(p0 + off_chain);
