@@ -8,8 +8,9 @@
 //   dP^T = V_j dO_i^T                 tcgen05.mma (smem x smem) -> TMEM [128, 256)
 //   P^T  = exp(scale S^T - LSE_i)     softmax warps, packed bf16 back into S^T's columns
 //   dV_j += P^T dO_i                  tcgen05.mma with A in TMEM, as soon as P^T is packed
-//   dS^T = P^T (dP^T - Delta_i)       softmax warps, into S^T's columns and shared memory
-//   dK_j += dS^T Q_i                  tcgen05.mma with A in TMEM
+//   dS^T = P^T (dP^T - Delta_i)       softmax warps, into shared memory (and at D = 128
+//                                     into S^T's columns)
+//   dK_j += dS^T Q_i                  tcgen05.mma, A in TMEM (D = 128) or smem (D = 64)
 //   dQp  = dS K_j                     tcgen05.mma (smem x smem) -> TMEM
 //   ordered reduction of dQp into an fp32 accumulator of block (b,h,i): wait
 //   until the accumulator's ticket says it is this pair's turn, add with plain
@@ -19,11 +20,13 @@
 //   so a contributor waits on the one two positions ahead of it; the last
 //   contributor adds the two sums, rounds once to bf16 and writes dQ.
 //
-// The MMA issuer queues S^T and dP^T of the next tile right behind dK and dQp,
-// so the exponentials of tile i+1 run while the tensor pipe finishes tile i,
-// and dV of tile i+1 runs while its dS is formed.  Taking P^T and dS^T from
-// TMEM keeps two of the five products off the shared-memory read path, which
-// bounds the 1-CTA tensor cores here.
+// D = 128: the MMA issuer queues S^T and dP^T of the next tile right behind dK
+// and dQp, so the exponentials of tile i+1 run while the tensor pipe finishes
+// tile i, and dV of tile i+1 runs while its dS is formed.  Taking P^T and dS^T
+// from TMEM keeps two of the five products off the shared-memory read path.
+// D = 64: TMEM has room for two S^T buffers, so S^T runs two tiles ahead; dK
+// reads dS^T from shared memory, which frees a tile's S^T buffer as soon as dV
+// and the softmax are done with its P^T, and the tile's dQp goes there.
 //
 // Warp roles (512 threads, four warpgroups):
 //   WG0, WG1  softmax / dS; WG0 owns Q columns 0-63, WG1 columns 64-127 (96 registers)
@@ -31,11 +34,13 @@
 //   WG3       warp 12 TMA producer, warp 13 MMA issuer and TMEM owner (96 registers)
 // TMEM lane quarter of a warp is (warp % 4), so each warpgroup covers the 128 lanes.
 //
-// TMEM columns (512): S^T [0,128) then packed P^T/dS^T, dP^T [128,256),
-// dV [256,256+D), dK after it; dQp in the dP^T columns (D = 128) or in two
-// buffers [384,448) [448,512) (D = 64).  Packed layout after the softmax: the
-// 32 fp32 columns of chunk c (Q columns 32c..32c+31) hold P^T of those columns
-// in 32c..32c+15 and dS^T in 32c+16..32c+31, two bf16 per column.
+// TMEM columns (512).  D = 128: S^T [0,128) then packed P^T/dS^T, dP^T
+// [128,256) then dQp, dV [256,384), dK [384,512).  D = 64: S^T of even tiles
+// [0,128), of odd tiles [128,256), each then packed P^T and then that tile's dQp
+// in its first 64 columns; dP^T [256,384), dV [384,448), dK [448,512).  Packed
+// layout after the softmax: the 32 fp32 columns of chunk c (Q columns
+// 32c..32c+31) hold P^T of those columns in 32c..32c+15 and (D = 128) dS^T in
+// 32c+16..32c+31, two bf16 per column.
 //
 // Shared-memory tiles are [128 rows][D] bf16 stored as D/64 column blocks of
 // 128 rows x 128 bytes with the 128-byte swizzle (the layout a TMA load with
@@ -104,14 +109,21 @@ struct BwdCfg {
   static constexpr int OFF_DO = OFF_Q + kStagesQ * kTile;
   static constexpr int OFF_DST = OFF_DO + kStagesDO * kTile;  // dS^T [128 kv][128 q]
   static constexpr int OFF_BAR = OFF_DST + 32768;
-  static constexpr int kBars = 16 + 2 * kStagesQ + 2 * kStagesDO;
+  static constexpr int kBars = 18 + 2 * kStagesQ + 2 * kStagesDO;
   static constexpr int OFF_TMEM_SLOT = OFF_BAR + kBars * 8;
   // The swizzled tiles need a 1 KiB aligned base; the kernel checks it.
   static constexpr int kSmemBytes = OFF_TMEM_SLOT + 16;
   static_assert(kSmemBytes <= 232448, "shared memory per block exceeded");
-  static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 256 + D;
-  static constexpr uint32_t TM_DQ = (D == 128) ? 128 : 384;
-  static constexpr bool kDqInDp = (D == 128);  // dQp reuses dP^T's columns
+  // TMEM columns.  D = 128: S^T [0,128), dP^T [128,256), dV, dK; dQp reuses dP^T's
+  // columns and dK takes dS^T from S^T's columns.  D = 64: S^T has two buffers [0,128)
+  // and [128,256) (the MMA issuer runs two tiles ahead on S^T), dP^T [256,384), dV, dK;
+  // dK takes dS^T from shared memory, so a tile's S^T buffer is free once dV and the
+  // softmax are done with its P^T, and the tile's dQp goes into its first 64 columns.
+  static constexpr bool kSDouble = (D == 64);
+  static constexpr uint32_t TM_S = 0, TM_DP = kSDouble ? 256 : 128;
+  static constexpr uint32_t TM_DV = TM_DP + 128, TM_DK = TM_DV + D;
+  static_assert(TM_DK + D == 512, "TMEM columns");
+  static constexpr bool kDqInDp = !kSDouble;
 };
 
 // Number of dQ accumulation chains (tickets, and fp32 accumulators of 128 x D):
@@ -125,7 +137,8 @@ constexpr long long dq_units(long long bh_times_n) {
 enum {
   B_KV_FULL = 0, B_KV_EMPTY, B_S_FULL, B_DP_FULL, B_DS_READY, B_DS_FREE, B_DQ_FULL0, B_DQ_FULL1,
   B_DQ_EMPTY0, B_DQ_EMPTY1, B_DVDK_DONE, B_DKDV_FULL, B_DKDV_EMPTY, B_FINAL, B_P_READY,
-  B_STAGE0 = 16
+  B_S_FULL1, B_P_READY1, B_DV_DONE,  // the second S^T buffer and dV done (D = 64)
+  B_STAGE0 = 18
 };
 
 // kTrace: record %globaltimer per pair of this CTA: 0 S^T issued, 1 softmax
@@ -158,6 +171,17 @@ __global__ void __launch_bounds__(512, 1)
   auto Q_EMPTY = [&](int s) { return BAR(B_STAGE0 + ST + s); };
   auto DO_FULL = [&](int s) { return BAR(B_STAGE0 + 2 * ST + s); };
   auto DO_EMPTY = [&](int s) { return BAR(B_STAGE0 + 2 * ST + SD + s); };
+  // Per-tile buffers: tile i's S^T columns and the barriers reporting them full and P^T
+  // packed; its dQp columns and the barriers reporting them full and drained.  With two
+  // buffers (D = 64) each barrier serves every other tile, so its phase parity is
+  // (i / 2) mod 2.
+  auto s_col = [&](int i) { return C::kSDouble ? 128u * (uint32_t)(i & 1) : 0u; };
+  auto S_FULL = [&](int i) { return BAR(C::kSDouble && (i & 1) ? B_S_FULL1 : B_S_FULL); };
+  auto P_READY = [&](int i) { return BAR(C::kSDouble && (i & 1) ? B_P_READY1 : B_P_READY); };
+  auto s_phase = [&](int i) { return C::kSDouble ? (i >> 1) & 1 : i & 1; };
+  auto dq_col = [&](int i) { return C::kDqInDp ? C::TM_DP : 128u * (uint32_t)(i & 1); };
+  auto DQ_FULL = [&](int i) { return BAR(C::kDqInDp ? B_DQ_FULL0 : B_DQ_FULL0 + (i & 1)); };
+  auto DQ_EMPTY = [&](int i) { return BAR(C::kDqInDp ? B_DQ_EMPTY0 : B_DQ_EMPTY0 + (i & 1)); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gb + C::OFF_TMEM_SLOT);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -177,6 +201,8 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(BAR(B_KV_FULL), 1);
     mbar_init(BAR(B_KV_EMPTY), 1);
     mbar_init(BAR(B_S_FULL), 1);
+    mbar_init(BAR(B_S_FULL1), 1);
+    mbar_init(BAR(B_DV_DONE), 1);
     mbar_init(BAR(B_DP_FULL), 1);
     mbar_init(BAR(B_DS_READY), 256);
     mbar_init(BAR(B_DS_FREE), 1);
@@ -189,6 +215,7 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(BAR(B_DKDV_EMPTY), 128);
     mbar_init(BAR(B_FINAL), 1);
     mbar_init(BAR(B_P_READY), 256);
+    mbar_init(BAR(B_P_READY1), 256);
     for (int s = 0; s < ST; ++s) {
       mbar_init(Q_FULL(s), 1);
       mbar_init(Q_EMPTY(s), 1);
@@ -289,90 +316,185 @@ __global__ void __launch_bounds__(512, 1)
       const uint32_t hi_none = sdesc_hi_none(128);
       const uint32_t kOnesS = sdesc_lo_none(sb + C::OFF_ONES, 2048);
       const uint32_t kOnesDP = sdesc_lo_none(sb + C::OFF_ONES + C::kColTile, 2048);
-      int it = 0, cn = 0;
-      for (int ci = cbeg; ci < cend; ++ci, ++cn) {
-        const int cnt = p.chains[ci].w;
-        wait(BAR(B_KV_FULL), cn & 1);
-        tc_fence_after();
-        // t = -1 only issues the chain's first S^T/dP^T; each later step finishes
-        // tile `it` and then issues S^T/dP^T of the next tile behind it
-        for (int t = -1; t < cnt; ++t) {
-          if (t >= 0) {
+      if constexpr (C::kSDouble) {
+        const uint32_t kDS = sdesc_lo(sDSt, 16);  // dS^T read K-major (M = kv, K = q) by dK
+        // S'^T = K Q^T - LSE/scale of tile i into its buffer, once the reducers have
+        // drained the dQp that tile i - 2 left there
+        auto issue_s = [&](int i) {
+          const int s = i % ST;
+          const uint32_t kQ = sdesc_lo(sQ + s * C::kTile, 16);
+          const uint32_t kCol = sdesc_lo_none(sb + C::OFF_COL + s * C::kColTile, 2048);
+          const uint32_t tSi = tS + s_col(i);
+          wait(Q_FULL(s), (i / ST) & 1);
+          if (i >= 2) wait(DQ_EMPTY(i - 2), s_phase(i - 2));
+          tc_fence_after();
+          trace(i, 0);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (uint32_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+            tc_mma_ss_w(tSi, kK + off, kQ + off, hi, ID_SS, kk > 0 ? 1u : 0u);
+          }
+          tc_mma_ss_w(tSi, kOnesS, kCol, hi_none, ID_SS, 1u);  // - LSE / scale
+          tc_commit(S_FULL(i));
+        };
+        // dP'^T = V dO^T - Delta of tile i (the issuer has already seen the softmax
+        // finish with tile i - 1's dP'^T)
+        auto issue_dp = [&](int i) {
+          const int s = i % ST, sd = i % SD;
+          const uint32_t kDO = sdesc_lo(sDO + sd * C::kTile, 16);
+          const uint32_t kCol = sdesc_lo_none(sb + C::OFF_COL + s * C::kColTile, 2048);
+          wait(DO_FULL(sd), (i / SD) & 1);
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (uint32_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+            tc_mma_ss_w(tDP, kV + off, kDO + off, hi, ID_SS, kk > 0 ? 1u : 0u);
+          }
+          tc_mma_ss_w(tDP, kOnesDP, kCol, hi_none, ID_SS, 1u);  // - Delta
+          tc_commit(BAR(B_DP_FULL));
+        };
+        int it = 0, cn = 0;
+        for (int ci = cbeg; ci < cend; ++ci, ++cn) {
+          const int cnt = p.chains[ci].w;
+          wait(BAR(B_KV_FULL), cn & 1);
+          tc_fence_after();
+          if (cnt > 0) {
+            issue_s(it);
+            if (cnt > 1) issue_s(it + 1);
+            issue_dp(it);
+          }
+          // Each step finishes tile `it`: dP'^T of the next tile first (the softmax's
+          // next wait), dQp into this tile's S^T buffer, dK; then S'^T two tiles ahead
+          // into that buffer once dQp has been drained.
+          for (int t = 0; t < cnt; ++t, ++it) {
             const int s = it % ST, sd = it % SD;
             const uint32_t mQ = sdesc_lo(sQ + s * C::kTile, 16384);
             const uint32_t mDO = sdesc_lo(sDO + sd * C::kTile, 16384);
-            // dV += P^T dO : M = kv, N = D, K = q (A in TMEM, B MN-major), once P is packed
-            wait(BAR(B_P_READY), it & 1);
-            // the previous chain's dV/dK must have been read out before they restart
+            const uint32_t tSi = tS + s_col(it);
+            // dV += P^T dO (A in TMEM), once P is packed
+            wait(P_READY(it), s_phase(it));
             if (t == 0 && cn > 0) wait(BAR(B_DKDV_EMPTY), (cn - 1) & 1);
             tc_fence_after();
             const uint32_t acc0 = t > 0 ? 1u : 0u;
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              tc_mma_ts_w(tDV, tS + 32 * (kk >> 1) + 8 * (kk & 1), mDO + kk * 128, hi, ID_KV,
+              tc_mma_ts_w(tDV, tSi + 32 * (kk >> 1) + 8 * (kk & 1), mDO + kk * 128, hi, ID_KV,
                           kk > 0 ? 1u : acc0);
             tc_commit(DO_EMPTY(sd));
-            // dK += dS^T Q
+            tc_commit(BAR(B_DV_DONE));
             wait(BAR(B_DS_READY), it & 1);
             trace(it, 1);
             tc_fence_after();
+            if (t + 1 < cnt) issue_dp(it + 1);
+            // dQp = dS K (both MN-major from shared memory) into the first 64 columns of
+            // this tile's S^T buffer, once dV has read P^T out of them
+            wait(BAR(B_DV_DONE), it & 1);
+            tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              tc_mma_ts_w(tDK, tS + 32 * (kk >> 1) + 16 + 8 * (kk & 1), mQ + kk * 128, hi, ID_KV,
-                          kk > 0 ? 1u : acc0);
+              tc_mma_ss_w(tmem + dq_col(it), mDS + kk * 128, mK + kk * 128, hi, ID_Q,
+                          kk > 0 ? 1u : 0u);
+            tc_commit(DQ_FULL(it));
+            // dK += dS^T Q : A = dS^T K-major, B = Q MN-major, both from shared memory
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t off = (uint32_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+              tc_mma_ss_w(tDK, kDS + off, mQ + kk * 128, hi, ID_KV, kk > 0 ? 1u : acc0);
+            }
             tc_commit(Q_EMPTY(s));
-            tc_commit(BAR(B_DVDK_DONE));
+            tc_commit(BAR(B_DS_FREE));  // dQp and dK have read dS^T
             if (t == cnt - 1) tc_commit(BAR(B_DKDV_FULL));
-            // dQp = dS K : M = q, N = D, K = kv (both operands MN-major)
-            const int buf = C::kDqInDp ? 0 : (it & 1);
-            if (!C::kDqInDp && it >= 2) {
-              wait(BAR(B_DQ_EMPTY0 + buf), ((it - 2) >> 1) & 1);
-              tc_fence_after();
-            }
-            const uint32_t tDQ = tmem + C::TM_DQ + 64 * buf;
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              tc_mma_ss_w(tDQ, mDS + kk * 128, mK + kk * 128, hi, ID_Q, kk > 0 ? 1u : 0u);
-            tc_commit(BAR(B_DQ_FULL0 + buf));
-            tc_commit(BAR(B_DS_FREE));
             trace(it, 2);
-            ++it;
+            if (t + 2 < cnt) issue_s(it + 2);
           }
-          if (t + 1 < cnt) {
-            // S^T = K Q^T of tile `it`: M = kv, N = q, K = D (both K-major), once dV/dK
-            // of the previous tile have read packed P^T/dS^T out of these columns
-            const int s = it % ST, sd = it % SD;
-            const uint32_t kQ = sdesc_lo(sQ + s * C::kTile, 16);
-            const uint32_t kDO = sdesc_lo(sDO + sd * C::kTile, 16);
-            const uint32_t kCol = sdesc_lo_none(sb + C::OFF_COL + s * C::kColTile, 2048);
-            wait(Q_FULL(s), (it / ST) & 1);
-            if (it > 0) wait(BAR(B_DVDK_DONE), (it - 1) & 1);
-            tc_fence_after();
-            trace(it, 0);
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = (uint32_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
-              tc_mma_ss_w(tS, kK + off, kQ + off, hi, ID_SS, kk > 0 ? 1u : 0u);
-            }
-            // S'^T = S^T - LSE / scale, so the softmax takes P = 2^(scale log2e S')
-            tc_mma_ss_w(tS, kOnesS, kCol, hi_none, ID_SS, 1u);
-            tc_commit(BAR(B_S_FULL));
-            // dP^T = V dO^T; at D = 128 these columns hold dQp of the previous tile
-            // until the reducers have drained it
-            wait(DO_FULL(sd), (it / SD) & 1);
-            if (C::kDqInDp && it > 0) wait(BAR(B_DQ_EMPTY0), (it - 1) & 1);
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = (uint32_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
-              tc_mma_ss_w(tDP, kV + off, kDO + off, hi, ID_SS, kk > 0 ? 1u : 0u);
-            }
-            // dP'^T = dP^T - Delta, so the softmax forms dS = P dP'
-            tc_mma_ss_w(tDP, kOnesDP, kCol, hi_none, ID_SS, 1u);
-            tc_commit(BAR(B_DP_FULL));
-          }
+          tc_commit(BAR(B_KV_EMPTY));
         }
-        tc_commit(BAR(B_KV_EMPTY));
+      } else {
+        int it = 0, cn = 0;
+        for (int ci = cbeg; ci < cend; ++ci, ++cn) {
+          const int cnt = p.chains[ci].w;
+          wait(BAR(B_KV_FULL), cn & 1);
+          tc_fence_after();
+          // t = -1 only issues the chain's first S^T/dP^T; each later step finishes
+          // tile `it` and then issues S^T/dP^T of the next tile behind it
+          for (int t = -1; t < cnt; ++t) {
+            if (t >= 0) {
+              const int s = it % ST, sd = it % SD;
+              const uint32_t mQ = sdesc_lo(sQ + s * C::kTile, 16384);
+              const uint32_t mDO = sdesc_lo(sDO + sd * C::kTile, 16384);
+              // dV += P^T dO : M = kv, N = D, K = q (A in TMEM, B MN-major), once P is packed
+              wait(BAR(B_P_READY), it & 1);
+              // the previous chain's dV/dK must have been read out before they restart
+              if (t == 0 && cn > 0) wait(BAR(B_DKDV_EMPTY), (cn - 1) & 1);
+              tc_fence_after();
+              const uint32_t acc0 = t > 0 ? 1u : 0u;
+  #pragma unroll
+              for (int kk = 0; kk < 8; ++kk)
+                tc_mma_ts_w(tDV, tS + 32 * (kk >> 1) + 8 * (kk & 1), mDO + kk * 128, hi, ID_KV,
+                            kk > 0 ? 1u : acc0);
+              tc_commit(DO_EMPTY(sd));
+              // dK += dS^T Q
+              wait(BAR(B_DS_READY), it & 1);
+              trace(it, 1);
+              tc_fence_after();
+  #pragma unroll
+              for (int kk = 0; kk < 8; ++kk)
+                tc_mma_ts_w(tDK, tS + 32 * (kk >> 1) + 16 + 8 * (kk & 1), mQ + kk * 128, hi, ID_KV,
+                            kk > 0 ? 1u : acc0);
+              tc_commit(Q_EMPTY(s));
+              tc_commit(BAR(B_DVDK_DONE));
+              if (t == cnt - 1) tc_commit(BAR(B_DKDV_FULL));
+              // dQp = dS K : M = q, N = D, K = kv (both operands MN-major)
+              const int buf = C::kDqInDp ? 0 : (it & 1);
+              if (!C::kDqInDp && it >= 2) {
+                wait(BAR(B_DQ_EMPTY0 + buf), ((it - 2) >> 1) & 1);
+                tc_fence_after();
+              }
+              const uint32_t tDQ = tmem + dq_col(it);
+  #pragma unroll
+              for (int kk = 0; kk < 8; ++kk)
+                tc_mma_ss_w(tDQ, mDS + kk * 128, mK + kk * 128, hi, ID_Q, kk > 0 ? 1u : 0u);
+              tc_commit(BAR(B_DQ_FULL0 + buf));
+              tc_commit(BAR(B_DS_FREE));
+              trace(it, 2);
+              ++it;
+            }
+            if (t + 1 < cnt) {
+              // S^T = K Q^T of tile `it`: M = kv, N = q, K = D (both K-major), once dV/dK
+              // of the previous tile have read packed P^T/dS^T out of these columns
+              const int s = it % ST, sd = it % SD;
+              const uint32_t kQ = sdesc_lo(sQ + s * C::kTile, 16);
+              const uint32_t kDO = sdesc_lo(sDO + sd * C::kTile, 16);
+              const uint32_t kCol = sdesc_lo_none(sb + C::OFF_COL + s * C::kColTile, 2048);
+              wait(Q_FULL(s), (it / ST) & 1);
+              if (it > 0) wait(BAR(B_DVDK_DONE), (it - 1) & 1);
+              tc_fence_after();
+              trace(it, 0);
+  #pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (uint32_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+                tc_mma_ss_w(tS, kK + off, kQ + off, hi, ID_SS, kk > 0 ? 1u : 0u);
+              }
+              // S'^T = S^T - LSE / scale, so the softmax takes P = 2^(scale log2e S')
+              tc_mma_ss_w(tS, kOnesS, kCol, hi_none, ID_SS, 1u);
+              tc_commit(BAR(B_S_FULL));
+              // dP^T = V dO^T; at D = 128 these columns hold dQp of the previous tile
+              // until the reducers have drained it
+              wait(DO_FULL(sd), (it / SD) & 1);
+              if (C::kDqInDp && it > 0) wait(BAR(B_DQ_EMPTY0), (it - 1) & 1);
+              tc_fence_after();
+  #pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (uint32_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+                tc_mma_ss_w(tDP, kV + off, kDO + off, hi, ID_SS, kk > 0 ? 1u : 0u);
+              }
+              // dP'^T = dP^T - Delta, so the softmax forms dS = P dP'
+              tc_mma_ss_w(tDP, kOnesDP, kCol, hi_none, ID_SS, 1u);
+              tc_commit(BAR(B_DP_FULL));
+            }
+          }
+          tc_commit(BAR(B_KV_EMPTY));
+        }
       }
       // drain: all issued MMAs complete before TMEM is released
       tc_commit(BAR(B_FINAL));
@@ -388,14 +510,15 @@ __global__ void __launch_bounds__(512, 1)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t rowoff =
         (uint32_t)half * 16384 + (uint32_t)(r >> 3) * 1024 + (uint32_t)(r & 7) * 128;
-    const uint32_t tS = tmem + lane_off + C::TM_S, tDP = tmem + lane_off + C::TM_DP;
+    const uint32_t tS0 = tmem + lane_off + C::TM_S, tDP = tmem + lane_off + C::TM_DP;
     const float sl2 = p.scale_log2;
     int it = 0;
     for (int ci = cbeg; ci < cend; ++ci) {
       const int4 ch = p.chains[ci];
       for (int t = 0; t < ch.w; ++t, ++it) {
         const int q = (int)(p.pairs[ch.z + t] & 0xffffu);
-        wait(BAR(B_S_FULL), it & 1);
+        const uint32_t tS = tS0 + s_col(it);
+        wait(S_FULL(it), s_phase(it));
         if (threadIdx.x == 0) trace(it, 3);
         tc_fence_after();
         // causal: on the diagonal tile Q column qc sees KV row r only if qc >= r
@@ -428,7 +551,7 @@ __global__ void __launch_bounds__(512, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(BAR(B_P_READY));
+        mbar_arrive(P_READY(it));
         wait(BAR(B_DP_FULL), it & 1);
         if (it > 0) wait(BAR(B_DS_FREE), (it - 1) & 1);
         tc_fence_after();
@@ -448,9 +571,9 @@ __global__ void __launch_bounds__(512, 1)
             const float p1 = __uint_as_float(pk[j >> 1] & 0xffff0000u);
             dk[j >> 1] = pack_bf16x2(p0 * __uint_as_float(dv[j]), p1 * __uint_as_float(dv[j + 1]));
           }
-          // dS^T into the last 16 columns of chunk c, and to shared memory
-          // (128-byte swizzle, 64-column block `half`)
-          tmem_st16(tS + 32 * c + 16, dk);
+          // dS^T into the last 16 columns of chunk c (D = 128, where dK reads it from
+          // TMEM), and to shared memory (128-byte swizzle, 64-column block `half`)
+          if constexpr (!C::kSDouble) tmem_st16(tS + 32 * c + 16, dk);
 #pragma unroll
           for (int m = 0; m < 4; ++m) {
             const uint32_t chunk = (uint32_t)(((cc * 4 + m) ^ (r & 7)) * 16);
@@ -458,7 +581,7 @@ __global__ void __launch_bounds__(512, 1)
                          dk[4 * m + 3]);
           }
         }
-        tmem_wait_st();
+        if constexpr (!C::kSDouble) tmem_wait_st();
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(BAR(B_DS_READY));
@@ -480,21 +603,19 @@ __global__ void __launch_bounds__(512, 1)
         const int q = (int)(w & 0xffffu), pos = (int)(w >> 16);
         const int ncontrib = p.causal ? q + 1 : N;
         const bool last = (pos == ncontrib - 1);
-        const int buf = C::kDqInDp ? 0 : (it & 1);
-        const int ph = C::kDqInDp ? (it & 1) : ((it >> 1) & 1);
-        wait(BAR(B_DQ_FULL0 + buf), ph);
+        wait(DQ_FULL(it), s_phase(it));
         if (threadIdx.x == 256) trace(it, 4);
         tc_fence_after();
         float a[D];
 #pragma unroll
         for (int c2 = 0; c2 < D / 32; ++c2) {
           uint32_t v[32];
-          tmem_ld32(tmem + lane_off + C::TM_DQ + 64 * buf + c2 * 32, v);
+          tmem_ld32(tmem + lane_off + dq_col(it) + c2 * 32, v);
 #pragma unroll
           for (int j = 0; j < 32; ++j) a[c2 * 32 + j] = __uint_as_float(v[j]);
         }
         tc_fence_before();
-        mbar_arrive(BAR(B_DQ_EMPTY0 + buf));
+        mbar_arrive(DQ_EMPTY(it));
         if (threadIdx.x == 256) trace(it, 5);
         const long long blk = (long long)ch.x * N + q;
         if constexpr (!kAtomic) {
