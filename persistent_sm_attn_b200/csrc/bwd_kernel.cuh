@@ -109,7 +109,7 @@ struct BwdCfg {
   static constexpr int OFF_DO = OFF_Q + kStagesQ * kTile;
   static constexpr int OFF_DST = OFF_DO + kStagesDO * kTile;  // dS^T [128 kv][128 q]
   static constexpr int OFF_BAR = OFF_DST + 32768;
-  static constexpr int kBars = 18 + 2 * kStagesQ + 2 * kStagesDO;
+  static constexpr int kBars = 22 + 2 * kStagesQ + 2 * kStagesDO;
   static constexpr int OFF_TMEM_SLOT = OFF_BAR + kBars * 8;
   // The swizzled tiles need a 1 KiB aligned base; the kernel checks it.
   static constexpr int kSmemBytes = OFF_TMEM_SLOT + 16;
@@ -124,6 +124,10 @@ struct BwdCfg {
   static constexpr uint32_t TM_DV = TM_DP + 128, TM_DK = TM_DV + D;
   static_assert(TM_DK + D == 512, "TMEM columns");
   static constexpr bool kDqInDp = !kSDouble;
+  // D = 64: a publisher warp releases the tickets, taking the release's wait for the
+  // stores off the reducers (at D = 128 the extra hand-off lengthens each link of the
+  // accumulation chains more than it saves)
+  static constexpr bool kPublisher = kSDouble;
 };
 
 // Number of dQ accumulation chains (tickets, and fp32 accumulators of 128 x D):
@@ -138,7 +142,8 @@ enum {
   B_KV_FULL = 0, B_KV_EMPTY, B_S_FULL, B_DP_FULL, B_DS_READY, B_DS_FREE, B_DQ_FULL0, B_DQ_FULL1,
   B_DQ_EMPTY0, B_DQ_EMPTY1, B_DVDK_DONE, B_DKDV_FULL, B_DKDV_EMPTY, B_FINAL, B_P_READY,
   B_S_FULL1, B_P_READY1, B_DV_DONE,  // the second S^T buffer and dV done (D = 64)
-  B_STAGE0 = 18
+  B_PUB_READY0, B_PUB_READY1, B_PUB_FREE0, B_PUB_FREE1,  // reducers -> publisher hand-off
+  B_STAGE0 = 22
 };
 
 // kTrace: record %globaltimer per pair of this CTA: 0 S^T issued, 1 softmax
@@ -216,6 +221,10 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(BAR(B_FINAL), 1);
     mbar_init(BAR(B_P_READY), 256);
     mbar_init(BAR(B_P_READY1), 256);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(BAR(B_PUB_READY0 + b), 128);
+      mbar_init(BAR(B_PUB_FREE0 + b), 1);
+    }
     for (int s = 0; s < ST; ++s) {
       mbar_init(Q_FULL(s), 1);
       mbar_init(Q_EMPTY(s), 1);
@@ -499,6 +508,30 @@ __global__ void __launch_bounds__(512, 1)
       // drain: all issued MMAs complete before TMEM is released
       tc_commit(BAR(B_FINAL));
       drain(BAR(B_FINAL), 0);
+    } else if (warp == 14 && lane == 0 && !kAtomic && C::kPublisher) {
+      // ---------------------------------------------------------- publisher
+      // Publishes the reducers' load-add-store results in their place: once all 128
+      // reducer threads have arrived after their stores (release at CTA scope,
+      // acquired here), a release store at gpu scope advances the chain's ticket and
+      // makes those stores visible with it.  The reducers go on to the next pair
+      // without waiting for the release.  Hand-off slot k mod 2; the reducers take a
+      // slot again only after this warp has freed it.
+      int it = 0, k = 0;
+      for (int ci = cbeg; ci < cend; ++ci) {
+        const int4 ch = p.chains[ci];
+        for (int t = 0; t < ch.w; ++t, ++it) {
+          const uint32_t w = p.pairs[ch.z + t];
+          const int q = (int)(w & 0xffffu), pos = (int)(w >> 16);
+          const int ncontrib = p.causal ? q + 1 : N;
+          if (pos == ncontrib - 1) continue;  // the last contributor writes dQ itself
+          const long long unit = ((long long)ch.x * N + q) * 2 + (pos & 1);
+          wait(BAR(B_PUB_READY0 + (k & 1)), (k >> 1) & 1);
+          st_release_gpu(p.tickets + unit, (uint32_t)((pos >> 1) + 1));
+          mbar_arrive(BAR(B_PUB_FREE0 + (k & 1)));
+          trace(it, 7);
+          ++k;
+        }
+      }
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------ softmax / dS
@@ -596,6 +629,7 @@ __global__ void __launch_bounds__(512, 1)
     constexpr int NV = D / 4;           // float4 per row
     constexpr int G = 24;               // loads in flight per group
     int it = 0, cn = 0;
+    int npub = 0;  // pairs handed to the publisher
     for (int ci = cbeg; ci < cend; ++ci, ++cn) {
       const int4 ch = p.chains[ci];
       for (int t = 0; t < ch.w; ++t, ++it) {
@@ -698,10 +732,18 @@ __global__ void __launch_bounds__(512, 1)
             for (int c4 = 0; c4 < NV; ++c4)
               st_cg_f4(accp + c4 * 128 + r,
                        make_float4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]));
-            // the barrier orders every thread's stores before thread 256's release,
-            // which publishes them at gpu scope
-            named_bar_sync(1, 128);
-            if (threadIdx.x == 256) st_release_gpu(p.tickets + unit, (uint32_t)(idx + 1));
+            if constexpr (C::kPublisher) {
+              // hand the publication of these stores to the publisher warp (slot k mod 2,
+              // free again once it has published pair k - 2)
+              if (npub >= 2) wait(BAR(B_PUB_FREE0 + (npub & 1)), ((npub - 2) >> 1) & 1);
+              mbar_arrive(BAR(B_PUB_READY0 + (npub & 1)));
+              ++npub;
+            } else {
+              // the barrier orders every thread's stores before thread 256's release,
+              // which publishes them at gpu scope
+              named_bar_sync(1, 128);
+              if (threadIdx.x == 256) st_release_gpu(p.tickets + unit, (uint32_t)(idx + 1));
+            }
           }
         } else {
           float4* accp = reinterpret_cast<float4*>(p.acc + blk * 128 * D);
@@ -710,7 +752,7 @@ __global__ void __launch_bounds__(512, 1)
             atomicAdd(accp + c4 * 128 + r,
                       make_float4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]));
         }
-        if (threadIdx.x == 256) trace(it, 7);
+        if (threadIdx.x == 256 && (kAtomic || last || !C::kPublisher)) trace(it, 7);
       }
       // chain epilogue: dV_j and scale * dK_j (rows of KV tile ch.y) to global bf16
       wait(BAR(B_DKDV_FULL), cn & 1);
