@@ -187,6 +187,35 @@ int dash_attn_bwd_noalloc(const void* q, const void* k, const void* v, const voi
                           int B, int H, int S, int D, int causal, int schedule, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Backward pass from host buffers.
+ *
+ * The paper has no counterpart to this entry point; it serves callers whose
+ * tensors live in host memory.  Same arguments, shapes, schedules and results
+ * as dash_attn_bwd, except that q, k, v, o, dout, lse and dq, dk, dv are HOST
+ * pointers (caller-owned, same layouts; page-locked memory lets the copies run
+ * asynchronously and overlap the compute, pageable memory works but copies
+ * synchronously).  The heads are split into up to 8 parts.  Each part's inputs
+ * are copied to the device on a library-owned stream while the previous part
+ * computes on `stream` and the part before that is copied back on a second
+ * library-owned stream, through two device staging slots.
+ *   - Results: every part runs the sub-table of the whole problem's schedule
+ *     table that covers its heads (same CTA for every chain, same position for
+ *     every dQ partial), so dq, dk, dv are bitwise identical to those of
+ *     dash_attn_bwd on device copies of the same inputs.
+ *   - Completion: the call returns once everything is queued; the results are
+ *     on the host when `stream` has completed (dash_attn_sync_status(stream)
+ *     waits for it and reports device-side timeouts as for dash_attn_bwd).
+ *   - Ownership: the staging slots (about 2 * (8*D*2 + 4) bytes per row of one
+ *     part), the copy streams and the per-part tables are cached per (device,
+ *     stream) and freed by dash_release_workspace().  Calls that use the same
+ *     stream are ordered; the host buffers must stay valid and unmodified until
+ *     `stream` has completed.
+ */
+int dash_attn_bwd_host(const void* q, const void* k, const void* v, const void* o,
+                       const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                       int H, int S, int D, int causal, int schedule, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Host-only entry points (no GPU needed).
  */
 
@@ -200,6 +229,17 @@ int dash_attn_bwd_noalloc(const void* q, const void* k, const void* v, const voi
  */
 long long dash_sched_table(int n_heads, int N, int causal, int schedule, int num_ctas,
                            int* rows, long long cap);
+
+/*
+ * The part of that table covering heads [h0, h1) (0 <= h0 < h1 <= n_heads), as the
+ * host-buffer path launches it: heads renumbered from 0, every chain on the same CTA
+ * and every pair at the same position in its dQ order as in the whole table.  Rows
+ * as for dash_sched_table.  Returns the number of rows, or -DASH_ERR_INVALID_ARG for
+ * a bad head range, -DASH_ERR_UNSUPPORTED, or -DASH_ERR_SCHEDULE if the part fails
+ * validation.
+ */
+long long dash_sched_table_part(int n_heads, int N, int causal, int schedule, int num_ctas,
+                                int h0, int h1, int* rows, long long cap);
 
 /*
  * DAG simulation of a schedule table (DASH summary §2.1): per pair the events

@@ -22,7 +22,8 @@ EXPORTS = ("dash_attn_fwd", "dash_attn_bwd", "dash_attn_sync_status", "dash_stat
            "dash_set_spin_limit_us", "dash_bwd_num_ctas", "dash_release_workspace",
            "dash_sched_table", "dash_sched_simulate", "dash_dag_longest_path",
            "dash_profile_begin", "dash_profile_end", "dash_attn_bwd_noalloc",
-           "dash_trace_bwd", "dash_inject_fault", "dash_sched_check")
+           "dash_trace_bwd", "dash_inject_fault", "dash_sched_check", "dash_attn_bwd_host",
+           "dash_sched_table_part")
 
 
 class DashError(RuntimeError):
@@ -53,6 +54,7 @@ def load(path: str | None = None):
     lib.dash_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, vp]
     lib.dash_attn_bwd.argtypes = [vp] * 9 + [i, i, i, i, i, i, vp]
     lib.dash_attn_bwd_noalloc.argtypes = [vp] * 9 + [i, i, i, i, i, i, vp]
+    lib.dash_attn_bwd_host.argtypes = [vp] * 9 + [i, i, i, i, i, i, vp]
     lib.dash_attn_sync_status.argtypes = [vp]
     lib.dash_status_string.argtypes = [i]
     lib.dash_status_string.restype = ctypes.c_char_p
@@ -62,6 +64,8 @@ def load(path: str | None = None):
     lib.dash_release_workspace.argtypes = []
     lib.dash_sched_table.argtypes = [i, i, i, i, i, vp, ll]
     lib.dash_sched_table.restype = ll
+    lib.dash_sched_table_part.argtypes = [i, i, i, i, i, i, i, vp, ll]
+    lib.dash_sched_table_part.restype = ll
     lib.dash_sched_simulate.argtypes = [i, i, i, i, i, d, d, i, i, P(d), P(d), P(d), P(ll)]
     lib.dash_sched_check.argtypes = [i, i, i, i, vp, ll]
     lib.dash_dag_longest_path.argtypes = [i, i, vp, vp, vp, vp, vp, P(d)]
@@ -69,7 +73,7 @@ def load(path: str | None = None):
     lib.dash_profile_begin.argtypes = []
     lib.dash_profile_end.argtypes = [P(d), P(d), P(ll)]
     for name in EXPORTS:
-        if name not in ("dash_status_string", "dash_sched_table"):
+        if name not in ("dash_status_string", "dash_sched_table", "dash_sched_table_part"):
             getattr(lib, name).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -132,6 +136,31 @@ def dash_attn_bwd(q, k, v, o, do, lse, causal: bool, schedule="shift", dq=None, 
     return dq, dk, dv
 
 
+def dash_attn_bwd_host(q, k, v, o, do, lse, causal: bool, schedule="shift", dq=None, dk=None,
+                       dv=None, stream=None):
+    """The backward from host (CPU) tensors, pipelined over parts of the heads;
+    results are bitwise those of dash_attn_bwd.  Page-locked tensors let the
+    copies overlap the compute.  The outputs are valid once `stream` (default:
+    torch's current stream) has completed."""
+    import torch
+    for t in (q, k, v, o, do, lse):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("inputs must be contiguous host tensors")
+    B, H, S, D = q.shape
+    pin = q.is_pinned()
+    dq = torch.empty(q.shape, dtype=q.dtype, pin_memory=pin) if dq is None else dq
+    dk = torch.empty(k.shape, dtype=k.dtype, pin_memory=pin) if dk is None else dk
+    dv = torch.empty(v.shape, dtype=v.dtype, pin_memory=pin) if dv is None else dv
+    for t in (dq, dk, dv):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("outputs must be contiguous host tensors")
+    rc = load().dash_attn_bwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse),
+                                   _ptr(dq), _ptr(dk), _ptr(dv), B, H, S, D, int(bool(causal)),
+                                   _sched_id(schedule), _stream_handle(stream))
+    _check(rc, "dash_attn_bwd_host")
+    return dq, dk, dv
+
+
 def dash_attn_bwd_noalloc(q, k, v, o, do, lse, causal: bool, schedule, dq, dk, dv,
                           stream=None):
     """The backward through the entry point that allocates no device memory.
@@ -181,6 +210,21 @@ def dash_sched_table(n_heads: int, N: int, causal: bool, schedule, num_ctas: int
         raise DashError(int(-n), "dash_sched_table")
     buf = (ctypes.c_int * (6 * n))()
     lib.dash_sched_table(n_heads, N, int(bool(causal)), sid, num_ctas, buf, n)
+    flat = list(buf)
+    return [tuple(flat[6 * r: 6 * r + 6]) for r in range(n)]
+
+
+def dash_sched_table_part(n_heads: int, N: int, causal: bool, schedule, num_ctas: int,
+                          h0: int, h1: int):
+    """Rows of the part of the table covering heads [h0, h1), heads renumbered
+    from 0, as the host-buffer path launches it."""
+    lib = load()
+    sid = _sched_id(schedule)
+    n = lib.dash_sched_table_part(n_heads, N, int(bool(causal)), sid, num_ctas, h0, h1, None, 0)
+    if n < 0:
+        raise DashError(int(-n), "dash_sched_table_part")
+    buf = (ctypes.c_int * (6 * max(n, 1)))()
+    lib.dash_sched_table_part(n_heads, N, int(bool(causal)), sid, num_ctas, h0, h1, buf, n)
     flat = list(buf)
     return [tuple(flat[6 * r: 6 * r + 6]) for r in range(n)]
 

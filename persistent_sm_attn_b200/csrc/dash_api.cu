@@ -118,6 +118,40 @@ int get_workspace(int dev, void* stream, size_t acc_bytes, size_t tk_bytes, size
   return DASH_OK;
 }
 
+void free_table(DevTable* d) {
+  cudaFree(d->cta_off);
+  cudaFree(d->chains);
+  cudaFree(d->pairs);
+  *d = DevTable{};
+}
+
+int upload_table(const dash::Table& t, DevTable* out) {
+  DevTable d;
+  // an empty chain or pair list still gets a valid (unused) allocation
+  const size_t nc = t.chains.empty() ? 1 : t.chains.size();
+  const size_t np = t.pairs.empty() ? 1 : t.pairs.size();
+  if (cudaMalloc(&d.cta_off, t.cta_off.size() * sizeof(int)) != cudaSuccess ||
+      cudaMalloc(&d.chains, nc * sizeof(int4)) != cudaSuccess ||
+      cudaMalloc(&d.pairs, np * sizeof(uint32_t)) != cudaSuccess) {
+    cudaGetLastError();
+    free_table(&d);
+    return DASH_ERR_OOM;
+  }
+  static_assert(sizeof(dash::Chain) == sizeof(int4), "chain layout");
+  if (cudaMemcpy(d.cta_off, t.cta_off.data(), t.cta_off.size() * sizeof(int),
+                 cudaMemcpyHostToDevice) != cudaSuccess ||
+      (!t.chains.empty() &&
+       cudaMemcpy(d.chains, t.chains.data(), t.chains.size() * sizeof(int4),
+                  cudaMemcpyHostToDevice) != cudaSuccess) ||
+      (!t.pairs.empty() && cudaMemcpy(d.pairs, t.pairs.data(), t.pairs.size() * sizeof(uint32_t),
+                                      cudaMemcpyHostToDevice) != cudaSuccess)) {
+    free_table(&d);
+    return DASH_ERR_CUDA;
+  }
+  *out = d;
+  return DASH_OK;
+}
+
 int get_table(int dev, int heads, int N, int causal, int sched, int ctas, DevTable** out) {
   auto key = std::make_tuple(dev, heads, N, causal, sched, ctas);
   auto itb = g_tables.find(key);
@@ -130,23 +164,46 @@ int get_table(int dev, int heads, int N, int causal, int sched, int ctas, DevTab
   if (!dash::build_table(heads, N, causal, sched, ctas, &t, &err)) return DASH_ERR_UNSUPPORTED;
   if (!dash::validate_table(t, &err)) return DASH_ERR_SCHEDULE;
   DevTable d;
-  if (cudaMalloc(&d.cta_off, t.cta_off.size() * sizeof(int)) != cudaSuccess ||
-      cudaMalloc(&d.chains, t.chains.size() * sizeof(int4)) != cudaSuccess ||
-      cudaMalloc(&d.pairs, t.pairs.size() * sizeof(uint32_t)) != cudaSuccess) {
-    cudaGetLastError();
-    cudaFree(d.cta_off);
-    cudaFree(d.chains);
-    cudaFree(d.pairs);
-    return DASH_ERR_OOM;
-  }
-  static_assert(sizeof(dash::Chain) == sizeof(int4), "chain layout");
-  DASH_CUDA(cudaMemcpy(d.cta_off, t.cta_off.data(), t.cta_off.size() * sizeof(int),
-                       cudaMemcpyHostToDevice));
-  DASH_CUDA(cudaMemcpy(d.chains, t.chains.data(), t.chains.size() * sizeof(int4),
-                       cudaMemcpyHostToDevice));
-  DASH_CUDA(cudaMemcpy(d.pairs, t.pairs.data(), t.pairs.size() * sizeof(uint32_t),
-                       cudaMemcpyHostToDevice));
+  int rc = upload_table(t, &d);
+  if (rc) return rc;
   auto res = g_tables.emplace(key, d);
+  *out = &res.first->second;
+  return DASH_OK;
+}
+
+// Tables of the host-buffer path: the whole grid's table split into parts of
+// `chunk` heads (split_table keeps every dQ block's order), one per part.
+std::map<std::tuple<int, int, int, int, int, int, int>, std::vector<DevTable>> g_chunk_tables;
+
+int get_chunk_tables(int dev, int heads, int N, int causal, int sched, int ctas, int chunk,
+                     std::vector<DevTable>** out) {
+  auto key = std::make_tuple(dev, heads, N, causal, sched, ctas, chunk);
+  auto itc = g_chunk_tables.find(key);
+  if (itc != g_chunk_tables.end()) {
+    *out = &itc->second;
+    return DASH_OK;
+  }
+  dash::Table full;
+  std::string err;
+  if (!dash::build_table(heads, N, causal, sched, ctas, &full, &err)) return DASH_ERR_UNSUPPORTED;
+  if (!dash::validate_table(full, &err)) return DASH_ERR_SCHEDULE;
+  std::vector<DevTable> parts;
+  int rc = DASH_OK;
+  for (int h0 = 0; h0 < heads && rc == DASH_OK; h0 += chunk) {
+    dash::Table t;
+    const int h1 = h0 + chunk < heads ? h0 + chunk : heads;
+    if (!dash::split_table(full, h0, h1, &t) || !dash::validate_table(t, &err)) {
+      rc = DASH_ERR_SCHEDULE;
+      break;
+    }
+    DevTable d;
+    if ((rc = upload_table(t, &d)) == DASH_OK) parts.push_back(d);
+  }
+  if (rc) {
+    for (DevTable& d : parts) free_table(&d);
+    return rc;
+  }
+  auto res = g_chunk_tables.emplace(key, std::move(parts));
   *out = &res.first->second;
   return DASH_OK;
 }
@@ -277,7 +334,7 @@ template <int D, bool kAtomic, bool kTrace = false>
 int launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                const float* lse, void* dq, void* dk, void* dv, int B, int H, int S, int causal,
                int sched, cudaStream_t stream, int dev, unsigned long long* trace = nullptr,
-               int trace_rows = 0) {
+               int trace_rows = 0, const DevTable* tab_override = nullptr) {
   using C = BwdCfg<D>;
   const int N = S / 128;
   const long long rows = (long long)B * H * S;
@@ -288,8 +345,10 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   Workspace* ws = nullptr;
   {
     std::lock_guard<std::mutex> lk(g_mu);
-    const int fault = g_fault.exchange(0);
-    if (fault == 1 && !kAtomic) {
+    const int fault = tab_override ? 0 : g_fault.exchange(0);
+    if (tab_override) {
+      tab = const_cast<DevTable*>(tab_override);
+    } else if (fault == 1 && !kAtomic) {
       if ((rc = get_fault_table(dev, B * H, N, causal, sched, ctas, &tab))) return rc;
     } else if ((rc = get_table(dev, B * H, N, causal, sched, ctas, &tab))) {
       return rc;
@@ -373,6 +432,126 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   return DASH_OK;
 }
 
+// ------------------------------------------------------------------ host-buffer path
+// Per (device, caller stream): two copy streams, events, and two slots of device
+// staging for one part's inputs and outputs.
+struct HostPipe {
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t entry = nullptr;
+  cudaEvent_t in_ready[2] = {}, comp_done[2] = {}, out_done[2] = {};
+  unsigned char* buf = nullptr;
+  size_t cap = 0;
+};
+std::map<std::pair<int, uintptr_t>, HostPipe> g_pipes;
+
+int get_pipe(int dev, void* stream, size_t bytes, HostPipe** out) {
+  HostPipe& hp = g_pipes[{dev, reinterpret_cast<uintptr_t>(stream)}];
+  if (!hp.h2d) {
+    bool ok = cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.entry, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; i < 2 && ok; ++i)
+      ok = cudaEventCreateWithFlags(&hp.in_ready[i], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&hp.comp_done[i], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&hp.out_done[i], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) {
+      cudaGetLastError();
+      return DASH_ERR_CUDA;
+    }
+  }
+  int rc = grow(reinterpret_cast<void**>(&hp.buf), &hp.cap, bytes);
+  if (rc) return rc;
+  *out = &hp;
+  return DASH_OK;
+}
+
+void free_pipe(HostPipe* hp) {
+  cudaFree(hp->buf);
+  for (int i = 0; i < 2; ++i) {
+    cudaEventDestroy(hp->in_ready[i]);
+    cudaEventDestroy(hp->comp_done[i]);
+    cudaEventDestroy(hp->out_done[i]);
+  }
+  cudaEventDestroy(hp->entry);
+  cudaStreamDestroy(hp->h2d);
+  cudaStreamDestroy(hp->d2h);
+  *hp = HostPipe{};
+}
+
+constexpr int kHostParts = 8;  // parts the heads are split into on the host-buffer path
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Backward from host buffers: the heads are split into parts; part p's inputs are
+// copied in on one stream while part p-1 computes on the caller's stream and the
+// results of part p-2 are copied out on a third, through two staging slots.
+template <int D, bool kAtomic>
+int host_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+             const float* lse, void* dq, void* dk, void* dv, int B, int H, int S, int causal,
+             int sched, cudaStream_t stream, int dev) {
+  const int BH = B * H, N = S / 128;
+  const int chunk = (BH + kHostParts - 1) / kHostParts;
+  int ctas = 0;
+  int rc = num_ctas_for<D, kAtomic>(dev, &ctas);
+  if (rc) return rc;
+  const size_t rows_c = (size_t)chunk * S;
+  const size_t tile = align256(rows_c * D * 2), lse_b = align256(rows_c * 4);
+  const size_t slot_bytes = 8 * tile + lse_b;  // q k v o dO, LSE; dQ dK dV
+  std::vector<DevTable>* parts = nullptr;
+  HostPipe* hp = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if ((rc = get_chunk_tables(dev, BH, N, causal, sched, ctas, chunk, &parts))) return rc;
+    if ((rc = get_pipe(dev, stream, 2 * slot_bytes, &hp))) return rc;
+  }
+  // the copy streams start after whatever the caller queued before this call
+  DASH_CUDA(cudaEventRecord(hp->entry, stream));
+  DASH_CUDA(cudaStreamWaitEvent(hp->h2d, hp->entry, 0));
+  DASH_CUDA(cudaStreamWaitEvent(hp->d2h, hp->entry, 0));
+  const unsigned char* hin[5] = {static_cast<const unsigned char*>(q),
+                                 static_cast<const unsigned char*>(k),
+                                 static_cast<const unsigned char*>(v),
+                                 static_cast<const unsigned char*>(o),
+                                 static_cast<const unsigned char*>(dout)};
+  unsigned char* hout[3] = {static_cast<unsigned char*>(dq), static_cast<unsigned char*>(dk),
+                            static_cast<unsigned char*>(dv)};
+  int c = 0;
+  for (int h0 = 0; h0 < BH; h0 += chunk, ++c) {
+    const int nh = (BH - h0 < chunk) ? BH - h0 : chunk;
+    const int slot = c & 1;
+    unsigned char* base = hp->buf + slot * slot_bytes;
+    unsigned char* din[5];
+    for (int i = 0; i < 5; ++i) din[i] = base + i * tile;
+    float* dlse = reinterpret_cast<float*>(base + 5 * tile);
+    unsigned char* dout3[3];
+    for (int i = 0; i < 3; ++i) dout3[i] = base + 5 * tile + lse_b + i * tile;
+    const size_t off = (size_t)h0 * S * D * 2, n = (size_t)nh * S * D * 2;
+    // inputs of part c, once the compute of part c - 2 has released the slot
+    if (c >= 2) DASH_CUDA(cudaStreamWaitEvent(hp->h2d, hp->comp_done[slot], 0));
+    for (int i = 0; i < 5; ++i)
+      DASH_CUDA(cudaMemcpyAsync(din[i], hin[i] + off, n, cudaMemcpyHostToDevice, hp->h2d));
+    DASH_CUDA(cudaMemcpyAsync(dlse, lse + (size_t)h0 * S, (size_t)nh * S * 4,
+                              cudaMemcpyHostToDevice, hp->h2d));
+    DASH_CUDA(cudaEventRecord(hp->in_ready[slot], hp->h2d));
+    // compute, once the inputs are in and the results of part c - 2 are out
+    DASH_CUDA(cudaStreamWaitEvent(stream, hp->in_ready[slot], 0));
+    if (c >= 2) DASH_CUDA(cudaStreamWaitEvent(stream, hp->out_done[slot], 0));
+    if ((rc = launch_bwd<D, kAtomic>(din[0], din[1], din[2], din[3], din[4], dlse, dout3[0],
+                                     dout3[1], dout3[2], 1, nh, S, causal, sched, stream, dev,
+                                     nullptr, 0, &(*parts)[c])))
+      return rc;
+    DASH_CUDA(cudaEventRecord(hp->comp_done[slot], stream));
+    // results of part c
+    DASH_CUDA(cudaStreamWaitEvent(hp->d2h, hp->comp_done[slot], 0));
+    for (int i = 0; i < 3; ++i)
+      DASH_CUDA(cudaMemcpyAsync(hout[i] + off, dout3[i], n, cudaMemcpyDeviceToHost, hp->d2h));
+    DASH_CUDA(cudaEventRecord(hp->out_done[slot], hp->d2h));
+  }
+  // the caller's stream completes once every result is on the host
+  for (int i = 0; i < 2 && i < c; ++i) DASH_CUDA(cudaStreamWaitEvent(stream, hp->out_done[i], 0));
+  return DASH_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -449,6 +628,31 @@ int dash_attn_bwd(const void* q, const void* k, const void* v, const void* o, co
                                         schedule, st, dev)
                 : launch_bwd<128, false>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
                                          schedule, st, dev);
+}
+
+int dash_attn_bwd_host(const void* q, const void* k, const void* v, const void* o,
+                       const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                       int H, int S, int D, int causal, int schedule, void* stream) {
+  int rc = check_shape(B, H, S, D);
+  if (rc) return rc;
+  if (causal != 0 && causal != 1) return DASH_ERR_INVALID_ARG;
+  if (schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_ATOMIC) return DASH_ERR_INVALID_ARG;
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return DASH_ERR_INVALID_ARG;
+  if (!dash::schedule_supported(schedule, S / 128, causal)) return DASH_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0) return DASH_OK;
+  int dev = 0;
+  DASH_CUDA(cudaGetDevice(&dev));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool atomic = (schedule == DASH_SCHED_ATOMIC);
+  if (D == 64)
+    return atomic ? host_bwd<64, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
+                                       schedule, st, dev)
+                  : host_bwd<64, false>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
+                                        schedule, st, dev);
+  return atomic ? host_bwd<128, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
+                                      schedule, st, dev)
+                : host_bwd<128, false>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
+                                       schedule, st, dev);
 }
 
 int dash_attn_sync_status(void* stream) {
@@ -537,12 +741,26 @@ int dash_release_workspace(void) {
   }
   for (auto itt = g_tables.begin(); itt != g_tables.end();) {
     if (std::get<0>(itt->first) == dev) {
-      cudaFree(itt->second.cta_off);
-      cudaFree(itt->second.chains);
-      cudaFree(itt->second.pairs);
+      free_table(&itt->second);
       itt = g_tables.erase(itt);
     } else {
       ++itt;
+    }
+  }
+  for (auto itc = g_chunk_tables.begin(); itc != g_chunk_tables.end();) {
+    if (std::get<0>(itc->first) == dev) {
+      for (DevTable& d : itc->second) free_table(&d);
+      itc = g_chunk_tables.erase(itc);
+    } else {
+      ++itc;
+    }
+  }
+  for (auto itp = g_pipes.begin(); itp != g_pipes.end();) {
+    if (itp->first.first == dev) {
+      free_pipe(&itp->second);
+      itp = g_pipes.erase(itp);
+    } else {
+      ++itp;
     }
   }
   return DASH_OK;
@@ -610,6 +828,35 @@ int dash_trace_bwd(const void* q, const void* k, const void* v, const void* o, c
   *num_ctas = ctas;
   *rows_per_cta = rows;
   return rc;
+}
+
+long long dash_sched_table_part(int n_heads, int N, int causal, int schedule, int num_ctas,
+                                int h0, int h1, int* rows, long long cap) {
+  dash::Table full, t;
+  std::string err;
+  if (!dash::build_table(n_heads, N, causal, schedule, num_ctas, &full, &err))
+    return -DASH_ERR_UNSUPPORTED;
+  if (!dash::validate_table(full, &err)) return -DASH_ERR_SCHEDULE;
+  if (!dash::split_table(full, h0, h1, &t)) return -DASH_ERR_INVALID_ARG;
+  if (!dash::validate_table(t, &err)) return -DASH_ERR_SCHEDULE;
+  long long n = 0;
+  for (int c = 0; c < t.num_ctas; ++c)
+    for (int ci = t.cta_off[c]; ci < t.cta_off[c + 1]; ++ci) {
+      const dash::Chain& ch = t.chains[ci];
+      for (int i = 0; i < ch.pair_cnt; ++i, ++n) {
+        if (rows && n < cap) {
+          const uint32_t w = t.pairs[ch.pair_off + i];
+          int* r = rows + 6 * n;
+          r[0] = c;
+          r[1] = ch.bh;
+          r[2] = ch.kv;
+          r[3] = dash::pair_q(w);
+          r[4] = dash::pair_pos(w);
+          r[5] = ci;
+        }
+      }
+    }
+  return n;
 }
 
 long long dash_sched_table(int n_heads, int N, int causal, int schedule, int num_ctas, int* rows,

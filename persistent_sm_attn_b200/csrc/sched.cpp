@@ -191,6 +191,32 @@ bool table_from_rows(int n_heads, int N, int causal, int num_ctas, const int* ro
   return true;
 }
 
+bool split_table(const Table& full, int h0, int h1, Table* out) {
+  if (h0 < 0 || h1 <= h0 || h1 > full.n_heads) return false;
+  Table t;
+  t.n_heads = h1 - h0;
+  t.N = full.N;
+  t.causal = full.causal;
+  t.schedule = full.schedule;
+  t.num_ctas = full.num_ctas;
+  t.cta_off.assign(full.num_ctas + 1, 0);
+  for (int c = 0; c < full.num_ctas; ++c) {
+    for (int i = full.cta_off[c]; i < full.cta_off[c + 1]; ++i) {
+      const Chain& ch = full.chains[i];
+      if (ch.bh < h0 || ch.bh >= h1) continue;
+      Chain n = ch;
+      n.bh = ch.bh - h0;
+      n.pair_off = (int32_t)t.pairs.size();
+      t.pairs.insert(t.pairs.end(), full.pairs.begin() + ch.pair_off,
+                     full.pairs.begin() + ch.pair_off + ch.pair_cnt);
+      t.chains.push_back(n);
+    }
+    t.cta_off[c + 1] = (int32_t)t.chains.size();
+  }
+  *out = std::move(t);
+  return true;
+}
+
 bool validate_table(const Table& t, std::string* err) {
   auto fail = [&](const char* m) { if (err) *err = m; return false; };
   const int N = t.N;

@@ -55,6 +55,13 @@ bool build_table(int n_heads, int N, int causal, int schedule, int num_ctas, Tab
 // its reductions in table order.  Returns false with a message on failure.
 bool validate_table(const Table& t, std::string* err);
 
+// The part of `full` that covers heads [h0, h1), renumbered to heads 0..h1-h0-1.
+// Every chain keeps its CTA, its place among that CTA's chains, and its pairs'
+// positions, so a launch over the part performs each dQ block's additions in
+// the same order as a launch over the whole table.  Returns false if the range
+// is empty or outside the table.
+bool split_table(const Table& full, int h0, int h1, Table* out);
+
 // Longest path of a general DAG (Kahn order).  Returns false on a cycle.
 bool dag_longest_path(int n_nodes, int n_edges, const int* src, const int* dst,
                       const double* w, double* depth, double* height, double* cp);

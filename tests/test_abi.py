@@ -60,6 +60,13 @@ def test_argument_errors_need_no_gpu(lib):
     assert lib.dash_sched_simulate(1, 4, 0, 2, 4, -1.0, 0.0, 0, 1, None, None, None, None) == 1
     assert lib.dash_sched_simulate(1, 4, 0, 2, 4, 1.0, 0.0, 0, 0, None, None, None, None) == 1
     assert lib.dash_sched_check(1, 4, 2, 4, None, 0) == 1
+    # host-buffer path: null host pointers and bad shapes fail before any copy
+    assert lib.dash_attn_bwd_host(*null, 1, 1, 128, 64, 0, 2, None) == 1
+    assert lib.dash_attn_bwd_host(*good, 1, 1, 128, 96, 0, 2, None) == 2
+    assert lib.dash_attn_bwd_host(*good, 1, 1, 128, 64, 1, 2, None) == 2
+    # a part outside the table's heads
+    for h0, h1 in ((0, 0), (2, 1), (-1, 1), (0, 5)):
+        assert lib.dash_sched_table_part(4, 4, 0, 2, 8, h0, h1, None, 0) == -1
 
 
 def test_dag_cycle_rejected():

@@ -34,6 +34,11 @@ SMALL = [
     (2, 3, 640, 64, False),     # odd tile count
     (3, 5, 640, 128, True),     # odd tile count, 15 heads on the persistent grid
     (1, 1, 1024, 64, True),
+    # more chains than CTAs: every CTA runs two or three chains back to back, so the
+    # chain hand-offs (K/V reload, dK/dV drain, S^T buffers carried across) all occur
+    (4, 40, 256, 64, False),
+    (2, 40, 384, 64, True),     # odd tile count, causal
+    (4, 40, 256, 128, False),
 ]
 
 

@@ -49,6 +49,27 @@ def test_full_size_tables_validate():
         assert len(rows) == heads * (N * (N + 1) // 2 if causal else N * N)
 
 
+@pytest.mark.parametrize("heads,N,causal,name,ctas,chunk", [
+    (32, 32, False, "shift", 148, 4),        # parts straddle rounds (32 chains per head)
+    (13, 6, False, "naive_asc", 7, 3),       # uneven last part, several rounds per CTA
+    (10, 8, True, "sym_shift", 9, 4),
+    (9, 5, True, "descending", 6, 2),
+])
+def test_table_parts_keep_every_position(heads, N, causal, name, ctas, chunk):
+    """The host-buffer path launches parts of the whole table: each part holds
+    exactly the whole table's rows of its heads (renumbered), with the same CTA,
+    KV tile, Q tile and dQ position, in the same per-CTA order."""
+    full = binding.dash_sched_table(heads, N, causal, name, ctas)
+    seen = 0
+    for h0 in range(0, heads, chunk):
+        h1 = min(heads, h0 + chunk)
+        part = binding.dash_sched_table_part(heads, N, causal, name, ctas, h0, h1)
+        want = [(c, h - h0, kv, q, pos) for c, h, kv, q, pos, _ in full if h0 <= h < h1]
+        assert [r[:5] for r in part] == want
+        seen += len(part)
+    assert seen == len(full)
+
+
 def test_more_units_than_ctas_never_deadlock():
     # a shift head of 8 chains on 4 CTAs runs in two rounds; its dQ blocks
     # accumulate round by round, so the table is valid
