@@ -3,8 +3,6 @@
 //                       terms the backward's S^T and dP^T products add (LSE_i / scale
 //                       and Delta_i, each as three bf16 parts)
 //   dash_dq_convert     fp32 accumulator -> bf16 dQ (atomic comparison variant only)
-//   dash_fwd_kernel     softmax-attention forward producing O and LSE; it only
-//                       feeds the backward, so it uses plain fp32 FMAs.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -122,95 +120,6 @@ __global__ void __launch_bounds__(256) dash_dq_convert(const float* __restrict__
   pk.x = *reinterpret_cast<uint32_t*>(&lo);
   pk.y = *reinterpret_cast<uint32_t*>(&hi);
   *reinterpret_cast<uint2*>(dq + (blk * 128 + r) * D + 4 * c4) = pk;
-}
-
-// Forward: a CTA of 256 threads owns 64 query rows of one head; 4 threads per
-// row, each holding the 16-byte column chunks sub, sub+4, sub+8, ... of q and
-// of the output accumulator.  Keys are streamed through shared memory in
-// chunks of 64 with an online (running max) softmax in the log2 domain.
-template <int D>
-__global__ void __launch_bounds__(256) dash_fwd_kernel(const __nv_bfloat16* __restrict__ q,
-                                                       const __nv_bfloat16* __restrict__ k,
-                                                       const __nv_bfloat16* __restrict__ v,
-                                                       __nv_bfloat16* __restrict__ o,
-                                                       float* __restrict__ lse, int S, int causal,
-                                                       float scale_log2) {
-  constexpr int KC = 64;          // keys per chunk
-  constexpr int NCH = D / 32;     // 8-element chunks per thread
-  __shared__ __align__(16) __nv_bfloat16 ks[KC * D];
-  __shared__ __align__(16) __nv_bfloat16 vs[KC * D];
-  const int bh = blockIdx.y;
-  const int row0 = blockIdx.x * 64;
-  const int tid = threadIdx.x, sub = tid & 3, lr = tid >> 2;
-  const int qi = row0 + lr;
-  const size_t head = (size_t)bh * S * D;
-  float qf[NCH * 8], of[NCH * 8];
-#pragma unroll
-  for (int c = 0; c < NCH; ++c) {
-    const uint4 t = reinterpret_cast<const uint4*>(q + head + (size_t)qi * D)[sub + 4 * c];
-    bf16x8_to_f32(t, qf + 8 * c);
-  }
-#pragma unroll
-  for (int i = 0; i < NCH * 8; ++i) of[i] = 0.f;
-  float m = -INFINITY, l = 0.f;
-  const int kend = causal ? (row0 + 64) : S;
-  for (int k0 = 0; k0 < kend; k0 += KC) {
-    __syncthreads();
-    for (int e = tid; e < KC * D / 8; e += 256) {
-      reinterpret_cast<uint4*>(ks)[e] = reinterpret_cast<const uint4*>(k + head + (size_t)k0 * D)[e];
-      reinterpret_cast<uint4*>(vs)[e] = reinterpret_cast<const uint4*>(v + head + (size_t)k0 * D)[e];
-    }
-    __syncthreads();
-    float s[KC];
-    float cmax = -INFINITY;
-#pragma unroll 4
-    for (int j = 0; j < KC; ++j) {
-      float part = 0.f;
-#pragma unroll
-      for (int c = 0; c < NCH; ++c) {
-        float kf[8];
-        bf16x8_to_f32(reinterpret_cast<const uint4*>(ks + j * D)[sub + 4 * c], kf);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) part = fmaf(qf[8 * c + i], kf[i], part);
-      }
-      part += __shfl_xor_sync(0xffffffffu, part, 1);
-      part += __shfl_xor_sync(0xffffffffu, part, 2);
-      const bool ok = !causal || (k0 + j <= qi);
-      s[j] = ok ? part * scale_log2 : -INFINITY;
-      cmax = fmaxf(cmax, s[j]);
-    }
-    const float mnew = fmaxf(m, cmax);
-    const float corr = exp2f(m - mnew);
-    l *= corr;
-#pragma unroll
-    for (int i = 0; i < NCH * 8; ++i) of[i] *= corr;
-#pragma unroll 4
-    for (int j = 0; j < KC; ++j) {
-      const float pj = exp2f(s[j] - mnew);
-      l += pj;
-#pragma unroll
-      for (int c = 0; c < NCH; ++c) {
-        float vf[8];
-        bf16x8_to_f32(reinterpret_cast<const uint4*>(vs + j * D)[sub + 4 * c], vf);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) of[8 * c + i] = fmaf(pj, vf[i], of[8 * c + i]);
-      }
-    }
-    m = mnew;
-  }
-  const float inv = 1.f / l;
-#pragma unroll
-  for (int c = 0; c < NCH; ++c) {
-    uint4 pk;
-    uint32_t* w = reinterpret_cast<uint32_t*>(&pk);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      __nv_bfloat162 t = __floats2bfloat162_rn(of[8 * c + 2 * i] * inv, of[8 * c + 2 * i + 1] * inv);
-      w[i] = *reinterpret_cast<uint32_t*>(&t);
-    }
-    reinterpret_cast<uint4*>(o + head + (size_t)qi * D)[sub + 4 * c] = pk;
-  }
-  if (sub == 0) lse[(size_t)bh * S + qi] = (m + log2f(l)) * 0.6931471805599453f;
 }
 
 }  // namespace dash

@@ -18,6 +18,7 @@
 #include "../../include/dash_attn.h"
 #include "aux_kernels.cuh"
 #include "bwd_kernel.cuh"
+#include "fwd_kernel.cuh"
 #include "sched.h"
 
 namespace {
@@ -432,6 +433,43 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   return DASH_OK;
 }
 
+// ------------------------------------------------------------------ forward
+template <int D>
+int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+               int S, int causal, cudaStream_t stream, int dev) {
+  using C = dash::FwdCfg<D>;
+  const int N = S / 128;
+  const long long rows = (long long)B * H * S;
+  if ((long long)N * B * H > 0x7fffffffLL) return DASH_ERR_UNSUPPORTED;
+  Workspace* ws = nullptr;
+  int rc;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if ((rc = get_workspace(dev, stream, 0, 0, 0, &ws))) return rc;
+  }
+  CUtensorMap tq, tk, tv;
+  if ((rc = make_tmap(&tq, q, rows, D, 128)) || (rc = make_tmap(&tk, k, rows, D, 128)) ||
+      (rc = make_tmap(&tv, v, rows, D, 128)))
+    return rc;
+  auto kern = dash::dash_fwd_tc_kernel<D>;
+  DASH_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes));
+  dash::FwdParams p;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.err = ws->err;
+  p.abort_flag = ws->err + 1;
+  p.S = S;
+  p.N = N;
+  p.BH = B * H;
+  p.causal = causal;
+  p.scale_log2 = (1.0f / sqrtf((float)D)) * 1.4426950408889634f;
+  p.spin_ns = (unsigned long long)spin_us() * 1000ull;
+  DASH_CUDA(cudaMemsetAsync(ws->err + 1, 0, sizeof(unsigned), stream));
+  kern<<<(unsigned)(N * B * H), C::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+  DASH_CUDA(cudaGetLastError());
+  return DASH_OK;
+}
+
 // ------------------------------------------------------------------ host-buffer path
 // Per (device, caller stream): two copy streams, events, and two slots of device
 // staging for one part's inputs and outputs.
@@ -588,19 +626,11 @@ int dash_attn_fwd(const void* q, const void* k, const void* v, void* o, float* l
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !lse)
     return DASH_ERR_INVALID_ARG;
   if (B == 0 || H == 0) return DASH_OK;
+  int dev = 0;
+  DASH_CUDA(cudaGetDevice(&dev));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  dim3 grid(S / 64, B * H);
-  const float sl2 = (1.0f / sqrtf((float)D)) * 1.4426950408889634f;
-  if (D == 64)
-    dash::dash_fwd_kernel<64><<<grid, 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-        static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(o), lse, S, causal, sl2);
-  else
-    dash::dash_fwd_kernel<128><<<grid, 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-        static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(o), lse, S, causal, sl2);
-  DASH_CUDA(cudaGetLastError());
-  return DASH_OK;
+  return D == 64 ? launch_fwd<64>(q, k, v, o, lse, B, H, S, causal, st, dev)
+                 : launch_fwd<128>(q, k, v, o, lse, B, H, S, causal, st, dev);
 }
 
 int dash_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
