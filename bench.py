@@ -202,6 +202,25 @@ def run_ours(args):
     for other in compare:
         results[other] = time_schedule(other, max(5, args.steps // 2), 3)[0]
 
+    # the attention block around it: the library forward (O, LSE) timed the same way,
+    # outside the backward's timed region
+    fo, fl = torch.empty_like(q), torch.empty_like(lse)
+    for _ in range(2):
+        binding.dash_attn_fwd(q, k, v, w.causal, fo, fl)
+    fwd_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(max(3, args.steps // 2))]
+    barrier()
+    for i, (a, b) in enumerate(fwd_ev):
+        flush.fill_(float(i))
+        a.record(stream)
+        binding.dash_attn_fwd(q, k, v, w.causal, fo, fl)
+        b.record(stream)
+    barrier()
+    if binding.dash_attn_sync_status() != 0:
+        raise RuntimeError("forward status")
+    fwd_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in fwd_ev) / len(fwd_ev), "cuda")
+    del fo, fl
+
     sim = None
     if rank == 0 and not args.no_compare:
         sim = simulator_vs_measured(w, q, k, v, o, do, lse, sched, results)
@@ -261,6 +280,13 @@ def run_ours(args):
             "e2e": {"value": round(tflops(e2e_ms), 2), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": int(n_calls) * (3 if sched == "atomic" else 2),
+            "fwd_bwd": {"fwd_ms": round(fwd_ms, 4),
+                        "fwd_tflops": round(0.4 * w.flops * world / (fwd_ms * 1e-3) / 1e12, 2),
+                        "block_ms": round(fwd_ms + ms, 4),
+                        "block_tflops": round(1.4 * w.flops * world /
+                                              ((fwd_ms + ms) * 1e-3) / 1e12, 2),
+                        "note": "library forward (4 B H S^2 D FLOPs, half causal) plus this "
+                                "line's backward step, each timed on its own"},
             "clocks": clocks.summary(),
         }
         if sim is not None:
