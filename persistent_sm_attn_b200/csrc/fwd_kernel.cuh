@@ -37,7 +37,7 @@ template <int D>
 struct FwdCfg {
   static constexpr int kThreads = 256;
   static constexpr int kTile = 128 * D * 2;               // one [128][D] bf16 tile
-  static constexpr int kStages = (D == 64) ? 3 : 2;        // K/V stages
+  static constexpr int kStages = 3;                         // K/V stages (224 KiB at D = 128)
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + kTile;
   static constexpr int OFF_V = OFF_K + kStages * kTile;
