@@ -192,15 +192,17 @@ __global__ void __launch_bounds__(256, 1)
       tc_fence_after();
       // causal: on the diagonal tile KV column c is visible to row r only if c <= r
       const int vis = (p.causal && j == qt) ? r : 127;
+      // the row's 128 scores, loaded two chunks at a time with one wait for each pair, and
+      // kept in registers for both passes
+      uint32_t sv[4][32];
+      tmem_ld32x2(tS, tS + 32, sv[0], sv[1]);
+      tmem_ld32x2(tS + 64, tS + 96, sv[2], sv[3]);
       float mx = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t sv[32];
-        tmem_ld32(tS + 32 * c, sv);
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
 #pragma unroll
         for (int k = 0; k < 32; ++k)
-          if (32 * c + k <= vis) mx = fmaxf(mx, __uint_as_float(sv[k]));
-      }
+          if (32 * c + k <= vis) mx = fmaxf(mx, __uint_as_float(sv[c][k]));
       const float mt = mx * sl2;
       // move the running maximum when this tile would push P above 2^kRescaleLog2;
       // the decision is per warp (TMEM loads and stores are warp-wide), each lane
@@ -228,20 +230,20 @@ __global__ void __launch_bounds__(256, 1)
         }
         m = mn;
       }
-#pragma unroll 1
+#pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t sv[32];
-        tmem_ld32(tS + 32 * c, sv);
         uint32_t pk[16];
 #pragma unroll
         for (int k = 0; k < 32; k += 2) {
-          float p0 = (32 * c + k <= vis) ? ex2_approx(__uint_as_float(sv[k]) * sl2 - m) : 0.f;
-          float p1 =
-              (32 * c + k + 1 <= vis) ? ex2_approx(__uint_as_float(sv[k + 1]) * sl2 - m) : 0.f;
+          float p0 = (32 * c + k <= vis) ? ex2_approx(__uint_as_float(sv[c][k]) * sl2 - m) : 0.f;
+          float p1 = (32 * c + k + 1 <= vis)
+                         ? ex2_approx(__uint_as_float(sv[c][k + 1]) * sl2 - m)
+                         : 0.f;
           l += p0 + p1;
           pk[k >> 1] = pack_bf16x2(p0, p1);
         }
-        // P_j into the first 16 columns of chunk c of its own buffer
+        // P_j into the first 16 columns of chunk c of its own buffer (chunk c's scores
+        // are already in registers)
         tmem_st16(tS + 32 * c, pk);
       }
       tmem_wait_st();
