@@ -113,6 +113,42 @@ def backward(q, k, v, do, causal: bool, scale: float | None = None, heads=None):
     return dq, dk, dv, delta
 
 
+def forward_gqa(q, k, v, causal: bool, scale: float | None = None):
+    """Grouped-query forward: q [B,H,S,D], k and v [B,Hkv,S,D]; query head h attends
+    with K/V head h // (H // Hkv).  Returns (O [B,H,S,D], LSE [B,H,S]) in float64."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, S, D = q.shape
+    g = H // k.shape[1]
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    o = np.empty((B, H, S, D))
+    lse = np.empty((B, H, S))
+    for b, h in np.ndindex(B, H):
+        o[b, h], lse[b, h] = head_forward(q[b, h], k[b, h // g], v[b, h // g], causal, scale)
+    return o, lse
+
+
+def backward_gqa(q, k, v, do, causal: bool, scale: float | None = None):
+    """Grouped-query backward: dQ [B,H,S,D] per query head; dK and dV [B,Hkv,S,D],
+    each the sum over the K/V head's query heads of that head's dK, dV (the
+    gradient of a K/V head used by several query heads).  float64."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, H, S, D = q.shape
+    Hkv = k.shape[1]
+    g = H // Hkv
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    dq = np.empty((B, H, S, D))
+    dk = np.zeros((B, Hkv, S, D))
+    dv = np.zeros((B, Hkv, S, D))
+    for b, h in np.ndindex(B, H):
+        dq[b, h], dk_h, dv_h, _ = head_backward(q[b, h], k[b, h // g], v[b, h // g], do[b, h],
+                                                causal, scale)
+        dk[b, h // g] += dk_h
+        dv[b, h // g] += dv_h
+    return dq, dk, dv
+
+
 def rel_fro(x, ref) -> float:
     """Relative Frobenius error ||x - ref||_F / ||ref||_F (the parity metric)."""
     x, ref = _f64(x), _f64(ref)
