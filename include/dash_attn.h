@@ -90,6 +90,26 @@ int dash_attn_bwd(const void* q, const void* k, const void* v, const void* o,
                   int B, int H, int S, int D, int causal, int schedule, void* stream);
 
 /*
+ * Grouped-query attention (no counterpart on the pages; their baseline models use
+ * it).  H query heads share Hkv key/value heads, H / Hkv query heads per K/V head
+ * (a power of two): query head h reads K/V head h / (H / Hkv).
+ *   q, o, dout, dq: bf16 [B, H, S, D];  k, v, dk, dv: bf16 [B, Hkv, S, D];
+ *   lse: fp32 [B, H, S].
+ * dK and dV sum over the K/V head's query heads.  The schedule table runs the chains
+ * that feed one dK/dV tile back to back on one CTA, so that sum accumulates in the
+ * kernel's fp32 accumulators in a fixed order (query heads in order) with no extra
+ * reduction; dQ is ordered per query head as for dash_attn_bwd.  Hkv == H is
+ * dash_attn_fwd / dash_attn_bwd.  Errors: DASH_ERR_INVALID_ARG if Hkv < 1 or does not
+ * divide H, DASH_ERR_UNSUPPORTED if H / Hkv is not a power of two; otherwise as
+ * dash_attn_fwd / dash_attn_bwd.
+ */
+int dash_attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                      int H, int Hkv, int S, int D, int causal, void* stream);
+int dash_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
+                      const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                      int H, int Hkv, int S, int D, int causal, int schedule, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device error word of
  * that stream's workspace: DASH_ERR_TIMEOUT if a ticket or pipeline wait of a
  * previous backward on this stream ran out (its outputs are then invalid),
@@ -240,6 +260,17 @@ long long dash_sched_table(int n_heads, int N, int causal, int schedule, int num
  */
 long long dash_sched_table_part(int n_heads, int N, int causal, int schedule, int num_ctas,
                                 int h0, int h1, int* rows, long long cap);
+
+/*
+ * The table of a grouped-query backward: n_heads query heads, `group` per K/V head
+ * (n_heads a multiple of group).  Rows as for dash_sched_table, heads being query
+ * heads; the chains that feed one dK/dV tile (K/V head = head / group, KV tile) are
+ * consecutive on one CTA.  group = 1 gives dash_sched_table's table.  Returns the
+ * number of rows, or -DASH_ERR_INVALID_ARG, -DASH_ERR_UNSUPPORTED or
+ * -DASH_ERR_SCHEDULE.
+ */
+long long dash_sched_table_gqa(int n_heads, int group, int N, int causal, int schedule,
+                               int num_ctas, int* rows, long long cap);
 
 /*
  * DAG simulation of a schedule table (DASH summary §2.1): per pair the events

@@ -23,7 +23,8 @@ EXPORTS = ("dash_attn_fwd", "dash_attn_bwd", "dash_attn_sync_status", "dash_stat
            "dash_sched_table", "dash_sched_simulate", "dash_dag_longest_path",
            "dash_profile_begin", "dash_profile_end", "dash_attn_bwd_noalloc",
            "dash_trace_bwd", "dash_inject_fault", "dash_sched_check", "dash_attn_bwd_host",
-           "dash_sched_table_part")
+           "dash_sched_table_part", "dash_attn_fwd_gqa", "dash_attn_bwd_gqa",
+           "dash_sched_table_gqa")
 
 
 class DashError(RuntimeError):
@@ -55,6 +56,8 @@ def load(path: str | None = None):
     lib.dash_attn_bwd.argtypes = [vp] * 9 + [i, i, i, i, i, i, vp]
     lib.dash_attn_bwd_noalloc.argtypes = [vp] * 9 + [i, i, i, i, i, i, vp]
     lib.dash_attn_bwd_host.argtypes = [vp] * 9 + [i, i, i, i, i, i, vp]
+    lib.dash_attn_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
+    lib.dash_attn_bwd_gqa.argtypes = [vp] * 9 + [i, i, i, i, i, i, i, vp]
     lib.dash_attn_sync_status.argtypes = [vp]
     lib.dash_status_string.argtypes = [i]
     lib.dash_status_string.restype = ctypes.c_char_p
@@ -66,6 +69,8 @@ def load(path: str | None = None):
     lib.dash_sched_table.restype = ll
     lib.dash_sched_table_part.argtypes = [i, i, i, i, i, i, i, vp, ll]
     lib.dash_sched_table_part.restype = ll
+    lib.dash_sched_table_gqa.argtypes = [i, i, i, i, i, i, vp, ll]
+    lib.dash_sched_table_gqa.restype = ll
     lib.dash_sched_simulate.argtypes = [i, i, i, i, i, d, d, i, i, P(d), P(d), P(d), P(ll)]
     lib.dash_sched_check.argtypes = [i, i, i, i, vp, ll]
     lib.dash_dag_longest_path.argtypes = [i, i, vp, vp, vp, vp, vp, P(d)]
@@ -73,7 +78,8 @@ def load(path: str | None = None):
     lib.dash_profile_begin.argtypes = []
     lib.dash_profile_end.argtypes = [P(d), P(d), P(ll)]
     for name in EXPORTS:
-        if name not in ("dash_status_string", "dash_sched_table", "dash_sched_table_part"):
+        if name not in ("dash_status_string", "dash_sched_table", "dash_sched_table_part",
+                        "dash_sched_table_gqa"):
             getattr(lib, name).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -133,6 +139,41 @@ def dash_attn_bwd(q, k, v, o, do, lse, causal: bool, schedule="shift", dq=None, 
                               _ptr(dk), _ptr(dv), B, H, S, D, int(bool(causal)),
                               _sched_id(schedule), _stream_handle(stream))
     _check(rc, "dash_attn_bwd")
+    return dq, dk, dv
+
+
+def dash_attn_fwd_gqa(q, k, v, causal: bool, out=None, lse=None, stream=None):
+    """O, LSE of grouped-query attention: q [B,H,S,D], k and v [B,Hkv,S,D] (bf16
+    CUDA tensors), query head h reading K/V head h // (H // Hkv)."""
+    import torch
+    B, H, S, D = q.shape
+    Hkv = k.shape[1]
+    out = torch.empty_like(q) if out is None else out
+    if lse is None:
+        lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    rc = load().dash_attn_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Hkv, S,
+                                  D, int(bool(causal)), _stream_handle(stream))
+    _check(rc, "dash_attn_fwd_gqa")
+    return out, lse
+
+
+def dash_attn_bwd_gqa(q, k, v, o, do, lse, causal: bool, schedule="shift", dq=None, dk=None,
+                      dv=None, stream=None):
+    """dQ [B,H,S,D], dK and dV [B,Hkv,S,D] of grouped-query attention (dK, dV summed
+    over each K/V head's query heads)."""
+    import torch
+    for t in (q, k, v, o, do, lse):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("inputs must be contiguous CUDA tensors")
+    B, H, S, D = q.shape
+    Hkv = k.shape[1]
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    rc = load().dash_attn_bwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse),
+                                  _ptr(dq), _ptr(dk), _ptr(dv), B, H, Hkv, S, D,
+                                  int(bool(causal)), _sched_id(schedule), _stream_handle(stream))
+    _check(rc, "dash_attn_bwd_gqa")
     return dq, dk, dv
 
 
@@ -225,6 +266,20 @@ def dash_sched_table_part(n_heads: int, N: int, causal: bool, schedule, num_ctas
         raise DashError(int(-n), "dash_sched_table_part")
     buf = (ctypes.c_int * (6 * max(n, 1)))()
     lib.dash_sched_table_part(n_heads, N, int(bool(causal)), sid, num_ctas, h0, h1, buf, n)
+    flat = list(buf)
+    return [tuple(flat[6 * r: 6 * r + 6]) for r in range(n)]
+
+
+def dash_sched_table_gqa(n_heads: int, group: int, N: int, causal: bool, schedule,
+                         num_ctas: int):
+    """Rows (cta, query head, kv, q, position, chain_index) of a grouped-query table."""
+    lib = load()
+    sid = _sched_id(schedule)
+    n = lib.dash_sched_table_gqa(n_heads, group, N, int(bool(causal)), sid, num_ctas, None, 0)
+    if n < 0:
+        raise DashError(int(-n), "dash_sched_table_gqa")
+    buf = (ctypes.c_int * (6 * max(n, 1)))()
+    lib.dash_sched_table_gqa(n_heads, group, N, int(bool(causal)), sid, num_ctas, buf, n)
     flat = list(buf)
     return [tuple(flat[6 * r: 6 * r + 6]) for r in range(n)]
 

@@ -58,6 +58,12 @@
 
 namespace dash {
 
+// Chain word w (pair count) as uploaded: the count in the low 16 bits and two flags for
+// grouped-query attention runs (chains that share one dK/dV tile on one CTA).
+constexpr int kChainCountMask = 0xffff;
+constexpr int kChainContPrev = 1 << 29;
+constexpr int kChainContNext = 1 << 30;
+
 struct BwdParams {
   const int* cta_off;     // [grid + 1]
   const int4* chains;     // {bh, kv, pair_off, pair_cnt}
@@ -71,6 +77,7 @@ struct BwdParams {
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   int S, N, causal;
+  int group_log2;         // log2 of the query heads per K/V head (0: one K/V head each)
   float scale, scale_log2;
   unsigned long long spin_ns;
   // Optional %globaltimer trace (kernels instantiated with kTrace only):
@@ -262,23 +269,35 @@ __global__ void __launch_bounds__(512, 1)
 
   const int cbeg = p.cta_off[blockIdx.x], cend = p.cta_off[blockIdx.x + 1];
   const int S = p.S, N = p.N;
+  // Grouped-query attention: the chains of one dK/dV tile (K/V head, KV tile) run back
+  // to back on this CTA; such a run loads K/V once and carries dK/dV in TMEM from one
+  // chain to the next.  With one K/V head per query head every run is one chain.
+  // The library marks this in the chain's pair-count word (kChainContPrev: the chain
+  // continues the previous chain's run, kChainContNext: the next chain continues its run).
+  const int gl2 = p.group_log2;
+  auto n_pairs = [](int w) { return w & kChainCountMask; };
+  auto cont_prev = [&](int ci) { return (p.chains[ci].w & kChainContPrev) != 0; };
+  auto cont_next = [&](int ci) { return (p.chains[ci].w & kChainContNext) != 0; };
 
   if (warp >= 12) {
     setmaxnreg_dec<C::kRegsCtrl>();
     if (warp == 12 && lane == 0) {
       // ---------------------------------------------------------- TMA producer
-      int it = 0, cn = 0;
-      for (int ci = cbeg; ci < cend; ++ci, ++cn) {
+      int it = 0, kn = 0;  // kn: K/V loads so far
+      for (int ci = cbeg; ci < cend; ++ci) {
         const int4 ch = p.chains[ci];
-        if (cn > 0) wait(BAR(B_KV_EMPTY), (cn - 1) & 1);
-        mbar_expect_tx(BAR(B_KV_FULL), 2 * C::kTile);
-        const int row_kv = ch.x * S + ch.y * 128;
+        if (!(ch.w & kChainContPrev)) {
+          if (kn > 0) wait(BAR(B_KV_EMPTY), (kn - 1) & 1);
+          mbar_expect_tx(BAR(B_KV_FULL), 2 * C::kTile);
+          const int row_kv = (ch.x >> gl2) * S + ch.y * 128;
 #pragma unroll
-        for (int cb = 0; cb < D / 64; ++cb) {
-          tma_load_2d(sK + cb * 16384, &tmK, cb * 64, row_kv, BAR(B_KV_FULL));
-          tma_load_2d(sV + cb * 16384, &tmV, cb * 64, row_kv, BAR(B_KV_FULL));
+          for (int cb = 0; cb < D / 64; ++cb) {
+            tma_load_2d(sK + cb * 16384, &tmK, cb * 64, row_kv, BAR(B_KV_FULL));
+            tma_load_2d(sV + cb * 16384, &tmV, cb * 64, row_kv, BAR(B_KV_FULL));
+          }
+          ++kn;
         }
-        for (int t = 0; t < ch.w; ++t, ++it) {
+        for (int t = 0; t < n_pairs(ch.w); ++t, ++it) {
           const int q = (int)(p.pairs[ch.z + t] & 0xffffu);
           const int s = it % ST, sd = it % SD;
           const int row_q = ch.x * S + q * 128;
@@ -306,7 +325,7 @@ __global__ void __launch_bounds__(512, 1)
         const int last_use = ((it - 1 - s) / SD) * SD + s;
         drain(DO_FULL(s), (last_use / SD) & 1);
       }
-      if (cn > 0) drain(BAR(B_KV_FULL), (cn - 1) & 1);
+      if (kn > 0) drain(BAR(B_KV_FULL), (kn - 1) & 1);
     } else if (warp == 13 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
       // One thread issues every MMA; its instruction stream between MMAs is the
@@ -362,10 +381,11 @@ __global__ void __launch_bounds__(512, 1)
           tc_mma_ss_w(tDP, kOnesDP, kCol, hi_none, ID_SS, 1u);  // - Delta
           tc_commit(BAR(B_DP_FULL));
         };
-        int it = 0, cn = 0;
-        for (int ci = cbeg; ci < cend; ++ci, ++cn) {
-          const int cnt = p.chains[ci].w;
-          wait(BAR(B_KV_FULL), cn & 1);
+        int it = 0, kn = 0;  // kn: runs started (K/V loads consumed)
+        for (int ci = cbeg; ci < cend; ++ci) {
+          const int cnt = n_pairs(p.chains[ci].w);
+          const bool cprev = cont_prev(ci);
+          if (!cprev) wait(BAR(B_KV_FULL), (kn++) & 1);
           tc_fence_after();
           if (cnt > 0) {
             issue_s(it);
@@ -382,9 +402,10 @@ __global__ void __launch_bounds__(512, 1)
             const uint32_t tSi = tS + s_col(it);
             // dV += P^T dO (A in TMEM), once P is packed
             wait(P_READY(it), s_phase(it));
-            if (t == 0 && cn > 0) wait(BAR(B_DKDV_EMPTY), (cn - 1) & 1);
+            // a run's first chain: the previous run's dV/dK must have been read out
+            if (t == 0 && !cprev && kn >= 2) wait(BAR(B_DKDV_EMPTY), (kn - 2) & 1);
             tc_fence_after();
-            const uint32_t acc0 = t > 0 ? 1u : 0u;
+            const uint32_t acc0 = (t > 0 || cprev) ? 1u : 0u;
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
               tc_mma_ts_w(tDV, tSi + 32 * (kk >> 1) + 8 * (kk & 1), mDO + kk * 128, hi, ID_KV,
@@ -412,17 +433,19 @@ __global__ void __launch_bounds__(512, 1)
             }
             tc_commit(Q_EMPTY(s));
             tc_commit(BAR(B_DS_FREE));  // dQp and dK have read dS^T
-            if (t == cnt - 1) tc_commit(BAR(B_DKDV_FULL));
+            if (t == cnt - 1 && !cont_next(ci)) tc_commit(BAR(B_DKDV_FULL));
             trace(it, 2);
             if (t + 2 < cnt) issue_s(it + 2);
           }
-          tc_commit(BAR(B_KV_EMPTY));
+          // the run's last chain: K/V are done with
+          if (!cont_next(ci)) tc_commit(BAR(B_KV_EMPTY));
         }
       } else {
-        int it = 0, cn = 0;
-        for (int ci = cbeg; ci < cend; ++ci, ++cn) {
-          const int cnt = p.chains[ci].w;
-          wait(BAR(B_KV_FULL), cn & 1);
+        int it = 0, kn = 0;  // kn: runs started (K/V loads consumed)
+        for (int ci = cbeg; ci < cend; ++ci) {
+          const int cnt = n_pairs(p.chains[ci].w);
+          const bool cprev = cont_prev(ci);
+          if (!cprev) wait(BAR(B_KV_FULL), (kn++) & 1);
           tc_fence_after();
           // t = -1 only issues the chain's first S^T/dP^T; each later step finishes
           // tile `it` and then issues S^T/dP^T of the next tile behind it
@@ -433,10 +456,10 @@ __global__ void __launch_bounds__(512, 1)
               const uint32_t mDO = sdesc_lo(sDO + sd * C::kTile, 16384);
               // dV += P^T dO : M = kv, N = D, K = q (A in TMEM, B MN-major), once P is packed
               wait(BAR(B_P_READY), it & 1);
-              // the previous chain's dV/dK must have been read out before they restart
-              if (t == 0 && cn > 0) wait(BAR(B_DKDV_EMPTY), (cn - 1) & 1);
+              // a run's first chain: the previous run's dV/dK must have been read out
+              if (t == 0 && !cprev && kn >= 2) wait(BAR(B_DKDV_EMPTY), (kn - 2) & 1);
               tc_fence_after();
-              const uint32_t acc0 = t > 0 ? 1u : 0u;
+              const uint32_t acc0 = (t > 0 || cprev) ? 1u : 0u;
   #pragma unroll
               for (int kk = 0; kk < 8; ++kk)
                 tc_mma_ts_w(tDV, tS + 32 * (kk >> 1) + 8 * (kk & 1), mDO + kk * 128, hi, ID_KV,
@@ -452,7 +475,7 @@ __global__ void __launch_bounds__(512, 1)
                             kk > 0 ? 1u : acc0);
               tc_commit(Q_EMPTY(s));
               tc_commit(BAR(B_DVDK_DONE));
-              if (t == cnt - 1) tc_commit(BAR(B_DKDV_FULL));
+              if (t == cnt - 1 && !cont_next(ci)) tc_commit(BAR(B_DKDV_FULL));
               // dQp = dS K : M = q, N = D, K = kv (both operands MN-major)
               const int buf = C::kDqInDp ? 0 : (it & 1);
               if (!C::kDqInDp && it >= 2) {
@@ -502,7 +525,8 @@ __global__ void __launch_bounds__(512, 1)
               tc_commit(BAR(B_DP_FULL));
             }
           }
-          tc_commit(BAR(B_KV_EMPTY));
+          // the run's last chain: K/V are done with
+          if (!cont_next(ci)) tc_commit(BAR(B_KV_EMPTY));
         }
       }
       // drain: all issued MMAs complete before TMEM is released
@@ -519,7 +543,7 @@ __global__ void __launch_bounds__(512, 1)
       int it = 0, k = 0;
       for (int ci = cbeg; ci < cend; ++ci) {
         const int4 ch = p.chains[ci];
-        for (int t = 0; t < ch.w; ++t, ++it) {
+        for (int t = 0; t < n_pairs(ch.w); ++t, ++it) {
           const uint32_t w = p.pairs[ch.z + t];
           const int q = (int)(w & 0xffffu), pos = (int)(w >> 16);
           const int ncontrib = p.causal ? q + 1 : N;
@@ -548,7 +572,7 @@ __global__ void __launch_bounds__(512, 1)
     int it = 0;
     for (int ci = cbeg; ci < cend; ++ci) {
       const int4 ch = p.chains[ci];
-      for (int t = 0; t < ch.w; ++t, ++it) {
+      for (int t = 0; t < n_pairs(ch.w); ++t, ++it) {
         const int q = (int)(p.pairs[ch.z + t] & 0xffffu);
         const uint32_t tS = tS0 + s_col(it);
         wait(S_FULL(it), s_phase(it));
@@ -628,11 +652,11 @@ __global__ void __launch_bounds__(512, 1)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     constexpr int NV = D / 4;           // float4 per row
     constexpr int G = 24;               // loads in flight per group
-    int it = 0, cn = 0;
-    int npub = 0;  // pairs handed to the publisher
-    for (int ci = cbeg; ci < cend; ++ci, ++cn) {
+    int it = 0, fn = 0;  // fn: dK/dV runs written out
+    int npub = 0;        // pairs handed to the publisher
+    for (int ci = cbeg; ci < cend; ++ci) {
       const int4 ch = p.chains[ci];
-      for (int t = 0; t < ch.w; ++t, ++it) {
+      for (int t = 0; t < n_pairs(ch.w); ++t, ++it) {
         const uint32_t w = p.pairs[ch.z + t];
         const int q = (int)(w & 0xffffu), pos = (int)(w >> 16);
         const int ncontrib = p.causal ? q + 1 : N;
@@ -754,10 +778,12 @@ __global__ void __launch_bounds__(512, 1)
         }
         if (threadIdx.x == 256 && (kAtomic || last || !C::kPublisher)) trace(it, 7);
       }
-      // chain epilogue: dV_j and scale * dK_j (rows of KV tile ch.y) to global bf16
-      wait(BAR(B_DKDV_FULL), cn & 1);
+      // run epilogue: dV_j and scale * dK_j (rows of KV tile ch.y of the chain's K/V
+      // head) to global bf16, after the run's last chain
+      if (ch.w & kChainContNext) continue;
+      wait(BAR(B_DKDV_FULL), (fn++) & 1);
       tc_fence_after();
-      const size_t row = (size_t)ch.x * S + (size_t)ch.y * 128 + r;
+      const size_t row = (size_t)(ch.x >> gl2) * S + (size_t)ch.y * 128 + r;
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         const uint32_t col = which ? C::TM_DK : C::TM_DV;

@@ -61,7 +61,7 @@ struct DevTable {
 
 std::mutex g_mu;
 std::map<std::pair<int, uintptr_t>, Workspace> g_ws;                  // (device, stream)
-std::map<std::tuple<int, int, int, int, int, int>, DevTable> g_tables;  // device,heads,N,causal,sched,ctas
+std::map<std::tuple<int, int, int, int, int, int, int>, DevTable> g_tables;  // device,heads,N,causal,sched,ctas,group
 std::map<std::pair<int, int>, int> g_num_ctas;                        // (device, D)
 
 // Optional per-launch device timing: while enabled, each backward records four
@@ -126,8 +126,25 @@ void free_table(DevTable* d) {
   *d = DevTable{};
 }
 
+// The device copy of a table's chains: the pair count of each chain carries the
+// kernel's run flags (a run: consecutive chains of one CTA that feed one dK/dV tile,
+// which only grouped-query tables have).
+std::vector<dash::Chain> device_chains(const dash::Table& t) {
+  std::vector<dash::Chain> c = t.chains;
+  auto same = [&](int a, int b) {
+    return t.chains[a].bh / t.group == t.chains[b].bh / t.group && t.chains[a].kv == t.chains[b].kv;
+  };
+  for (int k = 0; k < t.num_ctas; ++k)
+    for (int i = t.cta_off[k]; i < t.cta_off[k + 1]; ++i) {
+      if (i > t.cta_off[k] && same(i - 1, i)) c[i].pair_cnt |= dash::kChainContPrev;
+      if (i + 1 < t.cta_off[k + 1] && same(i, i + 1)) c[i].pair_cnt |= dash::kChainContNext;
+    }
+  return c;
+}
+
 int upload_table(const dash::Table& t, DevTable* out) {
   DevTable d;
+  const std::vector<dash::Chain> chains = device_chains(t);
   // an empty chain or pair list still gets a valid (unused) allocation
   const size_t nc = t.chains.empty() ? 1 : t.chains.size();
   const size_t np = t.pairs.empty() ? 1 : t.pairs.size();
@@ -141,8 +158,8 @@ int upload_table(const dash::Table& t, DevTable* out) {
   static_assert(sizeof(dash::Chain) == sizeof(int4), "chain layout");
   if (cudaMemcpy(d.cta_off, t.cta_off.data(), t.cta_off.size() * sizeof(int),
                  cudaMemcpyHostToDevice) != cudaSuccess ||
-      (!t.chains.empty() &&
-       cudaMemcpy(d.chains, t.chains.data(), t.chains.size() * sizeof(int4),
+      (!chains.empty() &&
+       cudaMemcpy(d.chains, chains.data(), chains.size() * sizeof(int4),
                   cudaMemcpyHostToDevice) != cudaSuccess) ||
       (!t.pairs.empty() && cudaMemcpy(d.pairs, t.pairs.data(), t.pairs.size() * sizeof(uint32_t),
                                       cudaMemcpyHostToDevice) != cudaSuccess)) {
@@ -153,8 +170,9 @@ int upload_table(const dash::Table& t, DevTable* out) {
   return DASH_OK;
 }
 
-int get_table(int dev, int heads, int N, int causal, int sched, int ctas, DevTable** out) {
-  auto key = std::make_tuple(dev, heads, N, causal, sched, ctas);
+int get_table(int dev, int heads, int N, int causal, int sched, int ctas, DevTable** out,
+              int group = 1) {
+  auto key = std::make_tuple(dev, heads, N, causal, sched, ctas, group);
   auto itb = g_tables.find(key);
   if (itb != g_tables.end()) {
     *out = &itb->second;
@@ -162,7 +180,8 @@ int get_table(int dev, int heads, int N, int causal, int sched, int ctas, DevTab
   }
   dash::Table t;
   std::string err;
-  if (!dash::build_table(heads, N, causal, sched, ctas, &t, &err)) return DASH_ERR_UNSUPPORTED;
+  if (!dash::build_table_grouped(heads, group, N, causal, sched, ctas, &t, &err))
+    return DASH_ERR_UNSUPPORTED;
   if (!dash::validate_table(t, &err)) return DASH_ERR_SCHEDULE;
   DevTable d;
   int rc = upload_table(t, &d);
@@ -335,7 +354,7 @@ template <int D, bool kAtomic, bool kTrace = false>
 int launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                const float* lse, void* dq, void* dk, void* dv, int B, int H, int S, int causal,
                int sched, cudaStream_t stream, int dev, unsigned long long* trace = nullptr,
-               int trace_rows = 0, const DevTable* tab_override = nullptr) {
+               int trace_rows = 0, const DevTable* tab_override = nullptr, int group = 1) {
   using C = BwdCfg<D>;
   const int N = S / 128;
   const long long rows = (long long)B * H * S;
@@ -346,12 +365,13 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   Workspace* ws = nullptr;
   {
     std::lock_guard<std::mutex> lk(g_mu);
-    const int fault = tab_override ? 0 : g_fault.exchange(0);
+    // an armed fault is kept for a multi-head call (its table has no run flags)
+    const int fault = (tab_override || group > 1) ? 0 : g_fault.exchange(0);
     if (tab_override) {
       tab = const_cast<DevTable*>(tab_override);
     } else if (fault == 1 && !kAtomic) {
       if ((rc = get_fault_table(dev, B * H, N, causal, sched, ctas, &tab))) return rc;
-    } else if ((rc = get_table(dev, B * H, N, causal, sched, ctas, &tab))) {
+    } else if ((rc = get_table(dev, B * H, N, causal, sched, ctas, &tab, group))) {
       return rc;
     }
     if ((rc = get_workspace(dev, stream, 2 * (size_t)rows * D * sizeof(float),
@@ -361,8 +381,8 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   }
   CUtensorMap tq, tk, tv, tdo, tc;
   if ((rc = make_tmap(&tq, q, rows, D, C::kQRows)) ||
-      (rc = make_tmap(&tk, k, rows, D, C::kKVRows)) ||
-      (rc = make_tmap(&tv, v, rows, D, C::kKVRows)) ||
+      (rc = make_tmap(&tk, k, rows / group, D, C::kKVRows)) ||
+      (rc = make_tmap(&tv, v, rows / group, D, C::kKVRows)) ||
       (rc = make_tmap(&tdo, dout, rows, D, C::kQRows)) ||
       (rc = make_tmap_cols(&tc, ws->rowbuf, rows)))
     return rc;
@@ -390,6 +410,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   p.S = S;
   p.N = N;
   p.causal = causal;
+  p.group_log2 = __builtin_ctz((unsigned)group);
   p.scale = scale;
   p.scale_log2 = p.scale * 1.4426950408889634f;
   p.spin_ns = (unsigned long long)spin_us() * 1000ull;
@@ -436,7 +457,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
 // ------------------------------------------------------------------ forward
 template <int D>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-               int S, int causal, cudaStream_t stream, int dev) {
+               int S, int causal, cudaStream_t stream, int dev, int group = 1) {
   using C = dash::FwdCfg<D>;
   const int N = S / 128;
   const long long rows = (long long)B * H * S;
@@ -448,8 +469,8 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     if ((rc = get_workspace(dev, stream, 0, 0, 0, &ws))) return rc;
   }
   CUtensorMap tq, tk, tv;
-  if ((rc = make_tmap(&tq, q, rows, D, 128)) || (rc = make_tmap(&tk, k, rows, D, 128)) ||
-      (rc = make_tmap(&tv, v, rows, D, 128)))
+  if ((rc = make_tmap(&tq, q, rows, D, 128)) || (rc = make_tmap(&tk, k, rows / group, D, 128)) ||
+      (rc = make_tmap(&tv, v, rows / group, D, 128)))
     return rc;
   auto kern = dash::dash_fwd_tc_kernel<D>;
   DASH_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes));
@@ -461,6 +482,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   p.S = S;
   p.N = N;
   p.BH = B * H;
+  p.group = group;
   p.causal = causal;
   p.scale_log2 = (1.0f / sqrtf((float)D)) * 1.4426950408889634f;
   p.spin_ns = (unsigned long long)spin_us() * 1000ull;
@@ -618,27 +640,36 @@ int dash_set_spin_limit_us(long long us) {
   return DASH_OK;
 }
 
-int dash_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-                  int S, int D, int causal, void* stream) {
+int dash_attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                      int H, int Hkv, int S, int D, int causal, void* stream) {
   int rc = check_shape(B, H, S, D);
   if (rc) return rc;
   if (causal != 0 && causal != 1) return DASH_ERR_INVALID_ARG;
+  if (H > 0 && (Hkv < 1 || H % Hkv != 0)) return DASH_ERR_INVALID_ARG;
+  if (H > 0 && ((H / Hkv) & (H / Hkv - 1)) != 0) return DASH_ERR_UNSUPPORTED;  // 2^k per K/V head
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !lse)
     return DASH_ERR_INVALID_ARG;
   if (B == 0 || H == 0) return DASH_OK;
   int dev = 0;
   DASH_CUDA(cudaGetDevice(&dev));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return D == 64 ? launch_fwd<64>(q, k, v, o, lse, B, H, S, causal, st, dev)
-                 : launch_fwd<128>(q, k, v, o, lse, B, H, S, causal, st, dev);
+  return D == 64 ? launch_fwd<64>(q, k, v, o, lse, B, H, S, causal, st, dev, H / Hkv)
+                 : launch_fwd<128>(q, k, v, o, lse, B, H, S, causal, st, dev, H / Hkv);
 }
 
-int dash_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
-                  const float* lse, void* dq, void* dk, void* dv, int B, int H, int S, int D,
-                  int causal, int schedule, void* stream) {
+int dash_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                  int S, int D, int causal, void* stream) {
+  return dash_attn_fwd_gqa(q, k, v, o, lse, B, H, H, S, D, causal, stream);
+}
+
+int dash_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
+                      const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                      int H, int Hkv, int S, int D, int causal, int schedule, void* stream) {
   int rc = check_shape(B, H, S, D);
   if (rc) return rc;
   if (causal != 0 && causal != 1) return DASH_ERR_INVALID_ARG;
+  if (H > 0 && (Hkv < 1 || H % Hkv != 0)) return DASH_ERR_INVALID_ARG;
+  if (H > 0 && ((H / Hkv) & (H / Hkv - 1)) != 0) return DASH_ERR_UNSUPPORTED;  // 2^k per K/V head
   if (schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_ATOMIC) return DASH_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
       !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
@@ -649,15 +680,23 @@ int dash_attn_bwd(const void* q, const void* k, const void* v, const void* o, co
   DASH_CUDA(cudaGetDevice(&dev));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool atomic = (schedule == DASH_SCHED_ATOMIC);
+  const int g = H / Hkv;
   if (D == 64)
     return atomic ? launch_bwd<64, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
-                                         schedule, st, dev)
+                                         schedule, st, dev, nullptr, 0, nullptr, g)
                   : launch_bwd<64, false>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
-                                          schedule, st, dev);
+                                          schedule, st, dev, nullptr, 0, nullptr, g);
   return atomic ? launch_bwd<128, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
-                                        schedule, st, dev)
+                                        schedule, st, dev, nullptr, 0, nullptr, g)
                 : launch_bwd<128, false>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
-                                         schedule, st, dev);
+                                         schedule, st, dev, nullptr, 0, nullptr, g);
+}
+
+int dash_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                  const float* lse, void* dq, void* dk, void* dv, int B, int H, int S, int D,
+                  int causal, int schedule, void* stream) {
+  return dash_attn_bwd_gqa(q, k, v, o, dout, lse, dq, dk, dv, B, H, H, S, D, causal, schedule,
+                           stream);
 }
 
 int dash_attn_bwd_host(const void* q, const void* k, const void* v, const void* o,
@@ -858,6 +897,34 @@ int dash_trace_bwd(const void* q, const void* k, const void* v, const void* o, c
   *num_ctas = ctas;
   *rows_per_cta = rows;
   return rc;
+}
+
+long long dash_sched_table_gqa(int n_heads, int group, int N, int causal, int schedule,
+                               int num_ctas, int* rows, long long cap) {
+  dash::Table t;
+  std::string err;
+  if (group < 1 || n_heads < 1 || n_heads % group != 0) return -DASH_ERR_INVALID_ARG;
+  if (!dash::build_table_grouped(n_heads, group, N, causal, schedule, num_ctas, &t, &err))
+    return -DASH_ERR_UNSUPPORTED;
+  if (!dash::validate_table(t, &err)) return -DASH_ERR_SCHEDULE;
+  long long n = 0;
+  for (int c = 0; c < t.num_ctas; ++c)
+    for (int ci = t.cta_off[c]; ci < t.cta_off[c + 1]; ++ci) {
+      const dash::Chain& ch = t.chains[ci];
+      for (int i = 0; i < ch.pair_cnt; ++i, ++n) {
+        if (rows && n < cap) {
+          const uint32_t w = t.pairs[ch.pair_off + i];
+          int* r = rows + 6 * n;
+          r[0] = c;
+          r[1] = ch.bh;
+          r[2] = ch.kv;
+          r[3] = dash::pair_q(w);
+          r[4] = dash::pair_pos(w);
+          r[5] = ci;
+        }
+      }
+    }
+  return n;
 }
 
 long long dash_sched_table_part(int n_heads, int N, int causal, int schedule, int num_ctas,

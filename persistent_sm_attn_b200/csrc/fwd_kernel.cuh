@@ -29,6 +29,7 @@ struct FwdParams {
   unsigned* err;         // device error word (shared with the backward's workspace)
   unsigned* abort_flag;  // cleared before each launch
   int S, N, BH, causal;
+  int group;             // query heads per K/V head
   float scale_log2;      // scale * log2(e)
   unsigned long long spin_ns;
 };
@@ -130,7 +131,7 @@ __global__ void __launch_bounds__(256, 1)
       const int s = j % KST;
       if (j >= KST) wait(KV_EMPTY(s), (uint32_t)(((j / KST) - 1) & 1));
       mbar_expect_tx(KV_FULL(s), 2 * C::kTile);
-      const int row_kv = bh * S + j * 128;
+      const int row_kv = (bh / p.group) * S + j * 128;
 #pragma unroll
       for (int cb = 0; cb < D / 64; ++cb) {
         tma_load_2d(sK + s * C::kTile + cb * 16384, &tmK, cb * 64, row_kv, KV_FULL(s));

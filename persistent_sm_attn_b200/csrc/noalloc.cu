@@ -221,6 +221,7 @@ int noalloc_launch(const void* q, const void* k, const void* v, const void* o, c
   p.S = S;
   p.N = N;
   p.causal = causal;
+  p.group_log2 = 0;
   p.scale = scale;
   p.scale_log2 = p.scale * 1.4426950408889634f;
   p.spin_ns = noalloc_spin_ns();

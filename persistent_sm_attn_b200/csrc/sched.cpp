@@ -94,40 +94,60 @@ std::vector<std::vector<std::pair<int, int>>> head_units(int schedule, int N, in
 
 bool build_table(int n_heads, int N, int causal, int schedule, int num_ctas, Table* out,
                  std::string* err) {
-  if (n_heads < 1 || num_ctas < 1 || !schedule_supported(schedule, N, causal)) {
-    if (err) *err = "schedule not defined for this mask / tile count";
+  return build_table_grouped(n_heads, 1, N, causal, schedule, num_ctas, out, err);
+}
+
+bool build_table_grouped(int n_heads, int group, int N, int causal, int schedule,
+                         int num_ctas, Table* out, std::string* err) {
+  if (n_heads < 1 || num_ctas < 1 || group < 1 || n_heads % group != 0 ||
+      !schedule_supported(schedule, N, causal)) {
+    if (err) *err = "schedule not defined for this mask / tile count / head grouping";
     return false;
   }
   const Units units = units_of(schedule, N, causal);
   const int U = (int)units.size();
-  // Positions within each dQ block, per head.  NAIVE_ASC / DESCENDING order a
-  // block by KV; SHIFT / SYM_SHIFT / ATOMIC by execution order: the round in
-  // which the unit runs (global unit g runs in round g / num_ctas), then the
-  // step.  The round only matters for heads whose units span two rounds;
-  // heads with the same first-unit offset in their round share one table.
+  // Group unit k: unit k's KV segments in order, each run for query heads 0..group-1
+  // of the K/V head in turn.  Entries (query head offset, kv, q) in execution order.
+  struct Step { int head, kv, q; };
+  std::vector<std::vector<Step>> gunits(U);
+  for (int k = 0; k < U; ++k) {
+    const auto& seq = units[k];
+    for (int a = 0; a < (int)seq.size();) {
+      int b = a;
+      while (b < (int)seq.size() && seq[b].first == seq[a].first) ++b;
+      for (int h = 0; h < group; ++h)
+        for (int i = a; i < b; ++i) gunits[k].push_back({h, seq[i].first, seq[i].second});
+      a = b;
+    }
+  }
+  // Positions within each dQ block, per query head.  NAIVE_ASC / DESCENDING order a
+  // block by KV; SHIFT / SYM_SHIFT / ATOMIC by execution order: the round in which
+  // the unit runs (global unit g runs in round g / num_ctas), then the step within
+  // the unit.  The round only matters for K/V heads whose units span two rounds;
+  // K/V heads with the same first-unit offset in their round share one table.
   const bool by_kv = (schedule == NAIVE_ASC || schedule == DESCENDING);
   auto head_positions = [&](long long first_g) {
-    std::vector<std::vector<std::pair<long long, int>>> contrib(N);  // per q: (key, unit*65536+step)
+    // per (query head offset, q): (key, unit * 65536 + step)
+    std::vector<std::vector<std::pair<long long, int>>> contrib((size_t)group * N);
     for (int k = 0; k < U; ++k) {
       const long long rnd = (first_g + k) / num_ctas - first_g / num_ctas;
-      for (int t = 0; t < (int)units[k].size(); ++t) {
-        const int kv = units[k][t].first, q = units[k][t].second;
-        const long long key = by_kv ? kv : (rnd << 40) + (long long)t * 65536 + k;
-        contrib[q].push_back({key, k * 65536 + t});
+      for (int t = 0; t < (int)gunits[k].size(); ++t) {
+        const Step& st = gunits[k][t];
+        const long long key = by_kv ? st.kv : (rnd << 40) + (long long)t * 65536 + k;
+        contrib[(size_t)st.head * N + st.q].push_back({key, k * 65536 + t});
       }
     }
     std::vector<std::vector<int>> pos(U);
-    for (int k = 0; k < U; ++k) pos[k].assign(units[k].size(), -1);
-    for (int q = 0; q < N; ++q) {
-      auto& c = contrib[q];
+    for (int k = 0; k < U; ++k) pos[k].assign(gunits[k].size(), -1);
+    for (auto& c : contrib) {
       std::sort(c.begin(), c.end());
       for (int p = 0; p < (int)c.size(); ++p) pos[c[p].second >> 16][c[p].second & 0xffff] = p;
     }
     return pos;
   };
   std::map<long long, std::vector<std::vector<int>>> pos_by_offset;
-  auto positions_of = [&](int bh) -> const std::vector<std::vector<int>>& {
-    const long long first_g = (long long)bh * U;
+  auto positions_of = [&](int kvh) -> const std::vector<std::vector<int>>& {
+    const long long first_g = (long long)kvh * U;
     const long long key = by_kv ? 0 : first_g % num_ctas;
     auto f = pos_by_offset.find(key);
     if (f == pos_by_offset.end()) f = pos_by_offset.emplace(key, head_positions(first_g)).first;
@@ -135,24 +155,26 @@ bool build_table(int n_heads, int N, int causal, int schedule, int num_ctas, Tab
   };
   Table t;
   t.n_heads = n_heads; t.N = N; t.causal = causal; t.schedule = schedule; t.num_ctas = num_ctas;
+  t.group = group;
   // per CTA, the global units it runs, in round order
   std::vector<std::vector<long long>> per_cta(num_ctas);
-  const long long total_units = (long long)n_heads * U;
+  const long long total_units = (long long)(n_heads / group) * U;
   for (long long g = 0; g < total_units; ++g) per_cta[g % num_ctas].push_back(g);
   t.cta_off.assign(num_ctas + 1, 0);
   for (int c = 0; c < num_ctas; ++c) {
     t.cta_off[c] = (int32_t)t.chains.size();
     for (long long g : per_cta[c]) {
-      const int bh = (int)(g / U), k = (int)(g % U);
-      const auto& seq = units[k];
-      const auto& pos = positions_of(bh);
+      const int kvh = (int)(g / U), k = (int)(g % U);
+      const auto& seq = gunits[k];
+      const auto& pos = positions_of(kvh);
       for (int i = 0; i < (int)seq.size(); ++i) {
-        if (i == 0 || seq[i].first != seq[i - 1].first) {
-          Chain ch{bh, seq[i].first, (int32_t)t.pairs.size(), 0};
+        const int bh = kvh * group + seq[i].head;
+        if (i == 0 || seq[i].kv != seq[i - 1].kv || seq[i].head != seq[i - 1].head) {
+          Chain ch{bh, seq[i].kv, (int32_t)t.pairs.size(), 0};
           t.chains.push_back(ch);
         }
         t.chains.back().pair_cnt++;
-        t.pairs.push_back(pack_pair(seq[i].second, pos[k][i]));
+        t.pairs.push_back(pack_pair(seq[i].q, pos[k][i]));
       }
     }
   }
@@ -193,12 +215,14 @@ bool table_from_rows(int n_heads, int N, int causal, int num_ctas, const int* ro
 
 bool split_table(const Table& full, int h0, int h1, Table* out) {
   if (h0 < 0 || h1 <= h0 || h1 > full.n_heads) return false;
+  if (h0 % full.group != 0 || h1 % full.group != 0) return false;  // whole K/V heads only
   Table t;
   t.n_heads = h1 - h0;
   t.N = full.N;
   t.causal = full.causal;
   t.schedule = full.schedule;
   t.num_ctas = full.num_ctas;
+  t.group = full.group;
   t.cta_off.assign(full.num_ctas + 1, 0);
   for (int c = 0; c < full.num_ctas; ++c) {
     for (int i = full.cta_off[c]; i < full.cta_off[c + 1]; ++i) {
@@ -253,6 +277,22 @@ bool validate_table(const Table& t, std::string* err) {
         n_contrib[blk]++;
       }
     }
+  }
+  if (t.group < 1 || t.n_heads % t.group != 0) return fail("bad head grouping");
+  if (t.group > 1) {
+    // the chains of one dK/dV tile (K/V head, KV tile) must run back to back on one CTA
+    std::vector<uint8_t> run_done((size_t)(t.n_heads / t.group) * N, 0);
+    for (int c = 0; c < t.num_ctas; ++c)
+      for (int ci = t.cta_off[c]; ci < t.cta_off[c + 1]; ++ci) {
+        const Chain& ch = t.chains[ci];
+        const size_t key = (size_t)(ch.bh / t.group) * N + ch.kv;
+        const bool cont = ci > t.cta_off[c] && t.chains[ci - 1].bh / t.group == ch.bh / t.group &&
+                          t.chains[ci - 1].kv == ch.kv;
+        if (!cont) {
+          if (run_done[key]) return fail("chains of one dK/dV tile split into two runs");
+          run_done[key] = 1;
+        }
+      }
   }
   for (long long blk = 0; blk < nblk; ++blk) {
     const int q = (int)(blk % N);

@@ -30,6 +30,7 @@ inline int pair_pos(uint32_t w) { return int(w >> 16); }
 
 struct Table {
   int n_heads = 0, N = 0, causal = 0, schedule = 0, num_ctas = 0;
+  int group = 1;  // query heads per K/V head (grouped-query attention); 1 = one K/V head each
   std::vector<int32_t> cta_off;   // num_ctas + 1 offsets into chains
   std::vector<Chain> chains;      // grouped by CTA, in execution order
   std::vector<uint32_t> pairs;    // packed (q, position)
@@ -48,6 +49,16 @@ std::vector<std::vector<std::pair<int, int>>> head_units(int schedule, int N, in
 // Returns false (with a message) if the combination is unsupported.
 bool build_table(int n_heads, int N, int causal, int schedule, int num_ctas, Table* out,
                  std::string* err);
+
+// The same for grouped-query attention: n_heads query heads, `group` of them per
+// K/V head (n_heads a multiple of group).  A unit covers one K/V head's KV tile (or
+// tiles) for all its query heads: each KV segment of the unit runs for every query
+// head of the group in turn, so the chains that feed one dK/dV tile run back to back
+// on one CTA and the kernel carries the accumulators across them.  Positions follow
+// the same keys (round, then step within the unit); group = 1 gives build_table's
+// table.
+bool build_table_grouped(int n_heads, int group, int N, int causal, int schedule,
+                         int num_ctas, Table* out, std::string* err);
 
 // Checks coverage (every allowed pair once), positions (a permutation per dQ
 // block), unbroken chains, pair-word ranges, and deadlock freedom of the

@@ -64,6 +64,17 @@ def test_argument_errors_need_no_gpu(lib):
     assert lib.dash_attn_bwd_host(*null, 1, 1, 128, 64, 0, 2, None) == 1
     assert lib.dash_attn_bwd_host(*good, 1, 1, 128, 96, 0, 2, None) == 2
     assert lib.dash_attn_bwd_host(*good, 1, 1, 128, 64, 1, 2, None) == 2
+    # grouped-query entries: Hkv must divide H, with a power-of-two group
+    gqa_b = lambda H, Hkv, S=128, D=64: lib.dash_attn_bwd_gqa(*good, 1, H, Hkv, S, D, 0, 2, None)
+    gqa_f = lambda H, Hkv: lib.dash_attn_fwd_gqa(*good[:5], 1, H, Hkv, 128, 64, 0, None)
+    for fn in (gqa_b, gqa_f):
+        assert fn(4, 3) == 1                          # 3 does not divide 4
+        assert fn(4, 0) == 1
+        assert fn(4, -2) == 1
+        assert fn(6, 2) == 2                          # 3 query heads per K/V head
+        assert fn(12, 1) == 2
+    assert gqa_b(8, 2, D=96) == 2
+    assert lib.dash_attn_bwd_gqa(*null, 1, 8, 2, 128, 64, 0, 2, None) == 1
     # a part outside the table's heads
     for h0, h1 in ((0, 0), (2, 1), (-1, 1), (0, 5)):
         assert lib.dash_sched_table_part(4, 4, 0, 2, 8, h0, h1, None, 0) == -1

@@ -1,0 +1,123 @@
+"""Grouped-query schedule tables (dash_sched_table_gqa).
+
+With a group of g query heads per K/V head, a CTA runs each KV segment of a unit
+for the g query heads in turn, so the dK/dV tile of that segment stays on one SM
+for the whole group.  These tests check, without a GPU:
+- group 1 gives the multi-head table;
+- every (query head, kv, q) pair of the mask appears once, and every dQ block's
+  positions are 0..n-1;
+- each K/V head's KV tile is one run of consecutive chains on one CTA, the group's
+  query heads in order, each with the multi-head unit's Q tiles for that segment;
+- the table's dependence graph (the oracle's event graph, two accumulation
+  chains per block as the kernel runs it) has no cycle, so no CTA waits forever;
+- the library's own validator accepts the rows.
+"""
+from collections import defaultdict
+
+import pytest
+
+from oracle import dag, schedules as sc
+from persistent_sm_attn_b200 import binding
+
+SID = {sc.NAIVE_ASC: "naive_asc", sc.DESCENDING: "descending", sc.SHIFT: "shift",
+       sc.SYM_SHIFT: "sym_shift"}
+
+
+def _mask_pairs(N, causal):
+    return [(kv, q) for kv in range(N) for q in range(N) if not causal or q >= kv]
+
+
+def _acyclic(n_nodes, edges):
+    indeg = [0] * n_nodes
+    out = defaultdict(list)
+    for u, v, _ in edges:
+        out[u].append(v)
+        indeg[v] += 1
+    ready = [x for x in range(n_nodes) if indeg[x] == 0]
+    seen = 0
+    while ready:
+        x = ready.pop()
+        seen += 1
+        for v in out[x]:
+            indeg[v] -= 1
+            if indeg[v] == 0:
+                ready.append(v)
+    return seen == n_nodes
+
+
+@pytest.mark.parametrize("name,N,causal,heads,ctas", [
+    (sc.SHIFT, 4, False, 3, 5), (sc.NAIVE_ASC, 3, True, 2, 7), (sc.DESCENDING, 5, True, 4, 6),
+    (sc.SYM_SHIFT, 4, True, 3, 4), (sc.SHIFT, 32, False, 32, 148)])
+def test_group_one_is_the_multi_head_table(name, N, causal, heads, ctas):
+    assert (binding.dash_sched_table_gqa(heads, 1, N, causal, SID[name], ctas)
+            == binding.dash_sched_table(heads, N, causal, SID[name], ctas))
+
+
+GQA_CASES = [(name, N, causal, heads, group, ctas)
+             for name in sc.ALL
+             for causal in (False, True)
+             for N, heads, group, ctas in ((4, 4, 2, 3), (6, 8, 4, 5), (4, 6, 2, 16),
+                                           (8, 4, 4, 2), (2, 2, 2, 1), (8, 16, 8, 148))
+             if sc.supported(name, N, causal)]
+
+
+@pytest.mark.parametrize("name,N,causal,heads,group,ctas", GQA_CASES)
+def test_grouped_table_invariants(name, N, causal, heads, group, ctas):
+    rows = binding.dash_sched_table_gqa(heads, group, N, causal, SID[name], ctas)
+    # coverage: each pair of every query head once
+    got = sorted((h, kv, q) for _, h, kv, q, _, _ in rows)
+    assert got == sorted((h, kv, q) for h in range(heads) for kv, q in _mask_pairs(N, causal))
+    # positions of each dQ block are a permutation of its contributors
+    pos = defaultdict(list)
+    for _, h, kv, q, p, _ in rows:
+        pos[(h, q)].append(p)
+    for (h, q), ps in pos.items():
+        assert sorted(ps) == list(range(q + 1 if causal else N))
+    # chains: consecutive rows of one chain index; runs of one (K/V head, kv) per CTA
+    chains = []  # (cta, chain, head, kv, [q...]) in table order
+    for cta, h, kv, q, _, ci in rows:
+        if not chains or chains[-1][1] != ci:
+            chains.append((cta, ci, h, kv, []))
+        chains[-1][4].append(q)
+    runs = []
+    for c in chains:
+        cta, _, h, kv, qs = c
+        if runs and runs[-1][0] == cta and runs[-1][1] == h // group and runs[-1][2] == kv:
+            runs[-1][3].append((h, qs))
+        else:
+            runs.append((cta, h // group, kv, [(h, qs)]))
+    keys = [(r[1], r[2]) for r in runs]
+    assert len(keys) == len(set(keys)) == (heads // group) * N   # one run per KV tile
+    mha = {}
+    for slot in sc.packed_table(name, 1, N, causal, len(sc.units(name, N, causal))):
+        for _, kv, q, _, _ in slot:
+            mha.setdefault(kv, []).append(q)
+    for _, kvh, kv, members in runs:
+        assert [h for h, _ in members] == [kvh * group + i for i in range(group)]
+        for _, qs in members:
+            assert qs == mha[kv]        # the multi-head unit's Q tiles of that segment
+    # no dependence cycle (two accumulation chains per block, as the kernel runs)
+    slots = [[] for _ in range(ctas)]
+    for cta, h, kv, q, p, _ in rows:
+        slots[cta].append((h, kv, q, p, q + 1 if causal else N))
+    for chains_per_block in (1, 2):
+        n, edges, _ = dag.schedule_graph(slots, 1.0, 0.3, None, chains_per_block)
+        assert _acyclic(n, edges)
+    assert binding.dash_sched_check(heads, N, causal, ctas, rows) == 0
+
+
+def test_grouped_tables_at_workload_shapes_validate():
+    # 32 query heads over 8 K/V heads (B=2 H=16 at S=4096 full; B=2 H=32 at S=8192 causal)
+    for heads, group, N, causal, name in ((32, 4, 32, False, "shift"),
+                                          (32, 4, 32, False, "descending"),
+                                          (64, 8, 64, True, "sym_shift"),
+                                          (64, 2, 64, True, "descending")):
+        rows = binding.dash_sched_table_gqa(heads, group, N, causal, name, 148)
+        assert len(rows) == heads * (N * (N + 1) // 2 if causal else N * N)
+
+
+def test_grouped_table_argument_errors():
+    with pytest.raises(binding.DashError):
+        binding.dash_sched_table_gqa(6, 4, 4, False, "shift", 4)     # 4 does not divide 6
+    with pytest.raises(binding.DashError):
+        binding.dash_sched_table_gqa(4, 0, 4, False, "shift", 4)
