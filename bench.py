@@ -153,10 +153,20 @@ def run_ours(args):
     if args.heads:
         # a smaller case of the same kernel (profiling): B=1 and the given head count
         w = dataclasses.replace(w, B=1, H=args.heads, name=f"{w.name}_as_b1_h{args.heads}")
+    gqa = bool(args.kv_heads) and args.kv_heads != w.H
+    if gqa:
+        # grouped-query attention: the same query heads over fewer K/V heads
+        w = dataclasses.replace(w, name=f"{w.name}_kv{args.kv_heads}")
     sched = args.schedule or w.schedules[0]
     q, k, v, do = draw(w.B, w.H, w.S, w.D, w.sigma, seed_of(args.workload) + 1000 * rank,
                        device="cuda")
-    o, lse = binding.dash_attn_fwd(q, k, v, w.causal)
+    if gqa:
+        _, k, v, _ = draw(w.B, args.kv_heads, w.S, w.D, w.sigma,
+                          seed_of(args.workload) + 1000 * rank + 1, device="cuda")
+        fwd_call, bwd_call = binding.dash_attn_fwd_gqa, binding.dash_attn_bwd_gqa
+    else:
+        fwd_call, bwd_call = binding.dash_attn_fwd, binding.dash_attn_bwd
+    o, lse = fwd_call(q, k, v, w.causal)
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
 
@@ -170,7 +180,7 @@ def run_ours(args):
         dk = torch.empty_like(k)
         dv = torch.empty_like(v)
         for _ in range(warmup):
-            binding.dash_attn_bwd(q, k, v, o, do, lse, w.causal, name, dq, dk, dv)
+            bwd_call(q, k, v, o, do, lse, w.causal, name, dq, dk, dv)
         st = binding.dash_attn_sync_status()
         if st != 0:
             raise RuntimeError(f"warm-up status {binding.dash_status_string(st)}")
@@ -183,7 +193,7 @@ def run_ours(args):
             for i in range(steps):
                 flush.fill_(float(i))
                 evs[i][0].record(stream)
-                binding.dash_attn_bwd(q, k, v, o, do, lse, w.causal, name, dq, dk, dv)
+                bwd_call(q, k, v, o, do, lse, w.causal, name, dq, dk, dv)
                 evs[i][1].record(stream)
             barrier()
         main_ms, aux_ms, n_calls = binding.dash_profile_end()
@@ -206,14 +216,14 @@ def run_ours(args):
     # outside the backward's timed region
     fo, fl = torch.empty_like(q), torch.empty_like(lse)
     for _ in range(2):
-        binding.dash_attn_fwd(q, k, v, w.causal, fo, fl)
+        fwd_call(q, k, v, w.causal, fo, fl)
     fwd_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(max(3, args.steps // 2))]
     barrier()
     for i, (a, b) in enumerate(fwd_ev):
         flush.fill_(float(i))
         a.record(stream)
-        binding.dash_attn_fwd(q, k, v, w.causal, fo, fl)
+        fwd_call(q, k, v, w.causal, fo, fl)
         b.record(stream)
     barrier()
     if binding.dash_attn_sync_status() != 0:
@@ -222,26 +232,30 @@ def run_ours(args):
     del fo, fl
 
     sim = None
-    if rank == 0 and not args.no_compare:
+    if rank == 0 and not args.no_compare and not gqa:
         sim = simulator_vs_measured(w, q, k, v, o, do, lse, sched, results)
 
     # end to end through the public API's host-buffer entry point: every step copies
     # the pinned host inputs in and the results out, overlapped with the compute
-    host_in = [t.cpu().pin_memory() for t in (q, k, v, o, do, lse)]
-    host_out = [torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(3)]
-    e2e_steps = max(3, args.steps // 2)
-    for it in range(e2e_steps + 2):
-        if it == 2:
-            barrier()
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-        binding.dash_attn_bwd_host(*host_in, w.causal, sched, *host_out)
-    e1.record(stream)
-    barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, "cuda")
-    h2d = sum(x.numel() * x.element_size() for x in host_in)
-    d2h = sum(x.numel() * x.element_size() for x in host_out)
+    # (multi-head only: there is no grouped-query host-buffer entry)
+    e2e = None
+    if not gqa:
+        host_in = [t.cpu().pin_memory() for t in (q, k, v, o, do, lse)]
+        host_out = [torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(3)]
+        e2e_steps = max(3, args.steps // 2)
+        for it in range(e2e_steps + 2):
+            if it == 2:
+                barrier()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            binding.dash_attn_bwd_host(*host_in, w.causal, sched, *host_out)
+        e1.record(stream)
+        barrier()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, "cuda")
+        e2e = {"value": round(w.flops * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in host_in),
+               "d2h_bytes_per_step": sum(x.numel() * x.element_size() for x in host_out)}
 
     if rank == 0:
         peak, _, peak_kind = _peaks()
@@ -264,7 +278,8 @@ def run_ours(args):
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic (seeded normal bf16 Q, K, V, dO; O and LSE from the library forward)",
-            "config": {"workload": w.name, "B": w.B, "H": w.H, "S": w.S, "D": w.D,
+            "config": {"workload": w.name, "B": w.B, "H": w.H,
+                       "H_kv": args.kv_heads if gqa else w.H, "S": w.S, "D": w.D,
                        "mask": "causal" if w.causal else "full", "sigma": w.sigma,
                        "schedule": sched, "parallelism": f"dp{world} (independent heads)",
                        "l2": "flushed before every timed step (512 MiB write)"},
@@ -277,8 +292,7 @@ def run_ours(args):
                          "traffic": _recorded_traffic(w.name, sched),
                          "kernel": "dash_bwd_kernel", "peak_kind": f"{peak_kind} bf16 burst",
                          "kernel_ms": round(main_ms, 4), "aux_ms": round(aux_ms, 4)},
-            "e2e": {"value": round(tflops(e2e_ms), 2), "unit": "TFLOP/s",
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "e2e": e2e,
             "gpu_launches": int(n_calls) * (3 if sched == "atomic" else 2),
             "fwd_bwd": {"fwd_ms": round(fwd_ms, 4),
                         "fwd_tflops": round(0.4 * w.flops * world / (fwd_ms * 1e-3) / 1e12, 2),
@@ -291,7 +305,7 @@ def run_ours(args):
         }
         if sim is not None:
             line["simulator"] = sim
-        if not args.no_cpu_baseline and world == 1:
+        if not args.no_cpu_baseline and world == 1 and not gqa:
             line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
         print(json.dumps(line), flush=True)
     if dist is not None:
@@ -419,6 +433,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--all-workloads", action="store_true",
                     help="one JSON line per workload (1-4), rank 0 only")
+    ap.add_argument("--kv-heads", type=int, default=0,
+                    help="time grouped-query attention with this many K/V heads (a side "
+                         "measurement: no host-buffer e2e, simulator or CPU baseline)")
     ap.add_argument("--heads", type=int, default=0,
                     help="run the workload's shape with B=1 and this many heads (a smaller "
                          "case of the same kernel, for profiling); 0 = the workload as named")
