@@ -293,6 +293,17 @@ int dash_sched_simulate(int n_heads, int N, int causal, int schedule, int num_ct
                         long long* stalls);
 
 /*
+ * The same simulation of the grouped-query table of dash_sched_table_gqa
+ * (n_heads query heads, `group` of them per K/V head): each pair's events and
+ * arcs as above, over the grouped table's CTA order and dQ positions.
+ * DASH_ERR_INVALID_ARG also when group < 1 or does not divide n_heads.
+ */
+int dash_sched_simulate_gqa(int n_heads, int group, int N, int causal, int schedule,
+                            int num_ctas, double w_compute, double w_reduce, int dq_buffers,
+                            int dq_chains, double* critical_path, double* makespan,
+                            double* bubble_time, long long* stalls);
+
+/*
  * Checks a schedule table supplied by the caller, in the row format of
  * dash_sched_table: n_rows rows of 6 ints (cta, head, kv_tile, q_tile,
  * position, chain_index), grouped by CTA in ascending order, each CTA's rows in

@@ -20,7 +20,8 @@ STATUS = {0: "DASH_OK", 1: "DASH_ERR_INVALID_ARG", 2: "DASH_ERR_UNSUPPORTED", 3:
 
 EXPORTS = ("dash_attn_fwd", "dash_attn_bwd", "dash_attn_sync_status", "dash_status_string",
            "dash_set_spin_limit_us", "dash_bwd_num_ctas", "dash_release_workspace",
-           "dash_sched_table", "dash_sched_simulate", "dash_dag_longest_path",
+           "dash_sched_table", "dash_sched_simulate", "dash_sched_simulate_gqa",
+           "dash_dag_longest_path",
            "dash_profile_begin", "dash_profile_end", "dash_attn_bwd_noalloc",
            "dash_trace_bwd", "dash_inject_fault", "dash_sched_check", "dash_attn_bwd_host",
            "dash_sched_table_part", "dash_attn_fwd_gqa", "dash_attn_bwd_gqa",
@@ -72,6 +73,8 @@ def load(path: str | None = None):
     lib.dash_sched_table_gqa.argtypes = [i, i, i, i, i, i, vp, ll]
     lib.dash_sched_table_gqa.restype = ll
     lib.dash_sched_simulate.argtypes = [i, i, i, i, i, d, d, i, i, P(d), P(d), P(d), P(ll)]
+    lib.dash_sched_simulate_gqa.argtypes = [i, i, i, i, i, i, d, d, i, i, P(d), P(d), P(d),
+                                            P(ll)]
     lib.dash_sched_check.argtypes = [i, i, i, i, vp, ll]
     lib.dash_dag_longest_path.argtypes = [i, i, vp, vp, vp, vp, vp, P(d)]
     lib.dash_trace_bwd.argtypes = [vp] * 9 + [i, i, i, i, i, i, vp, vp, ll, P(i), P(i)]
@@ -296,6 +299,20 @@ def dash_sched_simulate(n_heads: int, N: int, causal: bool, schedule, num_ctas: 
                                     int(dq_chains), ctypes.byref(cp), ctypes.byref(mk),
                                     ctypes.byref(bt), ctypes.byref(st))
     _check(rc, "dash_sched_simulate")
+    return cp.value, mk.value, bt.value, st.value
+
+
+def dash_sched_simulate_gqa(n_heads: int, group: int, N: int, causal: bool, schedule,
+                            num_ctas: int, w_compute: float, w_reduce: float,
+                            dq_buffers: int = 0, dq_chains: int = 1):
+    """dash_sched_simulate over the grouped-query table (`group` query heads per K/V head)."""
+    cp, mk, bt = ctypes.c_double(), ctypes.c_double(), ctypes.c_double()
+    st = ctypes.c_longlong()
+    rc = load().dash_sched_simulate_gqa(n_heads, group, N, int(bool(causal)), _sched_id(schedule),
+                                        num_ctas, float(w_compute), float(w_reduce),
+                                        int(dq_buffers), int(dq_chains), ctypes.byref(cp),
+                                        ctypes.byref(mk), ctypes.byref(bt), ctypes.byref(st))
+    _check(rc, "dash_sched_simulate_gqa")
     return cp.value, mk.value, bt.value, st.value
 
 

@@ -987,10 +987,20 @@ int dash_sched_simulate(int n_heads, int N, int causal, int schedule, int num_ct
                         double w_compute, double w_reduce, int dq_buffers, int dq_chains,
                         double* critical_path, double* makespan, double* bubble_time,
                         long long* stalls) {
+  return dash_sched_simulate_gqa(n_heads, 1, N, causal, schedule, num_ctas, w_compute, w_reduce,
+                                 dq_buffers, dq_chains, critical_path, makespan, bubble_time,
+                                 stalls);
+}
+
+int dash_sched_simulate_gqa(int n_heads, int group, int N, int causal, int schedule,
+                            int num_ctas, double w_compute, double w_reduce, int dq_buffers,
+                            int dq_chains, double* critical_path, double* makespan,
+                            double* bubble_time, long long* stalls) {
   if (w_compute < 0 || w_reduce < 0 || dq_chains < 1) return DASH_ERR_INVALID_ARG;
+  if (group < 1 || n_heads < 1 || n_heads % group != 0) return DASH_ERR_INVALID_ARG;
   dash::Table t;
   std::string err;
-  if (!dash::build_table(n_heads, N, causal, schedule, num_ctas, &t, &err))
+  if (!dash::build_table_grouped(n_heads, group, N, causal, schedule, num_ctas, &t, &err))
     return DASH_ERR_UNSUPPORTED;
   if (!dash::validate_table(t, &err)) return DASH_ERR_SCHEDULE;
   dash::SimResult r;

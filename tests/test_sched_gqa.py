@@ -121,3 +121,52 @@ def test_grouped_table_argument_errors():
         binding.dash_sched_table_gqa(6, 4, 4, False, "shift", 4)     # 4 does not divide 6
     with pytest.raises(binding.DashError):
         binding.dash_sched_table_gqa(4, 0, 4, False, "shift", 4)
+
+
+@pytest.mark.parametrize("name,N,causal,heads,group,ctas", [
+    (sc.SHIFT, 3, False, 2, 2, 3), (sc.SHIFT, 2, False, 4, 2, 3), (sc.NAIVE_ASC, 3, True, 2, 2, 2),
+    (sc.DESCENDING, 3, True, 2, 2, 2), (sc.DESCENDING, 2, False, 4, 4, 3),
+    (sc.SYM_SHIFT, 2, True, 4, 2, 3),
+    (sc.SYM_SHIFT, 4, True, 2, 2, 2)])
+@pytest.mark.parametrize("beta", [None, 1, 2])
+@pytest.mark.parametrize("chains", [1, 2])
+def test_grouped_simulator_matches_bruteforce(name, N, causal, heads, group, ctas, beta, chains):
+    c, r = 1.0, 0.35
+    rows = binding.dash_sched_table_gqa(heads, group, N, causal, SID[name], ctas)
+    slots = [[] for _ in range(ctas)]
+    for cta, h, kv, q, p, _ in rows:
+        slots[cta].append((h, kv, q, p, q + 1 if causal else N))
+    want = dag.simulate(slots, c, r, beta, chains)
+    got = binding.dash_sched_simulate_gqa(heads, group, N, causal, SID[name], ctas, c, r,
+                                          0 if beta is None else beta, chains)
+    assert got[0] == pytest.approx(want[0], abs=1e-9)
+    assert got[1] == pytest.approx(want[1], abs=1e-9)
+    assert got[2] == pytest.approx(want[2], abs=1e-9)
+    assert got[3] == want[3]
+
+
+def test_grouped_simulator_group_one_is_multi_head():
+    for name, N, causal in (("shift", 8, False), ("sym_shift", 8, True), ("descending", 6, True)):
+        assert (binding.dash_sched_simulate_gqa(12, 1, N, causal, name, 20, 1.0, 0.8, 2, 2)
+                == binding.dash_sched_simulate(12, N, causal, name, 20, 1.0, 0.8, 2, 2))
+
+
+@pytest.mark.parametrize("kv_heads,group,N", [(1, 4, 8), (3, 2, 16), (2, 8, 5)])
+def test_grouped_shift_closed_form(kv_heads, group, N):
+    """Full-mask shift with every unit in one round and r <= c: each dQ block's
+    contributors arrive one step apart, so nothing waits, and the last reduction
+    ends at g*N*c + r (g*N pairs per CTA)."""
+    c, r = 1.0, 0.6
+    ctas = kv_heads * N
+    cp, mk, bt, st = binding.dash_sched_simulate_gqa(kv_heads * group, group, N, False, "shift",
+                                                     ctas, c, r, 0, 1)
+    assert cp == pytest.approx(group * N * c + r)
+    assert mk == pytest.approx(group * N * c)
+    assert bt == pytest.approx(ctas * r)
+    assert st == 0
+
+
+def test_grouped_simulator_argument_errors():
+    for args in ((6, 4), (4, 0)):
+        with pytest.raises(binding.DashError):
+            binding.dash_sched_simulate_gqa(args[0], args[1], 4, False, "shift", 4, 1.0, 0.5)
