@@ -22,6 +22,18 @@ def head_range(n_heads: int, rank: int, world: int) -> tuple[int, int]:
     return start, start + base + (1 if rank < extra else 0)
 
 
+def group_head_range(n_heads: int, group: int, rank: int, world: int) -> tuple[int, int]:
+    """Contiguous [start, end) range of flattened query heads owned by `rank`
+    under grouped-query attention: whole K/V heads, each with its `group`
+    query heads, so a K/V head's dK/dV sum stays on one rank and the rank's
+    K/V slice is heads [start // group, end // group).
+    """
+    if group < 1 or n_heads % group != 0:
+        raise ValueError("group must divide the query head count")
+    a, b = head_range(n_heads // group, rank, world)
+    return a * group, b * group
+
+
 def max_over_ranks(value: float, device=None) -> float:
     """Maximum of a per-rank scalar (e.g. a timed duration) over all ranks;
     the value itself without an initialised process group."""

@@ -5,7 +5,7 @@ import pytest
 import torch
 import torch.multiprocessing as mp
 
-from persistent_sm_attn_b200.parallel import head_range, max_over_ranks
+from persistent_sm_attn_b200.parallel import group_head_range, head_range, max_over_ranks
 
 
 @pytest.mark.parametrize("n_heads", [0, 1, 5, 32, 128, 97])
@@ -19,6 +19,26 @@ def test_head_ranges_partition(n_heads, world):
         sizes.append(b - a)
     assert seen == list(range(n_heads))
     assert max(sizes) - min(sizes) <= 1
+
+
+@pytest.mark.parametrize("n_kv,group", [(0, 2), (1, 4), (5, 2), (8, 8), (7, 1)])
+@pytest.mark.parametrize("world", [1, 2, 3, 8])
+def test_group_head_ranges_keep_kv_heads_whole(n_kv, group, world):
+    seen, sizes = [], []
+    for r in range(world):
+        a, b = group_head_range(n_kv * group, group, r, world)
+        assert a % group == 0 and b % group == 0
+        seen.extend(range(a, b))
+        sizes.append((b - a) // group)
+    assert seen == list(range(n_kv * group))
+    assert max(sizes) - min(sizes) <= 1
+
+
+def test_group_head_range_rejects_partial_groups():
+    with pytest.raises(ValueError):
+        group_head_range(6, 4, 0, 1)
+    with pytest.raises(ValueError):
+        group_head_range(8, 0, 0, 2)
 
 
 def test_head_range_rejects_bad_ranks():
