@@ -109,6 +109,43 @@ def _sched_id(schedule) -> int:
     return SCHEDULES[schedule] if isinstance(schedule, str) else int(schedule)
 
 
+def _check_tensors(q, k, v, o=None, do=None, lse=None, outs=(), *, cuda=True, gqa=False):
+    """Reject tensors whose shape, dtype, layout or device differs from what the C
+    entry points read and write: q [B,H,S,D] bf16; k, v [B,Hkv,S,D] bf16 (Hkv = H
+    unless gqa); o, do like q; lse [B,H,S] fp32; outs (dq, dk, dv) or (o, lse).
+    The C ABI takes bare pointers, so a mismatch here would otherwise become an
+    out-of-bounds device access."""
+    import torch
+    if q.dim() != 4:
+        raise ValueError("q must be [B,H,S,D]")
+    B, H, S, D = q.shape
+    Hkv = k.shape[1] if gqa and k.dim() == 4 else H
+    bf, f32 = torch.bfloat16, torch.float32
+    want = [("q", q, (B, H, S, D), bf), ("k", k, (B, Hkv, S, D), bf), ("v", v, (B, Hkv, S, D), bf)]
+    if o is not None:
+        want.append(("o", o, (B, H, S, D), bf))
+    if do is not None:
+        want.append(("do", do, (B, H, S, D), bf))
+    if lse is not None:
+        want.append(("lse", lse, (B, H, S), f32))
+    names = ("dq", "dk", "dv") if len(outs) == 3 else ("out", "lse_out")
+    shapes = ((B, H, S, D), (B, Hkv, S, D), (B, Hkv, S, D)) if len(outs) == 3 else \
+        ((B, H, S, D), (B, H, S))
+    dtypes = (bf, bf, bf) if len(outs) == 3 else (bf, f32)
+    want += [(n, t, sh, dt) for n, t, sh, dt in zip(names, outs, shapes, dtypes) if t is not None]
+    for name, t, shape, dtype in want:
+        if tuple(t.shape) != shape:
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {shape}")
+        if t.dtype != dtype:
+            raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if cuda and (not t.is_cuda or t.device != q.device):
+            raise ValueError(f"{name} must be a CUDA tensor on {q.device}")
+        if not cuda and t.is_cuda:
+            raise ValueError(f"{name} must be a host tensor")
+
+
 def dash_status_string(status: int) -> str:
     return load().dash_status_string(int(status)).decode()
 
@@ -116,6 +153,7 @@ def dash_status_string(status: int) -> str:
 def dash_attn_fwd(q, k, v, causal: bool, out=None, lse=None, stream=None):
     """O, LSE = attention forward (bf16 [B,H,S,D] CUDA tensors)."""
     import torch
+    _check_tensors(q, k, v, outs=(out, lse))
     B, H, S, D = q.shape
     if out is None:
         out = torch.empty_like(q)
@@ -131,9 +169,7 @@ def dash_attn_bwd(q, k, v, o, do, lse, causal: bool, schedule="shift", dq=None, 
                   dv=None, stream=None):
     """dQ, dK, dV of attention (bf16 [B,H,S,D], lse fp32 [B,H,S]; CUDA tensors)."""
     import torch
-    for t in (q, k, v, o, do, lse):
-        if not t.is_cuda or not t.is_contiguous():
-            raise ValueError("inputs must be contiguous CUDA tensors")
+    _check_tensors(q, k, v, o, do, lse, (dq, dk, dv))
     B, H, S, D = q.shape
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
@@ -149,6 +185,7 @@ def dash_attn_fwd_gqa(q, k, v, causal: bool, out=None, lse=None, stream=None):
     """O, LSE of grouped-query attention: q [B,H,S,D], k and v [B,Hkv,S,D] (bf16
     CUDA tensors), query head h reading K/V head h // (H // Hkv)."""
     import torch
+    _check_tensors(q, k, v, outs=(out, lse), gqa=True)
     B, H, S, D = q.shape
     Hkv = k.shape[1]
     out = torch.empty_like(q) if out is None else out
@@ -165,9 +202,7 @@ def dash_attn_bwd_gqa(q, k, v, o, do, lse, causal: bool, schedule="shift", dq=No
     """dQ [B,H,S,D], dK and dV [B,Hkv,S,D] of grouped-query attention (dK, dV summed
     over each K/V head's query heads)."""
     import torch
-    for t in (q, k, v, o, do, lse):
-        if not t.is_cuda or not t.is_contiguous():
-            raise ValueError("inputs must be contiguous CUDA tensors")
+    _check_tensors(q, k, v, o, do, lse, (dq, dk, dv), gqa=True)
     B, H, S, D = q.shape
     Hkv = k.shape[1]
     dq = torch.empty_like(q) if dq is None else dq
@@ -187,17 +222,12 @@ def dash_attn_bwd_host(q, k, v, o, do, lse, causal: bool, schedule="shift", dq=N
     copies overlap the compute.  The outputs are valid once `stream` (default:
     torch's current stream) has completed."""
     import torch
-    for t in (q, k, v, o, do, lse):
-        if t.is_cuda or not t.is_contiguous():
-            raise ValueError("inputs must be contiguous host tensors")
+    _check_tensors(q, k, v, o, do, lse, (dq, dk, dv), cuda=False)
     B, H, S, D = q.shape
     pin = q.is_pinned()
     dq = torch.empty(q.shape, dtype=q.dtype, pin_memory=pin) if dq is None else dq
     dk = torch.empty(k.shape, dtype=k.dtype, pin_memory=pin) if dk is None else dk
     dv = torch.empty(v.shape, dtype=v.dtype, pin_memory=pin) if dv is None else dv
-    for t in (dq, dk, dv):
-        if t.is_cuda or not t.is_contiguous():
-            raise ValueError("outputs must be contiguous host tensors")
     rc = load().dash_attn_bwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse),
                                    _ptr(dq), _ptr(dk), _ptr(dv), B, H, S, D, int(bool(causal)),
                                    _sched_id(schedule), _stream_handle(stream))
@@ -210,9 +240,10 @@ def dash_attn_bwd_noalloc(q, k, v, o, do, lse, causal: bool, schedule, dq, dk, d
     """The backward through the entry point that allocates no device memory.
     Outputs must be preallocated; all scratch comes from the library's static
     device array (see include/dash_attn.h)."""
-    for t in (q, k, v, o, do, lse, dq, dk, dv):
-        if not t.is_cuda or not t.is_contiguous():
-            raise ValueError("tensors must be contiguous CUDA tensors")
+    for t in (dq, dk, dv):
+        if t is None:
+            raise ValueError("dash_attn_bwd_noalloc needs preallocated dq, dk, dv")
+    _check_tensors(q, k, v, o, do, lse, (dq, dk, dv))
     B, H, S, D = q.shape
     rc = load().dash_attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse),
                                       _ptr(dq), _ptr(dk), _ptr(dv), B, H, S, D,
@@ -355,6 +386,7 @@ def dash_trace_bwd(q, k, v, o, do, lse, causal: bool, schedule="shift", stream=N
     """One traced backward; returns (dq, dk, dv, trace [ctas, rows, 8] uint64 ns)."""
     import numpy as np
     import torch
+    _check_tensors(q, k, v, o, do, lse)
     B, H, S, D = q.shape
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     N = S // 128
