@@ -394,6 +394,12 @@ def run_reference(args):
     if rank != 0:
         return
     w = WORKLOADS[args.workload]
+    gqa = bool(args.kv_heads) and args.kv_heads != w.H
+    if gqa:
+        # the oracle's grouped-query backward is the per-head backward of every query
+        # head plus the sums of dK, dV over each group, so its cost per query head is
+        # the per-head backward timed here
+        w = dataclasses.replace(w, name=f"{w.name}_kv{args.kv_heads}")
     per_step = []
     last = None
     for _ in range(args.warmup):
@@ -408,7 +414,8 @@ def run_reference(args):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic (seeded normal bf16 Q, K, V, dO widened to fp64)",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "S": w.S, "D": w.D,
+        "config": {"workload": w.name, "B": w.B, "H": w.H,
+                   "H_kv": args.kv_heads if gqa else w.H, "S": w.S, "D": w.D,
                    "mask": "causal" if w.causal else "full", "schedule": "none (order-free)"},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores,
                          "kind": "oracle",

@@ -28,3 +28,14 @@ def test_reference_arm_prints_one_contract_line():
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_names_a_grouped_query_config():
+    out = subprocess.run(
+        [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+         "--warmup", "3", "--workload", "0", "--cpu-seconds", "0.2", "--kv-heads", "1"],
+        capture_output=True, text=True, timeout=600, cwd=ROOT, check=True).stdout
+    d = json.loads([l for l in out.splitlines() if l.strip().startswith("{")][-1])
+    assert d["config"]["workload"] == "full_b1_h2_s256_d64_kv1"
+    assert d["config"]["H"] == 2 and d["config"]["H_kv"] == 1
+    assert d["value"] > 0
