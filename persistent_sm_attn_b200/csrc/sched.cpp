@@ -18,6 +18,7 @@
 #include "sched.h"
 
 #include <algorithm>
+#include <climits>
 #include <cmath>
 #include <cstdio>
 #include <deque>
@@ -104,6 +105,13 @@ bool build_table_grouped(int n_heads, int group, int N, int causal, int schedule
     if (err) *err = "schedule not defined for this mask / tile count / head grouping";
     return false;
   }
+  // Chain offsets into the pair list are int32, and a grouped unit's step must fit the
+  // 24 bits the position keys below give it: refuse larger problems before building.
+  const long long per_head = causal ? (long long)N * (N + 1) / 2 : (long long)N * N;
+  if ((long long)n_heads * per_head > INT32_MAX || (long long)group * (N + 1) >= (1LL << 24)) {
+    if (err) *err = "table too large (more than 2^31 - 1 pairs, or 2^24 steps in a unit)";
+    return false;
+  }
   const Units units = units_of(schedule, N, causal);
   const int U = (int)units.size();
   // Group unit k: unit k's KV segments in order, each run for query heads 0..group-1
@@ -127,21 +135,23 @@ bool build_table_grouped(int n_heads, int group, int N, int causal, int schedule
   // K/V heads with the same first-unit offset in their round share one table.
   const bool by_kv = (schedule == NAIVE_ASC || schedule == DESCENDING);
   auto head_positions = [&](long long first_g) {
-    // per (query head offset, q): (key, unit * 65536 + step)
-    std::vector<std::vector<std::pair<long long, int>>> contrib((size_t)group * N);
+    // per (query head offset, q): (key, (unit, step)); keys are distinct within a block
+    // (by KV tile, or by round, step and unit, with step < 2^24 and unit < 2^16)
+    std::vector<std::vector<std::pair<long long, std::pair<int, int>>>> contrib(
+        (size_t)group * N);
     for (int k = 0; k < U; ++k) {
       const long long rnd = (first_g + k) / num_ctas - first_g / num_ctas;
       for (int t = 0; t < (int)gunits[k].size(); ++t) {
         const Step& st = gunits[k][t];
         const long long key = by_kv ? st.kv : (rnd << 40) + (long long)t * 65536 + k;
-        contrib[(size_t)st.head * N + st.q].push_back({key, k * 65536 + t});
+        contrib[(size_t)st.head * N + st.q].push_back({key, {k, t}});
       }
     }
     std::vector<std::vector<int>> pos(U);
     for (int k = 0; k < U; ++k) pos[k].assign(gunits[k].size(), -1);
     for (auto& c : contrib) {
       std::sort(c.begin(), c.end());
-      for (int p = 0; p < (int)c.size(); ++p) pos[c[p].second >> 16][c[p].second & 0xffff] = p;
+      for (int p = 0; p < (int)c.size(); ++p) pos[c[p].second.first][c[p].second.second] = p;
     }
     return pos;
   };

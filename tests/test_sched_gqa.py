@@ -170,3 +170,18 @@ def test_grouped_simulator_argument_errors():
     for args in ((6, 4), (4, 0)):
         with pytest.raises(binding.DashError):
             binding.dash_sched_simulate_gqa(args[0], args[1], 4, False, "shift", 4, 1.0, 0.5)
+
+
+def test_units_longer_than_two_to_the_sixteen_steps():
+    """512 query heads on one K/V head at N = 128, causal symmetric shift: each grouped
+    unit runs 512 * 129 pairs, more than a 16-bit step field holds.  The table still
+    builds and passes validation (positions, runs, deadlock)."""
+    lib = binding.load()
+    assert lib.dash_sched_table_gqa(512, 512, 128, 1, 3, 148, None, 0) == 512 * 128 * 129 // 2
+
+
+def test_tables_beyond_int32_pairs_are_refused_before_building():
+    lib = binding.load()
+    # 256 heads x 4096^2 pairs > 2^31 - 1: refused as unsupported, without building
+    assert lib.dash_sched_table_gqa(256, 1, 4096, 0, 2, 148, None, 0) == -2
+    assert lib.dash_sched_table(256, 4096, 0, 2, 148, None, 0) == -2
