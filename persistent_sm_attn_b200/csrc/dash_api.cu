@@ -112,8 +112,16 @@ int get_workspace(int dev, void* stream, size_t acc_bytes, size_t tk_bytes, size
     w.rows_cap = rows;
   }
   if (!w.err) {
-    if (cudaMalloc(&w.err, 2 * sizeof(unsigned)) != cudaSuccess) return DASH_ERR_OOM;
-    if (cudaMemset(w.err, 0, 2 * sizeof(unsigned)) != cudaSuccess) return DASH_ERR_CUDA;
+    if (cudaMalloc(&w.err, 2 * sizeof(unsigned)) != cudaSuccess) {
+      cudaGetLastError();
+      w.err = nullptr;
+      return DASH_ERR_OOM;
+    }
+    if (cudaMemset(w.err, 0, 2 * sizeof(unsigned)) != cudaSuccess) {
+      cudaFree(w.err);  // never keep an error word that was not cleared
+      w.err = nullptr;
+      return DASH_ERR_CUDA;
+    }
   }
   *out = &w;
   return DASH_OK;
@@ -504,6 +512,8 @@ struct HostPipe {
 };
 std::map<std::pair<int, uintptr_t>, HostPipe> g_pipes;
 
+void free_pipe(HostPipe* hp);
+
 int get_pipe(int dev, void* stream, size_t bytes, HostPipe** out) {
   HostPipe& hp = g_pipes[{dev, reinterpret_cast<uintptr_t>(stream)}];
   if (!hp.h2d) {
@@ -516,6 +526,7 @@ int get_pipe(int dev, void* stream, size_t bytes, HostPipe** out) {
            cudaEventCreateWithFlags(&hp.out_done[i], cudaEventDisableTiming) == cudaSuccess;
     if (!ok) {
       cudaGetLastError();
+      free_pipe(&hp);  // a later call starts from scratch, not from a half-made pipe
       return DASH_ERR_CUDA;
     }
   }
@@ -526,15 +537,15 @@ int get_pipe(int dev, void* stream, size_t bytes, HostPipe** out) {
 }
 
 void free_pipe(HostPipe* hp) {
-  cudaFree(hp->buf);
+  if (hp->buf) cudaFree(hp->buf);
   for (int i = 0; i < 2; ++i) {
-    cudaEventDestroy(hp->in_ready[i]);
-    cudaEventDestroy(hp->comp_done[i]);
-    cudaEventDestroy(hp->out_done[i]);
+    if (hp->in_ready[i]) cudaEventDestroy(hp->in_ready[i]);
+    if (hp->comp_done[i]) cudaEventDestroy(hp->comp_done[i]);
+    if (hp->out_done[i]) cudaEventDestroy(hp->out_done[i]);
   }
-  cudaEventDestroy(hp->entry);
-  cudaStreamDestroy(hp->h2d);
-  cudaStreamDestroy(hp->d2h);
+  if (hp->entry) cudaEventDestroy(hp->entry);
+  if (hp->h2d) cudaStreamDestroy(hp->h2d);
+  if (hp->d2h) cudaStreamDestroy(hp->d2h);
   *hp = HostPipe{};
 }
 
