@@ -11,6 +11,7 @@
 #include <cstdlib>
 #include <map>
 #include <mutex>
+#include <new>
 #include <string>
 #include <tuple>
 #include <vector>
@@ -623,6 +624,24 @@ int host_bwd(const void* q, const void* k, const void* v, const void* o, const v
   return DASH_OK;
 }
 
+// C++ exceptions (std::bad_alloc from a table, a map or a vector sized by the caller's
+// arguments) must not cross the C ABI: each entry point that allocates on the host
+// returns a status instead.
+template <class R, class F>
+R no_throw_impl(F&& f, R on_oom, R on_other) {
+  try {
+    return f();
+  } catch (const std::bad_alloc&) {
+    return on_oom;
+  } catch (...) {
+    return on_other;
+  }
+}
+template <class F>
+auto no_throw(F&& f, decltype(f()) on_oom, decltype(f()) on_other) -> decltype(f()) {
+  return no_throw_impl<decltype(f())>(static_cast<F&&>(f), on_oom, on_other);
+}
+
 }  // namespace
 
 extern "C" {
@@ -653,19 +672,21 @@ int dash_set_spin_limit_us(long long us) {
 
 int dash_attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                       int H, int Hkv, int S, int D, int causal, void* stream) {
-  int rc = check_shape(B, H, S, D);
-  if (rc) return rc;
-  if (causal != 0 && causal != 1) return DASH_ERR_INVALID_ARG;
-  if (H > 0 && (Hkv < 1 || H % Hkv != 0)) return DASH_ERR_INVALID_ARG;
-  if (H > 0 && ((H / Hkv) & (H / Hkv - 1)) != 0) return DASH_ERR_UNSUPPORTED;  // 2^k per K/V head
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !lse)
-    return DASH_ERR_INVALID_ARG;
-  if (B == 0 || H == 0) return DASH_OK;
-  int dev = 0;
-  DASH_CUDA(cudaGetDevice(&dev));
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return D == 64 ? launch_fwd<64>(q, k, v, o, lse, B, H, S, causal, st, dev, H / Hkv)
-                 : launch_fwd<128>(q, k, v, o, lse, B, H, S, causal, st, dev, H / Hkv);
+  return no_throw([&]() -> int {
+    int rc = check_shape(B, H, S, D);
+    if (rc) return rc;
+    if (causal != 0 && causal != 1) return DASH_ERR_INVALID_ARG;
+    if (H > 0 && (Hkv < 1 || H % Hkv != 0)) return DASH_ERR_INVALID_ARG;
+    if (H > 0 && ((H / Hkv) & (H / Hkv - 1)) != 0) return DASH_ERR_UNSUPPORTED;  // 2^k per K/V head
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !lse)
+      return DASH_ERR_INVALID_ARG;
+    if (B == 0 || H == 0) return DASH_OK;
+    int dev = 0;
+    DASH_CUDA(cudaGetDevice(&dev));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return D == 64 ? launch_fwd<64>(q, k, v, o, lse, B, H, S, causal, st, dev, H / Hkv)
+                   : launch_fwd<128>(q, k, v, o, lse, B, H, S, causal, st, dev, H / Hkv);
+  }, DASH_ERR_OOM, DASH_ERR_INVALID_ARG);
 }
 
 int dash_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
@@ -676,31 +697,34 @@ int dash_attn_fwd(const void* q, const void* k, const void* v, void* o, float* l
 int dash_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
                       const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
                       int H, int Hkv, int S, int D, int causal, int schedule, void* stream) {
-  int rc = check_shape(B, H, S, D);
-  if (rc) return rc;
-  if (causal != 0 && causal != 1) return DASH_ERR_INVALID_ARG;
-  if (H > 0 && (Hkv < 1 || H % Hkv != 0)) return DASH_ERR_INVALID_ARG;
-  if (H > 0 && ((H / Hkv) & (H / Hkv - 1)) != 0) return DASH_ERR_UNSUPPORTED;  // 2^k per K/V head
-  if (schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_ATOMIC) return DASH_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
-      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
-    return DASH_ERR_INVALID_ARG;
-  if (!dash::schedule_supported(schedule, S / 128, causal)) return DASH_ERR_UNSUPPORTED;
-  if (B == 0 || H == 0) return DASH_OK;
-  int dev = 0;
-  DASH_CUDA(cudaGetDevice(&dev));
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const bool atomic = (schedule == DASH_SCHED_ATOMIC);
-  const int g = H / Hkv;
-  if (D == 64)
-    return atomic ? launch_bwd<64, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
-                                         schedule, st, dev, nullptr, 0, nullptr, g)
-                  : launch_bwd<64, false>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
-                                          schedule, st, dev, nullptr, 0, nullptr, g);
-  return atomic ? launch_bwd<128, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
-                                        schedule, st, dev, nullptr, 0, nullptr, g)
-                : launch_bwd<128, false>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
-                                         schedule, st, dev, nullptr, 0, nullptr, g);
+  return no_throw([&]() -> int {
+    int rc = check_shape(B, H, S, D);
+    if (rc) return rc;
+    if (causal != 0 && causal != 1) return DASH_ERR_INVALID_ARG;
+    if (H > 0 && (Hkv < 1 || H % Hkv != 0)) return DASH_ERR_INVALID_ARG;
+    if (H > 0 && ((H / Hkv) & (H / Hkv - 1)) != 0) return DASH_ERR_UNSUPPORTED;  // 2^k per K/V head
+    if (schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_ATOMIC)
+      return DASH_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+        !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+      return DASH_ERR_INVALID_ARG;
+    if (!dash::schedule_supported(schedule, S / 128, causal)) return DASH_ERR_UNSUPPORTED;
+    if (B == 0 || H == 0) return DASH_OK;
+    int dev = 0;
+    DASH_CUDA(cudaGetDevice(&dev));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool atomic = (schedule == DASH_SCHED_ATOMIC);
+    const int g = H / Hkv;
+    if (D == 64)
+      return atomic ? launch_bwd<64, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
+                                           schedule, st, dev, nullptr, 0, nullptr, g)
+                    : launch_bwd<64, false>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
+                                            schedule, st, dev, nullptr, 0, nullptr, g);
+    return atomic ? launch_bwd<128, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
+                                          schedule, st, dev, nullptr, 0, nullptr, g)
+                  : launch_bwd<128, false>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
+                                           schedule, st, dev, nullptr, 0, nullptr, g);
+  }, DASH_ERR_OOM, DASH_ERR_INVALID_ARG);
 }
 
 int dash_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -713,26 +737,29 @@ int dash_attn_bwd(const void* q, const void* k, const void* v, const void* o, co
 int dash_attn_bwd_host(const void* q, const void* k, const void* v, const void* o,
                        const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
                        int H, int S, int D, int causal, int schedule, void* stream) {
-  int rc = check_shape(B, H, S, D);
-  if (rc) return rc;
-  if (causal != 0 && causal != 1) return DASH_ERR_INVALID_ARG;
-  if (schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_ATOMIC) return DASH_ERR_INVALID_ARG;
-  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return DASH_ERR_INVALID_ARG;
-  if (!dash::schedule_supported(schedule, S / 128, causal)) return DASH_ERR_UNSUPPORTED;
-  if (B == 0 || H == 0) return DASH_OK;
-  int dev = 0;
-  DASH_CUDA(cudaGetDevice(&dev));
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const bool atomic = (schedule == DASH_SCHED_ATOMIC);
-  if (D == 64)
-    return atomic ? host_bwd<64, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
-                                       schedule, st, dev)
-                  : host_bwd<64, false>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
-                                        schedule, st, dev);
-  return atomic ? host_bwd<128, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
-                                      schedule, st, dev)
-                : host_bwd<128, false>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
-                                       schedule, st, dev);
+  return no_throw([&]() -> int {
+    int rc = check_shape(B, H, S, D);
+    if (rc) return rc;
+    if (causal != 0 && causal != 1) return DASH_ERR_INVALID_ARG;
+    if (schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_ATOMIC)
+      return DASH_ERR_INVALID_ARG;
+    if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return DASH_ERR_INVALID_ARG;
+    if (!dash::schedule_supported(schedule, S / 128, causal)) return DASH_ERR_UNSUPPORTED;
+    if (B == 0 || H == 0) return DASH_OK;
+    int dev = 0;
+    DASH_CUDA(cudaGetDevice(&dev));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool atomic = (schedule == DASH_SCHED_ATOMIC);
+    if (D == 64)
+      return atomic ? host_bwd<64, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
+                                         schedule, st, dev)
+                    : host_bwd<64, false>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
+                                          schedule, st, dev);
+    return atomic ? host_bwd<128, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
+                                        schedule, st, dev)
+                  : host_bwd<128, false>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
+                                         schedule, st, dev);
+  }, DASH_ERR_OOM, DASH_ERR_INVALID_ARG);
 }
 
 int dash_attn_sync_status(void* stream) {
@@ -850,148 +877,161 @@ int dash_trace_bwd(const void* q, const void* k, const void* v, const void* o, c
                    const float* lse, void* dq, void* dk, void* dv, int B, int H, int S, int D,
                    int causal, int schedule, void* stream, unsigned long long* host_trace,
                    long long cap, int* num_ctas, int* rows_per_cta) {
-  int rc = check_shape(B, H, S, D);
-  if (rc) return rc;
-  if (causal != 0 && causal != 1) return DASH_ERR_INVALID_ARG;
-  if (schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_ATOMIC) return DASH_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
-      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !host_trace ||
-      !num_ctas || !rows_per_cta)
-    return DASH_ERR_INVALID_ARG;
-  if (!dash::schedule_supported(schedule, S / 128, causal)) return DASH_ERR_UNSUPPORTED;
-  if (B == 0 || H == 0) return DASH_ERR_INVALID_ARG;
-  int dev = 0;
-  DASH_CUDA(cudaGetDevice(&dev));
-  const bool atomic = (schedule == DASH_SCHED_ATOMIC);
-  int ctas = 0;
-  {
-    std::lock_guard<std::mutex> lk(g_mu);
-    rc = (D == 64) ? (atomic ? num_ctas_for<64, true>(dev, &ctas) : num_ctas_for<64, false>(dev, &ctas))
-                   : (atomic ? num_ctas_for<128, true>(dev, &ctas) : num_ctas_for<128, false>(dev, &ctas));
-  }
-  if (rc) return rc;
-  dash::Table t;
-  std::string err;
-  if (!dash::build_table(B * H, S / 128, causal, schedule, ctas, &t, &err)) return DASH_ERR_UNSUPPORTED;
-  int rows = 0;
-  for (int c = 0; c < ctas; ++c) {
-    int n = 0;
-    for (int ci = t.cta_off[c]; ci < t.cta_off[c + 1]; ++ci) n += t.chains[ci].pair_cnt;
-    rows = n > rows ? n : rows;
-  }
-  const size_t n_entries = (size_t)ctas * rows * 8;
-  unsigned long long* dtrace = nullptr;
-  if (cudaMalloc(&dtrace, n_entries * sizeof(unsigned long long)) != cudaSuccess) return DASH_ERR_OOM;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  rc = cudaMemsetAsync(dtrace, 0, n_entries * sizeof(unsigned long long), st) == cudaSuccess
-           ? DASH_OK : DASH_ERR_CUDA;
-  if (!rc) {
-    if (D == 64)
-      rc = atomic ? launch_bwd<64, true, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
-                                               schedule, st, dev, dtrace, rows)
-                  : launch_bwd<64, false, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
-                                                schedule, st, dev, dtrace, rows);
-    else
-      rc = atomic ? launch_bwd<128, true, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
-                                                schedule, st, dev, dtrace, rows)
-                  : launch_bwd<128, false, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S,
-                                                 causal, schedule, st, dev, dtrace, rows);
-  }
-  if (!rc && cudaStreamSynchronize(st) != cudaSuccess) rc = DASH_ERR_CUDA;
-  if (!rc) {
-    const size_t n = n_entries < (size_t)cap ? n_entries : (size_t)cap;
-    if (cudaMemcpy(host_trace, dtrace, n * sizeof(unsigned long long), cudaMemcpyDeviceToHost) !=
-        cudaSuccess)
-      rc = DASH_ERR_CUDA;
-  }
-  cudaFree(dtrace);
-  *num_ctas = ctas;
-  *rows_per_cta = rows;
-  return rc;
+  return no_throw([&]() -> int {
+    int rc = check_shape(B, H, S, D);
+    if (rc) return rc;
+    if (causal != 0 && causal != 1) return DASH_ERR_INVALID_ARG;
+    if (schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_ATOMIC)
+      return DASH_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+        !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !host_trace ||
+        !num_ctas || !rows_per_cta)
+      return DASH_ERR_INVALID_ARG;
+    if (!dash::schedule_supported(schedule, S / 128, causal)) return DASH_ERR_UNSUPPORTED;
+    if (B == 0 || H == 0) return DASH_ERR_INVALID_ARG;
+    int dev = 0;
+    DASH_CUDA(cudaGetDevice(&dev));
+    const bool atomic = (schedule == DASH_SCHED_ATOMIC);
+    int ctas = 0;
+    {
+      std::lock_guard<std::mutex> lk(g_mu);
+      if (D == 64)
+        rc = atomic ? num_ctas_for<64, true>(dev, &ctas) : num_ctas_for<64, false>(dev, &ctas);
+      else
+        rc = atomic ? num_ctas_for<128, true>(dev, &ctas) : num_ctas_for<128, false>(dev, &ctas);
+    }
+    if (rc) return rc;
+    dash::Table t;
+    std::string err;
+    if (!dash::build_table(B * H, S / 128, causal, schedule, ctas, &t, &err))
+      return DASH_ERR_UNSUPPORTED;
+    int rows = 0;
+    for (int c = 0; c < ctas; ++c) {
+      int n = 0;
+      for (int ci = t.cta_off[c]; ci < t.cta_off[c + 1]; ++ci) n += t.chains[ci].pair_cnt;
+      rows = n > rows ? n : rows;
+    }
+    const size_t n_entries = (size_t)ctas * rows * 8;
+    unsigned long long* dtrace = nullptr;
+    if (cudaMalloc(&dtrace, n_entries * sizeof(unsigned long long)) != cudaSuccess)
+      return DASH_ERR_OOM;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    rc = cudaMemsetAsync(dtrace, 0, n_entries * sizeof(unsigned long long), st) == cudaSuccess
+             ? DASH_OK : DASH_ERR_CUDA;
+    if (!rc) {
+      if (D == 64)
+        rc = atomic ? launch_bwd<64, true, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S,
+                                                 causal, schedule, st, dev, dtrace, rows)
+                    : launch_bwd<64, false, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S,
+                                                  causal, schedule, st, dev, dtrace, rows);
+      else
+        rc = atomic ? launch_bwd<128, true, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S,
+                                                  causal, schedule, st, dev, dtrace, rows)
+                    : launch_bwd<128, false, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S,
+                                                   causal, schedule, st, dev, dtrace, rows);
+    }
+    if (!rc && cudaStreamSynchronize(st) != cudaSuccess) rc = DASH_ERR_CUDA;
+    if (!rc) {
+      const size_t n = n_entries < (size_t)cap ? n_entries : (size_t)cap;
+      if (cudaMemcpy(host_trace, dtrace, n * sizeof(unsigned long long), cudaMemcpyDeviceToHost) !=
+          cudaSuccess)
+        rc = DASH_ERR_CUDA;
+    }
+    cudaFree(dtrace);
+    *num_ctas = ctas;
+    *rows_per_cta = rows;
+    return rc;
+  }, DASH_ERR_OOM, DASH_ERR_INVALID_ARG);
 }
 
 long long dash_sched_table_gqa(int n_heads, int group, int N, int causal, int schedule,
                                int num_ctas, int* rows, long long cap) {
-  dash::Table t;
-  std::string err;
-  if (group < 1 || n_heads < 1 || n_heads % group != 0) return -DASH_ERR_INVALID_ARG;
-  if (!dash::build_table_grouped(n_heads, group, N, causal, schedule, num_ctas, &t, &err))
-    return -DASH_ERR_UNSUPPORTED;
-  if (!dash::validate_table(t, &err)) return -DASH_ERR_SCHEDULE;
-  long long n = 0;
-  for (int c = 0; c < t.num_ctas; ++c)
-    for (int ci = t.cta_off[c]; ci < t.cta_off[c + 1]; ++ci) {
-      const dash::Chain& ch = t.chains[ci];
-      for (int i = 0; i < ch.pair_cnt; ++i, ++n) {
-        if (rows && n < cap) {
-          const uint32_t w = t.pairs[ch.pair_off + i];
-          int* r = rows + 6 * n;
-          r[0] = c;
-          r[1] = ch.bh;
-          r[2] = ch.kv;
-          r[3] = dash::pair_q(w);
-          r[4] = dash::pair_pos(w);
-          r[5] = ci;
+  return no_throw([&]() -> long long {
+    dash::Table t;
+    std::string err;
+    if (group < 1 || n_heads < 1 || n_heads % group != 0) return -DASH_ERR_INVALID_ARG;
+    if (!dash::build_table_grouped(n_heads, group, N, causal, schedule, num_ctas, &t, &err))
+      return -DASH_ERR_UNSUPPORTED;
+    if (!dash::validate_table(t, &err)) return -DASH_ERR_SCHEDULE;
+    long long n = 0;
+    for (int c = 0; c < t.num_ctas; ++c)
+      for (int ci = t.cta_off[c]; ci < t.cta_off[c + 1]; ++ci) {
+        const dash::Chain& ch = t.chains[ci];
+        for (int i = 0; i < ch.pair_cnt; ++i, ++n) {
+          if (rows && n < cap) {
+            const uint32_t w = t.pairs[ch.pair_off + i];
+            int* r = rows + 6 * n;
+            r[0] = c;
+            r[1] = ch.bh;
+            r[2] = ch.kv;
+            r[3] = dash::pair_q(w);
+            r[4] = dash::pair_pos(w);
+            r[5] = ci;
+          }
         }
       }
-    }
-  return n;
+    return n;
+  }, -DASH_ERR_OOM, -DASH_ERR_INVALID_ARG);
 }
 
 long long dash_sched_table_part(int n_heads, int N, int causal, int schedule, int num_ctas,
                                 int h0, int h1, int* rows, long long cap) {
-  dash::Table full, t;
-  std::string err;
-  if (!dash::build_table(n_heads, N, causal, schedule, num_ctas, &full, &err))
-    return -DASH_ERR_UNSUPPORTED;
-  if (!dash::validate_table(full, &err)) return -DASH_ERR_SCHEDULE;
-  if (!dash::split_table(full, h0, h1, &t)) return -DASH_ERR_INVALID_ARG;
-  if (!dash::validate_table(t, &err)) return -DASH_ERR_SCHEDULE;
-  long long n = 0;
-  for (int c = 0; c < t.num_ctas; ++c)
-    for (int ci = t.cta_off[c]; ci < t.cta_off[c + 1]; ++ci) {
-      const dash::Chain& ch = t.chains[ci];
-      for (int i = 0; i < ch.pair_cnt; ++i, ++n) {
-        if (rows && n < cap) {
-          const uint32_t w = t.pairs[ch.pair_off + i];
-          int* r = rows + 6 * n;
-          r[0] = c;
-          r[1] = ch.bh;
-          r[2] = ch.kv;
-          r[3] = dash::pair_q(w);
-          r[4] = dash::pair_pos(w);
-          r[5] = ci;
+  return no_throw([&]() -> long long {
+    dash::Table full, t;
+    std::string err;
+    if (!dash::build_table(n_heads, N, causal, schedule, num_ctas, &full, &err))
+      return -DASH_ERR_UNSUPPORTED;
+    if (!dash::validate_table(full, &err)) return -DASH_ERR_SCHEDULE;
+    if (!dash::split_table(full, h0, h1, &t)) return -DASH_ERR_INVALID_ARG;
+    if (!dash::validate_table(t, &err)) return -DASH_ERR_SCHEDULE;
+    long long n = 0;
+    for (int c = 0; c < t.num_ctas; ++c)
+      for (int ci = t.cta_off[c]; ci < t.cta_off[c + 1]; ++ci) {
+        const dash::Chain& ch = t.chains[ci];
+        for (int i = 0; i < ch.pair_cnt; ++i, ++n) {
+          if (rows && n < cap) {
+            const uint32_t w = t.pairs[ch.pair_off + i];
+            int* r = rows + 6 * n;
+            r[0] = c;
+            r[1] = ch.bh;
+            r[2] = ch.kv;
+            r[3] = dash::pair_q(w);
+            r[4] = dash::pair_pos(w);
+            r[5] = ci;
+          }
         }
       }
-    }
-  return n;
+    return n;
+  }, -DASH_ERR_OOM, -DASH_ERR_INVALID_ARG);
 }
 
 long long dash_sched_table(int n_heads, int N, int causal, int schedule, int num_ctas, int* rows,
                            long long cap) {
-  dash::Table t;
-  std::string err;
-  if (!dash::build_table(n_heads, N, causal, schedule, num_ctas, &t, &err))
-    return -DASH_ERR_UNSUPPORTED;
-  if (!dash::validate_table(t, &err)) return -DASH_ERR_SCHEDULE;
-  long long n = 0;
-  for (int c = 0; c < t.num_ctas; ++c)
-    for (int ci = t.cta_off[c]; ci < t.cta_off[c + 1]; ++ci) {
-      const dash::Chain& ch = t.chains[ci];
-      for (int i = 0; i < ch.pair_cnt; ++i, ++n) {
-        if (rows && n < cap) {
-          const uint32_t w = t.pairs[ch.pair_off + i];
-          int* r = rows + 6 * n;
-          r[0] = c;
-          r[1] = ch.bh;
-          r[2] = ch.kv;
-          r[3] = dash::pair_q(w);
-          r[4] = dash::pair_pos(w);
-          r[5] = ci;
+  return no_throw([&]() -> long long {
+    dash::Table t;
+    std::string err;
+    if (!dash::build_table(n_heads, N, causal, schedule, num_ctas, &t, &err))
+      return -DASH_ERR_UNSUPPORTED;
+    if (!dash::validate_table(t, &err)) return -DASH_ERR_SCHEDULE;
+    long long n = 0;
+    for (int c = 0; c < t.num_ctas; ++c)
+      for (int ci = t.cta_off[c]; ci < t.cta_off[c + 1]; ++ci) {
+        const dash::Chain& ch = t.chains[ci];
+        for (int i = 0; i < ch.pair_cnt; ++i, ++n) {
+          if (rows && n < cap) {
+            const uint32_t w = t.pairs[ch.pair_off + i];
+            int* r = rows + 6 * n;
+            r[0] = c;
+            r[1] = ch.bh;
+            r[2] = ch.kv;
+            r[3] = dash::pair_q(w);
+            r[4] = dash::pair_pos(w);
+            r[5] = ci;
+          }
         }
       }
-    }
-  return n;
+    return n;
+  }, -DASH_ERR_OOM, -DASH_ERR_INVALID_ARG);
 }
 
 int dash_sched_simulate(int n_heads, int N, int causal, int schedule, int num_ctas,
@@ -1007,40 +1047,46 @@ int dash_sched_simulate_gqa(int n_heads, int group, int N, int causal, int sched
                             int num_ctas, double w_compute, double w_reduce, int dq_buffers,
                             int dq_chains, double* critical_path, double* makespan,
                             double* bubble_time, long long* stalls) {
-  if (w_compute < 0 || w_reduce < 0 || dq_chains < 1) return DASH_ERR_INVALID_ARG;
-  if (group < 1 || n_heads < 1 || n_heads % group != 0) return DASH_ERR_INVALID_ARG;
-  dash::Table t;
-  std::string err;
-  if (!dash::build_table_grouped(n_heads, group, N, causal, schedule, num_ctas, &t, &err))
-    return DASH_ERR_UNSUPPORTED;
-  if (!dash::validate_table(t, &err)) return DASH_ERR_SCHEDULE;
-  dash::SimResult r;
-  if (!dash::simulate_table(t, w_compute, w_reduce, dq_buffers, dq_chains, &r, &err))
-    return DASH_ERR_SCHEDULE;
-  if (critical_path) *critical_path = r.critical_path;
-  if (makespan) *makespan = r.makespan;
-  if (bubble_time) *bubble_time = r.bubble_time;
-  if (stalls) *stalls = r.stalls;
-  return DASH_OK;
+  return no_throw([&]() -> int {
+    if (w_compute < 0 || w_reduce < 0 || dq_chains < 1) return DASH_ERR_INVALID_ARG;
+    if (group < 1 || n_heads < 1 || n_heads % group != 0) return DASH_ERR_INVALID_ARG;
+    dash::Table t;
+    std::string err;
+    if (!dash::build_table_grouped(n_heads, group, N, causal, schedule, num_ctas, &t, &err))
+      return DASH_ERR_UNSUPPORTED;
+    if (!dash::validate_table(t, &err)) return DASH_ERR_SCHEDULE;
+    dash::SimResult r;
+    if (!dash::simulate_table(t, w_compute, w_reduce, dq_buffers, dq_chains, &r, &err))
+      return DASH_ERR_SCHEDULE;
+    if (critical_path) *critical_path = r.critical_path;
+    if (makespan) *makespan = r.makespan;
+    if (bubble_time) *bubble_time = r.bubble_time;
+    if (stalls) *stalls = r.stalls;
+    return DASH_OK;
+  }, DASH_ERR_OOM, DASH_ERR_INVALID_ARG);
 }
 
 int dash_sched_check(int n_heads, int N, int causal, int num_ctas, const int* rows,
                      long long n_rows) {
-  if (causal != 0 && causal != 1) return DASH_ERR_INVALID_ARG;
-  dash::Table t;
-  std::string err;
-  if (!dash::table_from_rows(n_heads, N, causal, num_ctas, rows, n_rows, &t, &err))
-    return DASH_ERR_INVALID_ARG;
-  return dash::validate_table(t, &err) ? DASH_OK : DASH_ERR_SCHEDULE;
+  return no_throw([&]() -> int {
+    if (causal != 0 && causal != 1) return DASH_ERR_INVALID_ARG;
+    dash::Table t;
+    std::string err;
+    if (!dash::table_from_rows(n_heads, N, causal, num_ctas, rows, n_rows, &t, &err))
+      return DASH_ERR_INVALID_ARG;
+    return dash::validate_table(t, &err) ? DASH_OK : DASH_ERR_SCHEDULE;
+  }, DASH_ERR_OOM, DASH_ERR_INVALID_ARG);
 }
 
 int dash_dag_longest_path(int n_nodes, int n_edges, const int* src, const int* dst, const double* w,
                           double* depth, double* height, double* cp) {
-  if (n_nodes < 0 || n_edges < 0 || (n_edges > 0 && (!src || !dst || !w)))
-    return DASH_ERR_INVALID_ARG;
-  if (!dash::dag_longest_path(n_nodes, n_edges, src, dst, w, depth, height, cp))
-    return DASH_ERR_INVALID_ARG;
-  return DASH_OK;
+  return no_throw([&]() -> int {
+    if (n_nodes < 0 || n_edges < 0 || (n_edges > 0 && (!src || !dst || !w)))
+      return DASH_ERR_INVALID_ARG;
+    if (!dash::dag_longest_path(n_nodes, n_edges, src, dst, w, depth, height, cp))
+      return DASH_ERR_INVALID_ARG;
+    return DASH_OK;
+  }, DASH_ERR_OOM, DASH_ERR_INVALID_ARG);
 }
 
 }  // extern "C"

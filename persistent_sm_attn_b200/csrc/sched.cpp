@@ -254,7 +254,15 @@ bool split_table(const Table& full, int h0, int h1, Table* out) {
 bool validate_table(const Table& t, std::string* err) {
   auto fail = [&](const char* m) { if (err) *err = m; return false; };
   const int N = t.N;
-  if ((int)t.cta_off.size() != t.num_ctas + 1) return fail("bad cta offsets");
+  if (t.n_heads < 1 || N < 1 || N > 32767 || t.num_ctas < 1) return fail("bad table shape");
+  if ((int)t.cta_off.size() != t.num_ctas + 1 || t.cta_off[0] != 0 ||
+      t.cta_off[t.num_ctas] != (long long)t.chains.size())
+    return fail("bad cta offsets");
+  // the pair count is fixed by the mask; checking it first bounds the scratch below by
+  // the table's own size, whatever n_heads a caller-supplied table claims
+  const long long per_head = t.causal ? (long long)N * (N + 1) / 2 : (long long)N * N;
+  if ((long long)t.n_pairs() != (long long)t.n_heads * per_head)
+    return fail("table has missing or extra pairs");
   const long long nblk = (long long)t.n_heads * N;
   std::vector<uint8_t> seen((size_t)nblk * N, 0);       // (bh, kv, q)
   std::vector<uint8_t> chain_seen((size_t)nblk, 0);     // (bh, kv)

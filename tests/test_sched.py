@@ -114,6 +114,14 @@ def test_check_rejects_coverage_and_position_errors():
     assert binding.dash_sched_check(1, 4, False, 4, [(5, 0, 0, 0, 0, 0)]) == 1   # CTA out of range
 
 
+def test_check_bounds_its_scratch_by_the_rows_given():
+    """A caller's table that claims a million heads of 32767 tiles is rejected by its
+    pair count before any per-block scratch is sized from the claim."""
+    rows = binding.dash_sched_table(1, 4, False, "shift", 4)
+    assert binding.dash_sched_check(10**6, 32767, False, 4, rows) == 6
+    assert binding.dash_sched_check(1, 4, False, 4, rows + rows[-1:]) == 6   # an extra pair
+
+
 @pytest.mark.parametrize("name,N,causal,heads,ctas", [
     (sc.SHIFT, 3, False, 1, 3), (sc.SHIFT, 4, False, 2, 5), (sc.NAIVE_ASC, 3, False, 1, 3),
     (sc.NAIVE_ASC, 4, True, 2, 3), (sc.DESCENDING, 4, True, 1, 4), (sc.DESCENDING, 3, False, 2, 4),
