@@ -29,7 +29,10 @@
  *     The softmax scale is 1/sqrt(D).  Causal masks are top-left aligned:
  *     query i attends to keys j <= i.
  *   - Supported shapes: D in {64, 128}, S a positive multiple of 128,
- *     B * H * S < 2^31.  Other shapes return DASH_ERR_UNSUPPORTED.
+ *     B * H * S < 2^31, and a schedule table of at most 2^31 - 1 pairs
+ *     (B * H * N^2 for a full mask, half that plus the diagonal for a causal
+ *     one, N = S / 128).  Other shapes return DASH_ERR_UNSUPPORTED.
+ *   - No C++ exception leaves the library: every entry point returns a status.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
  *     asynchronous: DASH_OK means the work was enqueued.  Argument and launch
  *     errors are returned at once; errors found on the device (a spin wait
@@ -61,7 +64,7 @@ typedef enum {
   DASH_ERR_UNSUPPORTED = 2,   /* shape or schedule/mask combination not provided       */
   DASH_ERR_CUDA = 3,          /* a CUDA runtime call failed                            */
   DASH_ERR_TIMEOUT = 4,       /* a device spin wait ran out (see dash_attn_sync_status)*/
-  DASH_ERR_OOM = 5,           /* workspace allocation failed                           */
+  DASH_ERR_OOM = 5,           /* a device or host allocation failed                    */
   DASH_ERR_SCHEDULE = 6       /* schedule table failed validation (e.g. would deadlock)*/
 } dash_status_t;
 
