@@ -83,3 +83,21 @@ def test_argument_errors_need_no_gpu(lib):
 def test_dag_cycle_rejected():
     with pytest.raises(binding.DashError):
         binding.dash_dag_longest_path(2, [(0, 1, 1.0), (1, 0, 1.0)])
+
+
+def test_empty_batches_are_no_ops_without_a_device(lib):
+    """B = 0 or H = 0: nothing to compute, so every entry point returns DASH_OK after
+    its argument checks and before any CUDA call (none can succeed on this host)."""
+    buf = ctypes.create_string_buffer(64)
+    al = (ctypes.addressof(buf) + 15) // 16 * 16
+    good = [ctypes.c_void_p(al)] * 9
+    for B, H in ((0, 4), (2, 0)):
+        assert _bwd(lib, good, B=B, H=H) == 0
+        assert lib.dash_attn_fwd(*good[:5], B, H, 128, 64, 0, None) == 0
+        assert lib.dash_attn_bwd_gqa(*good, B, H, 1, 128, 64, 0, 2, None) == 0
+        assert lib.dash_attn_fwd_gqa(*good[:5], B, H, 1, 128, 64, 0, None) == 0
+        assert lib.dash_attn_bwd_host(*good, B, H, 256, 64, 1, 3, None) == 0
+        assert lib.dash_attn_bwd_noalloc(*good, B, H, 256, 128, 1, 1, None) == 0
+    # argument errors still come first
+    assert _bwd(lib, good, B=0, D=96) == 2
+    assert _bwd(lib, good, B=0, sched=9) == 1
