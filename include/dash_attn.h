@@ -244,7 +244,8 @@ int dash_attn_bwd_host(const void* q, const void* k, const void* v, const void* 
 
 /*
  * Schedule table of a whole grid (DASH summary §2.2), in CTA order.
- * n_heads = B*H heads of N = S/128 tiles on num_ctas persistent CTAs.
+ * n_heads = B*H heads of N = S/128 tiles on num_ctas persistent CTAs
+ * (1 <= num_ctas <= 65536; tables of at most 2^31 - 1 pairs).
  * If rows != NULL, writes up to cap rows of 6 ints:
  *   (cta, head, kv_tile, q_tile, position_in_dQ_order, chain_index).
  * Returns the total number of rows (pairs), or a negative dash_status_t

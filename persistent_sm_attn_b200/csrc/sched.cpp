@@ -100,8 +100,8 @@ bool build_table(int n_heads, int N, int causal, int schedule, int num_ctas, Tab
 
 bool build_table_grouped(int n_heads, int group, int N, int causal, int schedule,
                          int num_ctas, Table* out, std::string* err) {
-  if (n_heads < 1 || num_ctas < 1 || group < 1 || n_heads % group != 0 ||
-      !schedule_supported(schedule, N, causal)) {
+  if (n_heads < 1 || num_ctas < 1 || num_ctas > kMaxTableCtas || group < 1 ||
+      n_heads % group != 0 || !schedule_supported(schedule, N, causal)) {
     if (err) *err = "schedule not defined for this mask / tile count / head grouping";
     return false;
   }
@@ -196,7 +196,8 @@ bool build_table_grouped(int n_heads, int group, int N, int causal, int schedule
 bool table_from_rows(int n_heads, int N, int causal, int num_ctas, const int* rows,
                      long long n_rows, Table* out, std::string* err) {
   auto fail = [&](const char* m) { if (err) *err = m; return false; };
-  if (n_heads < 1 || N < 1 || N > 32767 || num_ctas < 1 || n_rows < 0 || (n_rows > 0 && !rows))
+  if (n_heads < 1 || N < 1 || N > 32767 || num_ctas < 1 || num_ctas > kMaxTableCtas ||
+      n_rows < 0 || (n_rows > 0 && !rows))
     return fail("bad table shape");
   Table t;
   t.n_heads = n_heads; t.N = N; t.causal = causal; t.schedule = NAIVE_ASC; t.num_ctas = num_ctas;

@@ -16,6 +16,10 @@ namespace dash {
 
 enum Schedule { NAIVE_ASC = 0, DESCENDING = 1, SHIFT = 2, SYM_SHIFT = 3, ATOMIC = 4 };
 
+// Upper bound on a table's CTA count (the kernel's grid is the SM count times the CTAs
+// resident per SM); larger requests are refused instead of sizing per-CTA lists by them.
+constexpr int kMaxTableCtas = 65536;
+
 struct Chain {           // one KV tile of one head, run back to back on one CTA
   int32_t bh;            // b * H + h
   int32_t kv;            // KV tile index

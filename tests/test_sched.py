@@ -178,3 +178,11 @@ def test_longest_path_matches_bruteforce_and_lemma():
                     assert cp2 == cp
                 if depth[v] + height[v] == cp:
                     assert (cp2 == cp) == (depth[u] <= depth[v])
+
+
+def test_table_cta_count_is_bounded():
+    lib = binding.load()
+    assert lib.dash_sched_table(2, 4, 0, 2, 65536, None, 0) == 32
+    assert lib.dash_sched_table(2, 4, 0, 2, 65537, None, 0) == -2
+    assert lib.dash_sched_table(2, 4, 0, 2, 2**31 - 1, None, 0) == -2
+    assert binding.dash_sched_check(1, 4, False, 2**31 - 1, []) == 1
