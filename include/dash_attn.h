@@ -196,6 +196,12 @@ int dash_release_workspace(void);
  *   - Set-up: the first call on a device (with that device current) looks up
  *     the array's device address and sizes the persistent grid; make that
  *     first call before any stream capture begins.
+ *   - Schedule tables: a call whose (B*H, S, causal, schedule) differs from
+ *     the previous call's uploads its table into the array.  On a capturing
+ *     stream that upload is refused with DASH_ERR_UNSUPPORTED: make one call
+ *     with the shape before capturing it.  A captured call reads the table the
+ *     array holds when the graph runs, so replay the graph only while no call
+ *     with another shape has run since its capture.
  *   - Sharing: every call uses the same array, which keeps the previous call's
  *     contents; the call clears what must start at zero.  Calls that overlap
  *     on the GPU (for example on two streams without ordering between them)

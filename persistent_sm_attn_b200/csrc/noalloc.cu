@@ -180,6 +180,14 @@ int noalloc_launch(const void* q, const void* k, const void* v, const void* o, c
   const size_t end = off_pair + align256(t.pairs.size() * sizeof(uint32_t));
   if (end > kNoallocScratchBytes) return DASH_ERR_OOM;
   if (std::memcmp(key, st->table_key, sizeof(key)) != 0) {
+    // A capturing stream would record the upload as a copy from host memory that is
+    // gone when the graph runs: a new table is only uploaded outside capture.
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) {
+      cudaGetLastError();
+      return DASH_ERR_CUDA;
+    }
+    if (cap != cudaStreamCaptureStatusNone) return DASH_ERR_UNSUPPORTED;
     if (!dash::validate_table(t, &msg)) return DASH_ERR_SCHEDULE;
     if (cudaMemcpyAsync(p0 + off_cta, t.cta_off.data(), t.cta_off.size() * sizeof(int),
                         cudaMemcpyHostToDevice, stream) != cudaSuccess ||
