@@ -33,6 +33,7 @@ sys.path.insert(0, ROOT)
 from persistent_sm_attn_b200.inputs import WORKLOADS, seed_of  # noqa: E402
 
 METRIC = "deterministic attn-bwd TFLOPS (% of B200 bf16 peak); det/nondet throughput ratio"
+DEFAULT_WORKLOAD = 3  # causal_b4_h32_s16384_d64, the workload with the most FLOPs
 
 
 def _peaks():
@@ -66,6 +67,15 @@ def _recorded_traffic(workload: str, schedule: str):
     except OSError:
         pass
     return None
+
+
+def _config(w, sched, world, h_kv):
+    """The config object of a JSON line; both arms print the same one, so the
+    reference arm's line names exactly the workload this arm times."""
+    return {"workload": w.name, "B": w.B, "H": w.H, "H_kv": h_kv, "S": w.S, "D": w.D,
+            "mask": "causal" if w.causal else "full", "sigma": w.sigma, "schedule": sched,
+            "parallelism": f"dp{world} (independent heads)",
+            "l2": "flushed before every timed step (512 MiB write)"}
 
 
 class ClockSampler:
@@ -278,11 +288,7 @@ def run_ours(args):
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic (seeded normal bf16 Q, K, V, dO; O and LSE from the library forward)",
-            "config": {"workload": w.name, "B": w.B, "H": w.H,
-                       "H_kv": args.kv_heads if gqa else w.H, "S": w.S, "D": w.D,
-                       "mask": "causal" if w.causal else "full", "sigma": w.sigma,
-                       "schedule": sched, "parallelism": f"dp{world} (independent heads)",
-                       "l2": "flushed before every timed step (512 MiB write)"},
+            "config": _config(w, sched, world, args.kv_heads if gqa else w.H),
             "pct_of_peak": round(100 * value / (peak * world), 2),
             "schedules_tflops": det,
             "det_nondet_ratio": (round(best_det / det["atomic"], 4)
@@ -414,9 +420,8 @@ def run_reference(args):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic (seeded normal bf16 Q, K, V, dO widened to fp64)",
-        "config": {"workload": w.name, "B": w.B, "H": w.H,
-                   "H_kv": args.kv_heads if gqa else w.H, "S": w.S, "D": w.D,
-                   "mask": "causal" if w.causal else "full", "schedule": "none (order-free)"},
+        "config": _config(w, args.schedule or w.schedules[0], world,
+                          args.kv_heads if gqa else w.H),
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores,
                          "kind": "oracle",
                          "sample": f"each step: >= {args.cpu_seconds / max(1, args.steps):.1f} s "
@@ -433,7 +438,8 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", type=int, default=1)
+    # the default is the largest workload: B=4 H=32 S=16384 D=64, causal
+    ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD)
     ap.add_argument("--schedule", default=None)
     ap.add_argument("--no-compare", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -81,6 +81,19 @@ def paths_longest(n_nodes: int, edges):
     return cp, depth, height
 
 
+def order_preds(p: int, nc: int, chains: int):
+    """Positions whose reductions must be done before position p of a dQ block
+    with nc contributors starts its own (the accumulation-order arcs).
+
+    Position p adds into chain p mod K after position p - K of the same chain.
+    The block's last position also waits for the last position of every other
+    chain, since it adds their sums (those are positions nc-K .. nc-2)."""
+    preds = [p - chains] if p >= chains else []
+    if p == nc - 1:
+        preds += list(range(max(0, p - chains + 1), p))
+    return preds
+
+
 def schedule_graph(table, c: float, r: float, beta: int | None, chains: int = 1):
     """Build the event graph of a packed schedule table.
 
@@ -105,10 +118,7 @@ def schedule_graph(table, c: float, r: float, beta: int | None, chains: int = 1)
         for n, (hd, kv, q, p, nc) in enumerate(seq):
             a = index[(sl, n)]
             edges += [(a, a + 1, c), (a + 1, a + 2, 0.0), (a + 2, a + 3, r)]
-            preds = [p - chains] if p >= chains else []
-            if p == nc - 1:
-                preds += list(range(max(0, p - chains + 1), p))
-            for pp in preds:
+            for pp in order_preds(p, nc, chains):
                 edges.append((by_block[(hd, q, pp)] + 3, a + 2, 0.0))
             if n > 0:
                 prev = index[(sl, n - 1)]

@@ -205,3 +205,142 @@ def test_buffer_depth_one_serialises_naive_order():
     _, _, _, st_naive = dag.simulate(_one_head(sc.NAIVE_ASC, N, False), c, r, 1)
     _, _, _, st_shift = dag.simulate(_one_head(sc.SHIFT, N, False), c, r, 1)
     assert st_naive > 0 and st_shift == 0
+
+
+# ---------------------------------------------------------------------------
+# Pins of the multi-chain accumulation order, the simulator's other outputs and
+# the multi-round positions
+
+def _closed_form(name, causal, N, c, r, chains):
+    """Critical path of one head, one CTA slot per unit, unbounded buffers,
+    r <= c / 2, derived by hand from the event graph's arcs:
+
+    * shift (full) and symmetric shift (causal): each reduction starts when its
+      own partial is ready, so the path is the longest chain plus one
+      reduction, N c + r and (N + 1) c + r, for any number of chains.
+    * descending, causal: every contributor of block q arrives at step N-1-q
+      (positions ascend in KV), the reductions of block q queue behind each
+      other, and block 0 (one contributor, last step) ends the path: N c + r.
+    * naive ascending (both masks) and descending (full): the reductions of the
+      last block queue at the end.  One chain: N c + N r.  Two chains: the
+      block's positions split into even and odd runs of ceil(N/2) and
+      floor(N/2) reductions; the last position waits for the other run, so
+      the path holds floor(N/2) + 1 reductions after N c.
+    """
+    if name == sc.SYM_SHIFT:
+        return (N + 1) * c + r
+    if name == sc.SHIFT or (name == sc.DESCENDING and causal):
+        return N * c + r
+    return N * c + (N * r if chains == 1 else (N // 2 + 1) * r)
+
+
+def _closed_forms_hold(chains_list=(1, 2)):
+    for c, r in ((1.0, 0.15), (1.0, 0.4)):
+        for N in range(1, 7):
+            for name in sc.ALL:
+                for causal in (False, True):
+                    if not sc.supported(name, N, causal):
+                        continue
+                    tab = _one_head(name, N, causal)
+                    for K in chains_list:
+                        cp, makespan, bubble, stalls = dag.simulate(tab, c, r, None, K)
+                        L = max(len(u) for u in tab)
+                        if abs(cp - _closed_form(name, causal, N, c, r, K)) > 1e-9:
+                            return False
+                        # unbounded buffers: compute never waits, and each slot
+                        # idles for the critical path minus its own compute
+                        if stalls != 0 or abs(makespan - L * c) > 1e-9:
+                            return False
+                        want_bubble = sum(cp - c * len(u) for u in tab if u)
+                        if abs(bubble - want_bubble) > 1e-9:
+                            return False
+    return True
+
+
+def test_dag_closed_forms_one_and_two_chains():
+    assert _closed_forms_hold()
+
+
+# Hand-worked: naive ascending, full mask, N = 2, c = 1, r = 1.5, one dQ buffer
+# per slot (beta = 1), two accumulation chains.  Slot k holds KV tile k and
+# visits Q tiles 0, 1; its pairs have position k in both blocks.  Position 0
+# has no predecessor; position 1 is the last of its block and waits for
+# position 0 (the other chain's last).  Event times (a, b, s, d):
+#   slot 0, q0: a 0, b 1, s 1, d 2.5
+#   slot 0, q1: a 1, b max(2, d_prev 2.5) = 2.5 (stall), s 2.5, d 4
+#   slot 1, q0: a 0, b 1, s max(1, d(slot 0, q0) 2.5) = 2.5, d 4
+#   slot 1, q1: a 1, b max(2, d_prev 4) = 4 (stall), s max(4, 4, d(slot 0, q1) 4) = 4, d 5.5
+# critical path 5.5; makespan (last compute end) max(2.5, 4) = 4;
+# bubble (5.5 - 2) + (5.5 - 2) = 7; stalls 2.
+HAND_NAIVE_N2 = ((1.0, 1.5, 1, 2), (5.5, 4.0, 7.0, 2))
+# Hand-worked: naive ascending, full mask, N = 3, c = 1, r = 0.4, beta = 1, two
+# chains.  Positions 0 and 1 start their reductions as soon as their partials
+# are ready: d = t + 1.4 at step t.  Position 2 (last) waits for positions 0
+# and 1: s = t + 1.4, d = t + 1.8; its own previous reduction (d = t + 0.8) never
+# holds up its next partial (b = t + 1), so nothing stalls.
+# critical path 3.8; makespan 3; bubble 3 x (3.8 - 3) = 2.4; stalls 0.
+HAND_NAIVE_N3 = ((1.0, 0.4, 1, 2), (3.8, 3.0, 2.4, 0))
+
+
+def _hand_tables_hold():
+    for N, ((c, r, beta, K), want) in ((2, HAND_NAIVE_N2), (3, HAND_NAIVE_N3)):
+        got = dag.simulate(_one_head(sc.NAIVE_ASC, N, False), c, r, beta, K)
+        if any(abs(g - w) > 1e-9 for g, w in zip(got, want)):
+            return False
+    return True
+
+
+def test_dag_hand_worked_tables():
+    assert _hand_tables_hold()
+
+
+@pytest.mark.parametrize("mutant", ["chain_pred_is_p_minus_1", "last_skips_other_chain",
+                                    "last_waits_only_first", "no_chain_pred"])
+def test_dag_pins_reject_planted_order_mistakes(monkeypatch, mutant):
+    """Each plausible mistake in the accumulation-order rule must fail a pin."""
+    real = dag.order_preds
+
+    def m_p1(p, nc, K):          # waits for the position one ahead, not K ahead
+        return ([p - 1] if p >= 1 else []) + \
+            ([q for q in range(max(0, p - K + 1), p) if q != p - 1] if p == nc - 1 else [])
+
+    def m_last(p, nc, K):        # the last contributor forgets the other chains
+        return [p - K] if p >= K else []
+
+    def m_first(p, nc, K):       # the last contributor waits for position 0 only
+        return ([p - K] if p >= K else []) + ([0] if p == nc - 1 and p > 0 else [])
+
+    def m_none(p, nc, K):        # no order within a chain
+        return list(range(max(0, p - K + 1), p)) if p == nc - 1 else []
+
+    fn = {"chain_pred_is_p_minus_1": m_p1, "last_skips_other_chain": m_last,
+          "last_waits_only_first": m_first, "no_chain_pred": m_none}[mutant]
+    assert real(5, 6, 2) == [3, 4]
+    monkeypatch.setattr(dag, "order_preds", fn)
+    assert not (_closed_forms_hold() and _hand_tables_hold())
+
+
+def _read_positions(name):
+    slots = []
+    for line in open(os.path.join(GOLD, name)):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        _, rest = line.split(":", 1)
+        slots.append([tuple(int(x) for x in t.split(":")) for t in rest.split()])
+    return slots
+
+
+@pytest.mark.parametrize("fname,name,heads,N,causal,slots", [
+    ("shift_n4_3slots_positions.txt", sc.SHIFT, 1, 4, False, 3),
+    ("sym_shift_n4_2heads_3slots_positions.txt", sc.SYM_SHIFT, 2, 4, True, 3),
+])
+def test_multi_round_positions_match_golden(fname, name, heads, N, causal, slots):
+    """Units that run in a later round come after every unit of an earlier
+    round in each dQ block's order (hand-worked tables)."""
+    got = sc.packed_table(name, heads, N, causal, slots)
+    want = _read_positions(fname)
+    assert [[e[:4] for e in s] for s in got] == want
+    for s in got:
+        for hd, kv, q, pos, nc in s:
+            assert nc == (q + 1 if causal else N)
