@@ -131,10 +131,11 @@ const char* dash_status_string(int status);
 int dash_set_spin_limit_us(long long us);
 
 /*
- * Failure-detection testing.  mode 1: the next deterministic dash_attn_bwd
- * (any stream) runs with a schedule table in which dQ block (head 0, Q tile 0)
- * never receives its first two partials, so its ticket waits run out; the kernel
- * still ends, with DASH_ERR_TIMEOUT reported by dash_attn_sync_status and
+ * Failure-detection testing.  mode 1: the next deterministic dash_attn_bwd or
+ * dash_attn_bwd_noalloc (any stream) runs with a schedule table in which dQ
+ * block (head 0, Q tile 0) never receives its first two partials, so its ticket
+ * waits run out; the kernel still ends, with DASH_ERR_TIMEOUT reported by
+ * dash_attn_sync_status (dash_attn_noalloc_sync_status for the second) and
  * invalid outputs.  The fault is made on the host; no memory outside the
  * call's buffers is touched.  mode 0 cancels.  Other modes: INVALID_ARG.
  */
@@ -178,42 +179,51 @@ int dash_release_workspace(void);
 /* ---------------------------------------------------------------------------
  * Backward pass that allocates nothing.
  *
- * The paper has no counterpart to this entry point; it serves callers that
- * cannot call cudaMalloc: code running while a stream is captured into a CUDA
- * graph, runtimes that hand out all device memory from their own pool, and
- * embedded users that must fix their device footprint in advance.
+ * The paper has no counterpart to this entry point.  It serves callers that
+ * cannot call cudaMalloc: runtimes that hand out all device memory from their
+ * own pool and forbid allocations outside it, and embedded or certified
+ * deployments that must fix their device footprint before they start.
  *
  * Same arguments, supported shapes, schedules and results as dash_attn_bwd
  * (q..dv caller-owned device memory; the caller still passes every input and
- * output).  All scratch memory comes from one statically allocated device
- * array of DASH_NOALLOC_SCRATCH_BYTES bytes, which every GPU that loads the
- * library holds until the process exits.  The call never calls cudaMalloc,
- * cudaFree or an allocating library routine.
+ * output), bit for bit on the deterministic schedules.  All scratch memory comes
+ * from one statically allocated device array of DASH_NOALLOC_SCRATCH_BYTES bytes,
+ * which every GPU that loads the library holds until the process exits.  The
+ * call never calls cudaMalloc, cudaFree or an allocating library routine.
  *   - Size limit: the array must hold the two fp32 dQ accumulators per block
  *     (2*B*H*S*D*4 bytes), 16 bytes of LSE and Delta terms per row (B*H*S*16), two
  *     tickets per 128-row dQ block and the schedule table; larger calls return
  *     DASH_ERR_OOM without touching the device.
  *   - Set-up: the first call on a device (with that device current) looks up
- *     the array's device address and sizes the persistent grid; make that
- *     first call before any stream capture begins.
- *   - Schedule tables: a call whose (B*H, S, causal, schedule) differs from
- *     the previous call's uploads its table into the array.  On a capturing
- *     stream that upload is refused with DASH_ERR_UNSUPPORTED: make one call
- *     with the shape before capturing it.  A captured call reads the table the
- *     array holds when the graph runs, so replay the graph only while no call
- *     with another shape has run since its capture.
+ *     the array's device address and sizes the persistent grid.
+ *   - Schedule tables: a call whose (B*H, S, causal, schedule) differs from the
+ *     previous call's copies its table from host memory into the array; while
+ *     the stream is being captured that copy is refused with
+ *     DASH_ERR_UNSUPPORTED.
  *   - Sharing: every call uses the same array, which keeps the previous call's
  *     contents; the call clears what must start at zero.  Calls that overlap
  *     on the GPU (for example on two streams without ordering between them)
  *     race on the array and give wrong results.
- *   - Device-side timeouts of this entry point are recorded in the array, not
- *     in the per-stream workspaces, so dash_attn_sync_status does not report
- *     them; the spin limit is DASH_SPIN_LIMIT_US (default 10 s).
+ *   - Errors: device-side timeouts of this entry point are recorded in the
+ *     array's error word, which dash_attn_noalloc_sync_status reads; the spin
+ *     limit is the one dash_set_spin_limit_us sets (else DASH_SPIN_LIMIT_US,
+ *     else 10 s).
  */
 #define DASH_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
 int dash_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
                           const void* dout, const float* lse, void* dq, void* dk, void* dv,
                           int B, int H, int S, int D, int causal, int schedule, void* stream);
+
+/*
+ * Status of dash_attn_bwd_noalloc on the current device: waits for `stream`,
+ * then returns and clears the array's error word.  DASH_ERR_TIMEOUT if a
+ * device wait ran out in a call since the word was last read (that call's
+ * outputs are invalid), DASH_ERR_UNSUPPORTED if a launch refused to run,
+ * DASH_OK otherwise (also before the first call on the device); DASH_ERR_CUDA
+ * if the stream reports an error.  Allocates nothing.  The paper has no
+ * counterpart to this call either.
+ */
+int dash_attn_noalloc_sync_status(void* stream);
 
 /* ---------------------------------------------------------------------------
  * Backward pass from host buffers.
@@ -296,6 +306,10 @@ long long dash_sched_table_gqa(int n_heads, int group, int N, int causal, int sc
  * CTAs of critical_path minus the CTA's compute time), stalls (pairs whose
  * partial waited for a free buffer).  Returns DASH_ERR_INVALID_ARG for
  * negative weights or dq_chains < 1.
+ * Argument mapping for a caller thinking in (B, H, S): n_heads = B * H and
+ * N = S / 128, since the table depends on those two alone; dq_chains has no
+ * counterpart in a single-order model (pass 1 for the pages' model); a bubble
+ * figure splits into bubble_time (idle time) and stalls (a count).
  */
 int dash_sched_simulate(int n_heads, int N, int causal, int schedule, int num_ctas,
                         double w_compute, double w_reduce, int dq_buffers, int dq_chains,

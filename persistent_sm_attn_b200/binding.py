@@ -25,7 +25,7 @@ EXPORTS = ("dash_attn_fwd", "dash_attn_bwd", "dash_attn_sync_status", "dash_stat
            "dash_profile_begin", "dash_profile_end", "dash_attn_bwd_noalloc",
            "dash_trace_bwd", "dash_inject_fault", "dash_sched_check", "dash_attn_bwd_host",
            "dash_sched_table_part", "dash_attn_fwd_gqa", "dash_attn_bwd_gqa",
-           "dash_sched_table_gqa")
+           "dash_sched_table_gqa", "dash_attn_noalloc_sync_status")
 
 
 class DashError(RuntimeError):
@@ -60,6 +60,7 @@ def load(path: str | None = None):
     lib.dash_attn_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
     lib.dash_attn_bwd_gqa.argtypes = [vp] * 9 + [i, i, i, i, i, i, i, vp]
     lib.dash_attn_sync_status.argtypes = [vp]
+    lib.dash_attn_noalloc_sync_status.argtypes = [vp]
     lib.dash_status_string.argtypes = [i]
     lib.dash_status_string.restype = ctypes.c_char_p
     lib.dash_set_spin_limit_us.argtypes = [ll]
@@ -82,7 +83,7 @@ def load(path: str | None = None):
     lib.dash_profile_end.argtypes = [P(d), P(d), P(ll)]
     for name in EXPORTS:
         if name not in ("dash_status_string", "dash_sched_table", "dash_sched_table_part",
-                        "dash_sched_table_gqa"):
+                        "dash_sched_table_gqa", "dash_attn_noalloc_sync_status"):
             getattr(lib, name).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -255,6 +256,12 @@ def dash_attn_bwd_noalloc(q, k, v, o, do, lse, causal: bool, schedule, dq, dk, d
 
 def dash_attn_sync_status(stream=None) -> int:
     return int(load().dash_attn_sync_status(_stream_handle(stream)))
+
+
+def dash_attn_noalloc_sync_status(stream=None) -> int:
+    """Waits for the stream and returns (and clears) the status that
+    dash_attn_bwd_noalloc's calls recorded on the current device."""
+    return int(load().dash_attn_noalloc_sync_status(_stream_handle(stream)))
 
 
 def dash_set_spin_limit_us(us: int) -> None:

@@ -20,6 +20,7 @@
 #include "aux_kernels.cuh"
 #include "bwd_kernel.cuh"
 #include "fwd_kernel.cuh"
+#include "internal.h"
 #include "sched.h"
 
 namespace {
@@ -245,14 +246,7 @@ int get_fault_table(int dev, int heads, int N, int causal, int sched, int ctas, 
   dash::Table t;
   std::string err;
   if (!dash::build_table(heads, N, causal, sched, ctas, &t, &err)) return DASH_ERR_UNSUPPORTED;
-  for (const dash::Chain& ch : t.chains)
-    if (ch.bh == 0)
-      for (int i = 0; i < ch.pair_cnt; ++i) {
-        uint32_t& w = t.pairs[ch.pair_off + i];
-        // the block's first two positions never arrive, so the first wait of both
-        // of its accumulation chains runs out
-        if (dash::pair_q(w) == 0) w = dash::pack_pair(0, dash::pair_pos(w) + 2);
-      }
+  dash::plant_missing_first_partials(&t);
   cudaFree(g_fault_table.cta_off);
   cudaFree(g_fault_table.chains);
   cudaFree(g_fault_table.pairs);
@@ -624,25 +618,16 @@ int host_bwd(const void* q, const void* k, const void* v, const void* o, const v
   return DASH_OK;
 }
 
-// C++ exceptions (std::bad_alloc from a table, a map or a vector sized by the caller's
-// arguments) must not cross the C ABI: each entry point that allocates on the host
-// returns a status instead.
-template <class R, class F>
-R no_throw_impl(F&& f, R on_oom, R on_other) {
-  try {
-    return f();
-  } catch (const std::bad_alloc&) {
-    return on_oom;
-  } catch (...) {
-    return on_other;
-  }
-}
-template <class F>
-auto no_throw(F&& f, decltype(f()) on_oom, decltype(f()) on_other) -> decltype(f()) {
-  return no_throw_impl<decltype(f())>(static_cast<F&&>(f), on_oom, on_other);
-}
-
 }  // namespace
+
+namespace dash {
+
+long long spin_limit_us() { return spin_us(); }
+int take_armed_fault() { return g_fault.exchange(0); }
+
+}  // namespace dash
+
+using dash::no_throw;
 
 extern "C" {
 

@@ -1,20 +1,18 @@
 // dash_attn_bwd_noalloc: the backward pass without any device allocation.
 //
-// Some callers cannot call cudaMalloc: code that runs while a stream is being
-// captured into a CUDA graph, runtimes that own all device memory through
-// their own pool and forbid other allocations, or embedded callers that must
-// know their whole device footprint up front.  This entry point runs the same
-// kernels as dash_attn_bwd, but takes every byte of scratch memory (the fp32
-// dQ accumulator, the tickets, the per-row Delta and scaled LSE, the error
-// words and the schedule table) from one statically allocated device array of
-// kNoallocScratchBytes.  Every device that loads the library holds that array
-// until the process exits.
+// Some callers cannot call cudaMalloc: runtimes that own all device memory
+// through their own pool and forbid allocations outside it, and embedded or
+// certified deployments that must fix their whole device footprint before
+// they start.  This entry point runs the same kernels as dash_attn_bwd, but
+// takes every byte of scratch memory (the fp32 dQ accumulators, the tickets,
+// the per-row LSE and Delta terms, the error words and the schedule table)
+// from one statically allocated device array of kNoallocScratchBytes.  Every
+// device that loads the library holds that array until the process exits.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
 #include <cstdint>
-#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -22,6 +20,7 @@
 #include "../../include/dash_attn.h"
 #include "aux_kernels.cuh"
 #include "bwd_kernel.cuh"
+#include "internal.h"
 #include "sched.h"
 
 namespace {
@@ -135,12 +134,6 @@ int noalloc_setup(int dev, DeviceState** out) {
   return DASH_OK;
 }
 
-// Spin limit of the device waits: DASH_SPIN_LIMIT_US if set, else 10 s.
-unsigned long long noalloc_spin_ns() {
-  const char* e = std::getenv("DASH_SPIN_LIMIT_US");
-  const long long us = e ? std::atoll(e) : 0;
-  return (unsigned long long)(us > 0 ? us : 10LL * 1000 * 1000) * 1000ull;
-}
 
 // Scratch bytes a call needs, table excluded.
 size_t fixed_scratch(long long rows, int D, long long blocks) {
@@ -169,17 +162,21 @@ int noalloc_launch(const void* q, const void* k, const void* v, const void* o, c
   off += align256((size_t)rows * 16);
   float* acc = reinterpret_cast<float*>(p0 + off);
   off += align256(2 * (size_t)rows * D * 4);
-  // the schedule table, built and checked on the host, then copied in
+  // the schedule table, built and checked on the host, then copied in.  A fault armed
+  // with dash_inject_fault replaces it, for this call only, by a table whose dQ block
+  // (head 0, Q tile 0) never receives its first partials.
   const long long key[6] = {B * (long long)H, N, causal, sched, ctas, (long long)off};
+  const int fault = kAtomic ? 0 : dash::take_armed_fault();
   dash::Table t;
   std::string msg;
   if (!dash::build_table(B * H, N, causal, sched, ctas, &t, &msg)) return DASH_ERR_UNSUPPORTED;
+  if (fault == 1) dash::plant_missing_first_partials(&t);
   const size_t off_cta = off;
   const size_t off_chain = off_cta + align256(t.cta_off.size() * sizeof(int));
   const size_t off_pair = off_chain + align256(t.chains.size() * sizeof(int4));
   const size_t end = off_pair + align256(t.pairs.size() * sizeof(uint32_t));
   if (end > kNoallocScratchBytes) return DASH_ERR_OOM;
-  if (std::memcmp(key, st->table_key, sizeof(key)) != 0) {
+  if (fault == 1 || std::memcmp(key, st->table_key, sizeof(key)) != 0) {
     // A capturing stream would record the upload as a copy from host memory that is
     // gone when the graph runs: a new table is only uploaded outside capture.
     cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
@@ -188,7 +185,7 @@ int noalloc_launch(const void* q, const void* k, const void* v, const void* o, c
       return DASH_ERR_CUDA;
     }
     if (cap != cudaStreamCaptureStatusNone) return DASH_ERR_UNSUPPORTED;
-    if (!dash::validate_table(t, &msg)) return DASH_ERR_SCHEDULE;
+    if (fault != 1 && !dash::validate_table(t, &msg)) return DASH_ERR_SCHEDULE;
     if (cudaMemcpyAsync(p0 + off_cta, t.cta_off.data(), t.cta_off.size() * sizeof(int),
                         cudaMemcpyHostToDevice, stream) != cudaSuccess ||
         cudaMemcpyAsync(p0 + off_chain, t.chains.data(), t.chains.size() * sizeof(int4),
@@ -196,7 +193,11 @@ int noalloc_launch(const void* q, const void* k, const void* v, const void* o, c
         cudaMemcpyAsync(p0 + off_pair, t.pairs.data(), t.pairs.size() * sizeof(uint32_t),
                         cudaMemcpyHostToDevice, stream) != cudaSuccess)
       return DASH_ERR_CUDA;
-    std::memcpy(st->table_key, key, sizeof(key));
+    // after a planted fault the next call uploads its table again
+    if (fault == 1)
+      for (long long& x : st->table_key) x = -1;
+    else
+      std::memcpy(st->table_key, key, sizeof(key));
   }
   CUtensorMap tq, tk, tv, tdo, tc;
   int rc;
@@ -207,14 +208,15 @@ int noalloc_launch(const void* q, const void* k, const void* v, const void* o, c
       (rc = noalloc_tmap_cols(&tc, cols, rows)))
     return rc;
   const float scale = 1.0f / sqrtf((float)D);
-  // The array keeps the previous call's contents: the Delta launch clears the error
-  // word, the abort flag and (deterministic path) the tickets; the atomic variant's
-  // accumulator is cleared here.
+  // The array keeps the previous call's contents: the Delta launch clears the abort
+  // flag and (deterministic path) the tickets; the atomic variant's accumulator is
+  // cleared here.  The error word (err[0]) keeps what earlier calls recorded until
+  // dash_attn_noalloc_sync_status reads and clears it.
   if (kAtomic && cudaMemsetAsync(acc, 0, (size_t)rows * D * 4, stream) != cudaSuccess)
     return DASH_ERR_CUDA;
   dash::dash_delta_kernel<D><<<dash::delta_grid<D>(rows, ctas), 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, cols,
-      rows, 1.0f / scale, tickets, kAtomic ? 0LL : blocks, err, 2);
+      rows, 1.0f / scale, tickets, kAtomic ? 0LL : blocks, err + 1, 1);
   dash::BwdParams p;
   p.cta_off = reinterpret_cast<const int*>(p0 + off_cta);
   p.chains = reinterpret_cast<const int4*>(p0 + off_chain);
@@ -232,7 +234,7 @@ int noalloc_launch(const void* q, const void* k, const void* v, const void* o, c
   p.group_log2 = 0;
   p.scale = scale;
   p.scale_log2 = p.scale * 1.4426950408889634f;
-  p.spin_ns = noalloc_spin_ns();
+  p.spin_ns = (unsigned long long)dash::spin_limit_us() * 1000ull;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ctas);
   cfg.blockDim = dim3(C::kThreads);
@@ -280,19 +282,39 @@ extern "C" int dash_attn_bwd_noalloc(const void* q, const void* k, const void* v
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return DASH_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return DASH_ERR_UNSUPPORTED;
+  // the table is built in host containers: no C++ exception may leave this function
+  return dash::no_throw([&]() -> int {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    DeviceState* st = nullptr;
+    int rc = noalloc_setup(dev, &st);
+    if (rc) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool atomic = (schedule == DASH_SCHED_ATOMIC);
+    if (D == 64)
+      return atomic ? noalloc_launch<64, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S,
+                                               causal, schedule, s, st)
+                    : noalloc_launch<64, false>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S,
+                                                causal, schedule, s, st);
+    return atomic ? noalloc_launch<128, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S,
+                                              causal, schedule, s, st)
+                  : noalloc_launch<128, false>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S,
+                                               causal, schedule, s, st);
+  }, DASH_ERR_OOM, DASH_ERR_INVALID_ARG);
+}
+
+extern "C" int dash_attn_noalloc_sync_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DASH_ERR_CUDA;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DASH_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return DASH_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  DeviceState* st = nullptr;
-  int rc = noalloc_setup(dev, &st);
-  if (rc) return rc;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const bool atomic = (schedule == DASH_SCHED_ATOMIC);
-  if (D == 64)
-    return atomic ? noalloc_launch<64, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
-                                             schedule, s, st)
-                  : noalloc_launch<64, false>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
-                                              schedule, s, st);
-  return atomic ? noalloc_launch<128, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
-                                            schedule, s, st)
-                : noalloc_launch<128, false>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
-                                             schedule, s, st);
+  const DeviceState& st = g_dev[dev];
+  if (!st.ready) return DASH_OK;  // no call has run on this device
+  unsigned h = 0;
+  if (cudaMemcpy(&h, st.base, sizeof(unsigned), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return DASH_ERR_CUDA;
+  if (h == 0) return DASH_OK;
+  if (cudaMemset(st.base, 0, sizeof(unsigned)) != cudaSuccess) return DASH_ERR_CUDA;
+  return (h & dash::dev::ERR_TIMEOUT) ? DASH_ERR_TIMEOUT : DASH_ERR_UNSUPPORTED;
 }

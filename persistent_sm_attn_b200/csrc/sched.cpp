@@ -474,4 +474,13 @@ bool simulate_table(const Table& t, double c, double r, int beta, int chains, Si
   return true;
 }
 
+void plant_missing_first_partials(Table* t) {
+  for (const Chain& ch : t->chains)
+    if (ch.bh == 0)
+      for (int i = 0; i < ch.pair_cnt; ++i) {
+        uint32_t& w = t->pairs[ch.pair_off + i];
+        if (pair_q(w) == 0) w = pack_pair(0, pair_pos(w) + 2);
+      }
+}
+
 }  // namespace dash

@@ -104,4 +104,10 @@ bool simulate_table(const Table& t, double c, double r, int beta, int chains, Si
 bool table_from_rows(int n_heads, int N, int causal, int num_ctas, const int* rows,
                      long long n_rows, Table* out, std::string* err);
 
+// Failure-detection testing: moves every partial of dQ block (head 0, Q tile 0)
+// two positions later, so the block's first two positions (the first of each
+// of its two accumulation chains) never arrive and the waits on them run out.
+// Every index stays in range; the table no longer passes validate_table.
+void plant_missing_first_partials(Table* t);
+
 }  // namespace dash

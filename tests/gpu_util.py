@@ -8,6 +8,14 @@ from persistent_sm_attn_b200.inputs import draw
 
 TOL = 5e-3  # relative Frobenius error bound on dQ, dK, dV (and O)
 
+# (label, {"dq": err, "dk": err, "dv": err}) of every parity check that ran; the
+# terminal summary prints them, so a run shows its margin to the bound
+MARGINS = []
+
+
+def log_margin(label, errs):
+    MARGINS.append((label, dict(errs)))
+
 
 def need_cuda():
     import pytest

@@ -1,36 +1,54 @@
 """Bitwise reproducibility of every deterministic schedule: 50 launches, and
-launches racing a concurrent load on another stream."""
+launches racing a concurrent load on another stream, on every workload at its
+full size (best schedule and the descending order, plus naive ascending where
+it is one of the workload's compared schedules) and on a reduced causal D = 64
+shape."""
 import pytest
 import torch
 
+from persistent_sm_attn_b200.inputs import WORKLOADS, seed_of
 from tests import gpu_util as G
 
 pytestmark = pytest.mark.gpu
 
-CASES = [
-    ((2, 16, 4096, 128, False), ("shift", "descending", "naive_asc")),
-    ((2, 8, 4096, 64, True), ("sym_shift", "descending", "naive_asc")),
-]
+
+def _det(w):
+    return tuple(s for s in w.schedules if s != "atomic")
+
+
+# (label, (B, H, S, D, causal, sigma, seed), schedules)
+CASES = [(w.name, (w.B, w.H, w.S, w.D, w.causal, w.sigma, seed_of(i)), _det(w))
+         for i, w in enumerate(WORKLOADS) if i >= 1]
+CASES.append(("causal_b2_h8_s4096_d64", (2, 8, 4096, 64, True, 1.0, 11),
+              ("sym_shift", "descending", "naive_asc")))
+IDS = [c[0] for c in CASES]
 
 
 def _same(a, b):
+    # torch.equal compares on the device
     return all(torch.equal(x, y) for x, y in zip(a, b))
 
 
-@pytest.mark.parametrize("shape,schedules", CASES)
-def test_fifty_launches_bit_identical(shape, schedules):
+def _case(shape):
+    B, H, S, D, causal, sigma, seed = shape
+    return G.make_case(B, H, S, D, causal, sigma, seed)
+
+
+@pytest.mark.parametrize("label,shape,schedules", CASES, ids=IDS)
+def test_fifty_launches_bit_identical(label, shape, schedules):
     G.need_cuda()
-    case = G.make_case(*shape, seed=11)
+    case = _case(shape)
     for sched in schedules:
         first = [t.clone() for t in G.bwd(case, sched)]
-        for _ in range(49):
-            assert _same(first, G.bwd(case, sched)), sched
+        for rep in range(49):
+            assert _same(first, G.bwd(case, sched)), (label, sched, rep)
+        del first
 
 
-@pytest.mark.parametrize("shape,schedules", CASES)
-def test_bit_identical_under_concurrent_load(shape, schedules):
+@pytest.mark.parametrize("label,shape,schedules", CASES, ids=IDS)
+def test_bit_identical_under_concurrent_load(label, shape, schedules):
     G.need_cuda()
-    case = G.make_case(*shape, seed=12)
+    case = _case(shape)
     side = torch.cuda.Stream()
     sizes = (1024, 3072, 8192)
     mats = {n: torch.randn(n, n, device="cuda", dtype=torch.bfloat16) for n in sizes}
@@ -41,8 +59,9 @@ def test_bit_identical_under_concurrent_load(shape, schedules):
             with torch.cuda.stream(side):
                 for _ in range(4):
                     mats[n] = (mats[n] @ mats[n]).clamp_(-1, 1)
-            assert _same(first, G.bwd(case, sched)), (sched, rep)
+            assert _same(first, G.bwd(case, sched)), (label, sched, rep)
         torch.cuda.synchronize()
+        del first
 
 
 def test_atomic_variant_runs_and_is_accurate():
@@ -51,4 +70,6 @@ def test_atomic_variant_runs_and_is_accurate():
     G.need_cuda()
     case = G.make_case(1, 2, 512, 64, False, seed=13)
     ref = G.oracle_full(case)
-    assert max(G.check_full(case, G.bwd(case, "atomic"), ref).values()) < G.TOL
+    errs = G.check_full(case, G.bwd(case, "atomic"), ref)
+    G.log_margin("B1 H2 S512 D64 full atomic", errs)
+    assert max(errs.values()) < G.TOL
