@@ -160,11 +160,15 @@ int dash_profile_end(double* main_ms, double* aux_ms, long long* launches);
  * a %globaltimer trace of every (KV tile, Q tile) pair, for measuring the
  * compute time c and the reduction time r of the DAG model (DASH summary
  * §2.1).  host_trace receives up to `cap` u64 entries laid out
- * [num_ctas][rows_per_cta][8] (unused rows stay 0); events per pair: 0 S^T
+ * [num_ctas][rows_per_cta][16] (unused rows stay 0); events per pair: 0 S^T
  * issued, 1 softmax done (seen by the MMA issuer), 2 tile MMAs issued, 3
  * softmax start, 4 dQ partial ready at the reducers, 5 partial drained from
  * TMEM, 6 ticket granted (0 for the first contributor of each of the block's
- * two accumulation chains), 7 reduction published or dQ written.
+ * two accumulation chains), 7 reduction published or dQ written, 8 P^T packed
+ * (end of the softmax's first phase), 9 start of its second phase, 10 dS ready,
+ * 11 P^T seen by the MMA issuer, 12 the issuer starts waiting for the S^T
+ * buffer, 13 load-add-store (or atomic adds) done, 14 the reducers start
+ * waiting for the ticket, 15 dP^T issued.
  * Allocates and frees its own trace buffer.
  */
 int dash_trace_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,

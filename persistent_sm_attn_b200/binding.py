@@ -390,14 +390,16 @@ def dash_profile_end():
 
 
 def dash_trace_bwd(q, k, v, o, do, lse, causal: bool, schedule="shift", stream=None):
-    """One traced backward; returns (dq, dk, dv, trace [ctas, rows, 8] uint64 ns)."""
+    """One traced backward; returns (dq, dk, dv, trace [ctas, rows, 16] uint64 ns),
+    the events per pair listed at dash_trace_bwd in include/dash_attn.h."""
     import numpy as np
     import torch
     _check_tensors(q, k, v, o, do, lse)
     B, H, S, D = q.shape
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     N = S // 128
-    cap = 8 * (B * H * N * N + 1024 * (N + 1))   # >= ctas * rows_per_cta * 8
+    EV = 16
+    cap = EV * (B * H * N * N + 1024 * (N + 1))   # >= ctas * rows_per_cta * EV
     buf = np.zeros(cap, dtype=np.uint64)
     nc, rows = ctypes.c_int(), ctypes.c_int()
     rc = load().dash_trace_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
@@ -406,7 +408,7 @@ def dash_trace_bwd(q, k, v, o, do, lse, causal: bool, schedule="shift", stream=N
                                buf.ctypes.data_as(ctypes.c_void_p), cap, ctypes.byref(nc),
                                ctypes.byref(rows))
     _check(rc, "dash_trace_bwd")
-    n = nc.value * rows.value * 8
+    n = nc.value * rows.value * EV
     if n > cap:
         raise RuntimeError("trace buffer too small")
-    return dq, dk, dv, buf[:n].reshape(nc.value, rows.value, 8)
+    return dq, dk, dv, buf[:n].reshape(nc.value, rows.value, EV)

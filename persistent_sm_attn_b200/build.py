@@ -12,7 +12,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libdash_attn.so")
 SOURCES = ["dash_api.cu", "noalloc.cu", "sched.cpp"]
-DEPS = SOURCES + ["sched.h", "ptx.cuh", "bwd_kernel.cuh", "fwd_kernel.cuh", "aux_kernels.cuh"]
+DEPS = SOURCES + ["sched.h", "internal.h", "ptx.cuh", "bwd_kernel.cuh", "fwd_kernel.cuh",
+                  "aux_kernels.cuh"]
 HEADER = os.path.join(os.path.dirname(HERE), "include", "dash_attn.h")
 
 NVCC_FLAGS = [

@@ -153,10 +153,16 @@ enum {
   B_STAGE0 = 22
 };
 
-// kTrace: record %globaltimer per pair of this CTA: 0 S^T issued, 1 softmax
-// done (seen by the MMA issuer), 2 tile MMAs issued, 3 softmax start, 4 dQ
-// partial ready (seen by the reducers), 5 partial drained, 6 ticket granted,
-// 7 reduction published.
+// kTrace: record %globaltimer per pair of this CTA, kTraceEvents slots per pair:
+//   0 S^T issued              1 softmax done (seen by the MMA issuer)
+//   2 tile MMAs issued        3 softmax start (S^T seen)
+//   4 dQ partial ready (seen by the reducers)       5 partial drained from TMEM
+//   6 ticket granted          7 reduction published (or dQ written)
+//   8 P^T packed (softmax, phase 1 end)             9 softmax phase 2 start
+//  10 dS ready (softmax, phase 2 end)              11 P^T seen by the MMA issuer
+//  12 MMA issuer starts waiting for the S^T buffer 13 load-add-store (or atomics) done
+//  14 reducers start waiting for the ticket        15 dP^T issued
+constexpr int kTraceEvents = 16;
 template <int D, bool kAtomic, bool kTrace = false>
 __global__ void __launch_bounds__(512, 1)
     dash_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -201,7 +207,7 @@ __global__ void __launch_bounds__(512, 1)
   auto trace = [&](int row, int ev) {
     if constexpr (kTrace) {
       if (row < p.trace_rows)
-        p.trace[((size_t)blockIdx.x * p.trace_rows + row) * 8 + ev] = globaltimer();
+        p.trace[((size_t)blockIdx.x * p.trace_rows + row) * kTraceEvents + ev] = globaltimer();
     }
   };
   auto wait = [&](uint32_t bar, uint32_t phase) { mbar_wait(bar, phase, lim, p.err, p.abort_flag); };
@@ -354,6 +360,7 @@ __global__ void __launch_bounds__(512, 1)
           const uint32_t kCol = sdesc_lo_none(sb + C::OFF_COL + s * C::kColTile, 2048);
           const uint32_t tSi = tS + s_col(i);
           wait(Q_FULL(s), (i / ST) & 1);
+          trace(i, 12);
           if (i >= 2) wait(DQ_EMPTY(i - 2), s_phase(i - 2));
           tc_fence_after();
           trace(i, 0);
@@ -380,6 +387,7 @@ __global__ void __launch_bounds__(512, 1)
           }
           tc_mma_ss_w(tDP, kOnesDP, kCol, hi_none, ID_SS, 1u);  // - Delta
           tc_commit(BAR(B_DP_FULL));
+          trace(i, 15);
         };
         int it = 0, kn = 0;  // kn: runs started (K/V loads consumed)
         for (int ci = cbeg; ci < cend; ++ci) {
@@ -402,6 +410,7 @@ __global__ void __launch_bounds__(512, 1)
             const uint32_t tSi = tS + s_col(it);
             // dV += P^T dO (A in TMEM), once P is packed
             wait(P_READY(it), s_phase(it));
+            trace(it, 11);
             // a run's first chain: the previous run's dV/dK must have been read out
             if (t == 0 && !cprev && kn >= 2) wait(BAR(B_DKDV_EMPTY), (kn - 2) & 1);
             tc_fence_after();
@@ -456,6 +465,7 @@ __global__ void __launch_bounds__(512, 1)
               const uint32_t mDO = sdesc_lo(sDO + sd * C::kTile, 16384);
               // dV += P^T dO : M = kv, N = D, K = q (A in TMEM, B MN-major), once P is packed
               wait(BAR(B_P_READY), it & 1);
+              trace(it, 11);
               // a run's first chain: the previous run's dV/dK must have been read out
               if (t == 0 && !cprev && kn >= 2) wait(BAR(B_DKDV_EMPTY), (kn - 2) & 1);
               tc_fence_after();
@@ -499,6 +509,7 @@ __global__ void __launch_bounds__(512, 1)
               const uint32_t kDO = sdesc_lo(sDO + sd * C::kTile, 16);
               const uint32_t kCol = sdesc_lo_none(sb + C::OFF_COL + s * C::kColTile, 2048);
               wait(Q_FULL(s), (it / ST) & 1);
+              trace(it, 12);
               if (it > 0) wait(BAR(B_DVDK_DONE), (it - 1) & 1);
               tc_fence_after();
               trace(it, 0);
@@ -523,6 +534,7 @@ __global__ void __launch_bounds__(512, 1)
               // dP'^T = dP^T - Delta, so the softmax forms dS = P dP'
               tc_mma_ss_w(tDP, kOnesDP, kCol, hi_none, ID_SS, 1u);
               tc_commit(BAR(B_DP_FULL));
+              trace(it, 15);
             }
           }
           // the run's last chain: K/V are done with
@@ -609,9 +621,11 @@ __global__ void __launch_bounds__(512, 1)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(P_READY(it));
+        if (threadIdx.x == 0) trace(it, 8);
         wait(BAR(B_DP_FULL), it & 1);
         if (it > 0) wait(BAR(B_DS_FREE), (it - 1) & 1);
         tc_fence_after();
+        if (threadIdx.x == 0) trace(it, 9);
         // dS from the bf16 P just packed: the registers are not there to keep P in
         // fp32 across the wait, and the extra rounding stays far inside the error bound
 #pragma unroll 1
@@ -642,6 +656,7 @@ __global__ void __launch_bounds__(512, 1)
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(BAR(B_DS_READY));
+        if (threadIdx.x == 0) trace(it, 10);
       }
     }
   } else {
@@ -727,6 +742,7 @@ __global__ void __launch_bounds__(512, 1)
             }
           };
           if (idx > 0) {
+            if (threadIdx.x == 256) trace(it, 14);
             ticket_wait(p.tickets + unit, (uint32_t)idx, ~0u);
             if (threadIdx.x == 256) trace(it, 6);
             add_from(accp);
@@ -756,6 +772,7 @@ __global__ void __launch_bounds__(512, 1)
             for (int c4 = 0; c4 < NV; ++c4)
               st_cg_f4(accp + c4 * 128 + r,
                        make_float4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]));
+            if (threadIdx.x == 256) trace(it, 13);
             if constexpr (C::kPublisher) {
               // hand the publication of these stores to the publisher warp (slot k mod 2,
               // free again once it has published pair k - 2)
@@ -775,6 +792,7 @@ __global__ void __launch_bounds__(512, 1)
           for (int c4 = 0; c4 < NV; ++c4)
             atomicAdd(accp + c4 * 128 + r,
                       make_float4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]));
+          if (threadIdx.x == 256) trace(it, 13);
         }
         if (threadIdx.x == 256 && (kAtomic || last || !C::kPublisher)) trace(it, 7);
       }

@@ -896,7 +896,7 @@ int dash_trace_bwd(const void* q, const void* k, const void* v, const void* o, c
       for (int ci = t.cta_off[c]; ci < t.cta_off[c + 1]; ++ci) n += t.chains[ci].pair_cnt;
       rows = n > rows ? n : rows;
     }
-    const size_t n_entries = (size_t)ctas * rows * 8;
+    const size_t n_entries = (size_t)ctas * rows * dash::kTraceEvents;
     unsigned long long* dtrace = nullptr;
     if (cudaMalloc(&dtrace, n_entries * sizeof(unsigned long long)) != cudaSuccess)
       return DASH_ERR_OOM;
