@@ -24,23 +24,30 @@
 // and dQp, so the exponentials of tile i+1 run while the tensor pipe finishes
 // tile i, and dV of tile i+1 runs while its dS is formed.  Taking P^T and dS^T
 // from TMEM keeps two of the five products off the shared-memory read path.
-// D = 64: TMEM has room for two S^T buffers, so S^T runs two tiles ahead; dK
-// reads dS^T from shared memory, which frees a tile's S^T buffer as soon as dV
-// and the softmax are done with its P^T, and the tile's dQp goes there.
+// D = 64: TMEM has room for two S^T buffers, so the two softmax warpgroups take
+// alternate tiles: one computes the exponentials of tile i+1 (bound by the MUFU
+// unit) while the other forms dS of tile i (bound by instruction issue).  A
+// tile's P^T goes into the upper half of its S^T buffer and its dQp into the
+// lower half; dK reads dS^T from shared memory (one buffer per warpgroup).
 //
 // Warp roles (512 threads, four warpgroups):
-//   WG0, WG1  softmax / dS; WG0 owns Q columns 0-63, WG1 columns 64-127 (96 registers)
-//   WG2       dQ reduction and the dK/dV epilogue (224 registers)
-//   WG3       warp 12 TMA producer, warp 13 MMA issuer and TMEM owner (96 registers)
+//   WG0, WG1  softmax / dS (96 registers at D = 128, 112 at D = 64); D = 128: WG0 owns Q columns 0-63 of every
+//             tile, WG1 columns 64-127; D = 64: WG0 takes the even tiles, WG1 the odd
+//             ones, all 128 columns
+//   WG2       dQ reduction and the dK/dV epilogue (224 registers at D = 128, 200 at D = 64)
+//   WG3       warp 12 TMA producer of K, V and Q, warp 13 MMA issuer and TMEM owner,
+//             warp 14 publisher of the ordered reduction (D = 64), warp 15 TMA producer
+//             of dO (96 registers at D = 128, 88 at D = 64)
 // TMEM lane quarter of a warp is (warp % 4), so each warpgroup covers the 128 lanes.
 //
 // TMEM columns (512).  D = 128: S^T [0,128) then packed P^T/dS^T, dP^T
 // [128,256) then dQp, dV [256,384), dK [384,512).  D = 64: S^T of even tiles
-// [0,128), of odd tiles [128,256), each then packed P^T and then that tile's dQp
-// in its first 64 columns; dP^T [256,384), dV [384,448), dK [448,512).  Packed
-// layout after the softmax: the 32 fp32 columns of chunk c (Q columns
-// 32c..32c+31) hold P^T of those columns in 32c..32c+15 and (D = 128) dS^T in
-// 32c+16..32c+31, two bf16 per column.
+// [0,128), of odd tiles [128,256), each then holding the packed P^T in its upper
+// 64 columns and that tile's dQp in its lower 64; dP^T [256,384), dV [384,448),
+// dK [448,512).  Packed layout after the softmax, two bf16 per column: D = 128,
+// the 32 fp32 columns of chunk c (Q columns 32c..32c+31) hold P^T of those
+// columns in 32c..32c+15 and dS^T in 32c+16..32c+31; D = 64, P^T of chunk c is
+// in the 16 columns at p_col64(c).
 //
 // Shared-memory tiles are [128 rows][D] bf16 stored as D/64 column blocks of
 // 128 rows x 128 bytes with the 128-byte swizzle (the layout a TMA load with
@@ -90,18 +97,22 @@ template <int D>
 struct BwdCfg {
   static constexpr int kThreads = 512;
   static constexpr int kLaunchRegs = 65536 / kThreads;   // 128: the setmaxnreg split below
-  static constexpr int kRegsSoftmax = 96;                // WG0, WG1
-  static constexpr int kRegsReduce = 224;                // WG2
-  static constexpr int kRegsCtrl = 96;                   // WG3
+  // D = 64: the softmax also stages dQp (64 fp32 per thread) out of TMEM
+  static constexpr int kRegsSoftmax = (D == 64) ? 104 : 96;  // WG0, WG1
+  static constexpr int kRegsReduce = (D == 64) ? 208 : 224;  // WG2
+  static constexpr int kRegsCtrl = 96;                       // WG3
   static_assert(2 * kRegsSoftmax + kRegsReduce + kRegsCtrl == 4 * kLaunchRegs,
                 "register split must equal the launch allocation");
   static constexpr int kKVRows = 128;                    // TMA box rows of K and V
   static constexpr int kQRows = 128;                     // TMA box rows of Q and dO
   static constexpr int kTile = 128 * D * 2;              // one [128][D] bf16 tile
-  // Q is double-buffered (the next S^T follows dK right away); at D = 128 dO has one
+  // D = 128: Q is double-buffered (the next S^T follows dK right away) and dO has one
   // buffer, refilled between dV of a tile and dP^T of the next, to fit the smem budget.
-  static constexpr int kStagesQ = (D == 64) ? 3 : 2;
-  static constexpr int kStagesDO = (D == 64) ? 3 : 1;
+  // D = 64: S^T runs two tiles ahead, so Q(i+2) reuses the stage of Q(i-2) (four stages)
+  // and its load has a whole tile to land; dO is read by dP^T(i+1) one tile ahead and
+  // released by dV, so two stages suffice.
+  static constexpr int kStagesQ = (D == 64) ? 4 : 2;
+  static constexpr int kStagesDO = (D == 64) ? 2 : 1;
   // LSE and Delta enter the S^T and dP^T products as one extra K-step each: a per-Q-row
   // column tile ([128 rows][8] bf16, loaded with Q) against a constant tile of ones.
   // Each tile is 2 KiB of core matrices (8 rows x 16 bytes, no swizzle) followed by
@@ -114,18 +125,22 @@ struct BwdCfg {
   static constexpr int OFF_V = OFF_K + kTile;
   static constexpr int OFF_Q = OFF_V + kTile;
   static constexpr int OFF_DO = OFF_Q + kStagesQ * kTile;
-  static constexpr int OFF_DST = OFF_DO + kStagesDO * kTile;  // dS^T [128 kv][128 q]
-  static constexpr int OFF_BAR = OFF_DST + 32768;
-  static constexpr int kBars = 22 + 2 * kStagesQ + 2 * kStagesDO;
+  // dS^T [128 kv][128 q]: one buffer per softmax warpgroup at D = 64, where the two
+  // warpgroups take alternate tiles; one at D = 128
+  static constexpr int kDsBufs = (D == 64) ? 2 : 1;
+  static constexpr int OFF_DST = OFF_DO + kStagesDO * kTile;
+  static constexpr int OFF_BAR = OFF_DST + kDsBufs * 32768;
+  static constexpr int kBars = 25 + 2 * kStagesQ + 2 * kStagesDO;
   static constexpr int OFF_TMEM_SLOT = OFF_BAR + kBars * 8;
   // The swizzled tiles need a 1 KiB aligned base; the kernel checks it.
   static constexpr int kSmemBytes = OFF_TMEM_SLOT + 16;
   static_assert(kSmemBytes <= 232448, "shared memory per block exceeded");
   // TMEM columns.  D = 128: S^T [0,128), dP^T [128,256), dV, dK; dQp reuses dP^T's
   // columns and dK takes dS^T from S^T's columns.  D = 64: S^T has two buffers [0,128)
-  // and [128,256) (the MMA issuer runs two tiles ahead on S^T), dP^T [256,384), dV, dK;
-  // dK takes dS^T from shared memory, so a tile's S^T buffer is free once dV and the
-  // softmax are done with its P^T, and the tile's dQp goes into its first 64 columns.
+  // and [128,256), one per softmax warpgroup (they take alternate tiles), dP^T
+  // [256,384), dV, dK.  The softmax packs a tile's P^T into the upper 64 columns of its
+  // S^T buffer, and the tile's dQp goes into the lower 64; dK takes dS^T from shared
+  // memory.
   static constexpr bool kSDouble = (D == 64);
   static constexpr uint32_t TM_S = 0, TM_DP = kSDouble ? 256 : 128;
   static constexpr uint32_t TM_DV = TM_DP + 128, TM_DK = TM_DV + D;
@@ -148,10 +163,16 @@ constexpr long long dq_units(long long bh_times_n) {
 enum {
   B_KV_FULL = 0, B_KV_EMPTY, B_S_FULL, B_DP_FULL, B_DS_READY, B_DS_FREE, B_DQ_FULL0, B_DQ_FULL1,
   B_DQ_EMPTY0, B_DQ_EMPTY1, B_DVDK_DONE, B_DKDV_FULL, B_DKDV_EMPTY, B_FINAL, B_P_READY,
-  B_S_FULL1, B_P_READY1, B_DV_DONE,  // the second S^T buffer and dV done (D = 64)
+  B_S_FULL1, B_P_READY1, B_UNUSED17,  // the second S^T buffer's barriers (D = 64)
   B_PUB_READY0, B_PUB_READY1, B_PUB_FREE0, B_PUB_FREE1,  // reducers -> publisher hand-off
-  B_STAGE0 = 22
+  B_DS_READY1, B_DP_FULL1, B_DS_FREE1,  // odd tiles' barriers (D = 64)
+  B_STAGE0 = 25
 };
+
+// D = 64: the TMEM column (within a tile's S^T buffer) where the softmax packs the
+// bf16 P^T of Q columns 32c..32c+31.  Chunks are packed in the order 2, 3, 0, 1 into
+// columns 64, 80, 96, 112, so each store lands on S^T columns already read.
+__host__ __device__ constexpr uint32_t p_col64(int c) { return 64u + 16u * (uint32_t)((c + 2) & 3); }
 
 // kTrace: record %globaltimer per pair of this CTA, kTraceEvents slots per pair:
 //   0 S^T issued              1 softmax done (seen by the MMA issuer)
@@ -197,6 +218,11 @@ __global__ void __launch_bounds__(512, 1)
   auto S_FULL = [&](int i) { return BAR(C::kSDouble && (i & 1) ? B_S_FULL1 : B_S_FULL); };
   auto P_READY = [&](int i) { return BAR(C::kSDouble && (i & 1) ? B_P_READY1 : B_P_READY); };
   auto s_phase = [&](int i) { return C::kSDouble ? (i >> 1) & 1 : i & 1; };
+  // D = 64 keeps one barrier per tile parity for dS ready, dP^T full and dS^T free, since
+  // the two softmax warpgroups take alternate tiles; D = 128 has one of each
+  auto DS_READY = [&](int i) { return BAR(C::kSDouble && (i & 1) ? B_DS_READY1 : B_DS_READY); };
+  auto DP_FULL = [&](int i) { return BAR(C::kSDouble && (i & 1) ? B_DP_FULL1 : B_DP_FULL); };
+  auto DS_FREE = [&](int i) { return BAR(C::kSDouble && (i & 1) ? B_DS_FREE1 : B_DS_FREE); };
   auto dq_col = [&](int i) { return C::kDqInDp ? C::TM_DP : 128u * (uint32_t)(i & 1); };
   auto DQ_FULL = [&](int i) { return BAR(C::kDqInDp ? B_DQ_FULL0 : B_DQ_FULL0 + (i & 1)); };
   auto DQ_EMPTY = [&](int i) { return BAR(C::kDqInDp ? B_DQ_EMPTY0 : B_DQ_EMPTY0 + (i & 1)); };
@@ -220,10 +246,16 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(BAR(B_KV_EMPTY), 1);
     mbar_init(BAR(B_S_FULL), 1);
     mbar_init(BAR(B_S_FULL1), 1);
-    mbar_init(BAR(B_DV_DONE), 1);
+    // D = 64: one softmax warpgroup (128 threads) per tile, D = 128: both
+    constexpr uint32_t kSoftmaxArrive = C::kSDouble ? 128u : 256u;
     mbar_init(BAR(B_DP_FULL), 1);
-    mbar_init(BAR(B_DS_READY), 256);
-    mbar_init(BAR(B_DS_FREE), 1);
+    mbar_init(BAR(B_DP_FULL1), 1);
+    mbar_init(BAR(B_DS_READY), kSoftmaxArrive);
+    mbar_init(BAR(B_DS_READY1), kSoftmaxArrive);
+    // D = 64: the reducers (128 threads) free a dS buffer once they have read the dQp
+    // staged there; D = 128: the commit of dQp and dK frees it
+    mbar_init(BAR(B_DS_FREE), C::kSDouble ? 128u : 1u);
+    mbar_init(BAR(B_DS_FREE1), C::kSDouble ? 128u : 1u);
     for (int b = 0; b < 2; ++b) {
       mbar_init(BAR(B_DQ_FULL0 + b), 1);
       mbar_init(BAR(B_DQ_EMPTY0 + b), 128);
@@ -232,8 +264,8 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(BAR(B_DKDV_FULL), 1);
     mbar_init(BAR(B_DKDV_EMPTY), 128);
     mbar_init(BAR(B_FINAL), 1);
-    mbar_init(BAR(B_P_READY), 256);
-    mbar_init(BAR(B_P_READY1), 256);
+    mbar_init(BAR(B_P_READY), kSoftmaxArrive);
+    mbar_init(BAR(B_P_READY1), kSoftmaxArrive);
     for (int b = 0; b < 2; ++b) {
       mbar_init(BAR(B_PUB_READY0 + b), 128);
       mbar_init(BAR(B_PUB_FREE0 + b), 1);
@@ -288,7 +320,10 @@ __global__ void __launch_bounds__(512, 1)
   if (warp >= 12) {
     setmaxnreg_dec<C::kRegsCtrl>();
     if (warp == 12 && lane == 0) {
-      // ---------------------------------------------------------- TMA producer
+      // ---------------------------------------------------------- TMA producer: K, V, Q
+      // K/V once per run; per pair Q with its column tile (LSE and Delta terms, read by
+      // S^T and dP^T, which finish before dK frees the stage).  dO has a producer of its
+      // own (warp 15), so a Q load never queues behind the wait for a dO stage.
       int it = 0, kn = 0;  // kn: K/V loads so far
       for (int ci = cbeg; ci < cend; ++ci) {
         const int4 ch = p.chains[ci];
@@ -305,21 +340,14 @@ __global__ void __launch_bounds__(512, 1)
         }
         for (int t = 0; t < n_pairs(ch.w); ++t, ++it) {
           const int q = (int)(p.pairs[ch.z + t] & 0xffffu);
-          const int s = it % ST, sd = it % SD;
+          const int s = it % ST;
           const int row_q = ch.x * S + q * 128;
-          // Q with its column tile (LSE and Delta terms, read by S^T and dP^T, which
-          // finish before dK frees the stage); dO is released earlier, after dV
           if (it >= ST) wait(Q_EMPTY(s), ((it / ST) - 1) & 1);
           mbar_expect_tx(Q_FULL(s), C::kTile + 2048);
 #pragma unroll
           for (int cb = 0; cb < D / 64; ++cb)
             tma_load_2d(sQ + s * C::kTile + cb * 16384, &tmQ, cb * 64, row_q, Q_FULL(s));
           tma_load_2d(sb + C::OFF_COL + s * C::kColTile, &tmC, 0, row_q, Q_FULL(s));
-          if (it >= SD) wait(DO_EMPTY(sd), ((it / SD) - 1) & 1);
-          mbar_expect_tx(DO_FULL(sd), C::kTile);
-#pragma unroll
-          for (int cb = 0; cb < D / 64; ++cb)
-            tma_load_2d(sDO + sd * C::kTile + cb * 16384, &tmDO, cb * 64, row_q, DO_FULL(sd));
         }
       }
       // drain: every issued load has landed before the CTA can exit
@@ -327,11 +355,27 @@ __global__ void __launch_bounds__(512, 1)
         const int last_use = ((it - 1 - s) / ST) * ST + s;
         drain(Q_FULL(s), (last_use / ST) & 1);
       }
+      if (kn > 0) drain(BAR(B_KV_FULL), (kn - 1) & 1);
+    } else if (warp == 15 && lane == 0) {
+      // ---------------------------------------------------------- TMA producer: dO
+      int it = 0;
+      for (int ci = cbeg; ci < cend; ++ci) {
+        const int4 ch = p.chains[ci];
+        for (int t = 0; t < n_pairs(ch.w); ++t, ++it) {
+          const int q = (int)(p.pairs[ch.z + t] & 0xffffu);
+          const int sd = it % SD;
+          const int row_q = ch.x * S + q * 128;
+          if (it >= SD) wait(DO_EMPTY(sd), ((it / SD) - 1) & 1);
+          mbar_expect_tx(DO_FULL(sd), C::kTile);
+#pragma unroll
+          for (int cb = 0; cb < D / 64; ++cb)
+            tma_load_2d(sDO + sd * C::kTile + cb * 16384, &tmDO, cb * 64, row_q, DO_FULL(sd));
+        }
+      }
       for (int s = 0; s < SD && s < it; ++s) {
         const int last_use = ((it - 1 - s) / SD) * SD + s;
         drain(DO_FULL(s), (last_use / SD) & 1);
       }
-      if (kn > 0) drain(BAR(B_KV_FULL), (kn - 1) & 1);
     } else if (warp == 13 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
       // One thread issues every MMA; its instruction stream between MMAs is the
@@ -351,9 +395,17 @@ __global__ void __launch_bounds__(512, 1)
       const uint32_t kOnesS = sdesc_lo_none(sb + C::OFF_ONES, 2048);
       const uint32_t kOnesDP = sdesc_lo_none(sb + C::OFF_ONES + C::kColTile, 2048);
       if constexpr (C::kSDouble) {
-        const uint32_t kDS = sdesc_lo(sDSt, 16);  // dS^T read K-major (M = kv, K = q) by dK
-        // S'^T = K Q^T - LSE/scale of tile i into its buffer, once the reducers have
-        // drained the dQp that tile i - 2 left there
+        // D = 64.  The two softmax warpgroups take alternate tiles, so tile i's S^T lives
+        // in buffer i mod 2 and the issuer keeps two tiles in flight: while one
+        // warpgroup forms dS of tile i, the other computes the exponentials of tile i+1.
+        // Per step i, once dS(i) is ready: dP'^T(i+1) (the buffer is free once the
+        // softmax has read dP'^T(i)), dQp(i) and dK(i), dV(i+1) once P^T(i+1) is packed,
+        // then S'^T(i+2) once the softmax has staged dQp(i) out of S^T buffer i mod 2.
+        // Each wait comes after the products that do not depend on it.
+        int it = 0, kn = 0;  // kn: runs started (K/V loads consumed)
+        auto dsbuf = [&](int i) { return sDSt + 32768u * (uint32_t)(i & 1); };
+        // S'^T = K Q^T - LSE/scale of tile i into its buffer, once the softmax has
+        // staged out the dQp that tile i - 2 left there
         auto issue_s = [&](int i) {
           const int s = i % ST;
           const uint32_t kQ = sdesc_lo(sQ + s * C::kTile, 16);
@@ -386,10 +438,25 @@ __global__ void __launch_bounds__(512, 1)
             tc_mma_ss_w(tDP, kV + off, kDO + off, hi, ID_SS, kk > 0 ? 1u : 0u);
           }
           tc_mma_ss_w(tDP, kOnesDP, kCol, hi_none, ID_SS, 1u);  // - Delta
-          tc_commit(BAR(B_DP_FULL));
+          tc_commit(DP_FULL(i));
           trace(i, 15);
         };
-        int it = 0, kn = 0;  // kn: runs started (K/V loads consumed)
+        // dV += P^T dO of tile i (A = P^T from the upper half of its S^T buffer), once
+        // P^T is packed; a run's first chain waits for the previous run's read-out
+        auto issue_dv = [&](int i, bool first_of_run, uint32_t acc0) {
+          const int sd = i % SD;
+          const uint32_t mDO = sdesc_lo(sDO + sd * C::kTile, 16384);
+          const uint32_t tSi = tS + s_col(i);
+          wait(P_READY(i), s_phase(i));
+          trace(i, 11);
+          if (first_of_run && kn >= 2) wait(BAR(B_DKDV_EMPTY), (kn - 2) & 1);
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            tc_mma_ts_w(tDV, tSi + p_col64(kk >> 1) + 8 * (kk & 1), mDO + kk * 128, hi, ID_KV,
+                        kk > 0 ? 1u : acc0);
+          tc_commit(DO_EMPTY(sd));  // dP'^T and dV have read dO
+        };
         for (int ci = cbeg; ci < cend; ++ci) {
           const int cnt = n_pairs(p.chains[ci].w);
           const bool cprev = cont_prev(ci);
@@ -399,51 +466,40 @@ __global__ void __launch_bounds__(512, 1)
             issue_s(it);
             if (cnt > 1) issue_s(it + 1);
             issue_dp(it);
+            issue_dv(it, !cprev, cprev ? 1u : 0u);
           }
-          // Each step finishes tile `it`: dP'^T of the next tile first (the softmax's
-          // next wait), dQp into this tile's S^T buffer, dK; then S'^T two tiles ahead
-          // into that buffer once dQp has been drained.
           for (int t = 0; t < cnt; ++t, ++it) {
-            const int s = it % ST, sd = it % SD;
+            const int s = it % ST;
             const uint32_t mQ = sdesc_lo(sQ + s * C::kTile, 16384);
-            const uint32_t mDO = sdesc_lo(sDO + sd * C::kTile, 16384);
-            const uint32_t tSi = tS + s_col(it);
-            // dV += P^T dO (A in TMEM), once P is packed
-            wait(P_READY(it), s_phase(it));
-            trace(it, 11);
-            // a run's first chain: the previous run's dV/dK must have been read out
-            if (t == 0 && !cprev && kn >= 2) wait(BAR(B_DKDV_EMPTY), (kn - 2) & 1);
-            tc_fence_after();
-            const uint32_t acc0 = (t > 0 || cprev) ? 1u : 0u;
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              tc_mma_ts_w(tDV, tSi + 32 * (kk >> 1) + 8 * (kk & 1), mDO + kk * 128, hi, ID_KV,
-                          kk > 0 ? 1u : acc0);
-            tc_commit(DO_EMPTY(sd));
-            tc_commit(BAR(B_DV_DONE));
-            wait(BAR(B_DS_READY), it & 1);
+            const uint32_t mDSi = sdesc_lo(dsbuf(it), 16384);  // dS MN-major (dQp)
+            const uint32_t kDSi = sdesc_lo(dsbuf(it), 16);     // dS^T K-major (dK)
+            wait(DS_READY(it), s_phase(it));
             trace(it, 1);
             tc_fence_after();
+            // the other warpgroup's next dS waits for dP'^T(it + 1) first
             if (t + 1 < cnt) issue_dp(it + 1);
-            // dQp = dS K (both MN-major from shared memory) into the first 64 columns of
-            // this tile's S^T buffer, once dV has read P^T out of them
-            wait(BAR(B_DV_DONE), it & 1);
-            tc_fence_after();
+            // dQp = dS K (both MN-major from shared memory) into the lower 64 columns of
+            // this tile's S^T buffer, which the softmax has finished reading
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              tc_mma_ss_w(tmem + dq_col(it), mDS + kk * 128, mK + kk * 128, hi, ID_Q,
+              tc_mma_ss_w(tmem + dq_col(it), mDSi + kk * 128, mK + kk * 128, hi, ID_Q,
                           kk > 0 ? 1u : 0u);
-            tc_commit(DQ_FULL(it));
             // dK += dS^T Q : A = dS^T K-major, B = Q MN-major, both from shared memory
+            const uint32_t acc0 = (t > 0 || cprev) ? 1u : 0u;
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
               const uint32_t off = (uint32_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
-              tc_mma_ss_w(tDK, kDS + off, mQ + kk * 128, hi, ID_KV, kk > 0 ? 1u : acc0);
+              tc_mma_ss_w(tDK, kDSi + off, mQ + kk * 128, hi, ID_KV, kk > 0 ? 1u : acc0);
             }
+            // dQp is ready, and dQp and dK have read dS: the softmax stages dQp into the
+            // dS buffer and then frees the S^T buffer (DQ_EMPTY)
+            tc_commit(DQ_FULL(it));
             tc_commit(Q_EMPTY(s));
-            tc_commit(BAR(B_DS_FREE));  // dQp and dK have read dS^T
             if (t == cnt - 1 && !cont_next(ci)) tc_commit(BAR(B_DKDV_FULL));
             trace(it, 2);
+            if (t + 1 < cnt) issue_dv(it + 1, false, 1u);
+            // S'^T(it + 2) last: by now the softmax has had dQp(it) and dK(it) to stage
+            // dQp(it) out of the buffer
             if (t + 2 < cnt) issue_s(it + 2);
           }
           // the run's last chain: K/V are done with
@@ -581,6 +637,116 @@ __global__ void __launch_bounds__(512, 1)
         (uint32_t)half * 16384 + (uint32_t)(r >> 3) * 1024 + (uint32_t)(r & 7) * 128;
     const uint32_t tS0 = tmem + lane_off + C::TM_S, tDP = tmem + lane_off + C::TM_DP;
     const float sl2 = p.scale_log2;
+    // P^T of 32 Q columns from S'^T: 2^(scale log2e S'), zero above the causal diagonal
+    // (Q column qc < lim_c), packed as bf16 pairs
+    auto exp_chunk = [&](const uint32_t (&sv)[32], uint32_t (&pk)[16], int c, int lim_c) {
+      auto body = [&](auto masked) {
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const int qc = 32 * c + j;
+          // S'^T already has LSE / scale taken off by the tensor core
+          float p0 = ex2_approx(__uint_as_float(sv[j]) * sl2);
+          float p1 = ex2_approx(__uint_as_float(sv[j + 1]) * sl2);
+          if constexpr (decltype(masked)::value) {
+            if (qc < lim_c) p0 = 0.f;
+            if (qc + 1 < lim_c) p1 = 0.f;
+          }
+          pk[j >> 1] = pack_bf16x2(p0, p1);
+        }
+      };
+      // the causal mask only touches chunks that reach the diagonal
+      if (lim_c > 32 * c) body(std::true_type{});
+      else body(std::false_type{});
+    };
+    // dS = P dP' of 32 Q columns from packed P and fp32 dP'^T (Delta already taken off
+    // by the tensor core), packed as bf16 pairs
+    auto ds_chunk = [&](const uint32_t (&pk)[16], const uint32_t (&dv)[32], uint32_t (&dk)[16]) {
+#pragma unroll
+      for (int j = 0; j < 32; j += 2) {
+        const float p0 = __uint_as_float(pk[j >> 1] << 16);
+        const float p1 = __uint_as_float(pk[j >> 1] & 0xffff0000u);
+        dk[j >> 1] = pack_bf16x2(p0 * __uint_as_float(dv[j]), p1 * __uint_as_float(dv[j + 1]));
+      }
+    };
+    if constexpr (C::kSDouble) {
+      // D = 64: warpgroup `half` takes the tiles of parity `half`, all 128 Q columns of
+      // them, so one warpgroup's exponentials (MUFU-bound) run beside the other's dS
+      // (issue-bound).  S'^T of its tiles is in buffer `half`; P^T goes into that
+      // buffer's upper 64 columns (p_col64), dS^T into shared-memory buffer `half`.
+      const uint32_t tS = tS0 + 128u * (uint32_t)half;
+      const uint32_t sDS = sDSt + 32768u * (uint32_t)half;
+      const uint32_t rowbase = (uint32_t)(r >> 3) * 1024 + (uint32_t)(r & 7) * 128;
+      const bool tracer = threadIdx.x == 128 * half;
+      int it = 0;
+      for (int ci = cbeg; ci < cend; ++ci) {
+        const int4 ch = p.chains[ci];
+        for (int t = 0; t < n_pairs(ch.w); ++t, ++it) {
+          if ((it & 1) != half) continue;
+          const int q = (int)(p.pairs[ch.z + t] & 0xffffu);
+          wait(S_FULL(it), s_phase(it));
+          if (tracer) trace(it, 3);
+          tc_fence_after();
+          const int lim_c = (p.causal && q == ch.y) ? r : -1;
+          // chunks 2, 3, 0, 1 into columns 64, 80, 96, 112: each store lands on columns
+          // this thread has already read
+#pragma unroll 1
+          for (int cc = 0; cc < 4; ++cc) {
+            const int c = (cc + 2) & 3;
+            uint32_t sv[32], pk[16];
+            tmem_ld32(tS + 32 * c, sv);
+            exp_chunk(sv, pk, c, lim_c);
+            tmem_st16(tS + 64 + 16 * cc, pk);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(P_READY(it));
+          if (tracer) trace(it, 8);
+          wait(DP_FULL(it), s_phase(it));
+          // the reducers have read tile it - 2's dQp out of this buffer
+          if (it >= 2) wait(DS_FREE(it - 2), s_phase(it - 2));
+          tc_fence_after();
+          if (tracer) trace(it, 9);
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t pk[16], dv[32], dk[16];
+            tmem_ld16(tS + p_col64(c), pk);
+            tmem_ld32(tDP + 32 * c, dv);
+            ds_chunk(pk, dv, dk);
+            // 128-byte swizzle, 64-column block c / 2
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+              const uint32_t unit = (uint32_t)((((c & 1) * 4 + m) ^ (r & 7)) * 16);
+              st_shared_v4(sDS + (uint32_t)(c >> 1) * 16384 + rowbase + unit, dk[4 * m],
+                           dk[4 * m + 1], dk[4 * m + 2], dk[4 * m + 3]);
+            }
+          }
+          fence_proxy_async_smem();
+          tc_fence_before();
+          mbar_arrive(DS_READY(it));
+          if (tracer) trace(it, 10);
+          // Stage this tile's dQp: once dQp and dK have read dS (their commit), move dQp
+          // out of the lower half of the S^T buffer into this warpgroup's dS buffer as
+          // fp32 [D/4][128 rows][4], the reducers' layout.  The S^T buffer is then free
+          // for tile it + 2 whatever the reducers are doing; they have until this
+          // warpgroup's next dS to read the staged copy.
+          wait(DQ_FULL(it), s_phase(it));
+          tc_fence_after();
+          {
+            uint32_t v[32];
+#pragma unroll
+            for (int c2 = 0; c2 < 2; ++c2) {
+              tmem_ld32(tS + 32 * c2, v);
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                st_shared_v4(sDS + (uint32_t)(((c2 * 8 + j) * 128 + r) * 16), v[4 * j],
+                             v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(DQ_EMPTY(it));
+        }
+      }
+    } else {
     int it = 0;
     for (int ci = cbeg; ci < cend; ++ci) {
       const int4 ch = p.chains[ci];
@@ -598,23 +764,7 @@ __global__ void __launch_bounds__(512, 1)
           uint32_t sv[32];
           tmem_ld32(tS + 32 * c, sv);
           uint32_t pk[16];
-          // the causal mask only touches chunks that reach the diagonal
-          auto body = [&](auto masked) {
-#pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-              const int qc = 32 * c + j;
-              // S'^T already has LSE / scale taken off by the tensor core
-              float p0 = ex2_approx(__uint_as_float(sv[j]) * sl2);
-              float p1 = ex2_approx(__uint_as_float(sv[j + 1]) * sl2);
-              if constexpr (decltype(masked)::value) {
-                if (qc < lim_c) p0 = 0.f;
-                if (qc + 1 < lim_c) p1 = 0.f;
-              }
-              pk[j >> 1] = pack_bf16x2(p0, p1);
-            }
-          };
-          if (lim_c > 32 * c) body(std::true_type{});
-          else body(std::false_type{});
+          exp_chunk(sv, pk, c, lim_c);
           // P^T into the first 16 columns of chunk c (this lane's own row)
           tmem_st16(tS + 32 * c, pk);
         }
@@ -628,36 +778,55 @@ __global__ void __launch_bounds__(512, 1)
         if (threadIdx.x == 0) trace(it, 9);
         // dS from the bf16 P just packed: the registers are not there to keep P in
         // fp32 across the wait, and the extra rounding stays far inside the error bound
-#pragma unroll 1
-        for (int cc = 0; cc < 2; ++cc) {
-          const int c = half * 2 + cc;
-          uint32_t pk[16], dv[32];
-          tmem_ld16(tS + 32 * c, pk);
-          tmem_ld32(tDP + 32 * c, dv);
-          uint32_t dk[16];
+        // in sub-chunks of 16 Q columns (h = 0..3 of this warpgroup's 64), the next
+        // sub-chunk's P and dP' loads in flight while this one is formed; dS^T goes into
+        // the last 16 columns of its 32-column chunk, where dK reads it from TMEM, and to
+        // shared memory (128-byte swizzle, 64-column block `half`)
+        {
+          uint32_t pa[8], da[16], pb[8], db[16];
+          auto load = [&](int h, uint32_t (&pp)[8], uint32_t (&dd)[16]) {
+            const int c = half * 2 + (h >> 1);
+            tmem_ld8_async(tS + 32 * c + 8 * (h & 1), pp);
+            tmem_ld16_async(tDP + 32 * c + 16 * (h & 1), dd);
+          };
+          auto form = [&](int h, const uint32_t (&pp)[8], const uint32_t (&dd)[16]) {
+            const int c = half * 2 + (h >> 1);
+            uint32_t dk[8];
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            // dP'^T already has Delta taken off by the tensor core
-            const float p0 = __uint_as_float(pk[j >> 1] << 16);
-            const float p1 = __uint_as_float(pk[j >> 1] & 0xffff0000u);
-            dk[j >> 1] = pack_bf16x2(p0 * __uint_as_float(dv[j]), p1 * __uint_as_float(dv[j + 1]));
-          }
-          // dS^T into the last 16 columns of chunk c (D = 128, where dK reads it from
-          // TMEM), and to shared memory (128-byte swizzle, 64-column block `half`)
-          if constexpr (!C::kSDouble) tmem_st16(tS + 32 * c + 16, dk);
+            for (int j = 0; j < 16; j += 2) {
+              const float p0 = __uint_as_float(pp[j >> 1] << 16);
+              const float p1 = __uint_as_float(pp[j >> 1] & 0xffff0000u);
+              dk[j >> 1] =
+                  pack_bf16x2(p0 * __uint_as_float(dd[j]), p1 * __uint_as_float(dd[j + 1]));
+            }
+            tmem_st8(tS + 32 * c + 16 + 8 * (h & 1), dk);
 #pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            const uint32_t chunk = (uint32_t)(((cc * 4 + m) ^ (r & 7)) * 16);
-            st_shared_v4(sDSt + rowoff + chunk, dk[4 * m], dk[4 * m + 1], dk[4 * m + 2],
-                         dk[4 * m + 3]);
-          }
+            for (int m = 0; m < 2; ++m) {
+              const uint32_t unit = (uint32_t)(((2 * h + m) ^ (r & 7)) * 16);
+              st_shared_v4(sDSt + rowoff + unit, dk[4 * m], dk[4 * m + 1], dk[4 * m + 2],
+                           dk[4 * m + 3]);
+            }
+          };
+          load(0, pa, da);
+          tmem_wait_ld();
+          load(1, pb, db);
+          form(0, pa, da);
+          tmem_wait_ld();
+          load(2, pa, da);
+          form(1, pb, db);
+          tmem_wait_ld();
+          load(3, pb, db);
+          form(2, pa, da);
+          tmem_wait_ld();
+          form(3, pb, db);
         }
-        if constexpr (!C::kSDouble) tmem_wait_st();
+        tmem_wait_st();
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(BAR(B_DS_READY));
         if (threadIdx.x == 0) trace(it, 10);
       }
+    }
     }
   } else {
     // ------------------------------------------------------------ dQ reduction + dK/dV epilogue
@@ -669,6 +838,13 @@ __global__ void __launch_bounds__(512, 1)
     constexpr int G = 24;               // loads in flight per group
     int it = 0, fn = 0;  // fn: dK/dV runs written out
     int npub = 0;        // pairs handed to the publisher
+    // D = 64, deterministic: once this pair is handed off, the accumulator loads of the
+    // next pair go out if its ticket is already granted (checked once, never waited
+    // for here), so their round trip overlaps the wait for the next partial and its
+    // drain.  The values loaded and the order of the additions are the same either way.
+    constexpr bool kLook = !kAtomic && D == 64;
+    float4 pre[NV];
+    bool pre_ok = false;  // pre holds this pair's accumulator, loaded ahead
     for (int ci = cbeg; ci < cend; ++ci) {
       const int4 ch = p.chains[ci];
       for (int t = 0; t < n_pairs(ch.w); ++t, ++it) {
@@ -676,19 +852,35 @@ __global__ void __launch_bounds__(512, 1)
         const int q = (int)(w & 0xffffu), pos = (int)(w >> 16);
         const int ncontrib = p.causal ? q + 1 : N;
         const bool last = (pos == ncontrib - 1);
-        wait(DQ_FULL(it), s_phase(it));
-        if (threadIdx.x == 256) trace(it, 4);
-        tc_fence_after();
         float a[D];
+        if constexpr (C::kSDouble) {
+          // D = 64: the softmax warpgroup of this tile has staged dQp in its dS buffer
+          wait(DQ_EMPTY(it), s_phase(it));
+          if (threadIdx.x == 256) trace(it, 4);
+          const uint32_t stage = sDSt + 32768u * (uint32_t)(it & 1);
 #pragma unroll
-        for (int c2 = 0; c2 < D / 32; ++c2) {
-          uint32_t v[32];
-          tmem_ld32(tmem + lane_off + dq_col(it) + c2 * 32, v);
+          for (int j = 0; j < D / 4; ++j) {
+            const float4 v = ld_shared_f4(stage + (uint32_t)((j * 128 + r) * 16));
+            a[4 * j] = v.x;
+            a[4 * j + 1] = v.y;
+            a[4 * j + 2] = v.z;
+            a[4 * j + 3] = v.w;
+          }
+          mbar_arrive(DS_FREE(it));
+        } else {
+          wait(DQ_FULL(it), s_phase(it));
+          if (threadIdx.x == 256) trace(it, 4);
+          tc_fence_after();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) a[c2 * 32 + j] = __uint_as_float(v[j]);
+          for (int c2 = 0; c2 < D / 32; ++c2) {
+            uint32_t v[32];
+            tmem_ld32(tmem + lane_off + dq_col(it) + c2 * 32, v);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) a[c2 * 32 + j] = __uint_as_float(v[j]);
+          }
+          tc_fence_before();
+          mbar_arrive(DQ_EMPTY(it));
         }
-        tc_fence_before();
-        mbar_arrive(DQ_EMPTY(it));
         if (threadIdx.x == 256) trace(it, 5);
         const long long blk = (long long)ch.x * N + q;
         if constexpr (!kAtomic) {
@@ -741,7 +933,25 @@ __global__ void __launch_bounds__(512, 1)
               }
             }
           };
-          if (idx > 0) {
+          if constexpr (kLook) {
+            if (idx > 0) {
+              if (!pre_ok) {
+                if (threadIdx.x == 256) trace(it, 14);
+                ticket_wait(p.tickets + unit, (uint32_t)idx, ~0u);
+                if (threadIdx.x == 256) trace(it, 6);
+#pragma unroll
+                for (int j = 0; j < NV; ++j) pre[j] = ld_cg_f4(accp + j * 128 + r);
+              }
+#pragma unroll
+              for (int j = 0; j < NV; ++j) {
+                float* x = a + 4 * j;
+                x[0] = pre[j].x + x[0];
+                x[1] = pre[j].y + x[1];
+                x[2] = pre[j].z + x[2];
+                x[3] = pre[j].w + x[3];
+              }
+            }
+          } else if (idx > 0) {
             if (threadIdx.x == 256) trace(it, 14);
             ticket_wait(p.tickets + unit, (uint32_t)idx, ~0u);
             if (threadIdx.x == 256) trace(it, 6);
@@ -784,6 +994,37 @@ __global__ void __launch_bounds__(512, 1)
               // which publishes them at gpu scope
               named_bar_sync(1, 128);
               if (threadIdx.x == 256) st_release_gpu(p.tickets + unit, (uint32_t)(idx + 1));
+            }
+          }
+          if constexpr (kLook) {
+            // the next pair (possibly in a later chain of this CTA): if its ticket is
+            // already granted, its accumulator loads go out now
+            pre_ok = false;
+            int nci = ci, nt = t + 1;
+            while (nci < cend && nt >= n_pairs(p.chains[nci].w)) {
+              ++nci;
+              nt = 0;
+            }
+            if (nci < cend) {
+              const int4 nch = p.chains[nci];
+              const uint32_t nw = p.pairs[nch.z + nt];
+              const int npos = (int)(nw >> 16);
+              if ((npos >> 1) > 0) {
+                const long long nunit =
+                    ((long long)nch.x * N + (int)(nw & 0xffffu)) * 2 + (npos & 1);
+                // lane 0 acquires (pairing with the publisher's release); the warp
+                // barrier orders the other lanes' loads after it
+                uint32_t okw = 0;
+                if (lane == 0)
+                  okw = ld_acquire_gpu(p.tickets + nunit) == (uint32_t)(npos >> 1) ? 1u : 0u;
+                pre_ok = __shfl_sync(0xffffffffu, okw, 0) != 0u;
+                __syncwarp();
+                if (pre_ok) {
+                  const float4* nacc = reinterpret_cast<const float4*>(p.acc) + nunit * (32 * D);
+#pragma unroll
+                  for (int j = 0; j < NV; ++j) pre[j] = ld_cg_f4(nacc + j * 128 + r);
+                }
+              }
             }
           }
         } else {
