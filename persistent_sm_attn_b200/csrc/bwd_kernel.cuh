@@ -31,13 +31,15 @@
 // lower half; dK reads dS^T from shared memory (one buffer per warpgroup).
 //
 // Warp roles (512 threads, four warpgroups):
-//   WG0, WG1  softmax / dS (96 registers at D = 128, 112 at D = 64); D = 128: WG0 owns Q columns 0-63 of every
-//             tile, WG1 columns 64-127; D = 64: WG0 takes the even tiles, WG1 the odd
-//             ones, all 128 columns
-//   WG2       dQ reduction and the dK/dV epilogue (224 registers at D = 128, 200 at D = 64)
-//   WG3       warp 12 TMA producer of K, V and Q, warp 13 MMA issuer and TMEM owner,
-//             warp 14 publisher of the ordered reduction (D = 64), warp 15 TMA producer
-//             of dO (96 registers at D = 128, 88 at D = 64)
+//   WG0, WG1  softmax / dS (96 registers at D = 128, 104 at D = 64); D = 128: WG0 owns
+//             Q columns 0-63 of every tile, WG1 columns 64-127; D = 64: WG0 takes the
+//             even tiles, WG1 the odd ones, all 128 columns, and stages each tile's dQp
+//             out of TMEM into its dS buffer
+//   WG2       dQ reduction and the dK/dV epilogue (224 registers at D = 128, 208 at D = 64)
+//   WG3       warp 12 TMA producer (K, V, Q; dO too at D = 64), warp 13 MMA issuer and
+//             TMEM owner (at D = 64 of the score products S^T, dP^T, dV only), warp 14
+//             publisher of the ordered reduction (D = 64), warp 15 TMA producer of dO
+//             (D = 128) or issuer of the gradient products dQp, dK (D = 64); 96 registers
 // TMEM lane quarter of a warp is (warp % 4), so each warpgroup covers the 128 lanes.
 //
 // TMEM columns (512).  D = 128: S^T [0,128) then packed P^T/dS^T, dP^T
@@ -108,11 +110,9 @@ struct BwdCfg {
   static constexpr int kTile = 128 * D * 2;              // one [128][D] bf16 tile
   // D = 128: Q is double-buffered (the next S^T follows dK right away) and dO has one
   // buffer, refilled between dV of a tile and dP^T of the next, to fit the smem budget.
-  // D = 64: S^T runs two tiles ahead, so Q(i+2) reuses the stage of Q(i-2) (four stages)
-  // and its load has a whole tile to land; dO is read by dP^T(i+1) one tile ahead and
-  // released by dV, so two stages suffice.
-  static constexpr int kStagesQ = (D == 64) ? 4 : 2;
-  static constexpr int kStagesDO = (D == 64) ? 2 : 1;
+  // D = 64: three stages each; S^T runs two tiles ahead and dP^T one.
+  static constexpr int kStagesQ = (D == 64) ? 3 : 2;
+  static constexpr int kStagesDO = (D == 64) ? 3 : 1;
   // LSE and Delta enter the S^T and dP^T products as one extra K-step each: a per-Q-row
   // column tile ([128 rows][8] bf16, loaded with Q) against a constant tile of ones.
   // Each tile is 2 KiB of core matrices (8 rows x 16 bytes, no swizzle) followed by
@@ -243,7 +243,7 @@ __global__ void __launch_bounds__(512, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(BAR(B_KV_FULL), 1);
-    mbar_init(BAR(B_KV_EMPTY), 1);
+    mbar_init(BAR(B_KV_EMPTY), C::kSDouble ? 2u : 1u);
     mbar_init(BAR(B_S_FULL), 1);
     mbar_init(BAR(B_S_FULL1), 1);
     // D = 64: one softmax warpgroup (128 threads) per tile, D = 128: both
@@ -261,9 +261,12 @@ __global__ void __launch_bounds__(512, 1)
       mbar_init(BAR(B_DQ_EMPTY0 + b), 128);
     }
     mbar_init(BAR(B_DVDK_DONE), 1);
-    mbar_init(BAR(B_DKDV_FULL), 1);
+    // D = 64: two threads issue the products (scores and gradients), and each commits
+    // its share of the shared barriers
+    constexpr uint32_t kIssuers = C::kSDouble ? 2u : 1u;
+    mbar_init(BAR(B_DKDV_FULL), kIssuers);
     mbar_init(BAR(B_DKDV_EMPTY), 128);
-    mbar_init(BAR(B_FINAL), 1);
+    mbar_init(BAR(B_FINAL), kIssuers);
     mbar_init(BAR(B_P_READY), kSoftmaxArrive);
     mbar_init(BAR(B_P_READY1), kSoftmaxArrive);
     for (int b = 0; b < 2; ++b) {
@@ -272,7 +275,7 @@ __global__ void __launch_bounds__(512, 1)
     }
     for (int s = 0; s < ST; ++s) {
       mbar_init(Q_FULL(s), 1);
-      mbar_init(Q_EMPTY(s), 1);
+      mbar_init(Q_EMPTY(s), kIssuers);
     }
     for (int s = 0; s < SD; ++s) {
       mbar_init(DO_FULL(s), 1);
@@ -322,8 +325,9 @@ __global__ void __launch_bounds__(512, 1)
     if (warp == 12 && lane == 0) {
       // ---------------------------------------------------------- TMA producer: K, V, Q
       // K/V once per run; per pair Q with its column tile (LSE and Delta terms, read by
-      // S^T and dP^T, which finish before dK frees the stage).  dO has a producer of its
-      // own (warp 15), so a Q load never queues behind the wait for a dO stage.
+      // S^T and dP^T, which finish before dK frees the stage), and at D = 64 dO.  At
+      // D = 128 dO has a producer of its own (warp 15), so a Q load never queues behind
+      // the wait for the single dO stage.
       int it = 0, kn = 0;  // kn: K/V loads so far
       for (int ci = cbeg; ci < cend; ++ci) {
         const int4 ch = p.chains[ci];
@@ -348,6 +352,14 @@ __global__ void __launch_bounds__(512, 1)
           for (int cb = 0; cb < D / 64; ++cb)
             tma_load_2d(sQ + s * C::kTile + cb * 16384, &tmQ, cb * 64, row_q, Q_FULL(s));
           tma_load_2d(sb + C::OFF_COL + s * C::kColTile, &tmC, 0, row_q, Q_FULL(s));
+          if constexpr (C::kSDouble) {
+            const int sd = it % SD;
+            if (it >= SD) wait(DO_EMPTY(sd), ((it / SD) - 1) & 1);
+            mbar_expect_tx(DO_FULL(sd), C::kTile);
+#pragma unroll
+            for (int cb = 0; cb < D / 64; ++cb)
+              tma_load_2d(sDO + sd * C::kTile + cb * 16384, &tmDO, cb * 64, row_q, DO_FULL(sd));
+          }
         }
       }
       // drain: every issued load has landed before the CTA can exit
@@ -355,8 +367,14 @@ __global__ void __launch_bounds__(512, 1)
         const int last_use = ((it - 1 - s) / ST) * ST + s;
         drain(Q_FULL(s), (last_use / ST) & 1);
       }
+      if constexpr (C::kSDouble) {
+        for (int s = 0; s < SD && s < it; ++s) {
+          const int last_use = ((it - 1 - s) / SD) * SD + s;
+          drain(DO_FULL(s), (last_use / SD) & 1);
+        }
+      }
       if (kn > 0) drain(BAR(B_KV_FULL), (kn - 1) & 1);
-    } else if (warp == 15 && lane == 0) {
+    } else if (warp == 15 && lane == 0 && !C::kSDouble) {
       // ---------------------------------------------------------- TMA producer: dO
       int it = 0;
       for (int ci = cbeg; ci < cend; ++ci) {
@@ -378,9 +396,11 @@ __global__ void __launch_bounds__(512, 1)
       }
     } else if (warp == 13 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
-      // One thread issues every MMA; its instruction stream between MMAs is the
-      // issue cost, so the loops are unrolled with constant operand offsets added
-      // to descriptor words, and each product is written out once.
+      // One thread issues every MMA at D = 128; at D = 64 this one issues the score
+      // products and warp 15 the gradient products.  An MMA is accepted only about as
+      // fast as the tensor core runs it, so a waiting issuer idles the tensor core:
+      // the loops are unrolled with constant operand offsets added to descriptor
+      // words, and each product is written out once.
       constexpr uint32_t ID_SS = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
       constexpr uint32_t ID_KV = idesc_bf16_f32(128, D, 0, 1);    // dV, dK (A in TMEM)
       constexpr uint32_t ID_Q = idesc_bf16_f32(128, D, 1, 1);     // dQ
@@ -395,15 +415,11 @@ __global__ void __launch_bounds__(512, 1)
       const uint32_t kOnesS = sdesc_lo_none(sb + C::OFF_ONES, 2048);
       const uint32_t kOnesDP = sdesc_lo_none(sb + C::OFF_ONES + C::kColTile, 2048);
       if constexpr (C::kSDouble) {
-        // D = 64.  The two softmax warpgroups take alternate tiles, so tile i's S^T lives
-        // in buffer i mod 2 and the issuer keeps two tiles in flight: while one
-        // warpgroup forms dS of tile i, the other computes the exponentials of tile i+1.
-        // Per step i, once dS(i) is ready: dP'^T(i+1) (the buffer is free once the
-        // softmax has read dP'^T(i)), dQp(i) and dK(i), dV(i+1) once P^T(i+1) is packed,
-        // then S'^T(i+2) once the softmax has staged dQp(i) out of S^T buffer i mod 2.
-        // Each wait comes after the products that do not depend on it.
+        // D = 64, the score products (S^T, dP^T, dV).  The two softmax warpgroups take
+        // alternate tiles, so tile i's S^T lives in buffer i mod 2 and two tiles are in
+        // flight: while one warpgroup forms dS of tile i, the other computes the
+        // exponentials of tile i+1.
         int it = 0, kn = 0;  // kn: runs started (K/V loads consumed)
-        auto dsbuf = [&](int i) { return sDSt + 32768u * (uint32_t)(i & 1); };
         // S'^T = K Q^T - LSE/scale of tile i into its buffer, once the softmax has
         // staged out the dQp that tile i - 2 left there
         auto issue_s = [&](int i) {
@@ -439,6 +455,7 @@ __global__ void __launch_bounds__(512, 1)
           }
           tc_mma_ss_w(tDP, kOnesDP, kCol, hi_none, ID_SS, 1u);  // - Delta
           tc_commit(DP_FULL(i));
+          tc_commit(Q_EMPTY(s));  // S'^T(i) and dP'^T(i) have read Q and the column tile
           trace(i, 15);
         };
         // dV += P^T dO of tile i (A = P^T from the upper half of its S^T buffer), once
@@ -457,6 +474,10 @@ __global__ void __launch_bounds__(512, 1)
                         kk > 0 ? 1u : acc0);
           tc_commit(DO_EMPTY(sd));  // dP'^T and dV have read dO
         };
+        // the score products' loop: dP'^T(it + 1) once the softmax has read dP'^T(it),
+        // dV(it + 1) once P^T(it + 1) is packed, S'^T(it + 2) once the softmax has
+        // staged dQp(it) out of S^T buffer it mod 2.  The gradient products (dQp, dK)
+        // come from warp 15, so none of these waits holds them up.
         for (int ci = cbeg; ci < cend; ++ci) {
           const int cnt = n_pairs(p.chains[ci].w);
           const bool cprev = cont_prev(ci);
@@ -469,41 +490,21 @@ __global__ void __launch_bounds__(512, 1)
             issue_dv(it, !cprev, cprev ? 1u : 0u);
           }
           for (int t = 0; t < cnt; ++t, ++it) {
-            const int s = it % ST;
-            const uint32_t mQ = sdesc_lo(sQ + s * C::kTile, 16384);
-            const uint32_t mDSi = sdesc_lo(dsbuf(it), 16384);  // dS MN-major (dQp)
-            const uint32_t kDSi = sdesc_lo(dsbuf(it), 16);     // dS^T K-major (dK)
             wait(DS_READY(it), s_phase(it));
             trace(it, 1);
             tc_fence_after();
-            // the other warpgroup's next dS waits for dP'^T(it + 1) first
-            if (t + 1 < cnt) issue_dp(it + 1);
-            // dQp = dS K (both MN-major from shared memory) into the lower 64 columns of
-            // this tile's S^T buffer, which the softmax has finished reading
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              tc_mma_ss_w(tmem + dq_col(it), mDSi + kk * 128, mK + kk * 128, hi, ID_Q,
-                          kk > 0 ? 1u : 0u);
-            // dK += dS^T Q : A = dS^T K-major, B = Q MN-major, both from shared memory
-            const uint32_t acc0 = (t > 0 || cprev) ? 1u : 0u;
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint32_t off = (uint32_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
-              tc_mma_ss_w(tDK, kDSi + off, mQ + kk * 128, hi, ID_KV, kk > 0 ? 1u : acc0);
+            if (t + 1 < cnt) {
+              issue_dp(it + 1);
+              issue_dv(it + 1, false, 1u);
             }
-            // dQp is ready, and dQp and dK have read dS: the softmax stages dQp into the
-            // dS buffer and then frees the S^T buffer (DQ_EMPTY)
-            tc_commit(DQ_FULL(it));
-            tc_commit(Q_EMPTY(s));
-            if (t == cnt - 1 && !cont_next(ci)) tc_commit(BAR(B_DKDV_FULL));
-            trace(it, 2);
-            if (t + 1 < cnt) issue_dv(it + 1, false, 1u);
-            // S'^T(it + 2) last: by now the softmax has had dQp(it) and dK(it) to stage
-            // dQp(it) out of the buffer
             if (t + 2 < cnt) issue_s(it + 2);
+            trace(it, 2);
           }
-          // the run's last chain: K/V are done with
-          if (!cont_next(ci)) tc_commit(BAR(B_KV_EMPTY));
+          // the run's last chain: its dV are all issued, and S^T / dP^T are done with K/V
+          if (!cont_next(ci)) {
+            tc_commit(BAR(B_DKDV_FULL));
+            tc_commit(BAR(B_KV_EMPTY));
+          }
         }
       } else {
         int it = 0, kn = 0;  // kn: runs started (K/V loads consumed)
@@ -598,6 +599,51 @@ __global__ void __launch_bounds__(512, 1)
         }
       }
       // drain: all issued MMAs complete before TMEM is released
+      tc_commit(BAR(B_FINAL));
+      drain(BAR(B_FINAL), 0);
+    } else if (warp == 15 && lane == 0 && C::kSDouble) {
+      // ---------------------------------------------------------- gradient products (D = 64)
+      // dQp(it) = dS K into the lower half of S^T buffer it mod 2 and dK += dS^T Q, once
+      // dS(it) is ready; their commit tells the softmax that dQp is ready to stage and
+      // that dS has been read.
+      constexpr uint32_t ID_KV = idesc_bf16_f32(128, D, 0, 1);  // dK (B = Q MN-major)
+      constexpr uint32_t ID_Q = idesc_bf16_f32(128, D, 1, 1);   // dQp
+      const uint32_t tDK = tmem + C::TM_DK;
+      const uint32_t hi = sdesc_hi(1024);
+      const uint32_t mK = sdesc_lo(sK, 16384);
+      int it = 0, kn = 0;  // kn: runs started
+      for (int ci = cbeg; ci < cend; ++ci) {
+        const int cnt = n_pairs(p.chains[ci].w);
+        const bool cprev = cont_prev(ci);
+        if (!cprev) wait(BAR(B_KV_FULL), (kn++) & 1);
+        for (int t = 0; t < cnt; ++t, ++it) {
+          const int s = it % ST;
+          const uint32_t dsb = sDSt + 32768u * (uint32_t)(it & 1);
+          const uint32_t mQ = sdesc_lo(sQ + s * C::kTile, 16384);
+          const uint32_t mDSi = sdesc_lo(dsb, 16384);  // dS MN-major (dQp)
+          const uint32_t kDSi = sdesc_lo(dsb, 16);     // dS^T K-major (dK)
+          wait(DS_READY(it), s_phase(it));
+          // a run's first chain: the previous run's dK must have been read out
+          if (t == 0 && !cprev && kn >= 2) wait(BAR(B_DKDV_EMPTY), (kn - 2) & 1);
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            tc_mma_ss_w(tmem + dq_col(it), mDSi + kk * 128, mK + kk * 128, hi, ID_Q,
+                        kk > 0 ? 1u : 0u);
+          const uint32_t acc0 = (t > 0 || cprev) ? 1u : 0u;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (uint32_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+            tc_mma_ss_w(tDK, kDSi + off, mQ + kk * 128, hi, ID_KV, kk > 0 ? 1u : acc0);
+          }
+          tc_commit(DQ_FULL(it));
+          tc_commit(Q_EMPTY(s));  // dK(it) has read Q
+        }
+        if (!cont_next(ci)) {
+          tc_commit(BAR(B_DKDV_FULL));
+          tc_commit(BAR(B_KV_EMPTY));  // dQp has read K
+        }
+      }
       tc_commit(BAR(B_FINAL));
       drain(BAR(B_FINAL), 0);
     } else if (warp == 14 && lane == 0 && !kAtomic && C::kPublisher) {
