@@ -173,7 +173,13 @@ def run_ours(args):
     if gqa:
         _, k, v, _ = draw(w.B, args.kv_heads, w.S, w.D, w.sigma,
                           seed_of(args.workload) + 1000 * rank + 1, device="cuda")
-        fwd_call, bwd_call = binding.dash_attn_fwd_gqa, binding.dash_attn_bwd_gqa
+        fwd_call = binding.dash_attn_fwd_gqa
+        split = args.gqa_split or binding.dash_bwd_gqa_split_for(
+            binding.dash_bwd_num_ctas(local, w.D), w.B, args.kv_heads, w.H // args.kv_heads,
+            w.S, w.causal, sched)
+
+        def bwd_call(*a):
+            return binding.dash_attn_bwd_gqa(*a, split=split)
     else:
         fwd_call, bwd_call = binding.dash_attn_fwd, binding.dash_attn_bwd
     o, lse = fwd_call(q, k, v, w.causal)
@@ -307,7 +313,8 @@ def run_ours(args):
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic (seeded normal bf16 Q, K, V, dO; O and LSE from the library forward)",
-            "config": _config(w, sched, world, args.kv_heads if gqa else w.H),
+            "config": dict(_config(w, sched, world, args.kv_heads if gqa else w.H),
+                           **({"gqa_split": split} if gqa else {})),
             "pct_of_peak": round(100 * value / (peak * world), 2),
             "schedules_tflops": det,
             "det_nondet_ratio": (round(best_det / det["atomic"], 4)
@@ -469,6 +476,8 @@ def main():
     ap.add_argument("--kv-heads", type=int, default=0,
                     help="time grouped-query attention with this many K/V heads (a side "
                          "measurement: no host-buffer e2e, simulator or CPU baseline)")
+    ap.add_argument("--gqa-split", type=int, default=0,
+                    help="with --kv-heads: sub-groups per K/V head (0 = the library's choice)")
     ap.add_argument("--heads", type=int, default=0,
                     help="run the workload's shape with B=1 and this many heads (a smaller "
                          "case of the same kernel, for profiling); 0 = the workload as named")

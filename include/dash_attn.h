@@ -98,19 +98,42 @@ int dash_attn_bwd(const void* q, const void* k, const void* v, const void* o,
  * (a power of two): query head h reads K/V head h / (H / Hkv).
  *   q, o, dout, dq: bf16 [B, H, S, D];  k, v, dk, dv: bf16 [B, Hkv, S, D];
  *   lse: fp32 [B, H, S].
- * dK and dV sum over the K/V head's query heads.  The schedule table runs the chains
- * that feed one dK/dV tile back to back on one CTA, so that sum accumulates in the
- * kernel's fp32 accumulators in a fixed order (query heads in order) with no extra
- * reduction; dQ is ordered per query head as for dash_attn_bwd.  Hkv == H is
- * dash_attn_fwd / dash_attn_bwd.  Errors: DASH_ERR_INVALID_ARG if Hkv < 1 or does not
- * divide H, DASH_ERR_UNSUPPORTED if H / Hkv is not a power of two; otherwise as
- * dash_attn_fwd / dash_attn_bwd.
+ * dK and dV sum over the K/V head's query heads.  The group of H / Hkv query heads is
+ * cut into `split` sub-groups of consecutive heads (a power of two dividing H / Hkv).
+ * The schedule table runs the chains that feed one dK/dV tile of one sub-group back
+ * to back on one CTA, so the sub-group's sum accumulates in the kernel's fp32
+ * accumulators, query heads in order.  With split > 1 each sub-group is a unit of
+ * its own (more units for the persistent grid, shorter runs); the sub-groups'
+ * fp32 partials of a dK/dV tile are added in sub-group order (sub-group s waits,
+ * bounded, for s - 1 under a ticket) and the last one rounds to bf16, so the
+ * result stays deterministic.  This uses 2 * B * Hkv * S * D fp32 of scratch.
+ * dQ is ordered per query head as for dash_attn_bwd.  Hkv == H is dash_attn_fwd /
+ * dash_attn_bwd.
+ * dash_attn_bwd_gqa lets the library choose split (the smallest power of two that
+ * fills the grid's rounds noticeably better; dash_bwd_gqa_split_for reports it);
+ * dash_attn_bwd_gqa_split takes it from the caller, 0 meaning the library's choice.
+ * Errors: DASH_ERR_INVALID_ARG if Hkv < 1 or does not divide H, or split is negative,
+ * not a power of two or does not divide H / Hkv; DASH_ERR_UNSUPPORTED if H / Hkv is
+ * not a power of two; otherwise as dash_attn_fwd / dash_attn_bwd.
  */
 int dash_attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                       int H, int Hkv, int S, int D, int causal, void* stream);
 int dash_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
                       const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
                       int H, int Hkv, int S, int D, int causal, int schedule, void* stream);
+int dash_attn_bwd_gqa_split(const void* q, const void* k, const void* v, const void* o,
+                            const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                            int B, int H, int Hkv, int S, int D, int causal, int schedule,
+                            int split, void* stream);
+/*
+ * The split dash_attn_bwd_gqa uses for B * Hkv K/V heads with `group` query heads
+ * each on a grid of num_ctas persistent CTAs (dash_bwd_num_ctas).  Host only: no
+ * device call.  Errors: DASH_ERR_INVALID_ARG for a NULL split, num_ctas, B, Hkv or
+ * group below 1, group not a power of two or causal not 0/1; DASH_ERR_UNSUPPORTED
+ * for a length or schedule the backward refuses.
+ */
+int dash_bwd_gqa_split_for(int num_ctas, int B, int Hkv, int group, int S, int causal,
+                           int schedule, int* split);
 
 /*
  * Synchronises `stream`, then returns and clears the device error word of

@@ -25,7 +25,8 @@ EXPORTS = ("dash_attn_fwd", "dash_attn_bwd", "dash_attn_sync_status", "dash_stat
            "dash_profile_begin", "dash_profile_end", "dash_attn_bwd_noalloc",
            "dash_trace_bwd", "dash_inject_fault", "dash_sched_check", "dash_attn_bwd_host",
            "dash_sched_table_part", "dash_attn_fwd_gqa", "dash_attn_bwd_gqa",
-           "dash_sched_table_gqa", "dash_attn_noalloc_sync_status")
+           "dash_sched_table_gqa", "dash_attn_noalloc_sync_status",
+           "dash_attn_bwd_gqa_split", "dash_bwd_gqa_split_for")
 
 
 class DashError(RuntimeError):
@@ -59,6 +60,8 @@ def load(path: str | None = None):
     lib.dash_attn_bwd_host.argtypes = [vp] * 9 + [i, i, i, i, i, i, vp]
     lib.dash_attn_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
     lib.dash_attn_bwd_gqa.argtypes = [vp] * 9 + [i, i, i, i, i, i, i, vp]
+    lib.dash_attn_bwd_gqa_split.argtypes = [vp] * 9 + [i, i, i, i, i, i, i, i, vp]
+    lib.dash_bwd_gqa_split_for.argtypes = [i, i, i, i, i, i, i, P(i)]
     lib.dash_attn_sync_status.argtypes = [vp]
     lib.dash_attn_noalloc_sync_status.argtypes = [vp]
     lib.dash_status_string.argtypes = [i]
@@ -83,7 +86,8 @@ def load(path: str | None = None):
     lib.dash_profile_end.argtypes = [P(d), P(d), P(ll)]
     for name in EXPORTS:
         if name not in ("dash_status_string", "dash_sched_table", "dash_sched_table_part",
-                        "dash_sched_table_gqa", "dash_attn_noalloc_sync_status"):
+                        "dash_sched_table_gqa", "dash_attn_noalloc_sync_status",
+           "dash_attn_bwd_gqa_split", "dash_bwd_gqa_split_for"):
             getattr(lib, name).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -199,9 +203,10 @@ def dash_attn_fwd_gqa(q, k, v, causal: bool, out=None, lse=None, stream=None):
 
 
 def dash_attn_bwd_gqa(q, k, v, o, do, lse, causal: bool, schedule="shift", dq=None, dk=None,
-                      dv=None, stream=None):
+                      dv=None, stream=None, split=None):
     """dQ [B,H,S,D], dK and dV [B,Hkv,S,D] of grouped-query attention (dK, dV summed
-    over each K/V head's query heads)."""
+    over each K/V head's query heads).  split: sub-groups per K/V head (a power of
+    two dividing H / Hkv); None or 0 lets the library choose."""
     import torch
     _check_tensors(q, k, v, o, do, lse, (dq, dk, dv), gqa=True)
     B, H, S, D = q.shape
@@ -209,11 +214,24 @@ def dash_attn_bwd_gqa(q, k, v, o, do, lse, causal: bool, schedule="shift", dq=No
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    rc = load().dash_attn_bwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse),
-                                  _ptr(dq), _ptr(dk), _ptr(dv), B, H, Hkv, S, D,
-                                  int(bool(causal)), _sched_id(schedule), _stream_handle(stream))
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk),
+            _ptr(dv), B, H, Hkv, S, D, int(bool(causal)), _sched_id(schedule))
+    if split is None:
+        rc = load().dash_attn_bwd_gqa(*args, _stream_handle(stream))
+    else:
+        rc = load().dash_attn_bwd_gqa_split(*args, int(split), _stream_handle(stream))
     _check(rc, "dash_attn_bwd_gqa")
     return dq, dk, dv
+
+
+def dash_bwd_gqa_split_for(num_ctas: int, B: int, Hkv: int, group: int, S: int, causal: bool,
+                           schedule="shift") -> int:
+    """The sub-group count dash_attn_bwd_gqa chooses (host only)."""
+    n = ctypes.c_int(0)
+    _check(load().dash_bwd_gqa_split_for(num_ctas, B, Hkv, group, S, int(bool(causal)),
+                                         _sched_id(schedule), ctypes.byref(n)),
+           "dash_bwd_gqa_split_for")
+    return n.value
 
 
 def dash_attn_bwd_host(q, k, v, o, do, lse, causal: bool, schedule="shift", dq=None, dk=None,

@@ -87,6 +87,14 @@ struct BwdParams {
   __nv_bfloat16* dv;
   int S, N, causal;
   int group_log2;         // log2 of the query heads per K/V head (0: one K/V head each)
+  // Grouped-query attention with each K/V head's group split into 2^split_log2 sub-groups
+  // that run as separate units: the sub-groups' dK/dV partials of a (K/V head, KV tile)
+  // add, in sub-group order, into fp32 accumulators [dV, dK][D/4][128][4] under one
+  // ticket each; the last sub-group writes bf16.  split_log2 = 0: dK/dV go straight
+  // to bf16.
+  int split_log2 = 0;
+  float* dkv_acc = nullptr;
+  uint32_t* dkv_tickets = nullptr;
   float scale, scale_log2;
   unsigned long long spin_ns;
   // Optional %globaltimer trace (kernels instantiated with kTrace only):
@@ -1089,6 +1097,85 @@ __global__ void __launch_bounds__(512, 1)
       wait(BAR(B_DKDV_FULL), (fn++) & 1);
       tc_fence_after();
       const size_t row = (size_t)(ch.x >> gl2) * S + (size_t)ch.y * 128 + r;
+      if (p.split_log2 > 0) {
+        // This run is sub-group s of its K/V head's group: it adds its dK/dV partials
+        // to the fp32 accumulator after sub-group s - 1 (an ordered load-add-store
+        // under the tile's ticket, as for dQ), and sub-group sp - 1 rounds to bf16.
+        // (A wait-free variant, where the last sub-group to finish adds every slot,
+        // made the whole kernel slower, also without a split.)
+        const int sp = 1 << p.split_log2;
+        const int s = (ch.x >> (gl2 - p.split_log2)) & (sp - 1);
+        const long long unit = (long long)(ch.x >> gl2) * N + ch.y;
+        float4* acc = reinterpret_cast<float4*>(p.dkv_acc) + unit * (2 * 32 * D);
+        uint32_t* tk = p.dkv_tickets + unit;
+        if (s > 0) {
+          // bounded wait: lane 0 acquires, the warp barrier orders the lanes' loads
+          if (lane == 0 && ld_acquire_gpu(tk) != (uint32_t)s) {
+            const uint64_t t0 = globaltimer();
+            bool ok = false;
+            while (!ok) {
+#pragma unroll 1
+              for (int i = 0; i < 32 && !ok; ++i) ok = (ld_acquire_gpu(tk) == (uint32_t)s);
+              if (!ok && (aborted(p.abort_flag) || globaltimer() - t0 > lim)) {
+                if (!aborted(p.abort_flag)) raise_timeout(p.err, p.abort_flag, ERR_WHERE_TICKET);
+                break;
+              }
+            }
+          }
+          __syncwarp();
+        }
+#pragma unroll 1
+        for (int which = 0; which < 2; ++which) {
+          const uint32_t col = which ? C::TM_DK : C::TM_DV;
+          const float sc = which ? p.scale : 1.0f;
+          __nv_bfloat16* out = (which ? p.dk : p.dv) + row * D;
+          float4* a = acc + which * 32 * D;
+#pragma unroll
+          for (int c2 = 0; c2 < D / 32; ++c2) {
+            uint32_t v[32];
+            tmem_ld32(tmem + lane_off + col + c2 * 32, v);
+            float x[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) x[j] = __uint_as_float(v[j]);
+            if (s > 0) {
+              float4 old[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) old[j] = ld_cg_f4(a + (c2 * 8 + j) * 128 + r);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                x[4 * j] = old[j].x + x[4 * j];
+                x[4 * j + 1] = old[j].y + x[4 * j + 1];
+                x[4 * j + 2] = old[j].z + x[4 * j + 2];
+                x[4 * j + 3] = old[j].w + x[4 * j + 3];
+              }
+            }
+            if (s < sp - 1) {
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                st_cg_f4(a + (c2 * 8 + j) * 128 + r,
+                         make_float4(x[4 * j], x[4 * j + 1], x[4 * j + 2], x[4 * j + 3]));
+            } else {
+#pragma unroll
+              for (int c8 = 0; c8 < 4; ++c8) {
+                uint4 pk;
+                pk.x = pack_bf16x2(x[8 * c8] * sc, x[8 * c8 + 1] * sc);
+                pk.y = pack_bf16x2(x[8 * c8 + 2] * sc, x[8 * c8 + 3] * sc);
+                pk.z = pack_bf16x2(x[8 * c8 + 4] * sc, x[8 * c8 + 5] * sc);
+                pk.w = pack_bf16x2(x[8 * c8 + 6] * sc, x[8 * c8 + 7] * sc);
+                *reinterpret_cast<uint4*>(out + c2 * 32 + c8 * 8) = pk;
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(BAR(B_DKDV_EMPTY));
+        if (s < sp - 1) {
+          // every reducer's stores precede thread 256's release, which publishes them
+          named_bar_sync(1, 128);
+          if (threadIdx.x == 256) st_release_gpu(tk, (uint32_t)(s + 1));
+        }
+        continue;
+      }
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         const uint32_t col = which ? C::TM_DK : C::TM_DV;

@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <array>
 #include <atomic>
 #include <cstdint>
@@ -52,6 +53,8 @@ struct Workspace {
   size_t tk_bytes = 0;
   float* rowbuf = nullptr;  // per-row column terms of the backward, 16 bytes per row
   size_t rows_cap = 0;
+  float* dkv = nullptr;     // fp32 dK/dV accumulators of split grouped-query sub-groups
+  size_t dkv_bytes = 0;
   unsigned* err = nullptr;   // [0] error word, [1] per-launch abort flag
 };
 
@@ -103,10 +106,11 @@ int grow(void** p, size_t* have, size_t need) {
 }
 
 int get_workspace(int dev, void* stream, size_t acc_bytes, size_t tk_bytes, size_t rows,
-                  Workspace** out) {
+                  Workspace** out, size_t dkv_bytes = 0) {
   Workspace& w = g_ws[{dev, reinterpret_cast<uintptr_t>(stream)}];
   int rc;
   if ((rc = grow(reinterpret_cast<void**>(&w.acc), &w.acc_bytes, acc_bytes))) return rc;
+  if ((rc = grow(reinterpret_cast<void**>(&w.dkv), &w.dkv_bytes, dkv_bytes))) return rc;
   if ((rc = grow(reinterpret_cast<void**>(&w.tickets), &w.tk_bytes, tk_bytes))) return rc;
   size_t rb = w.rows_cap * 16;
   if (rows > w.rows_cap) {
@@ -353,17 +357,53 @@ int num_ctas_for(int dev, int* out) {
   return DASH_OK;
 }
 
+// Sub-groups per K/V head for a grouped-query backward (split = 0 asks for this choice).
+// Each K/V head contributes `per_head` units per sub-group; a round is `ctas` units.
+// Two measured effects decide: a split whose units fill the grid's rounds better wins;
+// among splits that fill them equally (within 2 points), runs of two query heads are
+// fastest (longer runs stretch the schedule's dQ order, one-head runs send every dK/dV
+// tile through the ordered fp32 reduction).
+int choose_split(long long kv_heads, int group, long long per_head, int ctas) {
+  auto fill = [&](int sp) {
+    const long long u = kv_heads * sp * per_head;
+    const long long rounds = (u + ctas - 1) / ctas;
+    return (double)u / (double)(rounds * ctas);
+  };
+  double best_fill = 0.0;
+  for (int sp = 1; sp <= group; sp *= 2) best_fill = std::max(best_fill, fill(sp));
+  int best = 1, best_dist = 1 << 30;
+  for (int sp = 1; sp <= group; sp *= 2) {
+    if (fill(sp) < best_fill - 0.02) continue;
+    const int heads_log2 = __builtin_ctz((unsigned)(group / sp));  // log2 heads per run
+    const int dist = heads_log2 > 1 ? heads_log2 - 1 : 1 - heads_log2;
+    if (dist < best_dist) {
+      best = sp;
+      best_dist = dist;
+    }
+  }
+  return best;
+}
+
 template <int D, bool kAtomic, bool kTrace = false>
 int launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                const float* lse, void* dq, void* dk, void* dv, int B, int H, int S, int causal,
                int sched, cudaStream_t stream, int dev, unsigned long long* trace = nullptr,
-               int trace_rows = 0, const DevTable* tab_override = nullptr, int group = 1) {
+               int trace_rows = 0, const DevTable* tab_override = nullptr, int group = 1,
+               int split = 1) {
   using C = BwdCfg<D>;
   const int N = S / 128;
   const long long rows = (long long)B * H * S;
   int ctas = 0;
   int rc = num_ctas_for<D, kAtomic>(dev, &ctas);
   if (rc) return rc;
+  if (split == 0)
+    split = group > 1 ? choose_split((long long)B * (H / group), group,
+                                     (long long)dash::head_units(sched, N, causal).size(), ctas)
+                      : 1;
+  // a split group runs as group / split query heads per (virtual) K/V head in the table;
+  // the kernel still reads K/V of head / group
+  const long long dqn = dash::dq_units<D>((long long)B * H * N);
+  const long long dkvn = split > 1 ? (long long)B * (H / group) * N : 0;
   DevTable* tab = nullptr;
   Workspace* ws = nullptr;
   {
@@ -374,12 +414,12 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
       tab = const_cast<DevTable*>(tab_override);
     } else if (fault == 1 && !kAtomic) {
       if ((rc = get_fault_table(dev, B * H, N, causal, sched, ctas, &tab))) return rc;
-    } else if ((rc = get_table(dev, B * H, N, causal, sched, ctas, &tab, group))) {
+    } else if ((rc = get_table(dev, B * H, N, causal, sched, ctas, &tab, group / split))) {
       return rc;
     }
     if ((rc = get_workspace(dev, stream, 2 * (size_t)rows * D * sizeof(float),
-                            (size_t)dash::dq_units<D>((long long)B * H * N) * sizeof(uint32_t),
-                            (size_t)rows, &ws)))
+                            (size_t)(dqn + dkvn) * sizeof(uint32_t), (size_t)rows, &ws,
+                            2 * (size_t)(rows / group) * D * sizeof(float) * (split > 1))))
       return rc;
   }
   CUtensorMap tq, tk, tv, tdo, tc;
@@ -394,10 +434,11 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   if (!prof_record(0, &ev, stream)) return DASH_ERR_CUDA;
   // Delta and the column terms; the same launch clears the abort flag and, on the
   // deterministic path, the tickets
+  // (the dQ tickets on the deterministic path, the dK/dV tickets of a split group)
   dash::dash_delta_kernel<D><<<dash::delta_grid<D>(rows, ctas), 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse,
-      reinterpret_cast<uint4*>(ws->rowbuf), rows, 1.0f / scale, ws->tickets,
-      kAtomic ? 0LL : dash::dq_units<D>((long long)B * H * N), ws->err + 1, 1);
+      reinterpret_cast<uint4*>(ws->rowbuf), rows, 1.0f / scale, ws->tickets + (kAtomic ? dqn : 0),
+      (kAtomic ? 0LL : dqn) + dkvn, ws->err + 1, 1);
   if (kAtomic) DASH_CUDA(cudaMemsetAsync(ws->acc, 0, (size_t)rows * D * sizeof(float), stream));
   BwdParams p;
   p.cta_off = tab->cta_off;
@@ -414,6 +455,9 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   p.N = N;
   p.causal = causal;
   p.group_log2 = __builtin_ctz((unsigned)group);
+  p.split_log2 = __builtin_ctz((unsigned)split);
+  p.dkv_acc = ws->dkv;
+  p.dkv_tickets = ws->tickets + dqn;
   p.scale = scale;
   p.scale_log2 = p.scale * 1.4426950408889634f;
   p.spin_ns = (unsigned long long)spin_us() * 1000ull;
@@ -679,15 +723,20 @@ int dash_attn_fwd(const void* q, const void* k, const void* v, void* o, float* l
   return dash_attn_fwd_gqa(q, k, v, o, lse, B, H, H, S, D, causal, stream);
 }
 
-int dash_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
-                      const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
-                      int H, int Hkv, int S, int D, int causal, int schedule, void* stream) {
+int dash_attn_bwd_gqa_split(const void* q, const void* k, const void* v, const void* o,
+                            const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                            int B, int H, int Hkv, int S, int D, int causal, int schedule,
+                            int split, void* stream) {
   return no_throw([&]() -> int {
     int rc = check_shape(B, H, S, D);
     if (rc) return rc;
     if (causal != 0 && causal != 1) return DASH_ERR_INVALID_ARG;
     if (H > 0 && (Hkv < 1 || H % Hkv != 0)) return DASH_ERR_INVALID_ARG;
     if (H > 0 && ((H / Hkv) & (H / Hkv - 1)) != 0) return DASH_ERR_UNSUPPORTED;  // 2^k per K/V head
+    // split: 0 = chosen by the library, else a power of two dividing the group
+    if (split < 0 || (split > 0 && H > 0 &&
+                      ((split & (split - 1)) != 0 || (H / Hkv) % split != 0)))
+      return DASH_ERR_INVALID_ARG;
     if (schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_ATOMIC)
       return DASH_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
@@ -702,13 +751,34 @@ int dash_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o
     const int g = H / Hkv;
     if (D == 64)
       return atomic ? launch_bwd<64, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
-                                           schedule, st, dev, nullptr, 0, nullptr, g)
+                                           schedule, st, dev, nullptr, 0, nullptr, g, split)
                     : launch_bwd<64, false>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
-                                            schedule, st, dev, nullptr, 0, nullptr, g);
+                                            schedule, st, dev, nullptr, 0, nullptr, g, split);
     return atomic ? launch_bwd<128, true>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
-                                          schedule, st, dev, nullptr, 0, nullptr, g)
+                                          schedule, st, dev, nullptr, 0, nullptr, g, split)
                   : launch_bwd<128, false>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
-                                           schedule, st, dev, nullptr, 0, nullptr, g);
+                                           schedule, st, dev, nullptr, 0, nullptr, g, split);
+  }, DASH_ERR_OOM, DASH_ERR_INVALID_ARG);
+}
+
+int dash_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
+                      const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                      int H, int Hkv, int S, int D, int causal, int schedule, void* stream) {
+  return dash_attn_bwd_gqa_split(q, k, v, o, dout, lse, dq, dk, dv, B, H, Hkv, S, D, causal,
+                                 schedule, 0, stream);
+}
+
+int dash_bwd_gqa_split_for(int num_ctas, int B, int Hkv, int group, int S, int causal,
+                           int schedule, int* split) {
+  return no_throw([&]() -> int {
+    if (!split || num_ctas < 1 || B < 1 || Hkv < 1 || group < 1 || (group & (group - 1)) != 0 ||
+        (causal != 0 && causal != 1))
+      return DASH_ERR_INVALID_ARG;
+    if (S < 128 || S % 128 != 0) return DASH_ERR_UNSUPPORTED;
+    if (!dash::schedule_supported(schedule, S / 128, causal)) return DASH_ERR_UNSUPPORTED;
+    *split = choose_split((long long)B * Hkv, group,
+                          (long long)dash::head_units(schedule, S / 128, causal).size(), num_ctas);
+    return DASH_OK;
   }, DASH_ERR_OOM, DASH_ERR_INVALID_ARG);
 }
 
@@ -823,6 +893,7 @@ int dash_release_workspace(void) {
   for (auto itw = g_ws.begin(); itw != g_ws.end();) {
     if (itw->first.first == dev) {
       cudaFree(itw->second.acc);
+      cudaFree(itw->second.dkv);
       cudaFree(itw->second.tickets);
       cudaFree(itw->second.rowbuf);
       cudaFree(itw->second.err);

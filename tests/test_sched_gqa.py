@@ -185,3 +185,102 @@ def test_tables_beyond_int32_pairs_are_refused_before_building():
     # 256 heads x 4096^2 pairs > 2^31 - 1: refused as unsupported, without building
     assert lib.dash_sched_table_gqa(256, 1, 4096, 0, 2, 148, None, 0) == -2
     assert lib.dash_sched_table(256, 4096, 0, 2, 148, None, 0) == -2
+
+
+# ---------------------------------------------------------------------------
+# Split groups: each K/V head's group of g query heads cut into `split` sub-groups
+# of g / split consecutive heads, each a unit of its own (the table of g / split
+# query heads per virtual K/V head).  Sub-group s adds its dK/dV partials of a KV
+# tile after sub-group s - 1 has added its own.
+
+@pytest.mark.parametrize("name,N,causal,heads,group,split,ctas", [
+    (sc.SHIFT, 4, False, 8, 4, 2, 3), (sc.SHIFT, 4, False, 8, 4, 4, 5),
+    (sc.DESCENDING, 3, True, 4, 4, 2, 2), (sc.NAIVE_ASC, 5, True, 8, 8, 4, 7),
+    (sc.SYM_SHIFT, 4, True, 8, 2, 2, 4), (sc.SYM_SHIFT, 6, True, 16, 8, 8, 9),
+    (sc.SHIFT, 8, False, 16, 8, 4, 148), (sc.DESCENDING, 6, False, 4, 4, 4, 1)])
+def test_split_group_table(name, N, causal, heads, group, split, ctas):
+    """The virtual table of a split group: each (K/V head, KV tile) is one run per
+    sub-group, its g / split query heads in order; and every wait (the dQ tickets with
+    one or two chains per block, and sub-group s's dK/dV epilogue after s - 1's) points
+    back in the grid's execution order, so no CTA waits forever."""
+    sub = group // split
+    rows = binding.dash_sched_table_gqa(heads, sub, N, causal, SID[name], ctas)
+    slots = [[] for _ in range(ctas)]
+    for cta, h, kv, q, p, _ in rows:
+        slots[cta].append((h, kv, q, p, q + 1 if causal else N))
+    for chains in (1, 2):
+        n, edges, index = dag.schedule_graph(slots, 1.0, 0.3, None, chains)
+        # a run's epilogue follows its last reduction and precedes the CTA's next one
+        epi = {}
+        for sl, seq in enumerate(slots):
+            for i, (h, kv, _, _, _) in enumerate(seq):
+                nxt = seq[i + 1] if i + 1 < len(seq) else None
+                if nxt is not None and nxt[0] // sub == h // sub and nxt[1] == kv:
+                    continue
+                epi[(h // group, kv, (h // sub) % split)] = n
+                edges.append((index[(sl, i)] + 3, n, 0.0))
+                if nxt is not None:
+                    edges.append((n, index[(sl, i + 1)] + 2, 0.0))
+                n += 1
+        for (kvh, kv, s), e in epi.items():
+            if s > 0:
+                edges.append((epi[(kvh, kv, s - 1)], e, 0.0))
+        assert _acyclic(n, edges)
+        assert len(epi) == (heads // group) * N * split
+    runs = defaultdict(list)   # (K/V head, kv, sub-group) -> query heads, per chain
+    prev = None
+    for cta, h, kv, q, p, ci in rows:
+        if ci != prev:
+            runs[(h // group, kv, (h // sub) % split)].append((cta, h))
+            prev = ci
+    assert sorted(runs) == sorted((kvh, kv, s) for kvh in range(heads // group)
+                                  for kv in range(N) for s in range(split))
+    for (kvh, kv, s), members in runs.items():
+        assert len({c for c, _ in members}) == 1          # one CTA
+        assert [h for _, h in members] == [kvh * group + s * sub + i for i in range(sub)]
+
+
+def test_split_choice():
+    """dash_bwd_gqa_split_for: among the splits whose units fill the grid's rounds
+    within 2 points of the best, the one closest to two query heads per run
+    (hand-counted)."""
+    f = binding.dash_bwd_gqa_split_for
+    # 1 K/V head of 8, shift at S = 4096 (32 units per sub-group) on 148 CTAs:
+    # 32/148, 64/148, 128/148, 256/296 -> splits 4 and 8 fill best; 4 runs two heads
+    assert f(148, 1, 1, 8, 4096, False, "shift") == 4
+    # 4 K/V heads of 8, shift at S = 4096: 128/148, 256/296, 512/592 (0.865),
+    # 1024/1036 (0.988) -> only 8 fills best
+    assert f(148, 2, 2, 8, 4096, False, "shift") == 8
+    # 8 K/V heads of 8: 256/296, 512/592 (0.865), 1024/1036, 2048/2072 (0.988) -> 4
+    assert f(148, 1, 8, 8, 4096, False, "shift") == 4
+    # 4 K/V heads x 37 units (shift at S = 4736) fill every round at every split -> 4
+    assert f(148, 1, 4, 8, 4736, False, "shift") == 4
+    # 16 K/V heads of 8, sym_shift causal S = 16384 (64 units): 1024/1036 and up, all
+    # 0.988 -> 4
+    assert f(148, 4, 4, 8, 16384, True, "sym_shift") == 4
+    # 2 K/V heads of 4, sym_shift causal S = 8192 (32 units): 64/148, 128/148,
+    # 256/296 -> splits 2 and 4 fill best; 2 runs two heads
+    assert f(148, 1, 2, 4, 8192, True, "sym_shift") == 2
+    # 1 K/V head of 2, naive_asc at S = 16384: 128/148, 256/296 -> 1 (two heads a run)
+    assert f(148, 1, 1, 2, 16384, False, "naive_asc") == 1
+    assert f(148, 4, 8, 1, 4096, False, "shift") == 1      # no group to split
+    assert f(1, 1, 1, 16, 1024, True, "descending") == 8   # one CTA: always full
+    for bad in ((0, 1, 1, 2, 1024, False, "shift"), (148, 1, 1, 3, 1024, False, "shift"),
+                (148, 0, 1, 2, 1024, False, "shift")):
+        with pytest.raises(binding.DashError):
+            f(*bad)
+    with pytest.raises(binding.DashError):
+        f(148, 1, 1, 2, 1000, False, "shift")               # not a multiple of 128
+    with pytest.raises(binding.DashError):
+        f(148, 1, 1, 2, 1024, True, "shift")                # shift needs the full mask
+
+
+def test_split_argument_errors_before_the_device():
+    """A bad split is refused before any device call (dummy pointers, no GPU)."""
+    import ctypes
+    lib = binding.load()
+    buf = ctypes.create_string_buffer(64)
+    al = ctypes.c_void_p((ctypes.addressof(buf) + 15) // 16 * 16)
+    for split in (-1, 3, 8, 16):   # group 4: 3 not a power of two, 8 and 16 do not divide
+        rc = lib.dash_attn_bwd_gqa_split(*([al] * 9), 1, 8, 2, 256, 64, 0, 2, split, None)
+        assert rc == 1, split      # DASH_ERR_INVALID_ARG
