@@ -154,6 +154,18 @@ const char* dash_status_string(int status);
 int dash_set_spin_limit_us(long long us);
 
 /*
+ * How the deterministic backward adds a dQ partial at a middle position of an
+ * accumulation chain (DASH summary §1, the serialised accumulation): 0 (default) picks
+ * per launch, 1 always adds in L2 with red once the ticket grants the position, 2
+ * always loads, adds on the SM and stores.  The additions and their order are the
+ * same, so the results are bitwise the same; mode 0 takes red for the descending and
+ * naive ascending schedules from 64 tiles, where it measured faster.  Applies to later
+ * dash_attn_bwd / dash_attn_bwd_gqa / dash_attn_bwd_host calls on every stream
+ * (dash_attn_bwd_noalloc always loads and stores).  Other modes: INVALID_ARG.
+ */
+int dash_set_dq_chain_mode(int mode);
+
+/*
  * Failure-detection testing.  mode 1: the next deterministic dash_attn_bwd or
  * dash_attn_bwd_noalloc (any stream) runs with a schedule table in which dQ
  * block (head 0, Q tile 0) never receives its first two partials, so its ticket

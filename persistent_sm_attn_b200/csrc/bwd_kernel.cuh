@@ -192,7 +192,12 @@ __host__ __device__ constexpr uint32_t p_col64(int c) { return 64u + 16u * (uint
 //  12 MMA issuer starts waiting for the S^T buffer 13 load-add-store (or atomics) done
 //  14 reducers start waiting for the ticket        15 dP^T issued
 constexpr int kTraceEvents = 16;
-template <int D, bool kAtomic, bool kTrace = false>
+// kRed (deterministic only): a chain's middle positions add their partial into the
+// accumulator with red (fp32 addition performed in L2, no read back) once the ticket
+// grants them, instead of a load-add-store from the SM.  The additions and their order
+// are the same, so the results are bitwise the same; only the traffic and the latency
+// of each link differ.
+template <int D, bool kAtomic, bool kTrace = false, bool kRed = false>
 __global__ void __launch_bounds__(512, 1)
     dash_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -896,7 +901,7 @@ __global__ void __launch_bounds__(512, 1)
     // next pair go out if its ticket is already granted (checked once, never waited
     // for here), so their round trip overlaps the wait for the next partial and its
     // drain.  The values loaded and the order of the additions are the same either way.
-    constexpr bool kLook = !kAtomic && D == 64;
+    constexpr bool kLook = !kAtomic && D == 64 && !kRed;
     float4 pre[NV];
     bool pre_ok = false;  // pre holds this pair's accumulator, loaded ahead
     for (int ci = cbeg; ci < cend; ++ci) {
@@ -987,7 +992,15 @@ __global__ void __launch_bounds__(512, 1)
               }
             }
           };
-          if constexpr (kLook) {
+          if constexpr (kRed) {
+            // middle positions add with red in L2 below; only the last one loads
+            if (idx > 0 && last) {
+              if (threadIdx.x == 256) trace(it, 14);
+              ticket_wait(p.tickets + unit, (uint32_t)idx, ~0u);
+              if (threadIdx.x == 256) trace(it, 6);
+              add_from(accp);
+            }
+          } else if constexpr (kLook) {
             if (idx > 0) {
               if (!pre_ok) {
                 if (threadIdx.x == 256) trace(it, 14);
@@ -1032,10 +1045,23 @@ __global__ void __launch_bounds__(512, 1)
               *reinterpret_cast<uint4*>(out + 8 * c8) = pk;
             }
           } else {
+            if (kRed && idx > 0) {
+              // Once the ticket shows every earlier position's additions performed, this
+              // partial is added in L2 (red, no read back); the release below waits for
+              // these additions to be performed, so the chain's order is kept.
+              if (threadIdx.x == 256) trace(it, 14);
+              ticket_wait(p.tickets + unit, (uint32_t)idx, ~0u);
+              if (threadIdx.x == 256) trace(it, 6);
 #pragma unroll
-            for (int c4 = 0; c4 < NV; ++c4)
-              st_cg_f4(accp + c4 * 128 + r,
-                       make_float4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]));
+              for (int c4 = 0; c4 < NV; ++c4)
+                red_add_f4(accp + c4 * 128 + r,
+                           make_float4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]));
+            } else {
+#pragma unroll
+              for (int c4 = 0; c4 < NV; ++c4)
+                st_cg_f4(accp + c4 * 128 + r,
+                         make_float4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]));
+            }
             if (threadIdx.x == 256) trace(it, 13);
             if constexpr (C::kPublisher) {
               // hand the publication of these stores to the publisher warp (slot k mod 2,

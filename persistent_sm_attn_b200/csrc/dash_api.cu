@@ -332,6 +332,42 @@ int check_shape(int B, int H, int S, int D) {
   return DASH_OK;
 }
 
+// The backward kernel of one launch: the deterministic path takes the red chain
+// variant when `red` is set.
+template <int D, bool kAtomic, bool kTrace>
+auto bwd_kernel_for(bool red) {
+  if constexpr (kAtomic)
+    return dash::dash_bwd_kernel<D, true, kTrace, false>;
+  else
+    return red ? dash::dash_bwd_kernel<D, false, kTrace, true>
+               : dash::dash_bwd_kernel<D, false, kTrace, false>;
+}
+
+// Whether a deterministic launch adds its chains' middle positions with red in L2
+// (bitwise the same results): measured faster on B200 for descending and naive
+// ascending from 64 tiles, slower or equal for the step-ordered schedules and for
+// short sequences.  dash_set_dq_chain_mode overrides it.
+std::atomic<int> g_chain_mode{0};  // 0 by schedule and length, 1 always red, 2 never
+bool red_chain_for(int sched, int N) {
+  const int m = g_chain_mode.load();
+  if (m == 1) return true;
+  if (m == 2) return false;
+  return (sched == DASH_SCHED_DESCENDING || sched == DASH_SCHED_NAIVE_ASC) && N >= 64;
+}
+
+// The kernel moves registers between warpgroups with setmaxnreg; the split adds up
+// to exactly kLaunchRegs per thread, so refuse any other allocation.
+template <int D, bool kAtomic, bool kTrace>
+int prepare_kernel(bool red) {
+  using C = BwdCfg<D>;
+  auto kern = bwd_kernel_for<D, kAtomic, kTrace>(red);
+  DASH_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes));
+  cudaFuncAttributes fa;
+  DASH_CUDA(cudaFuncGetAttributes(&fa, kern));
+  if (fa.numRegs != C::kLaunchRegs) return DASH_ERR_UNSUPPORTED;
+  return DASH_OK;
+}
+
 template <int D, bool kAtomic>
 int num_ctas_for(int dev, int* out) {
   using C = BwdCfg<D>;
@@ -341,13 +377,10 @@ int num_ctas_for(int dev, int* out) {
     *out = itn->second;
     return DASH_OK;
   }
-  auto kern = dash::dash_bwd_kernel<D, kAtomic>;
-  DASH_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes));
-  // The kernel moves registers between warpgroups with setmaxnreg; the split
-  // adds up to exactly kLaunchRegs per thread, so refuse any other allocation.
-  cudaFuncAttributes fa;
-  DASH_CUDA(cudaFuncGetAttributes(&fa, kern));
-  if (fa.numRegs != C::kLaunchRegs) return DASH_ERR_UNSUPPORTED;
+  int rc;
+  if ((rc = prepare_kernel<D, kAtomic, false>(false))) return rc;
+  if (!kAtomic && (rc = prepare_kernel<D, kAtomic, false>(true))) return rc;
+  auto kern = bwd_kernel_for<D, kAtomic, false>(false);
   int per_sm = 0, sms = 0;
   DASH_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, C::kThreads, C::kSmemBytes));
   DASH_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
@@ -475,16 +508,10 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (!prof_record(1, &ev, stream)) return DASH_ERR_CUDA;
-  if (kTrace) {
-    auto kt = dash::dash_bwd_kernel<D, kAtomic, true>;
-    DASH_CUDA(cudaFuncSetAttribute(kt, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes));
-    cudaFuncAttributes fa;
-    DASH_CUDA(cudaFuncGetAttributes(&fa, kt));
-    if (fa.numRegs != C::kLaunchRegs) return DASH_ERR_UNSUPPORTED;
-    DASH_CUDA(cudaLaunchKernelEx(&cfg, kt, tq, tk, tv, tdo, tc, p));
-  } else {
-    DASH_CUDA(cudaLaunchKernelEx(&cfg, dash::dash_bwd_kernel<D, kAtomic>, tq, tk, tv, tdo, tc, p));
-  }
+  const bool red = !kAtomic && red_chain_for(sched, N);
+  if (kTrace && (rc = prepare_kernel<D, kAtomic, true>(red))) return rc;
+  DASH_CUDA(cudaLaunchKernelEx(&cfg, bwd_kernel_for<D, kAtomic, kTrace>(red), tq, tk, tv, tdo,
+                               tc, p));
   if (!prof_record(2, &ev, stream)) return DASH_ERR_CUDA;
   if (kAtomic) {
     const long long n_blocks = (long long)B * H * N;  // 128-row accumulator blocks
@@ -696,6 +723,12 @@ int dash_inject_fault(int mode) {
 
 int dash_set_spin_limit_us(long long us) {
   g_spin_us.store(us > 0 ? us : 0);
+  return DASH_OK;
+}
+
+int dash_set_dq_chain_mode(int mode) {
+  if (mode < 0 || mode > 2) return DASH_ERR_INVALID_ARG;
+  g_chain_mode.store(mode);
   return DASH_OK;
 }
 
