@@ -185,6 +185,7 @@ def run_ours(args):
     o, lse = fwd_call(q, k, v, w.causal)
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
+    binding.dash_set_dq_chain_mode(args.dq_chain_mode)
 
     def barrier():
         if dist is not None:
@@ -319,6 +320,8 @@ def run_ours(args):
             "schedules_tflops": det,
             "det_nondet_ratio": (round(best_det / det["atomic"], 4)
                                  if atomic_ms and best_det else None),
+            "dq_chain": ("red" if binding.dash_dq_chain_uses_red(sched, w.S)
+                         else "load-add-store") if sched != "atomic" else None,
             "roofline": {"bound": "tensor", "achieved": round(kern, 2), "peak": peak,
                          "unit": "TFLOP/s", "frac": round(kern / peak, 4),
                          "traffic": _recorded_traffic(w.name, sched),
@@ -476,6 +479,9 @@ def main():
     ap.add_argument("--kv-heads", type=int, default=0,
                     help="time grouped-query attention with this many K/V heads (a side "
                          "measurement: no host-buffer e2e, simulator or CPU baseline)")
+    ap.add_argument("--dq-chain-mode", type=int, default=0, choices=(0, 1, 2),
+                    help="how the ordered dQ chains add a middle position: 0 the library's "
+                         "choice, 1 red in L2, 2 load-add-store (bitwise the same results)")
     ap.add_argument("--gqa-split", type=int, default=0,
                     help="with --kv-heads: sub-groups per K/V head (0 = the library's choice)")
     ap.add_argument("--heads", type=int, default=0,

@@ -164,6 +164,11 @@ int dash_set_spin_limit_us(long long us);
  * (dash_attn_bwd_noalloc always loads and stores).  Other modes: INVALID_ARG.
  */
 int dash_set_dq_chain_mode(int mode);
+/* Whether a deterministic backward of this schedule and length, launched now, adds
+ * with red (*red = 1) or loads, adds and stores (*red = 0); 0 for ATOMIC.  Host only.
+ * Errors: INVALID_ARG for a NULL red, a bad schedule or S not a positive multiple of
+ * 128. */
+int dash_dq_chain_uses_red(int schedule, int S, int* red);
 
 /*
  * Failure-detection testing.  mode 1: the next deterministic dash_attn_bwd or

@@ -26,7 +26,8 @@ EXPORTS = ("dash_attn_fwd", "dash_attn_bwd", "dash_attn_sync_status", "dash_stat
            "dash_trace_bwd", "dash_inject_fault", "dash_sched_check", "dash_attn_bwd_host",
            "dash_sched_table_part", "dash_attn_fwd_gqa", "dash_attn_bwd_gqa",
            "dash_sched_table_gqa", "dash_attn_noalloc_sync_status",
-           "dash_attn_bwd_gqa_split", "dash_bwd_gqa_split_for", "dash_set_dq_chain_mode")
+           "dash_attn_bwd_gqa_split", "dash_bwd_gqa_split_for", "dash_set_dq_chain_mode",
+           "dash_dq_chain_uses_red")
 
 
 class DashError(RuntimeError):
@@ -63,6 +64,7 @@ def load(path: str | None = None):
     lib.dash_attn_bwd_gqa_split.argtypes = [vp] * 9 + [i, i, i, i, i, i, i, i, vp]
     lib.dash_bwd_gqa_split_for.argtypes = [i, i, i, i, i, i, i, P(i)]
     lib.dash_set_dq_chain_mode.argtypes = [i]
+    lib.dash_dq_chain_uses_red.argtypes = [i, i, P(i)]
     lib.dash_attn_sync_status.argtypes = [vp]
     lib.dash_attn_noalloc_sync_status.argtypes = [vp]
     lib.dash_status_string.argtypes = [i]
@@ -87,8 +89,7 @@ def load(path: str | None = None):
     lib.dash_profile_end.argtypes = [P(d), P(d), P(ll)]
     for name in EXPORTS:
         if name not in ("dash_status_string", "dash_sched_table", "dash_sched_table_part",
-                        "dash_sched_table_gqa", "dash_attn_noalloc_sync_status",
-           "dash_attn_bwd_gqa_split", "dash_bwd_gqa_split_for", "dash_set_dq_chain_mode"):
+                        "dash_sched_table_gqa", "dash_attn_noalloc_sync_status"):
             getattr(lib, name).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -302,6 +303,15 @@ def dash_set_dq_chain_mode(mode: int) -> None:
     """0: the library picks per launch; 1: middle positions of the ordered dQ chains
     add with red in L2; 2: load-add-store on the SM (bitwise the same results)."""
     _check(load().dash_set_dq_chain_mode(int(mode)), "dash_set_dq_chain_mode")
+
+
+def dash_dq_chain_uses_red(schedule: str, S: int) -> bool:
+    """Whether a deterministic backward of this schedule and length adds its chains'
+    middle positions with red under the current mode (host only)."""
+    r = ctypes.c_int(0)
+    _check(load().dash_dq_chain_uses_red(_sched_id(schedule), S, ctypes.byref(r)),
+           "dash_dq_chain_uses_red")
+    return bool(r.value)
 
 
 def dash_release_workspace() -> None:

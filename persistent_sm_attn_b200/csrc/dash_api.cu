@@ -732,6 +732,14 @@ int dash_set_dq_chain_mode(int mode) {
   return DASH_OK;
 }
 
+int dash_dq_chain_uses_red(int schedule, int S, int* red) {
+  if (!red || S < 128 || S % 128 != 0 || schedule < DASH_SCHED_NAIVE_ASC ||
+      schedule > DASH_SCHED_ATOMIC)
+    return DASH_ERR_INVALID_ARG;
+  *red = (schedule != DASH_SCHED_ATOMIC && red_chain_for(schedule, S / 128)) ? 1 : 0;
+  return DASH_OK;
+}
+
 int dash_attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                       int H, int Hkv, int S, int D, int causal, void* stream) {
   return no_throw([&]() -> int {
