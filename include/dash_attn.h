@@ -171,6 +171,28 @@ int dash_set_dq_chain_mode(int mode);
 int dash_dq_chain_uses_red(int schedule, int S, int* red);
 
 /*
+ * Head interleaving of a multi-head backward's schedule table (DASH summary §2.1: the
+ * schedule fixes each dQ block's accumulation order, and the table fixes the schedule's
+ * placement on the SMs).  With 2 (or 4) heads per unit, each KV segment of a unit of the
+ * schedule runs for 2 (or 4) consecutive heads in turn, K/V loaded again for each; the
+ * heads' dQ blocks then receive their contributions further apart in the grid's steps.
+ * The order of every dQ block is still fixed by the table, so results stay bitwise
+ * reproducible, but they differ in rounding from the uninterleaved table.
+ * mode 0 (default): the library picks, 2 for SYM_SHIFT at D = 64 when the units still
+ * fill the grid's rounds (measured faster there), else 1; mode 1: never; mode 2 or 4:
+ * that many heads per unit whenever it divides B * H.  Applies to later dash_attn_bwd,
+ * dash_attn_bwd_host, dash_attn_bwd_noalloc and dash_trace_bwd calls (the grouped-query
+ * entry points have their own grouping).  Other modes: INVALID_ARG.
+ */
+int dash_set_head_interleave(int mode);
+/* Heads per unit a multi-head backward takes under the current mode for n_heads = B*H
+ * heads on num_ctas persistent CTAs.  Host only.  Errors: INVALID_ARG for a NULL
+ * output, num_ctas or n_heads below 1, D not 64/128, a bad schedule or causal flag, or
+ * S not a positive multiple of 128. */
+int dash_bwd_head_interleave(int num_ctas, int D, int schedule, int n_heads, int S, int causal,
+                             int* heads_per_unit);
+
+/*
  * Failure-detection testing.  mode 1: the next deterministic dash_attn_bwd or
  * dash_attn_bwd_noalloc (any stream) runs with a schedule table in which dQ
  * block (head 0, Q tile 0) never receives its first two partials, so its ticket

@@ -27,7 +27,8 @@ EXPORTS = ("dash_attn_fwd", "dash_attn_bwd", "dash_attn_sync_status", "dash_stat
            "dash_sched_table_part", "dash_attn_fwd_gqa", "dash_attn_bwd_gqa",
            "dash_sched_table_gqa", "dash_attn_noalloc_sync_status",
            "dash_attn_bwd_gqa_split", "dash_bwd_gqa_split_for", "dash_set_dq_chain_mode",
-           "dash_dq_chain_uses_red")
+           "dash_dq_chain_uses_red", "dash_set_head_interleave",
+           "dash_bwd_head_interleave")
 
 
 class DashError(RuntimeError):
@@ -65,6 +66,8 @@ def load(path: str | None = None):
     lib.dash_bwd_gqa_split_for.argtypes = [i, i, i, i, i, i, i, P(i)]
     lib.dash_set_dq_chain_mode.argtypes = [i]
     lib.dash_dq_chain_uses_red.argtypes = [i, i, P(i)]
+    lib.dash_set_head_interleave.argtypes = [i]
+    lib.dash_bwd_head_interleave.argtypes = [i, i, i, i, i, i, P(i)]
     lib.dash_attn_sync_status.argtypes = [vp]
     lib.dash_attn_noalloc_sync_status.argtypes = [vp]
     lib.dash_status_string.argtypes = [i]
@@ -312,6 +315,22 @@ def dash_dq_chain_uses_red(schedule: str, S: int) -> bool:
     _check(load().dash_dq_chain_uses_red(_sched_id(schedule), S, ctypes.byref(r)),
            "dash_dq_chain_uses_red")
     return bool(r.value)
+
+
+def dash_set_head_interleave(mode: int) -> None:
+    """Heads per unit of a multi-head backward's table: 0 the library's choice, 1 never
+    interleave, 2 or 4 that many whenever it divides B * H."""
+    _check(load().dash_set_head_interleave(int(mode)), "dash_set_head_interleave")
+
+
+def dash_bwd_head_interleave(num_ctas: int, D: int, schedule: str, n_heads: int, S: int,
+                             causal: bool) -> int:
+    """Heads per unit a multi-head backward takes under the current mode (host only)."""
+    r = ctypes.c_int(0)
+    _check(load().dash_bwd_head_interleave(num_ctas, D, _sched_id(schedule), n_heads, S,
+                                           int(bool(causal)), ctypes.byref(r)),
+           "dash_bwd_head_interleave")
+    return r.value
 
 
 def dash_release_workspace() -> None:

@@ -66,7 +66,8 @@ struct DevTable {
 
 std::mutex g_mu;
 std::map<std::pair<int, uintptr_t>, Workspace> g_ws;                  // (device, stream)
-std::map<std::tuple<int, int, int, int, int, int, int>, DevTable> g_tables;  // device,heads,N,causal,sched,ctas,group
+// device, heads, N, causal, sched, ctas, group, run_group
+std::map<std::tuple<int, int, int, int, int, int, int, int>, DevTable> g_tables;
 std::map<std::pair<int, int>, int> g_num_ctas;                        // (device, D)
 
 // Optional per-launch device timing: while enabled, each backward records four
@@ -142,11 +143,13 @@ void free_table(DevTable* d) {
 
 // The device copy of a table's chains: the pair count of each chain carries the
 // kernel's run flags (a run: consecutive chains of one CTA that feed one dK/dV tile,
-// which only grouped-query tables have).
-std::vector<dash::Chain> device_chains(const dash::Table& t) {
+// which only grouped-query tables have).  run_group: query heads that share a K/V
+// head (the table's group, or 1 for a multi-head table that interleaves heads).
+std::vector<dash::Chain> device_chains(const dash::Table& t, int run_group) {
   std::vector<dash::Chain> c = t.chains;
   auto same = [&](int a, int b) {
-    return t.chains[a].bh / t.group == t.chains[b].bh / t.group && t.chains[a].kv == t.chains[b].kv;
+    return t.chains[a].bh / run_group == t.chains[b].bh / run_group &&
+           t.chains[a].kv == t.chains[b].kv;
   };
   for (int k = 0; k < t.num_ctas; ++k)
     for (int i = t.cta_off[k]; i < t.cta_off[k + 1]; ++i) {
@@ -156,9 +159,9 @@ std::vector<dash::Chain> device_chains(const dash::Table& t) {
   return c;
 }
 
-int upload_table(const dash::Table& t, DevTable* out) {
+int upload_table(const dash::Table& t, DevTable* out, int run_group) {
   DevTable d;
-  const std::vector<dash::Chain> chains = device_chains(t);
+  const std::vector<dash::Chain> chains = device_chains(t, run_group);
   // an empty chain or pair list still gets a valid (unused) allocation
   const size_t nc = t.chains.empty() ? 1 : t.chains.size();
   const size_t np = t.pairs.empty() ? 1 : t.pairs.size();
@@ -184,9 +187,11 @@ int upload_table(const dash::Table& t, DevTable* out) {
   return DASH_OK;
 }
 
+// group: query heads per unit of the table; run_group: query heads per K/V head
+// (group for a grouped-query table, 1 for a multi-head table that interleaves heads)
 int get_table(int dev, int heads, int N, int causal, int sched, int ctas, DevTable** out,
-              int group = 1) {
-  auto key = std::make_tuple(dev, heads, N, causal, sched, ctas, group);
+              int group, int run_group) {
+  auto key = std::make_tuple(dev, heads, N, causal, sched, ctas, group, run_group);
   auto itb = g_tables.find(key);
   if (itb != g_tables.end()) {
     *out = &itb->second;
@@ -198,7 +203,7 @@ int get_table(int dev, int heads, int N, int causal, int sched, int ctas, DevTab
     return DASH_ERR_UNSUPPORTED;
   if (!dash::validate_table(t, &err)) return DASH_ERR_SCHEDULE;
   DevTable d;
-  int rc = upload_table(t, &d);
+  int rc = upload_table(t, &d, run_group);
   if (rc) return rc;
   auto res = g_tables.emplace(key, d);
   *out = &res.first->second;
@@ -207,11 +212,11 @@ int get_table(int dev, int heads, int N, int causal, int sched, int ctas, DevTab
 
 // Tables of the host-buffer path: the whole grid's table split into parts of
 // `chunk` heads (split_table keeps every dQ block's order), one per part.
-std::map<std::tuple<int, int, int, int, int, int, int>, std::vector<DevTable>> g_chunk_tables;
+std::map<std::tuple<int, int, int, int, int, int, int, int>, std::vector<DevTable>> g_chunk_tables;
 
 int get_chunk_tables(int dev, int heads, int N, int causal, int sched, int ctas, int chunk,
-                     std::vector<DevTable>** out) {
-  auto key = std::make_tuple(dev, heads, N, causal, sched, ctas, chunk);
+                     int il, std::vector<DevTable>** out) {
+  auto key = std::make_tuple(dev, heads, N, causal, sched, ctas, chunk, il);
   auto itc = g_chunk_tables.find(key);
   if (itc != g_chunk_tables.end()) {
     *out = &itc->second;
@@ -219,7 +224,8 @@ int get_chunk_tables(int dev, int heads, int N, int causal, int sched, int ctas,
   }
   dash::Table full;
   std::string err;
-  if (!dash::build_table(heads, N, causal, sched, ctas, &full, &err)) return DASH_ERR_UNSUPPORTED;
+  if (!dash::build_table_grouped(heads, il, N, causal, sched, ctas, &full, &err))
+    return DASH_ERR_UNSUPPORTED;
   if (!dash::validate_table(full, &err)) return DASH_ERR_SCHEDULE;
   std::vector<DevTable> parts;
   int rc = DASH_OK;
@@ -231,7 +237,7 @@ int get_chunk_tables(int dev, int heads, int N, int causal, int sched, int ctas,
       break;
     }
     DevTable d;
-    if ((rc = upload_table(t, &d)) == DASH_OK) parts.push_back(d);
+    if ((rc = upload_table(t, &d, 1)) == DASH_OK) parts.push_back(d);
   }
   if (rc) {
     for (DevTable& d : parts) free_table(&d);
@@ -246,10 +252,12 @@ int get_chunk_tables(int dev, int heads, int N, int causal, int sched, int ctas,
 // dQ block (head 0, Q tile 0) moves one position later, so its first position
 // is never filled and the waits on it must run out.  All indices stay in range.
 DevTable g_fault_table;
-int get_fault_table(int dev, int heads, int N, int causal, int sched, int ctas, DevTable** out) {
+int get_fault_table(int dev, int heads, int N, int causal, int sched, int ctas, int il,
+                    DevTable** out) {
   dash::Table t;
   std::string err;
-  if (!dash::build_table(heads, N, causal, sched, ctas, &t, &err)) return DASH_ERR_UNSUPPORTED;
+  if (!dash::build_table_grouped(heads, il, N, causal, sched, ctas, &t, &err))
+    return DASH_ERR_UNSUPPORTED;
   dash::plant_missing_first_partials(&t);
   cudaFree(g_fault_table.cta_off);
   cudaFree(g_fault_table.chains);
@@ -348,6 +356,7 @@ auto bwd_kernel_for(bool red) {
 // ascending from 64 tiles, slower or equal for the step-ordered schedules and for
 // short sequences.  dash_set_dq_chain_mode overrides it.
 std::atomic<int> g_chain_mode{0};  // 0 by schedule and length, 1 always red, 2 never
+std::atomic<int> g_il_mode{0};     // dash_set_head_interleave: 0 the library's choice
 bool red_chain_for(int sched, int N) {
   const int m = g_chain_mode.load();
   if (m == 1) return true;
@@ -433,6 +442,12 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
     split = group > 1 ? choose_split((long long)B * (H / group), group,
                                      (long long)dash::head_units(sched, N, causal).size(), ctas)
                       : 1;
+  // the table's query heads per unit, and per K/V head (a multi-head launch may
+  // interleave heads in its units; each head keeps its own K/V)
+  const int tgroup = group > 1 ? group / split
+                               : dash::head_interleave(D, sched, B * H, N, causal, ctas,
+                                                       g_il_mode.load());
+  const int rgroup = group > 1 ? group / split : 1;
   // a split group runs as group / split query heads per (virtual) K/V head in the table;
   // the kernel still reads K/V of head / group
   const long long dqn = dash::dq_units<D>((long long)B * H * N);
@@ -446,8 +461,8 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
     if (tab_override) {
       tab = const_cast<DevTable*>(tab_override);
     } else if (fault == 1 && !kAtomic) {
-      if ((rc = get_fault_table(dev, B * H, N, causal, sched, ctas, &tab))) return rc;
-    } else if ((rc = get_table(dev, B * H, N, causal, sched, ctas, &tab, group / split))) {
+      if ((rc = get_fault_table(dev, B * H, N, causal, sched, ctas, tgroup, &tab))) return rc;
+    } else if ((rc = get_table(dev, B * H, N, causal, sched, ctas, &tab, tgroup, rgroup))) {
       return rc;
     }
     if ((rc = get_workspace(dev, stream, 2 * (size_t)rows * D * sizeof(float),
@@ -627,10 +642,13 @@ int host_bwd(const void* q, const void* k, const void* v, const void* o, const v
              const float* lse, void* dq, void* dk, void* dv, int B, int H, int S, int causal,
              int sched, cudaStream_t stream, int dev) {
   const int BH = B * H, N = S / 128;
-  const int chunk = (BH + kHostParts - 1) / kHostParts;
   int ctas = 0;
   int rc = num_ctas_for<D, kAtomic>(dev, &ctas);
   if (rc) return rc;
+  // the parts hold whole units of the launch's table, so its interleaved heads stay
+  // together and every dQ block keeps the order dash_attn_bwd gives it
+  const int il = dash::head_interleave(D, sched, BH, N, causal, ctas, g_il_mode.load());
+  const int chunk = ((BH + kHostParts - 1) / kHostParts + il - 1) / il * il;
   const size_t rows_c = (size_t)chunk * S;
   const size_t tile = align256(rows_c * D * 2), lse_b = align256(rows_c * 4);
   const size_t slot_bytes = 8 * tile + lse_b;  // q k v o dO, LSE; dQ dK dV
@@ -638,7 +656,7 @@ int host_bwd(const void* q, const void* k, const void* v, const void* o, const v
   HostPipe* hp = nullptr;
   {
     std::lock_guard<std::mutex> lk(g_mu);
-    if ((rc = get_chunk_tables(dev, BH, N, causal, sched, ctas, chunk, &parts))) return rc;
+    if ((rc = get_chunk_tables(dev, BH, N, causal, sched, ctas, chunk, il, &parts))) return rc;
     if ((rc = get_pipe(dev, stream, 2 * slot_bytes, &hp))) return rc;
   }
   // the copy streams start after whatever the caller queued before this call
@@ -695,6 +713,7 @@ namespace dash {
 
 long long spin_limit_us() { return spin_us(); }
 int take_armed_fault() { return g_fault.exchange(0); }
+int head_interleave_mode() { return g_il_mode.load(); }
 
 }  // namespace dash
 
@@ -723,6 +742,23 @@ int dash_inject_fault(int mode) {
 
 int dash_set_spin_limit_us(long long us) {
   g_spin_us.store(us > 0 ? us : 0);
+  return DASH_OK;
+}
+
+int dash_set_head_interleave(int mode) {
+  if (mode != 0 && mode != 1 && mode != 2 && mode != 4) return DASH_ERR_INVALID_ARG;
+  g_il_mode.store(mode);
+  return DASH_OK;
+}
+
+int dash_bwd_head_interleave(int num_ctas, int D, int schedule, int n_heads, int S, int causal,
+                             int* heads_per_unit) {
+  if (!heads_per_unit || num_ctas < 1 || n_heads < 1 || (D != 64 && D != 128) || S < 128 ||
+      S % 128 != 0 || schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_ATOMIC ||
+      (causal != 0 && causal != 1))
+    return DASH_ERR_INVALID_ARG;
+  *heads_per_unit =
+      dash::head_interleave(D, schedule, n_heads, S / 128, causal, num_ctas, g_il_mode.load());
   return DASH_OK;
 }
 
@@ -1000,7 +1036,9 @@ int dash_trace_bwd(const void* q, const void* k, const void* v, const void* o, c
     if (rc) return rc;
     dash::Table t;
     std::string err;
-    if (!dash::build_table(B * H, S / 128, causal, schedule, ctas, &t, &err))
+    const int il = dash::head_interleave(D, schedule, B * H, S / 128, causal, ctas,
+                                         g_il_mode.load());
+    if (!dash::build_table_grouped(B * H, il, S / 128, causal, schedule, ctas, &t, &err))
       return DASH_ERR_UNSUPPORTED;
     int rows = 0;
     for (int c = 0; c < ctas; ++c) {

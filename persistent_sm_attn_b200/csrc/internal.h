@@ -12,6 +12,9 @@ long long spin_limit_us();
 // The fault armed with dash_inject_fault (0: none), disarmed by this call.
 int take_armed_fault();
 
+// The mode set with dash_set_head_interleave (0: the library's choice).
+int head_interleave_mode();
+
 // C++ exceptions (std::bad_alloc from a table, a map or a vector sized by the
 // caller's arguments) must not cross the C ABI: each entry point that
 // allocates on the host returns a status instead.

@@ -38,7 +38,7 @@ struct DeviceState {
   unsigned char* base = nullptr;  // device address of g_noalloc_scratch on this device
   int ctas[2][2] = {{0, 0}, {0, 0}};  // [D==128][atomic]
   // key of the schedule table currently held in the scratch array
-  long long table_key[6] = {-1, -1, -1, -1, -1, -1};
+  long long table_key[7] = {-1, -1, -1, -1, -1, -1, -1};
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_noalloc_mu;
@@ -165,11 +165,16 @@ int noalloc_launch(const void* q, const void* k, const void* v, const void* o, c
   // the schedule table, built and checked on the host, then copied in.  A fault armed
   // with dash_inject_fault replaces it, for this call only, by a table whose dQ block
   // (head 0, Q tile 0) never receives its first partials.
-  const long long key[6] = {B * (long long)H, N, causal, sched, ctas, (long long)off};
+  // the allocating entry point's table (heads interleaved the same way), so the two
+  // add every dQ block in the same order
+  const int il =
+      dash::head_interleave(D, sched, B * H, N, causal, ctas, dash::head_interleave_mode());
+  const long long key[7] = {B * (long long)H, N, causal, sched, ctas, (long long)off, il};
   const int fault = kAtomic ? 0 : dash::take_armed_fault();
   dash::Table t;
   std::string msg;
-  if (!dash::build_table(B * H, N, causal, sched, ctas, &t, &msg)) return DASH_ERR_UNSUPPORTED;
+  if (!dash::build_table_grouped(B * H, il, N, causal, sched, ctas, &t, &msg))
+    return DASH_ERR_UNSUPPORTED;
   if (fault == 1) dash::plant_missing_first_partials(&t);
   const size_t off_cta = off;
   const size_t off_chain = off_cta + align256(t.cta_off.size() * sizeof(int));

@@ -98,6 +98,21 @@ bool build_table(int n_heads, int N, int causal, int schedule, int num_ctas, Tab
   return build_table_grouped(n_heads, 1, N, causal, schedule, num_ctas, out, err);
 }
 
+int head_interleave(int D, int schedule, int n_heads, int N, int causal, int num_ctas, int mode) {
+  if (n_heads < 1 || num_ctas < 1 || N < 1) return 1;
+  if (mode == 2 || mode == 4) return n_heads % mode == 0 ? mode : 1;
+  if (mode != 0 || D != 64 || schedule != SYM_SHIFT || n_heads % 2 != 0 ||
+      !schedule_supported(schedule, N, causal))
+    return 1;
+  const long long per_head = (long long)units_of(schedule, N, causal).size();
+  auto fill = [&](int il) {
+    const long long u = (long long)(n_heads / il) * per_head;
+    const long long rounds = (u + num_ctas - 1) / num_ctas;
+    return (double)u / (double)(rounds * num_ctas);
+  };
+  return fill(2) >= fill(1) - 0.02 ? 2 : 1;
+}
+
 bool build_table_grouped(int n_heads, int group, int N, int causal, int schedule,
                          int num_ctas, Table* out, std::string* err) {
   if (n_heads < 1 || num_ctas < 1 || num_ctas > kMaxTableCtas || group < 1 ||

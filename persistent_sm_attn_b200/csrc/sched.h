@@ -47,6 +47,15 @@ bool schedule_supported(int schedule, int N, int causal);
 // Units of one head: each a list of (kv, q) in visiting order.
 std::vector<std::vector<std::pair<int, int>>> head_units(int schedule, int N, int causal);
 
+// Query heads per unit of a multi-head launch's table.  With il > 1 the launch uses
+// build_table_grouped(n_heads, il, ...) although every head has K/V of its own: each KV
+// segment of a unit runs for il heads in turn (K/V loaded again for each), which
+// spaces successive contributions to a dQ block further apart in the persistent
+// grid's steps.  mode 0: the measured choice (2 for symmetric shift at D = 64 when
+// the units still fill the grid's rounds within 2 points, else 1); mode 1: 1; mode 2
+// or 4: that many where it divides n_heads, else 1.
+int head_interleave(int D, int schedule, int n_heads, int N, int causal, int num_ctas, int mode);
+
 // Build the whole-grid table: heads in order, unit g on CTA g mod num_ctas in
 // round g / num_ctas; step-ordered schedules accumulate each dQ block in
 // (round, step) order.
