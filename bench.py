@@ -186,6 +186,7 @@ def run_ours(args):
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
     binding.dash_set_dq_chain_mode(args.dq_chain_mode)
+    binding.dash_set_head_interleave(args.head_interleave)
 
     def barrier():
         if dist is not None:
@@ -301,6 +302,9 @@ def run_ours(args):
         atomic_ms = results.get("atomic")
         det = {s: round(tflops(m), 2) for s, m in results.items()}
         best_det = max((v_ for s, v_ in det.items() if s != "atomic"), default=None)
+        il = (binding.dash_bwd_head_interleave(binding.dash_bwd_num_ctas(local, w.D), w.D,
+                                               sched, w.B * w.H, w.S, w.causal)
+              if not gqa else 1)
         line = {
             "metric": METRIC,
             "value": round(value, 2),
@@ -320,8 +324,9 @@ def run_ours(args):
             "schedules_tflops": det,
             "det_nondet_ratio": (round(best_det / det["atomic"], 4)
                                  if atomic_ms and best_det else None),
-            "dq_chain": ("red" if binding.dash_dq_chain_uses_red(sched, w.S)
+            "dq_chain": ("red" if binding.dash_dq_chain_uses_red(sched, w.S, il)
                          else "load-add-store") if sched != "atomic" else None,
+            "heads_per_unit": il if not gqa else None,
             "roofline": {"bound": "tensor", "achieved": round(kern, 2), "peak": peak,
                          "unit": "TFLOP/s", "frac": round(kern / peak, 4),
                          "traffic": _recorded_traffic(w.name, sched),
@@ -482,6 +487,9 @@ def main():
     ap.add_argument("--dq-chain-mode", type=int, default=0, choices=(0, 1, 2),
                     help="how the ordered dQ chains add a middle position: 0 the library's "
                          "choice, 1 red in L2, 2 load-add-store (bitwise the same results)")
+    ap.add_argument("--head-interleave", type=int, default=0, choices=(0, 1, 2, 4),
+                    help="heads per unit of the multi-head table: 0 the library's choice, "
+                         "1 none, 2 or 4 forced")
     ap.add_argument("--gqa-split", type=int, default=0,
                     help="with --kv-heads: sub-groups per K/V head (0 = the library's choice)")
     ap.add_argument("--heads", type=int, default=0,

@@ -62,6 +62,7 @@ struct DevTable {
   int* cta_off = nullptr;
   int4* chains = nullptr;
   uint32_t* pairs = nullptr;
+  int group = 1;  // query heads per unit of the table it came from
 };
 
 std::mutex g_mu;
@@ -161,6 +162,7 @@ std::vector<dash::Chain> device_chains(const dash::Table& t, int run_group) {
 
 int upload_table(const dash::Table& t, DevTable* out, int run_group) {
   DevTable d;
+  d.group = t.group;
   const std::vector<dash::Chain> chains = device_chains(t, run_group);
   // an empty chain or pair list still gets a valid (unused) allocation
   const size_t nc = t.chains.empty() ? 1 : t.chains.size();
@@ -352,16 +354,19 @@ auto bwd_kernel_for(bool red) {
 }
 
 // Whether a deterministic launch adds its chains' middle positions with red in L2
-// (bitwise the same results): measured faster on B200 for descending and naive
-// ascending from 64 tiles, slower or equal for the step-ordered schedules and for
-// short sequences.  dash_set_dq_chain_mode overrides it.
-std::atomic<int> g_chain_mode{0};  // 0 by schedule and length, 1 always red, 2 never
+// (bitwise the same results): measured faster on B200 where consecutive positions of
+// a block have slack between them, i.e. descending and naive ascending from 64 tiles,
+// and tables that interleave heads (il > 1); slower or equal for the step-ordered
+// schedules with one head per unit and for short sequences.  dash_set_dq_chain_mode
+// overrides it.
+std::atomic<int> g_chain_mode{0};  // 0 by schedule, length and interleave, 1 red, 2 never
 std::atomic<int> g_il_mode{0};     // dash_set_head_interleave: 0 the library's choice
-bool red_chain_for(int sched, int N) {
+bool red_chain_for(int sched, int N, int il) {
   const int m = g_chain_mode.load();
   if (m == 1) return true;
   if (m == 2) return false;
-  return (sched == DASH_SCHED_DESCENDING || sched == DASH_SCHED_NAIVE_ASC) && N >= 64;
+  return ((sched == DASH_SCHED_DESCENDING || sched == DASH_SCHED_NAIVE_ASC) && N >= 64) ||
+         il > 1;
 }
 
 // The kernel moves registers between warpgroups with setmaxnreg; the split adds up
@@ -523,7 +528,9 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (!prof_record(1, &ev, stream)) return DASH_ERR_CUDA;
-  const bool red = !kAtomic && red_chain_for(sched, N);
+  // a multi-head table's interleave (the host-buffer path passes the parts of one)
+  const int il = group > 1 ? 1 : (tab_override ? tab_override->group : tgroup);
+  const bool red = !kAtomic && red_chain_for(sched, N, il);
   if (kTrace && (rc = prepare_kernel<D, kAtomic, true>(red))) return rc;
   DASH_CUDA(cudaLaunchKernelEx(&cfg, bwd_kernel_for<D, kAtomic, kTrace>(red), tq, tk, tv, tdo,
                                tc, p));
@@ -768,11 +775,12 @@ int dash_set_dq_chain_mode(int mode) {
   return DASH_OK;
 }
 
-int dash_dq_chain_uses_red(int schedule, int S, int* red) {
+int dash_dq_chain_uses_red(int schedule, int S, int heads_per_unit, int* red) {
   if (!red || S < 128 || S % 128 != 0 || schedule < DASH_SCHED_NAIVE_ASC ||
-      schedule > DASH_SCHED_ATOMIC)
+      schedule > DASH_SCHED_ATOMIC || heads_per_unit < 1)
     return DASH_ERR_INVALID_ARG;
-  *red = (schedule != DASH_SCHED_ATOMIC && red_chain_for(schedule, S / 128)) ? 1 : 0;
+  *red = (schedule != DASH_SCHED_ATOMIC && red_chain_for(schedule, S / 128, heads_per_unit))
+             ? 1 : 0;
   return DASH_OK;
 }
 

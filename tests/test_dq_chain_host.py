@@ -13,6 +13,9 @@ def test_default_choice():
     assert not f("descending", 63 * 128) and not f("naive_asc", 4096)
     assert not f("shift", 16384) and not f("sym_shift", 16384)
     assert not f("atomic", 16384)
+    # tables that interleave heads take red on every deterministic schedule
+    assert f("sym_shift", 16384, 2) and f("shift", 1024, 4) and f("descending", 512, 2)
+    assert not f("atomic", 16384, 2)
 
 
 def test_forced_modes():
@@ -31,6 +34,7 @@ def test_argument_errors():
     for bad in (lambda: binding.dash_set_dq_chain_mode(3),
                 lambda: binding.dash_set_dq_chain_mode(-1),
                 lambda: binding.dash_dq_chain_uses_red("descending", 100),
-                lambda: binding.dash_dq_chain_uses_red("descending", 0)):
+                lambda: binding.dash_dq_chain_uses_red("descending", 0),
+                lambda: binding.dash_dq_chain_uses_red("descending", 1024, 0)):
         with pytest.raises(binding.DashError):
             bad()
