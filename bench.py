@@ -304,7 +304,7 @@ def run_ours(args):
         best_det = max((v_ for s, v_ in det.items() if s != "atomic"), default=None)
         il = (binding.dash_bwd_head_interleave(binding.dash_bwd_num_ctas(local, w.D), w.D,
                                                sched, w.B * w.H, w.S, w.causal)
-              if not gqa else 1)
+              if not gqa else (w.H // args.kv_heads) // split)
         line = {
             "metric": METRIC,
             "value": round(value, 2),
@@ -324,7 +324,7 @@ def run_ours(args):
             "schedules_tflops": det,
             "det_nondet_ratio": (round(best_det / det["atomic"], 4)
                                  if atomic_ms and best_det else None),
-            "dq_chain": ("red" if binding.dash_dq_chain_uses_red(sched, w.S, il)
+            "dq_chain": ("red" if binding.dash_dq_chain_uses_red(sched, w.S, w.D, il)
                          else "load-add-store") if sched != "atomic" else None,
             "heads_per_unit": il if not gqa else None,
             "roofline": {"bound": "tensor", "achieved": round(kern, 2), "peak": peak,

@@ -159,18 +159,20 @@ int dash_set_spin_limit_us(long long us);
  * per launch, 1 always adds in L2 with red once the ticket grants the position, 2
  * always loads, adds on the SM and stores.  The additions and their order are the
  * same, so the results are bitwise the same; mode 0 takes red where it measured faster:
- * the descending and naive ascending schedules from 64 tiles, and multi-head launches
- * whose table interleaves heads (dash_set_head_interleave).  Applies to later
+ * the descending and naive ascending schedules from 64 tiles, and at D = 64 tables that
+ * run two or more query heads per unit (multi-head tables that interleave heads,
+ * dash_set_head_interleave; grouped-query sub-groups of two or more heads).  Applies to later
  * dash_attn_bwd / dash_attn_bwd_gqa / dash_attn_bwd_host calls on every stream
  * (dash_attn_bwd_noalloc always loads and stores).  Other modes: INVALID_ARG.
  */
 int dash_set_dq_chain_mode(int mode);
-/* Whether a deterministic backward of this schedule and length, launched now with
- * heads_per_unit heads per unit of its table (dash_bwd_head_interleave; 1 for the
- * grouped-query entry points), adds with red (*red = 1) or loads, adds and stores
- * (*red = 0); 0 for ATOMIC.  Host only.  Errors: INVALID_ARG for a NULL red, a bad
- * schedule, heads_per_unit below 1 or S not a positive multiple of 128. */
-int dash_dq_chain_uses_red(int schedule, int S, int heads_per_unit, int* red);
+/* Whether a deterministic backward of this schedule, length and head dim, launched
+ * now with heads_per_unit query heads per unit of its table (dash_bwd_head_interleave
+ * for the multi-head entry points; group / split for the grouped-query ones), adds with
+ * red (*red = 1) or loads, adds and stores (*red = 0); 0 for ATOMIC.  Host only.
+ * Errors: INVALID_ARG for a NULL red, a bad schedule, D not 64/128, heads_per_unit below
+ * 1 or S not a positive multiple of 128. */
+int dash_dq_chain_uses_red(int schedule, int S, int D, int heads_per_unit, int* red);
 
 /*
  * Head interleaving of a multi-head backward's schedule table (DASH summary §2.1: the

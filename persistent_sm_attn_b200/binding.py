@@ -65,7 +65,7 @@ def load(path: str | None = None):
     lib.dash_attn_bwd_gqa_split.argtypes = [vp] * 9 + [i, i, i, i, i, i, i, i, vp]
     lib.dash_bwd_gqa_split_for.argtypes = [i, i, i, i, i, i, i, P(i)]
     lib.dash_set_dq_chain_mode.argtypes = [i]
-    lib.dash_dq_chain_uses_red.argtypes = [i, i, i, P(i)]
+    lib.dash_dq_chain_uses_red.argtypes = [i, i, i, i, P(i)]
     lib.dash_set_head_interleave.argtypes = [i]
     lib.dash_bwd_head_interleave.argtypes = [i, i, i, i, i, i, P(i)]
     lib.dash_attn_sync_status.argtypes = [vp]
@@ -308,12 +308,12 @@ def dash_set_dq_chain_mode(mode: int) -> None:
     _check(load().dash_set_dq_chain_mode(int(mode)), "dash_set_dq_chain_mode")
 
 
-def dash_dq_chain_uses_red(schedule: str, S: int, heads_per_unit: int = 1) -> bool:
-    """Whether a deterministic backward of this schedule and length, with this many heads
-    per unit of its table, adds its chains' middle positions with red under the current
-    mode (host only)."""
+def dash_dq_chain_uses_red(schedule: str, S: int, D: int = 128, heads_per_unit: int = 1) -> bool:
+    """Whether a deterministic backward of this schedule, length and head dim, with this
+    many query heads per unit of its table, adds its chains' middle positions with red
+    under the current mode (host only)."""
     r = ctypes.c_int(0)
-    _check(load().dash_dq_chain_uses_red(_sched_id(schedule), S, int(heads_per_unit),
+    _check(load().dash_dq_chain_uses_red(_sched_id(schedule), S, int(D), int(heads_per_unit),
                                          ctypes.byref(r)),
            "dash_dq_chain_uses_red")
     return bool(r.value)

@@ -356,17 +356,17 @@ auto bwd_kernel_for(bool red) {
 // Whether a deterministic launch adds its chains' middle positions with red in L2
 // (bitwise the same results): measured faster on B200 where consecutive positions of
 // a block have slack between them, i.e. descending and naive ascending from 64 tiles,
-// and tables that interleave heads (il > 1); slower or equal for the step-ordered
-// schedules with one head per unit and for short sequences.  dash_set_dq_chain_mode
-// overrides it.
-std::atomic<int> g_chain_mode{0};  // 0 by schedule, length and interleave, 1 red, 2 never
+// and at D = 64 tables that run two or more query heads per unit (interleaved
+// multi-head tables, grouped-query sub-groups); slower or equal for the step-ordered
+// schedules otherwise and for short sequences.  dash_set_dq_chain_mode overrides it.
+std::atomic<int> g_chain_mode{0};  // 0 by schedule, length, head dim and heads per unit
 std::atomic<int> g_il_mode{0};     // dash_set_head_interleave: 0 the library's choice
-bool red_chain_for(int sched, int N, int il) {
+bool red_chain_for(int sched, int N, int D, int heads_per_unit) {
   const int m = g_chain_mode.load();
   if (m == 1) return true;
   if (m == 2) return false;
   return ((sched == DASH_SCHED_DESCENDING || sched == DASH_SCHED_NAIVE_ASC) && N >= 64) ||
-         il > 1;
+         (D == 64 && heads_per_unit > 1);
 }
 
 // The kernel moves registers between warpgroups with setmaxnreg; the split adds up
@@ -528,9 +528,9 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (!prof_record(1, &ev, stream)) return DASH_ERR_CUDA;
-  // a multi-head table's interleave (the host-buffer path passes the parts of one)
-  const int il = group > 1 ? 1 : (tab_override ? tab_override->group : tgroup);
-  const bool red = !kAtomic && red_chain_for(sched, N, il);
+  // query heads per unit of the table (the host-buffer path passes the parts of one)
+  const int hpu = tab_override ? tab_override->group : tgroup;
+  const bool red = !kAtomic && red_chain_for(sched, N, D, hpu);
   if (kTrace && (rc = prepare_kernel<D, kAtomic, true>(red))) return rc;
   DASH_CUDA(cudaLaunchKernelEx(&cfg, bwd_kernel_for<D, kAtomic, kTrace>(red), tq, tk, tv, tdo,
                                tc, p));
@@ -775,11 +775,11 @@ int dash_set_dq_chain_mode(int mode) {
   return DASH_OK;
 }
 
-int dash_dq_chain_uses_red(int schedule, int S, int heads_per_unit, int* red) {
+int dash_dq_chain_uses_red(int schedule, int S, int D, int heads_per_unit, int* red) {
   if (!red || S < 128 || S % 128 != 0 || schedule < DASH_SCHED_NAIVE_ASC ||
-      schedule > DASH_SCHED_ATOMIC || heads_per_unit < 1)
+      schedule > DASH_SCHED_ATOMIC || heads_per_unit < 1 || (D != 64 && D != 128))
     return DASH_ERR_INVALID_ARG;
-  *red = (schedule != DASH_SCHED_ATOMIC && red_chain_for(schedule, S / 128, heads_per_unit))
+  *red = (schedule != DASH_SCHED_ATOMIC && red_chain_for(schedule, S / 128, D, heads_per_unit))
              ? 1 : 0;
   return DASH_OK;
 }

@@ -13,9 +13,11 @@ def test_default_choice():
     assert not f("descending", 63 * 128) and not f("naive_asc", 4096)
     assert not f("shift", 16384) and not f("sym_shift", 16384)
     assert not f("atomic", 16384)
-    # tables that interleave heads take red on every deterministic schedule
-    assert f("sym_shift", 16384, 2) and f("shift", 1024, 4) and f("descending", 512, 2)
-    assert not f("atomic", 16384, 2)
+    # at D=64, tables with two or more query heads per unit take red on every
+    # deterministic schedule; at D=128 they do not
+    assert f("sym_shift", 16384, 64, 2) and f("shift", 1024, 64, 4) and f("descending", 512, 64, 2)
+    assert not f("sym_shift", 16384, 128, 2) and not f("sym_shift", 16384, 64, 1)
+    assert not f("atomic", 16384, 64, 2)
 
 
 def test_forced_modes():
@@ -35,6 +37,7 @@ def test_argument_errors():
                 lambda: binding.dash_set_dq_chain_mode(-1),
                 lambda: binding.dash_dq_chain_uses_red("descending", 100),
                 lambda: binding.dash_dq_chain_uses_red("descending", 0),
-                lambda: binding.dash_dq_chain_uses_red("descending", 1024, 0)):
+                lambda: binding.dash_dq_chain_uses_red("descending", 1024, 64, 0),
+                lambda: binding.dash_dq_chain_uses_red("descending", 1024, 96, 1)):
         with pytest.raises(binding.DashError):
             bad()
