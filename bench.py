@@ -187,6 +187,7 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
     binding.dash_set_dq_chain_mode(args.dq_chain_mode)
     binding.dash_set_head_interleave(args.head_interleave)
+    binding.dash_set_slot_placement(args.slot_placement)
 
     def barrier():
         if dist is not None:
@@ -327,6 +328,8 @@ def run_ours(args):
             "dq_chain": ("red" if binding.dash_dq_chain_uses_red(sched, w.S, w.D, il)
                          else "load-add-store") if sched != "atomic" else None,
             "heads_per_unit": il if not gqa else None,
+            "slot_placement": ("sm_id" if binding.dash_slot_placement_by_smid(w.S)
+                               else "launch_order"),
             "roofline": {"bound": "tensor", "achieved": round(kern, 2), "peak": peak,
                          "unit": "TFLOP/s", "frac": round(kern / peak, 4),
                          "traffic": _recorded_traffic(w.name, sched),
@@ -487,6 +490,9 @@ def main():
     ap.add_argument("--dq-chain-mode", type=int, default=0, choices=(0, 1, 2),
                     help="how the ordered dQ chains add a middle position: 0 the library's "
                          "choice, 1 red in L2, 2 load-add-store (bitwise the same results)")
+    ap.add_argument("--slot-placement", type=int, default=0, choices=(0, 1, 2),
+                    help="table slots on the SMs: 0 the library's choice, 1 by SM id, "
+                         "2 launch order (bitwise the same results)")
     ap.add_argument("--head-interleave", type=int, default=0, choices=(0, 1, 2, 4),
                     help="heads per unit of the multi-head table: 0 the library's choice, "
                          "1 none, 2 or 4 forced")

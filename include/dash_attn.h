@@ -175,6 +175,24 @@ int dash_set_dq_chain_mode(int mode);
 int dash_dq_chain_uses_red(int schedule, int S, int D, int heads_per_unit, int* red);
 
 /*
+ * Placement of the schedule table's CTA slots on the SMs (the die-aware placement the
+ * DASH summary §4 motivates: at 16k with a full mask, shift slows down through remote
+ * L2 segments).  By SM id: each CTA reads its SM id at start and runs the slot equal
+ * to that id's rank in the grid, so a head's consecutive units run on SMs with
+ * consecutive ids.  In launch order: the grid's CTA b runs slot b.  mode 0 (default):
+ * by SM id from 128 tiles (S >= 16384), where it measured faster, else in launch
+ * order; mode 1: always by SM id; mode 2: always in launch order.  The table fixes
+ * every order, so results are bitwise the same in every mode.  Applies to later
+ * dash_attn_bwd, dash_attn_bwd_gqa, dash_attn_bwd_host and dash_trace_bwd calls
+ * (dash_attn_bwd_noalloc keeps mode 0).  Other modes: INVALID_ARG.
+ */
+int dash_set_slot_placement(int mode);
+/* Whether a backward of length S, launched now, places slots by SM id (*by_smid = 1)
+ * or in launch order (0).  Host only.  Errors: INVALID_ARG for a NULL output or S not
+ * a positive multiple of 128. */
+int dash_slot_placement_by_smid(int S, int* by_smid);
+
+/*
  * Head interleaving of a multi-head backward's schedule table (DASH summary §2.1: the
  * schedule fixes each dQ block's accumulation order, and the table fixes the schedule's
  * placement on the SMs).  With 2 (or 4) heads per unit, each KV segment of a unit of the

@@ -28,7 +28,8 @@ EXPORTS = ("dash_attn_fwd", "dash_attn_bwd", "dash_attn_sync_status", "dash_stat
            "dash_sched_table_gqa", "dash_attn_noalloc_sync_status",
            "dash_attn_bwd_gqa_split", "dash_bwd_gqa_split_for", "dash_set_dq_chain_mode",
            "dash_dq_chain_uses_red", "dash_set_head_interleave",
-           "dash_bwd_head_interleave")
+           "dash_bwd_head_interleave", "dash_set_slot_placement",
+           "dash_slot_placement_by_smid")
 
 
 class DashError(RuntimeError):
@@ -67,6 +68,8 @@ def load(path: str | None = None):
     lib.dash_set_dq_chain_mode.argtypes = [i]
     lib.dash_dq_chain_uses_red.argtypes = [i, i, i, i, P(i)]
     lib.dash_set_head_interleave.argtypes = [i]
+    lib.dash_set_slot_placement.argtypes = [i]
+    lib.dash_slot_placement_by_smid.argtypes = [i, P(i)]
     lib.dash_bwd_head_interleave.argtypes = [i, i, i, i, i, i, P(i)]
     lib.dash_attn_sync_status.argtypes = [vp]
     lib.dash_attn_noalloc_sync_status.argtypes = [vp]
@@ -316,6 +319,21 @@ def dash_dq_chain_uses_red(schedule: str, S: int, D: int = 128, heads_per_unit: 
     _check(load().dash_dq_chain_uses_red(_sched_id(schedule), S, int(D), int(heads_per_unit),
                                          ctypes.byref(r)),
            "dash_dq_chain_uses_red")
+    return bool(r.value)
+
+
+def dash_set_slot_placement(mode: int) -> None:
+    """1: each CTA runs the table slot of its SM id's rank; 2: CTA b runs slot b; 0:
+    the library's choice (by SM id from 128 tiles).  Bitwise the same results."""
+    _check(load().dash_set_slot_placement(int(mode)), "dash_set_slot_placement")
+
+
+def dash_slot_placement_by_smid(S: int) -> bool:
+    """Whether a backward of length S places the table's slots by SM id under the
+    current mode (host only)."""
+    r = ctypes.c_int(0)
+    _check(load().dash_slot_placement_by_smid(int(S), ctypes.byref(r)),
+           "dash_slot_placement_by_smid")
     return bool(r.value)
 
 

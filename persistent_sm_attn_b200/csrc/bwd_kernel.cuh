@@ -97,6 +97,13 @@ struct BwdParams {
   uint32_t* dkv_tickets = nullptr;
   float scale, scale_log2;
   unsigned long long spin_ns;
+  // Placement of the table's slots on the SMs.  nullptr: CTA b runs slot b.  Else CTA
+  // b runs the slot equal to the rank of its SM id among the grid's (slot_smid holds
+  // gridDim.x ints, slot_arrive a counter that starts at 0), so consecutive slots, which
+  // hold a head's consecutive units, run on SMs with consecutive ids.  Which CTA runs a
+  // slot changes no result: the table fixes every order.
+  int* slot_smid = nullptr;
+  uint32_t* slot_arrive = nullptr;
   // Optional %globaltimer trace (kernels instantiated with kTrace only):
   // trace[(cta * trace_rows + pair) * 8 + event], events listed at kTrace.
   unsigned long long* trace = nullptr;
@@ -246,7 +253,7 @@ __global__ void __launch_bounds__(512, 1)
   auto trace = [&](int row, int ev) {
     if constexpr (kTrace) {
       if (row < p.trace_rows)
-        p.trace[((size_t)blockIdx.x * p.trace_rows + row) * kTraceEvents + ev] = globaltimer();
+        p.trace[((size_t)tmem_slot[1] * p.trace_rows + row) * kTraceEvents + ev] = globaltimer();
     }
   };
   auto wait = [&](uint32_t bar, uint32_t phase) { mbar_wait(bar, phase, lim, p.err, p.abort_flag); };
@@ -316,12 +323,40 @@ __global__ void __launch_bounds__(512, 1)
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
+  if (threadIdx.x == 0) {
+    int slot = (int)blockIdx.x;
+    if (p.slot_smid) {
+      // every CTA of the cooperative grid is resident: enter this SM's id, count in
+      // (release), wait (bounded) for all entries, and take the rank of this id
+      const int my = (int)smid_u32();
+      p.slot_smid[blockIdx.x] = my;
+      red_add_release_gpu(p.slot_arrive, 1u);
+      const uint64_t t0 = globaltimer();
+      bool all = false;
+      while (!(all = (ld_acquire_gpu(p.slot_arrive) >= gridDim.x))) {
+        if (aborted(p.abort_flag) || globaltimer() - t0 > lim) {
+          if (!aborted(p.abort_flag)) raise_timeout(p.err, p.abort_flag, ERR_WHERE_PIPE);
+          break;
+        }
+      }
+      if (all) {
+        int rank = 0;
+        for (int j = 0; j < (int)gridDim.x; ++j) {
+          const int o = ld_cg_s32(p.slot_smid + j);
+          rank += (o < my || (o == my && j < (int)blockIdx.x)) ? 1 : 0;
+        }
+        slot = rank;
+      }
+    }
+    reinterpret_cast<volatile uint32_t*>(tmem_slot)[1] = (uint32_t)slot;
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const int slot = (int)tmem_slot[1];  // the table slot this CTA runs
 
-  const int cbeg = p.cta_off[blockIdx.x], cend = p.cta_off[blockIdx.x + 1];
+  const int cbeg = p.cta_off[slot], cend = p.cta_off[slot + 1];
   const int S = p.S, N = p.N;
   // Grouped-query attention: the chains of one dK/dV tile (K/V head, KV tile) run back
   // to back on this CTA; such a run loads K/V once and carries dK/dV in TMEM from one

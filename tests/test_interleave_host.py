@@ -103,3 +103,22 @@ def test_interleaved_table(sched, N, causal, heads, il, ctas):
     for chains_per_block in (1, 2):
         n, edges, _ = dag.schedule_graph(slots, 1.0, 0.3, None, chains_per_block)
         assert _acyclic(n, edges)
+
+
+def test_slot_placement_choice():
+    """Slots are placed by SM id from 128 tiles by default; modes 1 and 2 force it."""
+    f = binding.dash_slot_placement_by_smid
+    try:
+        binding.dash_set_slot_placement(0)
+        assert f(16384) and f(32768) and not f(8192) and not f(128)
+        binding.dash_set_slot_placement(1)
+        assert f(128) and f(16384)
+        binding.dash_set_slot_placement(2)
+        assert not f(16384)
+        for bad in (lambda: binding.dash_set_slot_placement(3),
+                    lambda: binding.dash_set_slot_placement(-1),
+                    lambda: f(100), lambda: f(0)):
+            with pytest.raises(binding.DashError):
+                bad()
+    finally:
+        binding.dash_set_slot_placement(0)
