@@ -55,7 +55,8 @@ typedef enum {
   DASH_SCHED_DESCENDING = 1,  /* §2.2.A: Q tiles last to first, dQ order ascending KV  */
   DASH_SCHED_SHIFT = 2,       /* §2.2.B full masks: cyclic shift, conflict-free order  */
   DASH_SCHED_SYM_SHIFT = 3,   /* §2.2.B causal masks: KV i and N-1-i folded, 2 phases  */
-  DASH_SCHED_ATOMIC = 4       /* §1 nondeterministic counterpart: fp32 atomic dQ adds  */
+  DASH_SCHED_ATOMIC = 4,      /* §1 nondeterministic counterpart: fp32 atomic dQ adds  */
+  DASH_SCHED_SHIFT_PAIRS = 5  /* full masks, even N: CTA pairs pre-sum dQ (see below)  */
 } dash_schedule_t;
 
 typedef enum {
@@ -357,6 +358,22 @@ int dash_attn_bwd_host(const void* q, const void* k, const void* v, const void* 
  */
 long long dash_sched_table(int n_heads, int N, int causal, int schedule, int num_ctas,
                            int* rows, long long cap);
+
+/*
+ * DASH_SCHED_SHIFT_PAIRS.  The pages name 2-CTA pairs as the answer to the register
+ * and TMEM pressure of one KV tile per SM (DASH summary §4) and print no schedule for
+ * them; this is the library's.  CTAs 2i and 2i + 1 run KV tiles 2m and 2m + 1 of a
+ * head over the same Q tiles at the same steps, Q tile m + t mod N at step t, and the
+ * two dQ partials of a step are added together before the ordered accumulation, so a
+ * dQ block receives N / 2 contributions, in (round, step) order.  Full mask, N even.
+ * For this schedule dash_sched_table returns the half table, one row per pair of KV
+ * tiles (kv = m, num_ctas counting CTA pairs); dash_sched_table_pairs returns the grid's
+ * table for num_ctas CTAs (even): rows as for dash_sched_table, slot 2i with KV tile 2m
+ * and slot 2i + 1 with KV tile 2m + 1, both with the pair's Q tiles and positions.
+ * Returns the number of rows, or -DASH_ERR_INVALID_ARG (odd num_ctas),
+ * -DASH_ERR_UNSUPPORTED or -DASH_ERR_SCHEDULE.
+ */
+long long dash_sched_table_pairs(int n_heads, int N, int num_ctas, int* rows, long long cap);
 
 /*
  * The part of that table covering heads [h0, h1) (0 <= h0 < h1 <= n_heads), as the

@@ -24,6 +24,13 @@ Schedules (names follow the pages):
   visits k, k+1, ..., N-1, 0, ..., k-1 (the page prints this sequence; with one
   KV tile per SM it is read as the sequence of Q tiles, i.e. dQ blocks, that
   chain visits).  Each dQ block accumulates in step order.
+* ``shift_pairs`` -- the shift order for CTA pairs that pre-sum dQ (the "2-CTA
+  pairs" the pages' register-pressure remark in DASH summary §4 points to; the
+  pages print no such schedule, so this is this library's construction): unit m
+  stands for KV tiles 2m and 2m+1, run by two CTAs over the same Q tiles at the
+  same steps, m + t mod N at step t, so each step touches N/2 distinct dQ blocks.
+  A dQ block then receives N/2 pre-summed contributions, accumulated in step
+  order.  Full mask, even N.
 * ``sym_shift``  -- DASH summary §2.2.B, causal masks: KV tiles k and N-1-k are
   paired (one CTA serves both, one after the other) so the triangle of causal
   pairs folds into an N/2 x (N+1) rectangle, run in two phases: the dense
@@ -34,6 +41,7 @@ from __future__ import annotations
 
 NAIVE_ASC, DESCENDING, SHIFT, SYM_SHIFT = "naive_asc", "descending", "shift", "sym_shift"
 ALL = (NAIVE_ASC, DESCENDING, SHIFT, SYM_SHIFT)
+SHIFT_PAIRS = "shift_pairs"  # units stand for KV pairs; not in ALL (its units differ in kind)
 
 
 def supported(name: str, N: int, causal: bool) -> bool:
@@ -42,6 +50,8 @@ def supported(name: str, N: int, causal: bool) -> bool:
         return not causal
     if name == SYM_SHIFT:
         return causal and N % 2 == 0
+    if name == SHIFT_PAIRS:
+        return not causal and N % 2 == 0
     return name in (NAIVE_ASC, DESCENDING)
 
 
@@ -62,6 +72,10 @@ def units(name: str, N: int, causal: bool):
     elif name == SHIFT:
         for k in range(N):
             out.append([(k, (k + t) % N) for t in range(N)])
+    elif name == SHIFT_PAIRS:
+        # unit m: the KV pair (2m, 2m+1), written as m
+        for m in range(N // 2):
+            out.append([(m, (m + t) % N) for t in range(N)])
     elif name == SYM_SHIFT:
         h = N // 2
         for k in range(h):

@@ -14,7 +14,8 @@ import os
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libdash_attn.so")
 
-SCHEDULES = {"naive_asc": 0, "descending": 1, "shift": 2, "sym_shift": 3, "atomic": 4}
+SCHEDULES = {"naive_asc": 0, "descending": 1, "shift": 2, "sym_shift": 3, "atomic": 4,
+             "shift_pairs": 5}
 STATUS = {0: "DASH_OK", 1: "DASH_ERR_INVALID_ARG", 2: "DASH_ERR_UNSUPPORTED", 3: "DASH_ERR_CUDA",
           4: "DASH_ERR_TIMEOUT", 5: "DASH_ERR_OOM", 6: "DASH_ERR_SCHEDULE"}
 
@@ -29,7 +30,7 @@ EXPORTS = ("dash_attn_fwd", "dash_attn_bwd", "dash_attn_sync_status", "dash_stat
            "dash_attn_bwd_gqa_split", "dash_bwd_gqa_split_for", "dash_set_dq_chain_mode",
            "dash_dq_chain_uses_red", "dash_set_head_interleave",
            "dash_bwd_head_interleave", "dash_set_slot_placement",
-           "dash_slot_placement_by_smid")
+           "dash_slot_placement_by_smid", "dash_sched_table_pairs")
 
 
 class DashError(RuntimeError):
@@ -85,6 +86,8 @@ def load(path: str | None = None):
     lib.dash_sched_table_part.restype = ll
     lib.dash_sched_table_gqa.argtypes = [i, i, i, i, i, i, vp, ll]
     lib.dash_sched_table_gqa.restype = ll
+    lib.dash_sched_table_pairs.argtypes = [i, i, i, vp, ll]
+    lib.dash_sched_table_pairs.restype = ll
     lib.dash_sched_simulate.argtypes = [i, i, i, i, i, d, d, i, i, P(d), P(d), P(d), P(ll)]
     lib.dash_sched_simulate_gqa.argtypes = [i, i, i, i, i, i, d, d, i, i, P(d), P(d), P(d),
                                             P(ll)]
@@ -95,7 +98,8 @@ def load(path: str | None = None):
     lib.dash_profile_end.argtypes = [P(d), P(d), P(ll)]
     for name in EXPORTS:
         if name not in ("dash_status_string", "dash_sched_table", "dash_sched_table_part",
-                        "dash_sched_table_gqa", "dash_attn_noalloc_sync_status"):
+                        "dash_sched_table_gqa", "dash_attn_noalloc_sync_status",
+                        "dash_sched_table_pairs"):
             getattr(lib, name).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -395,6 +399,20 @@ def dash_sched_table_gqa(n_heads: int, group: int, N: int, causal: bool, schedul
         raise DashError(int(-n), "dash_sched_table_gqa")
     buf = (ctypes.c_int * (6 * max(n, 1)))()
     lib.dash_sched_table_gqa(n_heads, group, N, int(bool(causal)), sid, num_ctas, buf, n)
+    flat = list(buf)
+    return [tuple(flat[6 * r: 6 * r + 6]) for r in range(n)]
+
+
+def dash_sched_table_pairs(n_heads: int, N: int, num_ctas: int):
+    """Rows (cta, head, kv, q, position, chain_index) of the grid's SHIFT_PAIRS table for
+    num_ctas CTAs (even): CTAs 2i and 2i + 1 run KV tiles 2m and 2m + 1 over the same Q
+    tiles with the same positions."""
+    lib = load()
+    n = lib.dash_sched_table_pairs(n_heads, N, num_ctas, None, 0)
+    if n < 0:
+        raise DashError(int(-n), "dash_sched_table_pairs")
+    buf = (ctypes.c_int * (6 * max(n, 1)))()
+    lib.dash_sched_table_pairs(n_heads, N, num_ctas, buf, n)
     flat = list(buf)
     return [tuple(flat[6 * r: 6 * r + 6]) for r in range(n)]
 

@@ -1202,6 +1202,36 @@ long long dash_sched_table(int n_heads, int N, int causal, int schedule, int num
   }, -DASH_ERR_OOM, -DASH_ERR_INVALID_ARG);
 }
 
+long long dash_sched_table_pairs(int n_heads, int N, int num_ctas, int* rows, long long cap) {
+  return no_throw([&]() -> long long {
+    if (num_ctas < 2 || num_ctas % 2 != 0) return -DASH_ERR_INVALID_ARG;
+    dash::Table half, t;
+    std::string err;
+    if (!dash::build_table(n_heads, N, 0, dash::SHIFT_PAIRS, num_ctas / 2, &half, &err))
+      return -DASH_ERR_UNSUPPORTED;
+    if (!dash::validate_table(half, &err)) return -DASH_ERR_SCHEDULE;
+    if (!dash::expand_pair_table(half, &t)) return -DASH_ERR_SCHEDULE;
+    long long n = 0;
+    for (int c = 0; c < t.num_ctas; ++c)
+      for (int ci = t.cta_off[c]; ci < t.cta_off[c + 1]; ++ci) {
+        const dash::Chain& ch = t.chains[ci];
+        for (int i = 0; i < ch.pair_cnt; ++i, ++n) {
+          if (rows && n < cap) {
+            const uint32_t w = t.pairs[ch.pair_off + i];
+            int* r = rows + 6 * n;
+            r[0] = c;
+            r[1] = ch.bh;
+            r[2] = ch.kv;
+            r[3] = dash::pair_q(w);
+            r[4] = dash::pair_pos(w);
+            r[5] = ci;
+          }
+        }
+      }
+    return n;
+  }, -DASH_ERR_OOM, -DASH_ERR_INVALID_ARG);
+}
+
 int dash_sched_simulate(int n_heads, int N, int causal, int schedule, int num_ctas,
                         double w_compute, double w_reduce, int dq_buffers, int dq_chains,
                         double* critical_path, double* makespan, double* bubble_time,

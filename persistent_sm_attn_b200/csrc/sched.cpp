@@ -35,6 +35,7 @@ bool schedule_supported(int schedule, int N, int causal) {
     case ATOMIC: return true;
     case SHIFT: return !causal;
     case SYM_SHIFT: return causal && (N % 2 == 0);
+    case SHIFT_PAIRS: return !causal && (N % 2 == 0);
     default: return false;
   }
 }
@@ -66,6 +67,14 @@ static Units units_of(int schedule, int N, int causal) {
       for (int k = 0; k < N; ++k) {
         std::vector<std::pair<int, int>> seq;
         for (int t = 0; t < N; ++t) seq.push_back({k, (k + t) % N});
+        u.push_back(seq);
+      }
+      break;
+    case SHIFT_PAIRS:
+      // unit m: the pair of KV tiles 2m, 2m + 1 (written as m), Q tiles m + t mod N
+      for (int m = 0; m < N / 2; ++m) {
+        std::vector<std::pair<int, int>> seq;
+        for (int t = 0; t < N; ++t) seq.push_back({m, (m + t) % N});
         u.push_back(seq);
       }
       break;
@@ -181,6 +190,7 @@ bool build_table_grouped(int n_heads, int group, int N, int causal, int schedule
   Table t;
   t.n_heads = n_heads; t.N = N; t.causal = causal; t.schedule = schedule; t.num_ctas = num_ctas;
   t.group = group;
+  if (schedule == SHIFT_PAIRS) t.kv_units = N / 2;
   // per CTA, the global units it runs, in round order
   std::vector<std::vector<long long>> per_cta(num_ctas);
   const long long total_units = (long long)(n_heads / group) * U;
@@ -276,7 +286,11 @@ bool validate_table(const Table& t, std::string* err) {
     return fail("bad cta offsets");
   // the pair count is fixed by the mask; checking it first bounds the scratch below by
   // the table's own size, whatever n_heads a caller-supplied table claims
-  const long long per_head = t.causal ? (long long)N * (N + 1) / 2 : (long long)N * N;
+  // KV units per head: N, or N / 2 KV pairs for a pair schedule's half table
+  const int kvn = t.kv_units > 0 ? t.kv_units : N;
+  if (kvn > N || (t.kv_units > 0 && (t.causal || t.schedule != SHIFT_PAIRS)))
+    return fail("bad KV unit count");
+  const long long per_head = t.causal ? (long long)N * (N + 1) / 2 : (long long)kvn * N;
   if ((long long)t.n_pairs() != (long long)t.n_heads * per_head)
     return fail("table has missing or extra pairs");
   const long long nblk = (long long)t.n_heads * N;
@@ -288,7 +302,7 @@ bool validate_table(const Table& t, std::string* err) {
     if (t.cta_off[c] > t.cta_off[c + 1]) return fail("cta offsets not monotone");
     for (int ci = t.cta_off[c]; ci < t.cta_off[c + 1]; ++ci) {
       const Chain& ch = t.chains[ci];
-      if (ch.bh < 0 || ch.bh >= t.n_heads || ch.kv < 0 || ch.kv >= N || ch.pair_cnt < 1)
+      if (ch.bh < 0 || ch.bh >= t.n_heads || ch.kv < 0 || ch.kv >= kvn || ch.pair_cnt < 1)
         return fail("chain out of range");
       if (ch.pair_off < 0 || (long long)ch.pair_off + ch.pair_cnt > t.n_pairs())
         return fail("chain pair range out of bounds");
@@ -330,7 +344,7 @@ bool validate_table(const Table& t, std::string* err) {
   }
   for (long long blk = 0; blk < nblk; ++blk) {
     const int q = (int)(blk % N);
-    const int want = t.causal ? q + 1 : N;
+    const int want = t.causal ? q + 1 : kvn;
     if (n_contrib[blk] != want) return fail("dQ block has missing or extra contributors");
     for (int p = 0; p < want; ++p)
       if (!pos_seen[(size_t)blk * N + p]) return fail("positions are not a permutation");
@@ -486,6 +500,30 @@ bool simulate_table(const Table& t, double c, double r, int beta, int chains, Si
     out.bubble_time += cp - c * (double)nodes.size();
   }
   *res = out;
+  return true;
+}
+
+bool expand_pair_table(const Table& half, Table* out) {
+  if (half.schedule != SHIFT_PAIRS || half.kv_units * 2 != half.N || half.causal ||
+      half.group != 1 || (long long)half.num_ctas * 2 > kMaxTableCtas)
+    return false;
+  Table t;
+  t.n_heads = half.n_heads; t.N = half.N; t.causal = 0; t.schedule = SHIFT_PAIRS;
+  t.num_ctas = 2 * half.num_ctas;
+  t.group = 1;
+  t.kv_units = 0;  // the grid's table holds every KV tile
+  t.cta_off.assign(t.num_ctas + 1, 0);
+  for (int c = 0; c < half.num_ctas; ++c)
+    for (int r = 0; r < 2; ++r) {
+      t.cta_off[2 * c + r] = (int32_t)t.chains.size();
+      for (int ci = half.cta_off[c]; ci < half.cta_off[c + 1]; ++ci) {
+        const Chain& h = half.chains[ci];
+        t.chains.push_back(Chain{h.bh, 2 * h.kv + r, (int32_t)t.pairs.size(), h.pair_cnt});
+        for (int i = 0; i < h.pair_cnt; ++i) t.pairs.push_back(half.pairs[h.pair_off + i]);
+      }
+    }
+  t.cta_off[t.num_ctas] = (int32_t)t.chains.size();
+  *out = std::move(t);
   return true;
 }
 

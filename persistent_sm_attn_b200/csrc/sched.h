@@ -14,7 +14,8 @@
 
 namespace dash {
 
-enum Schedule { NAIVE_ASC = 0, DESCENDING = 1, SHIFT = 2, SYM_SHIFT = 3, ATOMIC = 4 };
+enum Schedule { NAIVE_ASC = 0, DESCENDING = 1, SHIFT = 2, SYM_SHIFT = 3, ATOMIC = 4,
+                SHIFT_PAIRS = 5 };
 
 // Upper bound on a table's CTA count (the kernel's grid is the SM count times the CTAs
 // resident per SM); larger requests are refused instead of sizing per-CTA lists by them.
@@ -35,6 +36,9 @@ inline int pair_pos(uint32_t w) { return int(w >> 16); }
 struct Table {
   int n_heads = 0, N = 0, causal = 0, schedule = 0, num_ctas = 0;
   int group = 1;  // query heads per K/V head (grouped-query attention); 1 = one K/V head each
+  // KV units per head when a unit stands for a pair of KV tiles (SHIFT_PAIRS' half table:
+  // N / 2, unit m = KV tiles 2m and 2m + 1); 0: one KV tile per unit, N of them
+  int kv_units = 0;
   std::vector<int32_t> cta_off;   // num_ctas + 1 offsets into chains
   std::vector<Chain> chains;      // grouped by CTA, in execution order
   std::vector<uint32_t> pairs;    // packed (q, position)
@@ -46,6 +50,15 @@ bool schedule_supported(int schedule, int N, int causal);
 
 // Units of one head: each a list of (kv, q) in visiting order.
 std::vector<std::vector<std::pair<int, int>>> head_units(int schedule, int N, int causal);
+
+// SHIFT_PAIRS (full mask, N even): CTA pairs (2i, 2i + 1) run KV tiles 2m and 2m + 1 of
+// a head over the same Q tiles at the same steps, m + t mod N at step t, and pre-sum
+// their two dQ partials before the ordered accumulation, so a dQ block receives N / 2
+// (pre-summed) contributions, in (round, step) order.  build_table_grouped builds the
+// half table (one unit per KV pair, num_ctas / 2 slots, kv = m); expand_pair_table
+// turns it into the grid's table, slot 2i running KV tile 2m and slot 2i + 1 KV tile
+// 2m + 1 with the same Q tiles and positions.
+bool expand_pair_table(const Table& half, Table* out);
 
 // Query heads per unit of a multi-head launch's table.  With il > 1 the launch uses
 // build_table_grouped(n_heads, il, ...) although every head has K/V of its own: each KV
