@@ -145,7 +145,7 @@ struct BwdCfg {
   static constexpr int kDsBufs = (D == 64) ? 2 : 1;
   static constexpr int OFF_DST = OFF_DO + kStagesDO * kTile;
   static constexpr int OFF_BAR = OFF_DST + kDsBufs * 32768;
-  static constexpr int kBars = 25 + 2 * kStagesQ + 2 * kStagesDO;
+  static constexpr int kBars = 26 + 2 * kStagesQ + 2 * kStagesDO;
   static constexpr int OFF_TMEM_SLOT = OFF_BAR + kBars * 8;
   // The swizzled tiles need a 1 KiB aligned base; the kernel checks it.
   static constexpr int kSmemBytes = OFF_TMEM_SLOT + 16;
@@ -178,10 +178,11 @@ constexpr long long dq_units(long long bh_times_n) {
 enum {
   B_KV_FULL = 0, B_KV_EMPTY, B_S_FULL, B_DP_FULL, B_DS_READY, B_DS_FREE, B_DQ_FULL0, B_DQ_FULL1,
   B_DQ_EMPTY0, B_DQ_EMPTY1, B_DVDK_DONE, B_DKDV_FULL, B_DKDV_EMPTY, B_FINAL, B_P_READY,
-  B_S_FULL1, B_P_READY1, B_UNUSED17,  // the second S^T buffer's barriers (D = 64)
+  B_S_FULL1, B_P_READY1, B_PEER0,  // the second S^T buffer's barriers (D = 64); see B_PEER1
   B_PUB_READY0, B_PUB_READY1, B_PUB_FREE0, B_PUB_FREE1,  // reducers -> publisher hand-off
   B_DS_READY1, B_DP_FULL1, B_DS_FREE1,  // odd tiles' barriers (D = 64)
-  B_STAGE0 = 25
+  B_PEER1,  // CTA pairs: the peer's tile of this parity is staged (with B_PEER0)
+  B_STAGE0 = 26
 };
 
 // D = 64: the TMEM column (within a tile's S^T buffer) where the softmax packs the
@@ -204,13 +205,22 @@ constexpr int kTraceEvents = 16;
 // grants them, instead of a load-add-store from the SM.  The additions and their order
 // are the same, so the results are bitwise the same; only the traffic and the latency
 // of each link differ.
-template <int D, bool kAtomic, bool kTrace = false, bool kRed = false>
+// kPair (D = 64, deterministic, load-add-store chains): the grid runs in clusters of two
+// CTAs, 2i and 2i + 1, with a SHIFT_PAIRS table: the pair runs KV tiles 2m and 2m + 1 over
+// the same Q tiles at the same steps.  Each CTA's reducers add the two staged dQ partials
+// of a step (its own, and the peer's read over distributed shared memory) for half of
+// the columns, CTA 2i + r taking columns [32r, 32r + 32), and run the ordered
+// accumulation of that half: one contribution per pair and step, so N / 2 per block and
+// half the accumulator bytes per CTA.  Both CTAs free a staged tile only after both
+// have read it.
+template <int D, bool kAtomic, bool kTrace = false, bool kRed = false, bool kPair = false>
 __global__ void __launch_bounds__(512, 1)
     dash_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                     const __grid_constant__ CUtensorMap tmC, const BwdParams p) {
   using namespace dev;
   using C = BwdCfg<D>;
+  static_assert(!kPair || (D == 64 && !kAtomic && !kRed), "CTA pairs: D = 64, load-add-store");
   constexpr int ST = C::kStagesQ, SD = C::kStagesDO;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t sb = smem_u32(smem_raw);
@@ -219,6 +229,7 @@ __global__ void __launch_bounds__(512, 1)
       atomicOr(p.err, ERR_MISALIGNED);
       atomicOr(p.abort_flag, 1u);
     }
+    if constexpr (kPair) cluster_sync_all();  // the peer takes the same branch
     return;
   }
   uint8_t* gb = smem_raw;
@@ -274,8 +285,13 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(BAR(B_DS_READY1), kSoftmaxArrive);
     // D = 64: the reducers (128 threads) free a dS buffer once they have read the dQp
     // staged there; D = 128: the commit of dQp and dK frees it
-    mbar_init(BAR(B_DS_FREE), C::kSDouble ? 128u : 1u);
-    mbar_init(BAR(B_DS_FREE1), C::kSDouble ? 128u : 1u);
+    // CTA pairs: both CTAs' reducers read each staged tile (128 + 128 arrivals)
+    constexpr uint32_t kDsFree = kPair ? 256u : (C::kSDouble ? 128u : 1u);
+    mbar_init(BAR(B_DS_FREE), kDsFree);
+    mbar_init(BAR(B_DS_FREE1), kDsFree);
+    // CTA pairs: the peer's softmax warpgroup (128 threads) has staged its tile's dQp
+    mbar_init(BAR(B_PEER0), 128);
+    mbar_init(BAR(B_PEER1), 128);
     for (int b = 0; b < 2; ++b) {
       mbar_init(BAR(B_DQ_FULL0 + b), 1);
       mbar_init(BAR(B_DQ_EMPTY0 + b), 128);
@@ -325,7 +341,7 @@ __global__ void __launch_bounds__(512, 1)
   }
   if (threadIdx.x == 0) {
     int slot = (int)blockIdx.x;
-    if (p.slot_smid) {
+    if (!kPair && p.slot_smid) {  // a pair's slots are its cluster's CTAs
       // every CTA of the cooperative grid is resident: enter this SM's id, count in
       // (release), wait (bounded) for all entries, and take the rank of this id
       const int my = (int)smid_u32();
@@ -353,8 +369,11 @@ __global__ void __launch_bounds__(512, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // CTA pairs: the peer's barriers are initialised before anything arrives on them
+  if constexpr (kPair) cluster_sync_all();
   const uint32_t tmem = *tmem_slot;
   const int slot = (int)tmem_slot[1];  // the table slot this CTA runs
+  const uint32_t prank = kPair ? cluster_ctarank() : 0u;  // this CTA's rank in its pair
 
   const int cbeg = p.cta_off[slot], cend = p.cta_off[slot + 1];
   const int S = p.S, N = p.N;
@@ -708,9 +727,12 @@ __global__ void __launch_bounds__(512, 1)
         for (int t = 0; t < n_pairs(ch.w); ++t, ++it) {
           const uint32_t w = p.pairs[ch.z + t];
           const int q = (int)(w & 0xffffu), pos = (int)(w >> 16);
-          const int ncontrib = p.causal ? q + 1 : N;
+          // CTA pairs: N / 2 contributions per block, tickets per (block, half, chain)
+          const int ncontrib = kPair ? N / 2 : (p.causal ? q + 1 : N);
           if (pos == ncontrib - 1) continue;  // the last contributor writes dQ itself
-          const long long unit = ((long long)ch.x * N + q) * 2 + (pos & 1);
+          const long long unit =
+              kPair ? (((long long)ch.x * N + q) * 2 + prank) * 2 + (pos & 1)
+                    : ((long long)ch.x * N + q) * 2 + (pos & 1);
           wait(BAR(B_PUB_READY0 + (k & 1)), (k >> 1) & 1);
           st_release_gpu(p.tickets + unit, (uint32_t)((pos >> 1) + 1));
           mbar_arrive(BAR(B_PUB_FREE0 + (k & 1)));
@@ -838,6 +860,9 @@ __global__ void __launch_bounds__(512, 1)
           }
           tc_fence_before();
           mbar_arrive(DQ_EMPTY(it));
+          // CTA pairs: tell the peer's reducers that this tile's dQp is staged here
+          if constexpr (kPair)
+            mbar_arrive_cluster(mapa_shared(BAR((it & 1) ? B_PEER1 : B_PEER0), prank ^ 1u));
         }
       }
     } else {
@@ -929,6 +954,8 @@ __global__ void __launch_bounds__(512, 1)
     const int r = quarter * 32 + lane;  // Q row for dQ, KV row for dK/dV
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     constexpr int NV = D / 4;           // float4 per row
+    // float4 per row of this CTA's share of a dQ block: all of it, or half for CTA pairs
+    constexpr int NA = kPair ? NV / 2 : NV;
     constexpr int G = 24;               // loads in flight per group
     int it = 0, fn = 0;  // fn: dK/dV runs written out
     int npub = 0;        // pairs handed to the publisher
@@ -936,7 +963,7 @@ __global__ void __launch_bounds__(512, 1)
     // next pair go out if its ticket is already granted (checked once, never waited
     // for here), so their round trip overlaps the wait for the next partial and its
     // drain.  The values loaded and the order of the additions are the same either way.
-    constexpr bool kLook = !kAtomic && D == 64 && !kRed;
+    constexpr bool kLook = !kAtomic && D == 64 && !kRed && !kPair;
     float4 pre[NV];
     bool pre_ok = false;  // pre holds this pair's accumulator, loaded ahead
     for (int ci = cbeg; ci < cend; ++ci) {
@@ -944,10 +971,34 @@ __global__ void __launch_bounds__(512, 1)
       for (int t = 0; t < n_pairs(ch.w); ++t, ++it) {
         const uint32_t w = p.pairs[ch.z + t];
         const int q = (int)(w & 0xffffu), pos = (int)(w >> 16);
-        const int ncontrib = p.causal ? q + 1 : N;
+        // CTA pairs: N / 2 (pre-summed) contributions per block
+        const int ncontrib = kPair ? N / 2 : (p.causal ? q + 1 : N);
         const bool last = (pos == ncontrib - 1);
         float a[D];
-        if constexpr (C::kSDouble) {
+        if constexpr (kPair) {
+          // this CTA's half of the columns of the two partials staged for this step, its
+          // own and the peer's (read over distributed shared memory once the peer says it
+          // is staged), added: a + b is the same sum in either CTA
+          wait(DQ_EMPTY(it), s_phase(it));
+          mbar_wait_cluster(BAR((it & 1) ? B_PEER1 : B_PEER0), s_phase(it), lim, p.err,
+                            p.abort_flag);
+          if (threadIdx.x == 256) trace(it, 4);
+          const uint32_t stage = sDSt + 32768u * (uint32_t)(it & 1);
+          const uint32_t pstage = mapa_shared(stage, prank ^ 1u);
+#pragma unroll
+          for (int j = 0; j < NA; ++j) {
+            const uint32_t off = (uint32_t)((((int)prank * NA + j) * 128 + r) * 16);
+            const float4 u = ld_shared_f4(stage + off);
+            const float4 v = ld_shared_cluster_f4(pstage + off);
+            a[4 * j] = u.x + v.x;
+            a[4 * j + 1] = u.y + v.y;
+            a[4 * j + 2] = u.z + v.z;
+            a[4 * j + 3] = u.w + v.w;
+          }
+          // both CTAs read both staged tiles: each frees both
+          mbar_arrive(DS_FREE(it));
+          mbar_arrive_cluster(mapa_shared(DS_FREE(it), prank ^ 1u));
+        } else if constexpr (C::kSDouble) {
           // D = 64: the softmax warpgroup of this tile has staged dQp in its dS buffer
           wait(DQ_EMPTY(it), s_phase(it));
           if (threadIdx.x == 256) trace(it, 4);
@@ -983,8 +1034,12 @@ __global__ void __launch_bounds__(512, 1)
           // their own, so consecutive contributors to a block do not wait on each
           // other.  The block's last contributor adds the two chain sums.
           const int chain = pos & 1, idx = pos >> 1;
-          const long long unit = blk * 2 + chain;
-          float4* accp = reinterpret_cast<float4*>(p.acc) + unit * (32 * D);
+          // CTA pairs: one chain per (block, half of the columns, parity), 128 x D/2 fp32
+          auto unit_of = [&](int ch_) -> long long {
+            return kPair ? (blk * 2 + (long long)prank) * 2 + ch_ : blk * 2 + ch_;
+          };
+          const long long unit = unit_of(chain);
+          float4* accp = reinterpret_cast<float4*>(p.acc) + unit * (128 * NA);
           // wait (bounded) until a chain's ticket reaches `want`.  Lane 0 acquires
           // (its acquire pairs with the publisher's release) and the warp barrier
           // orders the other lanes' accumulator loads after it.  `seen` is a value
@@ -1006,18 +1061,18 @@ __global__ void __launch_bounds__(512, 1)
             }
             __syncwarp();
           };
-          // a = acc + a over this thread's NV slots, up to G loads in flight before their
-          // adds (the last group holds the remaining NV mod G slots)
+          // a = acc + a over this thread's NA slots, up to G loads in flight before their
+          // adds (the last group holds the remaining NA mod G slots)
           auto add_from = [&](const float4* src) {
 #pragma unroll
-            for (int g0 = 0; g0 < NV; g0 += G) {
+            for (int g0 = 0; g0 < NA; g0 += G) {
               float4 old[G];
 #pragma unroll
               for (int j = 0; j < G; ++j)
-                if (g0 + j < NV) old[j] = ld_cg_f4(src + (g0 + j) * 128 + r);
+                if (g0 + j < NA) old[j] = ld_cg_f4(src + (g0 + j) * 128 + r);
 #pragma unroll
               for (int j = 0; j < G; ++j) {
-                if (g0 + j < NV) {
+                if (g0 + j < NA) {
                   float* x = a + 4 * (g0 + j);
                   x[0] = old[j].x + x[0];
                   x[1] = old[j].y + x[1];
@@ -1063,14 +1118,16 @@ __global__ void __launch_bounds__(512, 1)
             if (ncontrib > 1) {
               // the other chain is complete once its ticket counts all its positions
               const int other = chain ^ 1;
-              const long long ounit = blk * 2 + other;
+              const long long ounit = unit_of(other);
               ticket_wait(p.tickets + ounit, (uint32_t)((ncontrib + 1 - other) / 2), ~0u);
-              add_from(reinterpret_cast<const float4*>(p.acc) + ounit * (32 * D));
+              add_from(reinterpret_cast<const float4*>(p.acc) + ounit * (128 * NA));
             }
-            __nv_bfloat16* out = p.dq + ((size_t)ch.x * S + (size_t)q * 128 + r) * D;
+            // CTA pairs: this CTA's half of the columns
+            __nv_bfloat16* out = p.dq + ((size_t)ch.x * S + (size_t)q * 128 + r) * D +
+                                 (kPair ? (size_t)prank * (D / 2) : 0);
             const float sc = p.scale;
 #pragma unroll
-            for (int c8 = 0; c8 < D / 8; ++c8) {
+            for (int c8 = 0; c8 < NA / 2; ++c8) {
               const float* x = a + 8 * c8;
               uint4 pk;
               pk.x = pack_bf16x2(x[0] * sc, x[1] * sc);
@@ -1093,7 +1150,7 @@ __global__ void __launch_bounds__(512, 1)
                            make_float4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]));
             } else {
 #pragma unroll
-              for (int c4 = 0; c4 < NV; ++c4)
+              for (int c4 = 0; c4 < NA; ++c4)
                 st_cg_f4(accp + c4 * 128 + r,
                          make_float4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]));
             }
@@ -1264,6 +1321,9 @@ __global__ void __launch_bounds__(512, 1)
 
   tc_fence_before();
   __syncthreads();
+  // CTA pairs: neither CTA leaves while the other may still read its shared memory or
+  // arrive on its barriers
+  if constexpr (kPair) cluster_sync_all();
   if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);

@@ -563,6 +563,136 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   return DASH_OK;
 }
 
+// ------------------------------------------------------------------ CTA pairs
+// SHIFT_PAIRS at D = 64: the kernel runs in clusters of two CTAs, with as many
+// clusters as fit on the device at once (cooperative, so all are resident).
+std::map<int, int> g_pair_ctas;  // device -> CTAs of the pair launch
+int pair_ctas(int dev, int* out) {
+  auto it = g_pair_ctas.find(dev);
+  if (it != g_pair_ctas.end()) {
+    *out = it->second;
+    return DASH_OK;
+  }
+  using C = BwdCfg<64>;
+  auto kern = dash::dash_bwd_kernel<64, false, false, false, true>;
+  DASH_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes));
+  cudaFuncAttributes fa;
+  DASH_CUDA(cudaFuncGetAttributes(&fa, kern));
+  if (fa.numRegs != C::kLaunchRegs) return DASH_ERR_UNSUPPORTED;
+  int sms = 0;
+  DASH_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * sms));
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  DASH_CUDA(cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg));
+  if (clusters < 1) return DASH_ERR_UNSUPPORTED;
+  *out = 2 * clusters;
+  g_pair_ctas[dev] = *out;
+  return DASH_OK;
+}
+
+int launch_bwd_pairs(const void* q, const void* k, const void* v, const void* o,
+                     const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                     int H, int S, cudaStream_t stream, int dev) {
+  constexpr int D = 64;
+  using C = BwdCfg<D>;
+  const int N = S / 128;
+  const long long rows = (long long)B * H * S;
+  int ctas = 0;
+  int rc;
+  // tickets per (block, half of the columns, chain)
+  const long long dqn = 2 * dash::dq_units<D>((long long)B * H * N);
+  DevTable* tab = nullptr;
+  Workspace* ws = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if ((rc = pair_ctas(dev, &ctas))) return rc;
+    auto key = std::make_tuple(dev, B * H, N, 0, (int)dash::SHIFT_PAIRS, ctas, 1, 1);
+    auto itb = g_tables.find(key);
+    if (itb != g_tables.end()) {
+      tab = &itb->second;
+    } else {
+      dash::Table half, t;
+      std::string err;
+      if (!dash::build_table(B * H, N, 0, dash::SHIFT_PAIRS, ctas / 2, &half, &err))
+        return DASH_ERR_UNSUPPORTED;
+      if (!dash::validate_table(half, &err) || !dash::expand_pair_table(half, &t))
+        return DASH_ERR_SCHEDULE;
+      DevTable d;
+      if ((rc = upload_table(t, &d, 1))) return rc;
+      tab = &g_tables.emplace(key, d).first->second;
+    }
+    if ((rc = get_workspace(dev, stream, 2 * (size_t)rows * D * sizeof(float),
+                            (size_t)(dqn + 1) * sizeof(uint32_t), (size_t)rows, &ws)))
+      return rc;
+  }
+  CUtensorMap tq, tk, tv, tdo, tc;
+  if ((rc = make_tmap(&tq, q, rows, D, C::kQRows)) ||
+      (rc = make_tmap(&tk, k, rows, D, C::kKVRows)) ||
+      (rc = make_tmap(&tv, v, rows, D, C::kKVRows)) ||
+      (rc = make_tmap(&tdo, dout, rows, D, C::kQRows)) ||
+      (rc = make_tmap_cols(&tc, ws->rowbuf, rows)))
+    return rc;
+  const float scale = 1.0f / sqrtf((float)D);
+  std::array<cudaEvent_t, 4> ev{};
+  if (!prof_record(0, &ev, stream)) return DASH_ERR_CUDA;
+  dash::dash_delta_kernel<D><<<dash::delta_grid<D>(rows, ctas), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse,
+      reinterpret_cast<uint4*>(ws->rowbuf), rows, 1.0f / scale, ws->tickets, dqn, ws->err + 1,
+      1);
+  BwdParams p;
+  p.cta_off = tab->cta_off;
+  p.chains = tab->chains;
+  p.pairs = tab->pairs;
+  p.acc = ws->acc;
+  p.tickets = ws->tickets;
+  p.err = ws->err;
+  p.abort_flag = ws->err + 1;
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.S = S;
+  p.N = N;
+  p.causal = 0;
+  p.group_log2 = 0;
+  p.scale = scale;
+  p.scale_log2 = p.scale * 1.4426950408889634f;
+  p.spin_ns = (unsigned long long)spin_us() * 1000ull;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)ctas);
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  if (!prof_record(1, &ev, stream)) return DASH_ERR_CUDA;
+  DASH_CUDA(cudaLaunchKernelEx(&cfg, dash::dash_bwd_kernel<64, false, false, false, true>, tq,
+                               tk, tv, tdo, tc, p));
+  if (!prof_record(2, &ev, stream) || !prof_record(3, &ev, stream)) return DASH_ERR_CUDA;
+  if (g_prof_on.load()) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof.push_back(ev);
+  }
+  DASH_CUDA(cudaGetLastError());
+  return DASH_OK;
+}
+
 // ------------------------------------------------------------------ forward
 template <int D>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
@@ -895,6 +1025,23 @@ int dash_bwd_gqa_split_for(int num_ctas, int B, int Hkv, int group, int S, int c
 int dash_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                   const float* lse, void* dq, void* dk, void* dv, int B, int H, int S, int D,
                   int causal, int schedule, void* stream) {
+  if (schedule == DASH_SCHED_SHIFT_PAIRS)
+    return no_throw([&]() -> int {
+      int rc = check_shape(B, H, S, D);
+      if (rc) return rc;
+      if (causal != 0 && causal != 1) return DASH_ERR_INVALID_ARG;
+      if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+          !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+        return DASH_ERR_INVALID_ARG;
+      // CTA pairs exist for the full mask at D = 64 (the staged dQp they exchange)
+      if (D != 64 || !dash::schedule_supported(schedule, S / 128, causal))
+        return DASH_ERR_UNSUPPORTED;
+      if (B == 0 || H == 0) return DASH_OK;
+      int dev = 0;
+      DASH_CUDA(cudaGetDevice(&dev));
+      return launch_bwd_pairs(q, k, v, o, dout, lse, dq, dk, dv, B, H, S,
+                              static_cast<cudaStream_t>(stream), dev);
+    }, DASH_ERR_OOM, DASH_ERR_INVALID_ARG);
   return dash_attn_bwd_gqa(q, k, v, o, dout, lse, dq, dk, dv, B, H, H, S, D, causal, schedule,
                            stream);
 }

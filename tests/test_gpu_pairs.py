@@ -1,0 +1,40 @@
+"""CTA pairs that pre-sum dQ (DASH_SCHED_SHIFT_PAIRS, D = 64, full mask): the two dQ
+partials of a pair's step are added before the ordered accumulation, each CTA taking
+half of the columns.  Against the fp64 oracle on shapes with one or several rounds of
+CTA pairs, bitwise repeats, and the refusals for shapes the pairs do not serve."""
+import pytest
+import torch
+
+from oracle import attention as A
+from persistent_sm_attn_b200 import binding
+from tests import gpu_util as G
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("B,H,S", [
+    (1, 2, 256),     # one pair unit per head
+    (2, 3, 1024),    # 8 tiles: 4 pair units per head
+    (4, 40, 256),    # 160 pair units: more than one round of CTA pairs
+    (1, 4, 2048),
+])
+def test_pairs_match_oracle_and_repeat(B, H, S):
+    G.need_cuda()
+    case = G.make_case(B, H, S, 64, False, seed=700 + S + H)
+    _, _, *ref = G.oracle_full(case)
+    out = G.bwd(case, "shift_pairs")
+    errs = {n: A.rel_fro(x.float().cpu().numpy(), r) for n, x, r in zip(("dq", "dk", "dv"), out, ref)}
+    G.log_margin(f"shift_pairs B{B} H{H} S{S} D64 full", errs)
+    assert max(errs.values()) < G.TOL, errs
+    again = G.bwd(case, "shift_pairs")
+    for a, b in zip(out, again):
+        assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("S,D,causal", [(512, 128, False), (512, 64, True), (384, 64, False)])
+def test_pairs_refuse_other_shapes(S, D, causal):
+    G.need_cuda()
+    case = G.make_case(1, 2, S, D, causal, seed=5)
+    with pytest.raises(binding.DashError):
+        binding.dash_attn_bwd(case["q"], case["k"], case["v"], case["o"], case["do"],
+                              case["lse"], causal, "shift_pairs")
