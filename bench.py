@@ -69,6 +69,26 @@ def _recorded_traffic(workload: str, schedule: str):
     return None
 
 
+def _workload(args):
+    """The workload of this run: one of the configurations, or --shape B,H,S,D,mask (a
+    shape of the caller's, same input recipe and seed as the --workload configuration)."""
+    from persistent_sm_attn_b200.inputs import WORKLOADS, Workload
+    if not args.shape:
+        return WORKLOADS[args.workload]
+    b, h, s, d, mask = args.shape.split(",")
+    B, H, S, D, causal = int(b), int(h), int(s), int(d), mask.strip() == "causal"
+    N = S // 128
+    if causal:
+        scheds = ("sym_shift", "descending") if N % 2 == 0 else ("descending",)
+    elif D == 64 and N % 2 == 0:
+        scheds = ("shift", "shift_pairs", "descending")
+    else:
+        scheds = ("shift", "descending")
+    scheds = scheds + ("atomic",)
+    return Workload(f"{'causal' if causal else 'full'}_b{B}_h{H}_s{S}_d{D}", B, H, S, D, causal,
+                    1.0, scheds)
+
+
 def _config(w, sched, world, h_kv):
     """The config object of a JSON line; both arms print the same one, so the
     reference arm's line names exactly the workload this arm times."""
@@ -159,7 +179,7 @@ def run_ours(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-    w = WORKLOADS[args.workload]
+    w = _workload(args)
     if args.heads:
         # a smaller case of the same kernel (profiling): B=1 and the given head count
         w = dataclasses.replace(w, B=1, H=args.heads, name=f"{w.name}_as_b1_h{args.heads}")
@@ -328,7 +348,8 @@ def run_ours(args):
             "dq_chain": ("red" if binding.dash_dq_chain_uses_red(sched, w.S, w.D, il)
                          else "load-add-store") if sched != "atomic" else None,
             "heads_per_unit": il if not gqa else None,
-            "slot_placement": ("sm_id" if binding.dash_slot_placement_by_smid(w.S)
+            "slot_placement": ("cta_pairs" if sched == "shift_pairs" else
+                               "sm_id" if binding.dash_slot_placement_by_smid(w.S)
                                else "launch_order"),
             "roofline": {"bound": "tensor", "achieved": round(kern, 2), "peak": peak,
                          "unit": "TFLOP/s", "frac": round(kern / peak, 4),
@@ -437,7 +458,7 @@ def run_reference(args):
     world, rank, _ = _dist_init(args)
     if rank != 0:
         return
-    w = WORKLOADS[args.workload]
+    w = _workload(args)
     gqa = bool(args.kv_heads) and args.kv_heads != w.H
     if gqa:
         # the oracle's grouped-query backward is the per-head backward of every query
@@ -487,6 +508,9 @@ def main():
     ap.add_argument("--kv-heads", type=int, default=0,
                     help="time grouped-query attention with this many K/V heads (a side "
                          "measurement: no host-buffer e2e, simulator or CPU baseline)")
+    ap.add_argument("--shape", default="",
+                    help="B,H,S,D,mask (mask full or causal): time this shape instead of a "
+                         "configuration, with the same input recipe")
     ap.add_argument("--dq-chain-mode", type=int, default=0, choices=(0, 1, 2),
                     help="how the ordered dQ chains add a middle position: 0 the library's "
                          "choice, 1 red in L2, 2 load-add-store (bitwise the same results)")

@@ -372,6 +372,13 @@ long long dash_sched_table(int n_heads, int N, int causal, int schedule, int num
  * and slot 2i + 1 with KV tile 2m + 1, both with the pair's Q tiles and positions.
  * Returns the number of rows, or -DASH_ERR_INVALID_ARG (odd num_ctas),
  * -DASH_ERR_UNSUPPORTED or -DASH_ERR_SCHEDULE.
+ * The backward runs it through dash_attn_bwd only, at D = 64 (each CTA stages its dQ
+ * partial in shared memory, and the pair is a thread-block cluster of two CTAs that read
+ * each other's staged partial): each CTA adds the two partials for half of the columns
+ * and accumulates that half in order.  Other head dims, causal masks and odd N return
+ * DASH_ERR_UNSUPPORTED.  dash_attn_bwd_host takes it too (its parts are slices of the
+ * same table, so the bits are dash_attn_bwd's); the grouped-query, no-allocation and
+ * trace entry points return DASH_ERR_UNSUPPORTED.
  */
 long long dash_sched_table_pairs(int n_heads, int N, int num_ctas, int* rows, long long cap);
 

@@ -232,6 +232,18 @@ __global__ void __launch_bounds__(512, 1)
     if constexpr (kPair) cluster_sync_all();  // the peer takes the same branch
     return;
   }
+  if constexpr (kPair) {
+    // every CTA must sit in a cluster of two with the rank of its slot's parity; a launch
+    // without that (a tool that drops the cluster attribute, say) computes nothing and
+    // reports it, instead of reading a peer that is not there
+    if (cluster_nctarank() != 2u || cluster_ctarank() != (blockIdx.x & 1u)) {
+      if (threadIdx.x == 0) {
+        atomicOr(p.err, ERR_NO_CLUSTER);
+        atomicOr(p.abort_flag, 1u);
+      }
+      return;
+    }
+  }
   uint8_t* gb = smem_raw;
   const uint32_t sK = sb + C::OFF_K, sV = sb + C::OFF_V, sQ = sb + C::OFF_Q, sDO = sb + C::OFF_DO;
   const uint32_t sDSt = sb + C::OFF_DST;

@@ -250,6 +250,46 @@ int get_chunk_tables(int dev, int heads, int N, int causal, int sched, int ctas,
   return DASH_OK;
 }
 
+// The host-buffer path's parts of a SHIFT_PAIRS launch: the half table (one unit per
+// KV pair, ctas / 2 slots) split by heads, each part validated and expanded to the
+// grid's table, so every part keeps the whole launch's dQ orders.
+std::map<std::tuple<int, int, int, int, int>, std::vector<DevTable>> g_pair_chunk_tables;
+
+int get_pair_chunk_tables(int dev, int heads, int N, int ctas, int chunk,
+                          std::vector<DevTable>** out) {
+  auto key = std::make_tuple(dev, heads, N, ctas, chunk);
+  auto itc = g_pair_chunk_tables.find(key);
+  if (itc != g_pair_chunk_tables.end()) {
+    *out = &itc->second;
+    return DASH_OK;
+  }
+  dash::Table half;
+  std::string err;
+  if (!dash::build_table(heads, N, 0, dash::SHIFT_PAIRS, ctas / 2, &half, &err))
+    return DASH_ERR_UNSUPPORTED;
+  if (!dash::validate_table(half, &err)) return DASH_ERR_SCHEDULE;
+  std::vector<DevTable> parts;
+  int rc = DASH_OK;
+  for (int h0 = 0; h0 < heads && rc == DASH_OK; h0 += chunk) {
+    dash::Table t, g;
+    const int h1 = h0 + chunk < heads ? h0 + chunk : heads;
+    if (!dash::split_table(half, h0, h1, &t) || !dash::validate_table(t, &err) ||
+        !dash::expand_pair_table(t, &g)) {
+      rc = DASH_ERR_SCHEDULE;
+      break;
+    }
+    DevTable d;
+    if ((rc = upload_table(g, &d, 1)) == DASH_OK) parts.push_back(d);
+  }
+  if (rc) {
+    for (DevTable& d : parts) free_table(&d);
+    return rc;
+  }
+  auto res = g_pair_chunk_tables.emplace(key, std::move(parts));
+  *out = &res.first->second;
+  return DASH_OK;
+}
+
 // A deliberately broken table for failure-detection tests: every partial of
 // dQ block (head 0, Q tile 0) moves one position later, so its first position
 // is never filled and the waits on it must run out.  All indices stay in range.
@@ -602,7 +642,8 @@ int pair_ctas(int dev, int* out) {
 
 int launch_bwd_pairs(const void* q, const void* k, const void* v, const void* o,
                      const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
-                     int H, int S, cudaStream_t stream, int dev) {
+                     int H, int S, cudaStream_t stream, int dev,
+                     const DevTable* tab_override = nullptr) {
   constexpr int D = 64;
   using C = BwdCfg<D>;
   const int N = S / 128;
@@ -618,7 +659,9 @@ int launch_bwd_pairs(const void* q, const void* k, const void* v, const void* o,
     if ((rc = pair_ctas(dev, &ctas))) return rc;
     auto key = std::make_tuple(dev, B * H, N, 0, (int)dash::SHIFT_PAIRS, ctas, 1, 1);
     auto itb = g_tables.find(key);
-    if (itb != g_tables.end()) {
+    if (tab_override) {
+      tab = const_cast<DevTable*>(tab_override);
+    } else if (itb != g_tables.end()) {
       tab = &itb->second;
     } else {
       dash::Table half, t;
@@ -792,8 +835,13 @@ int host_bwd(const void* q, const void* k, const void* v, const void* o, const v
              const float* lse, void* dq, void* dk, void* dv, int B, int H, int S, int causal,
              int sched, cudaStream_t stream, int dev) {
   const int BH = B * H, N = S / 128;
+  const bool pairs = (sched == DASH_SCHED_SHIFT_PAIRS);  // CTA pairs (D = 64 only)
   int ctas = 0;
-  int rc = num_ctas_for<D, kAtomic>(dev, &ctas);
+  int rc;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    rc = pairs ? pair_ctas(dev, &ctas) : num_ctas_for<D, kAtomic>(dev, &ctas);
+  }
   if (rc) return rc;
   // the parts hold whole units of the launch's table, so its interleaved heads stay
   // together and every dQ block keeps the order dash_attn_bwd gives it
@@ -806,7 +854,9 @@ int host_bwd(const void* q, const void* k, const void* v, const void* o, const v
   HostPipe* hp = nullptr;
   {
     std::lock_guard<std::mutex> lk(g_mu);
-    if ((rc = get_chunk_tables(dev, BH, N, causal, sched, ctas, chunk, il, &parts))) return rc;
+    if ((rc = pairs ? get_pair_chunk_tables(dev, BH, N, ctas, chunk, &parts)
+                    : get_chunk_tables(dev, BH, N, causal, sched, ctas, chunk, il, &parts)))
+      return rc;
     if ((rc = get_pipe(dev, stream, 2 * slot_bytes, &hp))) return rc;
   }
   // the copy streams start after whatever the caller queued before this call
@@ -841,9 +891,11 @@ int host_bwd(const void* q, const void* k, const void* v, const void* o, const v
     // compute, once the inputs are in and the results of part c - 2 are out
     DASH_CUDA(cudaStreamWaitEvent(stream, hp->in_ready[slot], 0));
     if (c >= 2) DASH_CUDA(cudaStreamWaitEvent(stream, hp->out_done[slot], 0));
-    if ((rc = launch_bwd<D, kAtomic>(din[0], din[1], din[2], din[3], din[4], dlse, dout3[0],
-                                     dout3[1], dout3[2], 1, nh, S, causal, sched, stream, dev,
-                                     nullptr, 0, &(*parts)[c])))
+    if ((rc = pairs ? launch_bwd_pairs(din[0], din[1], din[2], din[3], din[4], dlse, dout3[0],
+                                       dout3[1], dout3[2], 1, nh, S, stream, dev, &(*parts)[c])
+                    : launch_bwd<D, kAtomic>(din[0], din[1], din[2], din[3], din[4], dlse,
+                                             dout3[0], dout3[1], dout3[2], 1, nh, S, causal,
+                                             sched, stream, dev, nullptr, 0, &(*parts)[c])))
       return rc;
     DASH_CUDA(cudaEventRecord(hp->comp_done[slot], stream));
     // results of part c
@@ -916,7 +968,7 @@ int dash_set_head_interleave(int mode) {
 int dash_bwd_head_interleave(int num_ctas, int D, int schedule, int n_heads, int S, int causal,
                              int* heads_per_unit) {
   if (!heads_per_unit || num_ctas < 1 || n_heads < 1 || (D != 64 && D != 128) || S < 128 ||
-      S % 128 != 0 || schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_ATOMIC ||
+      S % 128 != 0 || schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_SHIFT_PAIRS ||
       (causal != 0 && causal != 1))
     return DASH_ERR_INVALID_ARG;
   *heads_per_unit =
@@ -932,9 +984,11 @@ int dash_set_dq_chain_mode(int mode) {
 
 int dash_dq_chain_uses_red(int schedule, int S, int D, int heads_per_unit, int* red) {
   if (!red || S < 128 || S % 128 != 0 || schedule < DASH_SCHED_NAIVE_ASC ||
-      schedule > DASH_SCHED_ATOMIC || heads_per_unit < 1 || (D != 64 && D != 128))
+      schedule > DASH_SCHED_SHIFT_PAIRS || heads_per_unit < 1 || (D != 64 && D != 128))
     return DASH_ERR_INVALID_ARG;
-  *red = (schedule != DASH_SCHED_ATOMIC && red_chain_for(schedule, S / 128, D, heads_per_unit))
+  // the atomic variant has no chains; CTA pairs always load, add and store
+  *red = (schedule != DASH_SCHED_ATOMIC && schedule != DASH_SCHED_SHIFT_PAIRS &&
+          red_chain_for(schedule, S / 128, D, heads_per_unit))
              ? 1 : 0;
   return DASH_OK;
 }
@@ -977,8 +1031,9 @@ int dash_attn_bwd_gqa_split(const void* q, const void* k, const void* v, const v
     if (split < 0 || (split > 0 && H > 0 &&
                       ((split & (split - 1)) != 0 || (H / Hkv) % split != 0)))
       return DASH_ERR_INVALID_ARG;
-    if (schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_ATOMIC)
+    if (schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_SHIFT_PAIRS)
       return DASH_ERR_INVALID_ARG;
+    if (schedule == DASH_SCHED_SHIFT_PAIRS) return DASH_ERR_UNSUPPORTED;  // dash_attn_bwd only
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
         !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
       return DASH_ERR_INVALID_ARG;
@@ -1053,8 +1108,9 @@ int dash_attn_bwd_host(const void* q, const void* k, const void* v, const void* 
     int rc = check_shape(B, H, S, D);
     if (rc) return rc;
     if (causal != 0 && causal != 1) return DASH_ERR_INVALID_ARG;
-    if (schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_ATOMIC)
+    if (schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_SHIFT_PAIRS)
       return DASH_ERR_INVALID_ARG;
+    if (schedule == DASH_SCHED_SHIFT_PAIRS && D != 64) return DASH_ERR_UNSUPPORTED;
     if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return DASH_ERR_INVALID_ARG;
     if (!dash::schedule_supported(schedule, S / 128, causal)) return DASH_ERR_UNSUPPORTED;
     if (B == 0 || H == 0) return DASH_OK;
@@ -1194,8 +1250,9 @@ int dash_trace_bwd(const void* q, const void* k, const void* v, const void* o, c
     int rc = check_shape(B, H, S, D);
     if (rc) return rc;
     if (causal != 0 && causal != 1) return DASH_ERR_INVALID_ARG;
-    if (schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_ATOMIC)
+    if (schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_SHIFT_PAIRS)
       return DASH_ERR_INVALID_ARG;
+    if (schedule == DASH_SCHED_SHIFT_PAIRS) return DASH_ERR_UNSUPPORTED;  // dash_attn_bwd only
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
         !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !host_trace ||
         !num_ctas || !rows_per_cta)

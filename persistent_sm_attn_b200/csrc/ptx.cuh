@@ -51,6 +51,7 @@ enum : unsigned {
   ERR_WHERE_TICKET = 1u << 1,
   ERR_WHERE_PIPE = 1u << 2,
   ERR_MISALIGNED = 1u << 3,  // shared-memory base not 1 KiB aligned: nothing was computed
+  ERR_NO_CLUSTER = 1u << 4,  // a CTA-pair kernel launched without its pairs: nothing computed
 };
 
 // Bounded wait.  Returns false after limit_ns, recording the timeout in the
@@ -82,6 +83,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
 
 // ---------------------------------------------------------------- clusters
 // (CTA pairs that read each other's shared memory; launched with a cluster of 2)
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));

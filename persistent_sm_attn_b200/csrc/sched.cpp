@@ -259,6 +259,7 @@ bool split_table(const Table& full, int h0, int h1, Table* out) {
   t.schedule = full.schedule;
   t.num_ctas = full.num_ctas;
   t.group = full.group;
+  t.kv_units = full.kv_units;
   t.cta_off.assign(full.num_ctas + 1, 0);
   for (int c = 0; c < full.num_ctas; ++c) {
     for (int i = full.cta_off[c]; i < full.cta_off[c + 1]; ++i) {

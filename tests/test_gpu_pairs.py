@@ -38,3 +38,30 @@ def test_pairs_refuse_other_shapes(S, D, causal):
     with pytest.raises(binding.DashError):
         binding.dash_attn_bwd(case["q"], case["k"], case["v"], case["o"], case["do"],
                               case["lse"], causal, "shift_pairs")
+
+
+def test_host_path_gives_the_same_bits():
+    """The host-buffer path runs each part on a slice of the same pair table."""
+    G.need_cuda()
+    case = G.make_case(2, 8, 1024, 64, False, seed=19)
+    want = G.bwd(case, "shift_pairs")
+    host = [case[n].cpu().pin_memory() for n in ("q", "k", "v", "o", "do", "lse")]
+    got = binding.dash_attn_bwd_host(*host, False, "shift_pairs")
+    assert binding.dash_attn_sync_status() == 0
+    for a, b in zip(want, got):
+        assert torch.equal(a.cpu(), b)
+
+
+def test_other_entry_points_refuse_pairs():
+    """The no-allocation and grouped-query entry points refuse SHIFT_PAIRS
+    (DASH_ERR_UNSUPPORTED)."""
+    G.need_cuda()
+    case = G.make_case(1, 2, 512, 64, False, seed=9)
+    args = (case["q"], case["k"], case["v"], case["o"], case["do"], case["lse"], False,
+            "shift_pairs")
+    for call in (lambda: binding.dash_attn_bwd_noalloc(*args, *[torch.empty_like(case["q"])
+                                                               for _ in range(3)]),
+                 lambda: binding.dash_attn_bwd_gqa(*args)):
+        with pytest.raises(binding.DashError) as e:
+            call()
+        assert e.value.status == 2, e.value   # DASH_ERR_UNSUPPORTED
