@@ -65,3 +65,20 @@ def test_other_entry_points_refuse_pairs():
         with pytest.raises(binding.DashError) as e:
             call()
         assert e.value.status == 2, e.value   # DASH_ERR_UNSUPPORTED
+
+
+def test_pairs_repeat_at_a_larger_shape():
+    """20 launches at B=2 H=16 S=4096 D=64 (several rounds of CTA pairs) give the same
+    bits, and agree with the shift schedule to within rounding."""
+    G.need_cuda()
+    case = G.make_case(2, 16, 4096, 64, False, seed=808)
+    first = G.bwd(case, "shift_pairs")
+    for _ in range(19):
+        again = G.bwd(case, "shift_pairs")
+        for a, b in zip(first, again):
+            assert torch.equal(a, b)
+    plain = G.bwd(case, "shift")
+    for a, b in zip(first, plain):
+        rel = (torch.linalg.vector_norm(a.float() - b.float()) /
+               torch.linalg.vector_norm(b.float())).item()
+        assert rel < 4e-3
