@@ -205,7 +205,7 @@ constexpr int kTraceEvents = 16;
 // grants them, instead of a load-add-store from the SM.  The additions and their order
 // are the same, so the results are bitwise the same; only the traffic and the latency
 // of each link differ.
-// kPair (D = 64, deterministic, load-add-store chains): the grid runs in clusters of two
+// kPair (D = 64, deterministic): the grid runs in clusters of two
 // CTAs, 2i and 2i + 1, with a SHIFT_PAIRS table: the pair runs KV tiles 2m and 2m + 1 over
 // the same Q tiles at the same steps.  Each CTA's reducers add the two staged dQ partials
 // of a step (its own, and the peer's read over distributed shared memory) for half of
@@ -220,7 +220,7 @@ __global__ void __launch_bounds__(512, 1)
                     const __grid_constant__ CUtensorMap tmC, const BwdParams p) {
   using namespace dev;
   using C = BwdCfg<D>;
-  static_assert(!kPair || (D == 64 && !kAtomic && !kRed), "CTA pairs: D = 64, load-add-store");
+  static_assert(!kPair || (D == 64 && !kAtomic), "CTA pairs: D = 64, deterministic");
   constexpr int ST = C::kStagesQ, SD = C::kStagesDO;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t sb = smem_u32(smem_raw);
@@ -1157,7 +1157,7 @@ __global__ void __launch_bounds__(512, 1)
               ticket_wait(p.tickets + unit, (uint32_t)idx, ~0u);
               if (threadIdx.x == 256) trace(it, 6);
 #pragma unroll
-              for (int c4 = 0; c4 < NV; ++c4)
+              for (int c4 = 0; c4 < NA; ++c4)
                 red_add_f4(accp + c4 * 128 + r,
                            make_float4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]));
             } else {

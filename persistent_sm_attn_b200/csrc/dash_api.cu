@@ -413,6 +413,8 @@ bool red_chain_for(int sched, int N, int D, int heads_per_unit) {
   const int m = g_chain_mode.load();
   if (m == 1) return true;
   if (m == 2) return false;
+  // CTA pairs: red measured slower (2-5 % at D = 64, full 4k to 16k)
+  if (sched == DASH_SCHED_SHIFT_PAIRS) return false;
   return ((sched == DASH_SCHED_DESCENDING || sched == DASH_SCHED_NAIVE_ASC) && N >= 64) ||
          (D == 64 && heads_per_unit > 1);
 }
@@ -615,10 +617,13 @@ int pair_ctas(int dev, int* out) {
   }
   using C = BwdCfg<64>;
   auto kern = dash::dash_bwd_kernel<64, false, false, false, true>;
-  DASH_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes));
-  cudaFuncAttributes fa;
-  DASH_CUDA(cudaFuncGetAttributes(&fa, kern));
-  if (fa.numRegs != C::kLaunchRegs) return DASH_ERR_UNSUPPORTED;
+  for (auto k2 : {kern, dash::dash_bwd_kernel<64, false, false, true, true>}) {
+    DASH_CUDA(cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   C::kSmemBytes));
+    cudaFuncAttributes fa;
+    DASH_CUDA(cudaFuncGetAttributes(&fa, k2));
+    if (fa.numRegs != C::kLaunchRegs) return DASH_ERR_UNSUPPORTED;
+  }
   int sms = 0;
   DASH_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
   cudaLaunchConfig_t cfg = {};
@@ -725,8 +730,12 @@ int launch_bwd_pairs(const void* q, const void* k, const void* v, const void* o,
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   if (!prof_record(1, &ev, stream)) return DASH_ERR_CUDA;
-  DASH_CUDA(cudaLaunchKernelEx(&cfg, dash::dash_bwd_kernel<64, false, false, false, true>, tq,
-                               tk, tv, tdo, tc, p));
+  // middle links with red in L2 only where the chain mode forces it (bitwise the same)
+  const bool red = red_chain_for(DASH_SCHED_SHIFT_PAIRS, N, D, 1);
+  DASH_CUDA(cudaLaunchKernelEx(&cfg,
+                               red ? dash::dash_bwd_kernel<64, false, false, true, true>
+                                   : dash::dash_bwd_kernel<64, false, false, false, true>,
+                               tq, tk, tv, tdo, tc, p));
   if (!prof_record(2, &ev, stream) || !prof_record(3, &ev, stream)) return DASH_ERR_CUDA;
   if (g_prof_on.load()) {
     std::lock_guard<std::mutex> lk(g_prof_mu);
@@ -986,9 +995,8 @@ int dash_dq_chain_uses_red(int schedule, int S, int D, int heads_per_unit, int* 
   if (!red || S < 128 || S % 128 != 0 || schedule < DASH_SCHED_NAIVE_ASC ||
       schedule > DASH_SCHED_SHIFT_PAIRS || heads_per_unit < 1 || (D != 64 && D != 128))
     return DASH_ERR_INVALID_ARG;
-  // the atomic variant has no chains; CTA pairs always load, add and store
-  *red = (schedule != DASH_SCHED_ATOMIC && schedule != DASH_SCHED_SHIFT_PAIRS &&
-          red_chain_for(schedule, S / 128, D, heads_per_unit))
+  // the atomic variant has no chains
+  *red = (schedule != DASH_SCHED_ATOMIC && red_chain_for(schedule, S / 128, D, heads_per_unit))
              ? 1 : 0;
   return DASH_OK;
 }

@@ -18,13 +18,16 @@ def test_default_choice():
     assert f("sym_shift", 16384, 64, 2) and f("shift", 1024, 64, 4) and f("descending", 512, 64, 2)
     assert not f("sym_shift", 16384, 128, 2) and not f("sym_shift", 16384, 64, 1)
     assert not f("atomic", 16384, 64, 2)
+    # CTA pairs keep the load-add-store unless red is forced
+    assert not f("shift_pairs", 16384, 64, 1)
 
 
 def test_forced_modes():
     f = binding.dash_dq_chain_uses_red
     try:
         binding.dash_set_dq_chain_mode(1)
-        assert all(f(s, 256) for s in ("naive_asc", "descending", "shift", "sym_shift"))
+        assert all(f(s, 256) for s in ("naive_asc", "descending", "shift", "sym_shift",
+                                      "shift_pairs"))
         assert not f("atomic", 256)
         binding.dash_set_dq_chain_mode(2)
         assert not any(f(s, 16384) for s in ("naive_asc", "descending", "shift", "sym_shift"))
