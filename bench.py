@@ -78,7 +78,9 @@ def _workload(args):
     b, h, s, d, mask = args.shape.split(",")
     B, H, S, D, causal = int(b), int(h), int(s), int(d), mask.strip() == "causal"
     N = S // 128
-    if causal:
+    if causal and D == 64 and N % 4 == 0:
+        scheds = ("sym_shift", "sym_shift_pairs", "descending")
+    elif causal:
         scheds = ("sym_shift", "descending") if N % 2 == 0 else ("descending",)
     elif D == 64 and N % 2 == 0:
         scheds = ("shift", "shift_pairs", "descending")
@@ -348,7 +350,7 @@ def run_ours(args):
             "dq_chain": ("red" if binding.dash_dq_chain_uses_red(sched, w.S, w.D, il)
                          else "load-add-store") if sched != "atomic" else None,
             "heads_per_unit": il if not gqa else None,
-            "slot_placement": ("cta_pairs" if sched == "shift_pairs" else
+            "slot_placement": ("cta_pairs" if sched in ("shift_pairs", "sym_shift_pairs") else
                                "sm_id" if binding.dash_slot_placement_by_smid(w.S)
                                else "launch_order"),
             "roofline": {"bound": "tensor", "achieved": round(kern, 2), "peak": peak,

@@ -56,7 +56,8 @@ typedef enum {
   DASH_SCHED_SHIFT = 2,       /* §2.2.B full masks: cyclic shift, conflict-free order  */
   DASH_SCHED_SYM_SHIFT = 3,   /* §2.2.B causal masks: KV i and N-1-i folded, 2 phases  */
   DASH_SCHED_ATOMIC = 4,      /* §1 nondeterministic counterpart: fp32 atomic dQ adds  */
-  DASH_SCHED_SHIFT_PAIRS = 5  /* full masks, even N: CTA pairs pre-sum dQ (see below)  */
+  DASH_SCHED_SHIFT_PAIRS = 5, /* full masks, even N: CTA pairs pre-sum dQ (see below)  */
+  DASH_SCHED_SYM_SHIFT_PAIRS = 6 /* causal masks, N % 4 == 0: the same CTA pairs      */
 } dash_schedule_t;
 
 typedef enum {
@@ -366,21 +367,29 @@ long long dash_sched_table(int n_heads, int N, int causal, int schedule, int num
  * head over the same Q tiles at the same steps, Q tile m + t mod N at step t, and the
  * two dQ partials of a step are added together before the ordered accumulation, so a
  * dQ block receives N / 2 contributions, in (round, step) order.  Full mask, N even.
- * For this schedule dash_sched_table returns the half table, one row per pair of KV
+ * DASH_SCHED_SYM_SHIFT_PAIRS is the causal counterpart: KV pair m and Q pair j (Q tiles
+ * 2j and 2j + 1) form a pair-tile, present when j >= m; the half table runs
+ * DASH_SCHED_SYM_SHIFT over the N / 2 pair-tiles, each pair-tile as two steps (Q tile 2j,
+ * then 2j + 1).  On a diagonal pair-tile the step (KV 2m + 1, Q 2m) lies wholly above the
+ * diagonal: that CTA computes it as zeros, so both CTAs keep the same steps.  A dQ block
+ * q receives q / 2 + 1 contributions.  Causal mask, N a multiple of 4.
+ * For these schedules dash_sched_table returns the half table, one row per pair of KV
  * tiles (kv = m, num_ctas counting CTA pairs); dash_sched_table_pairs returns the grid's
- * table for num_ctas CTAs (even): rows as for dash_sched_table, slot 2i with KV tile 2m
- * and slot 2i + 1 with KV tile 2m + 1, both with the pair's Q tiles and positions.
- * Returns the number of rows, or -DASH_ERR_INVALID_ARG (odd num_ctas),
+ * table for num_ctas CTAs (even), SHIFT_PAIRS for causal = 0 and SYM_SHIFT_PAIRS for
+ * causal = 1: rows as for dash_sched_table, slot 2i with KV tile 2m and slot 2i + 1 with
+ * KV tile 2m + 1, both with the pair's Q tiles and positions.  Returns the number of
+ * rows, or -DASH_ERR_INVALID_ARG (odd num_ctas, causal not 0 or 1),
  * -DASH_ERR_UNSUPPORTED or -DASH_ERR_SCHEDULE.
- * The backward runs it through dash_attn_bwd only, at D = 64 (each CTA stages its dQ
+ * The backward runs them through dash_attn_bwd only, at D = 64 (each CTA stages its dQ
  * partial in shared memory, and the pair is a thread-block cluster of two CTAs that read
  * each other's staged partial): each CTA adds the two partials for half of the columns
- * and accumulates that half in order.  Other head dims, causal masks and odd N return
- * DASH_ERR_UNSUPPORTED.  dash_attn_bwd_host takes it too (its parts are slices of the
- * same table, so the bits are dash_attn_bwd's); the grouped-query, no-allocation and
- * trace entry points return DASH_ERR_UNSUPPORTED.
+ * and accumulates that half in order.  Other head dims, the other mask and unsupported
+ * N return DASH_ERR_UNSUPPORTED.  dash_attn_bwd_host takes them too (its parts are slices
+ * of the same table, so the bits are dash_attn_bwd's); the grouped-query, no-allocation
+ * and trace entry points return DASH_ERR_UNSUPPORTED.
  */
-long long dash_sched_table_pairs(int n_heads, int N, int num_ctas, int* rows, long long cap);
+long long dash_sched_table_pairs(int n_heads, int N, int causal, int num_ctas, int* rows,
+                                 long long cap);
 
 /*
  * The part of that table covering heads [h0, h1) (0 <= h0 < h1 <= n_heads), as the

@@ -36,12 +36,22 @@ Schedules (names follow the pages):
   pairs folds into an N/2 x (N+1) rectangle, run in two phases: the dense
   lower-left rectangle (Q in [N/2, N) x KV in [0, N/2)) and then the folded
   upper triangle.  Accumulation follows (phase, step).  Requires even N.
+* ``sym_shift_pairs`` -- the CTA pairs of ``shift_pairs`` under the causal mask
+  (this library's construction, like ``shift_pairs``): KV pair m (KV tiles 2m,
+  2m+1) against Q pair j (Q tiles 2j, 2j+1) is a pair-tile, present when
+  j >= m; ``sym_shift`` runs over the N/2 x N/2 pair-tiles, and each visited
+  pair-tile becomes two steps, Q tile 2j and then 2j+1.  A unit stands for KV
+  pairs, written as m; Q tile q >= 2m is visited by KV pair m, so dQ block q
+  receives q//2 + 1 pre-summed contributions, in (round, step) order.  On a
+  diagonal pair-tile the step (KV 2m+1, Q 2m) lies above the diagonal and adds
+  nothing.  Causal mask, N a multiple of 4.
 """
 from __future__ import annotations
 
 NAIVE_ASC, DESCENDING, SHIFT, SYM_SHIFT = "naive_asc", "descending", "shift", "sym_shift"
 ALL = (NAIVE_ASC, DESCENDING, SHIFT, SYM_SHIFT)
-SHIFT_PAIRS = "shift_pairs"  # units stand for KV pairs; not in ALL (its units differ in kind)
+# units stand for KV pairs; not in ALL (their units differ in kind)
+SHIFT_PAIRS, SYM_SHIFT_PAIRS = "shift_pairs", "sym_shift_pairs"
 
 
 def supported(name: str, N: int, causal: bool) -> bool:
@@ -52,6 +62,8 @@ def supported(name: str, N: int, causal: bool) -> bool:
         return causal and N % 2 == 0
     if name == SHIFT_PAIRS:
         return not causal and N % 2 == 0
+    if name == SYM_SHIFT_PAIRS:
+        return causal and N % 4 == 0
     return name in (NAIVE_ASC, DESCENDING)
 
 
@@ -76,6 +88,10 @@ def units(name: str, N: int, causal: bool):
         # unit m: the KV pair (2m, 2m+1), written as m
         for m in range(N // 2):
             out.append([(m, (m + t) % N) for t in range(N)])
+    elif name == SYM_SHIFT_PAIRS:
+        # pair-tile (m, j) of the half-size symmetric shift -> steps (m, 2j), (m, 2j+1)
+        for seq in units(SYM_SHIFT, N // 2, True):
+            out.append([(m, 2 * j + b) for (m, j) in seq for b in (0, 1)])
     elif name == SYM_SHIFT:
         h = N // 2
         for k in range(h):

@@ -15,7 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libdash_attn.so")
 
 SCHEDULES = {"naive_asc": 0, "descending": 1, "shift": 2, "sym_shift": 3, "atomic": 4,
-             "shift_pairs": 5}
+             "shift_pairs": 5, "sym_shift_pairs": 6}
 STATUS = {0: "DASH_OK", 1: "DASH_ERR_INVALID_ARG", 2: "DASH_ERR_UNSUPPORTED", 3: "DASH_ERR_CUDA",
           4: "DASH_ERR_TIMEOUT", 5: "DASH_ERR_OOM", 6: "DASH_ERR_SCHEDULE"}
 
@@ -86,7 +86,7 @@ def load(path: str | None = None):
     lib.dash_sched_table_part.restype = ll
     lib.dash_sched_table_gqa.argtypes = [i, i, i, i, i, i, vp, ll]
     lib.dash_sched_table_gqa.restype = ll
-    lib.dash_sched_table_pairs.argtypes = [i, i, i, vp, ll]
+    lib.dash_sched_table_pairs.argtypes = [i, i, i, i, vp, ll]
     lib.dash_sched_table_pairs.restype = ll
     lib.dash_sched_simulate.argtypes = [i, i, i, i, i, d, d, i, i, P(d), P(d), P(d), P(ll)]
     lib.dash_sched_simulate_gqa.argtypes = [i, i, i, i, i, i, d, d, i, i, P(d), P(d), P(d),
@@ -403,16 +403,16 @@ def dash_sched_table_gqa(n_heads: int, group: int, N: int, causal: bool, schedul
     return [tuple(flat[6 * r: 6 * r + 6]) for r in range(n)]
 
 
-def dash_sched_table_pairs(n_heads: int, N: int, num_ctas: int):
-    """Rows (cta, head, kv, q, position, chain_index) of the grid's SHIFT_PAIRS table for
-    num_ctas CTAs (even): CTAs 2i and 2i + 1 run KV tiles 2m and 2m + 1 over the same Q
-    tiles with the same positions."""
+def dash_sched_table_pairs(n_heads: int, N: int, causal: bool, num_ctas: int):
+    """Rows (cta, head, kv, q, position, chain_index) of the grid's CTA-pair table
+    (SHIFT_PAIRS, or SYM_SHIFT_PAIRS when causal) for num_ctas CTAs (even): CTAs 2i and
+    2i + 1 run KV tiles 2m and 2m + 1 over the same Q tiles with the same positions."""
     lib = load()
-    n = lib.dash_sched_table_pairs(n_heads, N, num_ctas, None, 0)
+    n = lib.dash_sched_table_pairs(n_heads, N, int(causal), num_ctas, None, 0)
     if n < 0:
         raise DashError(int(-n), "dash_sched_table_pairs")
     buf = (ctypes.c_int * (6 * max(n, 1)))()
-    lib.dash_sched_table_pairs(n_heads, N, num_ctas, buf, n)
+    lib.dash_sched_table_pairs(n_heads, N, int(causal), num_ctas, buf, n)
     flat = list(buf)
     return [tuple(flat[6 * r: 6 * r + 6]) for r in range(n)]
 

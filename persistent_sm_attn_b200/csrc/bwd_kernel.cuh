@@ -206,13 +206,15 @@ constexpr int kTraceEvents = 16;
 // are the same, so the results are bitwise the same; only the traffic and the latency
 // of each link differ.
 // kPair (D = 64, deterministic): the grid runs in clusters of two
-// CTAs, 2i and 2i + 1, with a SHIFT_PAIRS table: the pair runs KV tiles 2m and 2m + 1 over
-// the same Q tiles at the same steps.  Each CTA's reducers add the two staged dQ partials
-// of a step (its own, and the peer's read over distributed shared memory) for half of
-// the columns, CTA 2i + r taking columns [32r, 32r + 32), and run the ordered
-// accumulation of that half: one contribution per pair and step, so N / 2 per block and
-// half the accumulator bytes per CTA.  Both CTAs free a staged tile only after both
-// have read it.
+// CTAs, 2i and 2i + 1, with a SHIFT_PAIRS or SYM_SHIFT_PAIRS table: the pair runs KV tiles
+// 2m and 2m + 1 over the same Q tiles at the same steps.  Each CTA's reducers add the two
+// staged dQ partials of a step (its own, and the peer's read over distributed shared
+// memory) for half of the columns, CTA 2i + r taking columns [32r, 32r + 32), and run the
+// ordered accumulation of that half: one contribution per pair and step, so N / 2 per
+// block (q / 2 + 1 for block q under the causal mask) and half the accumulator bytes per
+// CTA.  Both CTAs free a staged tile only after both have read it.  Under the causal mask
+// CTA 2i + 1 meets one tile wholly above the diagonal per diagonal pair-tile (KV 2m + 1,
+// Q 2m): every probability of it is masked to zero, so its partials are zeros.
 template <int D, bool kAtomic, bool kTrace = false, bool kRed = false, bool kPair = false>
 __global__ void __launch_bounds__(512, 1)
     dash_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -739,8 +741,9 @@ __global__ void __launch_bounds__(512, 1)
         for (int t = 0; t < n_pairs(ch.w); ++t, ++it) {
           const uint32_t w = p.pairs[ch.z + t];
           const int q = (int)(w & 0xffffu), pos = (int)(w >> 16);
-          // CTA pairs: N / 2 contributions per block, tickets per (block, half, chain)
-          const int ncontrib = kPair ? N / 2 : (p.causal ? q + 1 : N);
+          // CTA pairs: N / 2 (causal: q / 2 + 1) contributions per block, tickets per
+          // (block, half, chain)
+          const int ncontrib = kPair ? (p.causal ? q / 2 + 1 : N / 2) : (p.causal ? q + 1 : N);
           if (pos == ncontrib - 1) continue;  // the last contributor writes dQ itself
           const long long unit =
               kPair ? (((long long)ch.x * N + q) * 2 + prank) * 2 + (pos & 1)
@@ -814,7 +817,9 @@ __global__ void __launch_bounds__(512, 1)
           wait(S_FULL(it), s_phase(it));
           if (tracer) trace(it, 3);
           tc_fence_after();
-          const int lim_c = (p.causal && q == ch.y) ? r : -1;
+          // causal: on the diagonal tile Q column qc sees KV row r only if qc >= r; a CTA
+          // pair's tile above the diagonal (q < kv) is masked whole
+          const int lim_c = !p.causal ? -1 : q == ch.y ? r : (kPair && q < ch.y) ? 128 : -1;
           // chunks 2, 3, 0, 1 into columns 64, 80, 96, 112: each store lands on columns
           // this thread has already read
 #pragma unroll 1
@@ -983,8 +988,8 @@ __global__ void __launch_bounds__(512, 1)
       for (int t = 0; t < n_pairs(ch.w); ++t, ++it) {
         const uint32_t w = p.pairs[ch.z + t];
         const int q = (int)(w & 0xffffu), pos = (int)(w >> 16);
-        // CTA pairs: N / 2 (pre-summed) contributions per block
-        const int ncontrib = kPair ? N / 2 : (p.causal ? q + 1 : N);
+        // CTA pairs: N / 2 (causal: q / 2 + 1) pre-summed contributions per block
+        const int ncontrib = kPair ? (p.causal ? q / 2 + 1 : N / 2) : (p.causal ? q + 1 : N);
         const bool last = (pos == ncontrib - 1);
         float a[D];
         if constexpr (kPair) {

@@ -250,14 +250,17 @@ int get_chunk_tables(int dev, int heads, int N, int causal, int sched, int ctas,
   return DASH_OK;
 }
 
-// The host-buffer path's parts of a SHIFT_PAIRS launch: the half table (one unit per
-// KV pair, ctas / 2 slots) split by heads, each part validated and expanded to the
-// grid's table, so every part keeps the whole launch's dQ orders.
-std::map<std::tuple<int, int, int, int, int>, std::vector<DevTable>> g_pair_chunk_tables;
+// The host-buffer path's parts of a CTA-pair launch (SHIFT_PAIRS, or SYM_SHIFT_PAIRS when
+// causal): the half table (one unit per KV pair, ctas / 2 slots) split by heads, each
+// part validated and expanded to the grid's table, so every part keeps the whole
+// launch's dQ orders.
+std::map<std::tuple<int, int, int, int, int, int>, std::vector<DevTable>> g_pair_chunk_tables;
 
-int get_pair_chunk_tables(int dev, int heads, int N, int ctas, int chunk,
+int pair_sched_of(int causal) { return causal ? dash::SYM_SHIFT_PAIRS : dash::SHIFT_PAIRS; }
+
+int get_pair_chunk_tables(int dev, int heads, int N, int causal, int ctas, int chunk,
                           std::vector<DevTable>** out) {
-  auto key = std::make_tuple(dev, heads, N, ctas, chunk);
+  auto key = std::make_tuple(dev, heads, N, causal, ctas, chunk);
   auto itc = g_pair_chunk_tables.find(key);
   if (itc != g_pair_chunk_tables.end()) {
     *out = &itc->second;
@@ -265,7 +268,7 @@ int get_pair_chunk_tables(int dev, int heads, int N, int ctas, int chunk,
   }
   dash::Table half;
   std::string err;
-  if (!dash::build_table(heads, N, 0, dash::SHIFT_PAIRS, ctas / 2, &half, &err))
+  if (!dash::build_table(heads, N, causal, pair_sched_of(causal), ctas / 2, &half, &err))
     return DASH_ERR_UNSUPPORTED;
   if (!dash::validate_table(half, &err)) return DASH_ERR_SCHEDULE;
   std::vector<DevTable> parts;
@@ -373,6 +376,9 @@ int make_tmap_cols(CUtensorMap* m, const void* base, long long rows) {
 
 // ------------------------------------------------------------------ helpers
 bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool pair_sched(int schedule) {
+  return schedule == DASH_SCHED_SHIFT_PAIRS || schedule == DASH_SCHED_SYM_SHIFT_PAIRS;
+}
 
 int check_shape(int B, int H, int S, int D) {
   if (B < 0 || H < 0 || S < 0 || D < 0) return DASH_ERR_INVALID_ARG;
@@ -414,7 +420,7 @@ bool red_chain_for(int sched, int N, int D, int heads_per_unit) {
   if (m == 1) return true;
   if (m == 2) return false;
   // CTA pairs: red measured slower (2-5 % at D = 64, full 4k to 16k)
-  if (sched == DASH_SCHED_SHIFT_PAIRS) return false;
+  if (pair_sched(sched)) return false;
   return ((sched == DASH_SCHED_DESCENDING || sched == DASH_SCHED_NAIVE_ASC) && N >= 64) ||
          (D == 64 && heads_per_unit > 1);
 }
@@ -606,7 +612,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
 }
 
 // ------------------------------------------------------------------ CTA pairs
-// SHIFT_PAIRS at D = 64: the kernel runs in clusters of two CTAs, with as many
+// SHIFT_PAIRS / SYM_SHIFT_PAIRS at D = 64: the kernel runs in clusters of two CTAs, with as many
 // clusters as fit on the device at once (cooperative, so all are resident).
 std::map<int, int> g_pair_ctas;  // device -> CTAs of the pair launch
 int pair_ctas(int dev, int* out) {
@@ -647,7 +653,7 @@ int pair_ctas(int dev, int* out) {
 
 int launch_bwd_pairs(const void* q, const void* k, const void* v, const void* o,
                      const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
-                     int H, int S, cudaStream_t stream, int dev,
+                     int H, int S, int causal, cudaStream_t stream, int dev,
                      const DevTable* tab_override = nullptr) {
   constexpr int D = 64;
   using C = BwdCfg<D>;
@@ -662,7 +668,7 @@ int launch_bwd_pairs(const void* q, const void* k, const void* v, const void* o,
   {
     std::lock_guard<std::mutex> lk(g_mu);
     if ((rc = pair_ctas(dev, &ctas))) return rc;
-    auto key = std::make_tuple(dev, B * H, N, 0, (int)dash::SHIFT_PAIRS, ctas, 1, 1);
+    auto key = std::make_tuple(dev, B * H, N, causal, pair_sched_of(causal), ctas, 1, 1);
     auto itb = g_tables.find(key);
     if (tab_override) {
       tab = const_cast<DevTable*>(tab_override);
@@ -671,7 +677,7 @@ int launch_bwd_pairs(const void* q, const void* k, const void* v, const void* o,
     } else {
       dash::Table half, t;
       std::string err;
-      if (!dash::build_table(B * H, N, 0, dash::SHIFT_PAIRS, ctas / 2, &half, &err))
+      if (!dash::build_table(B * H, N, causal, pair_sched_of(causal), ctas / 2, &half, &err))
         return DASH_ERR_UNSUPPORTED;
       if (!dash::validate_table(half, &err) || !dash::expand_pair_table(half, &t))
         return DASH_ERR_SCHEDULE;
@@ -710,7 +716,7 @@ int launch_bwd_pairs(const void* q, const void* k, const void* v, const void* o,
   p.dv = static_cast<__nv_bfloat16*>(dv);
   p.S = S;
   p.N = N;
-  p.causal = 0;
+  p.causal = causal;
   p.group_log2 = 0;
   p.scale = scale;
   p.scale_log2 = p.scale * 1.4426950408889634f;
@@ -731,7 +737,7 @@ int launch_bwd_pairs(const void* q, const void* k, const void* v, const void* o,
   cfg.numAttrs = 2;
   if (!prof_record(1, &ev, stream)) return DASH_ERR_CUDA;
   // middle links with red in L2 only where the chain mode forces it (bitwise the same)
-  const bool red = red_chain_for(DASH_SCHED_SHIFT_PAIRS, N, D, 1);
+  const bool red = red_chain_for(pair_sched_of(causal), N, D, 1);
   DASH_CUDA(cudaLaunchKernelEx(&cfg,
                                red ? dash::dash_bwd_kernel<64, false, false, true, true>
                                    : dash::dash_bwd_kernel<64, false, false, false, true>,
@@ -844,7 +850,7 @@ int host_bwd(const void* q, const void* k, const void* v, const void* o, const v
              const float* lse, void* dq, void* dk, void* dv, int B, int H, int S, int causal,
              int sched, cudaStream_t stream, int dev) {
   const int BH = B * H, N = S / 128;
-  const bool pairs = (sched == DASH_SCHED_SHIFT_PAIRS);  // CTA pairs (D = 64 only)
+  const bool pairs = pair_sched(sched);  // CTA pairs (D = 64 only)
   int ctas = 0;
   int rc;
   {
@@ -863,7 +869,7 @@ int host_bwd(const void* q, const void* k, const void* v, const void* o, const v
   HostPipe* hp = nullptr;
   {
     std::lock_guard<std::mutex> lk(g_mu);
-    if ((rc = pairs ? get_pair_chunk_tables(dev, BH, N, ctas, chunk, &parts)
+    if ((rc = pairs ? get_pair_chunk_tables(dev, BH, N, causal, ctas, chunk, &parts)
                     : get_chunk_tables(dev, BH, N, causal, sched, ctas, chunk, il, &parts)))
       return rc;
     if ((rc = get_pipe(dev, stream, 2 * slot_bytes, &hp))) return rc;
@@ -901,7 +907,8 @@ int host_bwd(const void* q, const void* k, const void* v, const void* o, const v
     DASH_CUDA(cudaStreamWaitEvent(stream, hp->in_ready[slot], 0));
     if (c >= 2) DASH_CUDA(cudaStreamWaitEvent(stream, hp->out_done[slot], 0));
     if ((rc = pairs ? launch_bwd_pairs(din[0], din[1], din[2], din[3], din[4], dlse, dout3[0],
-                                       dout3[1], dout3[2], 1, nh, S, stream, dev, &(*parts)[c])
+                                       dout3[1], dout3[2], 1, nh, S, causal, stream, dev,
+                                       &(*parts)[c])
                     : launch_bwd<D, kAtomic>(din[0], din[1], din[2], din[3], din[4], dlse,
                                              dout3[0], dout3[1], dout3[2], 1, nh, S, causal,
                                              sched, stream, dev, nullptr, 0, &(*parts)[c])))
@@ -977,7 +984,7 @@ int dash_set_head_interleave(int mode) {
 int dash_bwd_head_interleave(int num_ctas, int D, int schedule, int n_heads, int S, int causal,
                              int* heads_per_unit) {
   if (!heads_per_unit || num_ctas < 1 || n_heads < 1 || (D != 64 && D != 128) || S < 128 ||
-      S % 128 != 0 || schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_SHIFT_PAIRS ||
+      S % 128 != 0 || schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_SYM_SHIFT_PAIRS ||
       (causal != 0 && causal != 1))
     return DASH_ERR_INVALID_ARG;
   *heads_per_unit =
@@ -993,7 +1000,7 @@ int dash_set_dq_chain_mode(int mode) {
 
 int dash_dq_chain_uses_red(int schedule, int S, int D, int heads_per_unit, int* red) {
   if (!red || S < 128 || S % 128 != 0 || schedule < DASH_SCHED_NAIVE_ASC ||
-      schedule > DASH_SCHED_SHIFT_PAIRS || heads_per_unit < 1 || (D != 64 && D != 128))
+      schedule > DASH_SCHED_SYM_SHIFT_PAIRS || heads_per_unit < 1 || (D != 64 && D != 128))
     return DASH_ERR_INVALID_ARG;
   // the atomic variant has no chains
   *red = (schedule != DASH_SCHED_ATOMIC && red_chain_for(schedule, S / 128, D, heads_per_unit))
@@ -1039,9 +1046,9 @@ int dash_attn_bwd_gqa_split(const void* q, const void* k, const void* v, const v
     if (split < 0 || (split > 0 && H > 0 &&
                       ((split & (split - 1)) != 0 || (H / Hkv) % split != 0)))
       return DASH_ERR_INVALID_ARG;
-    if (schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_SHIFT_PAIRS)
+    if (schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_SYM_SHIFT_PAIRS)
       return DASH_ERR_INVALID_ARG;
-    if (schedule == DASH_SCHED_SHIFT_PAIRS) return DASH_ERR_UNSUPPORTED;  // dash_attn_bwd only
+    if (pair_sched(schedule)) return DASH_ERR_UNSUPPORTED;  // dash_attn_bwd only
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
         !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
       return DASH_ERR_INVALID_ARG;
@@ -1088,7 +1095,7 @@ int dash_bwd_gqa_split_for(int num_ctas, int B, int Hkv, int group, int S, int c
 int dash_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                   const float* lse, void* dq, void* dk, void* dv, int B, int H, int S, int D,
                   int causal, int schedule, void* stream) {
-  if (schedule == DASH_SCHED_SHIFT_PAIRS)
+  if (pair_sched(schedule))
     return no_throw([&]() -> int {
       int rc = check_shape(B, H, S, D);
       if (rc) return rc;
@@ -1096,13 +1103,14 @@ int dash_attn_bwd(const void* q, const void* k, const void* v, const void* o, co
       if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
           !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
         return DASH_ERR_INVALID_ARG;
-      // CTA pairs exist for the full mask at D = 64 (the staged dQp they exchange)
+      // CTA pairs exist at D = 64 (the staged dQp they exchange): SHIFT_PAIRS for the
+      // full mask, SYM_SHIFT_PAIRS for the causal one
       if (D != 64 || !dash::schedule_supported(schedule, S / 128, causal))
         return DASH_ERR_UNSUPPORTED;
       if (B == 0 || H == 0) return DASH_OK;
       int dev = 0;
       DASH_CUDA(cudaGetDevice(&dev));
-      return launch_bwd_pairs(q, k, v, o, dout, lse, dq, dk, dv, B, H, S,
+      return launch_bwd_pairs(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
                               static_cast<cudaStream_t>(stream), dev);
     }, DASH_ERR_OOM, DASH_ERR_INVALID_ARG);
   return dash_attn_bwd_gqa(q, k, v, o, dout, lse, dq, dk, dv, B, H, H, S, D, causal, schedule,
@@ -1116,9 +1124,9 @@ int dash_attn_bwd_host(const void* q, const void* k, const void* v, const void* 
     int rc = check_shape(B, H, S, D);
     if (rc) return rc;
     if (causal != 0 && causal != 1) return DASH_ERR_INVALID_ARG;
-    if (schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_SHIFT_PAIRS)
+    if (schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_SYM_SHIFT_PAIRS)
       return DASH_ERR_INVALID_ARG;
-    if (schedule == DASH_SCHED_SHIFT_PAIRS && D != 64) return DASH_ERR_UNSUPPORTED;
+    if (pair_sched(schedule) && D != 64) return DASH_ERR_UNSUPPORTED;
     if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return DASH_ERR_INVALID_ARG;
     if (!dash::schedule_supported(schedule, S / 128, causal)) return DASH_ERR_UNSUPPORTED;
     if (B == 0 || H == 0) return DASH_OK;
@@ -1258,9 +1266,9 @@ int dash_trace_bwd(const void* q, const void* k, const void* v, const void* o, c
     int rc = check_shape(B, H, S, D);
     if (rc) return rc;
     if (causal != 0 && causal != 1) return DASH_ERR_INVALID_ARG;
-    if (schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_SHIFT_PAIRS)
+    if (schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_SYM_SHIFT_PAIRS)
       return DASH_ERR_INVALID_ARG;
-    if (schedule == DASH_SCHED_SHIFT_PAIRS) return DASH_ERR_UNSUPPORTED;  // dash_attn_bwd only
+    if (pair_sched(schedule)) return DASH_ERR_UNSUPPORTED;  // dash_attn_bwd only
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
         !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !host_trace ||
         !num_ctas || !rows_per_cta)
@@ -1414,12 +1422,15 @@ long long dash_sched_table(int n_heads, int N, int causal, int schedule, int num
   }, -DASH_ERR_OOM, -DASH_ERR_INVALID_ARG);
 }
 
-long long dash_sched_table_pairs(int n_heads, int N, int num_ctas, int* rows, long long cap) {
+long long dash_sched_table_pairs(int n_heads, int N, int causal, int num_ctas, int* rows,
+                                 long long cap) {
   return no_throw([&]() -> long long {
-    if (num_ctas < 2 || num_ctas % 2 != 0) return -DASH_ERR_INVALID_ARG;
+    if (num_ctas < 2 || num_ctas % 2 != 0 || (causal != 0 && causal != 1))
+      return -DASH_ERR_INVALID_ARG;
     dash::Table half, t;
     std::string err;
-    if (!dash::build_table(n_heads, N, 0, dash::SHIFT_PAIRS, num_ctas / 2, &half, &err))
+    if (!dash::build_table(n_heads, N, causal, pair_sched_of(causal), num_ctas / 2, &half,
+                           &err))
       return -DASH_ERR_UNSUPPORTED;
     if (!dash::validate_table(half, &err)) return -DASH_ERR_SCHEDULE;
     if (!dash::expand_pair_table(half, &t)) return -DASH_ERR_SCHEDULE;

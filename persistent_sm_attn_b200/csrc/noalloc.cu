@@ -272,9 +272,10 @@ extern "C" int dash_attn_bwd_noalloc(const void* q, const void* k, const void* v
                                      int schedule, void* stream) {
   if (B < 0 || H < 0 || S < 0 || D < 0) return DASH_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return DASH_ERR_INVALID_ARG;
-  if (schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_SHIFT_PAIRS)
+  if (schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_SYM_SHIFT_PAIRS)
     return DASH_ERR_INVALID_ARG;
-  if (schedule == DASH_SCHED_SHIFT_PAIRS) return DASH_ERR_UNSUPPORTED;  // dash_attn_bwd only
+  if (schedule == DASH_SCHED_SHIFT_PAIRS || schedule == DASH_SCHED_SYM_SHIFT_PAIRS)
+    return DASH_ERR_UNSUPPORTED;  // dash_attn_bwd only
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
       !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return DASH_ERR_INVALID_ARG;

@@ -36,6 +36,7 @@ bool schedule_supported(int schedule, int N, int causal) {
     case SHIFT: return !causal;
     case SYM_SHIFT: return causal && (N % 2 == 0);
     case SHIFT_PAIRS: return !causal && (N % 2 == 0);
+    case SYM_SHIFT_PAIRS: return causal && (N % 4 == 0);
     default: return false;
   }
 }
@@ -78,6 +79,20 @@ static Units units_of(int schedule, int N, int causal) {
         u.push_back(seq);
       }
       break;
+    case SYM_SHIFT_PAIRS: {
+      // SYM_SHIFT over the N / 2 pair-tiles; each visited (KV pair, Q pair) becomes the two
+      // steps of its Q tiles, in order
+      const Units half = units_of(SYM_SHIFT, N / 2, 1);
+      for (const auto& hs : half) {
+        std::vector<std::pair<int, int>> seq;
+        for (const auto& e : hs) {
+          seq.push_back({e.first, 2 * e.second});
+          seq.push_back({e.first, 2 * e.second + 1});
+        }
+        u.push_back(seq);
+      }
+      break;
+    }
     case SYM_SHIFT: {
       const int h = N / 2;
       for (int k = 0; k < h; ++k) {
@@ -190,7 +205,7 @@ bool build_table_grouped(int n_heads, int group, int N, int causal, int schedule
   Table t;
   t.n_heads = n_heads; t.N = N; t.causal = causal; t.schedule = schedule; t.num_ctas = num_ctas;
   t.group = group;
-  if (schedule == SHIFT_PAIRS) t.kv_units = N / 2;
+  if (pair_schedule(schedule)) t.kv_units = N / 2;
   // per CTA, the global units it runs, in round order
   std::vector<std::vector<long long>> per_cta(num_ctas);
   const long long total_units = (long long)(n_heads / group) * U;
@@ -289,9 +304,14 @@ bool validate_table(const Table& t, std::string* err) {
   // the table's own size, whatever n_heads a caller-supplied table claims
   // KV units per head: N, or N / 2 KV pairs for a pair schedule's half table
   const int kvn = t.kv_units > 0 ? t.kv_units : N;
-  if (kvn > N || (t.kv_units > 0 && (t.causal || t.schedule != SHIFT_PAIRS)))
+  const bool half = t.kv_units > 0;  // a pair schedule's half table: kv is a KV pair
+  if (kvn > N || (half && (!pair_schedule(t.schedule) || 2 * kvn != N ||
+                           t.causal != (t.schedule == SYM_SHIFT_PAIRS))))
     return fail("bad KV unit count");
-  const long long per_head = t.causal ? (long long)N * (N + 1) / 2 : (long long)kvn * N;
+  // pairs per head: causal half tables hold Q tiles 2m .. N-1 for KV pair m
+  const long long per_head = !t.causal ? (long long)kvn * N
+                             : half    ? (long long)kvn * N - (long long)kvn * (kvn - 1)
+                                       : (long long)N * (N + 1) / 2;
   if ((long long)t.n_pairs() != (long long)t.n_heads * per_head)
     return fail("table has missing or extra pairs");
   const long long nblk = (long long)t.n_heads * N;
@@ -314,7 +334,7 @@ bool validate_table(const Table& t, std::string* err) {
         const uint32_t w = t.pairs[ch.pair_off + i];
         const int q = pair_q(w), p = pair_pos(w);
         if (q < 0 || q >= N) return fail("q tile out of range");
-        if (t.causal && q < ch.kv) return fail("pair above the causal diagonal");
+        if (t.causal && q < (half ? 2 * ch.kv : ch.kv)) return fail("pair above the causal diagonal");
         uint8_t& s = seen[((size_t)ch.bh * N + ch.kv) * N + q];
         if (s) return fail("pair visited twice");
         s = 1;
@@ -345,7 +365,7 @@ bool validate_table(const Table& t, std::string* err) {
   }
   for (long long blk = 0; blk < nblk; ++blk) {
     const int q = (int)(blk % N);
-    const int want = t.causal ? q + 1 : kvn;
+    const int want = t.causal ? (half ? q / 2 + 1 : q + 1) : kvn;
     if (n_contrib[blk] != want) return fail("dQ block has missing or extra contributors");
     for (int p = 0; p < want; ++p)
       if (!pos_seen[(size_t)blk * N + p]) return fail("positions are not a permutation");
@@ -505,11 +525,12 @@ bool simulate_table(const Table& t, double c, double r, int beta, int chains, Si
 }
 
 bool expand_pair_table(const Table& half, Table* out) {
-  if (half.schedule != SHIFT_PAIRS || half.kv_units * 2 != half.N || half.causal ||
-      half.group != 1 || (long long)half.num_ctas * 2 > kMaxTableCtas)
+  if (!pair_schedule(half.schedule) || half.kv_units * 2 != half.N ||
+      half.causal != (half.schedule == SYM_SHIFT_PAIRS) || half.group != 1 ||
+      (long long)half.num_ctas * 2 > kMaxTableCtas)
     return false;
   Table t;
-  t.n_heads = half.n_heads; t.N = half.N; t.causal = 0; t.schedule = SHIFT_PAIRS;
+  t.n_heads = half.n_heads; t.N = half.N; t.causal = half.causal; t.schedule = half.schedule;
   t.num_ctas = 2 * half.num_ctas;
   t.group = 1;
   t.kv_units = 0;  // the grid's table holds every KV tile

@@ -15,7 +15,10 @@
 namespace dash {
 
 enum Schedule { NAIVE_ASC = 0, DESCENDING = 1, SHIFT = 2, SYM_SHIFT = 3, ATOMIC = 4,
-                SHIFT_PAIRS = 5 };
+                SHIFT_PAIRS = 5, SYM_SHIFT_PAIRS = 6 };
+
+// The CTA-pair schedules, whose tables are built as half tables (one unit per KV pair).
+inline bool pair_schedule(int s) { return s == SHIFT_PAIRS || s == SYM_SHIFT_PAIRS; }
 
 // Upper bound on a table's CTA count (the kernel's grid is the SM count times the CTAs
 // resident per SM); larger requests are refused instead of sizing per-CTA lists by them.
@@ -51,6 +54,12 @@ bool schedule_supported(int schedule, int N, int causal);
 // Units of one head: each a list of (kv, q) in visiting order.
 std::vector<std::vector<std::pair<int, int>>> head_units(int schedule, int N, int causal);
 
+// SYM_SHIFT_PAIRS (causal, N a multiple of 4): the same pairing under the causal mask.
+// KV pair m and Q pair j (Q tiles 2j, 2j + 1) form a pair-tile, visible when j >= m; the
+// half table runs SYM_SHIFT over N / 2 pair-tiles, each pair-tile as two steps (Q tiles 2j
+// then 2j + 1).  On the diagonal pair-tile the odd KV tile's first step (KV 2m + 1, Q 2m)
+// is fully masked: it contributes zeros, so that both CTAs keep the same steps.  A dQ
+// block q receives q / 2 + 1 pre-summed contributions.
 // SHIFT_PAIRS (full mask, N even): CTA pairs (2i, 2i + 1) run KV tiles 2m and 2m + 1 of
 // a head over the same Q tiles at the same steps, m + t mod N at step t, and pre-sum
 // their two dQ partials before the ordered accumulation, so a dQ block receives N / 2
