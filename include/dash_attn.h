@@ -201,10 +201,11 @@ int dash_slot_placement_by_smid(int S, int* by_smid);
  * schedule runs for 2 (or 4) consecutive heads in turn, K/V loaded again for each; the
  * heads' dQ blocks then receive their contributions further apart in the grid's steps.
  * The order of every dQ block is still fixed by the table, so results stay bitwise
- * reproducible, but they differ in rounding from the uninterleaved table.
+ * reproducible, but they may differ in rounding from the uninterleaved table.
  * mode 0 (default): the library picks, 2 for SYM_SHIFT at D = 64 when the units still
  * fill the grid's rounds (measured faster there), else 1; mode 1: never; mode 2 or 4:
- * that many heads per unit whenever it divides B * H.  Applies to later dash_attn_bwd,
+ * that many heads per unit whenever it divides B * H, the CTA-pair schedules' half
+ * tables included.  Applies to later dash_attn_bwd,
  * dash_attn_bwd_host, dash_attn_bwd_noalloc and dash_trace_bwd calls (the grouped-query
  * entry points have their own grouping).  Other modes: INVALID_ARG.
  */

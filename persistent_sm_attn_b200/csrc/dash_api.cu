@@ -254,13 +254,14 @@ int get_chunk_tables(int dev, int heads, int N, int causal, int sched, int ctas,
 // causal): the half table (one unit per KV pair, ctas / 2 slots) split by heads, each
 // part validated and expanded to the grid's table, so every part keeps the whole
 // launch's dQ orders.
-std::map<std::tuple<int, int, int, int, int, int>, std::vector<DevTable>> g_pair_chunk_tables;
+std::map<std::tuple<int, int, int, int, int, int, int>, std::vector<DevTable>>
+    g_pair_chunk_tables;
 
 int pair_sched_of(int causal) { return causal ? dash::SYM_SHIFT_PAIRS : dash::SHIFT_PAIRS; }
 
-int get_pair_chunk_tables(int dev, int heads, int N, int causal, int ctas, int chunk,
+int get_pair_chunk_tables(int dev, int heads, int N, int causal, int ctas, int chunk, int il,
                           std::vector<DevTable>** out) {
-  auto key = std::make_tuple(dev, heads, N, causal, ctas, chunk);
+  auto key = std::make_tuple(dev, heads, N, causal, ctas, chunk, il);
   auto itc = g_pair_chunk_tables.find(key);
   if (itc != g_pair_chunk_tables.end()) {
     *out = &itc->second;
@@ -268,7 +269,8 @@ int get_pair_chunk_tables(int dev, int heads, int N, int causal, int ctas, int c
   }
   dash::Table half;
   std::string err;
-  if (!dash::build_table(heads, N, causal, pair_sched_of(causal), ctas / 2, &half, &err))
+  if (!dash::build_table_grouped(heads, il, N, causal, pair_sched_of(causal), ctas / 2, &half,
+                                 &err))
     return DASH_ERR_UNSUPPORTED;
   if (!dash::validate_table(half, &err)) return DASH_ERR_SCHEDULE;
   std::vector<DevTable> parts;
@@ -668,7 +670,10 @@ int launch_bwd_pairs(const void* q, const void* k, const void* v, const void* o,
   {
     std::lock_guard<std::mutex> lk(g_mu);
     if ((rc = pair_ctas(dev, &ctas))) return rc;
-    auto key = std::make_tuple(dev, B * H, N, causal, pair_sched_of(causal), ctas, 1, 1);
+    // heads per unit of the half table (1 unless dash_set_head_interleave forces more)
+    const int il = dash::head_interleave(D, pair_sched_of(causal), B * H, N, causal, ctas / 2,
+                                         g_il_mode.load());
+    auto key = std::make_tuple(dev, B * H, N, causal, pair_sched_of(causal), ctas, il, 1);
     auto itb = g_tables.find(key);
     if (tab_override) {
       tab = const_cast<DevTable*>(tab_override);
@@ -677,7 +682,8 @@ int launch_bwd_pairs(const void* q, const void* k, const void* v, const void* o,
     } else {
       dash::Table half, t;
       std::string err;
-      if (!dash::build_table(B * H, N, causal, pair_sched_of(causal), ctas / 2, &half, &err))
+      if (!dash::build_table_grouped(B * H, il, N, causal, pair_sched_of(causal), ctas / 2,
+                                     &half, &err))
         return DASH_ERR_UNSUPPORTED;
       if (!dash::validate_table(half, &err) || !dash::expand_pair_table(half, &t))
         return DASH_ERR_SCHEDULE;
@@ -860,7 +866,8 @@ int host_bwd(const void* q, const void* k, const void* v, const void* o, const v
   if (rc) return rc;
   // the parts hold whole units of the launch's table, so its interleaved heads stay
   // together and every dQ block keeps the order dash_attn_bwd gives it
-  const int il = dash::head_interleave(D, sched, BH, N, causal, ctas, g_il_mode.load());
+  const int il = dash::head_interleave(D, sched, BH, N, causal, pairs ? ctas / 2 : ctas,
+                                       g_il_mode.load());
   const int chunk = ((BH + kHostParts - 1) / kHostParts + il - 1) / il * il;
   const size_t rows_c = (size_t)chunk * S;
   const size_t tile = align256(rows_c * D * 2), lse_b = align256(rows_c * 4);
@@ -869,7 +876,7 @@ int host_bwd(const void* q, const void* k, const void* v, const void* o, const v
   HostPipe* hp = nullptr;
   {
     std::lock_guard<std::mutex> lk(g_mu);
-    if ((rc = pairs ? get_pair_chunk_tables(dev, BH, N, causal, ctas, chunk, &parts)
+    if ((rc = pairs ? get_pair_chunk_tables(dev, BH, N, causal, ctas, chunk, il, &parts)
                     : get_chunk_tables(dev, BH, N, causal, sched, ctas, chunk, il, &parts)))
       return rc;
     if ((rc = get_pipe(dev, stream, 2 * slot_bytes, &hp))) return rc;

@@ -526,13 +526,13 @@ bool simulate_table(const Table& t, double c, double r, int beta, int chains, Si
 
 bool expand_pair_table(const Table& half, Table* out) {
   if (!pair_schedule(half.schedule) || half.kv_units * 2 != half.N ||
-      half.causal != (half.schedule == SYM_SHIFT_PAIRS) || half.group != 1 ||
+      half.causal != (half.schedule == SYM_SHIFT_PAIRS) || half.group < 1 ||
       (long long)half.num_ctas * 2 > kMaxTableCtas)
     return false;
   Table t;
   t.n_heads = half.n_heads; t.N = half.N; t.causal = half.causal; t.schedule = half.schedule;
   t.num_ctas = 2 * half.num_ctas;
-  t.group = 1;
+  t.group = half.group;  // heads per unit: each KV segment runs for `group` heads in turn
   t.kv_units = 0;  // the grid's table holds every KV tile
   t.cta_off.assign(t.num_ctas + 1, 0);
   for (int c = 0; c < half.num_ctas; ++c)

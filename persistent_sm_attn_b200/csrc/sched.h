@@ -67,6 +67,8 @@ std::vector<std::vector<std::pair<int, int>>> head_units(int schedule, int N, in
 // half table (one unit per KV pair, num_ctas / 2 slots, kv = m); expand_pair_table
 // turns it into the grid's table, slot 2i running KV tile 2m and slot 2i + 1 KV tile
 // 2m + 1 with the same Q tiles and positions.
+// (A half table built with several heads per unit, build_table_grouped's group, expands
+// the same way: each CTA's chains keep the half table's head order.)
 bool expand_pair_table(const Table& half, Table* out);
 
 // Query heads per unit of a multi-head launch's table.  With il > 1 the launch uses

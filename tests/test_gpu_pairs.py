@@ -161,3 +161,28 @@ def test_causal_pairs_full_workload_sampled():
         rel = (torch.linalg.vector_norm(a.float() - b.float()) /
                torch.linalg.vector_norm(b.float())).item()
         assert rel < 1e-4, rel
+
+
+@pytest.mark.parametrize("causal,sched", [(False, "shift_pairs"), (True, "sym_shift_pairs")])
+def test_pairs_with_two_heads_per_unit(causal, sched):
+    """dash_set_head_interleave(2) builds the pair table with two heads per unit: parity
+    with the oracle on a multi-round grid, bitwise repeats, and the host-buffer path's
+    bits."""
+    G.need_cuda()
+    case = G.make_case(4, 40, 512, 64, causal, seed=31 + causal)
+    _, _, *ref = G.oracle_full(case)
+    binding.dash_set_head_interleave(2)
+    try:
+        out = G.bwd(case, sched)
+        again = G.bwd(case, sched)
+        host = [case[n].cpu().pin_memory() for n in ("q", "k", "v", "o", "do", "lse")]
+        got = binding.dash_attn_bwd_host(*host, causal, sched)
+        assert binding.dash_attn_sync_status() == 0
+    finally:
+        binding.dash_set_head_interleave(0)
+    errs = {n: A.rel_fro(x.float().cpu().numpy(), r) for n, x, r in zip(("dq", "dk", "dv"), out, ref)}
+    G.log_margin(f"{sched} B4 H40 S512 D64, two heads per unit", errs)
+    assert max(errs.values()) < G.TOL, errs
+    for a, b, c in zip(out, again, got):
+        assert torch.equal(a, b)
+        assert torch.equal(a.cpu(), c)
