@@ -1,8 +1,9 @@
 """Bitwise reproducibility of every deterministic schedule: 50 launches, and
 launches racing a concurrent load on another stream, on every workload at its
 full size (best schedule and the descending order, plus naive ascending where
-it is one of the workload's compared schedules) and on a reduced causal D = 64
-shape."""
+it is one of the workload's compared schedules), on a reduced causal D = 64
+shape, and for the CTA-pair schedules on a full-mask D = 64 shape and the causal
+16k workload."""
 import pytest
 import torch
 
@@ -21,6 +22,11 @@ CASES = [(w.name, (w.B, w.H, w.S, w.D, w.causal, w.sigma, seed_of(i)), _det(w))
          for i, w in enumerate(WORKLOADS) if i >= 1]
 CASES.append(("causal_b2_h8_s4096_d64", (2, 8, 4096, 64, True, 1.0, 11),
               ("sym_shift", "descending", "naive_asc")))
+# the CTA-pair schedules (D = 64): a full-mask shape, and the causal 16k workload
+CASES.append(("full_b2_h16_s4096_d64_pairs", (2, 16, 4096, 64, False, 1.0, 12), ("shift_pairs",)))
+_w3 = WORKLOADS[3]
+CASES.append((_w3.name + "_pairs", (_w3.B, _w3.H, _w3.S, _w3.D, _w3.causal, _w3.sigma, seed_of(3)),
+              ("sym_shift_pairs",)))
 IDS = [c[0] for c in CASES]
 
 
