@@ -50,6 +50,18 @@ def test_oracle_units(N):
     assert not sc.supported(sc.SHIFT_PAIRS, 4, True)
 
 
+def test_oracle_units_small_case_by_hand():
+    # N = 4: KV pairs 0 and 1; pair m starts at Q tile m and shifts by one per step
+    assert sc.units(sc.SHIFT_PAIRS, 4, False) == [
+        [(0, 0), (0, 1), (0, 2), (0, 3)],
+        [(1, 1), (1, 2), (1, 3), (1, 0)]]
+    # one round: each block's two contributions in step order.  Block q meets pair 0 at
+    # step q and pair 1 at step q - 1 mod 4, so pair 1 comes first except at block 0.
+    order = sc.accumulation_order(sc.SHIFT_PAIRS, 4, False)
+    assert order == {0: [(0, 0), (1, 3)], 1: [(1, 0), (0, 1)], 2: [(1, 1), (0, 2)],
+                     3: [(1, 2), (0, 3)]}
+
+
 @pytest.mark.parametrize("heads,N,slots", [(1, 4, 2), (3, 4, 5), (2, 8, 3), (5, 6, 7), (4, 16, 74)])
 def test_half_table_equals_oracle_and_has_no_cycle(heads, N, slots):
     rows = binding.dash_sched_table(heads, N, False, "shift_pairs", slots)
