@@ -145,6 +145,10 @@ def test_oracle_units_causal_small_case_by_hand():
     # runs the dense pair-tile (0, 1), then the diagonal pair-tile (0, 0), then (1, 1).
     assert sc.units(sc.SYM_SHIFT_PAIRS, 4, True) == [
         [(0, 2), (0, 3), (0, 0), (0, 1), (1, 2), (1, 3)]]
+    # blocks 0 and 1 hear from KV pair 0 only; blocks 2 and 3 from pair 0 (steps 0, 1)
+    # and then pair 1 (steps 4, 5)
+    assert sc.accumulation_order(sc.SYM_SHIFT_PAIRS, 4, True) == {
+        0: [(0, 2)], 1: [(0, 3)], 2: [(0, 0), (0, 4)], 3: [(0, 1), (0, 5)]}
 
 
 @pytest.mark.parametrize("heads,N,slots", [(1, 4, 1), (3, 4, 2), (2, 8, 3), (5, 12, 7),
