@@ -157,6 +157,22 @@ def rel_fro(x, ref) -> float:
     return float(num / den) if den > 0 else float(num)
 
 
+def head_forward_rows(q, k, v, causal: bool, scale: float, rows):
+    """The forward of one head evaluated only at chosen query rows, for heads too large
+    to hold S x S matrices: (O [len(rows), D], LSE [len(rows)]), each row from the same
+    definitions as ``head_forward`` (row i sees keys j <= i under the causal mask)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    S = k.shape[0]
+    rows = np.asarray(rows)
+    keys = np.arange(S)
+    allowed = (keys[None, :] <= rows[:, None]) if causal else np.ones((len(rows), S), bool)
+    s = np.where(allowed, scale * (q[rows] @ k.T), -np.inf)
+    m = s.max(axis=1, keepdims=True)
+    lse = (m + np.log(np.exp(s - m).sum(axis=1, keepdims=True)))[:, 0]
+    p = np.where(allowed, np.exp(s - lse[:, None]), 0.0)
+    return p @ v, lse
+
+
 def head_backward_rows(q, k, v, do, causal: bool, scale: float, rows_q, rows_kv, chunk=1024):
     """The backward of one head evaluated only at chosen rows, for heads too
     large to hold S x S matrices: dQ at query rows ``rows_q`` and dK, dV at

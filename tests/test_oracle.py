@@ -212,6 +212,25 @@ def test_pins_catch_planted_mistakes(mutant):
 
 
 @pytest.mark.parametrize("causal", [False, True])
+def test_row_sampled_forward_matches_torch_softmax(causal):
+    """The row-sampled forward used at full workload sizes equals torch float64
+    softmax and logsumexp on the sampled rows."""
+    import torch
+    S, D = 96, 16
+    q, k, v = (_rand((S, D), 600 + i) for i in range(3))
+    scale = 0.25
+    rows = np.array([0, 1, 31, 32, 63, 95])
+    o, lse = A.head_forward_rows(q, k, v, causal, scale, rows)
+    s = scale * (torch.from_numpy(q) @ torch.from_numpy(k).T)
+    if causal:
+        s = s.masked_fill(torch.ones(S, S, dtype=torch.bool).triu(1), float("-inf"))
+    want_o = (torch.softmax(s, dim=1) @ torch.from_numpy(v)).numpy()
+    want_lse = torch.logsumexp(s, dim=1).numpy()
+    assert np.abs(o - want_o[rows]).max() < 1e-12
+    assert np.abs(lse - want_lse[rows]).max() < 1e-12
+
+
+@pytest.mark.parametrize("causal", [False, True])
 def test_row_sampled_backward_matches_autograd(causal):
     """The row-sampled backward used at full workload sizes equals torch
     float64 autograd on the sampled rows."""
