@@ -410,6 +410,7 @@ __global__ void __launch_bounds__(512, 1)
       // D = 128 dO has a producer of its own (warp 15), so a Q load never queues behind
       // the wait for the single dO stage.
       int it = 0, kn = 0;  // kn: K/V loads so far
+      const uint64_t pol_first = policy_evict_first();  // K/V: one chain's use only
       for (int ci = cbeg; ci < cend; ++ci) {
         const int4 ch = p.chains[ci];
         if (!(ch.w & kChainContPrev)) {
@@ -418,8 +419,8 @@ __global__ void __launch_bounds__(512, 1)
           const int row_kv = (ch.x >> gl2) * S + ch.y * 128;
 #pragma unroll
           for (int cb = 0; cb < D / 64; ++cb) {
-            tma_load_2d(sK + cb * 16384, &tmK, cb * 64, row_kv, BAR(B_KV_FULL));
-            tma_load_2d(sV + cb * 16384, &tmV, cb * 64, row_kv, BAR(B_KV_FULL));
+            tma_load_2d_hint(sK + cb * 16384, &tmK, cb * 64, row_kv, BAR(B_KV_FULL), pol_first);
+            tma_load_2d_hint(sV + cb * 16384, &tmV, cb * 64, row_kv, BAR(B_KV_FULL), pol_first);
           }
           ++kn;
         }
@@ -976,6 +977,7 @@ __global__ void __launch_bounds__(512, 1)
     constexpr int G = 24;               // loads in flight per group
     int it = 0, fn = 0;  // fn: dK/dV runs written out
     int npub = 0;        // pairs handed to the publisher
+    const uint64_t pol_last = policy_evict_last();  // dQ accumulators: live for a whole head
     // D = 64, deterministic: once this pair is handed off, the accumulator loads of the
     // next pair go out if its ticket is already granted (checked once, never waited
     // for here), so their round trip overlaps the wait for the next partial and its
@@ -1086,7 +1088,7 @@ __global__ void __launch_bounds__(512, 1)
               float4 old[G];
 #pragma unroll
               for (int j = 0; j < G; ++j)
-                if (g0 + j < NA) old[j] = ld_cg_f4(src + (g0 + j) * 128 + r);
+                if (g0 + j < NA) old[j] = ld_cg_f4_hint(src + (g0 + j) * 128 + r, pol_last);
 #pragma unroll
               for (int j = 0; j < G; ++j) {
                 if (g0 + j < NA) {
@@ -1114,7 +1116,7 @@ __global__ void __launch_bounds__(512, 1)
                 ticket_wait(p.tickets + unit, (uint32_t)idx, ~0u);
                 if (threadIdx.x == 256) trace(it, 6);
 #pragma unroll
-                for (int j = 0; j < NV; ++j) pre[j] = ld_cg_f4(accp + j * 128 + r);
+                for (int j = 0; j < NV; ++j) pre[j] = ld_cg_f4_hint(accp + j * 128 + r, pol_last);
               }
 #pragma unroll
               for (int j = 0; j < NV; ++j) {
@@ -1163,13 +1165,15 @@ __global__ void __launch_bounds__(512, 1)
               if (threadIdx.x == 256) trace(it, 6);
 #pragma unroll
               for (int c4 = 0; c4 < NA; ++c4)
-                red_add_f4(accp + c4 * 128 + r,
-                           make_float4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]));
+                red_add_f4_hint(accp + c4 * 128 + r,
+                                make_float4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]),
+                                pol_last);
             } else {
 #pragma unroll
               for (int c4 = 0; c4 < NA; ++c4)
-                st_cg_f4(accp + c4 * 128 + r,
-                         make_float4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]));
+                st_cg_f4_hint(accp + c4 * 128 + r,
+                              make_float4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]),
+                              pol_last);
             }
             if (threadIdx.x == 256) trace(it, 13);
             if constexpr (C::kPublisher) {
@@ -1211,7 +1215,7 @@ __global__ void __launch_bounds__(512, 1)
                 if (pre_ok) {
                   const float4* nacc = reinterpret_cast<const float4*>(p.acc) + nunit * (32 * D);
 #pragma unroll
-                  for (int j = 0; j < NV; ++j) pre[j] = ld_cg_f4(nacc + j * 128 + r);
+                  for (int j = 0; j < NV; ++j) pre[j] = ld_cg_f4_hint(nacc + j * 128 + r, pol_last);
                 }
               }
             }
