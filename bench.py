@@ -78,11 +78,11 @@ def _workload(args):
     b, h, s, d, mask = args.shape.split(",")
     B, H, S, D, causal = int(b), int(h), int(s), int(d), mask.strip() == "causal"
     N = S // 128
-    if causal and D == 64 and N % 4 == 0:
+    if causal and N % 4 == 0:
         scheds = ("sym_shift", "sym_shift_pairs", "descending")
     elif causal:
         scheds = ("sym_shift", "descending") if N % 2 == 0 else ("descending",)
-    elif D == 64 and N % 2 == 0:
+    elif N % 2 == 0:
         scheds = ("shift", "shift_pairs", "descending")
     else:
         scheds = ("shift", "descending")

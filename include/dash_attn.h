@@ -381,11 +381,12 @@ long long dash_sched_table(int n_heads, int N, int causal, int schedule, int num
  * KV tile 2m + 1, both with the pair's Q tiles and positions.  Returns the number of
  * rows, or -DASH_ERR_INVALID_ARG (odd num_ctas, causal not 0 or 1),
  * -DASH_ERR_UNSUPPORTED or -DASH_ERR_SCHEDULE.
- * The backward runs them through dash_attn_bwd only, at D = 64 (each CTA stages its dQ
- * partial in shared memory, and the pair is a thread-block cluster of two CTAs that read
- * each other's staged partial): each CTA adds the two partials for half of the columns
- * and accumulates that half in order.  Other head dims, the other mask and unsupported
- * N return DASH_ERR_UNSUPPORTED.  dash_attn_bwd_host takes them too (its parts are slices
+ * The backward runs them through dash_attn_bwd, the pair being a thread-block cluster of
+ * two CTAs: each CTA adds the two partials for half of the columns and accumulates that
+ * half in order.  At D = 64 each CTA stages its dQ partial in shared memory and reads the
+ * peer's; at D = 128 (the partial stays in TMEM) each reducer thread writes the peer's
+ * half of its row into a 16 KiB buffer of the peer's shared memory, 32 columns a round.
+ * The other mask and unsupported N return DASH_ERR_UNSUPPORTED.  dash_attn_bwd_host takes them too (its parts are slices
  * of the same table, so the bits are dash_attn_bwd's); the grouped-query, no-allocation
  * and trace entry points return DASH_ERR_UNSUPPORTED.
  */

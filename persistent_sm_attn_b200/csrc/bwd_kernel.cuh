@@ -150,6 +150,11 @@ struct BwdCfg {
   // The swizzled tiles need a 1 KiB aligned base; the kernel checks it.
   static constexpr int kSmemBytes = OFF_TMEM_SLOT + 16;
   static_assert(kSmemBytes <= 232448, "shared memory per block exceeded");
+  // CTA pairs at D = 128: a 16 KiB buffer into which the peer writes 32 columns of its dQp
+  // rows at a time ([8 float4 groups][128 rows][float4]); pair launches only
+  static constexpr int OFF_XB = (kSmemBytes + 1023) / 1024 * 1024;
+  static constexpr int kSmemPairBytes = (D == 64) ? kSmemBytes : OFF_XB + 16384;
+  static_assert(kSmemPairBytes <= 232448, "shared memory per block exceeded (pairs)");
   // TMEM columns.  D = 128: S^T [0,128), dP^T [128,256), dV, dK; dQp reuses dP^T's
   // columns and dK takes dS^T from S^T's columns.  D = 64: S^T has two buffers [0,128)
   // and [128,256), one per softmax warpgroup (they take alternate tiles), dP^T
@@ -205,16 +210,19 @@ constexpr int kTraceEvents = 16;
 // grants them, instead of a load-add-store from the SM.  The additions and their order
 // are the same, so the results are bitwise the same; only the traffic and the latency
 // of each link differ.
-// kPair (D = 64, deterministic): the grid runs in clusters of two
+// kPair (deterministic): the grid runs in clusters of two
 // CTAs, 2i and 2i + 1, with a SHIFT_PAIRS or SYM_SHIFT_PAIRS table: the pair runs KV tiles
 // 2m and 2m + 1 over the same Q tiles at the same steps.  Each CTA's reducers add the two
-// staged dQ partials of a step (its own, and the peer's read over distributed shared
-// memory) for half of the columns, CTA 2i + r taking columns [32r, 32r + 32), and run the
-// ordered accumulation of that half: one contribution per pair and step, so N / 2 per
-// block (q / 2 + 1 for block q under the causal mask) and half the accumulator bytes per
-// CTA.  Both CTAs free a staged tile only after both have read it.  Under the causal mask
-// CTA 2i + 1 meets one tile wholly above the diagonal per diagonal pair-tile (KV 2m + 1,
-// Q 2m): every probability of it is masked to zero, so its partials are zeros.
+// dQ partials of a step (its own and the peer's) for half of the columns, CTA 2i + r taking
+// columns [rD/2, (r + 1)D/2), and run the ordered accumulation of that half: one
+// contribution per pair and step, so N / 2 per block (q / 2 + 1 for block q under the
+// causal mask) and half the accumulator bytes per CTA.  D = 64: each reducer reads the
+// peer's staged tile over distributed shared memory, and both CTAs free a staged tile only
+// after both have read it.  D = 128 (dQp only in TMEM): each reducer thread writes the
+// peer's half of its row into the peer's exchange buffer, 32 columns a round, two rounds
+// per step, and adds what the peer wrote into its own.  Under the causal mask CTA 2i + 1
+// meets one tile wholly above the diagonal per diagonal pair-tile (KV 2m + 1, Q 2m): every
+// probability of it is masked to zero, so its partials are zeros.
 template <int D, bool kAtomic, bool kTrace = false, bool kRed = false, bool kPair = false>
 __global__ void __launch_bounds__(512, 1)
     dash_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -222,7 +230,7 @@ __global__ void __launch_bounds__(512, 1)
                     const __grid_constant__ CUtensorMap tmC, const BwdParams p) {
   using namespace dev;
   using C = BwdCfg<D>;
-  static_assert(!kPair || (D == 64 && !kAtomic), "CTA pairs: D = 64, deterministic");
+  static_assert(!kPair || !kAtomic, "CTA pairs: deterministic only");
   constexpr int ST = C::kStagesQ, SD = C::kStagesDO;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t sb = smem_u32(smem_raw);
@@ -299,11 +307,13 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(BAR(B_DS_READY1), kSoftmaxArrive);
     // D = 64: the reducers (128 threads) free a dS buffer once they have read the dQp
     // staged there; D = 128: the commit of dQp and dK frees it
-    // CTA pairs: both CTAs' reducers read each staged tile (128 + 128 arrivals)
-    constexpr uint32_t kDsFree = kPair ? 256u : (C::kSDouble ? 128u : 1u);
+    // CTA pairs at D = 64: both CTAs' reducers read each staged tile (128 + 128 arrivals)
+    constexpr uint32_t kDsFree = C::kSDouble ? (kPair ? 256u : 128u) : 1u;
     mbar_init(BAR(B_DS_FREE), kDsFree);
     mbar_init(BAR(B_DS_FREE1), kDsFree);
-    // CTA pairs: the peer's softmax warpgroup (128 threads) has staged its tile's dQp
+    // CTA pairs: D = 64, the peer's softmax warpgroup (128 threads) has staged its tile's
+    // dQp; D = 128, the peer's reducers (128 threads) have filled this CTA's exchange
+    // buffer (B_PEER0), or have read theirs, so this CTA may write it again (B_PEER1)
     mbar_init(BAR(B_PEER0), 128);
     mbar_init(BAR(B_PEER1), 128);
     for (int b = 0; b < 2; ++b) {
@@ -893,8 +903,9 @@ __global__ void __launch_bounds__(512, 1)
         wait(S_FULL(it), s_phase(it));
         if (threadIdx.x == 0) trace(it, 3);
         tc_fence_after();
-        // causal: on the diagonal tile Q column qc sees KV row r only if qc >= r
-        const int lim_c = (p.causal && q == ch.y) ? r : -1;
+        // causal: on the diagonal tile Q column qc sees KV row r only if qc >= r; a CTA
+        // pair's tile above the diagonal (q < kv) is masked whole
+        const int lim_c = !p.causal ? -1 : q == ch.y ? r : (kPair && q < ch.y) ? 128 : -1;
 #pragma unroll 1
         for (int cc = 0; cc < 2; ++cc) {
           const int c = half * 2 + cc;  // 32-column chunk of the tile
@@ -994,7 +1005,7 @@ __global__ void __launch_bounds__(512, 1)
         const int ncontrib = kPair ? (p.causal ? q / 2 + 1 : N / 2) : (p.causal ? q + 1 : N);
         const bool last = (pos == ncontrib - 1);
         float a[D];
-        if constexpr (kPair) {
+        if constexpr (kPair && C::kSDouble) {
           // this CTA's half of the columns of the two partials staged for this step, its
           // own and the peer's (read over distributed shared memory once the peer says it
           // is staged), added: a + b is the same sum in either CTA
@@ -1044,6 +1055,44 @@ __global__ void __launch_bounds__(512, 1)
           }
           tc_fence_before();
           mbar_arrive(DQ_EMPTY(it));
+          if constexpr (kPair) {
+            // this CTA's half of the row in a[0, D/2), the peer's half in a[D/2, D)
+#pragma unroll
+            for (int j = 0; j < D / 2; ++j) {
+              const float lo = a[j], hi = a[D / 2 + j];
+              a[j] = prank ? hi : lo;
+              a[D / 2 + j] = prank ? lo : hi;
+            }
+            const uint32_t xb = sb + C::OFF_XB;
+            const uint32_t pxb = mapa_shared(xb, prank ^ 1u);
+#pragma unroll
+            for (int k = 0; k < D / 64; ++k) {
+              const int R = (D / 64) * it + k;  // exchange round
+              // the peer has read round R - 1 out of its buffer
+              if (R >= 1)
+                mbar_wait_cluster(BAR(B_PEER1), (uint32_t)((R - 1) & 1), lim, p.err,
+                                  p.abort_flag);
+#pragma unroll
+              for (int g = 0; g < 8; ++g) {
+                const float* x = a + D / 2 + 32 * k + 4 * g;
+                st_shared_cluster_f4(pxb + (uint32_t)((g * 128 + r) * 16),
+                                     make_float4(x[0], x[1], x[2], x[3]));
+              }
+              mbar_arrive_cluster(mapa_shared(BAR(B_PEER0), prank ^ 1u));
+              // the peer's columns of this CTA's half, round R
+              mbar_wait_cluster(BAR(B_PEER0), (uint32_t)(R & 1), lim, p.err, p.abort_flag);
+#pragma unroll
+              for (int g = 0; g < 8; ++g) {
+                const float4 v = ld_shared_f4(xb + (uint32_t)((g * 128 + r) * 16));
+                float* x = a + 32 * k + 4 * g;
+                x[0] = x[0] + v.x;
+                x[1] = x[1] + v.y;
+                x[2] = x[2] + v.z;
+                x[3] = x[3] + v.w;
+              }
+              mbar_arrive_cluster(mapa_shared(BAR(B_PEER1), prank ^ 1u));
+            }
+          }
         }
         if (threadIdx.x == 256) trace(it, 5);
         const long long blk = (long long)ch.x * N + q;

@@ -614,20 +614,21 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
 }
 
 // ------------------------------------------------------------------ CTA pairs
-// SHIFT_PAIRS / SYM_SHIFT_PAIRS at D = 64: the kernel runs in clusters of two CTAs, with as many
+// SHIFT_PAIRS / SYM_SHIFT_PAIRS: the kernel runs in clusters of two CTAs, with as many
 // clusters as fit on the device at once (cooperative, so all are resident).
-std::map<int, int> g_pair_ctas;  // device -> CTAs of the pair launch
+std::map<std::pair<int, int>, int> g_pair_ctas;  // (device, D) -> CTAs of the pair launch
+template <int D>
 int pair_ctas(int dev, int* out) {
-  auto it = g_pair_ctas.find(dev);
+  auto it = g_pair_ctas.find({dev, D});
   if (it != g_pair_ctas.end()) {
     *out = it->second;
     return DASH_OK;
   }
-  using C = BwdCfg<64>;
-  auto kern = dash::dash_bwd_kernel<64, false, false, false, true>;
-  for (auto k2 : {kern, dash::dash_bwd_kernel<64, false, false, true, true>}) {
+  using C = BwdCfg<D>;
+  auto kern = dash::dash_bwd_kernel<D, false, false, false, true>;
+  for (auto k2 : {kern, dash::dash_bwd_kernel<D, false, false, true, true>}) {
     DASH_CUDA(cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   C::kSmemBytes));
+                                   C::kSmemPairBytes));
     cudaFuncAttributes fa;
     DASH_CUDA(cudaFuncGetAttributes(&fa, k2));
     if (fa.numRegs != C::kLaunchRegs) return DASH_ERR_UNSUPPORTED;
@@ -637,7 +638,7 @@ int pair_ctas(int dev, int* out) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(2 * sms));
   cfg.blockDim = dim3(C::kThreads);
-  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.dynamicSmemBytes = C::kSmemPairBytes;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
@@ -649,15 +650,15 @@ int pair_ctas(int dev, int* out) {
   DASH_CUDA(cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg));
   if (clusters < 1) return DASH_ERR_UNSUPPORTED;
   *out = 2 * clusters;
-  g_pair_ctas[dev] = *out;
+  g_pair_ctas[{dev, D}] = *out;
   return DASH_OK;
 }
 
+template <int D>
 int launch_bwd_pairs(const void* q, const void* k, const void* v, const void* o,
                      const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
                      int H, int S, int causal, cudaStream_t stream, int dev,
                      const DevTable* tab_override = nullptr) {
-  constexpr int D = 64;
   using C = BwdCfg<D>;
   const int N = S / 128;
   const long long rows = (long long)B * H * S;
@@ -669,7 +670,7 @@ int launch_bwd_pairs(const void* q, const void* k, const void* v, const void* o,
   Workspace* ws = nullptr;
   {
     std::lock_guard<std::mutex> lk(g_mu);
-    if ((rc = pair_ctas(dev, &ctas))) return rc;
+    if ((rc = pair_ctas<D>(dev, &ctas))) return rc;
     // heads per unit of the half table (1 unless dash_set_head_interleave forces more)
     const int il = dash::head_interleave(D, pair_sched_of(causal), B * H, N, causal, ctas / 2,
                                          g_il_mode.load());
@@ -730,7 +731,7 @@ int launch_bwd_pairs(const void* q, const void* k, const void* v, const void* o,
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)ctas);
   cfg.blockDim = dim3(C::kThreads);
-  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.dynamicSmemBytes = C::kSmemPairBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
@@ -745,8 +746,8 @@ int launch_bwd_pairs(const void* q, const void* k, const void* v, const void* o,
   // middle links with red in L2 only where the chain mode forces it (bitwise the same)
   const bool red = red_chain_for(pair_sched_of(causal), N, D, 1);
   DASH_CUDA(cudaLaunchKernelEx(&cfg,
-                               red ? dash::dash_bwd_kernel<64, false, false, true, true>
-                                   : dash::dash_bwd_kernel<64, false, false, false, true>,
+                               red ? dash::dash_bwd_kernel<D, false, false, true, true>
+                                   : dash::dash_bwd_kernel<D, false, false, false, true>,
                                tq, tk, tv, tdo, tc, p));
   if (!prof_record(2, &ev, stream) || !prof_record(3, &ev, stream)) return DASH_ERR_CUDA;
   if (g_prof_on.load()) {
@@ -856,12 +857,12 @@ int host_bwd(const void* q, const void* k, const void* v, const void* o, const v
              const float* lse, void* dq, void* dk, void* dv, int B, int H, int S, int causal,
              int sched, cudaStream_t stream, int dev) {
   const int BH = B * H, N = S / 128;
-  const bool pairs = pair_sched(sched);  // CTA pairs (D = 64 only)
+  const bool pairs = pair_sched(sched);  // CTA pairs
   int ctas = 0;
   int rc;
   {
     std::lock_guard<std::mutex> lk(g_mu);
-    rc = pairs ? pair_ctas(dev, &ctas) : num_ctas_for<D, kAtomic>(dev, &ctas);
+    rc = pairs ? pair_ctas<D>(dev, &ctas) : num_ctas_for<D, kAtomic>(dev, &ctas);
   }
   if (rc) return rc;
   // the parts hold whole units of the launch's table, so its interleaved heads stay
@@ -913,7 +914,7 @@ int host_bwd(const void* q, const void* k, const void* v, const void* o, const v
     // compute, once the inputs are in and the results of part c - 2 are out
     DASH_CUDA(cudaStreamWaitEvent(stream, hp->in_ready[slot], 0));
     if (c >= 2) DASH_CUDA(cudaStreamWaitEvent(stream, hp->out_done[slot], 0));
-    if ((rc = pairs ? launch_bwd_pairs(din[0], din[1], din[2], din[3], din[4], dlse, dout3[0],
+    if ((rc = pairs ? launch_bwd_pairs<D>(din[0], din[1], din[2], din[3], din[4], dlse, dout3[0],
                                        dout3[1], dout3[2], 1, nh, S, causal, stream, dev,
                                        &(*parts)[c])
                     : launch_bwd<D, kAtomic>(din[0], din[1], din[2], din[3], din[4], dlse,
@@ -1110,15 +1111,15 @@ int dash_attn_bwd(const void* q, const void* k, const void* v, const void* o, co
       if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
           !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
         return DASH_ERR_INVALID_ARG;
-      // CTA pairs exist at D = 64 (the staged dQp they exchange): SHIFT_PAIRS for the
-      // full mask, SYM_SHIFT_PAIRS for the causal one
-      if (D != 64 || !dash::schedule_supported(schedule, S / 128, causal))
-        return DASH_ERR_UNSUPPORTED;
+      // CTA pairs: SHIFT_PAIRS for the full mask, SYM_SHIFT_PAIRS for the causal one
+      if (!dash::schedule_supported(schedule, S / 128, causal)) return DASH_ERR_UNSUPPORTED;
       if (B == 0 || H == 0) return DASH_OK;
       int dev = 0;
       DASH_CUDA(cudaGetDevice(&dev));
-      return launch_bwd_pairs(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
-                              static_cast<cudaStream_t>(stream), dev);
+      return D == 64 ? launch_bwd_pairs<64>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
+                                            static_cast<cudaStream_t>(stream), dev)
+                     : launch_bwd_pairs<128>(q, k, v, o, dout, lse, dq, dk, dv, B, H, S, causal,
+                                             static_cast<cudaStream_t>(stream), dev);
     }, DASH_ERR_OOM, DASH_ERR_INVALID_ARG);
   return dash_attn_bwd_gqa(q, k, v, o, dout, lse, dq, dk, dv, B, H, H, S, D, causal, schedule,
                            stream);
@@ -1133,7 +1134,6 @@ int dash_attn_bwd_host(const void* q, const void* k, const void* v, const void* 
     if (causal != 0 && causal != 1) return DASH_ERR_INVALID_ARG;
     if (schedule < DASH_SCHED_NAIVE_ASC || schedule > DASH_SCHED_SYM_SHIFT_PAIRS)
       return DASH_ERR_INVALID_ARG;
-    if (pair_sched(schedule) && D != 64) return DASH_ERR_UNSUPPORTED;
     if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return DASH_ERR_INVALID_ARG;
     if (!dash::schedule_supported(schedule, S / 128, causal)) return DASH_ERR_UNSUPPORTED;
     if (B == 0 || H == 0) return DASH_OK;

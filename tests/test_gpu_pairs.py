@@ -1,6 +1,6 @@
 """CTA pairs that pre-sum dQ (DASH_SCHED_SHIFT_PAIRS for the full mask,
-DASH_SCHED_SYM_SHIFT_PAIRS for the causal one; D = 64): the two dQ partials of a pair's
-step are added before the ordered accumulation, each CTA taking half of the columns.
+DASH_SCHED_SYM_SHIFT_PAIRS for the causal one; D = 64 and 128): the two dQ partials of a
+pair's step are added before the ordered accumulation, each CTA taking half of the columns.
 Against the fp64 oracle on shapes with one or several rounds of CTA pairs (and, causal,
 on sampled rows of the full 16k workload), bitwise repeats, and the refusals for shapes
 the pairs do not serve."""
@@ -35,9 +35,9 @@ def test_pairs_match_oracle_and_repeat(B, H, S):
 
 
 @pytest.mark.parametrize("S,D,causal,sched", [
-    (512, 128, False, "shift_pairs"), (512, 64, True, "shift_pairs"),
-    (384, 64, False, "shift_pairs"), (512, 128, True, "sym_shift_pairs"),
-    (512, 64, False, "sym_shift_pairs"), (768, 64, True, "sym_shift_pairs")])
+    (512, 64, True, "shift_pairs"), (384, 64, False, "shift_pairs"),
+    (384, 128, False, "shift_pairs"), (512, 64, False, "sym_shift_pairs"),
+    (768, 64, True, "sym_shift_pairs"), (768, 128, True, "sym_shift_pairs")])
 def test_pairs_refuse_other_shapes(S, D, causal, sched):
     G.need_cuda()
     case = G.make_case(1, 2, S, D, causal, seed=5)
@@ -186,3 +186,53 @@ def test_pairs_with_two_heads_per_unit(causal, sched):
     for a, b, c in zip(out, again, got):
         assert torch.equal(a, b)
         assert torch.equal(a.cpu(), c)
+
+
+# ---------------------------------------------------------------- D = 128
+# dQp stays in TMEM at D = 128; the pair exchanges the other half of each row through a
+# 16 KiB buffer in the peer's shared memory, 32 columns a round.
+
+@pytest.mark.parametrize("B,H,S,causal,sched", [
+    (1, 2, 256, False, "shift_pairs"),
+    (2, 3, 1024, False, "shift_pairs"),
+    (4, 40, 256, False, "shift_pairs"),      # more than one round of CTA pairs
+    (1, 2, 512, True, "sym_shift_pairs"),
+    (2, 3, 1024, True, "sym_shift_pairs"),
+    (4, 40, 512, True, "sym_shift_pairs"),
+])
+def test_pairs_d128_match_oracle_and_repeat(B, H, S, causal, sched):
+    G.need_cuda()
+    case = G.make_case(B, H, S, 128, causal, seed=1300 + S + H)
+    _, _, *ref = G.oracle_full(case)
+    out = G.bwd(case, sched)
+    errs = {n: A.rel_fro(x.float().cpu().numpy(), r) for n, x, r in zip(("dq", "dk", "dv"), out, ref)}
+    G.log_margin(f"{sched} B{B} H{H} S{S} D128 {'causal' if causal else 'full'}", errs)
+    assert max(errs.values()) < G.TOL, errs
+    again = G.bwd(case, sched)
+    for a, b in zip(out, again):
+        assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("causal,sched", [(False, "shift_pairs"), (True, "sym_shift_pairs")])
+def test_pairs_d128_host_path_and_repeats(causal, sched):
+    """20 launches at B=2 H=16 S=4096 D=128 give the same bits, and the host-buffer path
+    gives dash_attn_bwd's bits.  Against the one-CTA schedule the pairs differ only in the
+    order of the fp32 additions (partials pre-summed in pairs), which flips the rounding of
+    a few bf16 outputs: about 1e-4 relative, bounded here by 1e-3."""
+    G.need_cuda()
+    case = G.make_case(2, 16, 4096, 128, causal, seed=1700 + causal)
+    first = G.bwd(case, sched)
+    for _ in range(19):
+        again = G.bwd(case, sched)
+        for a, b in zip(first, again):
+            assert torch.equal(a, b)
+    plain = G.bwd(case, "sym_shift" if causal else "shift")
+    for a, b in zip(first, plain):
+        rel = (torch.linalg.vector_norm(a.float() - b.float()) /
+               torch.linalg.vector_norm(b.float())).item()
+        assert rel < 1e-3, rel
+    host = [case[n].cpu().pin_memory() for n in ("q", "k", "v", "o", "do", "lse")]
+    got = binding.dash_attn_bwd_host(*host, causal, sched)
+    assert binding.dash_attn_sync_status() == 0
+    for a, b in zip(first, got):
+        assert torch.equal(a.cpu(), b)
