@@ -2,8 +2,8 @@
 launches racing a concurrent load on another stream, on every workload at its
 full size (best schedule and the descending order, plus naive ascending where
 it is one of the workload's compared schedules), on a reduced causal D = 64
-shape, and for the CTA-pair schedules on a full-mask D = 64 shape and the causal
-16k workload."""
+shape, and for the CTA-pair schedules on a full-mask D = 64 shape, the causal 16k
+workload and the two D = 128 configurations (full 4k, causal 8k)."""
 import pytest
 import torch
 
@@ -27,6 +27,11 @@ CASES.append(("full_b2_h16_s4096_d64_pairs", (2, 16, 4096, 64, False, 1.0, 12), 
 _w3 = WORKLOADS[3]
 CASES.append((_w3.name + "_pairs", (_w3.B, _w3.H, _w3.S, _w3.D, _w3.causal, _w3.sigma, seed_of(3)),
               ("sym_shift_pairs",)))
+# and at D = 128, on the full-mask 4k and causal 8k configurations
+for _i, _sched in ((1, "shift_pairs"), (2, "sym_shift_pairs")):
+    _w = WORKLOADS[_i]
+    CASES.append((_w.name + "_pairs", (_w.B, _w.H, _w.S, _w.D, _w.causal, _w.sigma, seed_of(_i)),
+                  (_sched,)))
 IDS = [c[0] for c in CASES]
 
 
